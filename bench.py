@@ -1,0 +1,384 @@
+"""Benchmark of the routed MoE FFN layer (Gemma-4-26B-A4B shape) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config decode] [--impl reference]
+
+A step is one moe_forward over one batch (router, dispatch, GEMM-1 + GEGLU, GEMM-2,
+combine) with inputs resident in HBM.  L2 is flushed (256 MB write, untimed) before
+every step; each step is timed with CUDA events on the launching stream.  Rank 0 prints
+one JSON line.  With N > 1 (torchrun) every rank runs its own batch on its own GPU (weak
+scaling, no collective on the data path) and the reported time is the max over ranks.
+
+--impl reference times the fp64 CPU oracle instead (the only baseline this layer has),
+on rank 0 only, on the same config.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+from expert_routed_ffn_softmax_b200 import workloads as wl  # noqa: E402
+
+METRIC = "MoE-layer tokens/s; HBM GB/s (decode) & BF16 TFLOP/s (prefill) vs peak"
+UNIT = "tokens/s"
+KERNELS_PER_STEP = 9   # router 2, dispatch 4, GEMM-1, GEMM-2, combine
+PER_EXPERT_BYTES = 11_894_784   # 3 * 2816 * 704 * 2: weights one active expert reads
+L2_FLUSH_BYTES = 256 << 20
+
+
+def peaks() -> dict:
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained", d["bf16_tflops"]),
+                "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "source": "fallback"}
+
+
+# ----------------------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi clock/throttle samples while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.idx = gpu_index
+        self.proc = None
+        self.lines: list[str] = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except OSError:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self) -> dict | None:
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, mx, reasons = [], 0.0, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [s.strip() for s in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = max(mx, float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------- accounting
+def algorithmic(cfg: wl.MoEConfig, counts: np.ndarray, has_bias: bool) -> dict:
+    """Bytes/FLOPs the layer itself must move/compute (not Xp/Hbuf/O traffic)."""
+    active = int((counts > 0).sum())
+    P = cfg.T * cfg.k
+    ew = 3 * cfg.H * cfg.I * 2
+    step_bytes = (active * ew + cfg.H * cfg.E * 2 + 2 * cfg.T * cfg.H * 2
+                  + (cfg.E * 4 if has_bias else 0))
+    step_flops = cfg.T * 2 * cfg.H * cfg.E + P * (2 * cfg.H * 2 * cfg.I + 2 * cfg.I * cfg.H)
+    return {
+        "active_experts": active,
+        "step_bytes": step_bytes,
+        "step_flops": step_flops,
+        "gemm1_bytes": active * 2 * cfg.H * cfg.I * 2,
+        "gemm1_flops": P * 2 * cfg.H * 2 * cfg.I,
+        "gemm2_bytes": active * cfg.H * cfg.I * 2,
+        "gemm2_flops": P * 2 * cfg.I * cfg.H,
+    }
+
+
+def kernel_source_sha() -> str:
+    h = hashlib.sha256()
+    for f in ("grouped_gemm.cuh", "ptx.cuh", "moe.cu"):
+        h.update(open(os.path.join(ROOT, "expert_routed_ffn_softmax_b200", "csrc", f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(kernel: str, workload: str) -> float | None:
+    """DRAM bytes per launch recorded by ncu for this kernel source, else None."""
+    p = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    if not os.path.exists(p):
+        return None
+    try:
+        rows = json.load(open(p))
+    except ValueError:
+        return None
+    sha = kernel_source_sha()
+    for r in rows:
+        if r.get("kernel") == kernel and r.get("workload") == workload and r.get("source_sha") == sha:
+            return float(r["dram_bytes_per_launch"])
+    return None
+
+
+# ----------------------------------------------------------------------------- arms
+def run_reference(args, cfg) -> None:
+    import oracle
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    cores = len(os.sched_getaffinity(0))
+    oracle.set_threads(cores)
+    d = wl.make_inputs(cfg)
+    T_s = min(cfg.T, args.ref_tokens)
+    x = d["x"][:T_s].contiguous()
+
+    def step():
+        oracle.forward(x, d["w_router"], d["w_gate"], d["w_up"], d["w_down"], cfg.k, bias=d["bias"])
+
+    for _ in range(args.warmup):
+        step()
+    times = []
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        step()
+        times.append(time.perf_counter() - t0)
+    sec = sum(times) / len(times)
+    v = T_s / sec
+    sample = f"{T_s} of the {cfg.T} tokens of the {cfg.name} batch per step, fp64, all experts selected"
+    line = {
+        "impl": "reference", "metric": METRIC, "value": v, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": sec * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": f"{cfg.name}: T={cfg.T} H={cfg.H} E={cfg.E} k={cfg.k} I={cfg.I}",
+                   "global_batch": cfg.T, "parallelism": "cpu"},
+        "cpu_baseline": {"value": v, "unit": UNIT, "cores": oracle.get_threads(),
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def cpu_baseline(cfg, d, budget_s: float) -> dict:
+    import oracle
+    cores = len(os.sched_getaffinity(0))
+    oracle.set_threads(cores)
+    T_s = min(cfg.T, 64)
+    x = d["x"][:T_s].contiguous()
+    n, t_total = 0, 0.0
+    while t_total < budget_s or n == 0:
+        t0 = time.perf_counter()
+        oracle.forward(x, d["w_router"], d["w_gate"], d["w_up"], d["w_down"], cfg.k, bias=d["bias"])
+        t_total += time.perf_counter() - t0
+        n += 1
+    return {"value": n * T_s / t_total, "unit": UNIT, "cores": oracle.get_threads(),
+            "kind": "oracle",
+            "sample": f"{n} x forward of the first {T_s} tokens of the {cfg.name} batch "
+                      f"({t_total:.1f} s of fp64 CPU work)"}
+
+
+def run_native(args, cfg) -> None:
+    import expert_routed_ffn_softmax_b200 as moe
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+
+    d = wl.make_weights(cfg)
+    x_cpu = wl.make_x(cfg, seed=rank)
+    g = {k: (v.to(dev) if v is not None else None) for k, v in d.items()}
+    x = x_cpu.to(dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def fwd(xx, out=None, profile=False):
+        return moe.forward(xx, g["w_router"], g["w_gate"], g["w_up"], g["w_down"], cfg.k,
+                           bias=g["bias"], out=out, profile=profile)
+
+    y = torch.empty((cfg.T, cfg.H), dtype=torch.bfloat16, device=dev)
+    y0, aux = moe.forward(x, g["w_router"], g["w_gate"], g["w_up"], g["w_down"], cfg.k,
+                          bias=g["bias"], aux=True)
+    if moe.sync_status() != 0:
+        raise SystemExit("device status not OK after the first forward")
+    counts = aux["expert_counts"].cpu().numpy()
+    acc = algorithmic(cfg, counts, d["bias"] is not None)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        fwd(x, y)
+    torch.cuda.synchronize()
+
+    # ---- timed region: K steps, L2 flushed (untimed) before each
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    clocks = ClockSampler(local)
+    clocks.start()
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    for i in range(args.steps):
+        flush.zero_()
+        ev[i][0].record(stream)
+        fwd(x, y)
+        ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    clk = clocks.stop()
+    step_ms = [a.elapsed_time(b) for a, b in ev]
+    ms = sum(step_ms) / len(step_ms)
+    if moe.sync_status() != 0:
+        raise SystemExit("device status not OK after the timed steps")
+
+    # ---- per-stage device times (same calls with stage events), L2 flushed before each
+    stage_acc: dict[str, list[float]] = {}
+    for _ in range(max(3, min(args.steps, 20))):
+        flush.zero_()
+        fwd(x, y, profile=True)
+        for k, v in moe.last_stage_times().items():
+            stage_acc.setdefault(k, []).append(v)
+    stages = {k: sum(v) / len(v) for k, v in stage_acc.items()}
+
+    # ---- end to end through the public API with host buffers (pinned), L2 flushed
+    x_host = x_cpu.pin_memory()
+    y_host = torch.empty((cfg.T, cfg.H), dtype=torch.bfloat16).pin_memory()
+    x_dev = torch.empty_like(x)
+    e2e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(args.steps)]
+    for i in range(args.warmup + args.steps):
+        flush.zero_()
+        if i >= args.warmup:
+            e2e_ev[i - args.warmup][0].record(stream)
+        x_dev.copy_(x_host, non_blocking=True)
+        fwd(x_dev, y)
+        y_host.copy_(y, non_blocking=True)
+        if i >= args.warmup:
+            e2e_ev[i - args.warmup][1].record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = sum(a.elapsed_time(b) for a, b in e2e_ev) / args.steps
+
+    if dist:
+        t = torch.tensor([ms, e2e_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms, e2e_ms = float(t[0]), float(t[1])
+
+    if rank == 0:
+        pk = peaks()
+        g1, g2 = stages.get("gemm1_geglu", 0.0), stages.get("gemm2_down", 0.0)
+        dom = "gemm1_geglu" if g1 >= g2 else "gemm2_down"
+        dom_ms = max(g1, g2)
+        kb = acc["gemm1_bytes"] if dom == "gemm1_geglu" else acc["gemm2_bytes"]
+        kf = acc["gemm1_flops"] if dom == "gemm1_geglu" else acc["gemm2_flops"]
+        ridge = pk["bf16_tflops"] * 1e12 / (pk["hbm_gbs"] * 1e9)
+        kname = "grouped_gemm_kernel<4,0>" if dom == "gemm1_geglu" else "grouped_gemm_kernel<4,1>"
+        traffic = ncu_traffic(kname, cfg.name)
+        if kf / kb < ridge:
+            achieved = kb / (dom_ms * 1e-3) / 1e9
+            roof = {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                    "frac": achieved / pk["hbm_gbs"], "traffic": traffic,
+                    "kernel": kname, "peak_source": pk["source"] + " hbm_gbs"}
+        else:
+            achieved = kf / (dom_ms * 1e-3) / 1e12
+            roof = {"bound": "tensor", "achieved": achieved, "peak": pk["bf16_tflops"],
+                    "unit": "TFLOP/s", "frac": achieved / pk["bf16_tflops"], "traffic": traffic,
+                    "kernel": kname, "peak_source": pk["source"] + " bf16_tflops (burst)"}
+        step_s = ms * 1e-3
+        line = {
+            "metric": METRIC,
+            "value": world * cfg.T / step_s,
+            "unit": UNIT,
+            "n_gpus": world,
+            "steps": args.steps,
+            "warmup": args.warmup,
+            "ms_per_step": ms,
+            "higher_is_better": True,
+            "scaling": "weak",
+            "vs_baseline": None,
+            "dtype": "bf16",
+            "data": "synthetic",
+            "config": {"workload": f"{cfg.name}: T={cfg.T} H={cfg.H} E={cfg.E} k={cfg.k} "
+                                   f"I={cfg.I} (routed MoE FFN layer, Gemma-4-26B-A4B shape)",
+                       "global_batch": world * cfg.T, "tokens_per_gpu": cfg.T,
+                       "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                       "l2": "flushed before every step (256 MB write, untimed)"},
+            "roofline": roof,
+            "step_roofline": {
+                "hbm_frac": acc["step_bytes"] / step_s / (pk["hbm_gbs"] * 1e9),
+                "tensor_frac": acc["step_flops"] / step_s / (pk["bf16_tflops"] * 1e12),
+                "algorithmic_bytes": acc["step_bytes"], "algorithmic_flops": acc["step_flops"],
+                "active_experts": acc["active_experts"]},
+            "stages_ms": stages,
+            "e2e": {"value": world * cfg.T / (e2e_ms * 1e-3), "unit": UNIT,
+                    "h2d_bytes_per_step": cfg.T * cfg.H * 2,
+                    "d2h_bytes_per_step": cfg.T * cfg.H * 2},
+            "gpu_launches": KERNELS_PER_STEP * args.steps,
+            "clocks": clk,
+            "step_ms_p10_p50_p90": [float(np.percentile(step_ms, q)) for q in (10, 50, 90)],
+        }
+        if not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline(cfg, d, args.cpu_seconds)
+        print(json.dumps(line), flush=True)
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--config", default="decode", choices=sorted(wl.CONFIGS))
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--ref-tokens", type=int, default=8)
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)     # at least 3 untimed warm-up steps
+    cfg = wl.CONFIGS[args.config]
+    if args.impl == "reference":
+        run_reference(args, cfg)
+    else:
+        run_native(args, cfg)
+
+
+if __name__ == "__main__":
+    main()

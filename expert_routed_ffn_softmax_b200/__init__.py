@@ -1,1 +1,16 @@
+"""B200-native (sm_100a) routed Mixture-of-Experts FFN layer.
 
+The public calls mirror the C ABI of include/moe.h:
+
+    ids, weights = route(x, w_router, k, bias=None, renorm=True)
+    y            = forward(x, w_router, w_gate, w_up, w_down, k, bias=None, renorm=True)
+
+x, weights and outputs are CUDA tensors (bf16 operands, int32 ids, fp32 routing weights);
+all arithmetic runs in libmoe_b200.so.  ``workloads`` (seeded synthetic inputs) can be
+imported without a GPU.
+"""
+from ._abi import (MoEError, forward, last_stage_times, load, route, status_string,  # noqa: F401
+                   sync_status)
+
+__all__ = ["route", "forward", "sync_status", "last_stage_times", "load", "status_string",
+           "MoEError"]

@@ -1,0 +1,188 @@
+"""ctypes binding of include/moe.h (argument marshalling only).
+
+Every step of the layer runs in libmoe_b200.so; this module checks tensor types and
+shapes, owns a per-device workspace buffer, and passes raw pointers and the current
+CUDA stream across the C ABI.  There is no fallback: if the library cannot be loaded,
+every call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libmoe_b200.so")
+
+MOE_OK = 0
+MOE_ERR_INVALID_ARG = 1
+MOE_ERR_UNSUPPORTED = 2
+MOE_ERR_NO_WORKSPACE = 3
+MOE_ERR_CUDA = 4
+MOE_ERR_TIMEOUT = 5
+
+MOE_FLAG_NO_RENORM = 1 << 0
+MOE_FLAG_PROFILE_STAGES = 1 << 3
+
+# Every function the header declares, with (restype, argtypes).
+_P, _I, _U, _SZ = ctypes.c_void_p, ctypes.c_int, ctypes.c_uint, ctypes.c_size_t
+SIGNATURES = {
+    "moe_abi_version": (_I, []),
+    "moe_status_string": (ctypes.c_char_p, [_I]),
+    "moe_route_workspace_size": (_SZ, [_I, _I, _I, _I, _U]),
+    "moe_workspace_size": (_SZ, [_I, _I, _I, _I, _I, _U]),
+    "moe_route": (_I, [_P, _P, _P, _I, _I, _I, _I, _U, _P, _P, _P, _SZ, _P]),
+    "moe_forward": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _U, _P, _P, _P, _SZ, _P]),
+    "moe_sync_status": (_I, [_P]),
+    "moe_last_stage_times": (_I, [ctypes.POINTER(ctypes.c_float), _I]),
+    "moe_stage_name": (ctypes.c_char_p, [_I]),
+    "moe_debug_set_wait_limit_ns": (_I, [ctypes.c_ulonglong]),
+    "moe_debug_unsatisfied_wait": (_I, [_P]),
+}
+
+
+class MoEError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        self.code = code
+        super().__init__(f"{what}: {status_string(code)} ({code})")
+
+
+class AuxOut(ctypes.Structure):
+    _fields_ = [("expert_counts", _P), ("expert_offsets", _P), ("perm", _P),
+                ("topk_ids", _P), ("topk_weights", _P)]
+
+
+_lib = None
+_lock = threading.Lock()
+
+
+def load(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load the library (once).  Raises if it is missing or incomplete."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(path):
+                raise RuntimeError(f"{path} is missing: build it with "
+                                   "`python -m expert_routed_ffn_softmax_b200.build`")
+            L = ctypes.CDLL(path)
+            for name, (res, args) in SIGNATURES.items():
+                fn = getattr(L, name)
+                fn.restype, fn.argtypes = res, args
+            _lib = L
+    return _lib
+
+
+def status_string(code: int) -> str:
+    return load().moe_status_string(code).decode()
+
+
+def _check(code: int, what: str) -> None:
+    if code != MOE_OK:
+        raise MoEError(code, what)
+
+
+def _stream_ptr(stream) -> int:
+    s = torch.cuda.current_stream() if stream is None else stream
+    return s.cuda_stream
+
+
+_ws: dict[int, torch.Tensor] = {}
+
+
+def workspace(nbytes: int, device: torch.device) -> torch.Tensor:
+    """A per-device scratch buffer of at least nbytes (grown on demand, 256-byte aligned)."""
+    idx = device.index if device.index is not None else torch.cuda.current_device()
+    buf = _ws.get(idx)
+    if buf is None or buf.numel() < nbytes:
+        buf = torch.empty(max(nbytes, 1 << 20), dtype=torch.uint8, device=device)
+        _ws[idx] = buf
+    return buf
+
+
+def _dev(t: torch.Tensor, name: str, dtype: torch.dtype, shape: tuple) -> int:
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t.data_ptr()
+
+
+def route(x: torch.Tensor, w_router: torch.Tensor, k: int, bias: torch.Tensor | None = None,
+          renorm: bool = True, stream=None):
+    """Router of the MoE layer -> (topk_ids int32 [T,k], topk_weights float32 [T,k])."""
+    L = load()
+    T, H = x.shape
+    E = w_router.shape[1]
+    dev = x.device
+    px = _dev(x, "x", torch.bfloat16, (T, H))
+    pw = _dev(w_router, "w_router", torch.bfloat16, (H, E))
+    pb = None if bias is None else _dev(bias, "bias", torch.float32, (E,))
+    flags = 0 if renorm else MOE_FLAG_NO_RENORM
+    ids = torch.empty((T, k), dtype=torch.int32, device=dev)
+    wts = torch.empty((T, k), dtype=torch.float32, device=dev)
+    nbytes = L.moe_route_workspace_size(T, H, E, k, flags) if T > 0 else 0
+    if T > 0 and nbytes == 0:
+        raise MoEError(MOE_ERR_UNSUPPORTED, "moe_route_workspace_size")
+    ws = workspace(nbytes, dev)
+    _check(L.moe_route(px, pw, pb, T, H, E, k, flags, ids.data_ptr(), wts.data_ptr(),
+                       ws.data_ptr(), ws.numel(), _stream_ptr(stream)), "moe_route")
+    return ids, wts
+
+
+def forward(x: torch.Tensor, w_router: torch.Tensor, w_gate: torch.Tensor, w_up: torch.Tensor,
+            w_down: torch.Tensor, k: int, bias: torch.Tensor | None = None, renorm: bool = True,
+            aux: bool = False, out: torch.Tensor | None = None, profile: bool = False,
+            stream=None):
+    """The routed MoE FFN layer -> y bf16 [T,H] (and a dict of routing outputs if aux)."""
+    L = load()
+    T, H = x.shape
+    E, _, I = w_gate.shape
+    dev = x.device
+    px = _dev(x, "x", torch.bfloat16, (T, H))
+    pr = _dev(w_router, "w_router", torch.bfloat16, (H, E))
+    pg = _dev(w_gate, "w_gate", torch.bfloat16, (E, H, I))
+    pu = _dev(w_up, "w_up", torch.bfloat16, (E, H, I))
+    pd = _dev(w_down, "w_down", torch.bfloat16, (E, I, H))
+    pb = None if bias is None else _dev(bias, "bias", torch.float32, (E,))
+    y = torch.empty((T, H), dtype=torch.bfloat16, device=dev) if out is None else out
+    py = _dev(y, "out", torch.bfloat16, (T, H))
+    flags = (0 if renorm else MOE_FLAG_NO_RENORM) | (MOE_FLAG_PROFILE_STAGES if profile else 0)
+    a = None
+    aux_d = None
+    if aux:
+        aux_d = {
+            "expert_counts": torch.empty(E, dtype=torch.int32, device=dev),
+            "expert_offsets": torch.empty(E + 1, dtype=torch.int32, device=dev),
+            "perm": torch.empty(T * k, dtype=torch.int32, device=dev),
+            "topk_ids": torch.empty((T, k), dtype=torch.int32, device=dev),
+            "topk_weights": torch.empty((T, k), dtype=torch.float32, device=dev),
+        }
+        a = AuxOut(*(aux_d[n].data_ptr() for n, _ in AuxOut._fields_))
+    nbytes = L.moe_workspace_size(T, H, E, I, k, flags) if T > 0 else 0
+    if T > 0 and nbytes == 0:
+        raise MoEError(MOE_ERR_UNSUPPORTED, "moe_workspace_size")
+    ws = workspace(nbytes, dev)
+    _check(L.moe_forward(px, pr, pb, pg, pu, pd, T, H, E, I, k, flags, py,
+                         None if a is None else ctypes.byref(a), ws.data_ptr(), ws.numel(),
+                         _stream_ptr(stream)), "moe_forward")
+    return (y, aux_d) if aux else y
+
+
+def sync_status(stream=None) -> int:
+    """Synchronise the stream and return (and clear) the device-side status code."""
+    return load().moe_sync_status(_stream_ptr(stream))
+
+
+def last_stage_times() -> dict[str, float]:
+    L = load()
+    buf = (ctypes.c_float * 16)()
+    n = L.moe_last_stage_times(buf, 16)
+    if n < 0:
+        raise RuntimeError("no profiled moe_forward call yet")
+    return {L.moe_stage_name(i).decode(): float(buf[i]) for i in range(n)}

@@ -1,0 +1,171 @@
+// dispatch.cuh -- per-expert histogram, exclusive scan, stable permutation and the row
+// gather that makes each expert's tokens contiguous (the per-expert "split sizes" of the
+// double_routing dispatch, cann-recipes-infer Gemma-4-26B-A4B optimisation report §6.1
+// 方案), plus the unpermute-combine y[t] = sum_j w[t,j] * O[inv[t,j]].
+//
+// The permutation lists, expert by expert, the pairs q = t*k + j in ascending q, so it is
+// unique and identical to the definition: pairs are cut into fixed chunks, each chunk
+// counts its experts, a scan turns the counts into per-(chunk, expert) bases, and one
+// warp per chunk ranks its pairs in order with __match_any_sync.
+#pragma once
+#include "ptx.cuh"
+
+namespace moe {
+
+constexpr int kDispatchChunk = 2048;   // pairs per chunk
+
+// chunk_counts[c][e] = #pairs with id e in chunk c.
+__global__ void __launch_bounds__(256) dispatch_count_kernel(const int32_t* __restrict__ ids,
+                                                              int P, int E,
+                                                              int32_t* __restrict__ chunk_counts) {
+  extern __shared__ int hist[];
+  for (int e = threadIdx.x; e < E; e += blockDim.x) hist[e] = 0;
+  __syncthreads();
+  const int q0 = blockIdx.x * kDispatchChunk, q1 = min(P, q0 + kDispatchChunk);
+  for (int q = q0 + threadIdx.x; q < q1; q += blockDim.x) {
+    const int e = ids[q];
+    if ((unsigned)e < (unsigned)E)
+      atomicAdd(&hist[e], 1);
+    else
+      raise_error(MOE_DEVERR_BAD_INDEX);
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x)
+    chunk_counts[(size_t)blockIdx.x * E + e] = hist[e];
+}
+
+// One CTA (blockDim >= E).  counts, offsets, chunk_base[c][e] = offsets[e] + pairs of e in
+// chunks before c, and the GEMM tile list: for every expert with n_e > 0, tiles of BM rows
+// (expert, first sorted row, rows in tile), in expert order.
+__global__ void __launch_bounds__(256) dispatch_scan_kernel(
+    const int32_t* __restrict__ chunk_counts, int nchunks, int E, int P, int BM,
+    int32_t* __restrict__ counts, int32_t* __restrict__ offsets, int32_t* __restrict__ chunk_base,
+    int32_t* __restrict__ tile_num, int32_t* __restrict__ tile_expert,
+    int32_t* __restrict__ tile_row0, int32_t* __restrict__ tile_rows) {
+  __shared__ int s_cnt[256], s_off[256], s_tstart[256];
+  const int e = threadIdx.x;
+  int run = 0;
+  if (e < E) {
+    for (int c = 0; c < nchunks; ++c) {
+      chunk_base[(size_t)c * E + e] = run;
+      run += chunk_counts[(size_t)c * E + e];
+    }
+    s_cnt[e] = run;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int o = 0, ts = 0;
+    for (int i = 0; i < E; ++i) {
+      s_off[i] = o;
+      s_tstart[i] = ts;
+      o += s_cnt[i];
+      ts += (s_cnt[i] + BM - 1) / BM;
+    }
+    offsets[E] = o;
+    *tile_num = ts;
+  }
+  __syncthreads();
+  if (e < E) {
+    const int off = s_off[e];
+    counts[e] = run;
+    offsets[e] = off;
+    for (int c = 0; c < nchunks; ++c) chunk_base[(size_t)c * E + e] += off;
+    const int nt = (run + BM - 1) / BM;
+    for (int m = 0; m < nt; ++m) {
+      const int i = s_tstart[e] + m;
+      tile_expert[i] = e;
+      tile_row0[i] = off + m * BM;
+      tile_rows[i] = min(BM, run - m * BM);
+    }
+  }
+}
+
+// One warp per chunk: stable positions pos = chunk_base[c][e] + rank among earlier pairs
+// of the chunk with the same expert.  perm[pos] = q, inv[q] = pos.
+__global__ void __launch_bounds__(32) dispatch_rank_kernel(const int32_t* __restrict__ ids, int P,
+                                                           int E,
+                                                           const int32_t* __restrict__ chunk_base,
+                                                           int32_t* __restrict__ perm,
+                                                           int32_t* __restrict__ inv) {
+  extern __shared__ int base[];
+  const int lane = threadIdx.x;
+  for (int e = lane; e < E; e += 32) base[e] = chunk_base[(size_t)blockIdx.x * E + e];
+  __syncwarp();
+  const int q0 = blockIdx.x * kDispatchChunk, q1 = min(P, q0 + kDispatchChunk);
+  const unsigned lt = (1u << lane) - 1u;
+  for (int qb = q0; qb < q1; qb += 32) {
+    const int q = qb + lane;
+    const bool valid = q < q1;
+    int e = valid ? ids[q] : -1;
+    if (valid && (unsigned)e >= (unsigned)E) e = -2;  // counted as an error already
+    const unsigned grp = __match_any_sync(0xffffffffu, e);
+    const int rank = __popc(grp & lt);
+    int pos = 0;
+    if (e >= 0) pos = base[e] + rank;
+    __syncwarp();
+    if (e >= 0 && lane == 31 - __clz(grp)) base[e] += __popc(grp);
+    __syncwarp();
+    if (e >= 0) {
+      perm[pos] = q;
+      inv[q] = pos;
+    }
+  }
+}
+
+// Xp[pos, :] = x[perm[pos] / k, :]   (16-byte vectors; one warp per row, grid-stride)
+__global__ void __launch_bounds__(256) gather_rows_kernel(const uint4* __restrict__ x,
+                                                          const int32_t* __restrict__ perm, int P,
+                                                          int k, int nvec, uint4* __restrict__ xp) {
+  const int lane = threadIdx.x & 31;
+  const int wpb = blockDim.x >> 5;
+  for (int pos = blockIdx.x * wpb + (threadIdx.x >> 5); pos < P; pos += gridDim.x * wpb) {
+    const int t = perm[pos] / k;
+    const uint4* src = x + (size_t)t * nvec;
+    uint4* dst = xp + (size_t)pos * nvec;
+    for (int v = lane; v < nvec; v += 32) dst[v] = src[v];
+  }
+}
+
+// y[t, :] = sum_{j ascending} w[t,j] * O[inv[t,j], :]   (fp32, one bf16 rounding)
+__global__ void __launch_bounds__(256) combine_kernel(const uint4* __restrict__ O,
+                                                      const int32_t* __restrict__ inv,
+                                                      const float* __restrict__ w, int T, int k,
+                                                      int nvec, uint4* __restrict__ y) {
+  const int lane = threadIdx.x & 31;
+  const int wpb = blockDim.x >> 5;
+  for (int t = blockIdx.x * wpb + (threadIdx.x >> 5); t < T; t += gridDim.x * wpb) {
+    int pos[8];
+    float wj[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      pos[j] = j < k ? inv[(size_t)t * k + j] : 0;
+      wj[j] = j < k ? w[(size_t)t * k + j] : 0.f;
+    }
+    for (int v = lane; v < nvec; v += 32) {
+      float acc[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        if (j < k) {
+          const uint4 raw = O[(size_t)pos[j] * nvec + v];
+          const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&raw);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const float2 f = __bfloat1622float2(p[i]);
+            acc[2 * i] = fmaf(wj[j], f.x, acc[2 * i]);
+            acc[2 * i + 1] = fmaf(wj[j], f.y, acc[2 * i + 1]);
+          }
+        }
+      }
+      uint4 out;
+      out.x = pack_bf16x2(acc[0], acc[1]);
+      out.y = pack_bf16x2(acc[2], acc[3]);
+      out.z = pack_bf16x2(acc[4], acc[5]);
+      out.w = pack_bf16x2(acc[6], acc[7]);
+      y[(size_t)t * nvec + v] = out;
+    }
+  }
+}
+
+}  // namespace moe

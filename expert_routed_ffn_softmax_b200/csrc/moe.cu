@@ -1,0 +1,425 @@
+// moe.cu -- the C ABI of include/moe.h: argument checks, workspace layout, TMA tensor
+// maps and the launch sequence router -> dispatch -> GEMM-1 (+GEGLU) -> GEMM-2 -> combine.
+// All kernels live in this one translation unit so that they share the device error word.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "moe.h"
+#include "ptx.cuh"
+#include "router.cuh"
+#include "dispatch.cuh"
+#include "grouped_gemm.cuh"
+
+namespace moe {
+namespace {
+
+constexpr int kGemmStages = 4;
+constexpr int kMaxDevices = 64;
+
+size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
+
+bool shape_supported(int T, int H, int E, int I, int k, bool need_I) {
+  if (T < 1 || T > 1048576) return false;
+  if (H < 64 || H > 16384 || H % 64) return false;
+  if (need_I && (I < 64 || I > 8192 || I % 64)) return false;
+  if (E < 4 || E > 256 || E % 4 || (E > 128 && E % 8)) return false;
+  if (k < 1 || k > 8 || k > E) return false;
+  return true;
+}
+
+// Split of the router's H axis over CTAs: a divisor d of H/4 with 64 <= H/d <= 1408 (the
+// per-CTA x stage stays within 88 KB), the smallest one that gives ~2 CTAs per SM.
+int router_ksplit(int T, int H) {
+  const int ntg = (T + kRouterTokens - 1) / kRouterTokens;
+  const int target = (296 + ntg - 1) / ntg;
+  int first = -1, largest = -1;
+  for (int d = 1; d <= H / 4; ++d) {
+    if ((H / 4) % d) continue;
+    const int hs = H / d;
+    if (hs < 64 || hs > 1408) continue;
+    largest = d;
+    if (first < 0 && d >= target) first = d;
+  }
+  return first > 0 ? first : largest;
+}
+
+struct Layout {
+  int ks = 0, hs = 0, nchunks = 0, max_tiles = 0;
+  size_t part_logit = 0, part_xn2 = 0, part_wn2 = 0, n_exact = 0, ids = 0, wts = 0;
+  size_t chunk_counts = 0, chunk_base = 0, counts = 0, offsets = 0, perm = 0, inv = 0;
+  size_t tile_num = 0, tile_expert = 0, tile_row0 = 0, tile_rows = 0;
+  size_t xp = 0, hbuf = 0, obuf = 0;
+  size_t total = 0;
+};
+
+Layout make_layout(int T, int H, int E, int I, int k, bool forward) {
+  Layout L;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t at = off;
+    off = align256(off + bytes);
+    return at;
+  };
+  L.ks = router_ksplit(T, H);
+  L.hs = H / L.ks;
+  const size_t P = (size_t)T * k;
+  L.part_logit = take(sizeof(double) * L.ks * (size_t)T * E);
+  L.part_xn2 = take(sizeof(double) * L.ks * (size_t)T);
+  L.part_wn2 = take(sizeof(double) * L.ks * (size_t)E);
+  L.n_exact = take(sizeof(unsigned));
+  if (forward) {
+    L.nchunks = (int)((P + kDispatchChunk - 1) / kDispatchChunk);
+    L.max_tiles = (int)(P / GM_BM) + E;
+    L.ids = take(sizeof(int32_t) * P);
+    L.wts = take(sizeof(float) * P);
+    L.chunk_counts = take(sizeof(int32_t) * (size_t)L.nchunks * E);
+    L.chunk_base = take(sizeof(int32_t) * (size_t)L.nchunks * E);
+    L.counts = take(sizeof(int32_t) * E);
+    L.offsets = take(sizeof(int32_t) * (E + 1));
+    L.perm = take(sizeof(int32_t) * P);
+    L.inv = take(sizeof(int32_t) * P);
+    L.tile_num = take(sizeof(int32_t));
+    L.tile_expert = take(sizeof(int32_t) * L.max_tiles);
+    L.tile_row0 = take(sizeof(int32_t) * L.max_tiles);
+    L.tile_rows = take(sizeof(int32_t) * L.max_tiles);
+    L.xp = take(2 * P * H);
+    L.hbuf = take(2 * P * I);
+    L.obuf = take(2 * P * H);
+  }
+  L.total = off;
+  return L;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// --------------------------------------------------------------------------- TMA maps
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// Row-major [rows][cols] bf16, box = 64 columns x box_rows rows, 128-byte swizzle.
+bool make_map_2d(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, uint32_t box_rows) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * 2};
+  cuuint32_t box[2] = {64, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Stacked [E][rows][cols] bf16 (cols contiguous), box = 64 columns x 64 rows x 1 expert.
+bool make_map_3d(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, uint64_t E) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {cols, rows, E};
+  cuuint64_t strides[2] = {cols * 2, cols * rows * 2};
+  cuuint32_t box[3] = {64, 64, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// --------------------------------------------------------------------------- per device
+struct DeviceState {
+  bool attrs_set = false;
+  int num_sms = 0;
+  cudaEvent_t ev[8] = {};
+  int n_profiled = -1;
+};
+DeviceState g_dev[kMaxDevices];
+std::mutex g_dev_mu;
+
+const char* kStageNames[] = {"router", "dispatch", "gemm1_geglu", "gemm2_down", "combine"};
+constexpr int kNumStages = 5;
+
+DeviceState* device_state(int* dev_out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  *dev_out = dev;
+  std::lock_guard<std::mutex> lk(g_dev_mu);
+  DeviceState& d = g_dev[dev];
+  if (!d.attrs_set) {
+    cudaDeviceGetAttribute(&d.num_sms, cudaDevAttrMultiProcessorCount, dev);
+    const int gs = gemm_smem_bytes<kGemmStages>();
+    if (cudaFuncSetAttribute(grouped_gemm_kernel<kGemmStages, EPI_GEGLU>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, gs) != cudaSuccess ||
+        cudaFuncSetAttribute(grouped_gemm_kernel<kGemmStages, EPI_STORE>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, gs) != cudaSuccess ||
+        cudaFuncSetAttribute(router_partial_kernel<4>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, 1408 * 8 * 8) !=
+            cudaSuccess ||
+        cudaFuncSetAttribute(router_partial_kernel<8>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, 1408 * 8 * 8) !=
+            cudaSuccess)
+      return nullptr;
+    for (auto& e : d.ev)
+      if (cudaEventCreate(&e) != cudaSuccess) return nullptr;
+    d.attrs_set = true;
+  }
+  return &d;
+}
+
+struct Profiler {
+  DeviceState* d;
+  cudaStream_t st;
+  bool on;
+  int n = 0;
+  void mark() {
+    if (on) cudaEventRecord(d->ev[n++], st);
+  }
+  void finish() {
+    if (on) d->n_profiled = n - 1;
+  }
+};
+
+moe_status_t launched() {
+  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+moe_status_t launch_router(const __nv_bfloat16* x, const __nv_bfloat16* wr, const float* bias,
+                           int T, int H, int E, int k, unsigned flags, int32_t* ids, float* wts,
+                           uint8_t* ws, const Layout& L, const DeviceState& d, cudaStream_t st) {
+  double* part_logit = reinterpret_cast<double*>(ws + L.part_logit);
+  double* part_xn2 = reinterpret_cast<double*>(ws + L.part_xn2);
+  double* part_wn2 = reinterpret_cast<double*>(ws + L.part_wn2);
+  unsigned* n_exact = reinterpret_cast<unsigned*>(ws + L.n_exact);
+  const dim3 g1((T + kRouterTokens - 1) / kRouterTokens, L.ks);
+  const size_t sm1 =
+      sizeof(double) * std::max<size_t>((size_t)L.hs * kRouterTokens, (size_t)kRouterWarps * kRouterTokens * E);
+  if (E <= 128)
+    router_partial_kernel<4><<<g1, 128, sm1, st>>>(x, wr, T, H, E, L.hs, part_logit, part_xn2,
+                                                   part_wn2);
+  else
+    router_partial_kernel<8><<<g1, 128, sm1, st>>>(x, wr, T, H, E, L.hs, part_logit, part_xn2,
+                                                   part_wn2);
+  if (launched() != MOE_OK) return MOE_ERR_CUDA;
+  if (cudaMemsetAsync(n_exact, 0, sizeof(unsigned), st) != cudaSuccess) return MOE_ERR_CUDA;
+  const double u = std::ldexp(1.0, -53);
+  const double n = (double)H + 8.0;
+  const double gamma = n * u / (1.0 - n * u);
+  const double beta_scale = 2.0 * gamma * 1.01;
+  const int renorm = (flags & MOE_FLAG_NO_RENORM) ? 0 : 1;
+  const int g2 = std::min((T + 7) / 8, std::max(1, d.num_sms) * 8);
+  if (E <= 128)
+    router_select_kernel<4><<<g2, 256, 0, st>>>(part_logit, part_xn2, part_wn2, L.ks, bias, x, wr,
+                                                T, H, E, k, renorm, beta_scale, ids, wts, n_exact);
+  else
+    router_select_kernel<8><<<g2, 256, 0, st>>>(part_logit, part_xn2, part_wn2, L.ks, bias, x, wr,
+                                                T, H, E, k, renorm, beta_scale, ids, wts, n_exact);
+  return launched();
+}
+
+__global__ void unsatisfied_wait_kernel() {
+  __shared__ __align__(8) uint64_t bar;
+  const uint32_t b = smem_u32(&bar);
+  mbar_init(b, 1);
+  fence_barrier_init();
+  mbar_wait(b, 0);  // nothing arrives: runs out after the wait limit and raises the error
+}
+
+}  // namespace
+}  // namespace moe
+
+using namespace moe;
+
+extern "C" {
+
+int moe_abi_version(void) { return MOE_ABI_VERSION; }
+
+const char* moe_status_string(moe_status_t s) {
+  switch (s) {
+    case MOE_OK: return "MOE_OK";
+    case MOE_ERR_INVALID_ARG: return "MOE_ERR_INVALID_ARG";
+    case MOE_ERR_UNSUPPORTED: return "MOE_ERR_UNSUPPORTED";
+    case MOE_ERR_NO_WORKSPACE: return "MOE_ERR_NO_WORKSPACE";
+    case MOE_ERR_CUDA: return "MOE_ERR_CUDA";
+    case MOE_ERR_TIMEOUT: return "MOE_ERR_TIMEOUT";
+  }
+  return "MOE_ERR_UNKNOWN";
+}
+
+size_t moe_route_workspace_size(int T, int H, int E, int k, unsigned flags) {
+  (void)flags;
+  if (!shape_supported(T, H, E, 64, k, false)) return 0;
+  return make_layout(T, H, E, 64, k, false).total;
+}
+
+size_t moe_workspace_size(int T, int H, int E, int I, int k, unsigned flags) {
+  (void)flags;
+  if (!shape_supported(T, H, E, I, k, true)) return 0;
+  return make_layout(T, H, E, I, k, true).total;
+}
+
+moe_status_t moe_route(const void* x, const void* w_router, const float* router_bias, int T,
+                       int H, int E, int k, unsigned flags, int32_t* topk_ids,
+                       float* topk_weights, void* workspace, size_t workspace_bytes,
+                       void* stream) {
+  if (T < 0 || H <= 0 || E <= 0 || k < 1 || k > E) return MOE_ERR_INVALID_ARG;
+  if (flags & ~(unsigned)(MOE_FLAG_NO_RENORM | MOE_FLAG_PROFILE_STAGES)) return MOE_ERR_INVALID_ARG;
+  if (T == 0) return MOE_OK;
+  if (!x || !w_router || !topk_ids || !topk_weights || !workspace) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(w_router) || !aligned16(workspace)) return MOE_ERR_INVALID_ARG;
+  if (!shape_supported(T, H, E, 64, k, false)) return MOE_ERR_UNSUPPORTED;
+  const Layout L = make_layout(T, H, E, 64, k, false);
+  if (workspace_bytes < L.total) return MOE_ERR_NO_WORKSPACE;
+  int dev = 0;
+  DeviceState* d = device_state(&dev);
+  if (!d) return MOE_ERR_CUDA;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  return launch_router(static_cast<const __nv_bfloat16*>(x),
+                       static_cast<const __nv_bfloat16*>(w_router), router_bias, T, H, E, k, flags,
+                       topk_ids, topk_weights, static_cast<uint8_t*>(workspace), L, *d, st);
+}
+
+moe_status_t moe_forward(const void* x, const void* w_router, const float* router_bias,
+                         const void* w_gate, const void* w_up, const void* w_down, int T, int H,
+                         int E, int I, int k, unsigned flags, void* y, const moe_aux_t* aux,
+                         void* workspace, size_t workspace_bytes, void* stream) {
+  if (T < 0 || H <= 0 || E <= 0 || I <= 0 || k < 1 || k > E) return MOE_ERR_INVALID_ARG;
+  if (flags & ~(unsigned)(MOE_FLAG_NO_RENORM | MOE_FLAG_PROFILE_STAGES)) return MOE_ERR_INVALID_ARG;
+  if (T == 0) return MOE_OK;
+  if (!x || !w_router || !w_gate || !w_up || !w_down || !y || !workspace)
+    return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(w_router) || !aligned16(w_gate) || !aligned16(w_up) ||
+      !aligned16(w_down) || !aligned16(y) || !aligned16(workspace))
+    return MOE_ERR_INVALID_ARG;
+  if (x == y) return MOE_ERR_INVALID_ARG;
+  if (!shape_supported(T, H, E, I, k, true)) return MOE_ERR_UNSUPPORTED;
+  const Layout L = make_layout(T, H, E, I, k, true);
+  if (workspace_bytes < L.total) return MOE_ERR_NO_WORKSPACE;
+  int dev = 0;
+  DeviceState* d = device_state(&dev);
+  if (!d) return MOE_ERR_CUDA;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  const int P = T * k;
+
+  int32_t* ids = (aux && aux->topk_ids) ? aux->topk_ids : reinterpret_cast<int32_t*>(ws + L.ids);
+  float* wts = (aux && aux->topk_weights) ? aux->topk_weights : reinterpret_cast<float*>(ws + L.wts);
+  int32_t* counts =
+      (aux && aux->expert_counts) ? aux->expert_counts : reinterpret_cast<int32_t*>(ws + L.counts);
+  int32_t* offsets = (aux && aux->expert_offsets) ? aux->expert_offsets
+                                                  : reinterpret_cast<int32_t*>(ws + L.offsets);
+  int32_t* perm = (aux && aux->perm) ? aux->perm : reinterpret_cast<int32_t*>(ws + L.perm);
+  int32_t* inv = reinterpret_cast<int32_t*>(ws + L.inv);
+  int32_t* chunk_counts = reinterpret_cast<int32_t*>(ws + L.chunk_counts);
+  int32_t* chunk_base = reinterpret_cast<int32_t*>(ws + L.chunk_base);
+  int32_t* tile_num = reinterpret_cast<int32_t*>(ws + L.tile_num);
+  int32_t* tile_expert = reinterpret_cast<int32_t*>(ws + L.tile_expert);
+  int32_t* tile_row0 = reinterpret_cast<int32_t*>(ws + L.tile_row0);
+  int32_t* tile_rows = reinterpret_cast<int32_t*>(ws + L.tile_rows);
+  __nv_bfloat16* xp = reinterpret_cast<__nv_bfloat16*>(ws + L.xp);
+  __nv_bfloat16* hbuf = reinterpret_cast<__nv_bfloat16*>(ws + L.hbuf);
+  __nv_bfloat16* obuf = reinterpret_cast<__nv_bfloat16*>(ws + L.obuf);
+
+  CUtensorMap tm_xp, tm_wg, tm_wu, tm_h, tm_wd;
+  if (!make_map_2d(&tm_xp, xp, H, P, GM_BM) || !make_map_3d(&tm_wg, w_gate, I, H, E) ||
+      !make_map_3d(&tm_wu, w_up, I, H, E) || !make_map_2d(&tm_h, hbuf, I, P, GM_BM) ||
+      !make_map_3d(&tm_wd, w_down, H, I, E))
+    return MOE_ERR_CUDA;
+
+  Profiler prof{d, st, (flags & MOE_FLAG_PROFILE_STAGES) != 0};
+  prof.mark();
+  // 1. router
+  moe_status_t s = launch_router(static_cast<const __nv_bfloat16*>(x),
+                                 static_cast<const __nv_bfloat16*>(w_router), router_bias, T, H,
+                                 E, k, flags, ids, wts, ws, L, *d, st);
+  if (s != MOE_OK) return s;
+  prof.mark();
+  // 2. dispatch
+  dispatch_count_kernel<<<L.nchunks, 256, E * sizeof(int), st>>>(ids, P, E, chunk_counts);
+  dispatch_scan_kernel<<<1, 256, 0, st>>>(chunk_counts, L.nchunks, E, P, GM_BM, counts, offsets,
+                                          chunk_base, tile_num, tile_expert, tile_row0, tile_rows);
+  dispatch_rank_kernel<<<L.nchunks, 32, E * sizeof(int), st>>>(ids, P, E, chunk_base, perm, inv);
+  const int gsm = std::max(1, d->num_sms) * 8;
+  gather_rows_kernel<<<std::min((P + 7) / 8, gsm), 256, 0, st>>>(
+      static_cast<const uint4*>(x), perm, P, k, H / 8, reinterpret_cast<uint4*>(xp));
+  if (launched() != MOE_OK) return MOE_ERR_CUDA;
+  prof.mark();
+  // 3. GEMM-1 + GEGLU
+  const TileList tl{tile_num, tile_expert, tile_row0, tile_rows};
+  const int smem = gemm_smem_bytes<kGemmStages>();
+  const int n1 = (I + 127) / 128;
+  grouped_gemm_kernel<kGemmStages, EPI_GEGLU>
+      <<<n1 * L.max_tiles, 128, smem, st>>>(tm_xp, tm_wg, tm_wu, tl, n1, H, I, hbuf, I);
+  if (launched() != MOE_OK) return MOE_ERR_CUDA;
+  prof.mark();
+  // 4. GEMM-2 (down)
+  const int n2 = (H + 255) / 256;
+  grouped_gemm_kernel<kGemmStages, EPI_STORE>
+      <<<n2 * L.max_tiles, 128, smem, st>>>(tm_h, tm_wd, tm_wd, tl, n2, I, H, obuf, H);
+  if (launched() != MOE_OK) return MOE_ERR_CUDA;
+  prof.mark();
+  // 5. combine
+  combine_kernel<<<std::min((T + 7) / 8, gsm), 256, 0, st>>>(reinterpret_cast<const uint4*>(obuf),
+                                                            inv, wts, T, k, H / 8,
+                                                            static_cast<uint4*>(y));
+  if (launched() != MOE_OK) return MOE_ERR_CUDA;
+  prof.mark();
+  prof.finish();
+  return MOE_OK;
+}
+
+moe_status_t moe_sync_status(void* stream) {
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return MOE_ERR_CUDA;
+  unsigned w = 0;
+  if (cudaMemcpyFromSymbol(&w, g_error_word, sizeof w) != cudaSuccess) return MOE_ERR_CUDA;
+  if (w) {
+    const unsigned zero = 0;
+    if (cudaMemcpyToSymbol(g_error_word, &zero, sizeof zero) != cudaSuccess) return MOE_ERR_CUDA;
+  }
+  if (w & MOE_DEVERR_TIMEOUT) return MOE_ERR_TIMEOUT;
+  if (w) return MOE_ERR_CUDA;
+  return MOE_OK;
+}
+
+int moe_last_stage_times(float* ms, int n) {
+  int dev = 0;
+  DeviceState* d = device_state(&dev);
+  if (!d || d->n_profiled < 0) return -1;
+  const int ns = d->n_profiled;
+  if (cudaEventSynchronize(d->ev[ns]) != cudaSuccess) return -1;
+  for (int i = 0; i < ns && i < n; ++i) {
+    float t = 0.f;
+    cudaEventElapsedTime(&t, d->ev[i], d->ev[i + 1]);
+    ms[i] = t;
+  }
+  return ns;
+}
+
+const char* moe_stage_name(int i) {
+  return (i >= 0 && i < kNumStages) ? kStageNames[i] : "";
+}
+
+moe_status_t moe_debug_set_wait_limit_ns(unsigned long long ns) {
+  const unsigned long long v = ns ? ns : 2000000000ull;
+  return cudaMemcpyToSymbol(g_wait_limit_ns, &v, sizeof v) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+moe_status_t moe_debug_unsatisfied_wait(void* stream) {
+  unsatisfied_wait_kernel<<<1, 1, 0, static_cast<cudaStream_t>(stream)>>>();
+  return launched();
+}
+
+}  // extern "C"

@@ -1,0 +1,156 @@
+/*
+ * moe.h -- C ABI of the B200 (sm_100a) routed Mixture-of-Experts FFN layer.
+ *
+ * The layer is the MoE block of Gemma-4-26B-A4B: hidden H = 2816 in bf16, E = 128
+ * experts, top-k = 8 softmax routing, expert intermediate I = 704, GEGLU with the tanh
+ * form of GELU (cann-recipes-infer "Gemma-4-26B-A4B 模型优化报告" §1 模型概况 and §5 阶段3
+ * 融合算子 "MoE Router npu_moe_gating_top_k_softmax"; Gemma-4-26B-A4B-NVFP4 Ascend
+ * verification report §2.1 模型架构参数).  The shapes are runtime arguments; the limits
+ * each call accepts are listed below.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - Pointers marked (device) are CUDA device pointers OWNED BY THE CALLER; the library
+ *    never frees them and allocates nothing on the call path.  They must be 16-byte
+ *    aligned.  Arrays are dense and row-major in the layout stated at each argument.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = the legacy default stream).  All
+ *    work is enqueued asynchronously on it; a call returns before the GPU finishes.
+ *  - Argument errors are detected on the host before anything is launched and return
+ *    MOE_ERR_INVALID_ARG (null required pointer, negative size, k < 1, k > E,
+ *    misaligned pointer) or MOE_ERR_UNSUPPORTED (a shape outside the limits below).
+ *    T == 0 returns MOE_OK and launches nothing.
+ *  - A launch failure returns MOE_ERR_CUDA.  Device-side faults detected by the kernels
+ *    themselves (a bounded wait that ran out, an out-of-range index read from memory)
+ *    set a per-device error word; moe_sync_status() synchronises the stream, reads and
+ *    clears it, and returns MOE_ERR_TIMEOUT / MOE_ERR_CUDA.
+ *  - Inputs must be finite.  Calls on distinct workspaces may run concurrently.
+ *
+ * Shape limits (MOE_ERR_UNSUPPORTED otherwise):
+ *    1 <= T <= 1048576;  64 <= H <= 16384, H % 64 == 0;  64 <= I <= 8192, I % 64 == 0;
+ *    4 <= E <= 256, E % 4 == 0;  1 <= k <= min(8, E).
+ */
+#ifndef MOE_B200_H
+#define MOE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define MOE_ABI_VERSION 1
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = 1,
+  MOE_ERR_UNSUPPORTED = 2,
+  MOE_ERR_NO_WORKSPACE = 3,
+  MOE_ERR_CUDA = 4,
+  MOE_ERR_TIMEOUT = 5
+} moe_status_t;
+
+enum {
+  /* Return the raw softmax probabilities of the k selected experts instead of
+   * renormalising them to sum to one (renormalisation is the default). */
+  MOE_FLAG_NO_RENORM = 1u << 0,
+  /* Record a CUDA event at every stage boundary of the call; moe_last_stage_times()
+   * then reports the per-stage device times of the most recent such call. */
+  MOE_FLAG_PROFILE_STAGES = 1u << 3
+};
+
+/* Optional caller-owned device outputs of moe_forward (any member may be NULL). */
+typedef struct {
+  int32_t *expert_counts;  /* [E]    pairs routed to each expert ("split sizes")     */
+  int32_t *expert_offsets; /* [E+1]  exclusive scan of expert_counts                  */
+  int32_t *perm;           /* [T*k]  expert-sorted position -> pair index t*k+j       */
+  int32_t *topk_ids;       /* [T*k]  as moe_route                                     */
+  float *topk_weights;     /* [T*k]  as moe_route                                     */
+} moe_aux_t;
+
+/* ABI version of the loaded library (MOE_ABI_VERSION at build time). */
+int moe_abi_version(void);
+
+/* Human-readable name of a status code (static storage, never NULL). */
+const char *moe_status_string(moe_status_t s);
+
+/* Bytes of device workspace moe_route / moe_forward need for these sizes (0 when the
+ * shape is unsupported).  The workspace is caller-owned, 256-byte aligned device memory;
+ * its contents need no initialisation and are scratch between calls. */
+size_t moe_route_workspace_size(int T, int H, int E, int k, unsigned flags);
+size_t moe_workspace_size(int T, int H, int E, int I, int k, unsigned flags);
+
+/*
+ * moe_route -- the router: logits, softmax, top-k, renormalisation
+ * (optimisation report §5, "MoE Router npu_moe_gating_top_k_softmax"; top-8 of 128, §1).
+ *
+ *   logits   L[t,e] = sum_h x[t,h] * w_router[h,e] + router_bias[e]
+ *   ids      the k experts with the largest L[t,:], slot 0 largest, equal logits ordered
+ *            by the lower expert id.  The ranking is decided on values that agree with
+ *            a double-precision ascending-order sum of the exact bf16 products, so it is
+ *            reproducible bit for bit.
+ *   weights  p = softmax over all E logits; w_j = p[id_j] / sum_i p[id_i]
+ *            (or p[id_j] with MOE_FLAG_NO_RENORM).
+ *
+ *   x            (device) bf16 [T, H]
+ *   w_router     (device) bf16 [H, E]   (E contiguous)
+ *   router_bias  (device) fp32 [E], or NULL for no bias
+ *   topk_ids     (device) int32 [T, k]  output
+ *   topk_weights (device) fp32  [T, k]  output
+ *   workspace    (device) >= moe_route_workspace_size(T,H,E,k,flags) bytes, else
+ *                MOE_ERR_NO_WORKSPACE
+ */
+moe_status_t moe_route(const void *x, const void *w_router, const float *router_bias, int T,
+                       int H, int E, int k, unsigned flags, int32_t *topk_ids,
+                       float *topk_weights, void *workspace, size_t workspace_bytes,
+                       void *stream);
+
+/*
+ * moe_forward -- the whole routed FFN layer: route, dispatch, expert FFNs, combine.
+ *
+ *   route     as moe_route
+ *   dispatch  counts[e], offsets = exclusive scan, and a stable permutation that groups the
+ *             (token, slot) pairs expert by expert in ascending token order (the per-expert
+ *             "split sizes" of the double_routing dispatch, optimisation report §6.1)
+ *   expert e  h = gelu_tanh(x W_gate[e]) * (x W_up[e]);  o = h W_down[e]
+ *             (GEGLU, intermediate 704, §1; gelu_pytorch_tanh, verification report §2.1;
+ *             computed as a grouped matmul, the role of SwiftGMM in "MoE推理「王炸」组合：
+ *             昇腾×盘古让推理性能狂飙6-8倍", Group 4)
+ *   combine   y[t] = sum_j w[t,j] * o_{t,j}
+ *   Precision: bf16 operands, fp32 accumulation; h, o and y are rounded to bf16.
+ *
+ *   x, w_router, router_bias  as moe_route
+ *   w_gate, w_up  (device) bf16 [E, H, I]  (I contiguous)
+ *   w_down        (device) bf16 [E, I, H]  (H contiguous)
+ *   y             (device) bf16 [T, H]  output (may not alias x)
+ *   aux           NULL, or optional extra outputs (see moe_aux_t)
+ *   workspace     (device) >= moe_workspace_size(T,H,E,I,k,flags) bytes
+ */
+moe_status_t moe_forward(const void *x, const void *w_router, const float *router_bias,
+                         const void *w_gate, const void *w_up, const void *w_down, int T, int H,
+                         int E, int I, int k, unsigned flags, void *y, const moe_aux_t *aux,
+                         void *workspace, size_t workspace_bytes, void *stream);
+
+/* Synchronise `stream`, then read and clear this device's error word.
+ * MOE_OK, MOE_ERR_TIMEOUT (a bounded device wait ran out), or MOE_ERR_CUDA (a CUDA error,
+ * or an out-of-range index seen by a kernel). */
+moe_status_t moe_sync_status(void *stream);
+
+/* Stage timing of the most recent call made with MOE_FLAG_PROFILE_STAGES on this host
+ * thread's current device.  Synchronises on that call's last event.  Writes up to n
+ * per-stage times in milliseconds to ms (host) and returns the number of stages, or -1
+ * when no profiled call has been made.  moe_stage_name(i) names stage i. */
+int moe_last_stage_times(float *ms, int n);
+const char *moe_stage_name(int i);
+
+/* Testing aid for the failure path: set the wall-clock limit (ns) of every bounded wait
+ * in later launches on the current device (0 restores the default of 2 s), and launch a
+ * kernel that waits on a barrier nothing will ever complete, so that its bounded wait
+ * runs out and raises MOE_ERR_TIMEOUT in moe_sync_status().  No other state is touched. */
+moe_status_t moe_debug_set_wait_limit_ns(unsigned long long ns);
+moe_status_t moe_debug_unsatisfied_wait(void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MOE_B200_H */

@@ -1,0 +1,91 @@
+"""The C ABI without a GPU: the library loads, exports every function include/moe.h
+declares, and rejects bad arguments on the host before touching the device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from expert_routed_ffn_softmax_b200 import _abi, build
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(__file__)), "include", "moe.h")
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"^\s*[\w\s\*]*?\b(moe_\w+)\s*\(", src, flags=re.M)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return _abi.load()
+
+
+def test_header_declares_the_documented_calls():
+    names = declared_functions()
+    for n in ("moe_route", "moe_forward", "moe_workspace_size", "moe_route_workspace_size",
+              "moe_status_string", "moe_sync_status"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    names = declared_functions()
+    assert names
+    for n in names:
+        assert hasattr(lib, n), n
+        assert n in _abi.SIGNATURES, f"binding lacks {n}"
+
+
+def test_abi_version_and_status_strings(lib):
+    assert lib.moe_abi_version() == 1
+    assert _abi.status_string(0) == "MOE_OK"
+    assert _abi.status_string(5) == "MOE_ERR_TIMEOUT"
+    assert _abi.status_string(99) == "MOE_ERR_UNKNOWN"
+
+
+def test_workspace_sizes(lib):
+    small = lib.moe_workspace_size(8, 2816, 128, 704, 8, 0)
+    big = lib.moe_workspace_size(2048, 2816, 128, 704, 8, 0)
+    assert 0 < small < big
+    # Xp + Hbuf + O dominate: 2 bytes x pairs x (2H + I)
+    assert big >= 2 * 2048 * 8 * (2 * 2816 + 704)
+    assert lib.moe_workspace_size(8, 2816, 128, 700, 8, 0) == 0     # I % 64 != 0
+    assert lib.moe_workspace_size(8, 2800, 128, 704, 8, 0) == 0     # H % 64 != 0
+    assert lib.moe_workspace_size(8, 2816, 128, 704, 9, 0) == 0     # k > 8
+    assert lib.moe_workspace_size(8, 2816, 260, 704, 8, 0) == 0     # E > 256
+    assert lib.moe_route_workspace_size(8, 2816, 128, 8, 0) > 0
+    assert lib.moe_route_workspace_size(8, 2816, 6, 8, 0) == 0      # k > E
+
+
+FAKE = 1 << 20   # an aligned non-null address; never dereferenced (host checks fail first)
+
+
+def test_host_argument_checks(lib):
+    f = lib.moe_forward
+    ok = (FAKE, FAKE, None, FAKE, FAKE, FAKE)
+    # T == 0: nothing to do
+    assert f(*ok, 0, 2816, 128, 704, 8, 0, FAKE + 4096, None, FAKE, 1 << 30, None) == 0
+    # null required pointer
+    assert f(None, FAKE, None, FAKE, FAKE, FAKE, 8, 2816, 128, 704, 8, 0, FAKE + 4096, None,
+             FAKE, 1 << 30, None) == _abi.MOE_ERR_INVALID_ARG
+    # k > E, negative T, unknown flag
+    assert f(*ok, 8, 2816, 4, 704, 8, 0, FAKE + 4096, None, FAKE, 1 << 30, None) == 1
+    assert f(*ok, -1, 2816, 128, 704, 8, 0, FAKE + 4096, None, FAKE, 1 << 30, None) == 1
+    assert f(*ok, 8, 2816, 128, 704, 8, 1 << 7, FAKE + 4096, None, FAKE, 1 << 30, None) == 1
+    # misaligned pointer
+    assert f(FAKE + 2, *ok[1:], 8, 2816, 128, 704, 8, 0, FAKE + 4096, None, FAKE, 1 << 30,
+             None) == 1
+    # y aliasing x
+    assert f(*ok, 8, 2816, 128, 704, 8, 0, FAKE, None, FAKE, 1 << 30, None) == 1
+    # unsupported shape
+    assert f(*ok, 8, 2816, 128, 700, 8, 0, FAKE + 4096, None, FAKE, 1 << 30, None) == \
+        _abi.MOE_ERR_UNSUPPORTED
+    # too little workspace
+    assert f(*ok, 8, 2816, 128, 704, 8, 0, FAKE + 4096, None, FAKE, 1024, None) == \
+        _abi.MOE_ERR_NO_WORKSPACE
+    r = lib.moe_route
+    assert r(FAKE, FAKE, None, 8, 2816, 128, 8, 0, FAKE, FAKE, FAKE, 16, None) == \
+        _abi.MOE_ERR_NO_WORKSPACE
+    assert r(FAKE, None, None, 8, 2816, 128, 8, 0, FAKE, FAKE, FAKE, 1 << 30, None) == 1
