@@ -64,6 +64,8 @@ __global__ void __launch_bounds__(128, 1)
   const int tile = blockIdx.x / n_blocks;
   const int nb = blockIdx.x - tile * n_blocks;
   if (tile >= *tiles.num) return;
+  // After a device-side timeout anywhere, skip the work until the host clears the word.
+  if (*reinterpret_cast<volatile unsigned*>(&g_error_word) & MOE_DEVERR_TIMEOUT) return;
   const int e = tiles.expert[tile];
   const int row0 = tiles.row0[tile];
   const int rows = tiles.rows[tile];
