@@ -51,58 +51,66 @@ def peaks() -> dict:
 
 # ----------------------------------------------------------------------------- clocks
 class ClockSampler:
-    """nvidia-smi clock/throttle samples while the timed region runs."""
+    """SM clock and clock-event reasons sampled through NVML every few ms while the timed
+    region runs (reads only; nothing is set)."""
 
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown"}
 
-    def __init__(self, gpu_index: int):
-        self.idx = gpu_index
-        self.proc = None
-        self.lines: list[str] = []
+    def __init__(self, device: torch.device, period_s: float = 0.005):
+        self.period = period_s
+        self.samples: list[tuple[float, int, int]] = []
+        self.h = None
+        try:
+            import pynvml as nv
+            nv.nvmlInit()
+            p = torch.cuda.get_device_properties(device)
+            bus = f"{p.pci_domain_id:08X}:{p.pci_bus_id:02X}:{p.pci_device_id:02X}.0"
+            self.nv = nv
+            self.h = nv.nvmlDeviceGetHandleByPciBusId(bus)
+            self.max_mhz = nv.nvmlDeviceGetMaxClockInfo(self.h, nv.NVML_CLOCK_SM)
+        except Exception:   # no NVML: the line carries "clocks": null
+            self.h = None
+
+    def _reasons(self) -> int:
+        nv = self.nv
+        fn = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            nv.nvmlDeviceGetCurrentClocksThrottleReasons
+        return int(fn(self.h))
+
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append((time.perf_counter(),
+                                     nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM),
+                                     self._reasons()))
+            except Exception:
+                pass
+            time.sleep(self.period)
 
     def start(self):
-        try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "200"],
-                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-            self.t = threading.Thread(target=self._read, daemon=True)
-            self.t.start()
-        except OSError:
-            self.proc = None
-
-    def _read(self):
-        for line in self.proc.stdout:
-            self.lines.append(line.strip())
+        if self.h is None:
+            return
+        self._stop = threading.Event()
+        self.t = threading.Thread(target=self._run, daemon=True)
+        self.t.start()
 
     def stop(self) -> dict | None:
-        if self.proc is None:
+        if self.h is None:
             return None
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except subprocess.TimeoutExpired:
-            self.proc.kill()
-        sm, mx, reasons = [], 0.0, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
-            f = [s.strip() for s in ln.split(",")]
-            if len(f) < 9:
-                continue
-            try:
-                sm.append(float(f[1]))
-                mx = max(mx, float(f[2]))
-            except ValueError:
-                continue
-            for n, v in zip(names, f[5:9]):
-                if v.lower().startswith("active"):
-                    reasons.add(n)
-        if not sm:
+        self._stop.set()
+        self.t.join()
+        if not self.samples:
             return None
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
-                "samples": len(sm)}
+        sm = [s[1] for s in self.samples]
+        reasons = set()
+        for _, _, r in self.samples:
+            for bit, name in self.REASONS.items():
+                if r & bit:
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(reasons), "samples": len(sm), "source": "nvml"}
 
 
 # ----------------------------------------------------------------------------- accounting
@@ -127,7 +135,7 @@ def algorithmic(cfg: wl.MoEConfig, counts: np.ndarray, has_bias: bool) -> dict:
 
 def kernel_source_sha() -> str:
     h = hashlib.sha256()
-    for f in ("grouped_gemm.cuh", "ptx.cuh", "moe.cu"):
+    for f in ("grouped_gemm.cuh", "ptx.cuh"):
         h.update(open(os.path.join(ROOT, "expert_routed_ffn_softmax_b200", "csrc", f), "rb").read())
     return h.hexdigest()[:16]
 
@@ -187,12 +195,12 @@ def run_reference(args, cfg) -> None:
     print(json.dumps(line), flush=True)
 
 
-def cpu_baseline(cfg, d, budget_s: float) -> dict:
+def cpu_baseline(cfg, d, x_all, budget_s: float) -> dict:
     import oracle
     cores = len(os.sched_getaffinity(0))
     oracle.set_threads(cores)
     T_s = min(cfg.T, 64)
-    x = d["x"][:T_s].contiguous()
+    x = x_all[:T_s].contiguous()
     n, t_total = 0, 0.0
     while t_total < budget_s or n == 0:
         t0 = time.perf_counter()
@@ -229,11 +237,6 @@ def run_native(args, cfg) -> None:
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
 
-    def fwd(xx, out=None, profile=False):
-        return moe.forward(xx, g["w_router"], g["w_gate"], g["w_up"], g["w_down"], cfg.k,
-                           bias=g["bias"], out=out, profile=profile)
-
-    y = torch.empty((cfg.T, cfg.H), dtype=torch.bfloat16, device=dev)
     y0, aux = moe.forward(x, g["w_router"], g["w_gate"], g["w_up"], g["w_down"], cfg.k,
                           bias=g["bias"], aux=True)
     if moe.sync_status() != 0:
@@ -241,15 +244,20 @@ def run_native(args, cfg) -> None:
     counts = aux["expert_counts"].cpu().numpy()
     acc = algorithmic(cfg, counts, d["bias"] is not None)
 
+    # The step as a serving loop runs it: one captured moe_forward per batch (graph replay).
+    graph = moe.ForwardGraph(x, g["w_router"], g["w_gate"], g["w_up"], g["w_down"], cfg.k,
+                             bias=g["bias"])
     for _ in range(args.warmup):
         flush.zero_()
-        fwd(x, y)
+        graph.replay()
     torch.cuda.synchronize()
+    if not torch.equal(graph.y, y0):
+        raise SystemExit("graph replay differs from the direct call")
 
     # ---- timed region: K steps, L2 flushed (untimed) before each
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
           for _ in range(args.steps)]
-    clocks = ClockSampler(local)
+    clocks = ClockSampler(dev)
     clocks.start()
     if dist:
         dist.barrier()
@@ -257,7 +265,7 @@ def run_native(args, cfg) -> None:
     for i in range(args.steps):
         flush.zero_()
         ev[i][0].record(stream)
-        fwd(x, y)
+        graph.replay()
         ev[i][1].record(stream)
     torch.cuda.synchronize()
     if dist:
@@ -268,28 +276,30 @@ def run_native(args, cfg) -> None:
     if moe.sync_status() != 0:
         raise SystemExit("device status not OK after the timed steps")
 
-    # ---- per-stage device times (same calls with stage events), L2 flushed before each
+    # ---- per-stage device times: a graph of the same call with the library's stage events
+    pgraph = moe.ForwardGraph(x, g["w_router"], g["w_gate"], g["w_up"], g["w_down"], cfg.k,
+                              bias=g["bias"], profile=True)
     stage_acc: dict[str, list[float]] = {}
     for _ in range(max(3, min(args.steps, 20))):
         flush.zero_()
-        fwd(x, y, profile=True)
+        pgraph.replay()
         for k, v in moe.last_stage_times().items():
             stage_acc.setdefault(k, []).append(v)
     stages = {k: sum(v) / len(v) for k, v in stage_acc.items()}
+    del pgraph
 
     # ---- end to end through the public API with host buffers (pinned), L2 flushed
     x_host = x_cpu.pin_memory()
     y_host = torch.empty((cfg.T, cfg.H), dtype=torch.bfloat16).pin_memory()
-    x_dev = torch.empty_like(x)
     e2e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
               for _ in range(args.steps)]
     for i in range(args.warmup + args.steps):
         flush.zero_()
         if i >= args.warmup:
             e2e_ev[i - args.warmup][0].record(stream)
-        x_dev.copy_(x_host, non_blocking=True)
-        fwd(x_dev, y)
-        y_host.copy_(y, non_blocking=True)
+        graph.x.copy_(x_host, non_blocking=True)
+        graph.replay()
+        y_host.copy_(graph.y, non_blocking=True)
         if i >= args.warmup:
             e2e_ev[i - args.warmup][1].record(stream)
     torch.cuda.synchronize()
@@ -354,7 +364,7 @@ def run_native(args, cfg) -> None:
             "step_ms_p10_p50_p90": [float(np.percentile(step_ms, q)) for q in (10, 50, 90)],
         }
         if not args.no_cpu_baseline:
-            line["cpu_baseline"] = cpu_baseline(cfg, d, args.cpu_seconds)
+            line["cpu_baseline"] = cpu_baseline(cfg, d, x_cpu, args.cpu_seconds)
         print(json.dumps(line), flush=True)
     if dist:
         dist.barrier()

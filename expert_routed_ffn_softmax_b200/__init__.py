@@ -4,13 +4,14 @@ The public calls mirror the C ABI of include/moe.h:
 
     ids, weights = route(x, w_router, k, bias=None, renorm=True)
     y            = forward(x, w_router, w_gate, w_up, w_down, k, bias=None, renorm=True)
+    g            = ForwardGraph(x, w_router, w_gate, w_up, w_down, k); y = g.replay()
 
 x, weights and outputs are CUDA tensors (bf16 operands, int32 ids, fp32 routing weights);
 all arithmetic runs in libmoe_b200.so.  ``workloads`` (seeded synthetic inputs) can be
 imported without a GPU.
 """
-from ._abi import (MoEError, forward, last_stage_times, load, route, status_string,  # noqa: F401
-                   sync_status)
+from ._abi import (ForwardGraph, MoEError, forward, last_stage_times, load, route,  # noqa: F401
+                   status_string, sync_status)
 
-__all__ = ["route", "forward", "sync_status", "last_stage_times", "load", "status_string",
-           "MoEError"]
+__all__ = ["route", "forward", "ForwardGraph", "sync_status", "last_stage_times", "load",
+           "status_string", "MoEError"]

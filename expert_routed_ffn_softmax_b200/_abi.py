@@ -138,8 +138,11 @@ def route(x: torch.Tensor, w_router: torch.Tensor, k: int, bias: torch.Tensor | 
 def forward(x: torch.Tensor, w_router: torch.Tensor, w_gate: torch.Tensor, w_up: torch.Tensor,
             w_down: torch.Tensor, k: int, bias: torch.Tensor | None = None, renorm: bool = True,
             aux: bool = False, out: torch.Tensor | None = None, profile: bool = False,
-            stream=None):
-    """The routed MoE FFN layer -> y bf16 [T,H] (and a dict of routing outputs if aux)."""
+            stream=None, workspace_buf: torch.Tensor | None = None):
+    """The routed MoE FFN layer -> y bf16 [T,H] (and a dict of routing outputs if aux).
+
+    workspace_buf: optional caller-owned uint8 CUDA tensor used as the workspace (else a
+    per-device buffer cached by this module, which may be reallocated by a later call)."""
     L = load()
     T, H = x.shape
     E, _, I = w_gate.shape
@@ -164,14 +167,21 @@ def forward(x: torch.Tensor, w_router: torch.Tensor, w_gate: torch.Tensor, w_up:
             "topk_weights": torch.empty((T, k), dtype=torch.float32, device=dev),
         }
         a = AuxOut(*(aux_d[n].data_ptr() for n, _ in AuxOut._fields_))
-    nbytes = L.moe_workspace_size(T, H, E, I, k, flags) if T > 0 else 0
-    if T > 0 and nbytes == 0:
-        raise MoEError(MOE_ERR_UNSUPPORTED, "moe_workspace_size")
-    ws = workspace(nbytes, dev)
+    nbytes = workspace_bytes(T, H, E, I, k, flags)
+    ws = workspace(nbytes, dev) if workspace_buf is None else workspace_buf
     _check(L.moe_forward(px, pr, pb, pg, pu, pd, T, H, E, I, k, flags, py,
                          None if a is None else ctypes.byref(a), ws.data_ptr(), ws.numel(),
                          _stream_ptr(stream)), "moe_forward")
     return (y, aux_d) if aux else y
+
+
+def workspace_bytes(T: int, H: int, E: int, I: int, k: int, flags: int = 0) -> int:
+    if T == 0:
+        return 0
+    n = load().moe_workspace_size(T, H, E, I, k, flags)
+    if n == 0:
+        raise MoEError(MOE_ERR_UNSUPPORTED, "moe_workspace_size")
+    return n
 
 
 def sync_status(stream=None) -> int:
@@ -186,3 +196,36 @@ def last_stage_times() -> dict[str, float]:
     if n < 0:
         raise RuntimeError("no profiled moe_forward call yet")
     return {L.moe_stage_name(i).decode(): float(buf[i]) for i in range(n)}
+
+
+class ForwardGraph:
+    """One moe_forward captured in a CUDA graph for fixed shapes and buffers.
+
+    The layer is asynchronous, allocation-free and makes no host synchronisation on its
+    call path, so a captured call replays exactly: inputs are read from, and y is written
+    to, the same device buffers every replay (copy new activations into ``self.x``).  The
+    library's one-time device set-up runs in the warm-up call before capture.  The graph
+    owns its workspace.  profile=True records the library's stage events in every replay
+    (read them with last_stage_times()).
+    """
+
+    def __init__(self, x, w_router, w_gate, w_up, w_down, k, bias=None, renorm=True,
+                 profile=False):
+        self.x = x
+        T, H = x.shape
+        E, _, I = w_gate.shape
+        self.y = torch.empty((T, H), dtype=torch.bfloat16, device=x.device)
+        flags = MOE_FLAG_PROFILE_STAGES if profile else 0
+        self.workspace = torch.empty(max(1, workspace_bytes(T, H, E, I, k, flags)),
+                                     dtype=torch.uint8, device=x.device)
+        self._args = (w_router, w_gate, w_up, w_down, k)
+        self._kw = dict(bias=bias, renorm=renorm, profile=profile, workspace_buf=self.workspace)
+        forward(self.x, *self._args, out=self.y, **self._kw)    # set-up + workspace, uncaptured
+        torch.cuda.synchronize(x.device)
+        self.graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(self.graph):
+            forward(self.x, *self._args, out=self.y, **self._kw)
+
+    def replay(self) -> torch.Tensor:
+        self.graph.replay()
+        return self.y

@@ -112,6 +112,98 @@ __global__ void __launch_bounds__(32) dispatch_rank_kernel(const int32_t* __rest
   }
 }
 
+// Whole dispatch for a batch of at most one chunk (P <= kDispatchChunk) in one CTA of 256
+// threads: histogram, scan, tile list and the stable ranks, as the kernels above compute
+// them for many chunks.
+__global__ void __launch_bounds__(256) dispatch_small_kernel(
+    const int32_t* __restrict__ ids, int P, int E, int BM, int32_t* __restrict__ counts,
+    int32_t* __restrict__ offsets, int32_t* __restrict__ perm, int32_t* __restrict__ inv,
+    int32_t* __restrict__ tile_num, int32_t* __restrict__ tile_expert,
+    int32_t* __restrict__ tile_row0, int32_t* __restrict__ tile_rows) {
+  // s_base: running rank base per expert (advanced by the ranking warp); s_off stays the
+  // expert's first row for the tile list, which other threads build at the same time.
+  __shared__ int s_cnt[256], s_off[256], s_base[256], s_tstart[256];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  s_cnt[tid] = 0;
+  __syncthreads();
+  for (int q = tid; q < P; q += blockDim.x) {
+    const int e = ids[q];
+    if ((unsigned)e < (unsigned)E)
+      atomicAdd(&s_cnt[e], 1);
+    else
+      raise_error(MOE_DEVERR_BAD_INDEX);
+  }
+  __syncthreads();
+  if (warp == 0) {
+    // exclusive scans of counts and of tiles per expert; lane owns experts 8*lane..8*lane+7
+    int c[8], nt[8], cs = 0, ts = 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int e = lane * 8 + i;
+      c[i] = e < E ? s_cnt[e] : 0;
+      nt[i] = (c[i] + BM - 1) / BM;
+      cs += c[i];
+      ts += nt[i];
+    }
+    int ci = cs, ti = ts;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int a = __shfl_up_sync(0xffffffffu, ci, off);
+      const int b = __shfl_up_sync(0xffffffffu, ti, off);
+      if (lane >= off) {
+        ci += a;
+        ti += b;
+      }
+    }
+    int o = ci - cs, tt = ti - ts;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int e = lane * 8 + i;
+      if (e < E) {
+        s_off[e] = o;
+        s_base[e] = o;
+        s_tstart[e] = tt;
+        counts[e] = c[i];
+        offsets[e] = o;
+      }
+      o += c[i];
+      tt += nt[i];
+    }
+    if (lane == 31) {
+      offsets[E] = o;
+      *tile_num = tt;
+    }
+  }
+  __syncthreads();
+  if (tid < E) {
+    const int n = s_cnt[tid], off = s_off[tid], nt = (n + BM - 1) / BM;
+    for (int m = 0; m < nt; ++m) {
+      const int i = s_tstart[tid] + m;
+      tile_expert[i] = tid;
+      tile_row0[i] = off + m * BM;
+      tile_rows[i] = min(BM, n - m * BM);
+    }
+  }
+  if (warp == 0) {
+    const unsigned lt = (1u << lane) - 1u;
+    for (int qb = 0; qb < P; qb += 32) {
+      const int q = qb + lane;
+      int e = q < P ? ids[q] : -1;
+      if (q < P && (unsigned)e >= (unsigned)E) e = -2;
+      const unsigned grp = __match_any_sync(0xffffffffu, e);
+      int pos = 0;
+      if (e >= 0) pos = s_base[e] + __popc(grp & lt);
+      __syncwarp();
+      if (e >= 0 && lane == 31 - __clz(grp)) s_base[e] += __popc(grp);
+      __syncwarp();
+      if (e >= 0) {
+        perm[pos] = q;
+        inv[q] = pos;
+      }
+    }
+  }
+}
+
 // Xp[pos, :] = x[perm[pos] / k, :]   (16-byte vectors; one warp per row, grid-stride)
 __global__ void __launch_bounds__(256) gather_rows_kernel(const uint4* __restrict__ x,
                                                           const int32_t* __restrict__ perm, int P,
@@ -127,13 +219,15 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const uint4* __restric
 }
 
 // y[t, :] = sum_{j ascending} w[t,j] * O[inv[t,j], :]   (fp32, one bf16 rounding)
+// One thread per 8-element vector of y; the k rows it reads are loaded back to back.
 __global__ void __launch_bounds__(256) combine_kernel(const uint4* __restrict__ O,
                                                       const int32_t* __restrict__ inv,
                                                       const float* __restrict__ w, int T, int k,
                                                       int nvec, uint4* __restrict__ y) {
-  const int lane = threadIdx.x & 31;
-  const int wpb = blockDim.x >> 5;
-  for (int t = blockIdx.x * wpb + (threadIdx.x >> 5); t < T; t += gridDim.x * wpb) {
+  const size_t total = (size_t)T * nvec;
+  for (size_t idx = (size_t)blockIdx.x * blockDim.x + threadIdx.x; idx < total;
+       idx += (size_t)gridDim.x * blockDim.x) {
+    const int t = (int)(idx / nvec), v = (int)(idx - (size_t)t * nvec);
     int pos[8];
     float wj[8];
 #pragma unroll
@@ -141,7 +235,7 @@ __global__ void __launch_bounds__(256) combine_kernel(const uint4* __restrict__ 
       pos[j] = j < k ? inv[(size_t)t * k + j] : 0;
       wj[j] = j < k ? w[(size_t)t * k + j] : 0.f;
     }
-    for (int v = lane; v < nvec; v += 32) {
+    {
       float acc[8];
 #pragma unroll
       for (int i = 0; i < 8; ++i) acc[i] = 0.f;

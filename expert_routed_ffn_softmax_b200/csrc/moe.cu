@@ -348,10 +348,17 @@ moe_status_t moe_forward(const void* x, const void* w_router, const float* route
   if (s != MOE_OK) return s;
   prof.mark();
   // 2. dispatch
-  dispatch_count_kernel<<<L.nchunks, 256, E * sizeof(int), st>>>(ids, P, E, chunk_counts);
-  dispatch_scan_kernel<<<1, 256, 0, st>>>(chunk_counts, L.nchunks, E, P, GM_BM, counts, offsets,
-                                          chunk_base, tile_num, tile_expert, tile_row0, tile_rows);
-  dispatch_rank_kernel<<<L.nchunks, 32, E * sizeof(int), st>>>(ids, P, E, chunk_base, perm, inv);
+  if (L.nchunks == 1) {
+    dispatch_small_kernel<<<1, 256, 0, st>>>(ids, P, E, GM_BM, counts, offsets, perm, inv,
+                                             tile_num, tile_expert, tile_row0, tile_rows);
+  } else {
+    dispatch_count_kernel<<<L.nchunks, 256, E * sizeof(int), st>>>(ids, P, E, chunk_counts);
+    dispatch_scan_kernel<<<1, 256, 0, st>>>(chunk_counts, L.nchunks, E, P, GM_BM, counts,
+                                            offsets, chunk_base, tile_num, tile_expert, tile_row0,
+                                            tile_rows);
+    dispatch_rank_kernel<<<L.nchunks, 32, E * sizeof(int), st>>>(ids, P, E, chunk_base, perm,
+                                                                 inv);
+  }
   const int gsm = std::max(1, d->num_sms) * 8;
   gather_rows_kernel<<<std::min((P + 7) / 8, gsm), 256, 0, st>>>(
       static_cast<const uint4*>(x), perm, P, k, H / 8, reinterpret_cast<uint4*>(xp));
@@ -372,7 +379,9 @@ moe_status_t moe_forward(const void* x, const void* w_router, const float* route
   if (launched() != MOE_OK) return MOE_ERR_CUDA;
   prof.mark();
   // 5. combine
-  combine_kernel<<<std::min((T + 7) / 8, gsm), 256, 0, st>>>(reinterpret_cast<const uint4*>(obuf),
+  const long long cthreads = (long long)T * (H / 8);
+  combine_kernel<<<(int)std::min<long long>((cthreads + 255) / 256, gsm), 256, 0, st>>>(
+      reinterpret_cast<const uint4*>(obuf),
                                                             inv, wts, T, k, H / 8,
                                                             static_cast<uint4*>(y));
   if (launched() != MOE_OK) return MOE_ERR_CUDA;

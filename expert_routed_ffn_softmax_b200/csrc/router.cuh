@@ -209,20 +209,39 @@ __global__ void __launch_bounds__(256) router_select_kernel(
   const int warps_per_block = blockDim.x >> 5;
   for (int t = blockIdx.x * warps_per_block + (threadIdx.x >> 5); t < T;
        t += gridDim.x * warps_per_block) {
+    // Partials are added in ascending split order.  The loads of 8 splits are issued
+    // before their adds so that the latency of a long split list is paid once per 8.
     double L[EPL], beta[EPL];
     double xn2 = 0.0;
-    for (int s = 0; s < ks; ++s) xn2 += part_xn2[(size_t)s * T + t];
+    for (int s0 = 0; s0 < ks; s0 += 8) {
+      double p[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) p[u] = (s0 + u < ks) ? part_xn2[(size_t)(s0 + u) * T + t] : 0.0;
+#pragma unroll
+      for (int u = 0; u < 8; ++u)
+        if (s0 + u < ks) xn2 += p[u];
+    }
 #pragma unroll
     for (int i = 0; i < EPL; ++i) {
       const int e = lane + 32 * i;
       L[i] = -DBL_MAX;
       beta[i] = 0.0;
       if (e < E) {
-        double v = part_logit[(size_t)t * E + e];
-        double wn2 = part_wn2[e];
-        for (int s = 1; s < ks; ++s) {
-          v += part_logit[((size_t)s * T + t) * E + e];
-          wn2 += part_wn2[(size_t)s * E + e];
+        double v = 0.0, wn2 = 0.0;
+        for (int s0 = 0; s0 < ks; s0 += 8) {
+          double p[8], q[8];
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            const bool in = s0 + u < ks;
+            p[u] = in ? part_logit[((size_t)(s0 + u) * T + t) * E + e] : 0.0;
+            q[u] = in ? part_wn2[(size_t)(s0 + u) * E + e] : 0.0;
+          }
+#pragma unroll
+          for (int u = 0; u < 8; ++u)
+            if (s0 + u < ks) {
+              v = (s0 + u == 0) ? p[u] : v + p[u];
+              wn2 += q[u];
+            }
         }
         const double b = bias ? (double)bias[e] : 0.0;
         if (bias) v += b;

@@ -173,3 +173,18 @@ def test_bounded_wait_reports_timeout_and_context_survives(gemma_w):
     finally:
         assert lib.moe_debug_set_wait_limit_ns(0) == 0
     run_case(wl.CONFIGS["decode"], gemma_w, 10**9)                 # context still usable
+
+
+def test_graph_replay_matches_direct_call(gemma_w):
+    x, c, g = layer_inputs(wl.CONFIGS["decode"], gemma_w)
+    x = x.cuda()
+    y_direct = moe.forward(x, g["w_router"], g["w_gate"], g["w_up"], g["w_down"], 8)
+    fg = moe.ForwardGraph(x, g["w_router"], g["w_gate"], g["w_up"], g["w_down"], 8)
+    for _ in range(3):
+        assert torch.equal(fg.replay(), y_direct)
+    # new activations copied into the captured input buffer are picked up by the replay
+    x2 = wl.make_x(wl.CONFIGS["decode"], seed=7).cuda()
+    fg.x.copy_(x2)
+    y2 = fg.replay()
+    assert moe.sync_status() == 0
+    assert torch.equal(y2, moe.forward(x2, g["w_router"], g["w_gate"], g["w_up"], g["w_down"], 8))
