@@ -11,7 +11,7 @@ all arithmetic runs in libmoe_b200.so.  ``workloads`` (seeded synthetic inputs) 
 imported without a GPU.
 """
 from ._abi import (ForwardGraph, MoEError, forward, last_stage_times, load, route,  # noqa: F401
-                   status_string, sync_status)
+                   router_stats, status_string, sync_status)
 
 __all__ = ["route", "forward", "ForwardGraph", "sync_status", "last_stage_times", "load",
-           "status_string", "MoEError"]
+           "router_stats", "status_string", "MoEError"]

@@ -24,7 +24,11 @@ MOE_ERR_CUDA = 4
 MOE_ERR_TIMEOUT = 5
 
 MOE_FLAG_NO_RENORM = 1 << 0
+MOE_FLAG_ROUTER_FP64 = 1 << 1
+MOE_FLAG_ROUTER_SCREEN = 1 << 2
 MOE_FLAG_PROFILE_STAGES = 1 << 3
+
+_ROUTER_FLAGS = {"auto": 0, "fp64": MOE_FLAG_ROUTER_FP64, "screen": MOE_FLAG_ROUTER_SCREEN}
 
 # Every function the header declares, with (restype, argtypes).
 _P, _I, _U, _SZ = ctypes.c_void_p, ctypes.c_int, ctypes.c_uint, ctypes.c_size_t
@@ -51,7 +55,7 @@ class MoEError(RuntimeError):
 
 class AuxOut(ctypes.Structure):
     _fields_ = [("expert_counts", _P), ("expert_offsets", _P), ("perm", _P),
-                ("topk_ids", _P), ("topk_weights", _P)]
+                ("topk_ids", _P), ("topk_weights", _P), ("router_stats", _P)]
 
 
 _lib = None
@@ -113,9 +117,19 @@ def _dev(t: torch.Tensor, name: str, dtype: torch.dtype, shape: tuple) -> int:
     return t.data_ptr()
 
 
+def _flags(renorm: bool, router: str, profile: bool = False) -> int:
+    if router not in _ROUTER_FLAGS:
+        raise ValueError(f"router must be one of {sorted(_ROUTER_FLAGS)}")
+    return ((0 if renorm else MOE_FLAG_NO_RENORM) | _ROUTER_FLAGS[router]
+            | (MOE_FLAG_PROFILE_STAGES if profile else 0))
+
+
 def route(x: torch.Tensor, w_router: torch.Tensor, k: int, bias: torch.Tensor | None = None,
-          renorm: bool = True, stream=None):
-    """Router of the MoE layer -> (topk_ids int32 [T,k], topk_weights float32 [T,k])."""
+          renorm: bool = True, router: str = "auto", stream=None):
+    """Router of the MoE layer -> (topk_ids int32 [T,k], topk_weights float32 [T,k]).
+
+    router: "auto" (tensor-core screen + fp64 recheck for T >= 256, fp64 logits below),
+    "fp64" or "screen" to force a path; all give the same ids."""
     L = load()
     T, H = x.shape
     E = w_router.shape[1]
@@ -123,7 +137,7 @@ def route(x: torch.Tensor, w_router: torch.Tensor, k: int, bias: torch.Tensor | 
     px = _dev(x, "x", torch.bfloat16, (T, H))
     pw = _dev(w_router, "w_router", torch.bfloat16, (H, E))
     pb = None if bias is None else _dev(bias, "bias", torch.float32, (E,))
-    flags = 0 if renorm else MOE_FLAG_NO_RENORM
+    flags = _flags(renorm, router)
     ids = torch.empty((T, k), dtype=torch.int32, device=dev)
     wts = torch.empty((T, k), dtype=torch.float32, device=dev)
     nbytes = L.moe_route_workspace_size(T, H, E, k, flags) if T > 0 else 0
@@ -138,7 +152,7 @@ def route(x: torch.Tensor, w_router: torch.Tensor, k: int, bias: torch.Tensor | 
 def forward(x: torch.Tensor, w_router: torch.Tensor, w_gate: torch.Tensor, w_up: torch.Tensor,
             w_down: torch.Tensor, k: int, bias: torch.Tensor | None = None, renorm: bool = True,
             aux: bool = False, out: torch.Tensor | None = None, profile: bool = False,
-            stream=None, workspace_buf: torch.Tensor | None = None):
+            stream=None, workspace_buf: torch.Tensor | None = None, router: str = "auto"):
     """The routed MoE FFN layer -> y bf16 [T,H] (and a dict of routing outputs if aux).
 
     workspace_buf: optional caller-owned uint8 CUDA tensor used as the workspace (else a
@@ -155,7 +169,7 @@ def forward(x: torch.Tensor, w_router: torch.Tensor, w_gate: torch.Tensor, w_up:
     pb = None if bias is None else _dev(bias, "bias", torch.float32, (E,))
     y = torch.empty((T, H), dtype=torch.bfloat16, device=dev) if out is None else out
     py = _dev(y, "out", torch.bfloat16, (T, H))
-    flags = (0 if renorm else MOE_FLAG_NO_RENORM) | (MOE_FLAG_PROFILE_STAGES if profile else 0)
+    flags = _flags(renorm, router, profile)
     a = None
     aux_d = None
     if aux:
@@ -165,6 +179,7 @@ def forward(x: torch.Tensor, w_router: torch.Tensor, w_gate: torch.Tensor, w_up:
             "perm": torch.empty(T * k, dtype=torch.int32, device=dev),
             "topk_ids": torch.empty((T, k), dtype=torch.int32, device=dev),
             "topk_weights": torch.empty((T, k), dtype=torch.float32, device=dev),
+            "router_stats": torch.zeros(4, dtype=torch.int32, device=dev),
         }
         a = AuxOut(*(aux_d[n].data_ptr() for n, _ in AuxOut._fields_))
     nbytes = workspace_bytes(T, H, E, I, k, flags)
@@ -173,6 +188,16 @@ def forward(x: torch.Tensor, w_router: torch.Tensor, w_gate: torch.Tensor, w_up:
                          None if a is None else ctypes.byref(a), ws.data_ptr(), ws.numel(),
                          _stream_ptr(stream)), "moe_forward")
     return (y, aux_d) if aux else y
+
+
+def router_stats(aux: dict) -> dict:
+    """Decode aux["router_stats"] of a forward(..., aux=True) call."""
+    import struct
+    v = aux["router_stats"].cpu().tolist()
+    u = [x & 0xFFFFFFFF for x in v]
+    return {"candidates": u[0], "exact_recomputes": u[1],
+            "max_screen_err_ratio": struct.unpack("<f", struct.pack("<I", u[2]))[0],
+            "path": "screen" if u[3] == 1 else "fp64"}
 
 
 def workspace_bytes(T: int, H: int, E: int, I: int, k: int, flags: int = 0) -> int:
@@ -210,16 +235,17 @@ class ForwardGraph:
     """
 
     def __init__(self, x, w_router, w_gate, w_up, w_down, k, bias=None, renorm=True,
-                 profile=False):
+                 profile=False, router="auto"):
         self.x = x
         T, H = x.shape
         E, _, I = w_gate.shape
         self.y = torch.empty((T, H), dtype=torch.bfloat16, device=x.device)
-        flags = MOE_FLAG_PROFILE_STAGES if profile else 0
+        flags = _flags(renorm, router, profile)
         self.workspace = torch.empty(max(1, workspace_bytes(T, H, E, I, k, flags)),
                                      dtype=torch.uint8, device=x.device)
         self._args = (w_router, w_gate, w_up, w_down, k)
-        self._kw = dict(bias=bias, renorm=renorm, profile=profile, workspace_buf=self.workspace)
+        self._kw = dict(bias=bias, renorm=renorm, profile=profile, workspace_buf=self.workspace,
+                        router=router)
         forward(self.x, *self._args, out=self.y, **self._kw)    # set-up + workspace, uncaptured
         torch.cuda.synchronize(x.device)
         self.graph = torch.cuda.CUDAGraph()

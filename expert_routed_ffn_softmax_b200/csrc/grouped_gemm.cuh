@@ -26,26 +26,29 @@
 namespace moe {
 
 constexpr int GM_BM = 128;
-constexpr int GM_BN = 256;
 constexpr int GM_BK = 64;
 constexpr int GM_A_BYTES = GM_BM * GM_BK * 2;          // 16 KB
 constexpr int GM_SLAB_BYTES = GM_BK * 64 * 2;          // 8 KB: 64 K rows x 64 columns
-constexpr int GM_B_BYTES = 4 * GM_SLAB_BYTES;          // 32 KB
-constexpr int GM_STAGE_BYTES = GM_A_BYTES + GM_B_BYTES;
-constexpr uint32_t GM_TMEM_COLS = 256;
 
-enum { EPI_GEGLU = 0, EPI_STORE = 1 };
+// EPI_GEGLU: B = [gate | up] slabs, h = gelu_tanh(g) * u stored bf16 (N/2 columns out)
+// EPI_STORE: bf16 store of all N columns;  EPI_F32: fp32 store of all N columns.
+enum { EPI_GEGLU = 0, EPI_STORE = 1, EPI_F32 = 2 };
 
 struct TileList {
   const int32_t* num;     // [1] tiles in use
   const int32_t* expert;  // [cap]
   const int32_t* row0;    // [cap] first sorted row
   const int32_t* rows;    // [cap] rows in tile (1..128)
+  int uniform_rows;       // > 0: no list; tile m covers rows [128m, min(128m+128, uniform_rows)) of expert 0
 };
 
-template <int STAGES>
-constexpr int gemm_smem_bytes() {
-  return 1024 /*alignment slack*/ + STAGES * GM_STAGE_BYTES + 256 /*barriers*/;
+template <int NSLAB>
+__host__ __device__ constexpr int gemm_stage_bytes() {
+  return GM_A_BYTES + NSLAB * GM_SLAB_BYTES;
+}
+template <int STAGES, int NSLAB>
+__host__ __device__ constexpr int gemm_smem_bytes() {
+  return 1024 /*alignment slack*/ + STAGES * gemm_stage_bytes<NSLAB>() + 256 /*barriers*/;
 }
 
 __device__ __forceinline__ float gelu_tanh_f(float g) {
@@ -53,37 +56,49 @@ __device__ __forceinline__ float gelu_tanh_f(float g) {
   return 0.5f * g * (1.0f + tanh_approx(inner));
 }
 
-template <int STAGES, int MODE>
+template <int STAGES, int MODE, int NSLAB>
 __global__ void __launch_bounds__(128, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                         const __grid_constant__ CUtensorMap tmB0,
                         const __grid_constant__ CUtensorMap tmB1, TileList tiles, int n_blocks,
-                        int K, int N_total, __nv_bfloat16* __restrict__ out, int ldo) {
+                        int K, int N_total, void* __restrict__ out_ptr, int ldo) {
+  constexpr int BN = 64 * NSLAB;                       // MMA N
+  constexpr int STAGE_BYTES = gemm_stage_bytes<NSLAB>();
+  constexpr uint32_t TMEM_COLS = BN < 32 ? 32 : BN;
+  static_assert(MODE != EPI_GEGLU || NSLAB % 2 == 0, "GEGLU pairs gate and up slabs");
   // 1-D grid: n_blocks column blocks per row tile, column block fastest so that the CTAs
   // sharing one activation tile run together.
   const int tile = blockIdx.x / n_blocks;
   const int nb = blockIdx.x - tile * n_blocks;
-  if (tile >= *tiles.num) return;
+  int e, row0, rows;
+  if (tiles.uniform_rows > 0) {
+    if (tile * GM_BM >= tiles.uniform_rows) return;
+    e = 0;
+    row0 = tile * GM_BM;
+    rows = min(GM_BM, tiles.uniform_rows - row0);
+  } else {
+    if (tile >= *tiles.num) return;
+    e = tiles.expert[tile];
+    row0 = tiles.row0[tile];
+    rows = tiles.rows[tile];
+  }
   // After a device-side timeout anywhere, skip the work until the host clears the word.
   if (*reinterpret_cast<volatile unsigned*>(&g_error_word) & MOE_DEVERR_TIMEOUT) return;
-  const int e = tiles.expert[tile];
-  const int row0 = tiles.row0[tile];
-  const int rows = tiles.rows[tile];
-  // GEGLU: 128 output features per CTA; STORE: 256 output columns per CTA.
-  const int n0 = nb * (MODE == EPI_GEGLU ? 128 : 256);
+  // GEGLU: BN/2 output features per CTA; otherwise BN output columns per CTA.
+  const int n0 = nb * (MODE == EPI_GEGLU ? BN / 2 : BN);
 
   extern __shared__ uint8_t gsm_raw[];
   const uint32_t raw_addr = smem_u32(gsm_raw);
   const uint32_t base = (raw_addr + 1023u) & ~1023u;
   uint8_t* gsm = gsm_raw + (base - raw_addr);
-  const uint32_t bar_base = base + STAGES * GM_STAGE_BYTES;
+  const uint32_t bar_base = base + STAGES * STAGE_BYTES;
   auto full_bar = [&](int s) { return bar_base + 8u * s; };
   auto empty_bar = [&](int s) { return bar_base + 8u * (STAGES + s); };
   const uint32_t done_bar = bar_base + 8u * (2 * STAGES);
   volatile uint32_t* tmem_slot =
-      reinterpret_cast<volatile uint32_t*>(gsm + STAGES * GM_STAGE_BYTES + 8 * (2 * STAGES + 1));
+      reinterpret_cast<volatile uint32_t*>(gsm + STAGES * STAGE_BYTES + 8 * (2 * STAGES + 1));
   volatile int* abort_flag = reinterpret_cast<volatile int*>(
-      gsm + STAGES * GM_STAGE_BYTES + 8 * (2 * STAGES + 1) + 4);
+      gsm + STAGES * STAGE_BYTES + 8 * (2 * STAGES + 1) + 4);
   volatile int* n_issued = abort_flag + 1;
   volatile int* n_consumed = abort_flag + 2;
 
@@ -103,7 +118,7 @@ __global__ void __launch_bounds__(128, 1)
     tma_prefetch_desc(&tmB1);
   }
   if (warp == 0) {
-    tmem_alloc(smem_u32(const_cast<uint32_t*>(tmem_slot)), GM_TMEM_COLS);
+    tmem_alloc(smem_u32(const_cast<uint32_t*>(tmem_slot)), TMEM_COLS);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -122,25 +137,27 @@ __global__ void __launch_bounds__(128, 1)
         break;
       }
       if (*abort_flag) break;
-      const uint32_t sA = base + s * GM_STAGE_BYTES;
+      const uint32_t sA = base + s * STAGE_BYTES;
       const uint32_t sB = sA + GM_A_BYTES;
-      mbar_arrive_expect_tx(full_bar(s), GM_STAGE_BYTES);
+      mbar_arrive_expect_tx(full_bar(s), STAGE_BYTES);
       tma_load_2d(sA, &tmA, full_bar(s), kc * GM_BK, row0);
       if (MODE == EPI_GEGLU) {
-        tma_load_3d(sB + 0 * GM_SLAB_BYTES, &tmB0, full_bar(s), n0, kc * GM_BK, e);
-        tma_load_3d(sB + 1 * GM_SLAB_BYTES, &tmB0, full_bar(s), n0 + 64, kc * GM_BK, e);
-        tma_load_3d(sB + 2 * GM_SLAB_BYTES, &tmB1, full_bar(s), n0, kc * GM_BK, e);
-        tma_load_3d(sB + 3 * GM_SLAB_BYTES, &tmB1, full_bar(s), n0 + 64, kc * GM_BK, e);
+#pragma unroll
+        for (int j = 0; j < NSLAB / 2; ++j) {
+          tma_load_3d(sB + j * GM_SLAB_BYTES, &tmB0, full_bar(s), n0 + 64 * j, kc * GM_BK, e);
+          tma_load_3d(sB + (NSLAB / 2 + j) * GM_SLAB_BYTES, &tmB1, full_bar(s), n0 + 64 * j,
+                      kc * GM_BK, e);
+        }
       } else {
 #pragma unroll
-        for (int j = 0; j < 4; ++j)
+        for (int j = 0; j < NSLAB; ++j)
           tma_load_3d(sB + j * GM_SLAB_BYTES, &tmB0, full_bar(s), n0 + 64 * j, kc * GM_BK, e);
       }
       *n_issued = kc + 1;
     }
   } else if (warp == 1 && lane == 0) {
     // ---------------------------------------------------------------- MMA issuer
-    constexpr uint32_t idesc = idesc_bf16_f32(GM_BM, GM_BN, false, true);
+    constexpr uint32_t idesc = idesc_bf16_f32(GM_BM, BN, false, true);
     int kc = 0;
     for (; kc < nk; ++kc) {
       const int s = kc % STAGES;
@@ -150,7 +167,7 @@ __global__ void __launch_bounds__(128, 1)
       }
       *n_consumed = kc + 1;
       tc_fence_after();
-      const uint32_t sA = base + s * GM_STAGE_BYTES;
+      const uint32_t sA = base + s * STAGE_BYTES;
       const uint32_t sB = sA + GM_A_BYTES;
 #pragma unroll
       for (int kk = 0; kk < GM_BK / 16; ++kk) {
@@ -171,13 +188,13 @@ __global__ void __launch_bounds__(128, 1)
   const int r = warp * 32 + lane;
   const bool row_ok = store && r < rows;
   const uint32_t trow = tmem + (static_cast<uint32_t>(warp * 32) << 16);
-  __nv_bfloat16* orow = out + (size_t)(row0 + r) * ldo;
   if (MODE == EPI_GEGLU) {
+    __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(out_ptr) + (size_t)(row0 + r) * ldo;
 #pragma unroll 1
-    for (int c = 0; c < 128; c += 32) {
+    for (int c = 0; c < BN / 2; c += 32) {
       uint32_t g[32], u[32];
       tmem_ld_32x32b_x32(trow + c, g);
-      tmem_ld_32x32b_x32(trow + 128 + c, u);
+      tmem_ld_32x32b_x32(trow + BN / 2 + c, u);
       tmem_ld_wait();
       if (row_ok && n0 + c < N_total) {
         uint32_t pk[16];
@@ -194,9 +211,10 @@ __global__ void __launch_bounds__(128, 1)
           dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
       }
     }
-  } else {
+  } else if (MODE == EPI_STORE) {
+    __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(out_ptr) + (size_t)(row0 + r) * ldo;
 #pragma unroll 1
-    for (int c = 0; c < 256; c += 32) {
+    for (int c = 0; c < BN; c += 32) {
       uint32_t v[32];
       tmem_ld_32x32b_x32(trow + c, v);
       tmem_ld_wait();
@@ -211,6 +229,21 @@ __global__ void __launch_bounds__(128, 1)
           dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
       }
     }
+  } else {
+    float* orow = static_cast<float*>(out_ptr) + (size_t)(row0 + r) * ldo;
+#pragma unroll 1
+    for (int c = 0; c < BN; c += 32) {
+      uint32_t v[32];
+      tmem_ld_32x32b_x32(trow + c, v);
+      tmem_ld_wait();
+      if (row_ok) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+          if (n0 + c + 4 * i < N_total)
+            reinterpret_cast<uint4*>(orow + n0 + c)[i] =
+                make_uint4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+      }
+    }
   }
 
   // ------------------------------------------------------------------ teardown
@@ -223,7 +256,7 @@ __global__ void __launch_bounds__(128, 1)
   }
   __syncthreads();
   tc_fence_after();
-  if (warp == 0) tmem_dealloc(tmem, GM_TMEM_COLS);
+  if (warp == 0) tmem_dealloc(tmem, TMEM_COLS);
 }
 
 }  // namespace moe

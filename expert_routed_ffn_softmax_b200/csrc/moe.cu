@@ -22,6 +22,27 @@ namespace {
 
 constexpr int kGemmStages = 4;
 constexpr int kMaxDevices = 64;
+constexpr int kScreenMinTokens = 256;            // default router path switch
+constexpr double kScreenC = 1.0 / 1024.0;        // screen error bound / (|x| |w|)
+constexpr unsigned kKnownFlags = MOE_FLAG_NO_RENORM | MOE_FLAG_ROUTER_FP64 |
+                                 MOE_FLAG_ROUTER_SCREEN | MOE_FLAG_PROFILE_STAGES;
+
+#define GEMM_GEGLU grouped_gemm_kernel<kGemmStages, EPI_GEGLU, 4>
+#define GEMM_STORE grouped_gemm_kernel<kGemmStages, EPI_STORE, 4>
+#define GEMM_SCREEN grouped_gemm_kernel<kGemmStages, EPI_F32, 2>
+
+bool flags_ok(unsigned flags) {
+  if (flags & ~kKnownFlags) return false;
+  if ((flags & MOE_FLAG_ROUTER_FP64) && (flags & MOE_FLAG_ROUTER_SCREEN)) return false;
+  return true;
+}
+
+// Tensor-core screen + fp64 recheck, or fp64 logits for every expert.
+bool router_uses_screen(int T, unsigned flags) {
+  if (flags & (MOE_FLAG_NO_RENORM | MOE_FLAG_ROUTER_FP64)) return false;
+  if (flags & MOE_FLAG_ROUTER_SCREEN) return true;
+  return T >= kScreenMinTokens;
+}
 
 size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 
@@ -51,15 +72,17 @@ int router_ksplit(int T, int H) {
 }
 
 struct Layout {
+  bool screen = false;
   int ks = 0, hs = 0, nchunks = 0, max_tiles = 0;
-  size_t part_logit = 0, part_xn2 = 0, part_wn2 = 0, n_exact = 0, ids = 0, wts = 0;
+  size_t part_logit = 0, part_xn2 = 0, part_wn2 = 0, stats = 0, ids = 0, wts = 0;
+  size_t scr = 0, wrT = 0, wn2 = 0;
   size_t chunk_counts = 0, chunk_base = 0, counts = 0, offsets = 0, perm = 0, inv = 0;
   size_t tile_num = 0, tile_expert = 0, tile_row0 = 0, tile_rows = 0;
   size_t xp = 0, hbuf = 0, obuf = 0;
   size_t total = 0;
 };
 
-Layout make_layout(int T, int H, int E, int I, int k, bool forward) {
+Layout make_layout(int T, int H, int E, int I, int k, unsigned flags, bool forward) {
   Layout L;
   size_t off = 0;
   auto take = [&](size_t bytes) {
@@ -67,13 +90,20 @@ Layout make_layout(int T, int H, int E, int I, int k, bool forward) {
     off = align256(off + bytes);
     return at;
   };
-  L.ks = router_ksplit(T, H);
-  L.hs = H / L.ks;
   const size_t P = (size_t)T * k;
-  L.part_logit = take(sizeof(double) * L.ks * (size_t)T * E);
-  L.part_xn2 = take(sizeof(double) * L.ks * (size_t)T);
-  L.part_wn2 = take(sizeof(double) * L.ks * (size_t)E);
-  L.n_exact = take(sizeof(unsigned));
+  L.screen = router_uses_screen(T, flags);
+  L.stats = take(4 * sizeof(unsigned));
+  if (L.screen) {
+    L.scr = take(sizeof(float) * (size_t)T * E);
+    L.wrT = take(2 * (size_t)E * H);
+    L.wn2 = take(sizeof(double) * E);
+  } else {
+    L.ks = router_ksplit(T, H);
+    L.hs = H / L.ks;
+    L.part_logit = take(sizeof(double) * L.ks * (size_t)T * E);
+    L.part_xn2 = take(sizeof(double) * L.ks * (size_t)T);
+    L.part_wn2 = take(sizeof(double) * L.ks * (size_t)E);
+  }
   if (forward) {
     L.nchunks = (int)((P + kDispatchChunk - 1) / kDispatchChunk);
     L.max_tiles = (int)(P / GM_BM) + E;
@@ -161,11 +191,14 @@ DeviceState* device_state(int* dev_out) {
   DeviceState& d = g_dev[dev];
   if (!d.attrs_set) {
     cudaDeviceGetAttribute(&d.num_sms, cudaDevAttrMultiProcessorCount, dev);
-    const int gs = gemm_smem_bytes<kGemmStages>();
-    if (cudaFuncSetAttribute(grouped_gemm_kernel<kGemmStages, EPI_GEGLU>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, gs) != cudaSuccess ||
-        cudaFuncSetAttribute(grouped_gemm_kernel<kGemmStages, EPI_STORE>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, gs) != cudaSuccess ||
+    const int gs = gemm_smem_bytes<kGemmStages, 4>();
+    const int gs2 = gemm_smem_bytes<kGemmStages, 2>();
+    if (cudaFuncSetAttribute(GEMM_GEGLU, cudaFuncAttributeMaxDynamicSharedMemorySize, gs) !=
+            cudaSuccess ||
+        cudaFuncSetAttribute(GEMM_STORE, cudaFuncAttributeMaxDynamicSharedMemorySize, gs) !=
+            cudaSuccess ||
+        cudaFuncSetAttribute(GEMM_SCREEN, cudaFuncAttributeMaxDynamicSharedMemorySize, gs2) !=
+            cudaSuccess ||
         cudaFuncSetAttribute(router_partial_kernel<4>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, 1408 * 8 * 8) !=
             cudaSuccess ||
@@ -185,8 +218,11 @@ struct Profiler {
   cudaStream_t st;
   bool on;
   int n = 0;
+  // External records become event nodes when the call is captured into a CUDA graph, so
+  // every replay records the stage boundaries (a plain record would only be a capture
+  // dependency and never fire).
   void mark() {
-    if (on) cudaEventRecord(d->ev[n++], st);
+    if (on) cudaEventRecordWithFlags(d->ev[n++], st, cudaEventRecordExternal);
   }
   void finish() {
     if (on) d->n_profiled = n - 1;
@@ -199,14 +235,44 @@ moe_status_t launched() {
 
 moe_status_t launch_router(const __nv_bfloat16* x, const __nv_bfloat16* wr, const float* bias,
                            int T, int H, int E, int k, unsigned flags, int32_t* ids, float* wts,
-                           uint8_t* ws, const Layout& L, const DeviceState& d, cudaStream_t st) {
+                           unsigned* stats, uint8_t* ws, const Layout& L, const DeviceState& d,
+                           cudaStream_t st) {
+  if (cudaMemsetAsync(stats, 0, 4 * sizeof(unsigned), st) != cudaSuccess) return MOE_ERR_CUDA;
+  const double u = std::ldexp(1.0, -53);
+  const double n = (double)H + 8.0;
+  const double gamma = n * u / (1.0 - n * u);
+  const double beta_scale = 2.0 * gamma * 1.01;
+  const int renorm = (flags & MOE_FLAG_NO_RENORM) ? 0 : 1;
+  const int warps_blocks = std::min((T + 7) / 8, std::max(1, d.num_sms) * 8);
+  if (L.screen) {
+    float* scr = reinterpret_cast<float*>(ws + L.scr);
+    __nv_bfloat16* wrT = reinterpret_cast<__nv_bfloat16*>(ws + L.wrT);
+    double* wn2 = reinterpret_cast<double*>(ws + L.wn2);
+    router_transpose_kernel<<<dim3((H + 31) / 32, (E + 31) / 32), dim3(32, 8), 0, st>>>(wr, H, E,
+                                                                                      wrT);
+    router_wnorm_kernel<<<(E + 7) / 8, 256, 0, st>>>(wrT, H, E, wn2);
+    CUtensorMap tm_x, tm_wr;
+    if (!make_map_2d(&tm_x, x, H, T, GM_BM) || !make_map_3d(&tm_wr, wr, E, H, 1))
+      return MOE_ERR_CUDA;
+    const TileList tl{nullptr, nullptr, nullptr, nullptr, T};
+    const int nb = (E + 127) / 128;
+    const int mt = (T + GM_BM - 1) / GM_BM;
+    GEMM_SCREEN<<<nb * mt, 128, gemm_smem_bytes<kGemmStages, 2>(), st>>>(tm_x, tm_wr, tm_wr, tl,
+                                                                       nb, H, E, scr, E);
+    if (E <= 128)
+      router_screen_select_kernel<4><<<warps_blocks, 32 * kScreenWarps, 0, st>>>(
+          scr, x, wrT, wn2, bias, T, H, E, k, kScreenC, beta_scale, ids, wts, stats);
+    else
+      router_screen_select_kernel<8><<<warps_blocks, 32 * kScreenWarps, 0, st>>>(
+          scr, x, wrT, wn2, bias, T, H, E, k, kScreenC, beta_scale, ids, wts, stats);
+    return launched();
+  }
   double* part_logit = reinterpret_cast<double*>(ws + L.part_logit);
   double* part_xn2 = reinterpret_cast<double*>(ws + L.part_xn2);
   double* part_wn2 = reinterpret_cast<double*>(ws + L.part_wn2);
-  unsigned* n_exact = reinterpret_cast<unsigned*>(ws + L.n_exact);
   const dim3 g1((T + kRouterTokens - 1) / kRouterTokens, L.ks);
-  const size_t sm1 =
-      sizeof(double) * std::max<size_t>((size_t)L.hs * kRouterTokens, (size_t)kRouterWarps * kRouterTokens * E);
+  const size_t sm1 = sizeof(double) * std::max<size_t>((size_t)L.hs * kRouterTokens,
+                                                       (size_t)kRouterWarps * kRouterTokens * E);
   if (E <= 128)
     router_partial_kernel<4><<<g1, 128, sm1, st>>>(x, wr, T, H, E, L.hs, part_logit, part_xn2,
                                                    part_wn2);
@@ -214,19 +280,14 @@ moe_status_t launch_router(const __nv_bfloat16* x, const __nv_bfloat16* wr, cons
     router_partial_kernel<8><<<g1, 128, sm1, st>>>(x, wr, T, H, E, L.hs, part_logit, part_xn2,
                                                    part_wn2);
   if (launched() != MOE_OK) return MOE_ERR_CUDA;
-  if (cudaMemsetAsync(n_exact, 0, sizeof(unsigned), st) != cudaSuccess) return MOE_ERR_CUDA;
-  const double u = std::ldexp(1.0, -53);
-  const double n = (double)H + 8.0;
-  const double gamma = n * u / (1.0 - n * u);
-  const double beta_scale = 2.0 * gamma * 1.01;
-  const int renorm = (flags & MOE_FLAG_NO_RENORM) ? 0 : 1;
-  const int g2 = std::min((T + 7) / 8, std::max(1, d.num_sms) * 8);
   if (E <= 128)
-    router_select_kernel<4><<<g2, 256, 0, st>>>(part_logit, part_xn2, part_wn2, L.ks, bias, x, wr,
-                                                T, H, E, k, renorm, beta_scale, ids, wts, n_exact);
+    router_select_kernel<4><<<warps_blocks, 256, 0, st>>>(part_logit, part_xn2, part_wn2, L.ks,
+                                                          bias, x, wr, T, H, E, k, renorm,
+                                                          beta_scale, ids, wts, stats);
   else
-    router_select_kernel<8><<<g2, 256, 0, st>>>(part_logit, part_xn2, part_wn2, L.ks, bias, x, wr,
-                                                T, H, E, k, renorm, beta_scale, ids, wts, n_exact);
+    router_select_kernel<8><<<warps_blocks, 256, 0, st>>>(part_logit, part_xn2, part_wn2, L.ks,
+                                                          bias, x, wr, T, H, E, k, renorm,
+                                                          beta_scale, ids, wts, stats);
   return launched();
 }
 
@@ -260,15 +321,13 @@ const char* moe_status_string(moe_status_t s) {
 }
 
 size_t moe_route_workspace_size(int T, int H, int E, int k, unsigned flags) {
-  (void)flags;
-  if (!shape_supported(T, H, E, 64, k, false)) return 0;
-  return make_layout(T, H, E, 64, k, false).total;
+  if (!flags_ok(flags) || !shape_supported(T, H, E, 64, k, false)) return 0;
+  return make_layout(T, H, E, 64, k, flags, false).total;
 }
 
 size_t moe_workspace_size(int T, int H, int E, int I, int k, unsigned flags) {
-  (void)flags;
-  if (!shape_supported(T, H, E, I, k, true)) return 0;
-  return make_layout(T, H, E, I, k, true).total;
+  if (!flags_ok(flags) || !shape_supported(T, H, E, I, k, true)) return 0;
+  return make_layout(T, H, E, I, k, flags, true).total;
 }
 
 moe_status_t moe_route(const void* x, const void* w_router, const float* router_bias, int T,
@@ -276,12 +335,12 @@ moe_status_t moe_route(const void* x, const void* w_router, const float* router_
                        float* topk_weights, void* workspace, size_t workspace_bytes,
                        void* stream) {
   if (T < 0 || H <= 0 || E <= 0 || k < 1 || k > E) return MOE_ERR_INVALID_ARG;
-  if (flags & ~(unsigned)(MOE_FLAG_NO_RENORM | MOE_FLAG_PROFILE_STAGES)) return MOE_ERR_INVALID_ARG;
+  if (!flags_ok(flags)) return MOE_ERR_INVALID_ARG;
   if (T == 0) return MOE_OK;
   if (!x || !w_router || !topk_ids || !topk_weights || !workspace) return MOE_ERR_INVALID_ARG;
   if (!aligned16(x) || !aligned16(w_router) || !aligned16(workspace)) return MOE_ERR_INVALID_ARG;
   if (!shape_supported(T, H, E, 64, k, false)) return MOE_ERR_UNSUPPORTED;
-  const Layout L = make_layout(T, H, E, 64, k, false);
+  const Layout L = make_layout(T, H, E, 64, k, flags, false);
   if (workspace_bytes < L.total) return MOE_ERR_NO_WORKSPACE;
   int dev = 0;
   DeviceState* d = device_state(&dev);
@@ -289,7 +348,9 @@ moe_status_t moe_route(const void* x, const void* w_router, const float* router_
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   return launch_router(static_cast<const __nv_bfloat16*>(x),
                        static_cast<const __nv_bfloat16*>(w_router), router_bias, T, H, E, k, flags,
-                       topk_ids, topk_weights, static_cast<uint8_t*>(workspace), L, *d, st);
+                       topk_ids, topk_weights,
+                       reinterpret_cast<unsigned*>(static_cast<uint8_t*>(workspace) + L.stats),
+                       static_cast<uint8_t*>(workspace), L, *d, st);
 }
 
 moe_status_t moe_forward(const void* x, const void* w_router, const float* router_bias,
@@ -297,7 +358,7 @@ moe_status_t moe_forward(const void* x, const void* w_router, const float* route
                          int E, int I, int k, unsigned flags, void* y, const moe_aux_t* aux,
                          void* workspace, size_t workspace_bytes, void* stream) {
   if (T < 0 || H <= 0 || E <= 0 || I <= 0 || k < 1 || k > E) return MOE_ERR_INVALID_ARG;
-  if (flags & ~(unsigned)(MOE_FLAG_NO_RENORM | MOE_FLAG_PROFILE_STAGES)) return MOE_ERR_INVALID_ARG;
+  if (!flags_ok(flags)) return MOE_ERR_INVALID_ARG;
   if (T == 0) return MOE_OK;
   if (!x || !w_router || !w_gate || !w_up || !w_down || !y || !workspace)
     return MOE_ERR_INVALID_ARG;
@@ -306,7 +367,7 @@ moe_status_t moe_forward(const void* x, const void* w_router, const float* route
     return MOE_ERR_INVALID_ARG;
   if (x == y) return MOE_ERR_INVALID_ARG;
   if (!shape_supported(T, H, E, I, k, true)) return MOE_ERR_UNSUPPORTED;
-  const Layout L = make_layout(T, H, E, I, k, true);
+  const Layout L = make_layout(T, H, E, I, k, flags, true);
   if (workspace_bytes < L.total) return MOE_ERR_NO_WORKSPACE;
   int dev = 0;
   DeviceState* d = device_state(&dev);
@@ -322,6 +383,8 @@ moe_status_t moe_forward(const void* x, const void* w_router, const float* route
   int32_t* offsets = (aux && aux->expert_offsets) ? aux->expert_offsets
                                                   : reinterpret_cast<int32_t*>(ws + L.offsets);
   int32_t* perm = (aux && aux->perm) ? aux->perm : reinterpret_cast<int32_t*>(ws + L.perm);
+  unsigned* stats = (aux && aux->router_stats) ? aux->router_stats
+                                               : reinterpret_cast<unsigned*>(ws + L.stats);
   int32_t* inv = reinterpret_cast<int32_t*>(ws + L.inv);
   int32_t* chunk_counts = reinterpret_cast<int32_t*>(ws + L.chunk_counts);
   int32_t* chunk_base = reinterpret_cast<int32_t*>(ws + L.chunk_base);
@@ -344,7 +407,7 @@ moe_status_t moe_forward(const void* x, const void* w_router, const float* route
   // 1. router
   moe_status_t s = launch_router(static_cast<const __nv_bfloat16*>(x),
                                  static_cast<const __nv_bfloat16*>(w_router), router_bias, T, H,
-                                 E, k, flags, ids, wts, ws, L, *d, st);
+                                 E, k, flags, ids, wts, stats, ws, L, *d, st);
   if (s != MOE_OK) return s;
   prof.mark();
   // 2. dispatch
@@ -365,17 +428,15 @@ moe_status_t moe_forward(const void* x, const void* w_router, const float* route
   if (launched() != MOE_OK) return MOE_ERR_CUDA;
   prof.mark();
   // 3. GEMM-1 + GEGLU
-  const TileList tl{tile_num, tile_expert, tile_row0, tile_rows};
-  const int smem = gemm_smem_bytes<kGemmStages>();
+  const TileList tl{tile_num, tile_expert, tile_row0, tile_rows, 0};
+  const int smem = gemm_smem_bytes<kGemmStages, 4>();
   const int n1 = (I + 127) / 128;
-  grouped_gemm_kernel<kGemmStages, EPI_GEGLU>
-      <<<n1 * L.max_tiles, 128, smem, st>>>(tm_xp, tm_wg, tm_wu, tl, n1, H, I, hbuf, I);
+  GEMM_GEGLU<<<n1 * L.max_tiles, 128, smem, st>>>(tm_xp, tm_wg, tm_wu, tl, n1, H, I, hbuf, I);
   if (launched() != MOE_OK) return MOE_ERR_CUDA;
   prof.mark();
   // 4. GEMM-2 (down)
   const int n2 = (H + 255) / 256;
-  grouped_gemm_kernel<kGemmStages, EPI_STORE>
-      <<<n2 * L.max_tiles, 128, smem, st>>>(tm_h, tm_wd, tm_wd, tl, n2, I, H, obuf, H);
+  GEMM_STORE<<<n2 * L.max_tiles, 128, smem, st>>>(tm_h, tm_wd, tm_wd, tl, n2, I, H, obuf, H);
   if (launched() != MOE_OK) return MOE_ERR_CUDA;
   prof.mark();
   // 5. combine

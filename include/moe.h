@@ -52,8 +52,15 @@ typedef enum {
 
 enum {
   /* Return the raw softmax probabilities of the k selected experts instead of
-   * renormalising them to sum to one (renormalisation is the default). */
+   * renormalising them to sum to one (renormalisation is the default).  Implies the
+   * fp64 router path (the denominator needs every logit to fp64 accuracy). */
   MOE_FLAG_NO_RENORM = 1u << 0,
+  /* Router path.  By default batches of T >= 256 screen the logits on the tensor cores
+   * and recompute in fp64 only the experts that can still reach the top-k; smaller
+   * batches compute every logit in fp64.  Both give the same ids.  These flags force one
+   * path (testing and diagnosis); setting both is MOE_ERR_INVALID_ARG. */
+  MOE_FLAG_ROUTER_FP64 = 1u << 1,
+  MOE_FLAG_ROUTER_SCREEN = 1u << 2,
   /* Record a CUDA event at every stage boundary of the call; moe_last_stage_times()
    * then reports the per-stage device times of the most recent such call. */
   MOE_FLAG_PROFILE_STAGES = 1u << 3
@@ -66,6 +73,10 @@ typedef struct {
   int32_t *perm;           /* [T*k]  expert-sorted position -> pair index t*k+j       */
   int32_t *topk_ids;       /* [T*k]  as moe_route                                     */
   float *topk_weights;     /* [T*k]  as moe_route                                     */
+  uint32_t *router_stats;  /* [4]    {candidates recomputed in fp64, tokens that needed
+                            *         the exact sequential recomputation, largest screen
+                            *         error / (|x_t| |w_e|) seen (float bits), path:
+                            *         0 = fp64 logits, 1 = tensor-core screen}           */
 } moe_aux_t;
 
 /* ABI version of the loaded library (MOE_ABI_VERSION at build time). */

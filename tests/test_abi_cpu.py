@@ -57,6 +57,10 @@ def test_workspace_sizes(lib):
     assert lib.moe_workspace_size(8, 2816, 260, 704, 8, 0) == 0     # E > 256
     assert lib.moe_route_workspace_size(8, 2816, 128, 8, 0) > 0
     assert lib.moe_route_workspace_size(8, 2816, 6, 8, 0) == 0      # k > E
+    # the router path changes the scratch it needs: fp64 partials vs a screen buffer
+    fp64 = lib.moe_workspace_size(4096, 2816, 128, 704, 8, _abi.MOE_FLAG_ROUTER_FP64)
+    scr = lib.moe_workspace_size(4096, 2816, 128, 704, 8, _abi.MOE_FLAG_ROUTER_SCREEN)
+    assert fp64 > 0 and scr > 0 and fp64 != scr
 
 
 FAKE = 1 << 20   # an aligned non-null address; never dereferenced (host checks fail first)
@@ -74,6 +78,9 @@ def test_host_argument_checks(lib):
     assert f(*ok, 8, 2816, 4, 704, 8, 0, FAKE + 4096, None, FAKE, 1 << 30, None) == 1
     assert f(*ok, -1, 2816, 128, 704, 8, 0, FAKE + 4096, None, FAKE, 1 << 30, None) == 1
     assert f(*ok, 8, 2816, 128, 704, 8, 1 << 7, FAKE + 4096, None, FAKE, 1 << 30, None) == 1
+    both = _abi.MOE_FLAG_ROUTER_FP64 | _abi.MOE_FLAG_ROUTER_SCREEN      # contradictory paths
+    assert f(*ok, 8, 2816, 128, 704, 8, both, FAKE + 4096, None, FAKE, 1 << 30, None) == 1
+    assert lib.moe_workspace_size(8, 2816, 128, 704, 8, both) == 0
     # misaligned pointer
     assert f(FAKE + 2, *ok[1:], 8, 2816, 128, 704, 8, 0, FAKE + 4096, None, FAKE, 1 << 30,
              None) == 1

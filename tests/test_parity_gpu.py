@@ -42,10 +42,17 @@ def layer_inputs(cfg, gemma_w, seed=0, T=None):
     return x, cpu, gpu
 
 
-def gpu_forward(x, g, k, renorm=True):
+SCREEN_C = 2.0 ** -10     # the kernel's screen error bound, in units of |x_t| |w_e|
+
+
+def gpu_forward(x, g, k, renorm=True, router="auto"):
     y, aux = moe.forward(x.cuda(), g["w_router"], g["w_gate"], g["w_up"], g["w_down"], k,
-                         bias=g["bias"], renorm=renorm, aux=True)
+                         bias=g["bias"], renorm=renorm, aux=True, router=router)
     assert moe.sync_status() == 0
+    st = moe.router_stats(aux)
+    if st["path"] == "screen":
+        # the measured screen error stays 16x inside the bound the kernel assumes
+        assert st["max_screen_err_ratio"] <= SCREEN_C / 16, st
     return y, aux
 
 
@@ -78,10 +85,10 @@ def sample_tokens(T, n, seed=0):
     return np.unique(np.concatenate([[0, T - 1], s]))
 
 
-def run_case(cfg, gemma_w, n_sample, T=None, renorm=True):
+def run_case(cfg, gemma_w, n_sample, T=None, renorm=True, router="auto"):
     x, c, g = layer_inputs(cfg, gemma_w, T=T)
     T = x.shape[0]
-    y, aux = gpu_forward(x, g, cfg.k, renorm)
+    y, aux = gpu_forward(x, g, cfg.k, renorm, router)
     rows = sample_tokens(T, n_sample)
     ref = oracle.forward(x, c["w_router"], c["w_gate"], c["w_up"], c["w_down"], cfg.k,
                          bias=c["bias"], renorm=renorm, tokens=rows)
@@ -109,16 +116,23 @@ def test_forward_ragged_gemma(T, gemma_w):
     run_case(wl.CONFIGS["decode"], gemma_w, 64, T=T)
 
 
+@pytest.mark.parametrize("name,router", [("tiny", "screen"), ("decode", "screen"),
+                                         ("sweep_T512", "fp64"), ("prefill", "fp64")])
+def test_forward_forced_router_path(name, router, gemma_w):
+    run_case(wl.CONFIGS[name], gemma_w, 256, router=router)
+
+
 def test_forward_no_renorm(gemma_w):
     run_case(wl.CONFIGS["tiny"], gemma_w, 10**9, renorm=False)
     run_case(wl.CONFIGS["decode"], gemma_w, 10**9, renorm=False)
 
 
+@pytest.mark.parametrize("router", ["auto", "fp64", "screen"])
 @pytest.mark.parametrize("name", ["tiny", "decode", "prefill", "skewed", "sweep_T32768"])
-def test_route_parity_all_tokens(name, gemma_w):
+def test_route_parity_all_tokens(name, router, gemma_w):
     cfg = wl.CONFIGS[name]
     x, c, g = layer_inputs(cfg, gemma_w)
-    ids, w = moe.route(x.cuda(), g["w_router"], cfg.k, bias=g["bias"])
+    ids, w = moe.route(x.cuda(), g["w_router"], cfg.k, bias=g["bias"], router=router)
     assert moe.sync_status() == 0
     r_ids, r_w, L = oracle.route(x, c["w_router"], cfg.k, bias=c["bias"])
     assert np.array_equal(ids.cpu().numpy(), r_ids)
@@ -138,11 +152,13 @@ def test_k_equals_E_and_exact_ties():
     w["w_router"][:, 6] = w["w_router"][:, 2]
     w["w_router"][:, 7] = w["w_router"][:, 0]
     g = {k: (v.cuda() if v is not None else None) for k, v in w.items()}
-    for k in (2, cfg.E):
-        y, aux = gpu_forward(x, g, k)
-        ref = oracle.forward(x, w["w_router"], w["w_gate"], w["w_up"], w["w_down"], k)
-        check_routing(aux, ref, cfg.E)
-        check_y(y, ref["y"])
+    for router in ("fp64", "screen"):
+        for k in (2, cfg.E):
+            y, aux = gpu_forward(x, g, k, router=router)
+            ref = oracle.forward(x, w["w_router"], w["w_gate"], w["w_up"], w["w_down"], k)
+            check_routing(aux, ref, cfg.E)
+            check_y(y, ref["y"])
+            assert moe.router_stats(aux)["exact_recomputes"] > 0    # the ties went the exact way
 
 
 def test_determinism(gemma_w):
