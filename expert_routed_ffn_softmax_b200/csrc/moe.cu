@@ -218,11 +218,19 @@ struct Profiler {
   cudaStream_t st;
   bool on;
   int n = 0;
+  unsigned rec_flags = cudaEventRecordDefault;
   // External records become event nodes when the call is captured into a CUDA graph, so
   // every replay records the stage boundaries (a plain record would only be a capture
   // dependency and never fire).
   void mark() {
-    if (on) cudaEventRecordWithFlags(d->ev[n++], st, cudaEventRecordExternal);
+    if (!on) return;
+    if (n == 0) {
+      cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+      cudaStreamIsCapturing(st, &cs);
+      rec_flags = cs == cudaStreamCaptureStatusActive ? cudaEventRecordExternal
+                                                      : cudaEventRecordDefault;
+    }
+    cudaEventRecordWithFlags(d->ev[n++], st, rec_flags);
   }
   void finish() {
     if (on) d->n_profiled = n - 1;
