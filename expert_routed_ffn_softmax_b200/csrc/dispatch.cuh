@@ -36,13 +36,16 @@ __global__ void __launch_bounds__(256) dispatch_count_kernel(const int32_t* __re
 
 // One CTA (blockDim >= E).  counts, offsets, chunk_base[c][e] = offsets[e] + pairs of e in
 // chunks before c, and the GEMM tile list: for every expert with n_e > 0, tiles of BM rows
-// (expert, first sorted row, rows in tile), in expert order.
+// (expert, first sorted row, rows in tile), in expert order.  Also zeroes the split-unit
+// counters the grouped GEMMs use.
 __global__ void __launch_bounds__(256) dispatch_scan_kernel(
     const int32_t* __restrict__ chunk_counts, int nchunks, int E, int P, int BM,
     int32_t* __restrict__ counts, int32_t* __restrict__ offsets, int32_t* __restrict__ chunk_base,
     int32_t* __restrict__ tile_num, int32_t* __restrict__ tile_expert,
-    int32_t* __restrict__ tile_row0, int32_t* __restrict__ tile_rows) {
+    int32_t* __restrict__ tile_row0, int32_t* __restrict__ tile_rows,
+    int32_t* __restrict__ gemm_counters, int n_counters) {
   __shared__ int s_cnt[256], s_off[256], s_tstart[256];
+  for (int i = threadIdx.x; i < n_counters; i += blockDim.x) gemm_counters[i] = 0;
   const int e = threadIdx.x;
   int run = 0;
   if (e < E) {
@@ -119,7 +122,9 @@ __global__ void __launch_bounds__(256) dispatch_small_kernel(
     const int32_t* __restrict__ ids, int P, int E, int BM, int32_t* __restrict__ counts,
     int32_t* __restrict__ offsets, int32_t* __restrict__ perm, int32_t* __restrict__ inv,
     int32_t* __restrict__ tile_num, int32_t* __restrict__ tile_expert,
-    int32_t* __restrict__ tile_row0, int32_t* __restrict__ tile_rows) {
+    int32_t* __restrict__ tile_row0, int32_t* __restrict__ tile_rows,
+    int32_t* __restrict__ gemm_counters, int n_counters) {
+  for (int i = threadIdx.x; i < n_counters; i += blockDim.x) gemm_counters[i] = 0;
   // s_base: running rank base per expert (advanced by the ranking warp); s_off stays the
   // expert's first row for the tile list, which other threads build at the same time.
   __shared__ int s_cnt[256], s_off[256], s_base[256], s_tstart[256];

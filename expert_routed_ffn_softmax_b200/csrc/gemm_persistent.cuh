@@ -1,0 +1,395 @@
+// gemm_persistent.cuh -- persistent, warp-specialised grouped GEMM on tcgen05 (the expert
+// FFN matmuls; the role SwiftGMM plays on Ascend in "MoE推理「王炸」组合：昇腾×盘古让推理性能
+// 狂飙6-8倍", Group 4).  Same tiles, operand layouts and epilogues as grouped_gemm.cuh:
+// 128 rows of one expert x 64*NSLAB MMA columns, K staged 64 at a time by TMA (A K-major,
+// B MN-major slabs), fp32 accumulators in TMEM, GEGLU / bf16 / fp32 epilogues.
+//
+// One CTA per SM, 6 warps: warp 0 = TMA producer (lane 0) and TMEM owner, warp 1 = MMA
+// issuer (lane 0), warps 2-5 = epilogue (warp w reads TMEM lanes 32*(w%4)..+31).  Two TMEM
+// accumulators alternate between work items, so the epilogue of one item overlaps the
+// mainloop of the next.
+//
+// Schedule over U = tiles x column blocks units of nk k-steps each, G CTAs:
+//   * whole units, round robin (unit g + i*G), for all but the last one-to-two waves;
+//   * the remaining R units (G <= R < 2G, or all of them when U < 2G) are cut into G equal
+//     ranges of k-steps ("stream-K"), so every CTA streams the same number of weight bytes.
+//     A unit split between CTAs is finished by the CTA that completes its piece last: each
+//     epilogue warp stores its 32 rows of the fp32 partial tile and bumps that quadrant's
+//     counter; the warp that counts last adds the pieces in piece order (deterministic)
+//     and runs the epilogue.  Nothing waits on another CTA or another warp.
+#pragma once
+#include <cuda.h>
+#include "ptx.cuh"
+#include "grouped_gemm.cuh"
+
+namespace moe {
+
+constexpr int PG_THREADS = 192;
+constexpr int PG_EPI_THREADS = 128;
+
+template <int STAGES, int NSLAB>
+__host__ __device__ constexpr int pgemm_smem_bytes() {
+  return 1024 + STAGES * gemm_stage_bytes<NSLAB>() + 256;
+}
+
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
+struct PItem {
+  int unit;     // 0 .. U-1
+  int kb, ke;   // k-step range [kb, ke)
+  int r;        // remainder-unit index (stream-K part), -1 for whole units
+};
+
+// The work items of CTA g, in order.  Every role walks the same sequence.
+struct PSched {
+  int g, G, U, nk, n_dp, i_dp, dp_units;
+  long long c, e, Cr;
+
+  __device__ void init(int g_, int G_, int U_, int nk_) {
+    g = g_;
+    G = G_;
+    U = U_;
+    nk = nk_;
+    const int waves = U / G;
+    dp_units = waves >= 2 ? (waves - 1) * G : 0;
+    n_dp = dp_units / G;
+    i_dp = 0;
+    Cr = (long long)(U - dp_units) * nk;
+    c = (long long)g * Cr / G;
+    e = (long long)(g + 1) * Cr / G;
+  }
+  __device__ bool next(PItem& it) {
+    if (i_dp < n_dp) {
+      it.unit = g + i_dp * G;
+      it.kb = 0;
+      it.ke = nk;
+      it.r = -1;
+      ++i_dp;
+      return true;
+    }
+    if (c >= e) return false;
+    const int r = (int)(c / nk);
+    const int kb = (int)(c - (long long)r * nk);
+    const int ke = (int)min((long long)nk, kb + (e - c));
+    it.unit = dp_units + r;
+    it.kb = kb;
+    it.ke = ke;
+    it.r = (kb == 0 && ke == nk) ? -1 : r;   // covered whole by this CTA: no partial
+    c += ke - kb;
+    return true;
+  }
+  // CTA that owns remainder chunk q.
+  __device__ int owner(long long q) const { return (int)(((q + 1) * G - 1) / Cr); }
+  // Partial-tile slot of (CTA gg, remainder unit r): 2*gg for gg's first unit, else 2*gg+1.
+  __device__ int slot(int gg, int r) const {
+    const long long first = (long long)gg * Cr / G;
+    return (first / nk == r) ? 2 * gg : 2 * gg + 1;
+  }
+};
+
+template <int MODE, int NSLAB>
+__device__ __forceinline__ void pg_tile_info(const TileList& tiles, int n_blocks, int unit,
+                                             int& e, int& row0, int& rows, int& n0) {
+  constexpr int BN = 64 * NSLAB;
+  const int tile = unit / n_blocks;
+  const int nb = unit - tile * n_blocks;
+  if (tiles.uniform_rows > 0) {
+    e = 0;
+    row0 = tile * GM_BM;
+    rows = min(GM_BM, tiles.uniform_rows - row0);
+  } else {
+    e = tiles.expert[tile];
+    row0 = tiles.row0[tile];
+    rows = tiles.rows[tile];
+  }
+  n0 = nb * (MODE == EPI_GEGLU ? BN / 2 : BN);
+}
+
+// Epilogue of 32 consecutive accumulator columns [c, c+32) (and, for GEGLU, the up columns
+// [BN/2 + c, ...)) given as fp32 values, for one row.
+template <int MODE, int NSLAB>
+__device__ __forceinline__ void pg_store32(void* out_ptr, int ldo, int row, int n0, int c,
+                                           int N_total, const float* g, const float* u) {
+  if (MODE == EPI_F32) {
+    float* orow = static_cast<float*>(out_ptr) + (size_t)row * ldo + n0 + c;
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+      if (n0 + c + 4 * i < N_total)
+        reinterpret_cast<float4*>(orow)[i] = make_float4(g[4 * i], g[4 * i + 1], g[4 * i + 2],
+                                                         g[4 * i + 3]);
+    return;
+  }
+  if (n0 + c >= N_total) return;
+  uint32_t pk[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    if (MODE == EPI_GEGLU)
+      pk[i] = pack_bf16x2(gelu_tanh_f(g[2 * i]) * u[2 * i], gelu_tanh_f(g[2 * i + 1]) * u[2 * i + 1]);
+    else
+      pk[i] = pack_bf16x2(g[2 * i], g[2 * i + 1]);
+  }
+  uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(out_ptr) + (size_t)row * ldo +
+                                        n0 + c);
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+    dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+}
+
+template <int STAGES, int MODE, int NSLAB>
+__global__ void __launch_bounds__(PG_THREADS, 1)
+    grouped_gemm_persistent_kernel(const __grid_constant__ CUtensorMap tmA,
+                                   const __grid_constant__ CUtensorMap tmB0,
+                                   const __grid_constant__ CUtensorMap tmB1, TileList tiles,
+                                   int n_blocks, int K, int N_total, void* __restrict__ out_ptr,
+                                   int ldo, float* __restrict__ partials,
+                                   int* __restrict__ counters) {
+  constexpr int BN = 64 * NSLAB;
+  constexpr int STAGE_BYTES = gemm_stage_bytes<NSLAB>();
+  constexpr uint32_t TMEM_COLS = 2 * BN;   // two accumulators
+  static_assert(TMEM_COLS == 256 || TMEM_COLS == 512, "TMEM allocation must be a power of 2");
+  static_assert(MODE != EPI_GEGLU || NSLAB % 2 == 0, "GEGLU pairs gate and up slabs");
+
+  if (*reinterpret_cast<volatile unsigned*>(&g_error_word) & MOE_DEVERR_TIMEOUT) return;
+  const int n_tiles = tiles.uniform_rows > 0 ? (tiles.uniform_rows + GM_BM - 1) / GM_BM
+                                             : *tiles.num;
+  const int U = n_tiles * n_blocks;
+  const int nk = K / GM_BK;
+
+  extern __shared__ uint8_t psm_raw[];
+  const uint32_t raw_addr = smem_u32(psm_raw);
+  const uint32_t base = (raw_addr + 1023u) & ~1023u;
+  uint8_t* psm = psm_raw + (base - raw_addr);
+  const uint32_t bar_base = base + STAGES * STAGE_BYTES;
+  auto full_bar = [&](int s) { return bar_base + 8u * s; };
+  auto empty_bar = [&](int s) { return bar_base + 8u * (STAGES + s); };
+  auto tfull_bar = [&](int b) { return bar_base + 8u * (2 * STAGES + b); };
+  auto tempty_bar = [&](int b) { return bar_base + 8u * (2 * STAGES + 2 + b); };
+  uint8_t* misc = psm + STAGES * STAGE_BYTES + 8 * (2 * STAGES + 4);
+  volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(misc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 4);
+  volatile int* n_issued = reinterpret_cast<volatile int*>(misc + 8);
+  volatile int* n_consumed = reinterpret_cast<volatile int*>(misc + 12);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  if (tid == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(full_bar(s), 1);
+      mbar_init(empty_bar(s), 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(tfull_bar(b), 1);
+      mbar_init(tempty_bar(b), PG_EPI_THREADS);
+    }
+    *abort_flag = 0;
+    *n_issued = 0;
+    *n_consumed = 0;
+    fence_barrier_init();
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB0);
+    tma_prefetch_desc(&tmB1);
+  }
+  if (warp == 0) {
+    tmem_alloc(smem_u32(const_cast<uint32_t*>(tmem_slot)), TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  PSched sch;
+  sch.init(blockIdx.x, gridDim.x, U, nk);
+  PItem it;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ------------------------------------------------------------ TMA producer
+      int q = 0;
+      while (!*abort_flag && sch.next(it)) {
+        int e, row0, rows, n0;
+        pg_tile_info<MODE, NSLAB>(tiles, n_blocks, it.unit, e, row0, rows, n0);
+        for (int kc = it.kb; kc < it.ke; ++kc, ++q) {
+          const int s = q % STAGES;
+          if (q >= STAGES && !mbar_wait(empty_bar(s), ((q / STAGES) - 1) & 1)) {
+            *abort_flag = 1;
+            break;
+          }
+          const uint32_t sA = base + s * STAGE_BYTES;
+          const uint32_t sB = sA + GM_A_BYTES;
+          mbar_arrive_expect_tx(full_bar(s), STAGE_BYTES);
+          tma_load_2d(sA, &tmA, full_bar(s), kc * GM_BK, row0);
+          if (MODE == EPI_GEGLU) {
+#pragma unroll
+            for (int j = 0; j < NSLAB / 2; ++j) {
+              tma_load_3d(sB + j * GM_SLAB_BYTES, &tmB0, full_bar(s), n0 + 64 * j, kc * GM_BK, e);
+              tma_load_3d(sB + (NSLAB / 2 + j) * GM_SLAB_BYTES, &tmB1, full_bar(s), n0 + 64 * j,
+                          kc * GM_BK, e);
+            }
+          } else {
+#pragma unroll
+            for (int j = 0; j < NSLAB; ++j)
+              tma_load_3d(sB + j * GM_SLAB_BYTES, &tmB0, full_bar(s), n0 + 64 * j, kc * GM_BK, e);
+          }
+          *n_issued = q + 1;
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ------------------------------------------------------------ MMA issuer
+      constexpr uint32_t idesc = idesc_bf16_f32(GM_BM, BN, false, true);
+      int q = 0, j = 0;
+      while (!*abort_flag && sch.next(it)) {
+        const int b = j & 1, use = j >> 1;
+        if (use >= 1 && !mbar_wait(tempty_bar(b), (use - 1) & 1)) {
+          *abort_flag = 1;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t dt = tmem + b * BN;
+        bool ok = true;
+        for (int kc = it.kb; kc < it.ke; ++kc, ++q) {
+          const int s = q % STAGES;
+          if (!mbar_wait(full_bar(s), (q / STAGES) & 1)) {
+            ok = false;
+            break;
+          }
+          *n_consumed = q + 1;
+          tc_fence_after();
+          const uint32_t sA = base + s * STAGE_BYTES;
+          const uint32_t sB = sA + GM_A_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < GM_BK / 16; ++kk) {
+            const uint64_t adesc = smem_desc_sw128(sA + kk * 32, 16, 1024);
+            const uint64_t bdesc = smem_desc_sw128(sB + kk * 2048, GM_SLAB_BYTES, 1024);
+            umma_bf16(dt, adesc, bdesc, idesc, (kc != it.kb || kk != 0) ? 1u : 0u);
+          }
+          umma_commit(empty_bar(s));
+        }
+        umma_commit(tfull_bar(b));
+        ++j;
+        if (!ok) {
+          *abort_flag = 1;
+          break;
+        }
+      }
+    }
+  } else {
+    // -------------------------------------------------------------- epilogue (warps 2-5)
+    // Each warp owns 32 rows and works on its own: no barrier across the epilogue warps.
+    const int quad = warp & 3;
+    const int r_local = quad * 32 + lane;
+    int j = 0;
+    while (sch.next(it)) {
+      const int b = j & 1, use = j >> 1;
+      bool got = mbar_wait(tfull_bar(b), use & 1);
+      tc_fence_after();
+      got = __all_sync(0xffffffffu, got && !*abort_flag);   // warp-uniform decision
+      if (!got) {
+        *abort_flag = 1;
+        break;
+      }
+      int e, row0, rows, n0;
+      pg_tile_info<MODE, NSLAB>(tiles, n_blocks, it.unit, e, row0, rows, n0);
+      const bool row_ok = r_local < rows;
+      const int row = row0 + r_local;
+      const uint32_t trow = tmem + b * BN + (static_cast<uint32_t>(quad * 32) << 16);
+      constexpr int NC = MODE == EPI_GEGLU ? BN / 2 : BN;
+      if (it.r < 0) {
+        // whole unit: epilogue straight from TMEM
+#pragma unroll 1
+        for (int c = 0; c < NC; c += 32) {
+          uint32_t g[32], u[32];
+          tmem_ld_32x32b_x32(trow + c, g);
+          if (MODE == EPI_GEGLU) tmem_ld_32x32b_x32(trow + BN / 2 + c, u);
+          tmem_ld_wait();
+          if (row_ok)
+            pg_store32<MODE, NSLAB>(out_ptr, ldo, row, n0, c, N_total,
+                                    reinterpret_cast<const float*>(g),
+                                    reinterpret_cast<const float*>(u));
+        }
+        tc_fence_before();
+        mbar_arrive(tempty_bar(b));
+      } else {
+        // piece of a split unit: store this warp's 32 rows of the fp32 partial, count the
+        // piece, and let the warp that counts last add the pieces in order and finish.
+        const int slot = sch.slot(blockIdx.x, it.r);
+        float* prow = partials + ((size_t)slot * GM_BM + r_local) * BN;
+#pragma unroll 1
+        for (int c = 0; c < BN; c += 32) {
+          uint32_t v[32];
+          tmem_ld_32x32b_x32(trow + c, v);
+          tmem_ld_wait();
+          if (row_ok) {
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+              reinterpret_cast<uint4*>(prow + c)[i] =
+                  make_uint4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+          }
+        }
+        tc_fence_before();
+        mbar_arrive(tempty_bar(b));
+        __threadfence();
+        __syncwarp();
+        const long long cf = (long long)it.r * nk, cl = cf + nk - 1;
+        const int g_first = sch.owner(cf), n_pieces = sch.owner(cl) - g_first + 1;
+        int last = 0;
+        if (lane == 0) {
+          int* ctr = &counters[it.r * 4 + quad];
+          last = atomicAdd(ctr, 1) == n_pieces - 1;
+          if (last) *ctr = 0;   // ready for the next launch
+        }
+        last = __shfl_sync(0xffffffffu, last, 0);
+        if (last) {
+          __threadfence();
+          if (row_ok) {
+#pragma unroll 1
+            for (int c = 0; c < NC; c += 32) {
+              float gsum[32], usum[32];
+#pragma unroll
+              for (int i = 0; i < 32; ++i) gsum[i] = usum[i] = 0.f;
+              for (int p = 0; p < n_pieces; ++p) {
+                const float* src =
+                    partials + ((size_t)sch.slot(g_first + p, it.r) * GM_BM + r_local) * BN;
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                  const float4 a = __ldcg(reinterpret_cast<const float4*>(src + c) + i);
+                  gsum[4 * i] += a.x;
+                  gsum[4 * i + 1] += a.y;
+                  gsum[4 * i + 2] += a.z;
+                  gsum[4 * i + 3] += a.w;
+                  if (MODE == EPI_GEGLU) {
+                    const float4 bq =
+                        __ldcg(reinterpret_cast<const float4*>(src + BN / 2 + c) + i);
+                    usum[4 * i] += bq.x;
+                    usum[4 * i + 1] += bq.y;
+                    usum[4 * i + 2] += bq.z;
+                    usum[4 * i + 3] += bq.w;
+                  }
+                }
+              }
+              pg_store32<MODE, NSLAB>(out_ptr, ldo, row, n0, c, N_total, gsum, usum);
+            }
+          }
+        }
+      }
+      ++j;
+    }
+  }
+
+  // ------------------------------------------------------------------ teardown
+  tc_fence_before();
+  __syncthreads();
+  if (tid == 0 && *abort_flag) {
+    raise_error(MOE_DEVERR_TIMEOUT);
+    for (int q = *n_consumed; q < *n_issued; ++q)
+      mbar_wait_ns(full_bar(q % STAGES), (q / STAGES) & 1, kDrainLimitNs);
+  }
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 0) tmem_dealloc(tmem, TMEM_COLS);
+}
+
+}  // namespace moe

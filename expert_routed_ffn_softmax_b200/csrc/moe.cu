@@ -16,6 +16,7 @@
 #include "router.cuh"
 #include "dispatch.cuh"
 #include "grouped_gemm.cuh"
+#include "gemm_persistent.cuh"
 
 namespace moe {
 namespace {
@@ -23,12 +24,13 @@ namespace {
 constexpr int kGemmStages = 4;
 constexpr int kMaxDevices = 64;
 constexpr int kScreenMinTokens = 256;            // default router path switch
+constexpr int kMaxGemmCtas = 256;                // >= SMs per GPU (148 on B200)
 constexpr double kScreenC = 1.0 / 1024.0;        // screen error bound / (|x| |w|)
 constexpr unsigned kKnownFlags = MOE_FLAG_NO_RENORM | MOE_FLAG_ROUTER_FP64 |
                                  MOE_FLAG_ROUTER_SCREEN | MOE_FLAG_PROFILE_STAGES;
 
-#define GEMM_GEGLU grouped_gemm_kernel<kGemmStages, EPI_GEGLU, 4>
-#define GEMM_STORE grouped_gemm_kernel<kGemmStages, EPI_STORE, 4>
+#define GEMM_GEGLU grouped_gemm_persistent_kernel<kGemmStages, EPI_GEGLU, 4>
+#define GEMM_STORE grouped_gemm_persistent_kernel<kGemmStages, EPI_STORE, 4>
 #define GEMM_SCREEN grouped_gemm_kernel<kGemmStages, EPI_F32, 2>
 
 bool flags_ok(unsigned flags) {
@@ -79,6 +81,8 @@ struct Layout {
   size_t chunk_counts = 0, chunk_base = 0, counts = 0, offsets = 0, perm = 0, inv = 0;
   size_t tile_num = 0, tile_expert = 0, tile_row0 = 0, tile_rows = 0;
   size_t xp = 0, hbuf = 0, obuf = 0;
+  size_t partials = 0, counters = 0;
+  int n_counters = 0;
   size_t total = 0;
 };
 
@@ -122,6 +126,11 @@ Layout make_layout(int T, int H, int E, int I, int k, unsigned flags, bool forwa
     L.xp = take(2 * P * H);
     L.hbuf = take(2 * P * I);
     L.obuf = take(2 * P * H);
+    // stream-K split tiles of the persistent GEMMs: two fp32 tile slots per CTA, and
+    // per-(split unit, row quadrant) counters, one set per GEMM
+    L.partials = take(sizeof(float) * 2 * (size_t)kMaxGemmCtas * GM_BM * 256);
+    L.n_counters = 2 * 4 * 2 * kMaxGemmCtas;
+    L.counters = take(sizeof(int32_t) * L.n_counters);
   }
   L.total = off;
   return L;
@@ -191,7 +200,7 @@ DeviceState* device_state(int* dev_out) {
   DeviceState& d = g_dev[dev];
   if (!d.attrs_set) {
     cudaDeviceGetAttribute(&d.num_sms, cudaDevAttrMultiProcessorCount, dev);
-    const int gs = gemm_smem_bytes<kGemmStages, 4>();
+    const int gs = pgemm_smem_bytes<kGemmStages, 4>();
     const int gs2 = gemm_smem_bytes<kGemmStages, 2>();
     if (cudaFuncSetAttribute(GEMM_GEGLU, cudaFuncAttributeMaxDynamicSharedMemorySize, gs) !=
             cudaSuccess ||
@@ -419,14 +428,16 @@ moe_status_t moe_forward(const void* x, const void* w_router, const float* route
   if (s != MOE_OK) return s;
   prof.mark();
   // 2. dispatch
+  int32_t* gemm_counters = reinterpret_cast<int32_t*>(ws + L.counters);
   if (L.nchunks == 1) {
     dispatch_small_kernel<<<1, 256, 0, st>>>(ids, P, E, GM_BM, counts, offsets, perm, inv,
-                                             tile_num, tile_expert, tile_row0, tile_rows);
+                                             tile_num, tile_expert, tile_row0, tile_rows,
+                                             gemm_counters, L.n_counters);
   } else {
     dispatch_count_kernel<<<L.nchunks, 256, E * sizeof(int), st>>>(ids, P, E, chunk_counts);
     dispatch_scan_kernel<<<1, 256, 0, st>>>(chunk_counts, L.nchunks, E, P, GM_BM, counts,
                                             offsets, chunk_base, tile_num, tile_expert, tile_row0,
-                                            tile_rows);
+                                            tile_rows, gemm_counters, L.n_counters);
     dispatch_rank_kernel<<<L.nchunks, 32, E * sizeof(int), st>>>(ids, P, E, chunk_base, perm,
                                                                  inv);
   }
@@ -437,14 +448,18 @@ moe_status_t moe_forward(const void* x, const void* w_router, const float* route
   prof.mark();
   // 3. GEMM-1 + GEGLU
   const TileList tl{tile_num, tile_expert, tile_row0, tile_rows, 0};
-  const int smem = gemm_smem_bytes<kGemmStages, 4>();
+  const int smem = pgemm_smem_bytes<kGemmStages, 4>();
+  float* partials = reinterpret_cast<float*>(ws + L.partials);
+  const int G = std::min(std::max(1, d->num_sms), kMaxGemmCtas);
   const int n1 = (I + 127) / 128;
-  GEMM_GEGLU<<<n1 * L.max_tiles, 128, smem, st>>>(tm_xp, tm_wg, tm_wu, tl, n1, H, I, hbuf, I);
+  GEMM_GEGLU<<<G, PG_THREADS, smem, st>>>(tm_xp, tm_wg, tm_wu, tl, n1, H, I, hbuf, I, partials,
+                                          gemm_counters);
   if (launched() != MOE_OK) return MOE_ERR_CUDA;
   prof.mark();
   // 4. GEMM-2 (down)
   const int n2 = (H + 255) / 256;
-  GEMM_STORE<<<n2 * L.max_tiles, 128, smem, st>>>(tm_h, tm_wd, tm_wd, tl, n2, I, H, obuf, H);
+  GEMM_STORE<<<G, PG_THREADS, smem, st>>>(tm_h, tm_wd, tm_wd, tl, n2, I, H, obuf, H, partials,
+                                          gemm_counters + L.n_counters / 2);
   if (launched() != MOE_OK) return MOE_ERR_CUDA;
   prof.mark();
   // 5. combine

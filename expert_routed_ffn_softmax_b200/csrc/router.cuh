@@ -18,6 +18,7 @@
 #pragma once
 #include <cfloat>
 #include <climits>
+#include <type_traits>
 #include "ptx.cuh"
 
 namespace moe {
@@ -84,36 +85,36 @@ __global__ void __launch_bounds__(128) router_partial_kernel(
     for (int t = 0; t < TT; ++t) acc[t][i] = 0.0;
   }
   if (active) {
+    // 16 rows of W are loaded before any of them is used, so one memory latency covers 16
+    // h-steps; the FMAs still run in ascending h for every accumulator.
+    using Vec = typename std::conditional<EPL == 4, uint2, uint4>::type;
     const __nv_bfloat16* wp = wr + (size_t)(h0 + hb) * E + e0;
-#pragma unroll 2
-    for (int h = 0; h < sub; ++h, wp += E) {
-      double wv[EPL];
-      if constexpr (EPL == 4) {
-        const uint2 raw = *reinterpret_cast<const uint2*>(wp);
-        const __nv_bfloat162 a = *reinterpret_cast<const __nv_bfloat162*>(&raw.x);
-        const __nv_bfloat162 b = *reinterpret_cast<const __nv_bfloat162*>(&raw.y);
-        wv[0] = (double)__low2float(a);
-        wv[1] = (double)__high2float(a);
-        wv[2] = (double)__low2float(b);
-        wv[3] = (double)__high2float(b);
-      } else {
-        const uint4 raw = *reinterpret_cast<const uint4*>(wp);
-        const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&raw);
+    for (int hb0 = 0; hb0 < sub; hb0 += 16) {
+      Vec raw[16];
 #pragma unroll
-        for (int i = 0; i < EPL / 2; ++i) {
-          wv[2 * i] = (double)__low2float(p[i]);
-          wv[2 * i + 1] = (double)__high2float(p[i]);
+      for (int u = 0; u < 16; ++u)
+        if (hb0 + u < sub) raw[u] = *reinterpret_cast<const Vec*>(wp + (size_t)(hb0 + u) * E);
+#pragma unroll
+      for (int u = 0; u < 16; ++u) {
+        if (hb0 + u < sub) {
+          double wv[EPL];
+          const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&raw[u]);
+#pragma unroll
+          for (int i = 0; i < EPL / 2; ++i) {
+            wv[2 * i] = (double)__low2float(p[i]);
+            wv[2 * i + 1] = (double)__high2float(p[i]);
+          }
+          const double* xr = rsm + (hb + hb0 + u) * TT;
+#pragma unroll
+          for (int t = 0; t < TT; ++t) {
+            const double xv = xr[t];
+#pragma unroll
+            for (int i = 0; i < EPL; ++i) acc[t][i] = fma(xv, wv[i], acc[t][i]);
+          }
+#pragma unroll
+          for (int i = 0; i < EPL; ++i) wn[i] = fma(wv[i], wv[i], wn[i]);
         }
       }
-      const double* xr = rsm + (hb + h) * TT;
-#pragma unroll
-      for (int t = 0; t < TT; ++t) {
-        const double xv = xr[t];
-#pragma unroll
-        for (int i = 0; i < EPL; ++i) acc[t][i] = fma(xv, wv[i], acc[t][i]);
-      }
-#pragma unroll
-      for (int i = 0; i < EPL; ++i) wn[i] = fma(wv[i], wv[i], wn[i]);
     }
   }
   __syncthreads();  // x stage no longer needed: reuse smem for the cross-warp reduction
@@ -462,17 +463,37 @@ __global__ void __launch_bounds__(256) router_screen_select_kernel(
     }
     __syncwarp();
 
-    // fp64 recheck of the candidates, 4 at a time: lane sums h = lane + 32 j in ascending j,
-    // then a fixed xor tree.
+    // fp64 recheck of the candidates, 4 at a time.  Lane l owns h = 256 j + 8 l + i
+    // (i < 8), read as 16-byte vectors of x and of the transposed W rows; it sums its h in
+    // ascending order, then a fixed xor tree adds the lanes.
+    const int nj = (H + 255) / 256;
     for (int c0 = 0; c0 < nc; c0 += 4) {
-      const __nv_bfloat16* wrow[4];
+      const uint4* wrow[4];
       double acc[4] = {0.0, 0.0, 0.0, 0.0};
 #pragma unroll
-      for (int u = 0; u < 4; ++u) wrow[u] = wrT + (size_t)s_cand[warp][min(c0 + u, nc - 1)] * H;
-      for (int h = lane; h < H; h += 32) {
-        const double xv = (double)__bfloat162float(xr[h]);
+      for (int u = 0; u < 4; ++u)
+        wrow[u] = reinterpret_cast<const uint4*>(wrT + (size_t)s_cand[warp][min(c0 + u, nc - 1)] * H);
+      const uint4* xv4 = reinterpret_cast<const uint4*>(xr);
+#pragma unroll 4
+      for (int jj = 0; jj < nj; ++jj) {
+        const int v = jj * 32 + lane;           // 16-byte vector index within the row
+        if (v * 8 < H) {
+          const uint4 xq = __ldg(xv4 + v);
+          uint4 wq[4];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) acc[u] = fma(xv, (double)__bfloat162float(wrow[u][h]), acc[u]);
+          for (int u = 0; u < 4; ++u) wq[u] = __ldg(wrow[u] + v);
+          const __nv_bfloat162* xp2 = reinterpret_cast<const __nv_bfloat162*>(&xq);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const float2 xf = __bfloat1622float2(xp2[i]);
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              const float2 wf = __bfloat1622float2(reinterpret_cast<const __nv_bfloat162*>(&wq[u])[i]);
+              acc[u] = fma((double)xf.x, (double)wf.x, acc[u]);
+              acc[u] = fma((double)xf.y, (double)wf.y, acc[u]);
+            }
+          }
+        }
       }
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
