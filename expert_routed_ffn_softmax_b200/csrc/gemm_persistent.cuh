@@ -45,7 +45,7 @@ struct PItem {
 // The work items of CTA g, in order.  Every role walks the same sequence.
 struct PSched {
   int g, G, U, nk, n_dp, i_dp, dp_units;
-  long long c, e, Cr;
+  long long c, e, Cr, Gs;   // Gs: CTAs sharing the stream-K part, each with >= 1 k-step
 
   __device__ void init(int g_, int G_, int U_, int nk_) {
     g = g_;
@@ -57,8 +57,13 @@ struct PSched {
     n_dp = dp_units / G;
     i_dp = 0;
     Cr = (long long)(U - dp_units) * nk;
-    c = (long long)g * Cr / G;
-    e = (long long)(g + 1) * Cr / G;
+    Gs = Cr < G ? Cr : G;
+    if (g < Gs) {
+      c = (long long)g * Cr / Gs;
+      e = (long long)(g + 1) * Cr / Gs;
+    } else {
+      c = e = 0;
+    }
   }
   __device__ bool next(PItem& it) {
     if (i_dp < n_dp) {
@@ -80,11 +85,12 @@ struct PSched {
     c += ke - kb;
     return true;
   }
-  // CTA that owns remainder chunk q.
-  __device__ int owner(long long q) const { return (int)(((q + 1) * G - 1) / Cr); }
+  // CTA that owns remainder chunk q (the Gs ranges are all non-empty, so the owners of a
+  // unit's chunks are consecutive CTAs).
+  __device__ int owner(long long q) const { return (int)(((q + 1) * Gs - 1) / Cr); }
   // Partial-tile slot of (CTA gg, remainder unit r): 2*gg for gg's first unit, else 2*gg+1.
   __device__ int slot(int gg, int r) const {
-    const long long first = (long long)gg * Cr / G;
+    const long long first = (long long)gg * Cr / Gs;
     return (first / nk == r) ? 2 * gg : 2 * gg + 1;
   }
 };
