@@ -115,24 +115,25 @@ __global__ void __launch_bounds__(32) dispatch_rank_kernel(const int32_t* __rest
   }
 }
 
-// Whole dispatch for a batch of at most one chunk (P <= kDispatchChunk) in one CTA of 256
-// threads: histogram, scan, tile list and the stable ranks, as the kernels above compute
-// them for many chunks.
-__global__ void __launch_bounds__(256) dispatch_small_kernel(
+// Whole dispatch for a batch of at most one chunk (P <= kDispatchChunk) by one CTA (any
+// size >= 32 threads; warp 0 scans and ranks): histogram, scan, tile list and the stable
+// ranks, as the kernels above compute them for many chunks; also zeroes the split-unit
+// counters of the grouped GEMMs.  s_*: four shared arrays of 256 ints.
+__device__ __forceinline__ void dispatch_small_block(
     const int32_t* __restrict__ ids, int P, int E, int BM, int32_t* __restrict__ counts,
     int32_t* __restrict__ offsets, int32_t* __restrict__ perm, int32_t* __restrict__ inv,
     int32_t* __restrict__ tile_num, int32_t* __restrict__ tile_expert,
     int32_t* __restrict__ tile_row0, int32_t* __restrict__ tile_rows,
-    int32_t* __restrict__ gemm_counters, int n_counters) {
-  for (int i = threadIdx.x; i < n_counters; i += blockDim.x) gemm_counters[i] = 0;
+    int32_t* __restrict__ gemm_counters, int n_counters, int* s_cnt, int* s_off, int* s_base,
+    int* s_tstart) {
   // s_base: running rank base per expert (advanced by the ranking warp); s_off stays the
   // expert's first row for the tile list, which other threads build at the same time.
-  __shared__ int s_cnt[256], s_off[256], s_base[256], s_tstart[256];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  s_cnt[tid] = 0;
+  for (int i = tid; i < n_counters; i += blockDim.x) gemm_counters[i] = 0;
+  for (int i = tid; i < 256; i += blockDim.x) s_cnt[i] = 0;
   __syncthreads();
   for (int q = tid; q < P; q += blockDim.x) {
-    const int e = ids[q];
+    const int e = __ldcg(ids + q);
     if ((unsigned)e < (unsigned)E)
       atomicAdd(&s_cnt[e], 1);
     else
@@ -180,11 +181,11 @@ __global__ void __launch_bounds__(256) dispatch_small_kernel(
     }
   }
   __syncthreads();
-  if (tid < E) {
-    const int n = s_cnt[tid], off = s_off[tid], nt = (n + BM - 1) / BM;
+  for (int e = tid; e < E; e += blockDim.x) {
+    const int n = s_cnt[e], off = s_off[e], nt = (n + BM - 1) / BM;
     for (int m = 0; m < nt; ++m) {
-      const int i = s_tstart[tid] + m;
-      tile_expert[i] = tid;
+      const int i = s_tstart[e] + m;
+      tile_expert[i] = e;
       tile_row0[i] = off + m * BM;
       tile_rows[i] = min(BM, n - m * BM);
     }
@@ -193,7 +194,7 @@ __global__ void __launch_bounds__(256) dispatch_small_kernel(
     const unsigned lt = (1u << lane) - 1u;
     for (int qb = 0; qb < P; qb += 32) {
       const int q = qb + lane;
-      int e = q < P ? ids[q] : -1;
+      int e = q < P ? __ldcg(ids + q) : -1;
       if (q < P && (unsigned)e >= (unsigned)E) e = -2;
       const unsigned grp = __match_any_sync(0xffffffffu, e);
       int pos = 0;
@@ -207,6 +208,18 @@ __global__ void __launch_bounds__(256) dispatch_small_kernel(
       }
     }
   }
+}
+
+__global__ void __launch_bounds__(256) dispatch_small_kernel(
+    const int32_t* __restrict__ ids, int P, int E, int BM, int32_t* __restrict__ counts,
+    int32_t* __restrict__ offsets, int32_t* __restrict__ perm, int32_t* __restrict__ inv,
+    int32_t* __restrict__ tile_num, int32_t* __restrict__ tile_expert,
+    int32_t* __restrict__ tile_row0, int32_t* __restrict__ tile_rows,
+    int32_t* __restrict__ gemm_counters, int n_counters) {
+  __shared__ int s_cnt[256], s_off[256], s_base[256], s_tstart[256];
+  dispatch_small_block(ids, P, E, BM, counts, offsets, perm, inv, tile_num, tile_expert,
+                       tile_row0, tile_rows, gemm_counters, n_counters, s_cnt, s_off, s_base,
+                       s_tstart);
 }
 
 // Xp[pos, :] = x[perm[pos] / k, :]   (16-byte vectors; one warp per row, grid-stride)

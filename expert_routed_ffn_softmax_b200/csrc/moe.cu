@@ -17,6 +17,7 @@
 #include "dispatch.cuh"
 #include "grouped_gemm.cuh"
 #include "gemm_persistent.cuh"
+#include "decode_front.cuh"
 
 namespace moe {
 namespace {
@@ -25,6 +26,8 @@ constexpr int kGemmStages = 4;
 constexpr int kMaxDevices = 64;
 constexpr int kScreenMinTokens = 256;            // default router path switch
 constexpr int kMaxGemmCtas = 256;                // >= SMs per GPU (148 on B200)
+constexpr int kFrontSmemMax = 200 * 1024;        // decode front kernel's dynamic smem cap
+
 constexpr double kScreenC = 1.0 / 1024.0;        // screen error bound / (|x| |w|)
 constexpr unsigned kKnownFlags = MOE_FLAG_NO_RENORM | MOE_FLAG_ROUTER_FP64 |
                                  MOE_FLAG_ROUTER_SCREEN | MOE_FLAG_PROFILE_STAGES;
@@ -44,6 +47,12 @@ bool router_uses_screen(int T, unsigned flags) {
   if (flags & (MOE_FLAG_NO_RENORM | MOE_FLAG_ROUTER_FP64)) return false;
   if (flags & MOE_FLAG_ROUTER_SCREEN) return true;
   return T >= kScreenMinTokens;
+}
+
+// Batches of at most 8 tokens take the fused router + dispatch + gather launch.
+bool use_decode_front(int T, int H, int E, unsigned flags) {
+  return T <= kFrontMaxTokens && E <= 128 && !router_uses_screen(T, flags) &&
+         H % (kFrontRanks * 4) == 0 && decode_front_smem_bytes(H, E) <= (size_t)kFrontSmemMax;
 }
 
 size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
@@ -207,6 +216,9 @@ DeviceState* device_state(int* dev_out) {
         cudaFuncSetAttribute(GEMM_STORE, cudaFuncAttributeMaxDynamicSharedMemorySize, gs) !=
             cudaSuccess ||
         cudaFuncSetAttribute(GEMM_SCREEN, cudaFuncAttributeMaxDynamicSharedMemorySize, gs2) !=
+            cudaSuccess ||
+        cudaFuncSetAttribute(decode_front_kernel<4>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, kFrontSmemMax) !=
             cudaSuccess ||
         cudaFuncSetAttribute(router_partial_kernel<4>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, 1408 * 8 * 8) !=
@@ -421,31 +433,46 @@ moe_status_t moe_forward(const void* x, const void* w_router, const float* route
 
   Profiler prof{d, st, (flags & MOE_FLAG_PROFILE_STAGES) != 0};
   prof.mark();
-  // 1. router
-  moe_status_t s = launch_router(static_cast<const __nv_bfloat16*>(x),
-                                 static_cast<const __nv_bfloat16*>(w_router), router_bias, T, H,
-                                 E, k, flags, ids, wts, stats, ws, L, *d, st);
-  if (s != MOE_OK) return s;
-  prof.mark();
-  // 2. dispatch
   int32_t* gemm_counters = reinterpret_cast<int32_t*>(ws + L.counters);
-  if (L.nchunks == 1) {
-    dispatch_small_kernel<<<1, 256, 0, st>>>(ids, P, E, GM_BM, counts, offsets, perm, inv,
-                                             tile_num, tile_expert, tile_row0, tile_rows,
-                                             gemm_counters, L.n_counters);
-  } else {
-    dispatch_count_kernel<<<L.nchunks, 256, E * sizeof(int), st>>>(ids, P, E, chunk_counts);
-    dispatch_scan_kernel<<<1, 256, 0, st>>>(chunk_counts, L.nchunks, E, P, GM_BM, counts,
-                                            offsets, chunk_base, tile_num, tile_expert, tile_row0,
-                                            tile_rows, gemm_counters, L.n_counters);
-    dispatch_rank_kernel<<<L.nchunks, 32, E * sizeof(int), st>>>(ids, P, E, chunk_base, perm,
-                                                                 inv);
-  }
   const int gsm = std::max(1, d->num_sms) * 8;
-  gather_rows_kernel<<<std::min((P + 7) / 8, gsm), 256, 0, st>>>(
-      static_cast<const uint4*>(x), perm, P, k, H / 8, reinterpret_cast<uint4*>(xp));
-  if (launched() != MOE_OK) return MOE_ERR_CUDA;
-  prof.mark();
+  if (use_decode_front(T, H, E, flags)) {
+    // 1+2. router, dispatch and gather in one cluster launch
+    if (cudaMemsetAsync(stats, 0, 4 * sizeof(unsigned), st) != cudaSuccess) return MOE_ERR_CUDA;
+    const double u = std::ldexp(1.0, -53), n = (double)H + 8.0;
+    const double beta_scale = 2.0 * (n * u / (1.0 - n * u)) * 1.01;
+    decode_front_kernel<4><<<kFrontRanks, 128, decode_front_smem_bytes(H, E), st>>>(
+        static_cast<const __nv_bfloat16*>(x), static_cast<const __nv_bfloat16*>(w_router),
+        router_bias, T, H, E, k, (flags & MOE_FLAG_NO_RENORM) ? 0 : 1, beta_scale, ids, wts, stats,
+        counts, offsets, perm, inv, tile_num, tile_expert, tile_row0, tile_rows, gemm_counters,
+        L.n_counters, GM_BM, reinterpret_cast<uint4*>(xp), H / 8);
+    if (launched() != MOE_OK) return MOE_ERR_CUDA;
+    prof.mark();
+    prof.mark();
+  } else {
+    // 1. router
+    moe_status_t s = launch_router(static_cast<const __nv_bfloat16*>(x),
+                                   static_cast<const __nv_bfloat16*>(w_router), router_bias, T, H,
+                                   E, k, flags, ids, wts, stats, ws, L, *d, st);
+    if (s != MOE_OK) return s;
+    prof.mark();
+    // 2. dispatch
+    if (L.nchunks == 1) {
+      dispatch_small_kernel<<<1, 256, 0, st>>>(ids, P, E, GM_BM, counts, offsets, perm, inv,
+                                               tile_num, tile_expert, tile_row0, tile_rows,
+                                               gemm_counters, L.n_counters);
+    } else {
+      dispatch_count_kernel<<<L.nchunks, 256, E * sizeof(int), st>>>(ids, P, E, chunk_counts);
+      dispatch_scan_kernel<<<1, 256, 0, st>>>(chunk_counts, L.nchunks, E, P, GM_BM, counts,
+                                              offsets, chunk_base, tile_num, tile_expert, tile_row0,
+                                              tile_rows, gemm_counters, L.n_counters);
+      dispatch_rank_kernel<<<L.nchunks, 32, E * sizeof(int), st>>>(ids, P, E, chunk_base, perm,
+                                                                   inv);
+    }
+    gather_rows_kernel<<<std::min((P + 7) / 8, gsm), 256, 0, st>>>(
+        static_cast<const uint4*>(x), perm, P, k, H / 8, reinterpret_cast<uint4*>(xp));
+    if (launched() != MOE_OK) return MOE_ERR_CUDA;
+    prof.mark();
+  }
   // 3. GEMM-1 + GEGLU
   const TileList tl{tile_num, tile_expert, tile_row0, tile_rows, 0};
   const int smem = pgemm_smem_bytes<kGemmStages, 4>();

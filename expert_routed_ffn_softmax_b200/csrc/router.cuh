@@ -222,6 +222,83 @@ __device__ __forceinline__ double warp_value_of(const double (&V)[EPL], const in
   return __shfl_sync(0xffffffffu, mine, __ffs(m) - 1);
 }
 
+// Given a token's logits L (expert lane + 32 i) and their rounding bounds beta: select the
+// top-k by (value desc, id asc), verify every decision against the bounds, recompute the
+// token exactly when one is too close to call, then write ids and (renormalised) weights.
+template <int EPL>
+__device__ __forceinline__ void router_finish_token(
+    double (&L)[EPL], const double (&beta)[EPL], int t, const __nv_bfloat16* __restrict__ x,
+    const __nv_bfloat16* __restrict__ wr, const float* __restrict__ bias, int H, int E, int k,
+    int renorm, int32_t* __restrict__ ids, float* __restrict__ wts,
+    unsigned* __restrict__ stats) {
+  const int lane = threadIdx.x & 31;
+  bool taken[EPL];
+  int sel_e[8];
+  double sel_v[8];
+  warp_topk<EPL>(L, E, k, taken, sel_e, sel_v);
+
+  // Verify every decision against the rounding bound.
+  int eid[EPL];
+#pragma unroll
+  for (int i = 0; i < EPL; ++i) eid[i] = (lane + 32 * i < E) ? lane + 32 * i : INT_MAX;
+  double sel_b[8];
+  for (int r = 0; r < k; ++r) sel_b[r] = warp_value_of<EPL>(beta, eid, sel_e[r]);
+  bool ok = true;
+  for (int r = 0; r + 1 < k; ++r) ok = ok && (sel_v[r] - sel_v[r + 1] > sel_b[r] + sel_b[r + 1]);
+#pragma unroll
+  for (int i = 0; i < EPL; ++i) {
+    const int e = lane + 32 * i;
+    if (e < E && !taken[i]) ok = ok && (sel_v[k - 1] - L[i] > sel_b[k - 1] + beta[i]);
+  }
+  ok = __all_sync(0xffffffffu, ok);
+
+  if (!ok) {
+    // Too close to call: redo every logit of this token in ascending h (one FMA chain
+    // per expert, the product being exact), then rank those values.
+    if (lane == 0) atomicAdd(&stats[1], 1u);
+    double acc[EPL];
+#pragma unroll
+    for (int i = 0; i < EPL; ++i) acc[i] = 0.0;
+    const __nv_bfloat16* xr = x + (size_t)t * H;
+    for (int h = 0; h < H; ++h) {
+      const double xv = (double)__bfloat162float(xr[h]);
+#pragma unroll
+      for (int i = 0; i < EPL; ++i) {
+        const int e = lane + 32 * i;
+        if (e < E) acc[i] = fma(xv, (double)__bfloat162float(wr[(size_t)h * E + e]), acc[i]);
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < EPL; ++i) {
+      const int e = lane + 32 * i;
+      if (e < E) L[i] = bias ? acc[i] + (double)bias[e] : acc[i];
+    }
+    warp_topk<EPL>(L, E, k, taken, sel_e, sel_v);
+  }
+
+  // Weights: softmax over all E, renormalised over the k selected (or not).
+  const double m = sel_v[0];
+  double denom = 0.0;
+  if (renorm) {
+    for (int r = 0; r < k; ++r) denom += exp(sel_v[r] - m);
+  } else {
+    double s = 0.0;
+#pragma unroll
+    for (int i = 0; i < EPL; ++i)
+      if (lane + 32 * i < E) s += exp(L[i] - m);
+#pragma unroll
+    for (int off = 16; off; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+    denom = s;
+  }
+  for (int r = 0; r < k; ++r) {
+    if (lane == r) {
+      ids[(size_t)t * k + r] = sel_e[r];
+      wts[(size_t)t * k + r] = (float)(exp(sel_v[r] - m) / denom);
+    }
+  }
+
+}
+
 // One warp per token.  Finishes the logits, selects, verifies, computes the weights.
 template <int EPL>
 __global__ void __launch_bounds__(256) router_select_kernel(
@@ -235,110 +312,55 @@ __global__ void __launch_bounds__(256) router_select_kernel(
   const int warps_per_block = blockDim.x >> 5;
   for (int t = blockIdx.x * warps_per_block + (threadIdx.x >> 5); t < T;
        t += gridDim.x * warps_per_block) {
-    // Partials are added in ascending split order.  The loads of 8 splits are issued
-    // before their adds so that the latency of a long split list is paid once per 8.
-    double L[EPL], beta[EPL];
+    // Partials are added in ascending split order.  The loads of 4 splits (for every
+    // expert of the lane and the norms) are issued before their adds, so a long split list
+    // costs one memory latency per 4 splits.
+    double L[EPL], beta[EPL], wn2[EPL];
     double xn2 = 0.0;
-    for (int s0 = 0; s0 < ks; s0 += 8) {
-      double p[8];
-#pragma unroll
-      for (int u = 0; u < 8; ++u) p[u] = (s0 + u < ks) ? part_xn2[(size_t)(s0 + u) * T + t] : 0.0;
-#pragma unroll
-      for (int u = 0; u < 8; ++u)
-        if (s0 + u < ks) xn2 += p[u];
-    }
 #pragma unroll
     for (int i = 0; i < EPL; ++i) {
-      const int e = lane + 32 * i;
-      L[i] = -DBL_MAX;
-      beta[i] = 0.0;
-      if (e < E) {
-        double v = 0.0, wn2 = 0.0;
-        for (int s0 = 0; s0 < ks; s0 += 8) {
-          double p[8], q[8];
-#pragma unroll
-          for (int u = 0; u < 8; ++u) {
-            const bool in = s0 + u < ks;
-            p[u] = in ? part_logit[((size_t)(s0 + u) * T + t) * E + e] : 0.0;
-            q[u] = in ? part_wn2[(size_t)(s0 + u) * E + e] : 0.0;
-          }
-#pragma unroll
-          for (int u = 0; u < 8; ++u)
-            if (s0 + u < ks) {
-              v = (s0 + u == 0) ? p[u] : v + p[u];
-              wn2 += q[u];
-            }
-        }
-        const double b = bias ? (double)bias[e] : 0.0;
-        if (bias) v += b;
-        L[i] = v;
-        beta[i] = beta_scale * (sqrt(xn2 * wn2) * (1.0 + 1e-6) + fabs(b));
-      }
+      L[i] = 0.0;
+      wn2[i] = 0.0;
     }
-    bool taken[EPL];
-    int sel_e[8];
-    double sel_v[8];
-    warp_topk<EPL>(L, E, k, taken, sel_e, sel_v);
-
-    // Verify every decision against the rounding bound.
-    int eid[EPL];
+    for (int s0 = 0; s0 < ks; s0 += 4) {
+      double p[4][EPL], q[4][EPL], xq[4];
 #pragma unroll
-    for (int i = 0; i < EPL; ++i) eid[i] = (lane + 32 * i < E) ? lane + 32 * i : INT_MAX;
-    double sel_b[8];
-    for (int r = 0; r < k; ++r) sel_b[r] = warp_value_of<EPL>(beta, eid, sel_e[r]);
-    bool ok = true;
-    for (int r = 0; r + 1 < k; ++r) ok = ok && (sel_v[r] - sel_v[r + 1] > sel_b[r] + sel_b[r + 1]);
-#pragma unroll
-    for (int i = 0; i < EPL; ++i) {
-      const int e = lane + 32 * i;
-      if (e < E && !taken[i]) ok = ok && (sel_v[k - 1] - L[i] > sel_b[k - 1] + beta[i]);
-    }
-    ok = __all_sync(0xffffffffu, ok);
-
-    if (!ok) {
-      // Too close to call: redo every logit of this token in ascending h (one FMA chain
-      // per expert, the product being exact), then rank those values.
-      if (lane == 0) atomicAdd(&stats[1], 1u);
-      double acc[EPL];
-#pragma unroll
-      for (int i = 0; i < EPL; ++i) acc[i] = 0.0;
-      const __nv_bfloat16* xr = x + (size_t)t * H;
-      for (int h = 0; h < H; ++h) {
-        const double xv = (double)__bfloat162float(xr[h]);
+      for (int u = 0; u < 4; ++u) {
+        const bool in = s0 + u < ks;
+        xq[u] = in ? part_xn2[(size_t)(s0 + u) * T + t] : 0.0;
 #pragma unroll
         for (int i = 0; i < EPL; ++i) {
           const int e = lane + 32 * i;
-          if (e < E) acc[i] = fma(xv, (double)__bfloat162float(wr[(size_t)h * E + e]), acc[i]);
+          const bool ok = in && e < E;
+          p[u][i] = ok ? part_logit[((size_t)(s0 + u) * T + t) * E + e] : 0.0;
+          q[u][i] = ok ? part_wn2[(size_t)(s0 + u) * E + e] : 0.0;
         }
       }
 #pragma unroll
-      for (int i = 0; i < EPL; ++i) {
-        const int e = lane + 32 * i;
-        if (e < E) L[i] = bias ? acc[i] + (double)bias[e] : acc[i];
-      }
-      warp_topk<EPL>(L, E, k, taken, sel_e, sel_v);
-    }
-
-    // Weights: softmax over all E, renormalised over the k selected (or not).
-    const double m = sel_v[0];
-    double denom = 0.0;
-    if (renorm) {
-      for (int r = 0; r < k; ++r) denom += exp(sel_v[r] - m);
-    } else {
-      double s = 0.0;
+      for (int u = 0; u < 4; ++u) {
+        if (s0 + u < ks) {
+          xn2 += xq[u];
 #pragma unroll
-      for (int i = 0; i < EPL; ++i)
-        if (lane + 32 * i < E) s += exp(L[i] - m);
-#pragma unroll
-      for (int off = 16; off; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
-      denom = s;
-    }
-    for (int r = 0; r < k; ++r) {
-      if (lane == r) {
-        ids[(size_t)t * k + r] = sel_e[r];
-        wts[(size_t)t * k + r] = (float)(exp(sel_v[r] - m) / denom);
+          for (int i = 0; i < EPL; ++i) {
+            L[i] = (s0 + u == 0) ? p[u][i] : L[i] + p[u][i];
+            wn2[i] += q[u][i];
+          }
+        }
       }
     }
+#pragma unroll
+    for (int i = 0; i < EPL; ++i) {
+      const int e = lane + 32 * i;
+      beta[i] = 0.0;
+      if (e < E) {
+        const double b = bias ? (double)bias[e] : 0.0;
+        if (bias) L[i] += b;
+        beta[i] = beta_scale * (sqrt(xn2 * wn2[i]) * (1.0 + 1e-6) + fabs(b));
+      } else {
+        L[i] = -DBL_MAX;
+      }
+    }
+    router_finish_token<EPL>(L, beta, t, x, wr, bias, H, E, k, renorm, ids, wts, stats);
   }
 }
 
