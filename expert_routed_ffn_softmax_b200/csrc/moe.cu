@@ -18,6 +18,7 @@
 #include "grouped_gemm.cuh"
 #include "gemm_persistent.cuh"
 #include "decode_front.cuh"
+#include "gemm_decode.cuh"
 
 namespace moe {
 namespace {
@@ -47,6 +48,12 @@ bool router_uses_screen(int T, unsigned flags) {
   if (flags & (MOE_FLAG_NO_RENORM | MOE_FLAG_ROUTER_FP64)) return false;
   if (flags & MOE_FLAG_ROUTER_SCREEN) return true;
   return T >= kScreenMinTokens;
+}
+
+// Batches of at most 16 tokens (so at most 16 rows per expert) use the decode GEMMs.
+constexpr int kDecodeMaxTokens = 16;
+bool use_decode_gemm(int T, int H, int I) {
+  return T <= kDecodeMaxTokens && decode_shape_ok(I, true) && decode_shape_ok(H, false);
 }
 
 // Batches of at most 8 tokens take the fused router + dispatch + gather launch.
@@ -84,7 +91,7 @@ int router_ksplit(int T, int H) {
 
 struct Layout {
   bool screen = false;
-  int ks = 0, hs = 0, nchunks = 0, max_tiles = 0;
+  int ks = 0, hs = 0, nchunks = 0, max_tiles = 0, bm = 0;
   size_t part_logit = 0, part_xn2 = 0, part_wn2 = 0, stats = 0, ids = 0, wts = 0;
   size_t scr = 0, wrT = 0, wn2 = 0;
   size_t chunk_counts = 0, chunk_base = 0, counts = 0, offsets = 0, perm = 0, inv = 0;
@@ -119,7 +126,8 @@ Layout make_layout(int T, int H, int E, int I, int k, unsigned flags, bool forwa
   }
   if (forward) {
     L.nchunks = (int)((P + kDispatchChunk - 1) / kDispatchChunk);
-    L.max_tiles = (int)(P / GM_BM) + E;
+    L.bm = use_decode_gemm(T, H, I) ? DG_BN : GM_BM;
+    L.max_tiles = (int)(P / L.bm) + E;
     L.ids = take(sizeof(int32_t) * P);
     L.wts = take(sizeof(float) * P);
     L.chunk_counts = take(sizeof(int32_t) * (size_t)L.nchunks * E);
@@ -162,26 +170,30 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// Row-major [rows][cols] bf16, box = 64 columns x box_rows rows, 128-byte swizzle.
-bool make_map_2d(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, uint32_t box_rows) {
+// Row-major [rows][cols] bf16, box = box_cols x box_rows (64 columns with the 128-byte
+// swizzle, or 16 columns with the 32-byte swizzle).
+bool make_map_2d(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, uint32_t box_rows,
+                 uint32_t box_cols = 64) {
   auto fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[2] = {cols, rows};
   cuuint64_t strides[1] = {cols * 2};
-  cuuint32_t box[2] = {64, box_rows};
+  cuuint32_t box[2] = {box_cols, box_rows};
   cuuint32_t estr[2] = {1, 1};
+  const CUtensorMapSwizzle sw = box_cols == 16 ? CU_TENSOR_MAP_SWIZZLE_32B : CU_TENSOR_MAP_SWIZZLE_128B;
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
-            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// Stacked [E][rows][cols] bf16 (cols contiguous), box = 64 columns x 64 rows x 1 expert.
-bool make_map_3d(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, uint64_t E) {
+// Stacked [E][rows][cols] bf16 (cols contiguous), box = 64 columns x box_rows rows x 1 expert.
+bool make_map_3d(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, uint64_t E,
+                 uint32_t box_rows = 64) {
   auto fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[3] = {cols, rows, E};
   cuuint64_t strides[2] = {cols * 2, cols * rows * 2};
-  cuuint32_t box[3] = {64, 64, 1};
+  cuuint32_t box[3] = {64, box_rows, 1};
   cuuint32_t estr[3] = {1, 1, 1};
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -216,6 +228,12 @@ DeviceState* device_state(int* dev_out) {
         cudaFuncSetAttribute(GEMM_STORE, cudaFuncAttributeMaxDynamicSharedMemorySize, gs) !=
             cudaSuccess ||
         cudaFuncSetAttribute(GEMM_SCREEN, cudaFuncAttributeMaxDynamicSharedMemorySize, gs2) !=
+            cudaSuccess ||
+        cudaFuncSetAttribute(grouped_gemm_decode_kernel<EPI_GEGLU>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024) !=
+            cudaSuccess ||
+        cudaFuncSetAttribute(grouped_gemm_decode_kernel<EPI_STORE>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024) !=
             cudaSuccess ||
         cudaFuncSetAttribute(decode_front_kernel<4>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, kFrontSmemMax) !=
@@ -425,10 +443,14 @@ moe_status_t moe_forward(const void* x, const void* w_router, const float* route
   __nv_bfloat16* hbuf = reinterpret_cast<__nv_bfloat16*>(ws + L.hbuf);
   __nv_bfloat16* obuf = reinterpret_cast<__nv_bfloat16*>(ws + L.obuf);
 
+  const bool dec = L.bm == DG_BN;    // decode tiles: <= 16 rows per expert
   CUtensorMap tm_xp, tm_wg, tm_wu, tm_h, tm_wd;
-  if (!make_map_2d(&tm_xp, xp, H, P, GM_BM) || !make_map_3d(&tm_wg, w_gate, I, H, E) ||
-      !make_map_3d(&tm_wu, w_up, I, H, E) || !make_map_2d(&tm_h, hbuf, I, P, GM_BM) ||
-      !make_map_3d(&tm_wd, w_down, H, I, E))
+  const uint32_t act_rows = dec ? DG_BN : GM_BM, act_cols = dec ? DG_KS : 64;
+  const uint32_t w_rows = dec ? DG_KS : 64;
+  if (!make_map_2d(&tm_xp, xp, H, P, act_rows, act_cols) ||
+      !make_map_3d(&tm_wg, w_gate, I, H, E, w_rows) || !make_map_3d(&tm_wu, w_up, I, H, E, w_rows) ||
+      !make_map_2d(&tm_h, hbuf, I, P, act_rows, act_cols) ||
+      !make_map_3d(&tm_wd, w_down, H, I, E, w_rows))
     return MOE_ERR_CUDA;
 
   Profiler prof{d, st, (flags & MOE_FLAG_PROFILE_STAGES) != 0};
@@ -444,7 +466,7 @@ moe_status_t moe_forward(const void* x, const void* w_router, const float* route
         static_cast<const __nv_bfloat16*>(x), static_cast<const __nv_bfloat16*>(w_router),
         router_bias, T, H, E, k, (flags & MOE_FLAG_NO_RENORM) ? 0 : 1, beta_scale, ids, wts, stats,
         counts, offsets, perm, inv, tile_num, tile_expert, tile_row0, tile_rows, gemm_counters,
-        L.n_counters, GM_BM, reinterpret_cast<uint4*>(xp), H / 8);
+        L.n_counters, L.bm, reinterpret_cast<uint4*>(xp), H / 8);
     if (launched() != MOE_OK) return MOE_ERR_CUDA;
     prof.mark();
     prof.mark();
@@ -457,12 +479,12 @@ moe_status_t moe_forward(const void* x, const void* w_router, const float* route
     prof.mark();
     // 2. dispatch
     if (L.nchunks == 1) {
-      dispatch_small_kernel<<<1, 256, 0, st>>>(ids, P, E, GM_BM, counts, offsets, perm, inv,
+      dispatch_small_kernel<<<1, 256, 0, st>>>(ids, P, E, L.bm, counts, offsets, perm, inv,
                                                tile_num, tile_expert, tile_row0, tile_rows,
                                                gemm_counters, L.n_counters);
     } else {
       dispatch_count_kernel<<<L.nchunks, 256, E * sizeof(int), st>>>(ids, P, E, chunk_counts);
-      dispatch_scan_kernel<<<1, 256, 0, st>>>(chunk_counts, L.nchunks, E, P, GM_BM, counts,
+      dispatch_scan_kernel<<<1, 256, 0, st>>>(chunk_counts, L.nchunks, E, P, L.bm, counts,
                                               offsets, chunk_base, tile_num, tile_expert, tile_row0,
                                               tile_rows, gemm_counters, L.n_counters);
       dispatch_rank_kernel<<<L.nchunks, 32, E * sizeof(int), st>>>(ids, P, E, chunk_base, perm,
@@ -473,22 +495,34 @@ moe_status_t moe_forward(const void* x, const void* w_router, const float* route
     if (launched() != MOE_OK) return MOE_ERR_CUDA;
     prof.mark();
   }
-  // 3. GEMM-1 + GEGLU
+  // 3. GEMM-1 + GEGLU, 4. GEMM-2 (down)
   const TileList tl{tile_num, tile_expert, tile_row0, tile_rows, 0};
-  const int smem = pgemm_smem_bytes<kGemmStages, 4>();
   float* partials = reinterpret_cast<float*>(ws + L.partials);
   const int G = std::min(std::max(1, d->num_sms), kMaxGemmCtas);
-  const int n1 = (I + 127) / 128;
-  GEMM_GEGLU<<<G, PG_THREADS, smem, st>>>(tm_xp, tm_wg, tm_wu, tl, n1, H, I, hbuf, I, partials,
-                                          gemm_counters);
-  if (launched() != MOE_OK) return MOE_ERR_CUDA;
-  prof.mark();
-  // 4. GEMM-2 (down)
-  const int n2 = (H + 255) / 256;
-  GEMM_STORE<<<G, PG_THREADS, smem, st>>>(tm_h, tm_wd, tm_wd, tl, n2, I, H, obuf, H, partials,
-                                          gemm_counters + L.n_counters / 2);
-  if (launched() != MOE_OK) return MOE_ERR_CUDA;
-  prof.mark();
+  int32_t* ctr1 = gemm_counters;
+  int32_t* ctr2 = gemm_counters + L.n_counters / 2;
+  if (dec) {
+    grouped_gemm_decode_kernel<EPI_GEGLU><<<G, DG_THREADS, decode_smem_bytes(I, true), st>>>(
+        tm_xp, tm_wg, tm_wu, tl, H, I, hbuf, I, partials, ctr1);
+    if (launched() != MOE_OK) return MOE_ERR_CUDA;
+    prof.mark();
+    grouped_gemm_decode_kernel<EPI_STORE><<<G, DG_THREADS, decode_smem_bytes(H, false), st>>>(
+        tm_h, tm_wd, tm_wd, tl, I, H, obuf, H, partials, ctr2);
+    if (launched() != MOE_OK) return MOE_ERR_CUDA;
+    prof.mark();
+  } else {
+    const int smem = pgemm_smem_bytes<kGemmStages, 4>();
+    const int n1 = (I + 127) / 128;
+    GEMM_GEGLU<<<G, PG_THREADS, smem, st>>>(tm_xp, tm_wg, tm_wu, tl, n1, H, I, hbuf, I, partials,
+                                            ctr1);
+    if (launched() != MOE_OK) return MOE_ERR_CUDA;
+    prof.mark();
+    const int n2 = (H + 255) / 256;
+    GEMM_STORE<<<G, PG_THREADS, smem, st>>>(tm_h, tm_wd, tm_wd, tl, n2, I, H, obuf, H, partials,
+                                            ctr2);
+    if (launched() != MOE_OK) return MOE_ERR_CUDA;
+    prof.mark();
+  }
   // 5. combine
   const long long cthreads = (long long)T * (H / 8);
   combine_kernel<<<(int)std::min<long long>((cthreads + 255) / 256, gsm), 256, 0, st>>>(
