@@ -243,6 +243,7 @@ def run_native(args, cfg) -> None:
         raise SystemExit("device status not OK after the first forward")
     counts = aux["expert_counts"].cpu().numpy()
     acc = algorithmic(cfg, counts, d["bias"] is not None)
+    rstats = moe.router_stats(aux)
 
     # The step as a serving loop runs it: one captured moe_forward per batch (graph replay).
     graph = moe.ForwardGraph(x, g["w_router"], g["w_gate"], g["w_up"], g["w_down"], cfg.k,
@@ -321,7 +322,12 @@ def run_native(args, cfg) -> None:
         kb = acc["gemm1_bytes"] if dom == "gemm1_geglu" else acc["gemm2_bytes"]
         kf = acc["gemm1_flops"] if dom == "gemm1_geglu" else acc["gemm2_flops"]
         ridge = pk["bf16_tflops"] * 1e12 / (pk["hbm_gbs"] * 1e9)
-        kname = "grouped_gemm_kernel<4,0>" if dom == "gemm1_geglu" else "grouped_gemm_kernel<4,1>"
+        if cfg.T <= 16:   # the library's decode tiles (at most 16 rows per expert)
+            kname = ("grouped_gemm_decode_kernel<EPI_GEGLU>" if dom == "gemm1_geglu"
+                     else "grouped_gemm_decode_kernel<EPI_STORE>")
+        else:
+            kname = ("grouped_gemm_persistent_kernel<4,EPI_GEGLU,4>" if dom == "gemm1_geglu"
+                     else "grouped_gemm_persistent_kernel<4,EPI_STORE,4>")
         traffic = ncu_traffic(kname, cfg.name)
         if kf / kb < ridge:
             achieved = kb / (dom_ms * 1e-3) / 1e9
@@ -359,6 +365,7 @@ def run_native(args, cfg) -> None:
                 "algorithmic_bytes": acc["step_bytes"], "algorithmic_flops": acc["step_flops"],
                 "active_experts": acc["active_experts"]},
             "stages_ms": stages,
+            "router_stats": rstats,
             "e2e": {"value": world * cfg.T / (e2e_ms * 1e-3), "unit": UNIT,
                     "h2d_bytes_per_step": cfg.T * cfg.H * 2,
                     "d2h_bytes_per_step": cfg.T * cfg.H * 2},

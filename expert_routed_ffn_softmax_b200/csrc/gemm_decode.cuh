@@ -125,7 +125,7 @@ struct DSched {
 template <int MODE>
 __global__ void __launch_bounds__(DG_THREADS, 1)
     grouped_gemm_decode_kernel(const __grid_constant__ CUtensorMap tmX,   // activations, box 16x16
-                               const __grid_constant__ CUtensorMap tmW0,  // weights, box 64x16x1
+                               const __grid_constant__ CUtensorMap tmW0,  // weights, 16 rows x all slabs
                                const __grid_constant__ CUtensorMap tmW1,  // (up weights for GEGLU)
                                TileList tiles, int K, int N_out, void* __restrict__ out_ptr,
                                int ldo, float* __restrict__ partials,
@@ -212,11 +212,9 @@ __global__ void __launch_bounds__(DG_THREADS, 1)
           const uint32_t sB = sA + sh.nm * 2 * DG_SLAB;
           mbar_arrive_expect_tx(full_bar(s), tx);
           tma_load_2d(sB, &tmX, full_bar(s), ks * DG_KS, row0);
-          for (int j = 0; j < sh.nsl; ++j) {
-            tma_load_3d(sA + j * DG_SLAB, &tmW0, full_bar(s), 64 * j, ks * DG_KS, e);
-            if (GEGLU)
-              tma_load_3d(sA + (2 * sh.mt + j) * DG_SLAB, &tmW1, full_bar(s), 64 * j, ks * DG_KS, e);
-          }
+          // one load per projection: 16 K-rows x all nsl slabs of the expert
+          tma_load_4d(sA, &tmW0, full_bar(s), 0, ks * DG_KS, 0, e);
+          if (GEGLU) tma_load_4d(sA + 2 * sh.mt * DG_SLAB, &tmW1, full_bar(s), 0, ks * DG_KS, 0, e);
           *n_issued = q + 1;
         }
       }

@@ -226,17 +226,13 @@ __global__ void __launch_bounds__(PG_THREADS, 1)
           const uint32_t sB = sA + GM_A_BYTES;
           mbar_arrive_expect_tx(full_bar(s), STAGE_BYTES);
           tma_load_2d(sA, &tmA, full_bar(s), kc * GM_BK, row0);
+          // one load per projection: NSLAB/2 (gate, up) or NSLAB (down) 64-column slabs
           if (MODE == EPI_GEGLU) {
-#pragma unroll
-            for (int j = 0; j < NSLAB / 2; ++j) {
-              tma_load_3d(sB + j * GM_SLAB_BYTES, &tmB0, full_bar(s), n0 + 64 * j, kc * GM_BK, e);
-              tma_load_3d(sB + (NSLAB / 2 + j) * GM_SLAB_BYTES, &tmB1, full_bar(s), n0 + 64 * j,
-                          kc * GM_BK, e);
-            }
+            tma_load_4d(sB, &tmB0, full_bar(s), 0, kc * GM_BK, n0 / 64, e);
+            tma_load_4d(sB + (NSLAB / 2) * GM_SLAB_BYTES, &tmB1, full_bar(s), 0, kc * GM_BK,
+                        n0 / 64, e);
           } else {
-#pragma unroll
-            for (int j = 0; j < NSLAB; ++j)
-              tma_load_3d(sB + j * GM_SLAB_BYTES, &tmB0, full_bar(s), n0 + 64 * j, kc * GM_BK, e);
+            tma_load_4d(sB, &tmB0, full_bar(s), 0, kc * GM_BK, n0 / 64, e);
           }
           *n_issued = q + 1;
         }

@@ -200,6 +200,23 @@ bool make_map_3d(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Stacked [E][rows][cols] bf16 viewed as (64 columns, rows, cols/64 slabs, E), box = 64 columns
+// x box_rows rows x box_slabs slabs x 1: one load fills box_slabs consecutive 64-column slabs
+// of box_rows rows each (slab-major in shared memory, 128-byte swizzle), the layout of the
+// MN-major MMA operand.  Every in-bounds coordinate addresses memory inside the tensor.
+bool make_map_slabs(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, uint64_t E,
+                    uint32_t box_rows, uint32_t box_slabs) {
+  auto fn = encode_fn();
+  if (!fn || cols % 64) return false;
+  cuuint64_t dims[4] = {64, rows, cols / 64, E};
+  cuuint64_t strides[3] = {cols * 2, 128, cols * rows * 2};
+  cuuint32_t box[4] = {64, box_rows, box_slabs, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // --------------------------------------------------------------------------- per device
 struct DeviceState {
   bool attrs_set = false;
@@ -446,11 +463,15 @@ moe_status_t moe_forward(const void* x, const void* w_router, const float* route
   const bool dec = L.bm == DG_BN;    // decode tiles: <= 16 rows per expert
   CUtensorMap tm_xp, tm_wg, tm_wu, tm_h, tm_wd;
   const uint32_t act_rows = dec ? DG_BN : GM_BM, act_cols = dec ? DG_KS : 64;
+  // weight boxes: decode = 16 rows x every slab of the expert; prefill = 64 rows x 2 (gate,
+  // up) or 4 (down) slabs
   const uint32_t w_rows = dec ? DG_KS : 64;
+  const uint32_t gu_slabs = dec ? (uint32_t)(I / 64) : 2u, d_slabs = dec ? (uint32_t)(H / 64) : 4u;
   if (!make_map_2d(&tm_xp, xp, H, P, act_rows, act_cols) ||
-      !make_map_3d(&tm_wg, w_gate, I, H, E, w_rows) || !make_map_3d(&tm_wu, w_up, I, H, E, w_rows) ||
+      !make_map_slabs(&tm_wg, w_gate, I, H, E, w_rows, gu_slabs) ||
+      !make_map_slabs(&tm_wu, w_up, I, H, E, w_rows, gu_slabs) ||
       !make_map_2d(&tm_h, hbuf, I, P, act_rows, act_cols) ||
-      !make_map_3d(&tm_wd, w_down, H, I, E, w_rows))
+      !make_map_slabs(&tm_wd, w_down, H, I, E, w_rows, d_slabs))
     return MOE_ERR_CUDA;
 
   Profiler prof{d, st, (flags & MOE_FLAG_PROFILE_STAGES) != 0};
