@@ -54,11 +54,34 @@ __global__ void __cluster_dims__(kFrontRanks, 1, 1) __launch_bounds__(128, 1)
   const int nt = T;
 
   // ---- 1. partial logits over this CTA's h-slice
-  for (int i = tid; i < hs * TT; i += blockDim.x) {
-    const int tt = i / hs, hh = i - tt * hs;
-    double v = 0.0;
-    if (tt < nt) v = (double)__bfloat162float(x[(size_t)tt * H + h0 + hh]);
-    work[hh * TT + tt] = v;
+  // x slice as 16-byte vectors, 4 per thread in flight before any is used.
+  {
+    const int nv = hs / 8, total = TT * nv;
+    for (int b0 = tid; b0 < total; b0 += 4 * blockDim.x) {
+      uint4 r[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int idx = b0 + u * blockDim.x;
+        const int tt = idx / nv, v = idx - tt * nv;
+        r[u] = make_uint4(0, 0, 0, 0);
+        if (idx < total && tt < nt)
+          r[u] = __ldg(reinterpret_cast<const uint4*>(x + (size_t)tt * H + h0) + v);
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int idx = b0 + u * blockDim.x;
+        if (idx < total) {
+          const int tt = idx / nv, v = idx - tt * nv;
+          const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&r[u]);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const float2 f = __bfloat1622float2(p2[i]);
+            work[(8 * v + 2 * i) * TT + tt] = (double)f.x;
+            work[(8 * v + 2 * i + 1) * TT + tt] = (double)f.y;
+          }
+        }
+      }
+    }
   }
   __syncthreads();
   for (int tt = warp; tt < TT; tt += NW) {
@@ -176,13 +199,26 @@ __global__ void __cluster_dims__(kFrontRanks, 1, 1) __launch_bounds__(128, 1)
   }
   cluster_sync();
 
-  // ---- 3. gather the x rows of the sorted pairs
+  // ---- 3. gather the x rows of the sorted pairs (16-byte vectors, 8 per thread in flight)
   const int P = nt * k;
-  for (int pos = rank * NW + warp; pos < P; pos += kFrontRanks * NW) {
-    const int t = __ldcg(perm + pos) / k;
-    const uint4* src = reinterpret_cast<const uint4*>(x) + (size_t)t * nvec;
-    uint4* dst = xp + (size_t)pos * nvec;
-    for (int v = lane; v < nvec; v += 32) dst[v] = src[v];
+  const long long total = (long long)P * nvec;
+  const int nthr = kFrontRanks * blockDim.x;
+  for (long long b0 = rank * blockDim.x + tid; b0 < total; b0 += 8LL * nthr) {
+    uint4 r[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const long long idx = b0 + (long long)u * nthr;
+      if (idx < total) {
+        const int pos = (int)(idx / nvec), v = (int)(idx - (long long)pos * nvec);
+        const int t = __ldcg(perm + pos) / k;
+        r[u] = __ldg(reinterpret_cast<const uint4*>(x) + (size_t)t * nvec + v);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const long long idx = b0 + (long long)u * nthr;
+      if (idx < total) xp[idx] = r[u];
+    }
   }
 }
 

@@ -222,17 +222,29 @@ __global__ void __launch_bounds__(256) dispatch_small_kernel(
                        s_tstart);
 }
 
-// Xp[pos, :] = x[perm[pos] / k, :]   (16-byte vectors; one warp per row, grid-stride)
+// Xp[pos, :] = x[perm[pos] / k, :]   (16-byte vectors over all (row, vector) pairs,
+// 8 loads per thread issued before the stores)
 __global__ void __launch_bounds__(256) gather_rows_kernel(const uint4* __restrict__ x,
                                                           const int32_t* __restrict__ perm, int P,
                                                           int k, int nvec, uint4* __restrict__ xp) {
-  const int lane = threadIdx.x & 31;
-  const int wpb = blockDim.x >> 5;
-  for (int pos = blockIdx.x * wpb + (threadIdx.x >> 5); pos < P; pos += gridDim.x * wpb) {
-    const int t = perm[pos] / k;
-    const uint4* src = x + (size_t)t * nvec;
-    uint4* dst = xp + (size_t)pos * nvec;
-    for (int v = lane; v < nvec; v += 32) dst[v] = src[v];
+  const long long total = (long long)P * nvec;
+  const long long nthr = (long long)gridDim.x * blockDim.x;
+  for (long long b0 = (long long)blockIdx.x * blockDim.x + threadIdx.x; b0 < total;
+       b0 += 8 * nthr) {
+    uint4 r[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const long long idx = b0 + u * nthr;
+      if (idx < total) {
+        const int pos = (int)(idx / nvec), v = (int)(idx - (long long)pos * nvec);
+        r[u] = x[(size_t)(perm[pos] / k) * nvec + v];
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const long long idx = b0 + u * nthr;
+      if (idx < total) xp[idx] = r[u];
+    }
   }
 }
 

@@ -295,19 +295,48 @@ __global__ void __launch_bounds__(DG_THREADS, 1)
       last = __shfl_sync(0xffffffffu, last, 0);
       if (last) {
         __threadfence();
-        for (int m = 0; m < sh.mt; ++m) {
-          const int f = m * 128 + fl;
-          if (f >= N_out) continue;
-          for (int t = 0; t < rows; ++t) {
-            float g = 0.f, u = 0.f;
-            for (int p = 0; p < n_pieces; ++p) {
-              const float* src =
-                  partials + (size_t)sch.slot(g_first + p, it.tile) * DG_BN * prow + (size_t)t * prow;
-              g += __ldcg(src + m * 128 + fl);
-              if (GEGLU) u += __ldcg(src + (sh.mt + m) * 128 + fl);
+        // (m, t) pairs of this thread, 4 at a time, with the loads of up to 8 pieces each
+        // issued before they are added (in piece order)
+        const int npair = sh.mt * rows;
+        for (int q0 = 0; q0 < npair; q0 += 4) {
+          float g[4], u[4];
+#pragma unroll
+          for (int a = 0; a < 4; ++a) g[a] = u[a] = 0.f;
+          for (int p0 = 0; p0 < n_pieces; p0 += 8) {
+            float gp[4][8], up[4][8];
+#pragma unroll
+            for (int a = 0; a < 4; ++a) {
+              const int qq = q0 + a, m = qq / rows, t = qq - m * rows;
+#pragma unroll
+              for (int b = 0; b < 8; ++b) {
+                gp[a][b] = up[a][b] = 0.f;
+                if (qq < npair && p0 + b < n_pieces && m * 128 + fl < N_out) {
+                  const float* src = partials +
+                                     (size_t)sch.slot(g_first + p0 + b, it.tile) * DG_BN * prow +
+                                     (size_t)t * prow;
+                  gp[a][b] = __ldcg(src + m * 128 + fl);
+                  if (GEGLU) up[a][b] = __ldcg(src + (sh.mt + m) * 128 + fl);
+                }
+              }
             }
-            const float o = GEGLU ? gelu_tanh_f(g) * u : g;
-            static_cast<__nv_bfloat16*>(out_ptr)[(size_t)(row0 + t) * ldo + f] = __float2bfloat16_rn(o);
+#pragma unroll
+            for (int a = 0; a < 4; ++a)
+#pragma unroll
+              for (int b = 0; b < 8; ++b)
+                if (p0 + b < n_pieces) {
+                  g[a] += gp[a][b];
+                  u[a] += up[a][b];
+                }
+          }
+#pragma unroll
+          for (int a = 0; a < 4; ++a) {
+            const int qq = q0 + a, m = qq / rows, t = qq - m * rows;
+            const int f = m * 128 + fl;
+            if (qq < npair && f < N_out) {
+              const float o = GEGLU ? gelu_tanh_f(g[a]) * u[a] : g[a];
+              static_cast<__nv_bfloat16*>(out_ptr)[(size_t)(row0 + t) * ldo + f] =
+                  __float2bfloat16_rn(o);
+            }
           }
         }
       }

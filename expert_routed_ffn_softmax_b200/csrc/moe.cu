@@ -73,14 +73,15 @@ bool shape_supported(int T, int H, int E, int I, int k, bool need_I) {
   return true;
 }
 
-// Split of the router's H axis over CTAs: a divisor d of H/4 with 64 <= H/d <= 1408 (the
-// per-CTA x stage stays within 88 KB), the smallest one that gives ~2 CTAs per SM.
+// Split of the router's H axis over CTAs: a divisor d of H/32 (so every warp's share is a
+// whole number of 8-element vectors) with 64 <= H/d <= 1408 (the per-CTA x stage stays
+// within 88 KB), the smallest one that gives ~2 CTAs per SM.
 int router_ksplit(int T, int H) {
   const int ntg = (T + kRouterTokens - 1) / kRouterTokens;
   const int target = (296 + ntg - 1) / ntg;
   int first = -1, largest = -1;
-  for (int d = 1; d <= H / 4; ++d) {
-    if ((H / 4) % d) continue;
+  for (int d = 1; d <= H / 32; ++d) {
+    if ((H / 32) % d) continue;
     const int hs = H / d;
     if (hs < 64 || hs > 1408) continue;
     largest = d;

@@ -41,11 +41,34 @@ __global__ void __launch_bounds__(128) router_partial_kernel(
   const int nt = min(TT, T - t0);
 
   // Stage x[t0:t0+TT, h0:h0+hs] as double, layout [h][t]; missing tokens are zero.
-  for (int i = tid; i < hs * TT; i += blockDim.x) {
-    const int tt = i / hs, hh = i - tt * hs;
-    double v = 0.0;
-    if (tt < nt) v = (double)__bfloat162float(x[(size_t)(t0 + tt) * H + h0 + hh]);
-    rsm[hh * TT + tt] = v;
+  // 16-byte vectors, 4 per thread in flight before any is used (hs % 8 == 0).
+  {
+    const int nv = hs / 8, total = TT * nv;
+    for (int b0 = tid; b0 < total; b0 += 4 * blockDim.x) {
+      uint4 r[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int idx = b0 + u * blockDim.x;
+        const int tt = idx / nv, v = idx - tt * nv;
+        r[u] = make_uint4(0, 0, 0, 0);
+        if (idx < total && tt < nt)
+          r[u] = __ldg(reinterpret_cast<const uint4*>(x + (size_t)(t0 + tt) * H + h0) + v);
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int idx = b0 + u * blockDim.x;
+        if (idx < total) {
+          const int tt = idx / nv, v = idx - tt * nv;
+          const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&r[u]);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const float2 f = __bfloat1622float2(p2[i]);
+            rsm[(8 * v + 2 * i) * TT + tt] = (double)f.x;
+            rsm[(8 * v + 2 * i + 1) * TT + tt] = (double)f.y;
+          }
+        }
+      }
+    }
   }
   __syncthreads();
 
