@@ -247,7 +247,7 @@ def run_native(args, cfg) -> None:
 
     # The step as a serving loop runs it: one captured moe_forward per batch (graph replay).
     graph = moe.ForwardGraph(x, g["w_router"], g["w_gate"], g["w_up"], g["w_down"], cfg.k,
-                             bias=g["bias"])
+                             bias=g["bias"], tiles=args.tiles)
     for _ in range(args.warmup):
         flush.zero_()
         graph.replay()
@@ -279,7 +279,7 @@ def run_native(args, cfg) -> None:
 
     # ---- per-stage device times: a graph of the same call with the library's stage events
     pgraph = moe.ForwardGraph(x, g["w_router"], g["w_gate"], g["w_up"], g["w_down"], cfg.k,
-                              bias=g["bias"], profile=True)
+                              bias=g["bias"], profile=True, tiles=args.tiles)
     stage_acc: dict[str, list[float]] = {}
     try:
         for _ in range(max(3, min(args.steps, 20))):
@@ -322,7 +322,7 @@ def run_native(args, cfg) -> None:
         kb = acc["gemm1_bytes"] if dom == "gemm1_geglu" else acc["gemm2_bytes"]
         kf = acc["gemm1_flops"] if dom == "gemm1_geglu" else acc["gemm2_flops"]
         ridge = pk["bf16_tflops"] * 1e12 / (pk["hbm_gbs"] * 1e9)
-        if cfg.T <= 16:   # the library's decode tiles (at most 16 rows per expert)
+        if (cfg.T <= 16 and args.tiles != "prefill"):   # decode tiles (<= 16 rows per expert)
             kname = ("grouped_gemm_decode_kernel<EPI_GEGLU>" if dom == "gemm1_geglu"
                      else "grouped_gemm_decode_kernel<EPI_STORE>")
         else:
@@ -391,6 +391,8 @@ def main():
     ap.add_argument("--ref-tokens", type=int, default=8)
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--tiles", default="auto", choices=["auto", "decode", "prefill"],
+                    help="expert-GEMM tile family (default: the library's choice)")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)     # at least 3 untimed warm-up steps
     cfg = wl.CONFIGS[args.config]

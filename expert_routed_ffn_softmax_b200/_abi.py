@@ -27,8 +27,11 @@ MOE_FLAG_NO_RENORM = 1 << 0
 MOE_FLAG_ROUTER_FP64 = 1 << 1
 MOE_FLAG_ROUTER_SCREEN = 1 << 2
 MOE_FLAG_PROFILE_STAGES = 1 << 3
+MOE_FLAG_DECODE_TILES = 1 << 4
+MOE_FLAG_PREFILL_TILES = 1 << 5
 
 _ROUTER_FLAGS = {"auto": 0, "fp64": MOE_FLAG_ROUTER_FP64, "screen": MOE_FLAG_ROUTER_SCREEN}
+_TILE_FLAGS = {"auto": 0, "decode": MOE_FLAG_DECODE_TILES, "prefill": MOE_FLAG_PREFILL_TILES}
 
 # Every function the header declares, with (restype, argtypes).
 _P, _I, _U, _SZ = ctypes.c_void_p, ctypes.c_int, ctypes.c_uint, ctypes.c_size_t
@@ -117,10 +120,12 @@ def _dev(t: torch.Tensor, name: str, dtype: torch.dtype, shape: tuple) -> int:
     return t.data_ptr()
 
 
-def _flags(renorm: bool, router: str, profile: bool = False) -> int:
+def _flags(renorm: bool, router: str, profile: bool = False, tiles: str = "auto") -> int:
     if router not in _ROUTER_FLAGS:
         raise ValueError(f"router must be one of {sorted(_ROUTER_FLAGS)}")
-    return ((0 if renorm else MOE_FLAG_NO_RENORM) | _ROUTER_FLAGS[router]
+    if tiles not in _TILE_FLAGS:
+        raise ValueError(f"tiles must be one of {sorted(_TILE_FLAGS)}")
+    return ((0 if renorm else MOE_FLAG_NO_RENORM) | _ROUTER_FLAGS[router] | _TILE_FLAGS[tiles]
             | (MOE_FLAG_PROFILE_STAGES if profile else 0))
 
 
@@ -152,7 +157,8 @@ def route(x: torch.Tensor, w_router: torch.Tensor, k: int, bias: torch.Tensor | 
 def forward(x: torch.Tensor, w_router: torch.Tensor, w_gate: torch.Tensor, w_up: torch.Tensor,
             w_down: torch.Tensor, k: int, bias: torch.Tensor | None = None, renorm: bool = True,
             aux: bool = False, out: torch.Tensor | None = None, profile: bool = False,
-            stream=None, workspace_buf: torch.Tensor | None = None, router: str = "auto"):
+            stream=None, workspace_buf: torch.Tensor | None = None, router: str = "auto",
+            tiles: str = "auto"):
     """The routed MoE FFN layer -> y bf16 [T,H] (and a dict of routing outputs if aux).
 
     workspace_buf: optional caller-owned uint8 CUDA tensor used as the workspace (else a
@@ -169,7 +175,7 @@ def forward(x: torch.Tensor, w_router: torch.Tensor, w_gate: torch.Tensor, w_up:
     pb = None if bias is None else _dev(bias, "bias", torch.float32, (E,))
     y = torch.empty((T, H), dtype=torch.bfloat16, device=dev) if out is None else out
     py = _dev(y, "out", torch.bfloat16, (T, H))
-    flags = _flags(renorm, router, profile)
+    flags = _flags(renorm, router, profile, tiles)
     a = None
     aux_d = None
     if aux:
@@ -235,17 +241,17 @@ class ForwardGraph:
     """
 
     def __init__(self, x, w_router, w_gate, w_up, w_down, k, bias=None, renorm=True,
-                 profile=False, router="auto"):
+                 profile=False, router="auto", tiles="auto"):
         self.x = x
         T, H = x.shape
         E, _, I = w_gate.shape
         self.y = torch.empty((T, H), dtype=torch.bfloat16, device=x.device)
-        flags = _flags(renorm, router, profile)
+        flags = _flags(renorm, router, profile, tiles)
         self.workspace = torch.empty(max(1, workspace_bytes(T, H, E, I, k, flags)),
                                      dtype=torch.uint8, device=x.device)
         self._args = (w_router, w_gate, w_up, w_down, k)
         self._kw = dict(bias=bias, renorm=renorm, profile=profile, workspace_buf=self.workspace,
-                        router=router)
+                        router=router, tiles=tiles)
         forward(self.x, *self._args, out=self.y, **self._kw)    # set-up + workspace, uncaptured
         torch.cuda.synchronize(x.device)
         self.graph = torch.cuda.CUDAGraph()

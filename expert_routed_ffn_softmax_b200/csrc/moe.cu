@@ -31,7 +31,8 @@ constexpr int kFrontSmemMax = 200 * 1024;        // decode front kernel's dynami
 
 constexpr double kScreenC = 1.0 / 1024.0;        // screen error bound / (|x| |w|)
 constexpr unsigned kKnownFlags = MOE_FLAG_NO_RENORM | MOE_FLAG_ROUTER_FP64 |
-                                 MOE_FLAG_ROUTER_SCREEN | MOE_FLAG_PROFILE_STAGES;
+                                 MOE_FLAG_ROUTER_SCREEN | MOE_FLAG_PROFILE_STAGES |
+                                 MOE_FLAG_DECODE_TILES | MOE_FLAG_PREFILL_TILES;
 
 #define GEMM_GEGLU grouped_gemm_persistent_kernel<kGemmStages, EPI_GEGLU, 4>
 #define GEMM_STORE grouped_gemm_persistent_kernel<kGemmStages, EPI_STORE, 4>
@@ -40,6 +41,7 @@ constexpr unsigned kKnownFlags = MOE_FLAG_NO_RENORM | MOE_FLAG_ROUTER_FP64 |
 bool flags_ok(unsigned flags) {
   if (flags & ~kKnownFlags) return false;
   if ((flags & MOE_FLAG_ROUTER_FP64) && (flags & MOE_FLAG_ROUTER_SCREEN)) return false;
+  if ((flags & MOE_FLAG_DECODE_TILES) && (flags & MOE_FLAG_PREFILL_TILES)) return false;
   return true;
 }
 
@@ -52,8 +54,13 @@ bool router_uses_screen(int T, unsigned flags) {
 
 // Batches of at most 16 tokens (so at most 16 rows per expert) use the decode GEMMs.
 constexpr int kDecodeMaxTokens = 16;
-bool use_decode_gemm(int T, int H, int I) {
+bool decode_gemm_ok(int T, int H, int I) {
   return T <= kDecodeMaxTokens && decode_shape_ok(I, true) && decode_shape_ok(H, false);
+}
+bool use_decode_gemm(int T, int H, int I, unsigned flags) {
+  if (flags & MOE_FLAG_PREFILL_TILES) return false;
+  if (flags & MOE_FLAG_DECODE_TILES) return decode_gemm_ok(T, H, I);
+  return decode_gemm_ok(T, H, I);
 }
 
 // Batches of at most 8 tokens take the fused router + dispatch + gather launch.
@@ -127,7 +134,7 @@ Layout make_layout(int T, int H, int E, int I, int k, unsigned flags, bool forwa
   }
   if (forward) {
     L.nchunks = (int)((P + kDispatchChunk - 1) / kDispatchChunk);
-    L.bm = use_decode_gemm(T, H, I) ? DG_BN : GM_BM;
+    L.bm = use_decode_gemm(T, H, I, flags) ? DG_BN : GM_BM;
     L.max_tiles = (int)(P / L.bm) + E;
     L.ids = take(sizeof(int32_t) * P);
     L.wts = take(sizeof(float) * P);
@@ -432,6 +439,7 @@ moe_status_t moe_forward(const void* x, const void* w_router, const float* route
     return MOE_ERR_INVALID_ARG;
   if (x == y) return MOE_ERR_INVALID_ARG;
   if (!shape_supported(T, H, E, I, k, true)) return MOE_ERR_UNSUPPORTED;
+  if ((flags & MOE_FLAG_DECODE_TILES) && !decode_gemm_ok(T, H, I)) return MOE_ERR_INVALID_ARG;
   const Layout L = make_layout(T, H, E, I, k, flags, true);
   if (workspace_bytes < L.total) return MOE_ERR_NO_WORKSPACE;
   int dev = 0;

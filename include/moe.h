@@ -63,7 +63,13 @@ enum {
   MOE_FLAG_ROUTER_SCREEN = 1u << 2,
   /* Record a CUDA event at every stage boundary of the call; moe_last_stage_times()
    * then reports the per-stage device times of the most recent such call. */
-  MOE_FLAG_PROFILE_STAGES = 1u << 3
+  MOE_FLAG_PROFILE_STAGES = 1u << 3,
+  /* Expert-GEMM tile family (moe_forward).  Decode tiles (weights as the 128-row MMA
+   * operand, at most 16 tokens as the other; T <= 16 only) or prefill tiles (128 sorted
+   * rows x 256 columns).  By default the library picks; setting both, or decode tiles for
+   * T > 16, is MOE_ERR_INVALID_ARG. */
+  MOE_FLAG_DECODE_TILES = 1u << 4,
+  MOE_FLAG_PREFILL_TILES = 1u << 5
 };
 
 /* Optional caller-owned device outputs of moe_forward (any member may be NULL). */

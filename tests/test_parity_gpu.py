@@ -45,9 +45,9 @@ def layer_inputs(cfg, gemma_w, seed=0, T=None):
 SCREEN_C = 2.0 ** -10     # the kernel's screen error bound, in units of |x_t| |w_e|
 
 
-def gpu_forward(x, g, k, renorm=True, router="auto"):
+def gpu_forward(x, g, k, renorm=True, router="auto", tiles="auto"):
     y, aux = moe.forward(x.cuda(), g["w_router"], g["w_gate"], g["w_up"], g["w_down"], k,
-                         bias=g["bias"], renorm=renorm, aux=True, router=router)
+                         bias=g["bias"], renorm=renorm, aux=True, router=router, tiles=tiles)
     assert moe.sync_status() == 0
     st = moe.router_stats(aux)
     if st["path"] == "screen":
@@ -85,10 +85,10 @@ def sample_tokens(T, n, seed=0):
     return np.unique(np.concatenate([[0, T - 1], s]))
 
 
-def run_case(cfg, gemma_w, n_sample, T=None, renorm=True, router="auto"):
+def run_case(cfg, gemma_w, n_sample, T=None, renorm=True, router="auto", tiles="auto"):
     x, c, g = layer_inputs(cfg, gemma_w, T=T)
     T = x.shape[0]
-    y, aux = gpu_forward(x, g, cfg.k, renorm, router)
+    y, aux = gpu_forward(x, g, cfg.k, renorm, router, tiles)
     rows = sample_tokens(T, n_sample)
     ref = oracle.forward(x, c["w_router"], c["w_gate"], c["w_up"], c["w_down"], cfg.k,
                          bias=c["bias"], renorm=renorm, tokens=rows)
@@ -120,6 +120,13 @@ def test_forward_ragged_gemma(T, gemma_w):
                                          ("sweep_T512", "fp64"), ("prefill", "fp64")])
 def test_forward_forced_router_path(name, router, gemma_w):
     run_case(wl.CONFIGS[name], gemma_w, 256, router=router)
+
+
+@pytest.mark.parametrize("tiles", ["decode", "prefill"])
+@pytest.mark.parametrize("name,T", [("tiny", 16), ("tiny", 3), ("decode", 8), ("decode", 1),
+                                    ("decode", 16)])
+def test_forward_tile_families(name, T, tiles, gemma_w):
+    run_case(wl.CONFIGS[name], gemma_w, 64, T=T, tiles=tiles)
 
 
 def test_forward_no_renorm(gemma_w):
