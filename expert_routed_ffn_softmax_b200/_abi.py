@@ -41,6 +41,7 @@ SIGNATURES = {
     "moe_route_workspace_size": (_SZ, [_I, _I, _I, _I, _U]),
     "moe_workspace_size": (_SZ, [_I, _I, _I, _I, _I, _U]),
     "moe_route": (_I, [_P, _P, _P, _I, _I, _I, _I, _U, _P, _P, _P, _SZ, _P]),
+    "moe_route_static": (_I, [_P, _P, _P, _I, _I, _I, _I, _U, _P, _P, _P]),
     "moe_forward": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _U, _P, _P, _P, _SZ, _P]),
     "moe_sync_status": (_I, [_P]),
     "moe_last_stage_times": (_I, [ctypes.POINTER(ctypes.c_float), _I]),

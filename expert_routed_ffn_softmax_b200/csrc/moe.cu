@@ -363,6 +363,13 @@ moe_status_t launch_router(const __nv_bfloat16* x, const __nv_bfloat16* wr, cons
   return launched();
 }
 
+// Scratch of moe_route_static: a file-scope device array (every GPU that loads this
+// library holds it until the process exits).  Host code must not use the symbol itself as a
+// device address; moe_route_static looks its address up once per device.
+constexpr size_t kStaticScratchBytes = 4u << 20;
+__device__ __align__(256) uint8_t g_static_scratch[kStaticScratchBytes];
+void* g_static_scratch_ptr[kMaxDevices] = {};
+
 __global__ void unsatisfied_wait_kernel() {
   __shared__ __align__(8) uint64_t bar;
   const uint32_t b = smem_u32(&bar);
@@ -563,6 +570,41 @@ moe_status_t moe_forward(const void* x, const void* w_router, const float* route
   prof.mark();
   prof.finish();
   return MOE_OK;
+}
+
+moe_status_t moe_route_static(const void* x, const void* w_router, const float* router_bias,
+                              int T, int H, int E, int k, unsigned flags, int32_t* topk_ids,
+                              float* topk_weights, void* stream) {
+  if (T < 0 || H <= 0 || E <= 0 || k < 1 || k > E) return MOE_ERR_INVALID_ARG;
+  if (!flags_ok(flags) || (flags & (MOE_FLAG_ROUTER_SCREEN | MOE_FLAG_PROFILE_STAGES)))
+    return MOE_ERR_INVALID_ARG;
+  if (T == 0) return MOE_OK;
+  if (!x || !w_router || !topk_ids || !topk_weights) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(w_router)) return MOE_ERR_INVALID_ARG;
+  if (!shape_supported(T, H, E, 64, k, false)) return MOE_ERR_UNSUPPORTED;
+  const unsigned f = flags | MOE_FLAG_ROUTER_FP64;   // fp64 logits: no screen buffers
+  const Layout L = make_layout(T, H, E, 64, k, f, false);
+  if (L.total > kStaticScratchBytes) return MOE_ERR_NO_WORKSPACE;
+  int dev = 0;
+  DeviceState* d = device_state(&dev);
+  if (!d) return MOE_ERR_CUDA;
+  void* scratch = nullptr;
+  {
+    // First call on this device: look up the array's device address (with this device
+    // current).  Later calls reuse it.
+    std::lock_guard<std::mutex> lk(g_dev_mu);
+    if (!g_static_scratch_ptr[dev]) {
+      void* p = nullptr;
+      if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || !p) return MOE_ERR_CUDA;
+      g_static_scratch_ptr[dev] = p;
+    }
+    scratch = g_static_scratch_ptr[dev];
+  }
+  uint8_t* ws = static_cast<uint8_t*>(scratch);
+  return launch_router(static_cast<const __nv_bfloat16*>(x),
+                       static_cast<const __nv_bfloat16*>(w_router), router_bias, T, H, E, k, f,
+                       topk_ids, topk_weights, reinterpret_cast<unsigned*>(ws + L.stats), ws, L,
+                       *d, static_cast<cudaStream_t>(stream));
 }
 
 moe_status_t moe_sync_status(void* stream) {

@@ -148,6 +148,34 @@ moe_status_t moe_forward(const void *x, const void *w_router, const float *route
                          int E, int I, int k, unsigned flags, void *y, const moe_aux_t *aux,
                          void *workspace, size_t workspace_bytes, void *stream);
 
+/*
+ * moe_route_static -- moe_route for callers that cannot allocate device memory.
+ *
+ * The pages have no counterpart of this call; it exists for the library's users.  Some
+ * callers have no way to provide the workspace moe_route needs: code that runs while a
+ * stream is being captured into a CUDA graph (cudaMalloc is not allowed there and would
+ * synchronise the device), plugin hosts that hand a kernel only its inputs and outputs,
+ * and runtimes with a fixed memory budget that forbid allocations after start-up.  This
+ * entry point takes the same inputs and outputs as moe_route (all caller-owned device
+ * memory) and allocates nothing: its scratch is a 4 MiB array compiled into the library,
+ * which every GPU that loads the library holds until the process exits.
+ *
+ *   Same arguments, results and ranking guarantee as moe_route, always on the fp64 logits
+ *   path.  MOE_FLAG_ROUTER_SCREEN and MOE_FLAG_PROFILE_STAGES are MOE_ERR_INVALID_ARG.
+ *   The scratch a call needs is moe_route_workspace_size(T, H, E, k, MOE_FLAG_ROUTER_FP64);
+ *   above 4 MiB the call returns MOE_ERR_NO_WORKSPACE and launches nothing (at the Gemma-4
+ *   shape, H = 2816, E = 128, k = 8, batches of T = 1..64, 128 and 256 tokens fit).
+ *   The first call on a device looks up the array's device address (cudaGetSymbolAddress
+ *   with that device current); make that first call before any stream capture.
+ *   All calls on a device share the one array and it keeps the last call's contents (the
+ *   counters that must start at zero are cleared by every call): calls whose GPU work
+ *   overlaps -- on different streams, or from several host threads -- race on it and must
+ *   be serialised by the caller.
+ */
+moe_status_t moe_route_static(const void *x, const void *w_router, const float *router_bias,
+                              int T, int H, int E, int k, unsigned flags, int32_t *topk_ids,
+                              float *topk_weights, void *stream);
+
 /* Synchronise `stream`, then read and clear this device's error word.
  * MOE_OK, MOE_ERR_TIMEOUT (a bounded device wait ran out), or MOE_ERR_CUDA (a CUDA error,
  * or an out-of-range index seen by a kernel). */
