@@ -238,7 +238,7 @@ def run_native(args, cfg) -> None:
     stream = torch.cuda.current_stream()
 
     y0, aux = moe.forward(x, g["w_router"], g["w_gate"], g["w_up"], g["w_down"], cfg.k,
-                          bias=g["bias"], aux=True)
+                          bias=g["bias"], aux=True, tiles=args.tiles)
     if moe.sync_status() != 0:
         raise SystemExit("device status not OK after the first forward")
     counts = aux["expert_counts"].cpu().numpy()
@@ -322,7 +322,7 @@ def run_native(args, cfg) -> None:
         kb = acc["gemm1_bytes"] if dom == "gemm1_geglu" else acc["gemm2_bytes"]
         kf = acc["gemm1_flops"] if dom == "gemm1_geglu" else acc["gemm2_flops"]
         ridge = pk["bf16_tflops"] * 1e12 / (pk["hbm_gbs"] * 1e9)
-        if (cfg.T <= 16 and args.tiles != "prefill"):   # decode tiles (<= 16 rows per expert)
+        if args.tiles == "decode":   # decode tiles (<= 16 rows per expert)
             kname = ("grouped_gemm_decode_kernel<EPI_GEGLU>" if dom == "gemm1_geglu"
                      else "grouped_gemm_decode_kernel<EPI_STORE>")
         else:

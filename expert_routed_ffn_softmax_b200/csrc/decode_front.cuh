@@ -2,7 +2,7 @@
 // launch: one cluster of 8 CTAs.
 //
 //   1. CTA r computes fp64 partial logits of all 8 tokens x E experts over the h-slice
-//      [r*H/8, (r+1)*H/8) (4 warps, each an FMA chain in ascending h over a quarter of the
+//      [r*H/8, (r+1)*H/8) (8 warps, each an FMA chain in ascending h over an eighth of the
 //      slice, added in warp order), plus partial squared norms, and writes them into CTA 0's
 //      shared memory through distributed shared memory (st.shared::cluster);
 //   2. cluster barrier; CTA 0 adds the 8 partials in rank order and finishes every token
@@ -10,7 +10,7 @@
 //      sequential exact recomputation when too close, renormalised weights), then runs the
 //      single-CTA dispatch (counts, offsets, stable permutation, tile list);
 //   3. cluster barrier; all 32 warps of the cluster copy the x rows into Xp.
-// The summation depth per logit is H/32 + 3 + 7 + 1 (<= H + 8), inside the bound the
+// The summation depth per logit is H/64 + 7 + 7 + 1 (<= H + 8), inside the bound the
 // verification uses.
 #pragma once
 #include "ptx.cuh"
@@ -21,17 +21,19 @@ namespace moe {
 
 constexpr int kFrontRanks = 8;
 constexpr int kFrontMaxTokens = 8;
+constexpr int kFrontWarps = 8;      // one token per warp in the finishing CTA
 
 // Dynamic shared memory (doubles): part [8][8][E] | pxn [8][8] | pwn [8][E] | work region
-// max(hs*8, 4*8*E) (x stage, then the cross-warp reduction).
+// max(hs*8, warps*8*E) (x stage, then the cross-warp reduction).
 __host__ __device__ inline size_t decode_front_smem_bytes(int H, int E) {
   const size_t hs = (size_t)H / kFrontRanks;
-  const size_t work = hs * 8 > (size_t)4 * 8 * E ? hs * 8 : (size_t)4 * 8 * E;
+  const size_t red = (size_t)kFrontWarps * 8 * E;
+  const size_t work = hs * 8 > red ? hs * 8 : red;
   return sizeof(double) * ((size_t)kFrontRanks * 8 * E + kFrontRanks * 8 + (size_t)kFrontRanks * E + work);
 }
 
 template <int EPL>
-__global__ void __cluster_dims__(kFrontRanks, 1, 1) __launch_bounds__(128, 1)
+__global__ void __cluster_dims__(kFrontRanks, 1, 1) __launch_bounds__(32 * kFrontWarps, 1)
     decode_front_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __restrict__ wr,
                         const float* __restrict__ bias, int T, int H, int E, int k, int renorm,
                         double beta_scale, int32_t* __restrict__ ids, float* __restrict__ wts,
@@ -41,7 +43,9 @@ __global__ void __cluster_dims__(kFrontRanks, 1, 1) __launch_bounds__(128, 1)
                         int32_t* __restrict__ tile_expert, int32_t* __restrict__ tile_row0,
                         int32_t* __restrict__ tile_rows, int32_t* __restrict__ gemm_counters,
                         int n_counters, int BM, uint4* __restrict__ xp, int nvec) {
-  constexpr int TT = kFrontMaxTokens, NW = 4;
+  pdl_trigger();
+  pdl_wait();
+  constexpr int TT = kFrontMaxTokens, NW = kFrontWarps;
   extern __shared__ double fsm[];
   __shared__ int s_cnt[256], s_off[256], s_base[256], s_tstart[256];
   double* part = fsm;                                   // [8][TT][E]   (filled in CTA 0)

@@ -18,6 +18,8 @@ constexpr int kDispatchChunk = 2048;   // pairs per chunk
 __global__ void __launch_bounds__(256) dispatch_count_kernel(const int32_t* __restrict__ ids,
                                                               int P, int E,
                                                               int32_t* __restrict__ chunk_counts) {
+  pdl_trigger();
+  pdl_wait();
   extern __shared__ int hist[];
   for (int e = threadIdx.x; e < E; e += blockDim.x) hist[e] = 0;
   __syncthreads();
@@ -44,6 +46,8 @@ __global__ void __launch_bounds__(256) dispatch_scan_kernel(
     int32_t* __restrict__ tile_num, int32_t* __restrict__ tile_expert,
     int32_t* __restrict__ tile_row0, int32_t* __restrict__ tile_rows,
     int32_t* __restrict__ gemm_counters, int n_counters) {
+  pdl_trigger();
+  pdl_wait();
   __shared__ int s_cnt[256], s_off[256], s_tstart[256];
   for (int i = threadIdx.x; i < n_counters; i += blockDim.x) gemm_counters[i] = 0;
   const int e = threadIdx.x;
@@ -90,6 +94,8 @@ __global__ void __launch_bounds__(32) dispatch_rank_kernel(const int32_t* __rest
                                                            const int32_t* __restrict__ chunk_base,
                                                            int32_t* __restrict__ perm,
                                                            int32_t* __restrict__ inv) {
+  pdl_trigger();
+  pdl_wait();
   extern __shared__ int base[];
   const int lane = threadIdx.x;
   for (int e = lane; e < E; e += 32) base[e] = chunk_base[(size_t)blockIdx.x * E + e];
@@ -216,6 +222,8 @@ __global__ void __launch_bounds__(256) dispatch_small_kernel(
     int32_t* __restrict__ tile_num, int32_t* __restrict__ tile_expert,
     int32_t* __restrict__ tile_row0, int32_t* __restrict__ tile_rows,
     int32_t* __restrict__ gemm_counters, int n_counters) {
+  pdl_trigger();
+  pdl_wait();
   __shared__ int s_cnt[256], s_off[256], s_base[256], s_tstart[256];
   dispatch_small_block(ids, P, E, BM, counts, offsets, perm, inv, tile_num, tile_expert,
                        tile_row0, tile_rows, gemm_counters, n_counters, s_cnt, s_off, s_base,
@@ -227,6 +235,8 @@ __global__ void __launch_bounds__(256) dispatch_small_kernel(
 __global__ void __launch_bounds__(256) gather_rows_kernel(const uint4* __restrict__ x,
                                                           const int32_t* __restrict__ perm, int P,
                                                           int k, int nvec, uint4* __restrict__ xp) {
+  pdl_trigger();
+  pdl_wait();
   const long long total = (long long)P * nvec;
   const long long nthr = (long long)gridDim.x * blockDim.x;
   for (long long b0 = (long long)blockIdx.x * blockDim.x + threadIdx.x; b0 < total;
@@ -254,6 +264,8 @@ __global__ void __launch_bounds__(256) combine_kernel(const uint4* __restrict__ 
                                                       const int32_t* __restrict__ inv,
                                                       const float* __restrict__ w, int T, int k,
                                                       int nvec, uint4* __restrict__ y) {
+  pdl_trigger();
+  pdl_wait();
   const size_t total = (size_t)T * nvec;
   for (size_t idx = (size_t)blockIdx.x * blockDim.x + threadIdx.x; idx < total;
        idx += (size_t)gridDim.x * blockDim.x) {

@@ -131,10 +131,9 @@ __global__ void __launch_bounds__(DG_THREADS, 1)
                                int ldo, float* __restrict__ partials,
                                int* __restrict__ counters) {
   constexpr bool GEGLU = MODE == EPI_GEGLU;
-  if (*reinterpret_cast<volatile unsigned*>(&g_error_word) & MOE_DEVERR_TIMEOUT) return;
+  pdl_trigger();
   const DecodeShape sh = decode_shape(N_out, GEGLU);
   const int STAGES = sh.stages;
-  const int n_tiles = *tiles.num;
   const int nk = K / DG_KS;
   const int prow = sh.nm * 128;   // floats per token row of a partial tile
 
@@ -190,6 +189,10 @@ __global__ void __launch_bounds__(DG_THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // The prologue above overlaps the previous kernel; the tile list is its output.
+  pdl_wait();
+  const int n_tiles =
+      (*reinterpret_cast<volatile unsigned*>(&g_error_word) & MOE_DEVERR_TIMEOUT) ? 0 : *tiles.num;
 
   DSched sch;
   sch.init(blockIdx.x, gridDim.x, n_tiles, nk);

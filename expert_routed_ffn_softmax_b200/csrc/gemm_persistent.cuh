@@ -157,10 +157,7 @@ __global__ void __launch_bounds__(PG_THREADS, 1)
   static_assert(TMEM_COLS == 256 || TMEM_COLS == 512, "TMEM allocation must be a power of 2");
   static_assert(MODE != EPI_GEGLU || NSLAB % 2 == 0, "GEGLU pairs gate and up slabs");
 
-  if (*reinterpret_cast<volatile unsigned*>(&g_error_word) & MOE_DEVERR_TIMEOUT) return;
-  const int n_tiles = tiles.uniform_rows > 0 ? (tiles.uniform_rows + GM_BM - 1) / GM_BM
-                                             : *tiles.num;
-  const int U = n_tiles * n_blocks;
+  pdl_trigger();
   const int nk = K / GM_BK;
 
   extern __shared__ uint8_t psm_raw[];
@@ -204,6 +201,14 @@ __global__ void __launch_bounds__(PG_THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // The prologue above overlaps the previous kernel; the tile list is its output.
+  pdl_wait();
+  int U = 0;
+  if (!(*reinterpret_cast<volatile unsigned*>(&g_error_word) & MOE_DEVERR_TIMEOUT)) {
+    const int n_tiles = tiles.uniform_rows > 0 ? (tiles.uniform_rows + GM_BM - 1) / GM_BM
+                                               : *tiles.num;
+    U = n_tiles * n_blocks;
+  }
 
   PSched sch;
   sch.init(blockIdx.x, gridDim.x, U, nk);

@@ -62,6 +62,8 @@ __global__ void __launch_bounds__(128, 1)
                         const __grid_constant__ CUtensorMap tmB0,
                         const __grid_constant__ CUtensorMap tmB1, TileList tiles, int n_blocks,
                         int K, int N_total, void* __restrict__ out_ptr, int ldo) {
+  pdl_trigger();
+  pdl_wait();
   constexpr int BN = 64 * NSLAB;                       // MMA N
   constexpr int STAGE_BYTES = gemm_stage_bytes<NSLAB>();
   constexpr uint32_t TMEM_COLS = BN < 32 ? 32 : BN;

@@ -57,16 +57,17 @@ constexpr int kDecodeMaxTokens = 16;
 bool decode_gemm_ok(int T, int H, int I) {
   return T <= kDecodeMaxTokens && decode_shape_ok(I, true) && decode_shape_ok(H, false);
 }
+// Decode tiles only on request: measured on B200 the persistent 128-row tiles stream the
+// weights faster at every batch size so far.
 bool use_decode_gemm(int T, int H, int I, unsigned flags) {
-  if (flags & MOE_FLAG_PREFILL_TILES) return false;
-  if (flags & MOE_FLAG_DECODE_TILES) return decode_gemm_ok(T, H, I);
-  return decode_gemm_ok(T, H, I);
+  return (flags & MOE_FLAG_DECODE_TILES) && decode_gemm_ok(T, H, I);
 }
 
 // Batches of at most 8 tokens take the fused router + dispatch + gather launch.
 bool use_decode_front(int T, int H, int E, unsigned flags) {
   return T <= kFrontMaxTokens && E <= 128 && !router_uses_screen(T, flags) &&
-         H % (kFrontRanks * 4) == 0 && decode_front_smem_bytes(H, E) <= (size_t)kFrontSmemMax;
+         H % (kFrontRanks * kFrontWarps) == 0 &&
+         decode_front_smem_bytes(H, E) <= (size_t)kFrontSmemMax;
 }
 
 size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
@@ -305,11 +306,35 @@ moe_status_t launched() {
   return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
+// Kernel launch; with `dependent` the kernel may start launching while the previous kernel
+// on the stream is still running (programmatic stream serialisation): it runs its prologue
+// and then waits in pdl_wait() for that kernel's results.
+struct Launch {
+  cudaStream_t st;
+  bool pdl;   // allowed for this call (off while stage events sit between kernels)
+  template <typename... KArgs, typename... Args>
+  void operator()(bool dependent, void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                  Args... args) const {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = (dependent && pdl) ? 1 : 0;
+    cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+  }
+};
+
 moe_status_t launch_router(const __nv_bfloat16* x, const __nv_bfloat16* wr, const float* bias,
                            int T, int H, int E, int k, unsigned flags, int32_t* ids, float* wts,
                            unsigned* stats, uint8_t* ws, const Layout& L, const DeviceState& d,
-                           cudaStream_t st) {
+                           cudaStream_t st, bool pdl) {
   if (cudaMemsetAsync(stats, 0, 4 * sizeof(unsigned), st) != cudaSuccess) return MOE_ERR_CUDA;
+  const Launch launch{st, pdl};
   const double u = std::ldexp(1.0, -53);
   const double n = (double)H + 8.0;
   const double gamma = n * u / (1.0 - n * u);
@@ -320,23 +345,25 @@ moe_status_t launch_router(const __nv_bfloat16* x, const __nv_bfloat16* wr, cons
     float* scr = reinterpret_cast<float*>(ws + L.scr);
     __nv_bfloat16* wrT = reinterpret_cast<__nv_bfloat16*>(ws + L.wrT);
     double* wn2 = reinterpret_cast<double*>(ws + L.wn2);
-    router_transpose_kernel<<<dim3((H + 31) / 32, (E + 31) / 32), dim3(32, 8), 0, st>>>(wr, H, E,
-                                                                                      wrT);
-    router_wnorm_kernel<<<(E + 7) / 8, 256, 0, st>>>(wrT, H, E, wn2);
+    launch(false, router_transpose_kernel, dim3((H + 31) / 32, (E + 31) / 32), dim3(32, 8), 0, wr,
+           H, E, wrT);
+    launch(true, router_wnorm_kernel, dim3((E + 7) / 8), dim3(256), 0, wrT, H, E, wn2);
     CUtensorMap tm_x, tm_wr;
     if (!make_map_2d(&tm_x, x, H, T, GM_BM) || !make_map_3d(&tm_wr, wr, E, H, 1))
       return MOE_ERR_CUDA;
     const TileList tl{nullptr, nullptr, nullptr, nullptr, T};
     const int nb = (E + 127) / 128;
     const int mt = (T + GM_BM - 1) / GM_BM;
-    GEMM_SCREEN<<<nb * mt, 128, gemm_smem_bytes<kGemmStages, 2>(), st>>>(tm_x, tm_wr, tm_wr, tl,
-                                                                       nb, H, E, scr, E);
+    launch(true, GEMM_SCREEN, dim3(nb * mt), dim3(128), gemm_smem_bytes<kGemmStages, 2>(), tm_x,
+           tm_wr, tm_wr, tl, nb, H, E, (void*)scr, E);
     if (E <= 128)
-      router_screen_select_kernel<4><<<warps_blocks, 32 * kScreenWarps, 0, st>>>(
-          scr, x, wrT, wn2, bias, T, H, E, k, kScreenC, beta_scale, ids, wts, stats);
+      launch(true, router_screen_select_kernel<4>, dim3(warps_blocks), dim3(32 * kScreenWarps), 0,
+             (const float*)scr, x, (const __nv_bfloat16*)wrT, (const double*)wn2, bias, T, H, E, k,
+             kScreenC, beta_scale, ids, wts, stats);
     else
-      router_screen_select_kernel<8><<<warps_blocks, 32 * kScreenWarps, 0, st>>>(
-          scr, x, wrT, wn2, bias, T, H, E, k, kScreenC, beta_scale, ids, wts, stats);
+      launch(true, router_screen_select_kernel<8>, dim3(warps_blocks), dim3(32 * kScreenWarps), 0,
+             (const float*)scr, x, (const __nv_bfloat16*)wrT, (const double*)wn2, bias, T, H, E, k,
+             kScreenC, beta_scale, ids, wts, stats);
     return launched();
   }
   double* part_logit = reinterpret_cast<double*>(ws + L.part_logit);
@@ -346,20 +373,20 @@ moe_status_t launch_router(const __nv_bfloat16* x, const __nv_bfloat16* wr, cons
   const size_t sm1 = sizeof(double) * std::max<size_t>((size_t)L.hs * kRouterTokens,
                                                        (size_t)kRouterWarps * kRouterTokens * E);
   if (E <= 128)
-    router_partial_kernel<4><<<g1, 128, sm1, st>>>(x, wr, T, H, E, L.hs, part_logit, part_xn2,
-                                                   part_wn2);
+    launch(false, router_partial_kernel<4>, g1, dim3(128), sm1, x, wr, T, H, E, L.hs, part_logit,
+           part_xn2, part_wn2);
   else
-    router_partial_kernel<8><<<g1, 128, sm1, st>>>(x, wr, T, H, E, L.hs, part_logit, part_xn2,
-                                                   part_wn2);
+    launch(false, router_partial_kernel<8>, g1, dim3(128), sm1, x, wr, T, H, E, L.hs, part_logit,
+           part_xn2, part_wn2);
   if (launched() != MOE_OK) return MOE_ERR_CUDA;
   if (E <= 128)
-    router_select_kernel<4><<<warps_blocks, 256, 0, st>>>(part_logit, part_xn2, part_wn2, L.ks,
-                                                          bias, x, wr, T, H, E, k, renorm,
-                                                          beta_scale, ids, wts, stats);
+    launch(true, router_select_kernel<4>, dim3(warps_blocks), dim3(256), 0,
+           (const double*)part_logit, (const double*)part_xn2, (const double*)part_wn2, L.ks, bias,
+           x, wr, T, H, E, k, renorm, beta_scale, ids, wts, stats);
   else
-    router_select_kernel<8><<<warps_blocks, 256, 0, st>>>(part_logit, part_xn2, part_wn2, L.ks,
-                                                          bias, x, wr, T, H, E, k, renorm,
-                                                          beta_scale, ids, wts, stats);
+    launch(true, router_select_kernel<8>, dim3(warps_blocks), dim3(256), 0,
+           (const double*)part_logit, (const double*)part_xn2, (const double*)part_wn2, L.ks, bias,
+           x, wr, T, H, E, k, renorm, beta_scale, ids, wts, stats);
   return launched();
 }
 
@@ -429,7 +456,7 @@ moe_status_t moe_route(const void* x, const void* w_router, const float* router_
                        static_cast<const __nv_bfloat16*>(w_router), router_bias, T, H, E, k, flags,
                        topk_ids, topk_weights,
                        reinterpret_cast<unsigned*>(static_cast<uint8_t*>(workspace) + L.stats),
-                       static_cast<uint8_t*>(workspace), L, *d, st);
+                       static_cast<uint8_t*>(workspace), L, *d, st, true);
 }
 
 moe_status_t moe_forward(const void* x, const void* w_router, const float* router_bias,
@@ -494,16 +521,19 @@ moe_status_t moe_forward(const void* x, const void* w_router, const float* route
   prof.mark();
   int32_t* gemm_counters = reinterpret_cast<int32_t*>(ws + L.counters);
   const int gsm = std::max(1, d->num_sms) * 8;
+  // Dependent launches, except while stage events sit between the kernels.
+  const Launch launch{st, !prof.on};
   if (use_decode_front(T, H, E, flags)) {
     // 1+2. router, dispatch and gather in one cluster launch
     if (cudaMemsetAsync(stats, 0, 4 * sizeof(unsigned), st) != cudaSuccess) return MOE_ERR_CUDA;
     const double u = std::ldexp(1.0, -53), n = (double)H + 8.0;
     const double beta_scale = 2.0 * (n * u / (1.0 - n * u)) * 1.01;
-    decode_front_kernel<4><<<kFrontRanks, 128, decode_front_smem_bytes(H, E), st>>>(
-        static_cast<const __nv_bfloat16*>(x), static_cast<const __nv_bfloat16*>(w_router),
-        router_bias, T, H, E, k, (flags & MOE_FLAG_NO_RENORM) ? 0 : 1, beta_scale, ids, wts, stats,
-        counts, offsets, perm, inv, tile_num, tile_expert, tile_row0, tile_rows, gemm_counters,
-        L.n_counters, L.bm, reinterpret_cast<uint4*>(xp), H / 8);
+    launch(false, decode_front_kernel<4>, dim3(kFrontRanks), dim3(32 * kFrontWarps),
+           decode_front_smem_bytes(H, E), static_cast<const __nv_bfloat16*>(x),
+           static_cast<const __nv_bfloat16*>(w_router), router_bias, T, H, E, k,
+           (flags & MOE_FLAG_NO_RENORM) ? 0 : 1, beta_scale, ids, wts, stats, counts, offsets, perm,
+           inv, tile_num, tile_expert, tile_row0, tile_rows, gemm_counters, L.n_counters, L.bm,
+           reinterpret_cast<uint4*>(xp), H / 8);
     if (launched() != MOE_OK) return MOE_ERR_CUDA;
     prof.mark();
     prof.mark();
@@ -511,24 +541,26 @@ moe_status_t moe_forward(const void* x, const void* w_router, const float* route
     // 1. router
     moe_status_t s = launch_router(static_cast<const __nv_bfloat16*>(x),
                                    static_cast<const __nv_bfloat16*>(w_router), router_bias, T, H,
-                                   E, k, flags, ids, wts, stats, ws, L, *d, st);
+                                   E, k, flags, ids, wts, stats, ws, L, *d, st, !prof.on);
     if (s != MOE_OK) return s;
     prof.mark();
     // 2. dispatch
     if (L.nchunks == 1) {
-      dispatch_small_kernel<<<1, 256, 0, st>>>(ids, P, E, L.bm, counts, offsets, perm, inv,
-                                               tile_num, tile_expert, tile_row0, tile_rows,
-                                               gemm_counters, L.n_counters);
+      launch(true, dispatch_small_kernel, dim3(1), dim3(256), 0, (const int32_t*)ids, P, E, L.bm,
+             counts, offsets, perm, inv, tile_num, tile_expert, tile_row0, tile_rows,
+             gemm_counters, L.n_counters);
     } else {
-      dispatch_count_kernel<<<L.nchunks, 256, E * sizeof(int), st>>>(ids, P, E, chunk_counts);
-      dispatch_scan_kernel<<<1, 256, 0, st>>>(chunk_counts, L.nchunks, E, P, L.bm, counts,
-                                              offsets, chunk_base, tile_num, tile_expert, tile_row0,
-                                              tile_rows, gemm_counters, L.n_counters);
-      dispatch_rank_kernel<<<L.nchunks, 32, E * sizeof(int), st>>>(ids, P, E, chunk_base, perm,
-                                                                   inv);
+      launch(true, dispatch_count_kernel, dim3(L.nchunks), dim3(256), E * sizeof(int),
+             (const int32_t*)ids, P, E, chunk_counts);
+      launch(true, dispatch_scan_kernel, dim3(1), dim3(256), 0, (const int32_t*)chunk_counts,
+             L.nchunks, E, P, L.bm, counts, offsets, chunk_base, tile_num, tile_expert, tile_row0,
+             tile_rows, gemm_counters, L.n_counters);
+      launch(true, dispatch_rank_kernel, dim3(L.nchunks), dim3(32), E * sizeof(int),
+             (const int32_t*)ids, P, E, (const int32_t*)chunk_base, perm, inv);
     }
-    gather_rows_kernel<<<std::min((P + 7) / 8, gsm), 256, 0, st>>>(
-        static_cast<const uint4*>(x), perm, P, k, H / 8, reinterpret_cast<uint4*>(xp));
+    launch(true, gather_rows_kernel, dim3(std::min((P + 7) / 8, gsm)), dim3(256), 0,
+           static_cast<const uint4*>(x), (const int32_t*)perm, P, k, H / 8,
+           reinterpret_cast<uint4*>(xp));
     if (launched() != MOE_OK) return MOE_ERR_CUDA;
     prof.mark();
   }
@@ -539,33 +571,34 @@ moe_status_t moe_forward(const void* x, const void* w_router, const float* route
   int32_t* ctr1 = gemm_counters;
   int32_t* ctr2 = gemm_counters + L.n_counters / 2;
   if (dec) {
-    grouped_gemm_decode_kernel<EPI_GEGLU><<<G, DG_THREADS, decode_smem_bytes(I, true), st>>>(
-        tm_xp, tm_wg, tm_wu, tl, H, I, hbuf, I, partials, ctr1);
+    launch(true, grouped_gemm_decode_kernel<EPI_GEGLU>, dim3(G), dim3(DG_THREADS),
+           decode_smem_bytes(I, true), tm_xp, tm_wg, tm_wu, tl, H, I, (void*)hbuf, I, partials,
+           ctr1);
     if (launched() != MOE_OK) return MOE_ERR_CUDA;
     prof.mark();
-    grouped_gemm_decode_kernel<EPI_STORE><<<G, DG_THREADS, decode_smem_bytes(H, false), st>>>(
-        tm_h, tm_wd, tm_wd, tl, I, H, obuf, H, partials, ctr2);
+    launch(true, grouped_gemm_decode_kernel<EPI_STORE>, dim3(G), dim3(DG_THREADS),
+           decode_smem_bytes(H, false), tm_h, tm_wd, tm_wd, tl, I, H, (void*)obuf, H, partials,
+           ctr2);
     if (launched() != MOE_OK) return MOE_ERR_CUDA;
     prof.mark();
   } else {
     const int smem = pgemm_smem_bytes<kGemmStages, 4>();
     const int n1 = (I + 127) / 128;
-    GEMM_GEGLU<<<G, PG_THREADS, smem, st>>>(tm_xp, tm_wg, tm_wu, tl, n1, H, I, hbuf, I, partials,
-                                            ctr1);
+    launch(true, GEMM_GEGLU, dim3(G), dim3(PG_THREADS), smem, tm_xp, tm_wg, tm_wu, tl, n1, H, I,
+           (void*)hbuf, I, partials, ctr1);
     if (launched() != MOE_OK) return MOE_ERR_CUDA;
     prof.mark();
     const int n2 = (H + 255) / 256;
-    GEMM_STORE<<<G, PG_THREADS, smem, st>>>(tm_h, tm_wd, tm_wd, tl, n2, I, H, obuf, H, partials,
-                                            ctr2);
+    launch(true, GEMM_STORE, dim3(G), dim3(PG_THREADS), smem, tm_h, tm_wd, tm_wd, tl, n2, I, H,
+           (void*)obuf, H, partials, ctr2);
     if (launched() != MOE_OK) return MOE_ERR_CUDA;
     prof.mark();
   }
   // 5. combine
   const long long cthreads = (long long)T * (H / 8);
-  combine_kernel<<<(int)std::min<long long>((cthreads + 255) / 256, gsm), 256, 0, st>>>(
-      reinterpret_cast<const uint4*>(obuf),
-                                                            inv, wts, T, k, H / 8,
-                                                            static_cast<uint4*>(y));
+  launch(true, combine_kernel, dim3((int)std::min<long long>((cthreads + 255) / 256, gsm)),
+         dim3(256), 0, reinterpret_cast<const uint4*>(obuf), (const int32_t*)inv,
+         (const float*)wts, T, k, H / 8, static_cast<uint4*>(y));
   if (launched() != MOE_OK) return MOE_ERR_CUDA;
   prof.mark();
   prof.finish();
@@ -604,7 +637,7 @@ moe_status_t moe_route_static(const void* x, const void* w_router, const float* 
   return launch_router(static_cast<const __nv_bfloat16*>(x),
                        static_cast<const __nv_bfloat16*>(w_router), router_bias, T, H, E, k, f,
                        topk_ids, topk_weights, reinterpret_cast<unsigned*>(ws + L.stats), ws, L,
-                       *d, static_cast<cudaStream_t>(stream));
+                       *d, static_cast<cudaStream_t>(stream), true);
 }
 
 moe_status_t moe_sync_status(void* stream) {

@@ -31,6 +31,17 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
+// ----------------------------------------------------------------------------- dependent launch
+// A kernel launched with programmatic stream serialisation may start while its predecessor
+// is still running; pdl_wait() blocks until the predecessor grid has completed and its
+// memory is visible (a no-op otherwise).  pdl_trigger() lets the next kernel start
+// launching.  Every kernel here calls pdl_wait() before it reads anything an earlier
+// kernel wrote.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ----------------------------------------------------------------------------- mbarrier
 __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");

@@ -34,6 +34,8 @@ __global__ void __launch_bounds__(128) router_partial_kernel(
     const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __restrict__ wr, int T, int H,
     int E, int hs, double* __restrict__ part_logit, double* __restrict__ part_xn2,
     double* __restrict__ part_wn2) {
+  pdl_trigger();
+  pdl_wait();
   constexpr int TT = kRouterTokens;
   extern __shared__ double rsm[];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -299,11 +301,16 @@ __device__ __forceinline__ void router_finish_token(
     warp_topk<EPL>(L, E, k, taken, sel_e, sel_v);
   }
 
-  // Weights: softmax over all E, renormalised over the k selected (or not).
+  // Weights: softmax over all E, renormalised over the k selected (or not).  Lane r < k
+  // evaluates slot r's exponential; the denominator is summed in slot (or expert) order.
   const double m = sel_v[0];
+  double mine = 0.0;
+  for (int r = 0; r < k; ++r)
+    if (lane == r) mine = sel_v[r];
+  const double ex = lane < k ? exp(mine - m) : 0.0;
   double denom = 0.0;
   if (renorm) {
-    for (int r = 0; r < k; ++r) denom += exp(sel_v[r] - m);
+    for (int r = 0; r < k; ++r) denom += __shfl_sync(0xffffffffu, ex, r);
   } else {
     double s = 0.0;
 #pragma unroll
@@ -316,7 +323,7 @@ __device__ __forceinline__ void router_finish_token(
   for (int r = 0; r < k; ++r) {
     if (lane == r) {
       ids[(size_t)t * k + r] = sel_e[r];
-      wts[(size_t)t * k + r] = (float)(exp(sel_v[r] - m) / denom);
+      wts[(size_t)t * k + r] = (float)(ex / denom);
     }
   }
 
@@ -330,6 +337,8 @@ __global__ void __launch_bounds__(256) router_select_kernel(
     const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __restrict__ wr, int T, int H,
     int E, int k, int renorm, double beta_scale, int32_t* __restrict__ ids,
     float* __restrict__ wts, unsigned* __restrict__ stats) {
+  pdl_trigger();
+  pdl_wait();
   if (blockIdx.x == 0 && threadIdx.x == 0) stats[3] = 0;   // path: fp64 logits
   const int lane = threadIdx.x & 31;
   const int warps_per_block = blockDim.x >> 5;
@@ -409,6 +418,8 @@ __global__ void __launch_bounds__(256) router_select_kernel(
 __global__ void __launch_bounds__(256) router_transpose_kernel(const __nv_bfloat16* __restrict__ wr,
                                                                int H, int E,
                                                                __nv_bfloat16* __restrict__ wrT) {
+  pdl_trigger();
+  pdl_wait();
   __shared__ __nv_bfloat16 tile[32][33];
   const int h0 = blockIdx.x * 32, e0 = blockIdx.y * 32;
   for (int i = threadIdx.y; i < 32; i += blockDim.y) {
@@ -425,6 +436,8 @@ __global__ void __launch_bounds__(256) router_transpose_kernel(const __nv_bfloat
 // wn2[e] = sum_h Wr[h][e]^2 in fp64 (one warp per expert, over the transposed rows).
 __global__ void __launch_bounds__(256) router_wnorm_kernel(const __nv_bfloat16* __restrict__ wrT,
                                                            int H, int E, double* __restrict__ wn2) {
+  pdl_trigger();
+  pdl_wait();
   const int lane = threadIdx.x & 31;
   const int e = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   if (e >= E) return;
@@ -450,6 +463,8 @@ __global__ void __launch_bounds__(256) router_screen_select_kernel(
     const float* __restrict__ bias, int T, int H, int E, int k, double screen_c,
     double beta_scale, int32_t* __restrict__ ids, float* __restrict__ wts,
     unsigned* __restrict__ stats) {
+  pdl_trigger();
+  pdl_wait();
   if (blockIdx.x == 0 && threadIdx.x == 0) stats[3] = 1;   // path: screen + fp64 recheck
   __shared__ int s_cand[kScreenWarps][32 * EPL];
   __shared__ double s_val[kScreenWarps][32 * EPL];

@@ -66,8 +66,8 @@ enum {
   MOE_FLAG_PROFILE_STAGES = 1u << 3,
   /* Expert-GEMM tile family (moe_forward).  Decode tiles (weights as the 128-row MMA
    * operand, at most 16 tokens as the other; T <= 16 only) or prefill tiles (128 sorted
-   * rows x 256 columns).  By default the library picks; setting both, or decode tiles for
-   * T > 16, is MOE_ERR_INVALID_ARG. */
+   * rows x 256 columns, the default).  Setting both, or decode tiles for T > 16, is
+   * MOE_ERR_INVALID_ARG. */
   MOE_FLAG_DECODE_TILES = 1u << 4,
   MOE_FLAG_PREFILL_TILES = 1u << 5
 };
