@@ -156,6 +156,22 @@ def ncu_traffic(kernel: str, workload: str) -> float | None:
     return None
 
 
+# ----------------------------------------------------------------------------- ranks
+def max_over_ranks(values: list[float], dist=None, device=None) -> list[float]:
+    """Element-wise max of per-rank timings (every rank gets the result).  With one rank
+    (dist None or world size 1) the values come back unchanged."""
+    if dist is None or dist.get_world_size() == 1:
+        return [float(v) for v in values]
+    t = torch.tensor(values, dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t.tolist()]
+
+
+def job_throughput(world: int, tokens_per_rank: int, max_ms: float) -> float:
+    """Whole-job tokens/s: every rank's tokens over the slowest rank's step time."""
+    return world * tokens_per_rank / (max_ms * 1e-3)
+
+
 # ----------------------------------------------------------------------------- arms
 def run_reference(args, cfg) -> None:
     import oracle
@@ -309,10 +325,7 @@ def run_native(args, cfg) -> None:
     torch.cuda.synchronize()
     e2e_ms = sum(a.elapsed_time(b) for a, b in e2e_ev) / args.steps
 
-    if dist:
-        t = torch.tensor([ms, e2e_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms, e2e_ms = float(t[0]), float(t[1])
+    ms, e2e_ms = max_over_ranks([ms, e2e_ms], dist, dev)
 
     if rank == 0:
         pk = peaks()
@@ -342,7 +355,7 @@ def run_native(args, cfg) -> None:
         step_s = ms * 1e-3
         line = {
             "metric": METRIC,
-            "value": world * cfg.T / step_s,
+            "value": job_throughput(world, cfg.T, ms),
             "unit": UNIT,
             "n_gpus": world,
             "steps": args.steps,
@@ -366,7 +379,7 @@ def run_native(args, cfg) -> None:
                 "active_experts": acc["active_experts"]},
             "stages_ms": stages,
             "router_stats": rstats,
-            "e2e": {"value": world * cfg.T / (e2e_ms * 1e-3), "unit": UNIT,
+            "e2e": {"value": job_throughput(world, cfg.T, e2e_ms), "unit": UNIT,
                     "h2d_bytes_per_step": cfg.T * cfg.H * 2,
                     "d2h_bytes_per_step": cfg.T * cfg.H * 2},
             "gpu_launches": KERNELS_PER_STEP * args.steps,

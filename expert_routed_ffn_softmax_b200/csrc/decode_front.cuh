@@ -9,7 +9,8 @@
 //      exactly as router_select_kernel does (rank, verify against the rounding bound,
 //      sequential exact recomputation when too close, renormalised weights), then runs the
 //      single-CTA dispatch (counts, offsets, stable permutation, tile list);
-//   3. cluster barrier; all 32 warps of the cluster copy the x rows into Xp.
+//   3. (only when an Xp buffer is given) cluster barrier; all warps of the cluster copy the
+//      x rows into Xp.  By default GEMM-1 gathers the rows itself and this step is skipped.
 // The summation depth per logit is H/64 + 7 + 7 + 1 (<= H + 8), inside the bound the
 // verification uses.
 #pragma once
@@ -201,6 +202,7 @@ __global__ void __cluster_dims__(kFrontRanks, 1, 1) __launch_bounds__(32 * kFron
                          s_tstart);
     __threadfence();
   }
+  if (xp == nullptr) return;   // the grouped GEMM gathers the rows itself
   cluster_sync();
 
   // ---- 3. gather the x rows of the sorted pairs (16-byte vectors, 8 per thread in flight)

@@ -29,7 +29,7 @@ constexpr int PG_EPI_THREADS = 128;
 
 template <int STAGES, int NSLAB>
 __host__ __device__ constexpr int pgemm_smem_bytes() {
-  return 1024 + STAGES * gemm_stage_bytes<NSLAB>() + 256;
+  return 1024 + STAGES * gemm_stage_bytes<NSLAB>() + 1024;   // + barriers, flags, token rows
 }
 
 __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
@@ -143,7 +143,10 @@ __device__ __forceinline__ void pg_store32(void* out_ptr, int ldo, int row, int 
     dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
 }
 
-template <int STAGES, int MODE, int NSLAB>
+// GATHER: the A operand's rows are gathered from the unpermuted activations (tmA maps x
+// [T][K] with a 1-row box) by tile::gather4: row r of a tile is x[perm[row0 + r] / k], and
+// only the first ceil(rows/4)*4 rows are loaded (the others are never stored).
+template <int STAGES, int MODE, int NSLAB, bool GATHER = false>
 __global__ void __launch_bounds__(PG_THREADS, 1)
     grouped_gemm_persistent_kernel(const __grid_constant__ CUtensorMap tmA,
                                    const __grid_constant__ CUtensorMap tmB0,
@@ -215,22 +218,41 @@ __global__ void __launch_bounds__(PG_THREADS, 1)
   PItem it;
 
   if (warp == 0) {
-    if (lane == 0) {
-      // ------------------------------------------------------------ TMA producer
-      int q = 0;
-      while (!*abort_flag && sch.next(it)) {
-        int e, row0, rows, n0;
-        pg_tile_info<MODE, NSLAB>(tiles, n_blocks, it.unit, e, row0, rows, n0);
+    // -------------------------------------------------------------- TMA producer (lane 0;
+    // with GATHER the whole warp first reads the tile's token rows into shared memory)
+    int* tok = reinterpret_cast<int*>(misc + 32);   // [128] token row of every tile row
+    int q = 0;
+    while (sch.next(it)) {
+      int e, row0, rows, n0;
+      pg_tile_info<MODE, NSLAB>(tiles, n_blocks, it.unit, e, row0, rows, n0);
+      int a_bytes = GM_A_BYTES;
+      if (GATHER) {
+        __syncwarp();
+        for (int r = lane; r < GM_BM; r += 32)
+          tok[r] = __ldg(tiles.perm + row0 + min(r, rows - 1)) / tiles.k;
+        __syncwarp();
+        a_bytes = ((rows + 3) / 4) * 4 * 128;
+      }
+      bool stop = false;
+      if (lane == 0) {
         for (int kc = it.kb; kc < it.ke; ++kc, ++q) {
           const int s = q % STAGES;
-          if (q >= STAGES && !mbar_wait(empty_bar(s), ((q / STAGES) - 1) & 1)) {
+          if (*abort_flag ||
+              (q >= STAGES && !mbar_wait(empty_bar(s), ((q / STAGES) - 1) & 1))) {
             *abort_flag = 1;
+            stop = true;
             break;
           }
           const uint32_t sA = base + s * STAGE_BYTES;
           const uint32_t sB = sA + GM_A_BYTES;
-          mbar_arrive_expect_tx(full_bar(s), STAGE_BYTES);
-          tma_load_2d(sA, &tmA, full_bar(s), kc * GM_BK, row0);
+          mbar_arrive_expect_tx(full_bar(s), a_bytes + NSLAB * GM_SLAB_BYTES);
+          if (GATHER) {
+            for (int g = 0; g < (rows + 3) / 4; ++g)
+              tma_gather4(sA + g * 512, &tmA, full_bar(s), kc * GM_BK, tok[4 * g], tok[4 * g + 1],
+                          tok[4 * g + 2], tok[4 * g + 3]);
+          } else {
+            tma_load_2d(sA, &tmA, full_bar(s), kc * GM_BK, row0);
+          }
           // one load per projection: NSLAB/2 (gate, up) or NSLAB (down) 64-column slabs
           if (MODE == EPI_GEGLU) {
             tma_load_4d(sB, &tmB0, full_bar(s), 0, kc * GM_BK, n0 / 64, e);
@@ -242,6 +264,8 @@ __global__ void __launch_bounds__(PG_THREADS, 1)
           *n_issued = q + 1;
         }
       }
+      stop = __shfl_sync(0xffffffffu, stop, 0);
+      if (stop) break;
     }
   } else if (warp == 1) {
     if (lane == 0) {

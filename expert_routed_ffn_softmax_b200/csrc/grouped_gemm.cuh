@@ -40,6 +40,8 @@ struct TileList {
   const int32_t* row0;    // [cap] first sorted row
   const int32_t* rows;    // [cap] rows in tile (1..128)
   int uniform_rows;       // > 0: no list; tile m covers rows [128m, min(128m+128, uniform_rows)) of expert 0
+  const int32_t* perm = nullptr;   // gathering GEMMs: sorted row -> pair index t*k + j
+  int k = 1;                       //                  (row r of a tile reads x[perm[r] / k])
 };
 
 template <int NSLAB>

@@ -34,7 +34,7 @@ constexpr unsigned kKnownFlags = MOE_FLAG_NO_RENORM | MOE_FLAG_ROUTER_FP64 |
                                  MOE_FLAG_ROUTER_SCREEN | MOE_FLAG_PROFILE_STAGES |
                                  MOE_FLAG_DECODE_TILES | MOE_FLAG_PREFILL_TILES;
 
-#define GEMM_GEGLU grouped_gemm_persistent_kernel<kGemmStages, EPI_GEGLU, 4>
+#define GEMM_GEGLU grouped_gemm_persistent_kernel<kGemmStages, EPI_GEGLU, 4, true>
 #define GEMM_STORE grouped_gemm_persistent_kernel<kGemmStages, EPI_STORE, 4>
 #define GEMM_SCREEN grouped_gemm_kernel<kGemmStages, EPI_F32, 2>
 
@@ -149,7 +149,9 @@ Layout make_layout(int T, int H, int E, int I, int k, unsigned flags, bool forwa
     L.tile_expert = take(sizeof(int32_t) * L.max_tiles);
     L.tile_row0 = take(sizeof(int32_t) * L.max_tiles);
     L.tile_rows = take(sizeof(int32_t) * L.max_tiles);
-    L.xp = take(2 * P * H);
+    // Xp (expert-sorted copies of the x rows) only for the decode tiles; the prefill tiles
+    // gather the rows straight from x
+    if (L.bm == DG_BN) L.xp = take(2 * P * H);
     L.hbuf = take(2 * P * I);
     L.obuf = take(2 * P * H);
     // stream-K split tiles of the persistent GEMMs: two fp32 tile slots per CTA, and
@@ -247,7 +249,7 @@ DeviceState* device_state(int* dev_out) {
   DeviceState& d = g_dev[dev];
   if (!d.attrs_set) {
     cudaDeviceGetAttribute(&d.num_sms, cudaDevAttrMultiProcessorCount, dev);
-    const int gs = pgemm_smem_bytes<kGemmStages, 4>();
+    const int gs = pgemm_smem_bytes<kGemmStages, 4>();   // both persistent variants
     const int gs2 = gemm_smem_bytes<kGemmStages, 2>();
     if (cudaFuncSetAttribute(GEMM_GEGLU, cudaFuncAttributeMaxDynamicSharedMemorySize, gs) !=
             cudaSuccess ||
@@ -510,7 +512,9 @@ moe_status_t moe_forward(const void* x, const void* w_router, const float* route
   // up) or 4 (down) slabs
   const uint32_t w_rows = dec ? DG_KS : 64;
   const uint32_t gu_slabs = dec ? (uint32_t)(I / 64) : 2u, d_slabs = dec ? (uint32_t)(H / 64) : 4u;
-  if (!make_map_2d(&tm_xp, xp, H, P, act_rows, act_cols) ||
+  const bool ok_x = dec ? make_map_2d(&tm_xp, xp, H, P, act_rows, act_cols)
+                       : make_map_2d(&tm_xp, x, H, T, 1, 64);   // gather4: 1-row box over x
+  if (!ok_x ||
       !make_map_slabs(&tm_wg, w_gate, I, H, E, w_rows, gu_slabs) ||
       !make_map_slabs(&tm_wu, w_up, I, H, E, w_rows, gu_slabs) ||
       !make_map_2d(&tm_h, hbuf, I, P, act_rows, act_cols) ||
@@ -533,7 +537,7 @@ moe_status_t moe_forward(const void* x, const void* w_router, const float* route
            static_cast<const __nv_bfloat16*>(w_router), router_bias, T, H, E, k,
            (flags & MOE_FLAG_NO_RENORM) ? 0 : 1, beta_scale, ids, wts, stats, counts, offsets, perm,
            inv, tile_num, tile_expert, tile_row0, tile_rows, gemm_counters, L.n_counters, L.bm,
-           reinterpret_cast<uint4*>(xp), H / 8);
+           dec ? reinterpret_cast<uint4*>(xp) : nullptr, H / 8);
     if (launched() != MOE_OK) return MOE_ERR_CUDA;
     prof.mark();
     prof.mark();
@@ -558,14 +562,15 @@ moe_status_t moe_forward(const void* x, const void* w_router, const float* route
       launch(true, dispatch_rank_kernel, dim3(L.nchunks), dim3(32), E * sizeof(int),
              (const int32_t*)ids, P, E, (const int32_t*)chunk_base, perm, inv);
     }
-    launch(true, gather_rows_kernel, dim3(std::min((P + 7) / 8, gsm)), dim3(256), 0,
-           static_cast<const uint4*>(x), (const int32_t*)perm, P, k, H / 8,
-           reinterpret_cast<uint4*>(xp));
+    if (dec)
+      launch(true, gather_rows_kernel, dim3(std::min((P + 7) / 8, gsm)), dim3(256), 0,
+             static_cast<const uint4*>(x), (const int32_t*)perm, P, k, H / 8,
+             reinterpret_cast<uint4*>(xp));
     if (launched() != MOE_OK) return MOE_ERR_CUDA;
     prof.mark();
   }
   // 3. GEMM-1 + GEGLU, 4. GEMM-2 (down)
-  const TileList tl{tile_num, tile_expert, tile_row0, tile_rows, 0};
+  const TileList tl{tile_num, tile_expert, tile_row0, tile_rows, 0, perm, k};
   float* partials = reinterpret_cast<float*>(ws + L.partials);
   const int G = std::min(std::max(1, d->num_sms), kMaxGemmCtas);
   int32_t* ctr1 = gemm_counters;

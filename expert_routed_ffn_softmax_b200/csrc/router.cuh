@@ -470,6 +470,9 @@ __global__ void __launch_bounds__(256) router_screen_select_kernel(
   __shared__ double s_val[kScreenWarps][32 * EPL];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const unsigned lt = (1u << lane) - 1u;
+  // statistics are gathered per warp and published once, not per token
+  unsigned st_cand = 0, st_exact = 0;
+  float st_err = 0.f;
   for (int t = blockIdx.x * kScreenWarps + warp; t < T; t += gridDim.x * kScreenWarps) {
     const __nv_bfloat16* xr = x + (size_t)t * H;
     double xn2 = 0.0;
@@ -617,11 +620,9 @@ __global__ void __launch_bounds__(256) router_screen_select_kernel(
     }
 #pragma unroll
     for (int off = 16; off; off >>= 1) err = fmaxf(err, __shfl_xor_sync(0xffffffffu, err, off));
-    if (lane == 0) {
-      atomicAdd(&stats[0], (unsigned)nc);
-      if (!ok) atomicAdd(&stats[1], 1u);
-      atomicMax(&stats[2], __float_as_uint(err));
-    }
+    st_cand += (unsigned)nc;
+    st_exact += ok ? 0u : 1u;
+    st_err = fmaxf(st_err, err);
 
     // Renormalised weights: softmax over the k selected logits.
     const double m = sel_v[0];
@@ -633,6 +634,11 @@ __global__ void __launch_bounds__(256) router_screen_select_kernel(
         wts[(size_t)t * k + r] = (float)(exp(sel_v[r] - m) / denom);
       }
     __syncwarp();
+  }
+  if (lane == 0 && st_cand) {
+    atomicAdd(&stats[0], st_cand);
+    if (st_exact) atomicAdd(&stats[1], st_exact);
+    atomicMax(&stats[2], __float_as_uint(st_err));
   }
 }
 
