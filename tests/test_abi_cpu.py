@@ -49,8 +49,11 @@ def test_workspace_sizes(lib):
     small = lib.moe_workspace_size(8, 2816, 128, 704, 8, 0)
     big = lib.moe_workspace_size(2048, 2816, 128, 704, 8, 0)
     assert 0 < small < big
-    # Xp + Hbuf + O dominate: 2 bytes x pairs x (2H + I)
-    assert big >= 2 * 2048 * 8 * (2 * 2816 + 704)
+    # Hbuf + O dominate: 2 bytes x pairs x (H + I); GEMM-1 gathers its rows straight from x
+    assert big >= 2 * 2048 * 8 * (2816 + 704)
+    # decode tiles (at most 16 tokens) also keep a gathered copy Xp of the routed rows
+    dec = lib.moe_workspace_size(8, 2816, 128, 704, 8, 1 << 4)
+    assert dec >= small + 2 * 8 * 8 * 2816
     assert lib.moe_workspace_size(8, 2816, 128, 700, 8, 0) == 0     # I % 64 != 0
     assert lib.moe_workspace_size(8, 2800, 128, 704, 8, 0) == 0     # H % 64 != 0
     assert lib.moe_workspace_size(8, 2816, 128, 704, 9, 0) == 0     # k > 8
