@@ -33,7 +33,6 @@ from expert_routed_ffn_softmax_b200 import workloads as wl  # noqa: E402
 
 METRIC = "MoE-layer tokens/s; HBM GB/s (decode) & BF16 TFLOP/s (prefill) vs peak"
 UNIT = "tokens/s"
-KERNELS_PER_STEP = 9   # router 2, dispatch 4, GEMM-1, GEMM-2, combine
 PER_EXPERT_BYTES = 11_894_784   # 3 * 2816 * 704 * 2: weights one active expert reads
 L2_FLUSH_BYTES = 256 << 20
 
@@ -382,7 +381,7 @@ def run_native(args, cfg) -> None:
             "e2e": {"value": job_throughput(world, cfg.T, e2e_ms), "unit": UNIT,
                     "h2d_bytes_per_step": cfg.T * cfg.H * 2,
                     "d2h_bytes_per_step": cfg.T * cfg.H * 2},
-            "gpu_launches": KERNELS_PER_STEP * args.steps,
+            "gpu_launches": graph.kernels_per_replay * args.steps,
             "clocks": clk,
             "step_ms_p10_p50_p90": [float(np.percentile(step_ms, q)) for q in (10, 50, 90)],
         }

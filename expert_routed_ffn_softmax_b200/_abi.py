@@ -46,15 +46,22 @@ SIGNATURES = {
     "moe_sync_status": (_I, [_P]),
     "moe_last_stage_times": (_I, [ctypes.POINTER(ctypes.c_float), _I]),
     "moe_stage_name": (ctypes.c_char_p, [_I]),
+    "moe_last_cuda_error": (_I, []),
+    "moe_last_kernel_count": (_I, []),
+    "moe_cuda_error_name": (ctypes.c_char_p, [_I]),
     "moe_debug_set_wait_limit_ns": (_I, [ctypes.c_ulonglong]),
     "moe_debug_unsatisfied_wait": (_I, [_P]),
 }
 
 
 class MoEError(RuntimeError):
-    def __init__(self, code: int, what: str):
+    def __init__(self, code: int, what: str, cuda_error: int = 0):
         self.code = code
-        super().__init__(f"{what}: {status_string(code)} ({code})")
+        self.cuda_error = cuda_error
+        msg = f"{what}: {status_string(code)} ({code})"
+        if cuda_error:
+            msg += f" [{load().moe_cuda_error_name(cuda_error).decode()}]"
+        super().__init__(msg)
 
 
 class AuxOut(ctypes.Structure):
@@ -88,7 +95,7 @@ def status_string(code: int) -> str:
 
 def _check(code: int, what: str) -> None:
     if code != MOE_OK:
-        raise MoEError(code, what)
+        raise MoEError(code, what, load().moe_last_cuda_error() if code == MOE_ERR_CUDA else 0)
 
 
 def _stream_ptr(stream) -> int:
@@ -230,6 +237,11 @@ def last_stage_times() -> dict[str, float]:
     return {L.moe_stage_name(i).decode(): float(buf[i]) for i in range(n)}
 
 
+def last_kernel_count() -> int:
+    """Kernels launched by this thread's most recent route/forward call."""
+    return int(load().moe_last_kernel_count())
+
+
 class ForwardGraph:
     """One moe_forward captured in a CUDA graph for fixed shapes and buffers.
 
@@ -258,6 +270,7 @@ class ForwardGraph:
         self.graph = torch.cuda.CUDAGraph()
         with torch.cuda.graph(self.graph):
             forward(self.x, *self._args, out=self.y, **self._kw)
+        self.kernels_per_replay = last_kernel_count()
 
     def replay(self) -> torch.Tensor:
         self.graph.replay()

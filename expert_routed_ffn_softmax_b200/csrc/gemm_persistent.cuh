@@ -7,7 +7,10 @@
 // One CTA per SM, 6 warps: warp 0 = TMA producer (lane 0) and TMEM owner, warp 1 = MMA
 // issuer (lane 0), warps 2-5 = epilogue (warp w reads TMEM lanes 32*(w%4)..+31).  Two TMEM
 // accumulators alternate between work items, so the epilogue of one item overlaps the
-// mainloop of the next.
+// mainloop of the next.  A gathering GEMM adds warps 6-7, which copy the A rows of each
+// stage from the unpermuted activations with cp.async (TMA then loads only the weights).
+// Eight warps put two on each SM sub-partition, whose 16K registers then allow up to 255
+// per thread (ten warps would put three on one and cap every thread at 168).
 //
 // Schedule over U = tiles x column blocks units of nk k-steps each, G CTAs:
 //   * whole units, round robin (unit g + i*G), for all but the last one-to-two waves;
@@ -25,11 +28,17 @@
 namespace moe {
 
 constexpr int PG_THREADS = 192;
+constexpr int PG_GATHER_THREADS = 64;
+constexpr int PG_MAX_THREADS = PG_THREADS + PG_GATHER_THREADS;
 constexpr int PG_EPI_THREADS = 128;
+
+__host__ __device__ constexpr int pgemm_threads(bool gather) {
+  return gather ? PG_MAX_THREADS : PG_THREADS;
+}
 
 template <int STAGES, int NSLAB>
 __host__ __device__ constexpr int pgemm_smem_bytes() {
-  return 1024 + STAGES * gemm_stage_bytes<NSLAB>() + 1024;   // + barriers, flags, token rows
+  return 1024 + STAGES * gemm_stage_bytes<NSLAB>() + 1024;   // + barriers and flags
 }
 
 __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
@@ -143,11 +152,12 @@ __device__ __forceinline__ void pg_store32(void* out_ptr, int ldo, int row, int 
     dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
 }
 
-// GATHER: the A operand's rows are gathered from the unpermuted activations (tmA maps x
-// [T][K] with a 1-row box) by tile::gather4: row r of a tile is x[perm[row0 + r] / k], and
-// only the first ceil(rows/4)*4 rows are loaded (the others are never stored).
+// GATHER: row r of a tile's A operand is tiles.src[perm[row0 + r] / k] (tmA is unused).
+// Rows past the tile's end are not loaded: their accumulator rows hold whatever the stage
+// held before and are never stored.  (One TMA tile::gather4 per four rows was measured
+// first; its per-instruction cost capped a 128-row tile at about a sixth of the MMA rate.)
 template <int STAGES, int MODE, int NSLAB, bool GATHER = false>
-__global__ void __launch_bounds__(PG_THREADS, 1)
+__global__ void __launch_bounds__(PG_MAX_THREADS, 1)
     grouped_gemm_persistent_kernel(const __grid_constant__ CUtensorMap tmA,
                                    const __grid_constant__ CUtensorMap tmB0,
                                    const __grid_constant__ CUtensorMap tmB1, TileList tiles,
@@ -181,7 +191,7 @@ __global__ void __launch_bounds__(PG_THREADS, 1)
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   if (tid == 0) {
     for (int s = 0; s < STAGES; ++s) {
-      mbar_init(full_bar(s), 1);
+      mbar_init(full_bar(s), GATHER ? 1 + PG_GATHER_THREADS : 1);
       mbar_init(empty_bar(s), 1);
     }
     for (int b = 0; b < 2; ++b) {
@@ -192,7 +202,7 @@ __global__ void __launch_bounds__(PG_THREADS, 1)
     *n_issued = 0;
     *n_consumed = 0;
     fence_barrier_init();
-    tma_prefetch_desc(&tmA);
+    if (!GATHER) tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB0);
     tma_prefetch_desc(&tmB1);
   }
@@ -218,23 +228,13 @@ __global__ void __launch_bounds__(PG_THREADS, 1)
   PItem it;
 
   if (warp == 0) {
-    // -------------------------------------------------------------- TMA producer (lane 0;
-    // with GATHER the whole warp first reads the tile's token rows into shared memory)
-    int* tok = reinterpret_cast<int*>(misc + 32);   // [128] token row of every tile row
-    int q = 0;
-    while (sch.next(it)) {
-      int e, row0, rows, n0;
-      pg_tile_info<MODE, NSLAB>(tiles, n_blocks, it.unit, e, row0, rows, n0);
-      int a_bytes = GM_A_BYTES;
-      if (GATHER) {
-        __syncwarp();
-        for (int r = lane; r < GM_BM; r += 32)
-          tok[r] = __ldg(tiles.perm + row0 + min(r, rows - 1)) / tiles.k;
-        __syncwarp();
-        a_bytes = ((rows + 3) / 4) * 4 * 128;
-      }
+    // -------------------------------------------------------------- TMA producer (lane 0)
+    if (lane == 0) {
+      int q = 0;
       bool stop = false;
-      if (lane == 0) {
+      while (!stop && sch.next(it)) {
+        int e, row0, rows, n0;
+        pg_tile_info<MODE, NSLAB>(tiles, n_blocks, it.unit, e, row0, rows, n0);
         for (int kc = it.kb; kc < it.ke; ++kc, ++q) {
           const int s = q % STAGES;
           if (*abort_flag ||
@@ -245,14 +245,8 @@ __global__ void __launch_bounds__(PG_THREADS, 1)
           }
           const uint32_t sA = base + s * STAGE_BYTES;
           const uint32_t sB = sA + GM_A_BYTES;
-          mbar_arrive_expect_tx(full_bar(s), a_bytes + NSLAB * GM_SLAB_BYTES);
-          if (GATHER) {
-            for (int g = 0; g < (rows + 3) / 4; ++g)
-              tma_gather4(sA + g * 512, &tmA, full_bar(s), kc * GM_BK, tok[4 * g], tok[4 * g + 1],
-                          tok[4 * g + 2], tok[4 * g + 3]);
-          } else {
-            tma_load_2d(sA, &tmA, full_bar(s), kc * GM_BK, row0);
-          }
+          mbar_arrive_expect_tx(full_bar(s), (GATHER ? 0 : GM_A_BYTES) + NSLAB * GM_SLAB_BYTES);
+          if (!GATHER) tma_load_2d(sA, &tmA, full_bar(s), kc * GM_BK, row0);
           // one load per projection: NSLAB/2 (gate, up) or NSLAB (down) 64-column slabs
           if (MODE == EPI_GEGLU) {
             tma_load_4d(sB, &tmB0, full_bar(s), 0, kc * GM_BK, n0 / 64, e);
@@ -264,8 +258,6 @@ __global__ void __launch_bounds__(PG_THREADS, 1)
           *n_issued = q + 1;
         }
       }
-      stop = __shfl_sync(0xffffffffu, stop, 0);
-      if (stop) break;
     }
   } else if (warp == 1) {
     if (lane == 0) {
@@ -288,6 +280,7 @@ __global__ void __launch_bounds__(PG_THREADS, 1)
             break;
           }
           *n_consumed = q + 1;
+          if (GATHER) fence_proxy_async_smem();   // A arrived through the generic proxy
           tc_fence_after();
           const uint32_t sA = base + s * STAGE_BYTES;
           const uint32_t sB = sA + GM_A_BYTES;
@@ -307,7 +300,7 @@ __global__ void __launch_bounds__(PG_THREADS, 1)
         }
       }
     }
-  } else {
+  } else if (warp < 6) {
     // -------------------------------------------------------------- epilogue (warps 2-5)
     // Each warp owns 32 rows and works on its own: no barrier across the epilogue warps.
     const int quad = warp & 3;
@@ -408,6 +401,49 @@ __global__ void __launch_bounds__(PG_THREADS, 1)
       }
       ++j;
     }
+  } else if (GATHER) {
+    // -------------------------------------------------------------- A-row gather (warps 6-7)
+    // Gather warp w' = warp - 6 copies tile rows 64w'..64w'+63, four rows per instruction:
+    // lane = (sub-row lane/8, 16-byte chunk lane%8).  Chunk c of row r lands where a
+    // 128-byte-swizzled TMA box of 64 columns puts it: byte 128 r + 16 (c ^ (r % 8)).
+    const int gw = warp - 6, sub = lane >> 3, ch = lane & 7;
+    int q = 0;
+    bool stop = false;
+    while (!stop && sch.next(it)) {
+      int e, row0, rows, n0;
+      pg_tile_info<MODE, NSLAB>(tiles, n_blocks, it.unit, e, row0, rows, n0);
+      constexpr int NI = GM_BM / (4 * (PG_GATHER_THREADS / 32));   // instructions per stage
+      const __nv_bfloat16* src[NI];
+      uint32_t doff[NI];
+#pragma unroll
+      for (int i = 0; i < NI; ++i) {
+        const int r = gw * (4 * NI) + 4 * i + sub;
+        src[i] = nullptr;
+        if (r < rows) {
+          const int t = __ldg(tiles.perm + row0 + r) / tiles.k;
+          if (t >= 0 && t < tiles.src_rows)
+            src[i] = tiles.src + (size_t)t * tiles.ld + 8 * ch;
+          else
+            raise_error(MOE_DEVERR_BAD_INDEX);   // row left uncopied
+        }
+        doff[i] = static_cast<uint32_t>(r * 128 + ((ch ^ (r & 7)) << 4));
+      }
+      for (int kc = it.kb; kc < it.ke; ++kc, ++q) {
+        const int s = q % STAGES;
+        bool ok = !*abort_flag && (q < STAGES || mbar_wait(empty_bar(s), ((q / STAGES) - 1) & 1));
+        if (!__all_sync(0xffffffffu, ok)) {
+          *abort_flag = 1;
+          stop = true;
+          break;
+        }
+        const uint32_t sA = base + s * STAGE_BYTES;
+#pragma unroll
+        for (int i = 0; i < NI; ++i)
+          if (src[i] != nullptr) cp_async_16(sA + doff[i], src[i] + kc * GM_BK);
+        cp_async_arrive_noinc(full_bar(s));
+      }
+    }
+    cp_async_wait_all();   // nothing of ours lands in shared memory after this CTA ends
   }
 
   // ------------------------------------------------------------------ teardown

@@ -40,8 +40,13 @@ struct TileList {
   const int32_t* row0;    // [cap] first sorted row
   const int32_t* rows;    // [cap] rows in tile (1..128)
   int uniform_rows;       // > 0: no list; tile m covers rows [128m, min(128m+128, uniform_rows)) of expert 0
-  const int32_t* perm = nullptr;   // gathering GEMMs: sorted row -> pair index t*k + j
-  int k = 1;                       //                  (row r of a tile reads x[perm[r] / k])
+  // Gathering GEMMs: sorted row r of the A operand is row perm[r] / k of src (row stride ld
+  // elements), i.e. x[t] for the pair (t, j) = divmod(perm[r], k).
+  const int32_t* perm = nullptr;
+  int k = 1;
+  const __nv_bfloat16* src = nullptr;
+  int ld = 0;         // row stride of src (elements; a multiple of 8)
+  int src_rows = 0;   // rows of src
 };
 
 template <int NSLAB>

@@ -241,6 +241,20 @@ std::mutex g_dev_mu;
 const char* kStageNames[] = {"router", "dispatch", "gemm1_geglu", "gemm2_down", "combine"};
 constexpr int kNumStages = 5;
 
+thread_local int t_last_cuda_error = 0;
+thread_local int t_kernels = 0;   // kernels launched by this thread's current/last call
+
+moe_status_t cuda_failed(int code) {
+  t_last_cuda_error = code;
+  return MOE_ERR_CUDA;
+}
+
+#define MOE_TRY_CUDA(call)                          \
+  do {                                              \
+    const cudaError_t e_ = (call);                  \
+    if (e_ != cudaSuccess) return cuda_failed(e_);  \
+  } while (0)
+
 DeviceState* device_state(int* dev_out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
@@ -271,10 +285,15 @@ DeviceState* device_state(int* dev_out) {
             cudaSuccess ||
         cudaFuncSetAttribute(router_partial_kernel<8>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, 1408 * 8 * 8) !=
-            cudaSuccess)
+            cudaSuccess) {
+      cuda_failed(cudaGetLastError());
       return nullptr;
+    }
     for (auto& e : d.ev)
-      if (cudaEventCreate(&e) != cudaSuccess) return nullptr;
+      if (const cudaError_t err = cudaEventCreate(&e); err != cudaSuccess) {
+        cuda_failed(err);
+        return nullptr;
+      }
     d.attrs_set = true;
   }
   return &d;
@@ -305,7 +324,8 @@ struct Profiler {
 };
 
 moe_status_t launched() {
-  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+  const cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? MOE_OK : cuda_failed(e);
 }
 
 // Kernel launch; with `dependent` the kernel may start launching while the previous kernel
@@ -328,6 +348,7 @@ struct Launch {
     cfg.attrs = attr;
     cfg.numAttrs = (dependent && pdl) ? 1 : 0;
     cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+    ++t_kernels;
   }
 };
 
@@ -335,7 +356,7 @@ moe_status_t launch_router(const __nv_bfloat16* x, const __nv_bfloat16* wr, cons
                            int T, int H, int E, int k, unsigned flags, int32_t* ids, float* wts,
                            unsigned* stats, uint8_t* ws, const Layout& L, const DeviceState& d,
                            cudaStream_t st, bool pdl) {
-  if (cudaMemsetAsync(stats, 0, 4 * sizeof(unsigned), st) != cudaSuccess) return MOE_ERR_CUDA;
+  MOE_TRY_CUDA(cudaMemsetAsync(stats, 0, 4 * sizeof(unsigned), st));
   const Launch launch{st, pdl};
   const double u = std::ldexp(1.0, -53);
   const double n = (double)H + 8.0;
@@ -352,7 +373,7 @@ moe_status_t launch_router(const __nv_bfloat16* x, const __nv_bfloat16* wr, cons
     launch(true, router_wnorm_kernel, dim3((E + 7) / 8), dim3(256), 0, wrT, H, E, wn2);
     CUtensorMap tm_x, tm_wr;
     if (!make_map_2d(&tm_x, x, H, T, GM_BM) || !make_map_3d(&tm_wr, wr, E, H, 1))
-      return MOE_ERR_CUDA;
+      return cuda_failed(-1);   // a tensor map could not be encoded
     const TileList tl{nullptr, nullptr, nullptr, nullptr, T};
     const int nb = (E + 127) / 128;
     const int mt = (T + GM_BM - 1) / GM_BM;
@@ -380,7 +401,7 @@ moe_status_t launch_router(const __nv_bfloat16* x, const __nv_bfloat16* wr, cons
   else
     launch(false, router_partial_kernel<8>, g1, dim3(128), sm1, x, wr, T, H, E, L.hs, part_logit,
            part_xn2, part_wn2);
-  if (launched() != MOE_OK) return MOE_ERR_CUDA;
+  if (const moe_status_t ls = launched(); ls != MOE_OK) return ls;
   if (E <= 128)
     launch(true, router_select_kernel<4>, dim3(warps_blocks), dim3(256), 0,
            (const double*)part_logit, (const double*)part_xn2, (const double*)part_wn2, L.ks, bias,
@@ -453,6 +474,7 @@ moe_status_t moe_route(const void* x, const void* w_router, const float* router_
   int dev = 0;
   DeviceState* d = device_state(&dev);
   if (!d) return MOE_ERR_CUDA;
+  t_kernels = 0;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   return launch_router(static_cast<const __nv_bfloat16*>(x),
                        static_cast<const __nv_bfloat16*>(w_router), router_bias, T, H, E, k, flags,
@@ -481,6 +503,7 @@ moe_status_t moe_forward(const void* x, const void* w_router, const float* route
   int dev = 0;
   DeviceState* d = device_state(&dev);
   if (!d) return MOE_ERR_CUDA;
+  t_kernels = 0;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   const int P = T * k;
@@ -512,14 +535,15 @@ moe_status_t moe_forward(const void* x, const void* w_router, const float* route
   // up) or 4 (down) slabs
   const uint32_t w_rows = dec ? DG_KS : 64;
   const uint32_t gu_slabs = dec ? (uint32_t)(I / 64) : 2u, d_slabs = dec ? (uint32_t)(H / 64) : 4u;
+  // Prefill tiles gather their A rows from x inside GEMM-1; their A map is a placeholder.
   const bool ok_x = dec ? make_map_2d(&tm_xp, xp, H, P, act_rows, act_cols)
-                       : make_map_2d(&tm_xp, x, H, T, 1, 64);   // gather4: 1-row box over x
+                        : make_map_2d(&tm_xp, x, H, T, 1, 64);
   if (!ok_x ||
       !make_map_slabs(&tm_wg, w_gate, I, H, E, w_rows, gu_slabs) ||
       !make_map_slabs(&tm_wu, w_up, I, H, E, w_rows, gu_slabs) ||
       !make_map_2d(&tm_h, hbuf, I, P, act_rows, act_cols) ||
       !make_map_slabs(&tm_wd, w_down, H, I, E, w_rows, d_slabs))
-    return MOE_ERR_CUDA;
+    return cuda_failed(-1);   // a tensor map could not be encoded
 
   Profiler prof{d, st, (flags & MOE_FLAG_PROFILE_STAGES) != 0};
   prof.mark();
@@ -529,7 +553,7 @@ moe_status_t moe_forward(const void* x, const void* w_router, const float* route
   const Launch launch{st, !prof.on};
   if (use_decode_front(T, H, E, flags)) {
     // 1+2. router, dispatch and gather in one cluster launch
-    if (cudaMemsetAsync(stats, 0, 4 * sizeof(unsigned), st) != cudaSuccess) return MOE_ERR_CUDA;
+    MOE_TRY_CUDA(cudaMemsetAsync(stats, 0, 4 * sizeof(unsigned), st));
     const double u = std::ldexp(1.0, -53), n = (double)H + 8.0;
     const double beta_scale = 2.0 * (n * u / (1.0 - n * u)) * 1.01;
     launch(false, decode_front_kernel<4>, dim3(kFrontRanks), dim3(32 * kFrontWarps),
@@ -538,7 +562,7 @@ moe_status_t moe_forward(const void* x, const void* w_router, const float* route
            (flags & MOE_FLAG_NO_RENORM) ? 0 : 1, beta_scale, ids, wts, stats, counts, offsets, perm,
            inv, tile_num, tile_expert, tile_row0, tile_rows, gemm_counters, L.n_counters, L.bm,
            dec ? reinterpret_cast<uint4*>(xp) : nullptr, H / 8);
-    if (launched() != MOE_OK) return MOE_ERR_CUDA;
+    if (const moe_status_t ls = launched(); ls != MOE_OK) return ls;
     prof.mark();
     prof.mark();
   } else {
@@ -566,11 +590,12 @@ moe_status_t moe_forward(const void* x, const void* w_router, const float* route
       launch(true, gather_rows_kernel, dim3(std::min((P + 7) / 8, gsm)), dim3(256), 0,
              static_cast<const uint4*>(x), (const int32_t*)perm, P, k, H / 8,
              reinterpret_cast<uint4*>(xp));
-    if (launched() != MOE_OK) return MOE_ERR_CUDA;
+    if (const moe_status_t ls = launched(); ls != MOE_OK) return ls;
     prof.mark();
   }
   // 3. GEMM-1 + GEGLU, 4. GEMM-2 (down)
-  const TileList tl{tile_num, tile_expert, tile_row0, tile_rows, 0, perm, k};
+  const TileList tl{tile_num, tile_expert, tile_row0, tile_rows, 0, perm, k,
+                    static_cast<const __nv_bfloat16*>(x), H, T};
   float* partials = reinterpret_cast<float*>(ws + L.partials);
   const int G = std::min(std::max(1, d->num_sms), kMaxGemmCtas);
   int32_t* ctr1 = gemm_counters;
@@ -579,24 +604,24 @@ moe_status_t moe_forward(const void* x, const void* w_router, const float* route
     launch(true, grouped_gemm_decode_kernel<EPI_GEGLU>, dim3(G), dim3(DG_THREADS),
            decode_smem_bytes(I, true), tm_xp, tm_wg, tm_wu, tl, H, I, (void*)hbuf, I, partials,
            ctr1);
-    if (launched() != MOE_OK) return MOE_ERR_CUDA;
+    if (const moe_status_t ls = launched(); ls != MOE_OK) return ls;
     prof.mark();
     launch(true, grouped_gemm_decode_kernel<EPI_STORE>, dim3(G), dim3(DG_THREADS),
            decode_smem_bytes(H, false), tm_h, tm_wd, tm_wd, tl, I, H, (void*)obuf, H, partials,
            ctr2);
-    if (launched() != MOE_OK) return MOE_ERR_CUDA;
+    if (const moe_status_t ls = launched(); ls != MOE_OK) return ls;
     prof.mark();
   } else {
     const int smem = pgemm_smem_bytes<kGemmStages, 4>();
     const int n1 = (I + 127) / 128;
-    launch(true, GEMM_GEGLU, dim3(G), dim3(PG_THREADS), smem, tm_xp, tm_wg, tm_wu, tl, n1, H, I,
+    launch(true, GEMM_GEGLU, dim3(G), dim3(pgemm_threads(true)), smem, tm_xp, tm_wg, tm_wu, tl, n1, H, I,
            (void*)hbuf, I, partials, ctr1);
-    if (launched() != MOE_OK) return MOE_ERR_CUDA;
+    if (const moe_status_t ls = launched(); ls != MOE_OK) return ls;
     prof.mark();
     const int n2 = (H + 255) / 256;
     launch(true, GEMM_STORE, dim3(G), dim3(PG_THREADS), smem, tm_h, tm_wd, tm_wd, tl, n2, I, H,
            (void*)obuf, H, partials, ctr2);
-    if (launched() != MOE_OK) return MOE_ERR_CUDA;
+    if (const moe_status_t ls = launched(); ls != MOE_OK) return ls;
     prof.mark();
   }
   // 5. combine
@@ -604,7 +629,7 @@ moe_status_t moe_forward(const void* x, const void* w_router, const float* route
   launch(true, combine_kernel, dim3((int)std::min<long long>((cthreads + 255) / 256, gsm)),
          dim3(256), 0, reinterpret_cast<const uint4*>(obuf), (const int32_t*)inv,
          (const float*)wts, T, k, H / 8, static_cast<uint4*>(y));
-  if (launched() != MOE_OK) return MOE_ERR_CUDA;
+  if (const moe_status_t ls = launched(); ls != MOE_OK) return ls;
   prof.mark();
   prof.finish();
   return MOE_OK;
@@ -626,6 +651,7 @@ moe_status_t moe_route_static(const void* x, const void* w_router, const float* 
   int dev = 0;
   DeviceState* d = device_state(&dev);
   if (!d) return MOE_ERR_CUDA;
+  t_kernels = 0;
   void* scratch = nullptr;
   {
     // First call on this device: look up the array's device address (with this device
@@ -646,16 +672,26 @@ moe_status_t moe_route_static(const void* x, const void* w_router, const float* 
 }
 
 moe_status_t moe_sync_status(void* stream) {
-  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return MOE_ERR_CUDA;
+  MOE_TRY_CUDA(cudaStreamSynchronize(static_cast<cudaStream_t>(stream)));
   unsigned w = 0;
-  if (cudaMemcpyFromSymbol(&w, g_error_word, sizeof w) != cudaSuccess) return MOE_ERR_CUDA;
+  MOE_TRY_CUDA(cudaMemcpyFromSymbol(&w, g_error_word, sizeof w));
   if (w) {
     const unsigned zero = 0;
-    if (cudaMemcpyToSymbol(g_error_word, &zero, sizeof zero) != cudaSuccess) return MOE_ERR_CUDA;
+    MOE_TRY_CUDA(cudaMemcpyToSymbol(g_error_word, &zero, sizeof zero));
   }
   if (w & MOE_DEVERR_TIMEOUT) return MOE_ERR_TIMEOUT;
   if (w) return MOE_ERR_CUDA;
   return MOE_OK;
+}
+
+int moe_last_cuda_error(void) { return t_last_cuda_error; }
+
+int moe_last_kernel_count(void) { return t_kernels; }
+
+const char* moe_cuda_error_name(int code) {
+  if (code == 0) return "";
+  if (code == -1) return "tensor map encoding failed";
+  return cudaGetErrorName(static_cast<cudaError_t>(code));
 }
 
 int moe_last_stage_times(float* ms, int n) {

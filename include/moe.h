@@ -181,6 +181,17 @@ moe_status_t moe_route_static(const void *x, const void *w_router, const float *
  * or an out-of-range index seen by a kernel). */
 moe_status_t moe_sync_status(void *stream);
 
+/* The CUDA error behind the most recent MOE_ERR_CUDA returned to this host thread: its
+ * cudaError_t value (0 if none has occurred; -1 when a TMA tensor map could not be encoded),
+ * and its name (static string, "" for 0).  Reading it does not clear it. */
+int moe_last_cuda_error(void);
+const char *moe_cuda_error_name(int code);
+
+/* Number of kernels the most recent moe_route / moe_route_static / moe_forward call on this
+ * host thread launched (memsets not counted).  A CUDA graph captured from a call replays
+ * the same kernels. */
+int moe_last_kernel_count(void);
+
 /* Stage timing of the most recent call made with MOE_FLAG_PROFILE_STAGES on this host
  * thread's current device.  Synchronises on that call's last event.  Writes up to n
  * per-stage times in milliseconds to ms (host) and returns the number of stages, or -1

@@ -211,3 +211,17 @@ def test_graph_replay_matches_direct_call(gemma_w):
     y2 = fg.replay()
     assert moe.sync_status() == 0
     assert torch.equal(y2, moe.forward(x2, g["w_router"], g["w_gate"], g["w_up"], g["w_down"], 8))
+
+
+@pytest.mark.parametrize("T,router,expected", [
+    (8, "auto", 4),        # decode front end (router + dispatch), GEMM-1, GEMM-2, combine
+    (64, "auto", 6),       # fp64 router 2, single-CTA dispatch, GEMM-1, GEMM-2, combine
+    (4096, "auto", 10),    # screen router 4, dispatch 3, GEMM-1, GEMM-2, combine
+])
+def test_kernel_count_per_forward(T, router, expected, gemma_w):
+    x, c, g = layer_inputs(wl.CONFIGS["decode"], gemma_w, T=T)
+    moe.forward(x.cuda(), g["w_router"], g["w_gate"], g["w_up"], g["w_down"], 8, router=router)
+    assert moe.sync_status() == 0
+    assert moe.last_kernel_count() == expected
+    moe.route(x.cuda(), g["w_router"], 8, router="fp64")   # partial logits + select
+    assert moe.last_kernel_count() == 2
