@@ -29,9 +29,15 @@ MOE_FLAG_ROUTER_SCREEN = 1 << 2
 MOE_FLAG_PROFILE_STAGES = 1 << 3
 MOE_FLAG_DECODE_TILES = 1 << 4
 MOE_FLAG_PREFILL_TILES = 1 << 5
+MOE_FLAG_UNFUSED_FFN = 1 << 6
+MOE_FLAG_FUSED_FFN = 1 << 7
 
 _ROUTER_FLAGS = {"auto": 0, "fp64": MOE_FLAG_ROUTER_FP64, "screen": MOE_FLAG_ROUTER_SCREEN}
-_TILE_FLAGS = {"auto": 0, "decode": MOE_FLAG_DECODE_TILES, "prefill": MOE_FLAG_PREFILL_TILES}
+# Prefill tiles run GEMM-1 and GEMM-2 as one persistent launch ("fused") or two
+# ("unfused"); "prefill" leaves that choice to the library (fused for T*k <= 1024).
+_TILE_FLAGS = {"auto": 0, "decode": MOE_FLAG_DECODE_TILES, "prefill": MOE_FLAG_PREFILL_TILES,
+               "fused": MOE_FLAG_PREFILL_TILES | MOE_FLAG_FUSED_FFN,
+               "unfused": MOE_FLAG_PREFILL_TILES | MOE_FLAG_UNFUSED_FFN}
 
 # Every function the header declares, with (restype, argtypes).
 _P, _I, _U, _SZ = ctypes.c_void_p, ctypes.c_int, ctypes.c_uint, ctypes.c_size_t

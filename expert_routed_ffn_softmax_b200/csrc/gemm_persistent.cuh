@@ -152,26 +152,141 @@ __device__ __forceinline__ void pg_store32(void* out_ptr, int ldo, int row, int 
     dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
 }
 
-// GATHER: row r of a tile's A operand is tiles.src[perm[row0 + r] / k] (tmA is unused).
-// Rows past the tile's end are not loaded: their accumulator rows hold whatever the stage
-// held before and are never stored.  (One TMA tile::gather4 per four rows was measured
-// first; its per-instruction cost capped a 128-row tile at about a sixth of the MMA rate.)
-template <int STAGES, int MODE, int NSLAB, bool GATHER = false>
+// One GEMM of a persistent launch.
+struct PGemm {
+  int n_blocks;      // output column blocks (BN/2 GEGLU features, or BN columns, each)
+  int K;             // reduction depth, a multiple of 64
+  int N_total;       // output columns
+  void* out;         // output rows, ldo elements apart (bf16; fp32 for EPI_F32)
+  int ldo;
+  float* partials;   // stream-K partial tiles: 2 per CTA, 128 x BN fp32 each
+  int* counters;     // stream-K counters, 4 per split unit; zero at launch, left zero
+};
+
+// Epilogue of one work item by one epilogue warp (accumulator rows 32*quad .. +31, in
+// TMEM at trow).  Frees the TMEM buffer (arrives on tempty) once it has been read.
+// Returns true (warp-uniform) when this warp stored the item's final rows: a whole unit,
+// or the last piece of a split unit after adding the pieces in order.
+template <int MODE, int NSLAB>
+__device__ __forceinline__ bool pg_epilogue(const PGemm& g, const PSched& sch, const PItem& it,
+                                            int row0, int rows, int n0, uint32_t trow,
+                                            uint32_t tempty, int quad, int lane) {
+  constexpr int BN = 64 * NSLAB;
+  constexpr int NC = MODE == EPI_GEGLU ? BN / 2 : BN;
+  const int r_local = quad * 32 + lane;
+  const bool row_ok = r_local < rows;
+  const int row = row0 + r_local;
+  if (it.r < 0) {
+    // whole unit: epilogue straight from TMEM
+#pragma unroll 1
+    for (int c = 0; c < NC; c += 32) {
+      uint32_t gv[32], uv[32];
+      tmem_ld_32x32b_x32(trow + c, gv);
+      if (MODE == EPI_GEGLU) tmem_ld_32x32b_x32(trow + BN / 2 + c, uv);
+      tmem_ld_wait();
+      if (row_ok)
+        pg_store32<MODE, NSLAB>(g.out, g.ldo, row, n0, c, g.N_total,
+                                reinterpret_cast<const float*>(gv),
+                                reinterpret_cast<const float*>(uv));
+    }
+    tc_fence_before();
+    mbar_arrive(tempty);
+    return true;
+  }
+  // piece of a split unit: store this warp's 32 rows of the fp32 partial, count the piece,
+  // and let the warp that counts last add the pieces in order and finish.
+  const int slot = sch.slot(blockIdx.x, it.r);
+  float* prow = g.partials + ((size_t)slot * GM_BM + r_local) * BN;
+#pragma unroll 1
+  for (int c = 0; c < BN; c += 32) {
+    uint32_t v[32];
+    tmem_ld_32x32b_x32(trow + c, v);
+    tmem_ld_wait();
+    if (row_ok) {
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+        reinterpret_cast<uint4*>(prow + c)[i] =
+            make_uint4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+    }
+  }
+  tc_fence_before();
+  mbar_arrive(tempty);
+  __threadfence();
+  __syncwarp();
+  const int nk = sch.nk;
+  const long long cf = (long long)it.r * nk, cl = cf + nk - 1;
+  const int g_first = sch.owner(cf), n_pieces = sch.owner(cl) - g_first + 1;
+  int last = 0;
+  if (lane == 0) {
+    int* ctr = &g.counters[it.r * 4 + quad];
+    last = atomicAdd(ctr, 1) == n_pieces - 1;
+    if (last) *ctr = 0;   // ready for the next launch
+  }
+  last = __shfl_sync(0xffffffffu, last, 0);
+  if (!last) return false;
+  __threadfence();
+  if (row_ok) {
+#pragma unroll 1
+    for (int c = 0; c < NC; c += 32) {
+      float gsum[32], usum[32];
+#pragma unroll
+      for (int i = 0; i < 32; ++i) gsum[i] = usum[i] = 0.f;
+      for (int p = 0; p < n_pieces; ++p) {
+        const float* src = g.partials + ((size_t)sch.slot(g_first + p, it.r) * GM_BM + r_local) * BN;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const float4 a = __ldcg(reinterpret_cast<const float4*>(src + c) + i);
+          gsum[4 * i] += a.x;
+          gsum[4 * i + 1] += a.y;
+          gsum[4 * i + 2] += a.z;
+          gsum[4 * i + 3] += a.w;
+          if (MODE == EPI_GEGLU) {
+            const float4 bq = __ldcg(reinterpret_cast<const float4*>(src + BN / 2 + c) + i);
+            usum[4 * i] += bq.x;
+            usum[4 * i + 1] += bq.y;
+            usum[4 * i + 2] += bq.z;
+            usum[4 * i + 3] += bq.w;
+          }
+        }
+      }
+      pg_store32<MODE, NSLAB>(g.out, g.ldo, row, n0, c, g.N_total, gsum, usum);
+    }
+  }
+  return true;
+}
+
+// One launch runs one GEMM (g0), or with FUSED both expert GEMMs: phase 0 = GEMM-1 + GEGLU
+// (g0: h = gelu(x Wg) * (x Wu), A gathered from x), then phase 1 = GEMM-2 (g1: O = h Wd, A
+// = rows of h by TMA through tmA2, B through tmB2).  Every CTA runs all its phase-0 items
+// before its phase-1 items; a phase-1 item waits until the four epilogue warps of every
+// phase-0 column block of its tile have stored their h rows (h_ready[tile] = 4 n_blocks).
+// Those are always items that run earlier on their CTAs, and every CTA is resident (one
+// per SM), so the waits end.  h_ready[n_tiles] counts the same stores over all tiles: once
+// a CTA has seen it complete, its later phase-1 items skip the per-tile check (a global
+// acquire per item would stall the producer for a memory round trip each time).
+//
+// GATHER: row r of a tile's phase-0 A operand is tiles.src[perm[row0 + r] / k] (tmA is
+// unused).  Rows past the tile's end are not loaded: their accumulator rows hold whatever
+// the stage held before and are never stored.  (One TMA tile::gather4 per four rows was
+// measured first; its per-instruction cost capped a 128-row tile at about a sixth of the
+// MMA rate.)
+template <int STAGES, int MODE, int NSLAB, bool GATHER = false, bool FUSED = false>
 __global__ void __launch_bounds__(PG_MAX_THREADS, 1)
     grouped_gemm_persistent_kernel(const __grid_constant__ CUtensorMap tmA,
                                    const __grid_constant__ CUtensorMap tmB0,
-                                   const __grid_constant__ CUtensorMap tmB1, TileList tiles,
-                                   int n_blocks, int K, int N_total, void* __restrict__ out_ptr,
-                                   int ldo, float* __restrict__ partials,
-                                   int* __restrict__ counters) {
+                                   const __grid_constant__ CUtensorMap tmB1,
+                                   const __grid_constant__ CUtensorMap tmA2,
+                                   const __grid_constant__ CUtensorMap tmB2, TileList tiles,
+                                   PGemm g0, PGemm g1, int* __restrict__ h_ready) {
   constexpr int BN = 64 * NSLAB;
   constexpr int STAGE_BYTES = gemm_stage_bytes<NSLAB>();
   constexpr uint32_t TMEM_COLS = 2 * BN;   // two accumulators
+  constexpr int NPH = FUSED ? 2 : 1;
   static_assert(TMEM_COLS == 256 || TMEM_COLS == 512, "TMEM allocation must be a power of 2");
   static_assert(MODE != EPI_GEGLU || NSLAB % 2 == 0, "GEGLU pairs gate and up slabs");
+  static_assert(!FUSED || (MODE == EPI_GEGLU && GATHER), "the fused launch is GEMM-1 then GEMM-2");
 
   pdl_trigger();
-  const int nk = K / GM_BK;
 
   extern __shared__ uint8_t psm_raw[];
   const uint32_t raw_addr = smem_u32(psm_raw);
@@ -205,6 +320,10 @@ __global__ void __launch_bounds__(PG_MAX_THREADS, 1)
     if (!GATHER) tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB0);
     tma_prefetch_desc(&tmB1);
+    if (FUSED) {
+      tma_prefetch_desc(&tmA2);
+      tma_prefetch_desc(&tmB2);
+    }
   }
   if (warp == 0) {
     tmem_alloc(smem_u32(const_cast<uint32_t*>(tmem_slot)), TMEM_COLS);
@@ -216,46 +335,69 @@ __global__ void __launch_bounds__(PG_MAX_THREADS, 1)
   const uint32_t tmem = *tmem_slot;
   // The prologue above overlaps the previous kernel; the tile list is its output.
   pdl_wait();
-  int U = 0;
-  if (!(*reinterpret_cast<volatile unsigned*>(&g_error_word) & MOE_DEVERR_TIMEOUT)) {
-    const int n_tiles = tiles.uniform_rows > 0 ? (tiles.uniform_rows + GM_BM - 1) / GM_BM
-                                               : *tiles.num;
-    U = n_tiles * n_blocks;
-  }
-
-  PSched sch;
-  sch.init(blockIdx.x, gridDim.x, U, nk);
+  int n_tiles = 0;
+  if (!(*reinterpret_cast<volatile unsigned*>(&g_error_word) & MOE_DEVERR_TIMEOUT))
+    n_tiles = tiles.uniform_rows > 0 ? (tiles.uniform_rows + GM_BM - 1) / GM_BM : *tiles.num;
+  const int h_target = 4 * g0.n_blocks;
+  // Phase p's schedule (every role walks the same sequence of items).
+  auto sched = [&](int p) {
+    const PGemm& g = p ? g1 : g0;
+    PSched sc;
+    sc.init(blockIdx.x, gridDim.x, n_tiles * g.n_blocks, g.K / GM_BK);
+    return sc;
+  };
   PItem it;
 
   if (warp == 0) {
     // -------------------------------------------------------------- TMA producer (lane 0)
     if (lane == 0) {
       int q = 0;
-      bool stop = false;
-      while (!stop && sch.next(it)) {
-        int e, row0, rows, n0;
-        pg_tile_info<MODE, NSLAB>(tiles, n_blocks, it.unit, e, row0, rows, n0);
-        for (int kc = it.kb; kc < it.ke; ++kc, ++q) {
-          const int s = q % STAGES;
-          if (*abort_flag ||
-              (q >= STAGES && !mbar_wait(empty_bar(s), ((q / STAGES) - 1) & 1))) {
-            *abort_flag = 1;
-            stop = true;
-            break;
+      bool stop = false, all_h_ready = false;
+      for (int p = 0; p < NPH && !stop; ++p) {
+        const PGemm& g = p ? g1 : g0;
+        const bool a_tma = !(GATHER && p == 0);
+        PSched sch = sched(p);
+        while (!stop && sch.next(it)) {
+          int e, row0, rows, n0;
+          if (p == 0)
+            pg_tile_info<MODE, NSLAB>(tiles, g.n_blocks, it.unit, e, row0, rows, n0);
+          else
+            pg_tile_info<EPI_STORE, NSLAB>(tiles, g.n_blocks, it.unit, e, row0, rows, n0);
+          if (FUSED && p == 1 && !all_h_ready) {
+            // this tile's h rows come from phase-0 items of (possibly) other CTAs
+            if (ld_acquire_gpu(h_ready + n_tiles) >= h_target * n_tiles) {
+              all_h_ready = true;
+            } else if (!wait_counter_geq(h_ready + it.unit / g.n_blocks, h_target)) {
+              *abort_flag = 1;
+              stop = true;
+              break;
+            }
+            fence_proxy_async_global();   // TMA reads of h after the generic acquire
           }
-          const uint32_t sA = base + s * STAGE_BYTES;
-          const uint32_t sB = sA + GM_A_BYTES;
-          mbar_arrive_expect_tx(full_bar(s), (GATHER ? 0 : GM_A_BYTES) + NSLAB * GM_SLAB_BYTES);
-          if (!GATHER) tma_load_2d(sA, &tmA, full_bar(s), kc * GM_BK, row0);
-          // one load per projection: NSLAB/2 (gate, up) or NSLAB (down) 64-column slabs
-          if (MODE == EPI_GEGLU) {
-            tma_load_4d(sB, &tmB0, full_bar(s), 0, kc * GM_BK, n0 / 64, e);
-            tma_load_4d(sB + (NSLAB / 2) * GM_SLAB_BYTES, &tmB1, full_bar(s), 0, kc * GM_BK,
-                        n0 / 64, e);
-          } else {
-            tma_load_4d(sB, &tmB0, full_bar(s), 0, kc * GM_BK, n0 / 64, e);
+          for (int kc = it.kb; kc < it.ke; ++kc, ++q) {
+            const int s = q % STAGES;
+            if (*abort_flag ||
+                (q >= STAGES && !mbar_wait(empty_bar(s), ((q / STAGES) - 1) & 1))) {
+              *abort_flag = 1;
+              stop = true;
+              break;
+            }
+            const uint32_t sA = base + s * STAGE_BYTES;
+            const uint32_t sB = sA + GM_A_BYTES;
+            mbar_arrive_expect_tx(full_bar(s), (a_tma ? GM_A_BYTES : 0) + NSLAB * GM_SLAB_BYTES);
+            // phase 1: the gather warps have left; arrive in their place
+            if (FUSED && p == 1) mbar_arrive_cnt(full_bar(s), PG_GATHER_THREADS);
+            if (a_tma) tma_load_2d(sA, p ? &tmA2 : &tmA, full_bar(s), kc * GM_BK, row0);
+            // one load per projection: NSLAB/2 (gate, up) or NSLAB (down) 64-column slabs
+            if (p == 0 && MODE == EPI_GEGLU) {
+              tma_load_4d(sB, &tmB0, full_bar(s), 0, kc * GM_BK, n0 / 64, e);
+              tma_load_4d(sB + (NSLAB / 2) * GM_SLAB_BYTES, &tmB1, full_bar(s), 0, kc * GM_BK,
+                          n0 / 64, e);
+            } else {
+              tma_load_4d(sB, p ? &tmB2 : &tmB0, full_bar(s), 0, kc * GM_BK, n0 / 64, e);
+            }
+            *n_issued = q + 1;
           }
-          *n_issued = q + 1;
         }
       }
     }
@@ -264,39 +406,45 @@ __global__ void __launch_bounds__(PG_MAX_THREADS, 1)
       // ------------------------------------------------------------ MMA issuer
       constexpr uint32_t idesc = idesc_bf16_f32(GM_BM, BN, false, true);
       int q = 0, j = 0;
-      while (!*abort_flag && sch.next(it)) {
-        const int b = j & 1, use = j >> 1;
-        if (use >= 1 && !mbar_wait(tempty_bar(b), (use - 1) & 1)) {
-          *abort_flag = 1;
-          break;
-        }
-        tc_fence_after();
-        const uint32_t dt = tmem + b * BN;
-        bool ok = true;
-        for (int kc = it.kb; kc < it.ke; ++kc, ++q) {
-          const int s = q % STAGES;
-          if (!mbar_wait(full_bar(s), (q / STAGES) & 1)) {
-            ok = false;
+      bool stop = false;
+      for (int p = 0; p < NPH && !stop; ++p) {
+        PSched sch = sched(p);
+        while (!*abort_flag && sch.next(it)) {
+          const int b = j & 1, use = j >> 1;
+          if (use >= 1 && !mbar_wait(tempty_bar(b), (use - 1) & 1)) {
+            *abort_flag = 1;
+            stop = true;
             break;
           }
-          *n_consumed = q + 1;
-          if (GATHER) fence_proxy_async_smem();   // A arrived through the generic proxy
           tc_fence_after();
-          const uint32_t sA = base + s * STAGE_BYTES;
-          const uint32_t sB = sA + GM_A_BYTES;
+          const uint32_t dt = tmem + b * BN;
+          bool ok = true;
+          for (int kc = it.kb; kc < it.ke; ++kc, ++q) {
+            const int s = q % STAGES;
+            if (!mbar_wait(full_bar(s), (q / STAGES) & 1)) {
+              ok = false;
+              break;
+            }
+            *n_consumed = q + 1;
+            if (GATHER && p == 0) fence_proxy_async_smem();   // A came through the generic proxy
+            tc_fence_after();
+            const uint32_t sA = base + s * STAGE_BYTES;
+            const uint32_t sB = sA + GM_A_BYTES;
 #pragma unroll
-          for (int kk = 0; kk < GM_BK / 16; ++kk) {
-            const uint64_t adesc = smem_desc_sw128(sA + kk * 32, 16, 1024);
-            const uint64_t bdesc = smem_desc_sw128(sB + kk * 2048, GM_SLAB_BYTES, 1024);
-            umma_bf16(dt, adesc, bdesc, idesc, (kc != it.kb || kk != 0) ? 1u : 0u);
+            for (int kk = 0; kk < GM_BK / 16; ++kk) {
+              const uint64_t adesc = smem_desc_sw128(sA + kk * 32, 16, 1024);
+              const uint64_t bdesc = smem_desc_sw128(sB + kk * 2048, GM_SLAB_BYTES, 1024);
+              umma_bf16(dt, adesc, bdesc, idesc, (kc != it.kb || kk != 0) ? 1u : 0u);
+            }
+            umma_commit(empty_bar(s));
           }
-          umma_commit(empty_bar(s));
-        }
-        umma_commit(tfull_bar(b));
-        ++j;
-        if (!ok) {
-          *abort_flag = 1;
-          break;
+          umma_commit(tfull_bar(b));
+          ++j;
+          if (!ok) {
+            *abort_flag = 1;
+            stop = true;
+            break;
+          }
         }
       }
     }
@@ -304,117 +452,61 @@ __global__ void __launch_bounds__(PG_MAX_THREADS, 1)
     // -------------------------------------------------------------- epilogue (warps 2-5)
     // Each warp owns 32 rows and works on its own: no barrier across the epilogue warps.
     const int quad = warp & 3;
-    const int r_local = quad * 32 + lane;
     int j = 0;
-    while (sch.next(it)) {
-      const int b = j & 1, use = j >> 1;
-      bool got = mbar_wait(tfull_bar(b), use & 1);
-      tc_fence_after();
-      got = __all_sync(0xffffffffu, got && !*abort_flag);   // warp-uniform decision
-      if (!got) {
-        *abort_flag = 1;
-        break;
-      }
-      int e, row0, rows, n0;
-      pg_tile_info<MODE, NSLAB>(tiles, n_blocks, it.unit, e, row0, rows, n0);
-      const bool row_ok = r_local < rows;
-      const int row = row0 + r_local;
-      const uint32_t trow = tmem + b * BN + (static_cast<uint32_t>(quad * 32) << 16);
-      constexpr int NC = MODE == EPI_GEGLU ? BN / 2 : BN;
-      if (it.r < 0) {
-        // whole unit: epilogue straight from TMEM
-#pragma unroll 1
-        for (int c = 0; c < NC; c += 32) {
-          uint32_t g[32], u[32];
-          tmem_ld_32x32b_x32(trow + c, g);
-          if (MODE == EPI_GEGLU) tmem_ld_32x32b_x32(trow + BN / 2 + c, u);
-          tmem_ld_wait();
-          if (row_ok)
-            pg_store32<MODE, NSLAB>(out_ptr, ldo, row, n0, c, N_total,
-                                    reinterpret_cast<const float*>(g),
-                                    reinterpret_cast<const float*>(u));
+    bool stop = false;
+    for (int p = 0; p < NPH && !stop; ++p) {
+      const PGemm& g = p ? g1 : g0;
+      PSched sch = sched(p);
+      while (sch.next(it)) {
+        const int b = j & 1, use = j >> 1;
+        bool got = mbar_wait(tfull_bar(b), use & 1);
+        tc_fence_after();
+        got = __all_sync(0xffffffffu, got && !*abort_flag);   // warp-uniform decision
+        if (!got) {
+          *abort_flag = 1;
+          stop = true;
+          break;
         }
-        tc_fence_before();
-        mbar_arrive(tempty_bar(b));
-      } else {
-        // piece of a split unit: store this warp's 32 rows of the fp32 partial, count the
-        // piece, and let the warp that counts last add the pieces in order and finish.
-        const int slot = sch.slot(blockIdx.x, it.r);
-        float* prow = partials + ((size_t)slot * GM_BM + r_local) * BN;
-#pragma unroll 1
-        for (int c = 0; c < BN; c += 32) {
-          uint32_t v[32];
-          tmem_ld_32x32b_x32(trow + c, v);
-          tmem_ld_wait();
-          if (row_ok) {
-#pragma unroll
-            for (int i = 0; i < 8; ++i)
-              reinterpret_cast<uint4*>(prow + c)[i] =
-                  make_uint4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
-          }
-        }
-        tc_fence_before();
-        mbar_arrive(tempty_bar(b));
-        __threadfence();
-        __syncwarp();
-        const long long cf = (long long)it.r * nk, cl = cf + nk - 1;
-        const int g_first = sch.owner(cf), n_pieces = sch.owner(cl) - g_first + 1;
-        int last = 0;
-        if (lane == 0) {
-          int* ctr = &counters[it.r * 4 + quad];
-          last = atomicAdd(ctr, 1) == n_pieces - 1;
-          if (last) *ctr = 0;   // ready for the next launch
-        }
-        last = __shfl_sync(0xffffffffu, last, 0);
-        if (last) {
-          __threadfence();
-          if (row_ok) {
-#pragma unroll 1
-            for (int c = 0; c < NC; c += 32) {
-              float gsum[32], usum[32];
-#pragma unroll
-              for (int i = 0; i < 32; ++i) gsum[i] = usum[i] = 0.f;
-              for (int p = 0; p < n_pieces; ++p) {
-                const float* src =
-                    partials + ((size_t)sch.slot(g_first + p, it.r) * GM_BM + r_local) * BN;
-#pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                  const float4 a = __ldcg(reinterpret_cast<const float4*>(src + c) + i);
-                  gsum[4 * i] += a.x;
-                  gsum[4 * i + 1] += a.y;
-                  gsum[4 * i + 2] += a.z;
-                  gsum[4 * i + 3] += a.w;
-                  if (MODE == EPI_GEGLU) {
-                    const float4 bq =
-                        __ldcg(reinterpret_cast<const float4*>(src + BN / 2 + c) + i);
-                    usum[4 * i] += bq.x;
-                    usum[4 * i + 1] += bq.y;
-                    usum[4 * i + 2] += bq.z;
-                    usum[4 * i + 3] += bq.w;
-                  }
-                }
-              }
-              pg_store32<MODE, NSLAB>(out_ptr, ldo, row, n0, c, N_total, gsum, usum);
+        int e, row0, rows, n0;
+        const uint32_t trow = tmem + b * BN + (static_cast<uint32_t>(quad * 32) << 16);
+        if (p == 0) {
+          pg_tile_info<MODE, NSLAB>(tiles, g.n_blocks, it.unit, e, row0, rows, n0);
+          const bool done = pg_epilogue<MODE, NSLAB>(g, sch, it, row0, rows, n0, trow,
+                                                     tempty_bar(b), quad, lane);
+          if (FUSED && done) {
+            // publish this warp's h rows of the tile to the phase-1 TMA loads
+            fence_proxy_async_global();
+            __threadfence();
+            __syncwarp();
+            if (lane == 0) {
+              red_release_add_gpu(h_ready + it.unit / g.n_blocks, 1);
+              red_release_add_gpu(h_ready + n_tiles, 1);
             }
           }
+        } else {
+          pg_tile_info<EPI_STORE, NSLAB>(tiles, g.n_blocks, it.unit, e, row0, rows, n0);
+          pg_epilogue<EPI_STORE, NSLAB>(g, sch, it, row0, rows, n0, trow, tempty_bar(b), quad,
+                                        lane);
         }
+        ++j;
       }
-      ++j;
     }
   } else if (GATHER) {
     // -------------------------------------------------------------- A-row gather (warps 6-7)
     // Gather warp w' = warp - 6 copies tile rows 64w'..64w'+63, four rows per instruction:
     // lane = (sub-row lane/8, 16-byte chunk lane%8).  Chunk c of row r lands where a
     // 128-byte-swizzled TMA box of 64 columns puts it: byte 128 r + 16 (c ^ (r % 8)).
+    // Phase 0 only: in phase 1 the TMA thread arrives for these warps.
     const int gw = warp - 6, sub = lane >> 3, ch = lane & 7;
     int q = 0;
     bool stop = false;
+    PSched sch = sched(0);
     while (!stop && sch.next(it)) {
-      int e, row0, rows, n0;
-      pg_tile_info<MODE, NSLAB>(tiles, n_blocks, it.unit, e, row0, rows, n0);
       constexpr int NI = GM_BM / (4 * (PG_GATHER_THREADS / 32));   // instructions per stage
       const __nv_bfloat16* src[NI];
       uint32_t doff[NI];
+      int e, row0, rows, n0;
+      pg_tile_info<MODE, NSLAB>(tiles, g0.n_blocks, it.unit, e, row0, rows, n0);
 #pragma unroll
       for (int i = 0; i < NI; ++i) {
         const int r = gw * (4 * NI) + 4 * i + sub;

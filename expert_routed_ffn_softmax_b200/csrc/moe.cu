@@ -27,14 +27,17 @@ constexpr int kGemmStages = 4;
 constexpr int kMaxDevices = 64;
 constexpr int kScreenMinTokens = 256;            // default router path switch
 constexpr int kMaxGemmCtas = 256;                // >= SMs per GPU (148 on B200)
+constexpr int kStreamKCounters = 4 * 2 * kMaxGemmCtas;   // per GEMM: 4 per split unit
 constexpr int kFrontSmemMax = 200 * 1024;        // decode front kernel's dynamic smem cap
 
 constexpr double kScreenC = 1.0 / 1024.0;        // screen error bound / (|x| |w|)
 constexpr unsigned kKnownFlags = MOE_FLAG_NO_RENORM | MOE_FLAG_ROUTER_FP64 |
                                  MOE_FLAG_ROUTER_SCREEN | MOE_FLAG_PROFILE_STAGES |
-                                 MOE_FLAG_DECODE_TILES | MOE_FLAG_PREFILL_TILES;
+                                 MOE_FLAG_DECODE_TILES | MOE_FLAG_PREFILL_TILES |
+                                 MOE_FLAG_UNFUSED_FFN | MOE_FLAG_FUSED_FFN;
 
 #define GEMM_GEGLU grouped_gemm_persistent_kernel<kGemmStages, EPI_GEGLU, 4, true>
+#define GEMM_FFN grouped_gemm_persistent_kernel<kGemmStages, EPI_GEGLU, 4, true, true>
 #define GEMM_STORE grouped_gemm_persistent_kernel<kGemmStages, EPI_STORE, 4>
 #define GEMM_SCREEN grouped_gemm_kernel<kGemmStages, EPI_F32, 2>
 
@@ -42,6 +45,7 @@ bool flags_ok(unsigned flags) {
   if (flags & ~kKnownFlags) return false;
   if ((flags & MOE_FLAG_ROUTER_FP64) && (flags & MOE_FLAG_ROUTER_SCREEN)) return false;
   if ((flags & MOE_FLAG_DECODE_TILES) && (flags & MOE_FLAG_PREFILL_TILES)) return false;
+  if ((flags & MOE_FLAG_UNFUSED_FFN) && (flags & MOE_FLAG_FUSED_FFN)) return false;
   return true;
 }
 
@@ -50,6 +54,15 @@ bool router_uses_screen(int T, unsigned flags) {
   if (flags & (MOE_FLAG_NO_RENORM | MOE_FLAG_ROUTER_FP64)) return false;
   if (flags & MOE_FLAG_ROUTER_SCREEN) return true;
   return T >= kScreenMinTokens;
+}
+
+// GEMM-1 and GEMM-2 in one launch for small batches (measured on B200: one kernel ramp less
+// pays at T*k <= 512; from T*k = 4096 up two launches were faster).
+constexpr long long kFusedFfnMaxPairs = 1024;
+bool use_fused_ffn(int T, int k, unsigned flags) {
+  if (flags & MOE_FLAG_FUSED_FFN) return true;
+  if (flags & MOE_FLAG_UNFUSED_FFN) return false;
+  return (long long)T * k <= kFusedFfnMaxPairs;
 }
 
 // Batches of at most 16 tokens (so at most 16 rows per expert) use the decode GEMMs.
@@ -106,7 +119,7 @@ struct Layout {
   size_t chunk_counts = 0, chunk_base = 0, counts = 0, offsets = 0, perm = 0, inv = 0;
   size_t tile_num = 0, tile_expert = 0, tile_row0 = 0, tile_rows = 0;
   size_t xp = 0, hbuf = 0, obuf = 0;
-  size_t partials = 0, counters = 0;
+  size_t partials = 0, partials2 = 0, counters = 0;
   int n_counters = 0;
   size_t total = 0;
 };
@@ -154,10 +167,12 @@ Layout make_layout(int T, int H, int E, int I, int k, unsigned flags, bool forwa
     if (L.bm == DG_BN) L.xp = take(2 * P * H);
     L.hbuf = take(2 * P * I);
     L.obuf = take(2 * P * H);
-    // stream-K split tiles of the persistent GEMMs: two fp32 tile slots per CTA, and
-    // per-(split unit, row quadrant) counters, one set per GEMM
+    // stream-K split tiles of the persistent GEMMs: two fp32 tile slots per CTA and
+    // per-(split unit, row quadrant) counters, one set per GEMM (the fused launch runs both
+    // at once); then one h-ready counter per tile for the fused launch
     L.partials = take(sizeof(float) * 2 * (size_t)kMaxGemmCtas * GM_BM * 256);
-    L.n_counters = 2 * 4 * 2 * kMaxGemmCtas;
+    L.partials2 = take(sizeof(float) * 2 * (size_t)kMaxGemmCtas * GM_BM * 256);
+    L.n_counters = 2 * kStreamKCounters + L.max_tiles + 1;
     L.counters = take(sizeof(int32_t) * L.n_counters);
   }
   L.total = off;
@@ -238,8 +253,8 @@ struct DeviceState {
 DeviceState g_dev[kMaxDevices];
 std::mutex g_dev_mu;
 
-const char* kStageNames[] = {"router", "dispatch", "gemm1_geglu", "gemm2_down", "combine"};
-constexpr int kNumStages = 5;
+const char* kStageNames[] = {"router", "dispatch", "expert_ffn", "combine"};
+constexpr int kNumStages = 4;
 
 thread_local int t_last_cuda_error = 0;
 thread_local int t_kernels = 0;   // kernels launched by this thread's current/last call
@@ -266,6 +281,8 @@ DeviceState* device_state(int* dev_out) {
     const int gs = pgemm_smem_bytes<kGemmStages, 4>();   // both persistent variants
     const int gs2 = gemm_smem_bytes<kGemmStages, 2>();
     if (cudaFuncSetAttribute(GEMM_GEGLU, cudaFuncAttributeMaxDynamicSharedMemorySize, gs) !=
+            cudaSuccess ||
+        cudaFuncSetAttribute(GEMM_FFN, cudaFuncAttributeMaxDynamicSharedMemorySize, gs) !=
             cudaSuccess ||
         cudaFuncSetAttribute(GEMM_STORE, cudaFuncAttributeMaxDynamicSharedMemorySize, gs) !=
             cudaSuccess ||
@@ -597,33 +614,37 @@ moe_status_t moe_forward(const void* x, const void* w_router, const float* route
   const TileList tl{tile_num, tile_expert, tile_row0, tile_rows, 0, perm, k,
                     static_cast<const __nv_bfloat16*>(x), H, T};
   float* partials = reinterpret_cast<float*>(ws + L.partials);
+  float* partials2 = reinterpret_cast<float*>(ws + L.partials2);
   const int G = std::min(std::max(1, d->num_sms), kMaxGemmCtas);
   int32_t* ctr1 = gemm_counters;
-  int32_t* ctr2 = gemm_counters + L.n_counters / 2;
+  int32_t* ctr2 = gemm_counters + kStreamKCounters;
+  int32_t* h_ready = gemm_counters + 2 * kStreamKCounters;
   if (dec) {
     launch(true, grouped_gemm_decode_kernel<EPI_GEGLU>, dim3(G), dim3(DG_THREADS),
            decode_smem_bytes(I, true), tm_xp, tm_wg, tm_wu, tl, H, I, (void*)hbuf, I, partials,
            ctr1);
     if (const moe_status_t ls = launched(); ls != MOE_OK) return ls;
-    prof.mark();
     launch(true, grouped_gemm_decode_kernel<EPI_STORE>, dim3(G), dim3(DG_THREADS),
            decode_smem_bytes(H, false), tm_h, tm_wd, tm_wd, tl, I, H, (void*)obuf, H, partials,
            ctr2);
     if (const moe_status_t ls = launched(); ls != MOE_OK) return ls;
-    prof.mark();
   } else {
     const int smem = pgemm_smem_bytes<kGemmStages, 4>();
-    const int n1 = (I + 127) / 128;
-    launch(true, GEMM_GEGLU, dim3(G), dim3(pgemm_threads(true)), smem, tm_xp, tm_wg, tm_wu, tl, n1, H, I,
-           (void*)hbuf, I, partials, ctr1);
+    const PGemm g1{(I + 127) / 128, H, I, hbuf, I, partials, ctr1};
+    const PGemm g2{(H + 255) / 256, I, H, obuf, H, partials2, ctr2};
+    if (!use_fused_ffn(T, k, flags)) {
+      launch(true, GEMM_GEGLU, dim3(G), dim3(pgemm_threads(true)), smem, tm_xp, tm_wg, tm_wu,
+             tm_xp, tm_wg, tl, g1, g1, h_ready);
+      if (const moe_status_t ls = launched(); ls != MOE_OK) return ls;
+      launch(true, GEMM_STORE, dim3(G), dim3(pgemm_threads(false)), smem, tm_h, tm_wd, tm_wd,
+             tm_h, tm_wd, tl, g2, g2, h_ready);
+    } else {
+      launch(true, GEMM_FFN, dim3(G), dim3(pgemm_threads(true)), smem, tm_xp, tm_wg, tm_wu, tm_h,
+             tm_wd, tl, g1, g2, h_ready);
+    }
     if (const moe_status_t ls = launched(); ls != MOE_OK) return ls;
-    prof.mark();
-    const int n2 = (H + 255) / 256;
-    launch(true, GEMM_STORE, dim3(G), dim3(PG_THREADS), smem, tm_h, tm_wd, tm_wd, tl, n2, I, H,
-           (void*)obuf, H, partials, ctr2);
-    if (const moe_status_t ls = launched(); ls != MOE_OK) return ls;
-    prof.mark();
   }
+  prof.mark();
   // 5. combine
   const long long cthreads = (long long)T * (H / 8);
   launch(true, combine_kernel, dim3((int)std::min<long long>((cthreads + 255) / 256, gsm)),

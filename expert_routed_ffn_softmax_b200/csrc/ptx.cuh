@@ -57,6 +57,11 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t byt
                : "memory");
 }
 
+// `count` arrivals at once (on behalf of threads that do not take part in this phase).
+__device__ __forceinline__ void mbar_arrive_cnt(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
@@ -86,6 +91,37 @@ __device__ __forceinline__ bool mbar_wait_ns(uint32_t bar, uint32_t parity, uint
 
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
   return mbar_wait_ns(bar, parity, g_wait_limit_ns);
+}
+
+// ----------------------------------------------------------------------------- global flags
+__device__ __forceinline__ int ld_acquire_gpu(const int* p) {
+  int v;
+  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ void red_release_add_gpu(int* p, int v) {
+  asm volatile("red.release.gpu.global.add.s32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+// Orders this thread's generic-proxy global accesses with its later async-proxy ones
+// (TMA), and the reverse.
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
+// Wait until *p >= target (another CTA's release), at most the bounded-wait limit.
+__device__ __forceinline__ bool wait_counter_geq(const int* p, int target) {
+  if (ld_acquire_gpu(p) >= target) return true;
+  const uint64_t t0 = global_timer_ns();
+  while (ld_acquire_gpu(p) < target) {
+    if (global_timer_ns() - t0 > g_wait_limit_ns) {
+      raise_error(MOE_DEVERR_TIMEOUT);
+      return false;
+    }
+    __nanosleep(128);
+  }
+  return true;
 }
 
 // ----------------------------------------------------------------------------- TMA

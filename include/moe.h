@@ -69,7 +69,13 @@ enum {
    * rows x 256 columns, the default).  Setting both, or decode tiles for T > 16, is
    * MOE_ERR_INVALID_ARG. */
   MOE_FLAG_DECODE_TILES = 1u << 4,
-  MOE_FLAG_PREFILL_TILES = 1u << 5
+  MOE_FLAG_PREFILL_TILES = 1u << 5,
+  /* Prefill tiles run GEMM-1 (+GEGLU) and GEMM-2 either as one persistent launch (a CTA
+   * moves on to GEMM-2 tiles as soon as the GEMM-1 tiles they read are stored; the default
+   * for T*k <= 1024) or as two launches (the default above).  Both give the same bytes.
+   * These flags force one form; setting both is MOE_ERR_INVALID_ARG. */
+  MOE_FLAG_UNFUSED_FFN = 1u << 6,
+  MOE_FLAG_FUSED_FFN = 1u << 7
 };
 
 /* Optional caller-owned device outputs of moe_forward (any member may be NULL). */
@@ -195,7 +201,8 @@ int moe_last_kernel_count(void);
 /* Stage timing of the most recent call made with MOE_FLAG_PROFILE_STAGES on this host
  * thread's current device.  Synchronises on that call's last event.  Writes up to n
  * per-stage times in milliseconds to ms (host) and returns the number of stages, or -1
- * when no profiled call has been made.  moe_stage_name(i) names stage i. */
+ * when no profiled call has been made.  moe_stage_name(i) names stage i: "router",
+ * "dispatch", "expert_ffn" (GEMM-1 + GEGLU and GEMM-2, one or two kernels), "combine". */
 int moe_last_stage_times(float *ms, int n);
 const char *moe_stage_name(int i);
 

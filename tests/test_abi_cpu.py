@@ -80,10 +80,12 @@ def test_host_argument_checks(lib):
     # k > E, negative T, unknown flag
     assert f(*ok, 8, 2816, 4, 704, 8, 0, FAKE + 4096, None, FAKE, 1 << 30, None) == 1
     assert f(*ok, -1, 2816, 128, 704, 8, 0, FAKE + 4096, None, FAKE, 1 << 30, None) == 1
-    assert f(*ok, 8, 2816, 128, 704, 8, 1 << 7, FAKE + 4096, None, FAKE, 1 << 30, None) == 1
-    both = _abi.MOE_FLAG_ROUTER_FP64 | _abi.MOE_FLAG_ROUTER_SCREEN      # contradictory paths
-    assert f(*ok, 8, 2816, 128, 704, 8, both, FAKE + 4096, None, FAKE, 1 << 30, None) == 1
-    assert lib.moe_workspace_size(8, 2816, 128, 704, 8, both) == 0
+    assert f(*ok, 8, 2816, 128, 704, 8, 1 << 12, FAKE + 4096, None, FAKE, 1 << 30, None) == 1
+    for both in (_abi.MOE_FLAG_ROUTER_FP64 | _abi.MOE_FLAG_ROUTER_SCREEN,   # contradictory
+                 _abi.MOE_FLAG_FUSED_FFN | _abi.MOE_FLAG_UNFUSED_FFN,
+                 _abi.MOE_FLAG_DECODE_TILES | _abi.MOE_FLAG_PREFILL_TILES):
+        assert f(*ok, 8, 2816, 128, 704, 8, both, FAKE + 4096, None, FAKE, 1 << 30, None) == 1
+        assert lib.moe_workspace_size(8, 2816, 128, 704, 8, both) == 0
     # misaligned pointer
     assert f(FAKE + 2, *ok[1:], 8, 2816, 128, 704, 8, 0, FAKE + 4096, None, FAKE, 1 << 30,
              None) == 1

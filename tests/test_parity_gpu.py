@@ -122,7 +122,7 @@ def test_forward_forced_router_path(name, router, gemma_w):
     run_case(wl.CONFIGS[name], gemma_w, 256, router=router)
 
 
-@pytest.mark.parametrize("tiles", ["decode", "prefill"])
+@pytest.mark.parametrize("tiles", ["decode", "prefill", "fused", "unfused"])
 @pytest.mark.parametrize("name,T", [("tiny", 16), ("tiny", 3), ("decode", 8), ("decode", 1),
                                     ("decode", 16)])
 def test_forward_tile_families(name, T, tiles, gemma_w):
@@ -213,15 +213,29 @@ def test_graph_replay_matches_direct_call(gemma_w):
     assert torch.equal(y2, moe.forward(x2, g["w_router"], g["w_gate"], g["w_up"], g["w_down"], 8))
 
 
-@pytest.mark.parametrize("T,router,expected", [
-    (8, "auto", 4),        # decode front end (router + dispatch), GEMM-1, GEMM-2, combine
-    (64, "auto", 6),       # fp64 router 2, single-CTA dispatch, GEMM-1, GEMM-2, combine
+@pytest.mark.parametrize("T,tiles,expected", [
+    (8, "auto", 3),        # decode front end (router + dispatch), expert FFN, combine
+    (8, "unfused", 4),     # ... with GEMM-1 and GEMM-2 as two launches
+    (64, "auto", 5),       # fp64 router 2, single-CTA dispatch, expert FFN, combine
     (4096, "auto", 10),    # screen router 4, dispatch 3, GEMM-1, GEMM-2, combine
+    (4096, "fused", 9),    # ... with GEMM-1 and GEMM-2 in one launch
 ])
-def test_kernel_count_per_forward(T, router, expected, gemma_w):
+def test_kernel_count_per_forward(T, tiles, expected, gemma_w):
     x, c, g = layer_inputs(wl.CONFIGS["decode"], gemma_w, T=T)
-    moe.forward(x.cuda(), g["w_router"], g["w_gate"], g["w_up"], g["w_down"], 8, router=router)
+    moe.forward(x.cuda(), g["w_router"], g["w_gate"], g["w_up"], g["w_down"], 8, tiles=tiles)
     assert moe.sync_status() == 0
     assert moe.last_kernel_count() == expected
     moe.route(x.cuda(), g["w_router"], 8, router="fp64")   # partial logits + select
     assert moe.last_kernel_count() == 2
+
+
+@pytest.mark.parametrize("T", [1, 8, 64, 300, 2048])
+def test_fused_ffn_matches_two_launches_bitwise(T, gemma_w):
+    """GEMM-1 and GEMM-2 in one persistent launch give the same bytes as two launches (same
+    tiles, same stream-K split, same summation order)."""
+    x, c, g = layer_inputs(wl.CONFIGS["decode"], gemma_w, T=T)
+    x = x.cuda()
+    y1 = moe.forward(x, g["w_router"], g["w_gate"], g["w_up"], g["w_down"], 8, tiles="fused")
+    y2 = moe.forward(x, g["w_router"], g["w_gate"], g["w_up"], g["w_down"], 8, tiles="unfused")
+    assert moe.sync_status() == 0
+    assert torch.equal(y1, y2)
