@@ -338,6 +338,7 @@ def run_native(args, cfg) -> None:
         fused = args.tiles == "fused" or (args.tiles in ("auto", "prefill")
                                           and cfg.T * cfg.k <= FUSED_FFN_MAX_PAIRS)
         kname = ("grouped_gemm_decode_kernel<EPI_GEGLU>+<EPI_STORE>" if args.tiles == "decode"
+                 else "grouped_gemm_persistent_kernel<6,EPI_GEGLU,4,1,1,1>" if fused and cfg.T <= 8
                  else "grouped_gemm_persistent_kernel<4,EPI_GEGLU,4,1,1>" if fused
                  else "grouped_gemm_persistent_kernel<4,EPI_GEGLU,4,1,0>+<4,EPI_STORE,4,0,0>")
         traffic = ncu_traffic(kname, cfg.name)

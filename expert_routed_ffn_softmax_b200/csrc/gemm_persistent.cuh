@@ -36,9 +36,27 @@ __host__ __device__ constexpr int pgemm_threads(bool gather) {
   return gather ? PG_MAX_THREADS : PG_THREADS;
 }
 
-template <int STAGES, int NSLAB>
+// SMALL_A: every tile has at most 8 rows (batches of at most 8 tokens).  A stage then
+// holds only 8 A rows (1 KB) and the MMA reads them as all 128 rows of its A operand (the
+// descriptor's stride between 8-row groups is 0), so accumulator rows 8..127 repeat rows
+// 0..7 and are never stored.  The stages shrink from 48 KB to 33 KB and 6 fit instead of 4:
+// half as many weight bytes again in flight per SM, which is what a weight-streaming
+// decode step needs.
+constexpr int PG_SMALL_ROWS = 8;
+
+template <int NSLAB, bool SMALL_A>
+__host__ __device__ constexpr int pgemm_a_bytes() {
+  return SMALL_A ? PG_SMALL_ROWS * GM_BK * 2 : GM_A_BYTES;
+}
+
+template <int NSLAB, bool SMALL_A>
+__host__ __device__ constexpr int pgemm_stage_bytes() {
+  return pgemm_a_bytes<NSLAB, SMALL_A>() + NSLAB * GM_SLAB_BYTES;
+}
+
+template <int STAGES, int NSLAB, bool SMALL_A = false>
 __host__ __device__ constexpr int pgemm_smem_bytes() {
-  return 1024 + STAGES * gemm_stage_bytes<NSLAB>() + 1024;   // + barriers and flags
+  return 1024 + STAGES * pgemm_stage_bytes<NSLAB, SMALL_A>() + 1024;   // + barriers, flags
 }
 
 __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
@@ -270,7 +288,8 @@ __device__ __forceinline__ bool pg_epilogue(const PGemm& g, const PSched& sch, c
 // the stage held before and are never stored.  (One TMA tile::gather4 per four rows was
 // measured first; its per-instruction cost capped a 128-row tile at about a sixth of the
 // MMA rate.)
-template <int STAGES, int MODE, int NSLAB, bool GATHER = false, bool FUSED = false>
+template <int STAGES, int MODE, int NSLAB, bool GATHER = false, bool FUSED = false,
+          bool SMALL_A = false>
 __global__ void __launch_bounds__(PG_MAX_THREADS, 1)
     grouped_gemm_persistent_kernel(const __grid_constant__ CUtensorMap tmA,
                                    const __grid_constant__ CUtensorMap tmB0,
@@ -279,9 +298,12 @@ __global__ void __launch_bounds__(PG_MAX_THREADS, 1)
                                    const __grid_constant__ CUtensorMap tmB2, TileList tiles,
                                    PGemm g0, PGemm g1, int* __restrict__ h_ready) {
   constexpr int BN = 64 * NSLAB;
-  constexpr int STAGE_BYTES = gemm_stage_bytes<NSLAB>();
+  constexpr int A_BYTES = pgemm_a_bytes<NSLAB, SMALL_A>();
+  constexpr int STAGE_BYTES = pgemm_stage_bytes<NSLAB, SMALL_A>();
+  constexpr uint32_t A_SBO = SMALL_A ? 0u : 1024u;   // stride between 8-row groups of A
   constexpr uint32_t TMEM_COLS = 2 * BN;   // two accumulators
   constexpr int NPH = FUSED ? 2 : 1;
+  static_assert(STAGE_BYTES % 1024 == 0, "stages keep the 1 KB alignment of swizzled tiles");
   static_assert(TMEM_COLS == 256 || TMEM_COLS == 512, "TMEM allocation must be a power of 2");
   static_assert(MODE != EPI_GEGLU || NSLAB % 2 == 0, "GEGLU pairs gate and up slabs");
   static_assert(!FUSED || (MODE == EPI_GEGLU && GATHER), "the fused launch is GEMM-1 then GEMM-2");
@@ -383,8 +405,8 @@ __global__ void __launch_bounds__(PG_MAX_THREADS, 1)
               break;
             }
             const uint32_t sA = base + s * STAGE_BYTES;
-            const uint32_t sB = sA + GM_A_BYTES;
-            mbar_arrive_expect_tx(full_bar(s), (a_tma ? GM_A_BYTES : 0) + NSLAB * GM_SLAB_BYTES);
+            const uint32_t sB = sA + A_BYTES;
+            mbar_arrive_expect_tx(full_bar(s), (a_tma ? A_BYTES : 0) + NSLAB * GM_SLAB_BYTES);
             // phase 1: the gather warps have left; arrive in their place
             if (FUSED && p == 1) mbar_arrive_cnt(full_bar(s), PG_GATHER_THREADS);
             if (a_tma) tma_load_2d(sA, p ? &tmA2 : &tmA, full_bar(s), kc * GM_BK, row0);
@@ -429,10 +451,10 @@ __global__ void __launch_bounds__(PG_MAX_THREADS, 1)
             if (GATHER && p == 0) fence_proxy_async_smem();   // A came through the generic proxy
             tc_fence_after();
             const uint32_t sA = base + s * STAGE_BYTES;
-            const uint32_t sB = sA + GM_A_BYTES;
+            const uint32_t sB = sA + A_BYTES;
 #pragma unroll
             for (int kk = 0; kk < GM_BK / 16; ++kk) {
-              const uint64_t adesc = smem_desc_sw128(sA + kk * 32, 16, 1024);
+              const uint64_t adesc = smem_desc_sw128(sA + kk * 32, 16, A_SBO);
               const uint64_t bdesc = smem_desc_sw128(sB + kk * 2048, GM_SLAB_BYTES, 1024);
               umma_bf16(dt, adesc, bdesc, idesc, (kc != it.kb || kk != 0) ? 1u : 0u);
             }
@@ -507,6 +529,10 @@ __global__ void __launch_bounds__(PG_MAX_THREADS, 1)
       uint32_t doff[NI];
       int e, row0, rows, n0;
       pg_tile_info<MODE, NSLAB>(tiles, g0.n_blocks, it.unit, e, row0, rows, n0);
+      if (SMALL_A && rows > PG_SMALL_ROWS) {   // the host never launches this; stay in the slot
+        raise_error(MOE_DEVERR_BAD_INDEX);
+        rows = PG_SMALL_ROWS;
+      }
 #pragma unroll
       for (int i = 0; i < NI; ++i) {
         const int r = gw * (4 * NI) + 4 * i + sub;

@@ -38,6 +38,9 @@ constexpr unsigned kKnownFlags = MOE_FLAG_NO_RENORM | MOE_FLAG_ROUTER_FP64 |
 
 #define GEMM_GEGLU grouped_gemm_persistent_kernel<kGemmStages, EPI_GEGLU, 4, true>
 #define GEMM_FFN grouped_gemm_persistent_kernel<kGemmStages, EPI_GEGLU, 4, true, true>
+// batches of at most 8 tokens (<= 8 rows per tile): 1 KB A slots, 6 stages
+constexpr int kSmallStages = 6;
+#define GEMM_FFN_SMALL grouped_gemm_persistent_kernel<kSmallStages, EPI_GEGLU, 4, true, true, true>
 #define GEMM_STORE grouped_gemm_persistent_kernel<kGemmStages, EPI_STORE, 4>
 #define GEMM_SCREEN grouped_gemm_kernel<kGemmStages, EPI_F32, 2>
 
@@ -284,6 +287,8 @@ DeviceState* device_state(int* dev_out) {
             cudaSuccess ||
         cudaFuncSetAttribute(GEMM_FFN, cudaFuncAttributeMaxDynamicSharedMemorySize, gs) !=
             cudaSuccess ||
+        cudaFuncSetAttribute(GEMM_FFN_SMALL, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             pgemm_smem_bytes<kSmallStages, 4, true>()) != cudaSuccess ||
         cudaFuncSetAttribute(GEMM_STORE, cudaFuncAttributeMaxDynamicSharedMemorySize, gs) !=
             cudaSuccess ||
         cudaFuncSetAttribute(GEMM_SCREEN, cudaFuncAttributeMaxDynamicSharedMemorySize, gs2) !=
@@ -638,6 +643,13 @@ moe_status_t moe_forward(const void* x, const void* w_router, const float* route
       if (const moe_status_t ls = launched(); ls != MOE_OK) return ls;
       launch(true, GEMM_STORE, dim3(G), dim3(pgemm_threads(false)), smem, tm_h, tm_wd, tm_wd,
              tm_h, tm_wd, tl, g2, g2, h_ready);
+    } else if (T <= PG_SMALL_ROWS) {
+      // every tile has at most T <= 8 rows: 8-row A slots (and an 8-row box over h)
+      CUtensorMap tm_h8;
+      if (!make_map_2d(&tm_h8, hbuf, I, P, PG_SMALL_ROWS, 64)) return cuda_failed(-1);
+      launch(true, GEMM_FFN_SMALL, dim3(G), dim3(pgemm_threads(true)),
+             pgemm_smem_bytes<kSmallStages, 4, true>(), tm_xp, tm_wg, tm_wu, tm_h8, tm_wd, tl, g1,
+             g2, h_ready);
     } else {
       launch(true, GEMM_FFN, dim3(G), dim3(pgemm_threads(true)), smem, tm_xp, tm_wg, tm_wu, tm_h,
              tm_wd, tl, g1, g2, h_ready);

@@ -232,6 +232,49 @@ __device__ __forceinline__ void warp_topk(const double (&L)[EPL], int E, int k, 
   warp_topk_ids<EPL>(L, id, k, taken, sel_e, sel_v);
 }
 
+// The same selection by rank counting through shared memory: every lane ranks its own
+// experts against all E values (broadcast reads of `scratch`), and the expert of rank r < k
+// takes slot r.  Ranks are unique because ties go to the lower id.  NaN logits rank below
+// every number.  One pass of E comparisons instead of k dependent shuffle reductions.
+// scratch: this warp's E + 16 doubles.
+template <int EPL>
+__device__ __forceinline__ void warp_topk_ranked(const double (&L)[EPL], int E, int k,
+                                                 double* scratch, bool (&taken)[EPL],
+                                                 int (&sel_e)[8], double (&sel_v)[8]) {
+  const int lane = threadIdx.x & 31;
+  double* s_sv = scratch + E;
+  int* s_se = reinterpret_cast<int*>(s_sv + 8);
+  double v[EPL];
+#pragma unroll
+  for (int i = 0; i < EPL; ++i) {
+    v[i] = isnan(L[i]) ? -INFINITY : L[i];
+    if (lane + 32 * i < E) scratch[lane + 32 * i] = v[i];
+  }
+  __syncwarp();
+  int rank[EPL];
+#pragma unroll
+  for (int i = 0; i < EPL; ++i) rank[i] = 0;
+  for (int e2 = 0; e2 < E; ++e2) {
+    const double v2 = scratch[e2];
+#pragma unroll
+    for (int i = 0; i < EPL; ++i) rank[i] += rank_before(v2, e2, v[i], lane + 32 * i) ? 1 : 0;
+  }
+#pragma unroll
+  for (int i = 0; i < EPL; ++i) {
+    taken[i] = lane + 32 * i < E && rank[i] < k;
+    if (taken[i]) {
+      s_sv[rank[i]] = L[i];
+      s_se[rank[i]] = lane + 32 * i;
+    }
+  }
+  __syncwarp();
+  for (int r = 0; r < k; ++r) {
+    sel_v[r] = s_sv[r];
+    sel_e[r] = s_se[r];
+  }
+  __syncwarp();   // scratch free again
+}
+
 // Value held by the lane/slot whose id is `e` (every lane gets it).
 template <int EPL>
 __device__ __forceinline__ double warp_value_of(const double (&V)[EPL], const int (&id)[EPL], int e) {
@@ -250,17 +293,18 @@ __device__ __forceinline__ double warp_value_of(const double (&V)[EPL], const in
 // Given a token's logits L (expert lane + 32 i) and their rounding bounds beta: select the
 // top-k by (value desc, id asc), verify every decision against the bounds, recompute the
 // token exactly when one is too close to call, then write ids and (renormalised) weights.
+// scratch: this warp's E + 16 doubles of shared memory.
 template <int EPL>
 __device__ __forceinline__ void router_finish_token(
     double (&L)[EPL], const double (&beta)[EPL], int t, const __nv_bfloat16* __restrict__ x,
     const __nv_bfloat16* __restrict__ wr, const float* __restrict__ bias, int H, int E, int k,
     int renorm, int32_t* __restrict__ ids, float* __restrict__ wts,
-    unsigned* __restrict__ stats) {
+    unsigned* __restrict__ stats, double* scratch) {
   const int lane = threadIdx.x & 31;
   bool taken[EPL];
   int sel_e[8];
   double sel_v[8];
-  warp_topk<EPL>(L, E, k, taken, sel_e, sel_v);
+  warp_topk_ranked<EPL>(L, E, k, scratch, taken, sel_e, sel_v);
 
   // Verify every decision against the rounding bound.
   int eid[EPL];
@@ -298,7 +342,7 @@ __device__ __forceinline__ void router_finish_token(
       const int e = lane + 32 * i;
       if (e < E) L[i] = bias ? acc[i] + (double)bias[e] : acc[i];
     }
-    warp_topk<EPL>(L, E, k, taken, sel_e, sel_v);
+    warp_topk_ranked<EPL>(L, E, k, scratch, taken, sel_e, sel_v);
   }
 
   // Weights: softmax over all E, renormalised over the k selected (or not).  Lane r < k
@@ -340,6 +384,7 @@ __global__ void __launch_bounds__(256) router_select_kernel(
   pdl_trigger();
   pdl_wait();
   if (blockIdx.x == 0 && threadIdx.x == 0) stats[3] = 0;   // path: fp64 logits
+  __shared__ double s_topk[8][256 + 16];   // per-warp top-k scratch (blocks of 8 warps)
   const int lane = threadIdx.x & 31;
   const int warps_per_block = blockDim.x >> 5;
   for (int t = blockIdx.x * warps_per_block + (threadIdx.x >> 5); t < T;
@@ -392,7 +437,8 @@ __global__ void __launch_bounds__(256) router_select_kernel(
         L[i] = -DBL_MAX;
       }
     }
-    router_finish_token<EPL>(L, beta, t, x, wr, bias, H, E, k, renorm, ids, wts, stats);
+    router_finish_token<EPL>(L, beta, t, x, wr, bias, H, E, k, renorm, ids, wts, stats,
+                             s_topk[threadIdx.x >> 5]);
   }
 }
 
