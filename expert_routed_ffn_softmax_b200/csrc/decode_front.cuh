@@ -14,7 +14,8 @@
 //      verified against the rounding bound; a token too close to call goes to the warp path
 //      of router_select_kernel, which recomputes it exactly); its ids also go to CTA 0;
 //   3. cluster barrier; CTA 0 runs the dispatch of the T*k <= 64 pairs from shared memory
-//      (counts, offsets, stable permutation, tile list) and zeroes the GEMM counters;
+//      (counts, offsets, stable permutation, tile list); the GEMM counters were zeroed by
+//      all CTAs in step 1;
 //   4. (only when an Xp buffer is given, for decode tiles) cluster barrier; all warps of
 //      the cluster copy the x rows into Xp.  By default GEMM-1 gathers the rows itself.
 // The summation depth per logit is H/64 + 7 + 7 + 1 (<= H + 8), inside the bound the
@@ -161,6 +162,10 @@ __global__ void __cluster_dims__(kFrontRanks, 1, 1) __launch_bounds__(32 * kFron
       }
     }
   }
+  // The GEMM counters are zeroed by all CTAs while the W_router copies are in flight (this
+  // launch runs in plain stream order: no earlier GEMM is still using them).
+  for (int i = rank * blockDim.x + tid; i < n_counters; i += kFrontRanks * blockDim.x)
+    gemm_counters[i] = 0;
   __syncthreads();   // also publishes the barrier initialisation
   // |x_t|^2 over the slice -> CTA t
   for (int tt = warp; tt < nt; tt += NW) {
@@ -331,7 +336,6 @@ __global__ void __cluster_dims__(kFrontRanks, 1, 1) __launch_bounds__(32 * kFron
   // ---- 3. CTA 0: dispatch of the P = T*k <= 64 pairs from shared memory, all threads
   if (rank == 0) {
     const int P = nt * k;
-    for (int i = tid; i < n_counters; i += blockDim.x) gemm_counters[i] = 0;
     if (tid < E) {   // pairs of expert tid
       int c = 0;
 #pragma unroll 8
@@ -340,6 +344,7 @@ __global__ void __cluster_dims__(kFrontRanks, 1, 1) __launch_bounds__(32 * kFron
     } else if (tid >= 128 && tid - 128 < P) {   // pair q's rank among its expert's pairs
       const int q = tid - 128, e = s_ids[q];
       int before = 0;
+#pragma unroll 8
       for (int q2 = 0; q2 < q; ++q2) before += (s_ids[q2] == e);
       s_bef[q] = before;
       if ((unsigned)e >= (unsigned)E) raise_error(MOE_DEVERR_BAD_INDEX);
