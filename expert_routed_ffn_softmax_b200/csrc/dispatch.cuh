@@ -39,7 +39,8 @@ __global__ void __launch_bounds__(256) dispatch_count_kernel(const int32_t* __re
 // One CTA (blockDim >= E).  counts, offsets, chunk_base[c][e] = offsets[e] + pairs of e in
 // chunks before c, and the GEMM tile list: for every expert with n_e > 0, tiles of BM rows
 // (expert, first sorted row, rows in tile), in expert order.  Also zeroes the split-unit
-// counters the grouped GEMMs use.
+// counters the grouped GEMMs use.  Thread e walks its column of chunk counts with 8 loads
+// in flight; warp 0 scans the experts (8 per lane) with shuffles.
 __global__ void __launch_bounds__(256) dispatch_scan_kernel(
     const int32_t* __restrict__ chunk_counts, int nchunks, int E, int P, int BM,
     int32_t* __restrict__ counts, int32_t* __restrict__ offsets, int32_t* __restrict__ chunk_base,
@@ -50,26 +51,59 @@ __global__ void __launch_bounds__(256) dispatch_scan_kernel(
   pdl_wait();
   __shared__ int s_cnt[256], s_off[256], s_tstart[256];
   for (int i = threadIdx.x; i < n_counters; i += blockDim.x) gemm_counters[i] = 0;
-  const int e = threadIdx.x;
+  const int e = threadIdx.x, lane = threadIdx.x & 31;
   int run = 0;
   if (e < E) {
-    for (int c = 0; c < nchunks; ++c) {
-      chunk_base[(size_t)c * E + e] = run;
-      run += chunk_counts[(size_t)c * E + e];
+    for (int c0 = 0; c0 < nchunks; c0 += 8) {
+      int v[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u)
+        v[u] = c0 + u < nchunks ? __ldcg(chunk_counts + (size_t)(c0 + u) * E + e) : 0;
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        if (c0 + u < nchunks) chunk_base[(size_t)(c0 + u) * E + e] = run;
+        run += v[u];
+      }
     }
     s_cnt[e] = run;
   }
   __syncthreads();
-  if (threadIdx.x == 0) {
-    int o = 0, ts = 0;
-    for (int i = 0; i < E; ++i) {
-      s_off[i] = o;
-      s_tstart[i] = ts;
-      o += s_cnt[i];
-      ts += (s_cnt[i] + BM - 1) / BM;
+  if (threadIdx.x < 32) {
+    // exclusive scans of counts and tiles over the experts; lane owns 8*lane .. 8*lane+7
+    int c[8], nt[8], cs = 0, ts = 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int ee = 8 * lane + i;
+      c[i] = ee < E ? s_cnt[ee] : 0;
+      nt[i] = (c[i] + BM - 1) / BM;
+      cs += c[i];
+      ts += nt[i];
     }
-    offsets[E] = o;
-    *tile_num = ts;
+    int ci = cs, ti = ts;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int a = __shfl_up_sync(0xffffffffu, ci, off);
+      const int b = __shfl_up_sync(0xffffffffu, ti, off);
+      if (lane >= off) {
+        ci += a;
+        ti += b;
+      }
+    }
+    int o = ci - cs, tt = ti - ts;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int ee = 8 * lane + i;
+      if (ee < E) {
+        s_off[ee] = o;
+        s_tstart[ee] = tt;
+      }
+      o += c[i];
+      tt += nt[i];
+    }
+    if (lane == 31) {
+      offsets[E] = o;
+      *tile_num = tt;
+    }
   }
   __syncthreads();
   if (e < E) {
@@ -87,32 +121,65 @@ __global__ void __launch_bounds__(256) dispatch_scan_kernel(
   }
 }
 
-// One warp per chunk: stable positions pos = chunk_base[c][e] + rank among earlier pairs
-// of the chunk with the same expert.  perm[pos] = q, inv[q] = pos.
-__global__ void __launch_bounds__(32) dispatch_rank_kernel(const int32_t* __restrict__ ids, int P,
-                                                           int E,
-                                                           const int32_t* __restrict__ chunk_base,
-                                                           int32_t* __restrict__ perm,
-                                                           int32_t* __restrict__ inv) {
+// One CTA of 8 warps per chunk: warp w takes pairs [256 w, 256 w + 256) of the chunk
+// (8 per lane, loaded up front), counts them per expert, the warps' counts are scanned in
+// warp order per expert, and each warp ranks its pairs in order with __match_any_sync:
+// pos = chunk_base[c][e] + pairs of e in earlier warps + rank within the warp's earlier
+// pairs.  perm[pos] = q, inv[q] = pos.  Dynamic shared memory: 9 * E ints.
+constexpr int kRankWarps = 8;
+__global__ void __launch_bounds__(32 * kRankWarps) dispatch_rank_kernel(
+    const int32_t* __restrict__ ids, int P, int E, const int32_t* __restrict__ chunk_base,
+    int32_t* __restrict__ perm, int32_t* __restrict__ inv) {
   pdl_trigger();
   pdl_wait();
-  extern __shared__ int base[];
-  const int lane = threadIdx.x;
-  for (int e = lane; e < E; e += 32) base[e] = chunk_base[(size_t)blockIdx.x * E + e];
-  __syncwarp();
-  const int q0 = blockIdx.x * kDispatchChunk, q1 = min(P, q0 + kDispatchChunk);
+  extern __shared__ int rank_sm[];
+  int* wcnt = rank_sm;                   // [kRankWarps][E] pairs of e in warp w
+  int* base = rank_sm + kRankWarps * E;  // [E] chunk base
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  constexpr int kSub = kDispatchChunk / kRankWarps;   // 256 pairs per warp
+  const int q0 = blockIdx.x * kDispatchChunk + warp * kSub;
+  for (int i = threadIdx.x; i < kRankWarps * E; i += blockDim.x) wcnt[i] = 0;
+  for (int i = threadIdx.x; i < E; i += blockDim.x) base[i] = chunk_base[(size_t)blockIdx.x * E + i];
+  int ev[kSub / 32];
+#pragma unroll
+  for (int it = 0; it < kSub / 32; ++it) {
+    const int q = q0 + 32 * it + lane;
+    int e = q < P ? __ldcg(ids + q) : -1;
+    if (q < P && (unsigned)e >= (unsigned)E) e = -2;   // counted as an error already
+    ev[it] = e;
+  }
+  __syncthreads();
   const unsigned lt = (1u << lane) - 1u;
-  for (int qb = q0; qb < q1; qb += 32) {
-    const int q = qb + lane;
-    const bool valid = q < q1;
-    int e = valid ? ids[q] : -1;
-    if (valid && (unsigned)e >= (unsigned)E) e = -2;  // counted as an error already
+  // per-warp counts
+#pragma unroll
+  for (int it = 0; it < kSub / 32; ++it) {
+    const int e = ev[it];
     const unsigned grp = __match_any_sync(0xffffffffu, e);
-    const int rank = __popc(grp & lt);
-    int pos = 0;
-    if (e >= 0) pos = base[e] + rank;
+    if (e >= 0 && lane == 31 - __clz(grp)) wcnt[warp * E + e] += __popc(grp);
     __syncwarp();
-    if (e >= 0 && lane == 31 - __clz(grp)) base[e] += __popc(grp);
+  }
+  __syncthreads();
+  // exclusive scan over the warps, per expert (in place): wcnt[w][e] = pairs of e in warps < w
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    int run = base[e];
+#pragma unroll
+    for (int w = 0; w < kRankWarps; ++w) {
+      const int v = wcnt[w * E + e];
+      wcnt[w * E + e] = run;
+      run += v;
+    }
+  }
+  __syncthreads();
+  int* wb = wcnt + warp * E;   // this warp's running base per expert
+#pragma unroll
+  for (int it = 0; it < kSub / 32; ++it) {
+    const int q = q0 + 32 * it + lane;
+    const int e = ev[it];
+    const unsigned grp = __match_any_sync(0xffffffffu, e);
+    int pos = 0;
+    if (e >= 0) pos = wb[e] + __popc(grp & lt);
+    __syncwarp();
+    if (e >= 0 && lane == 31 - __clz(grp)) wb[e] += __popc(grp);
     __syncwarp();
     if (e >= 0) {
       perm[pos] = q;

@@ -605,7 +605,8 @@ moe_status_t moe_forward(const void* x, const void* w_router, const float* route
       launch(true, dispatch_scan_kernel, dim3(1), dim3(256), 0, (const int32_t*)chunk_counts,
              L.nchunks, E, P, L.bm, counts, offsets, chunk_base, tile_num, tile_expert, tile_row0,
              tile_rows, gemm_counters, L.n_counters);
-      launch(true, dispatch_rank_kernel, dim3(L.nchunks), dim3(32), E * sizeof(int),
+      launch(true, dispatch_rank_kernel, dim3(L.nchunks), dim3(32 * kRankWarps),
+             (kRankWarps + 1) * E * sizeof(int),
              (const int32_t*)ids, P, E, (const int32_t*)chunk_base, perm, inv);
     }
     if (dec)
