@@ -326,33 +326,55 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const uint4* __restric
 }
 
 // y[t, :] = sum_{j ascending} w[t,j] * O[inv[t,j], :]   (fp32, one bf16 rounding)
-// One thread per 8-element vector of y; the k rows it reads are loaded back to back.
+// One warp per item (token t, chunk c of 64 16-byte vectors of the row): lanes j < k fetch
+// slot j's row and weight, which the warp shares by shuffles; then each lane loads its two
+// vectors of all k rows (16 loads in flight) and sums them in slot order.
+constexpr int kCombineChunkVec = 64;
 __global__ void __launch_bounds__(256) combine_kernel(const uint4* __restrict__ O,
                                                       const int32_t* __restrict__ inv,
                                                       const float* __restrict__ w, int T, int k,
                                                       int nvec, uint4* __restrict__ y) {
   pdl_trigger();
   pdl_wait();
-  const size_t total = (size_t)T * nvec;
-  for (size_t idx = (size_t)blockIdx.x * blockDim.x + threadIdx.x; idx < total;
-       idx += (size_t)gridDim.x * blockDim.x) {
-    const int t = (int)(idx / nvec), v = (int)(idx - (size_t)t * nvec);
+  const int lane = threadIdx.x & 31;
+  const int nch = (nvec + kCombineChunkVec - 1) / kCombineChunkVec;
+  const long long items = (long long)T * nch;
+  const long long nwarps = (long long)gridDim.x * (blockDim.x >> 5);
+  for (long long it = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); it < items;
+       it += nwarps) {
+    const int t = (int)(it / nch), c = (int)(it - (long long)t * nch);
+    int myp = 0;
+    float myw = 0.f;
+    if (lane < k) {
+      myp = __ldg(inv + (size_t)t * k + lane);
+      myw = __ldg(w + (size_t)t * k + lane);
+    }
     int pos[8];
     float wj[8];
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
-      pos[j] = j < k ? inv[(size_t)t * k + j] : 0;
-      wj[j] = j < k ? w[(size_t)t * k + j] : 0.f;
+      pos[j] = __shfl_sync(0xffffffffu, myp, j);
+      wj[j] = __shfl_sync(0xffffffffu, myw, j);
     }
-    {
+    const int v0 = c * kCombineChunkVec + lane, v1 = v0 + 32;
+    const bool ok0 = v0 < nvec, ok1 = v1 < nvec;
+    uint4 r0[8], r1[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      if (j < k && ok0) r0[j] = __ldcs(O + (size_t)pos[j] * nvec + v0);
+      if (j < k && ok1) r1[j] = __ldcs(O + (size_t)pos[j] * nvec + v1);
+    }
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+      if (half == 0 ? !ok0 : !ok1) continue;
+      const uint4* r = half == 0 ? r0 : r1;
       float acc[8];
 #pragma unroll
       for (int i = 0; i < 8; ++i) acc[i] = 0.f;
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
         if (j < k) {
-          const uint4 raw = O[(size_t)pos[j] * nvec + v];
-          const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&raw);
+          const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&r[j]);
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
             const float2 f = __bfloat1622float2(p[i]);
@@ -366,7 +388,7 @@ __global__ void __launch_bounds__(256) combine_kernel(const uint4* __restrict__ 
       out.y = pack_bf16x2(acc[2], acc[3]);
       out.z = pack_bf16x2(acc[4], acc[5]);
       out.w = pack_bf16x2(acc[6], acc[7]);
-      y[(size_t)t * nvec + v] = out;
+      y[(size_t)t * nvec + (half == 0 ? v0 : v1)] = out;
     }
   }
 }

@@ -658,11 +658,11 @@ moe_status_t moe_forward(const void* x, const void* w_router, const float* route
     if (const moe_status_t ls = launched(); ls != MOE_OK) return ls;
   }
   prof.mark();
-  // 5. combine
-  const long long cthreads = (long long)T * (H / 8);
-  launch(true, combine_kernel, dim3((int)std::min<long long>((cthreads + 255) / 256, gsm)),
-         dim3(256), 0, reinterpret_cast<const uint4*>(obuf), (const int32_t*)inv,
-         (const float*)wts, T, k, H / 8, static_cast<uint4*>(y));
+  // 5. combine: one warp per (token, 64-vector chunk), 8 warps per block
+  const long long citems = (long long)T * ((H / 8 + kCombineChunkVec - 1) / kCombineChunkVec);
+  launch(true, combine_kernel, dim3((int)std::min<long long>((citems + 7) / 8, gsm)), dim3(256),
+         0, reinterpret_cast<const uint4*>(obuf), (const int32_t*)inv, (const float*)wts, T, k,
+         H / 8, static_cast<uint4*>(y));
   if (const moe_status_t ls = launched(); ls != MOE_OK) return ls;
   prof.mark();
   prof.finish();
