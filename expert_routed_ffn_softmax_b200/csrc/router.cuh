@@ -503,7 +503,7 @@ constexpr int kScreenWarps = 8;
 // stats[2] = max over candidates of |screen - L| / (|x| |w|) (float bits, atomicMax),
 // stats[3] = 1 (the screen path).
 template <int EPL>
-__global__ void __launch_bounds__(256) router_screen_select_kernel(
+__global__ void __launch_bounds__(256, 3) router_screen_select_kernel(
     const float* __restrict__ screen, const __nv_bfloat16* __restrict__ x,
     const __nv_bfloat16* __restrict__ wrT, const double* __restrict__ wn2,
     const float* __restrict__ bias, int T, int H, int E, int k, double screen_c,
