@@ -53,8 +53,17 @@ bool flags_ok(unsigned flags) {
 }
 
 // Tensor-core screen + fp64 recheck, or fp64 logits for every expert.
-bool router_uses_screen(int T, unsigned flags) {
+// The screen's TMA map over W_router [H][E] needs 16-byte rows: E % 8 == 0.
+bool screen_shape_ok(int E) { return E % 8 == 0; }
+
+// A forced screen path needs a shape the screen supports.
+bool forced_path_ok(int E, unsigned flags) {
+  return !(flags & MOE_FLAG_ROUTER_SCREEN) || screen_shape_ok(E);
+}
+
+bool router_uses_screen(int T, int E, unsigned flags) {
   if (flags & (MOE_FLAG_NO_RENORM | MOE_FLAG_ROUTER_FP64)) return false;
+  if (!screen_shape_ok(E)) return false;
   if (flags & MOE_FLAG_ROUTER_SCREEN) return true;
   return T >= kScreenMinTokens;
 }
@@ -81,7 +90,7 @@ bool use_decode_gemm(int T, int H, int I, unsigned flags) {
 
 // Batches of at most 8 tokens take the fused router + dispatch + gather launch.
 bool use_decode_front(int T, int H, int E, unsigned flags) {
-  return T <= kFrontMaxTokens && E <= 128 && !router_uses_screen(T, flags) &&
+  return T <= kFrontMaxTokens && E <= 128 && !router_uses_screen(T, E, flags) &&
          H % (kFrontRanks * kFrontWarps) == 0 &&
          decode_front_smem_bytes(H, E) <= (size_t)kFrontSmemMax;
 }
@@ -136,7 +145,7 @@ Layout make_layout(int T, int H, int E, int I, int k, unsigned flags, bool forwa
     return at;
   };
   const size_t P = (size_t)T * k;
-  L.screen = router_uses_screen(T, flags);
+  L.screen = router_uses_screen(T, E, flags);
   L.stats = take(4 * sizeof(unsigned));
   if (L.screen) {
     L.scr = take(sizeof(float) * (size_t)T * E);
@@ -472,12 +481,14 @@ const char* moe_status_string(moe_status_t s) {
 }
 
 size_t moe_route_workspace_size(int T, int H, int E, int k, unsigned flags) {
-  if (!flags_ok(flags) || !shape_supported(T, H, E, 64, k, false)) return 0;
+  if (!flags_ok(flags) || !shape_supported(T, H, E, 64, k, false) || !forced_path_ok(E, flags))
+    return 0;
   return make_layout(T, H, E, 64, k, flags, false).total;
 }
 
 size_t moe_workspace_size(int T, int H, int E, int I, int k, unsigned flags) {
-  if (!flags_ok(flags) || !shape_supported(T, H, E, I, k, true)) return 0;
+  if (!flags_ok(flags) || !shape_supported(T, H, E, I, k, true) || !forced_path_ok(E, flags))
+    return 0;
   return make_layout(T, H, E, I, k, flags, true).total;
 }
 
@@ -490,7 +501,8 @@ moe_status_t moe_route(const void* x, const void* w_router, const float* router_
   if (T == 0) return MOE_OK;
   if (!x || !w_router || !topk_ids || !topk_weights || !workspace) return MOE_ERR_INVALID_ARG;
   if (!aligned16(x) || !aligned16(w_router) || !aligned16(workspace)) return MOE_ERR_INVALID_ARG;
-  if (!shape_supported(T, H, E, 64, k, false)) return MOE_ERR_UNSUPPORTED;
+  if (!shape_supported(T, H, E, 64, k, false) || !forced_path_ok(E, flags))
+    return MOE_ERR_UNSUPPORTED;
   const Layout L = make_layout(T, H, E, 64, k, flags, false);
   if (workspace_bytes < L.total) return MOE_ERR_NO_WORKSPACE;
   int dev = 0;
@@ -518,7 +530,8 @@ moe_status_t moe_forward(const void* x, const void* w_router, const float* route
       !aligned16(w_down) || !aligned16(y) || !aligned16(workspace))
     return MOE_ERR_INVALID_ARG;
   if (x == y) return MOE_ERR_INVALID_ARG;
-  if (!shape_supported(T, H, E, I, k, true)) return MOE_ERR_UNSUPPORTED;
+  if (!shape_supported(T, H, E, I, k, true) || !forced_path_ok(E, flags))
+    return MOE_ERR_UNSUPPORTED;
   if ((flags & MOE_FLAG_DECODE_TILES) && !decode_gemm_ok(T, H, I)) return MOE_ERR_INVALID_ARG;
   const Layout L = make_layout(T, H, E, I, k, flags, true);
   if (workspace_bytes < L.total) return MOE_ERR_NO_WORKSPACE;

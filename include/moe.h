@@ -58,7 +58,9 @@ enum {
   /* Router path.  By default batches of T >= 256 screen the logits on the tensor cores
    * and recompute in fp64 only the experts that can still reach the top-k; smaller
    * batches compute every logit in fp64.  Both give the same ids.  These flags force one
-   * path (testing and diagnosis); setting both is MOE_ERR_INVALID_ARG. */
+   * path (testing and diagnosis); setting both is MOE_ERR_INVALID_ARG.  The screen needs
+   * E % 8 == 0 (16-byte rows of W_router for its TMA loads): the default takes the fp64
+   * path otherwise, and forcing the screen is then MOE_ERR_UNSUPPORTED. */
   MOE_FLAG_ROUTER_FP64 = 1u << 1,
   MOE_FLAG_ROUTER_SCREEN = 1u << 2,
   /* Record a CUDA event at every stage boundary of the call; moe_last_stage_times()

@@ -239,3 +239,32 @@ def test_fused_ffn_matches_two_launches_bitwise(T, gemma_w):
     y2 = moe.forward(x, g["w_router"], g["w_gate"], g["w_up"], g["w_down"], 8, tiles="unfused")
     assert moe.sync_status() == 0
     assert torch.equal(y1, y2)
+
+
+# Other layer shapes the ABI accepts: 256 experts (8 per lane in the routers), few experts,
+# short hidden/intermediate sizes with ragged 128-column blocks, k from 1 to 8, every router
+# path and both FFN forms.  Inputs follow the same seeded recipe.
+OTHER_SHAPES = [
+    wl.MoEConfig("e256_k6", 40, 512, 256, 6, 192),
+    wl.MoEConfig("e256_T300", 300, 512, 256, 8, 128),
+    wl.MoEConfig("e64_T300", 300, 1024, 64, 4, 256),
+    wl.MoEConfig("e32_decode", 8, 2048, 32, 2, 128),
+    wl.MoEConfig("e12_h768", 5, 768, 12, 3, 64),
+    wl.MoEConfig("k1", 33, 1024, 16, 1, 320),
+]
+
+
+@pytest.mark.parametrize("router", ["auto", "fp64", "screen"])
+@pytest.mark.parametrize("cfg", OTHER_SHAPES, ids=[c.name for c in OTHER_SHAPES])
+def test_other_shapes(cfg, router, gemma_w):
+    if router == "screen" and cfg.E % 8:
+        # the screen needs 16-byte W_router rows; forcing it is refused, not run
+        x, c, g = layer_inputs(cfg, gemma_w)
+        with pytest.raises(moe.MoEError) as ei:
+            gpu_forward(x, g, cfg.k, True, router, "auto")
+        assert ei.value.code == 2   # MOE_ERR_UNSUPPORTED
+        return
+    run_case(cfg, gemma_w, 10**9, router=router)
+    run_case(cfg, gemma_w, 10**9, router=router, tiles="unfused")
+    if router != "screen":   # the screen path renormalises only
+        run_case(cfg, gemma_w, 10**9, router=router, renorm=False)
