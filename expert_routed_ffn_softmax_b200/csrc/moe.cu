@@ -17,6 +17,7 @@
 #include "dispatch.cuh"
 #include "grouped_gemm.cuh"
 #include "gemm_persistent.cuh"
+#include "ffn_dynamic.cuh"
 #include "decode_front.cuh"
 #include "gemm_decode.cuh"
 
@@ -131,7 +132,8 @@ struct Layout {
   size_t chunk_counts = 0, chunk_base = 0, counts = 0, offsets = 0, perm = 0, inv = 0;
   size_t tile_num = 0, tile_expert = 0, tile_row0 = 0, tile_rows = 0;
   size_t xp = 0, hbuf = 0, obuf = 0;
-  size_t partials = 0, partials2 = 0, counters = 0;
+  size_t partials = 0, partials2 = 0, counters = 0, dy_part1 = 0, dy_part2 = 0;
+  int dy_u1 = 0, dy_u2 = 0, dy_ctr = 0;   // dynamic small-batch FFN: units, counter offset
   int n_counters = 0;
   size_t total = 0;
 };
@@ -185,6 +187,17 @@ Layout make_layout(int T, int H, int E, int I, int k, unsigned flags, bool forwa
     L.partials = take(sizeof(float) * 2 * (size_t)kMaxGemmCtas * GM_BM * 256);
     L.partials2 = take(sizeof(float) * 2 * (size_t)kMaxGemmCtas * GM_BM * 256);
     L.n_counters = 2 * kStreamKCounters + L.max_tiles + 1;
+    if (T <= PG_SMALL_ROWS) {
+      // dynamic small-batch FFN: per-chunk partial tiles and per-unit chunk counts (+ the
+      // chunk counter).  A tile has >= 1 pair, so at most min(max_tiles, P) tiles.
+      const int mt = (int)std::min<long long>(L.max_tiles, P);
+      L.dy_u1 = mt * ((I + 127) / 128);
+      L.dy_u2 = mt * ((H + 255) / 256);
+      L.dy_part1 = take(sizeof(float) * (size_t)L.dy_u1 * DY_CH1 * DY_PART_FLOATS);
+      L.dy_part2 = take(sizeof(float) * (size_t)L.dy_u2 * DY_CH2 * DY_PART_FLOATS);
+      L.dy_ctr = L.n_counters;
+      L.n_counters += 1 + L.dy_u1 + L.dy_u2;
+    }
     L.counters = take(sizeof(int32_t) * L.n_counters);
   }
   L.total = off;
@@ -296,6 +309,8 @@ DeviceState* device_state(int* dev_out) {
             cudaSuccess ||
         cudaFuncSetAttribute(GEMM_FFN, cudaFuncAttributeMaxDynamicSharedMemorySize, gs) !=
             cudaSuccess ||
+        cudaFuncSetAttribute(expert_ffn_dynamic_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             dy_smem_bytes()) != cudaSuccess ||
         cudaFuncSetAttribute(GEMM_FFN_SMALL, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              pgemm_smem_bytes<kSmallStages, 4, true>()) != cudaSuccess ||
         cudaFuncSetAttribute(GEMM_STORE, cudaFuncAttributeMaxDynamicSharedMemorySize, gs) !=
@@ -657,6 +672,16 @@ moe_status_t moe_forward(const void* x, const void* w_router, const float* route
       if (const moe_status_t ls = launched(); ls != MOE_OK) return ls;
       launch(true, GEMM_STORE, dim3(G), dim3(pgemm_threads(false)), smem, tm_h, tm_wd, tm_wd,
              tm_h, tm_wd, tl, g2, g2, h_ready);
+    } else if (T <= PG_SMALL_ROWS && !(flags & MOE_FLAG_FUSED_FFN)) {
+      // at most 8 rows per tile, work handed out dynamically in k-chunks
+      CUtensorMap tm_h8;
+      if (!make_map_2d(&tm_h8, hbuf, I, P, PG_SMALL_ROWS, 64)) return cuda_failed(-1);
+      int32_t* dctr = gemm_counters + L.dy_ctr;
+      const DyState dys{dctr, dctr + 1, dctr + 1 + L.dy_u1,
+                        reinterpret_cast<float*>(ws + L.dy_part1),
+                        reinterpret_cast<float*>(ws + L.dy_part2)};
+      launch(true, expert_ffn_dynamic_kernel, dim3(G), dim3(pgemm_threads(true)), dy_smem_bytes(),
+             tm_wg, tm_wu, tm_h8, tm_wd, tl, g1, g2, h_ready, dys);
     } else if (T <= PG_SMALL_ROWS) {
       // every tile has at most T <= 8 rows: 8-row A slots (and an 8-row box over h)
       CUtensorMap tm_h8;
