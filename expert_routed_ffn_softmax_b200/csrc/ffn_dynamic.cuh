@@ -173,20 +173,13 @@ __global__ void __launch_bounds__(PG_MAX_THREADS, 1)
           pg_tile_info<EPI_GEGLU, NSLAB>(tiles, g1.n_blocks, d.unit, e, row0, rows, n0);
         else
           pg_tile_info<EPI_STORE, NSLAB>(tiles, g2.n_blocks, d.unit, e, row0, rows, n0);
-        if (d.phase == 1 && !all_h_ready) {
-          if (ld_acquire_gpu(h_ready + n_tiles) >= h_target * n_tiles) {
-            all_h_ready = true;
-          } else if (!wait_counter_geq(h_ready + d.unit / g2.n_blocks, h_target)) {
-            *abort_flag = 1;
-          }
-          fence_proxy_async_global();   // TMA reads of h after the generic acquire
-        }
-        for (int kc = d.kb; kc < d.ke; ++kc, ++q) {
-          const int s = q % DY_STAGES;
+        // Issue stage `kc` of the chunk: wait for the slot; B (and, unless deferred, A).
+        auto stage_in = [&](int kc, int qq, bool with_a) -> bool {
+          const int s = qq % DY_STAGES;
           if (*abort_flag ||
-              (q >= DY_STAGES && !mbar_wait(empty_bar(s), ((q / DY_STAGES) - 1) & 1))) {
+              (qq >= DY_STAGES && !mbar_wait(empty_bar(s), ((qq / DY_STAGES) - 1) & 1))) {
             *abort_flag = 1;
-            break;
+            return false;
           }
           const uint32_t sA = base + s * STAGE_BYTES;
           const uint32_t sB = sA + A_BYTES;
@@ -198,11 +191,37 @@ __global__ void __launch_bounds__(PG_MAX_THREADS, 1)
           } else {
             mbar_arrive_expect_tx(full_bar(s), A_BYTES + NSLAB * GM_SLAB_BYTES);
             mbar_arrive_cnt(full_bar(s), PG_GATHER_THREADS);   // in place of the gather warps
-            tma_load_2d(sA, &tmH8, full_bar(s), kc * GM_BK, row0);
             tma_load_4d(sB, &tmWd, full_bar(s), 0, kc * GM_BK, n0 / 64, e);
+            if (with_a) tma_load_2d(sA, &tmH8, full_bar(s), kc * GM_BK, row0);
           }
-          *n_issued = q + 1;
+          *n_issued = qq + 1;
+          return true;
+        };
+        bool ok = true;
+        int kc = d.kb;
+        if (d.phase == 1 && !all_h_ready) {
+          // GEMM-2 needs this tile's h rows (GEMM-1 units of any CTA).  The W_down tiles do
+          // not: load them for the first stages, then wait for h, then load its rows.
+          const int pre = min(d.ke - d.kb, DY_STAGES);
+          for (int t2 = 0; t2 < pre && ok; ++t2) ok = stage_in(d.kb + t2, q + t2, false);
+          if (ok) {
+            if (!wait_counter_geq(h_ready + d.unit / g2.n_blocks, h_target)) {
+              *abort_flag = 1;
+              ok = false;
+            } else {
+              all_h_ready = ld_acquire_gpu(h_ready + n_tiles) >= h_target * n_tiles;
+              fence_proxy_async_global();   // TMA reads of h after the generic acquire
+              for (int t2 = 0; t2 < pre; ++t2) {
+                const int s = (q + t2) % DY_STAGES;
+                tma_load_2d(base + s * STAGE_BYTES, &tmH8, full_bar(s), (d.kb + t2) * GM_BK, row0);
+              }
+            }
+          }
+          kc += pre;
+          q += pre;
         }
+        for (; ok && kc < d.ke; ++kc, ++q) ok = stage_in(kc, q, true);
+        if (!ok) break;
         c = cnext;
         ++i;
       }
