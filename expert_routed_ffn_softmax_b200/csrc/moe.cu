@@ -148,7 +148,7 @@ Layout make_layout(int T, int H, int E, int I, int k, unsigned flags, bool forwa
   };
   const size_t P = (size_t)T * k;
   L.screen = router_uses_screen(T, E, flags);
-  L.stats = take(4 * sizeof(unsigned));
+  L.stats = take(8 * sizeof(unsigned));   // router statistics [4], front-end counter [1]
   if (L.screen) {
     L.scr = take(sizeof(float) * (size_t)T * E);
     L.wrT = take(2 * (size_t)E * H);
@@ -602,16 +602,21 @@ moe_status_t moe_forward(const void* x, const void* w_router, const float* route
   // Dependent launches, except while stage events sit between the kernels.
   const Launch launch{st, !prof.on};
   if (use_decode_front(T, H, E, flags)) {
-    // 1+2. router, dispatch and gather in one cluster launch
-    MOE_TRY_CUDA(cudaMemsetAsync(stats, 0, 4 * sizeof(unsigned), st));
+    // 1+2. router and dispatch in one launch: one 8-CTA cluster per token.  stats[4] is the
+    // front end's token counter (zero at launch, left zero).
+    MOE_TRY_CUDA(cudaMemsetAsync(stats, 0, 8 * sizeof(unsigned), st));
     const double u = std::ldexp(1.0, -53), n = (double)H + 8.0;
     const double beta_scale = 2.0 * (n * u / (1.0 - n * u)) * 1.01;
-    launch(false, decode_front_kernel<4>, dim3(kFrontRanks), dim3(32 * kFrontWarps),
+    launch(false, decode_front_kernel<4>, dim3(kFrontRanks * T), dim3(32 * kFrontWarps),
            decode_front_smem_bytes(H, E), static_cast<const __nv_bfloat16*>(x),
            static_cast<const __nv_bfloat16*>(w_router), router_bias, T, H, E, k,
            (flags & MOE_FLAG_NO_RENORM) ? 0 : 1, beta_scale, ids, wts, stats, counts, offsets, perm,
            inv, tile_num, tile_expert, tile_row0, tile_rows, gemm_counters, L.n_counters, L.bm,
-           dec ? reinterpret_cast<uint4*>(xp) : nullptr, H / 8);
+           stats + 4);
+    if (dec)   // decode tiles read a gathered copy of the routed rows
+      launch(true, gather_rows_kernel, dim3(std::min((P + 7) / 8, gsm)), dim3(256), 0,
+             static_cast<const uint4*>(x), (const int32_t*)perm, P, k, H / 8,
+             reinterpret_cast<uint4*>(xp));
     if (const moe_status_t ls = launched(); ls != MOE_OK) return ls;
     prof.mark();
     prof.mark();

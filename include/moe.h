@@ -72,10 +72,14 @@ enum {
    * MOE_ERR_INVALID_ARG. */
   MOE_FLAG_DECODE_TILES = 1u << 4,
   MOE_FLAG_PREFILL_TILES = 1u << 5,
-  /* Prefill tiles run GEMM-1 (+GEGLU) and GEMM-2 either as one persistent launch (a CTA
-   * moves on to GEMM-2 tiles as soon as the GEMM-1 tiles they read are stored; the default
-   * for T*k <= 1024) or as two launches (the default above).  Both give the same bytes.
-   * These flags force one form; setting both is MOE_ERR_INVALID_ARG. */
+  /* Prefill tiles run GEMM-1 (+GEGLU) and GEMM-2 as one persistent launch for T*k <= 1024
+   * (a CTA moves on to GEMM-2 tiles as soon as the GEMM-1 tiles they read are stored) and
+   * as two launches above.  For T <= 8 the default single launch hands its work out
+   * dynamically (CTAs take k-chunks from a shared counter); its GEMM-1 sums are split in
+   * two chunks, so its bytes can differ from the other forms in the last bit of a few
+   * elements (it is deterministic).  MOE_FLAG_FUSED_FFN forces the single launch with a
+   * static schedule, MOE_FLAG_UNFUSED_FFN two launches; these two give the same bytes.
+   * Setting both is MOE_ERR_INVALID_ARG. */
   MOE_FLAG_UNFUSED_FFN = 1u << 6,
   MOE_FLAG_FUSED_FFN = 1u << 7
 };
