@@ -135,7 +135,8 @@ def algorithmic(cfg: wl.MoEConfig, counts: np.ndarray, has_bias: bool) -> dict:
 
 def kernel_source_sha() -> str:
     h = hashlib.sha256()
-    for f in ("grouped_gemm.cuh", "gemm_persistent.cuh", "gemm_decode.cuh", "ptx.cuh"):
+    for f in ("grouped_gemm.cuh", "gemm_persistent.cuh", "ffn_dynamic.cuh", "gemm_decode.cuh",
+              "ptx.cuh"):
         h.update(open(os.path.join(ROOT, "expert_routed_ffn_softmax_b200", "csrc", f), "rb").read())
     return h.hexdigest()[:16]
 
@@ -338,6 +339,7 @@ def run_native(args, cfg) -> None:
         fused = args.tiles == "fused" or (args.tiles in ("auto", "prefill")
                                           and cfg.T * cfg.k <= FUSED_FFN_MAX_PAIRS)
         kname = ("grouped_gemm_decode_kernel<EPI_GEGLU>+<EPI_STORE>" if args.tiles == "decode"
+                 else "expert_ffn_dynamic_kernel" if cfg.T <= 8 and args.tiles in ("auto", "prefill")
                  else "grouped_gemm_persistent_kernel<6,EPI_GEGLU,4,1,1,1>" if fused and cfg.T <= 8
                  else "grouped_gemm_persistent_kernel<4,EPI_GEGLU,4,1,1>" if fused
                  else "grouped_gemm_persistent_kernel<4,EPI_GEGLU,4,1,0>+<4,EPI_STORE,4,0,0>")
