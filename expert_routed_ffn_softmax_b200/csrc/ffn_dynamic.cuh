@@ -8,13 +8,13 @@
 // (CH1 chunks per GEMM-1 unit = (tile, 128 features), CH2 per GEMM-2 unit = (tile, 256
 // columns)), handed out in order from one global counter: every GEMM-1 chunk before any
 // GEMM-2 chunk, so a CTA never waits for work that is handed out after its own.  A chunk's
-// fp32 partial (at most 8 rows x 256 columns) goes to global memory; the CTA that completes
+// fp32 partial (at most R rows x 256 columns) goes to global memory; the CTA that completes
 // a unit's last chunk adds the unit's partials in chunk order (deterministic whatever the
 // timing), applies GEGLU (GEMM-1) or rounds (GEMM-2) and stores the rows.  GEMM-1 units
 // publish h_ready[tile]; a GEMM-2 chunk's TMA load of h waits for it.
 //
 // Roles as in gemm_persistent.cuh (TMA thread, MMA thread, 4 epilogue warps, 2 gather
-// warps), with the 8-row A slots of its SMALL_A form.  The TMA thread takes chunk ids and
+// warps), with A slots of R <= 64 rows (batches of T <= R tokens).  The TMA thread takes chunk ids and
 // passes them to the other roles through a ring of descriptors in shared memory (full /
 // empty mbarriers).  Every wait is bounded.
 #pragma once
@@ -22,24 +22,35 @@
 
 namespace moe {
 
-constexpr int DY_STAGES = 6;
 constexpr int DY_RING = 8;                           // chunk descriptors in flight per CTA
 constexpr int DY_CH1 = 2;                            // chunks per GEMM-1 unit
 constexpr int DY_CH2 = 1;                            // chunks per GEMM-2 unit
-constexpr int DY_ROWS = PG_SMALL_ROWS;               // rows per tile (<= 8 tokens)
-constexpr int DY_PART_FLOATS = DY_ROWS * 256;        // one chunk's partial tile
-constexpr int DY_EPI_WARP = 4;                       // warp 4 reads TMEM lanes 0..31
+
+// R = rows of a tile's A slot (a batch of T <= R tokens has at most T rows per tile):
+// 8, 16, 32 or 64.  The MMA still reads 128 rows of A; rows past R read the stage's weight
+// bytes, which follow the slot, and their accumulator rows are never stored.
+template <int R>
+struct DyShape {
+  static_assert(R == 8 || R == 16 || R == 32 || R == 64, "A slot rows");
+  static constexpr int A_BYTES = R * GM_BK * 2;
+  static constexpr int STAGE_BYTES = A_BYTES + 4 * GM_SLAB_BYTES;
+  static constexpr int STAGES = R <= 32 ? 6 : 5;
+  static constexpr int ROW_WARPS = (R + 31) / 32;    // epilogue warps holding rows
+  static constexpr int PART_FLOATS = R * 256;        // one chunk's partial tile
+  static constexpr int SMEM = 1024 + STAGES * STAGE_BYTES + 2048;
+};
 
 struct DyState {
   int* next;       // [1] next chunk id; zero at launch
-  int* done1;      // [U1] finished chunks per GEMM-1 unit; zero at launch
-  int* done2;      // [U2] finished chunks per GEMM-2 unit; zero at launch
-  float* part1;    // [U1 * CH1][8][256]
-  float* part2;    // [U2 * CH2][8][256]
+  int* done1;      // [U1][ROW_WARPS] finished chunks per GEMM-1 unit; zero at launch
+  int* done2;      // [U2][ROW_WARPS] finished chunks per GEMM-2 unit; zero at launch
+  float* part1;    // [U1 * CH1][R][256] (unused when CH1 == 1)
+  float* part2;    // [U2 * CH2][R][256] (unused when CH2 == 1)
 };
 
+template <int R>
 __host__ __device__ inline int dy_smem_bytes() {
-  return pgemm_smem_bytes<DY_STAGES, 4, true>() + 1024;   // + descriptor ring
+  return DyShape<R>::SMEM;
 }
 
 // A chunk: phase 0 = GEMM-1, 1 = GEMM-2; unit; chunk index j within the unit; k-steps
@@ -68,15 +79,21 @@ __device__ __forceinline__ DyChunk dy_decode(int c, int U1, int nk1, int nk2, in
   return d;
 }
 
+// tmH: h rows, box R rows x 64 columns.
+template <int R>
 __global__ void __launch_bounds__(PG_MAX_THREADS, 1)
     expert_ffn_dynamic_kernel(const __grid_constant__ CUtensorMap tmWg,
                               const __grid_constant__ CUtensorMap tmWu,
-                              const __grid_constant__ CUtensorMap tmH8,
+                              const __grid_constant__ CUtensorMap tmH,
                               const __grid_constant__ CUtensorMap tmWd, TileList tiles,
                               PGemm g1, PGemm g2, int* __restrict__ h_ready, DyState dy) {
+  using SH = DyShape<R>;
   constexpr int NSLAB = 4, BN = 256;
-  constexpr int A_BYTES = pgemm_a_bytes<NSLAB, true>();
-  constexpr int STAGE_BYTES = pgemm_stage_bytes<NSLAB, true>();
+  constexpr int A_BYTES = SH::A_BYTES;
+  constexpr int STAGE_BYTES = SH::STAGE_BYTES;
+  constexpr int DY_STAGES = SH::STAGES;
+  constexpr int NRW = SH::ROW_WARPS;
+  constexpr int PARTF = SH::PART_FLOATS;
   constexpr uint32_t TMEM_COLS = 2 * BN;
   static_assert(DY_CH1 >= 1 && DY_CH2 >= 1, "chunks");
 
@@ -121,7 +138,7 @@ __global__ void __launch_bounds__(PG_MAX_THREADS, 1)
     fence_barrier_init();
     tma_prefetch_desc(&tmWg);
     tma_prefetch_desc(&tmWu);
-    tma_prefetch_desc(&tmH8);
+    tma_prefetch_desc(&tmH);
     tma_prefetch_desc(&tmWd);
   }
   if (warp == 0) {
@@ -140,7 +157,7 @@ __global__ void __launch_bounds__(PG_MAX_THREADS, 1)
   const int nk1 = g1.K / GM_BK, nk2 = g2.K / GM_BK;
   const int ch1 = min(DY_CH1, nk1), ch2 = min(DY_CH2, nk2);
   const int total = U1 * ch1 + U2 * ch2;
-  const int h_target = g1.n_blocks;   // one release per GEMM-1 unit of the tile
+  const int h_target = NRW * g1.n_blocks;   // one release per (GEMM-1 unit, row warp)
 
   // Read descriptor i (bounded wait); every reader then releases it.  -1 = no more work,
   // -2 = a wait ran out.
@@ -192,7 +209,7 @@ __global__ void __launch_bounds__(PG_MAX_THREADS, 1)
             mbar_arrive_expect_tx(full_bar(s), A_BYTES + NSLAB * GM_SLAB_BYTES);
             mbar_arrive_cnt(full_bar(s), PG_GATHER_THREADS);   // in place of the gather warps
             tma_load_4d(sB, &tmWd, full_bar(s), 0, kc * GM_BK, n0 / 64, e);
-            if (with_a) tma_load_2d(sA, &tmH8, full_bar(s), kc * GM_BK, row0);
+            if (with_a) tma_load_2d(sA, &tmH, full_bar(s), kc * GM_BK, row0);
           }
           *n_issued = qq + 1;
           return true;
@@ -213,7 +230,7 @@ __global__ void __launch_bounds__(PG_MAX_THREADS, 1)
               fence_proxy_async_global();   // TMA reads of h after the generic acquire
               for (int t2 = 0; t2 < pre; ++t2) {
                 const int s = (q + t2) % DY_STAGES;
-                tma_load_2d(base + s * STAGE_BYTES, &tmH8, full_bar(s), (d.kb + t2) * GM_BK, row0);
+                tma_load_2d(base + s * STAGE_BYTES, &tmH, full_bar(s), (d.kb + t2) * GM_BK, row0);
               }
             }
           }
@@ -260,7 +277,7 @@ __global__ void __launch_bounds__(PG_MAX_THREADS, 1)
           const uint32_t sB = sA + A_BYTES;
 #pragma unroll
           for (int kk = 0; kk < GM_BK / 16; ++kk) {
-            const uint64_t adesc = smem_desc_sw128(sA + kk * 32, 16, 0);   // 8 rows, repeated
+            const uint64_t adesc = smem_desc_sw128(sA + kk * 32, 16, 1024);
             const uint64_t bdesc = smem_desc_sw128(sB + kk * 2048, GM_SLAB_BYTES, 1024);
             umma_bf16(dt, adesc, bdesc, idesc, (kc != d.kb || kk != 0) ? 1u : 0u);
           }
@@ -275,9 +292,10 @@ __global__ void __launch_bounds__(PG_MAX_THREADS, 1)
     }
   } else if (warp < 6) {
     // -------------------------------------------------------------- epilogue (warps 2-5)
-    // Rows 0..7 of every tile are TMEM lanes 0..7, read by warp 4; the other warps only
-    // keep the accumulator hand-off going.
-    const bool rows_warp = warp == DY_EPI_WARP;
+    // Warp w reads TMEM lanes 32 (w % 4) .. +31; the rows of a tile (< R) sit in the first
+    // NRW of those quadrants.  The other warps only keep the accumulator hand-off going.
+    const int quad = warp & 3;
+    const bool rows_warp = quad < NRW;
     for (int i = 0;; ++i) {
       int c = 0;
       if (lane == 0) c = read_desc(i);
@@ -304,75 +322,103 @@ __global__ void __launch_bounds__(PG_MAX_THREADS, 1)
       else
         pg_tile_info<EPI_STORE, NSLAB>(tiles, g.n_blocks, d.unit, e, row0, rows, n0);
       const int nch = d.phase == 0 ? ch1 : ch2;
-      float* part = d.phase == 0 ? dy.part1 + (size_t)d.unit * DY_CH1 * DY_PART_FLOATS
-                                 : dy.part2 + (size_t)d.unit * DY_CH2 * DY_PART_FLOATS;
-      const bool row_ok = rows_warp && lane < rows && lane < DY_ROWS;
-      if (rows_warp) {
-        // this chunk's partial rows -> global
-        const uint32_t trow = tmem + b * BN;   // warp 4 reads lanes 0..31
-        float* prow = part + (size_t)d.j * DY_PART_FLOATS + (size_t)lane * 256;
+      const int r_local = quad * 32 + lane;
+      const bool row_ok = rows_warp && r_local < rows && r_local < R;
+      const uint32_t trow = tmem + b * BN + (static_cast<uint32_t>(quad * 32) << 16);
+      if (nch == 1) {
+        // the whole unit in one chunk: epilogue straight from TMEM
+        if (rows_warp) {
+          const int NC = d.phase == 0 ? BN / 2 : BN;
 #pragma unroll 1
-        for (int cc = 0; cc < BN; cc += 32) {
-          uint32_t v[32];
-          tmem_ld_32x32b_x32(trow + cc, v);
-          tmem_ld_wait();
-          if (row_ok) {
-#pragma unroll
-            for (int k4 = 0; k4 < 8; ++k4)
-              reinterpret_cast<uint4*>(prow + cc)[k4] =
-                  make_uint4(v[4 * k4], v[4 * k4 + 1], v[4 * k4 + 2], v[4 * k4 + 3]);
-          }
-        }
-      }
-      tc_fence_before();
-      mbar_arrive(tempty_bar(b));
-      if (!rows_warp) continue;
-      __threadfence();
-      __syncwarp();
-      int last = 0;
-      if (lane == 0) {
-        int* ctr = (d.phase == 0 ? dy.done1 : dy.done2) + d.unit;
-        last = atomicAdd(ctr, 1) == nch - 1;
-      }
-      last = __shfl_sync(0xffffffffu, last, 0);
-      if (!last) continue;
-      // the unit's last chunk: add the partials in chunk order and finish the rows
-      __threadfence();
-      if (row_ok) {
-        const int row = row0 + lane;
-        constexpr int NC1 = BN / 2;
-        const int NC = d.phase == 0 ? NC1 : BN;
-#pragma unroll 1
-        for (int cc = 0; cc < NC; cc += 32) {
-          float gsum[32], usum[32];
-#pragma unroll
-          for (int k2 = 0; k2 < 32; ++k2) gsum[k2] = usum[k2] = 0.f;
-          for (int jj = 0; jj < nch; ++jj) {
-            const float* src = part + (size_t)jj * DY_PART_FLOATS + (size_t)lane * 256;
-#pragma unroll
-            for (int k4 = 0; k4 < 8; ++k4) {
-              const float4 a = __ldcg(reinterpret_cast<const float4*>(src + cc) + k4);
-              gsum[4 * k4] += a.x;
-              gsum[4 * k4 + 1] += a.y;
-              gsum[4 * k4 + 2] += a.z;
-              gsum[4 * k4 + 3] += a.w;
-              if (d.phase == 0) {
-                const float4 bq = __ldcg(reinterpret_cast<const float4*>(src + NC1 + cc) + k4);
-                usum[4 * k4] += bq.x;
-                usum[4 * k4 + 1] += bq.y;
-                usum[4 * k4 + 2] += bq.z;
-                usum[4 * k4 + 3] += bq.w;
-              }
+          for (int cc = 0; cc < NC; cc += 32) {
+            uint32_t gv[32], uv[32];
+            tmem_ld_32x32b_x32(trow + cc, gv);
+            if (d.phase == 0) tmem_ld_32x32b_x32(trow + BN / 2 + cc, uv);
+            tmem_ld_wait();
+            if (row_ok) {
+              if (d.phase == 0)
+                pg_store32<EPI_GEGLU, NSLAB>(g.out, g.ldo, row0 + r_local, n0, cc, g.N_total,
+                                             reinterpret_cast<const float*>(gv),
+                                             reinterpret_cast<const float*>(uv));
+              else
+                pg_store32<EPI_STORE, NSLAB>(g.out, g.ldo, row0 + r_local, n0, cc, g.N_total,
+                                             reinterpret_cast<const float*>(gv),
+                                             reinterpret_cast<const float*>(uv));
             }
           }
-          if (d.phase == 0)
-            pg_store32<EPI_GEGLU, NSLAB>(g.out, g.ldo, row, n0, cc, g.N_total, gsum, usum);
-          else
-            pg_store32<EPI_STORE, NSLAB>(g.out, g.ldo, row, n0, cc, g.N_total, gsum, usum);
+        }
+        tc_fence_before();
+        mbar_arrive(tempty_bar(b));
+      } else {
+        float* part = (d.phase == 0 ? dy.part1 + (size_t)d.unit * DY_CH1 * PARTF
+                                    : dy.part2 + (size_t)d.unit * DY_CH2 * PARTF);
+        if (rows_warp) {
+          // this chunk's partial rows -> global
+          float* prow = part + (size_t)d.j * PARTF + (size_t)r_local * 256;
+#pragma unroll 1
+          for (int cc = 0; cc < BN; cc += 32) {
+            uint32_t v[32];
+            tmem_ld_32x32b_x32(trow + cc, v);
+            tmem_ld_wait();
+            if (row_ok) {
+#pragma unroll
+              for (int k4 = 0; k4 < 8; ++k4)
+                reinterpret_cast<uint4*>(prow + cc)[k4] =
+                    make_uint4(v[4 * k4], v[4 * k4 + 1], v[4 * k4 + 2], v[4 * k4 + 3]);
+            }
+          }
+        }
+        tc_fence_before();
+        mbar_arrive(tempty_bar(b));
+        if (!rows_warp) continue;
+        __threadfence();
+        __syncwarp();
+        int last = 0;
+        if (lane == 0) {
+          int* ctr = (d.phase == 0 ? dy.done1 : dy.done2) + d.unit * NRW + quad;
+          last = atomicAdd(ctr, 1) == nch - 1;
+        }
+        last = __shfl_sync(0xffffffffu, last, 0);
+        if (!last) continue;
+        // the unit's last chunk: add the partials in chunk order and finish the rows
+        __threadfence();
+        if (row_ok) {
+          constexpr int NC1 = BN / 2;
+          const int NC = d.phase == 0 ? NC1 : BN;
+#pragma unroll 1
+          for (int cc = 0; cc < NC; cc += 32) {
+            float gsum[32], usum[32];
+#pragma unroll
+            for (int k2 = 0; k2 < 32; ++k2) gsum[k2] = usum[k2] = 0.f;
+            for (int jj = 0; jj < nch; ++jj) {
+              const float* src = part + (size_t)jj * PARTF + (size_t)r_local * 256;
+#pragma unroll
+              for (int k4 = 0; k4 < 8; ++k4) {
+                const float4 a4 = __ldcg(reinterpret_cast<const float4*>(src + cc) + k4);
+                gsum[4 * k4] += a4.x;
+                gsum[4 * k4 + 1] += a4.y;
+                gsum[4 * k4 + 2] += a4.z;
+                gsum[4 * k4 + 3] += a4.w;
+                if (d.phase == 0) {
+                  const float4 bq = __ldcg(reinterpret_cast<const float4*>(src + NC1 + cc) + k4);
+                  usum[4 * k4] += bq.x;
+                  usum[4 * k4 + 1] += bq.y;
+                  usum[4 * k4 + 2] += bq.z;
+                  usum[4 * k4 + 3] += bq.w;
+                }
+              }
+            }
+            if (d.phase == 0)
+              pg_store32<EPI_GEGLU, NSLAB>(g.out, g.ldo, row0 + r_local, n0, cc, g.N_total, gsum,
+                                           usum);
+            else
+              pg_store32<EPI_STORE, NSLAB>(g.out, g.ldo, row0 + r_local, n0, cc, g.N_total, gsum,
+                                           usum);
+          }
         }
       }
-      if (d.phase == 0) {
-        // publish the tile's h rows of this unit to the GEMM-2 TMA loads
+      if (d.phase == 0 && rows_warp) {
+        // publish this warp's h rows of the unit to the GEMM-2 TMA loads
         fence_proxy_async_global();
         __threadfence();
         __syncwarp();
@@ -384,7 +430,7 @@ __global__ void __launch_bounds__(PG_MAX_THREADS, 1)
     }
   } else {
     // -------------------------------------------------------------- A-row gather (warps 6-7)
-    // GEMM-1 chunks: the <= 8 rows of the tile, 16-byte cp.async into the 128-byte-swizzled
+    // GEMM-1 chunks: the <= R rows of the tile, 16-byte cp.async into the 128-byte-swizzled
     // slot (chunk c of row r at byte 128 r + 16 (c ^ r)).  GEMM-2 chunks: nothing (the TMA
     // thread arrives in their place), but the stage count must follow.
     const int gw = warp - 6, sub = lane >> 3, ch = lane & 7;
@@ -406,16 +452,17 @@ __global__ void __launch_bounds__(PG_MAX_THREADS, 1)
       }
       int e, row0, rows, n0;
       pg_tile_info<EPI_GEGLU, NSLAB>(tiles, g1.n_blocks, d.unit, e, row0, rows, n0);
-      if (rows > DY_ROWS) {   // never launched so; stay inside the slot
+      if (rows > R) {   // never launched so; stay inside the slot
         raise_error(MOE_DEVERR_BAD_INDEX);
-        rows = DY_ROWS;
+        rows = R;
       }
-      // warp 6 lanes cover rows 0..3 and 4..7 (two instructions); warp 7 has none
-      const __nv_bfloat16* src[2];
-      uint32_t doff[2];
+      // warp 6 copies rows 0 .. R/2-1, warp 7 rows R/2 .. R-1, four rows per instruction
+      constexpr int NI = R / 8;
+      const __nv_bfloat16* src[NI];
+      uint32_t doff[NI];
 #pragma unroll
-      for (int u = 0; u < 2; ++u) {
-        const int r = gw * 64 + 4 * u + sub;
+      for (int u = 0; u < NI; ++u) {
+        const int r = gw * (R / 2) + 4 * u + sub;
         src[u] = nullptr;
         if (r < rows) {
           const int t = __ldg(tiles.perm + row0 + r) / tiles.k;
@@ -438,7 +485,7 @@ __global__ void __launch_bounds__(PG_MAX_THREADS, 1)
         }
         const uint32_t sA = base + s * STAGE_BYTES;
 #pragma unroll
-        for (int u = 0; u < 2; ++u)
+        for (int u = 0; u < NI; ++u)
           if (src[u] != nullptr) cp_async_16(sA + doff[u], src[u] + kc * GM_BK);
         cp_async_arrive_noinc(full_bar(s));
       }

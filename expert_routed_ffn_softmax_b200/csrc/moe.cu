@@ -78,6 +78,13 @@ bool use_fused_ffn(int T, int k, unsigned flags) {
   return (long long)T * k <= kFusedFfnMaxPairs;
 }
 
+// The dynamically scheduled expert FFN takes batches of at most 64 tokens (A slots of
+// R = 8, 16, 32 or 64 rows) unless a flag asks for another form; 0 = not used.
+int dy_rows(int T, unsigned flags) {
+  if (flags & (MOE_FLAG_FUSED_FFN | MOE_FLAG_UNFUSED_FFN | MOE_FLAG_DECODE_TILES)) return 0;
+  return T <= 8 ? 8 : T <= 16 ? 16 : T <= 32 ? 32 : T <= 64 ? 64 : 0;
+}
+
 // Batches of at most 16 tokens (so at most 16 rows per expert) use the decode GEMMs.
 constexpr int kDecodeMaxTokens = 16;
 bool decode_gemm_ok(int T, int H, int I) {
@@ -187,16 +194,17 @@ Layout make_layout(int T, int H, int E, int I, int k, unsigned flags, bool forwa
     L.partials = take(sizeof(float) * 2 * (size_t)kMaxGemmCtas * GM_BM * 256);
     L.partials2 = take(sizeof(float) * 2 * (size_t)kMaxGemmCtas * GM_BM * 256);
     L.n_counters = 2 * kStreamKCounters + L.max_tiles + 1;
-    if (T <= PG_SMALL_ROWS) {
-      // dynamic small-batch FFN: per-chunk partial tiles and per-unit chunk counts (+ the
-      // chunk counter).  A tile has >= 1 pair, so at most min(max_tiles, P) tiles.
+    if (const int R = dy_rows(T, flags); R > 0) {
+      // dynamic small-batch FFN: per-chunk partial tiles and per-(unit, row warp) chunk
+      // counts (+ the chunk counter).  A tile has >= 1 pair: at most min(max_tiles, P).
       const int mt = (int)std::min<long long>(L.max_tiles, P);
+      const int nrw = (R + 31) / 32;
       L.dy_u1 = mt * ((I + 127) / 128);
       L.dy_u2 = mt * ((H + 255) / 256);
-      L.dy_part1 = take(sizeof(float) * (size_t)L.dy_u1 * DY_CH1 * DY_PART_FLOATS);
-      L.dy_part2 = take(sizeof(float) * (size_t)L.dy_u2 * DY_CH2 * DY_PART_FLOATS);
+      if (DY_CH1 > 1) L.dy_part1 = take(sizeof(float) * (size_t)L.dy_u1 * DY_CH1 * R * 256);
+      if (DY_CH2 > 1) L.dy_part2 = take(sizeof(float) * (size_t)L.dy_u2 * DY_CH2 * R * 256);
       L.dy_ctr = L.n_counters;
-      L.n_counters += 1 + L.dy_u1 + L.dy_u2;
+      L.n_counters += 1 + (L.dy_u1 + L.dy_u2) * nrw;
     }
     L.counters = take(sizeof(int32_t) * L.n_counters);
   }
@@ -309,8 +317,18 @@ DeviceState* device_state(int* dev_out) {
             cudaSuccess ||
         cudaFuncSetAttribute(GEMM_FFN, cudaFuncAttributeMaxDynamicSharedMemorySize, gs) !=
             cudaSuccess ||
-        cudaFuncSetAttribute(expert_ffn_dynamic_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             dy_smem_bytes()) != cudaSuccess ||
+        cudaFuncSetAttribute(expert_ffn_dynamic_kernel<8>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, dy_smem_bytes<8>()) !=
+            cudaSuccess ||
+        cudaFuncSetAttribute(expert_ffn_dynamic_kernel<16>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, dy_smem_bytes<16>()) !=
+            cudaSuccess ||
+        cudaFuncSetAttribute(expert_ffn_dynamic_kernel<32>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, dy_smem_bytes<32>()) !=
+            cudaSuccess ||
+        cudaFuncSetAttribute(expert_ffn_dynamic_kernel<64>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, dy_smem_bytes<64>()) !=
+            cudaSuccess ||
         cudaFuncSetAttribute(GEMM_FFN_SMALL, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              pgemm_smem_bytes<kSmallStages, 4, true>()) != cudaSuccess ||
         cudaFuncSetAttribute(GEMM_STORE, cudaFuncAttributeMaxDynamicSharedMemorySize, gs) !=
@@ -677,16 +695,23 @@ moe_status_t moe_forward(const void* x, const void* w_router, const float* route
       if (const moe_status_t ls = launched(); ls != MOE_OK) return ls;
       launch(true, GEMM_STORE, dim3(G), dim3(pgemm_threads(false)), smem, tm_h, tm_wd, tm_wd,
              tm_h, tm_wd, tl, g2, g2, h_ready);
-    } else if (T <= PG_SMALL_ROWS && !(flags & MOE_FLAG_FUSED_FFN)) {
-      // at most 8 rows per tile, work handed out dynamically in k-chunks
-      CUtensorMap tm_h8;
-      if (!make_map_2d(&tm_h8, hbuf, I, P, PG_SMALL_ROWS, 64)) return cuda_failed(-1);
+    } else if (const int R = dy_rows(T, flags); R > 0) {
+      // at most R rows per tile, work handed out dynamically in k-chunks
+      CUtensorMap tm_hr;
+      if (!make_map_2d(&tm_hr, hbuf, I, P, R, 64)) return cuda_failed(-1);
       int32_t* dctr = gemm_counters + L.dy_ctr;
-      const DyState dys{dctr, dctr + 1, dctr + 1 + L.dy_u1,
+      const int nrw = (R + 31) / 32;
+      const DyState dys{dctr, dctr + 1, dctr + 1 + L.dy_u1 * nrw,
                         reinterpret_cast<float*>(ws + L.dy_part1),
                         reinterpret_cast<float*>(ws + L.dy_part2)};
-      launch(true, expert_ffn_dynamic_kernel, dim3(G), dim3(pgemm_threads(true)), dy_smem_bytes(),
-             tm_wg, tm_wu, tm_h8, tm_wd, tl, g1, g2, h_ready, dys);
+      auto go = [&](auto kernel, int smem) {
+        launch(true, kernel, dim3(G), dim3(pgemm_threads(true)), smem, tm_wg, tm_wu, tm_hr, tm_wd,
+               tl, g1, g2, h_ready, dys);
+      };
+      if (R == 8) go(expert_ffn_dynamic_kernel<8>, dy_smem_bytes<8>());
+      else if (R == 16) go(expert_ffn_dynamic_kernel<16>, dy_smem_bytes<16>());
+      else if (R == 32) go(expert_ffn_dynamic_kernel<32>, dy_smem_bytes<32>());
+      else go(expert_ffn_dynamic_kernel<64>, dy_smem_bytes<64>());
     } else if (T <= PG_SMALL_ROWS) {
       // every tile has at most T <= 8 rows: 8-row A slots (and an 8-row box over h)
       CUtensorMap tm_h8;

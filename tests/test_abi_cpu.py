@@ -52,8 +52,12 @@ def test_workspace_sizes(lib):
     # Hbuf + O dominate: 2 bytes x pairs x (H + I); GEMM-1 gathers its rows straight from x
     assert big >= 2 * 2048 * 8 * (2816 + 704)
     # decode tiles (at most 16 tokens) also keep a gathered copy Xp of the routed rows
+    # (compared with the static single launch, which keeps no chunk partials)
     dec = lib.moe_workspace_size(8, 2816, 128, 704, 8, 1 << 4)
-    assert dec >= small + 2 * 8 * 8 * 2816
+    static = lib.moe_workspace_size(8, 2816, 128, 704, 8, 1 << 7)
+    assert dec >= static + 2 * 8 * 8 * 2816
+    # the dynamically scheduled FFN (T <= 64) keeps fp32 chunk partials of its tiles
+    assert small > static
     assert lib.moe_workspace_size(8, 2816, 128, 700, 8, 0) == 0     # I % 64 != 0
     assert lib.moe_workspace_size(8, 2800, 128, 704, 8, 0) == 0     # H % 64 != 0
     assert lib.moe_workspace_size(8, 2816, 128, 704, 9, 0) == 0     # k > 8
