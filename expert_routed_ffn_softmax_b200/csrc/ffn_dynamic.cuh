@@ -23,7 +23,7 @@
 namespace moe {
 
 constexpr int DY_RING = 8;                           // chunk descriptors in flight per CTA
-constexpr int DY_CH1 = 2;                            // chunks per GEMM-1 unit
+constexpr int DY_CH1 = 1;                            // chunks per GEMM-1 unit
 constexpr int DY_CH2 = 1;                            // chunks per GEMM-2 unit
 
 // R = rows of a tile's A slot (a batch of T <= R tokens has at most T rows per tile):
