@@ -35,7 +35,6 @@ METRIC = "MoE-layer tokens/s; HBM GB/s (decode) & BF16 TFLOP/s (prefill) vs peak
 UNIT = "tokens/s"
 PER_EXPERT_BYTES = 11_894_784   # 3 * 2816 * 704 * 2: weights one active expert reads
 L2_FLUSH_BYTES = 256 << 20
-FUSED_FFN_MAX_PAIRS = 1024   # the library runs GEMM-1 and GEMM-2 as one launch up to T*k = 1024
 
 
 def peaks() -> dict:
@@ -131,6 +130,19 @@ def algorithmic(cfg: wl.MoEConfig, counts: np.ndarray, has_bias: bool) -> dict:
         "gemm2_bytes": active * cfg.H * cfg.I * 2,
         "gemm2_flops": P * 2 * cfg.I * cfg.H,
     }
+
+
+def ffn_kernel_name(T: int, tiles: str) -> str:
+    """The expert-FFN kernel(s) the library launches for T tokens and a tile family."""
+    if tiles == "decode":
+        return "grouped_gemm_decode_kernel<EPI_GEGLU>+<EPI_STORE>"
+    if tiles == "unfused":
+        return "grouped_gemm_persistent_kernel<4,EPI_GEGLU,4,1,0>+<4,EPI_STORE,4,0,0>"
+    if tiles == "fused":
+        return ("grouped_gemm_persistent_kernel<6,EPI_GEGLU,4,1,1,1>" if T <= 8
+                else "grouped_gemm_persistent_kernel<4,EPI_GEGLU,4,1,1>")
+    rows = next(r for r in (8, 16, 32, 64, 128) if T <= r or r == 128)
+    return f"expert_ffn_dynamic_kernel<{rows}>"
 
 
 def kernel_source_sha() -> str:
@@ -336,13 +348,7 @@ def run_native(args, cfg) -> None:
         kb = acc["gemm1_bytes"] + acc["gemm2_bytes"]
         kf = acc["gemm1_flops"] + acc["gemm2_flops"]
         ridge = pk["bf16_tflops"] * 1e12 / (pk["hbm_gbs"] * 1e9)
-        fused = args.tiles == "fused" or (args.tiles in ("auto", "prefill")
-                                          and cfg.T * cfg.k <= FUSED_FFN_MAX_PAIRS)
-        kname = ("grouped_gemm_decode_kernel<EPI_GEGLU>+<EPI_STORE>" if args.tiles == "decode"
-                 else "expert_ffn_dynamic_kernel" if cfg.T <= 8 and args.tiles in ("auto", "prefill")
-                 else "grouped_gemm_persistent_kernel<6,EPI_GEGLU,4,1,1,1>" if fused and cfg.T <= 8
-                 else "grouped_gemm_persistent_kernel<4,EPI_GEGLU,4,1,1>" if fused
-                 else "grouped_gemm_persistent_kernel<4,EPI_GEGLU,4,1,0>+<4,EPI_STORE,4,0,0>")
+        kname = ffn_kernel_name(cfg.T, args.tiles)
         traffic = ncu_traffic(kname, cfg.name)
         if kf / kb < ridge:
             achieved = kb / (dom_ms * 1e-3) / 1e9

@@ -26,15 +26,16 @@ constexpr int DY_RING = 8;                           // chunk descriptors in fli
 constexpr int DY_CH1 = 1;                            // chunks per GEMM-1 unit
 constexpr int DY_CH2 = 1;                            // chunks per GEMM-2 unit
 
-// R = rows of a tile's A slot (a batch of T <= R tokens has at most T rows per tile):
-// 8, 16, 32 or 64.  The MMA still reads 128 rows of A; rows past R read the stage's weight
-// bytes, which follow the slot, and their accumulator rows are never stored.
+// R = rows of a tile's A slot: 8, 16, 32 or 64 for batches of T <= R tokens (at most T
+// rows per tile), 128 for any batch (tiles are at most 128 rows).  The MMA reads 128 rows
+// of A; rows past R read the stage's weight bytes, which follow the slot, and their
+// accumulator rows are never stored.
 template <int R>
 struct DyShape {
-  static_assert(R == 8 || R == 16 || R == 32 || R == 64, "A slot rows");
+  static_assert(R == 8 || R == 16 || R == 32 || R == 64 || R == 128, "A slot rows");
   static constexpr int A_BYTES = R * GM_BK * 2;
   static constexpr int STAGE_BYTES = A_BYTES + 4 * GM_SLAB_BYTES;
-  static constexpr int STAGES = R <= 32 ? 6 : 5;
+  static constexpr int STAGES = R <= 32 ? 6 : R == 64 ? 5 : 4;
   static constexpr int ROW_WARPS = (R + 31) / 32;    // epilogue warps holding rows
   static constexpr int PART_FLOATS = R * 256;        // one chunk's partial tile
   static constexpr int SMEM = 1024 + STAGES * STAGE_BYTES + 2048;

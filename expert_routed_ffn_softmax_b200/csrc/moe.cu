@@ -69,20 +69,12 @@ bool router_uses_screen(int T, int E, unsigned flags) {
   return T >= kScreenMinTokens;
 }
 
-// GEMM-1 and GEMM-2 in one launch for small batches (measured on B200: one kernel ramp less
-// pays at T*k <= 512; from T*k = 4096 up two launches were faster).
-constexpr long long kFusedFfnMaxPairs = 1024;
-bool use_fused_ffn(int T, int k, unsigned flags) {
-  if (flags & MOE_FLAG_FUSED_FFN) return true;
-  if (flags & MOE_FLAG_UNFUSED_FFN) return false;
-  return (long long)T * k <= kFusedFfnMaxPairs;
-}
-
-// The dynamically scheduled expert FFN takes batches of at most 64 tokens (A slots of
-// R = 8, 16, 32 or 64 rows) unless a flag asks for another form; 0 = not used.
+// The dynamically scheduled expert FFN unless a flag asks for another form (0 = not used).
+// Its A slot holds R = 8, 16, 32, 64 or 128 rows: a tile never has more rows than T.
+// Measured on B200 it beat the static schedules at every T from 1 to 32768.
 int dy_rows(int T, unsigned flags) {
   if (flags & (MOE_FLAG_FUSED_FFN | MOE_FLAG_UNFUSED_FFN | MOE_FLAG_DECODE_TILES)) return 0;
-  return T <= 8 ? 8 : T <= 16 ? 16 : T <= 32 ? 32 : T <= 64 ? 64 : 0;
+  return T <= 8 ? 8 : T <= 16 ? 16 : T <= 32 ? 32 : T <= 64 ? 64 : 128;
 }
 
 // Batches of at most 16 tokens (so at most 16 rows per expert) use the decode GEMMs.
@@ -188,15 +180,19 @@ Layout make_layout(int T, int H, int E, int I, int k, unsigned flags, bool forwa
     if (L.bm == DG_BN) L.xp = take(2 * P * H);
     L.hbuf = take(2 * P * I);
     L.obuf = take(2 * P * H);
-    // stream-K split tiles of the persistent GEMMs: two fp32 tile slots per CTA and
-    // per-(split unit, row quadrant) counters, one set per GEMM (the fused launch runs both
-    // at once); then one h-ready counter per tile for the fused launch
-    L.partials = take(sizeof(float) * 2 * (size_t)kMaxGemmCtas * GM_BM * 256);
-    L.partials2 = take(sizeof(float) * 2 * (size_t)kMaxGemmCtas * GM_BM * 256);
+    // stream-K split tiles of the statically scheduled GEMMs: two fp32 tile slots per CTA
+    // and per-(split unit, row quadrant) counters, one set per GEMM (the fused launch runs
+    // both at once); then one h-ready counter per tile for the single-launch forms
+    const int R = dy_rows(T, flags);
+    if (R == 0) {
+      L.partials = take(sizeof(float) * 2 * (size_t)kMaxGemmCtas * GM_BM * 256);
+      L.partials2 = take(sizeof(float) * 2 * (size_t)kMaxGemmCtas * GM_BM * 256);
+    }
     L.n_counters = 2 * kStreamKCounters + L.max_tiles + 1;
-    if (const int R = dy_rows(T, flags); R > 0) {
-      // dynamic small-batch FFN: per-chunk partial tiles and per-(unit, row warp) chunk
-      // counts (+ the chunk counter).  A tile has >= 1 pair: at most min(max_tiles, P).
+    if (R > 0) {
+      // dynamic FFN: the unit counter, and per-chunk partial tiles and per-(unit, row warp)
+      // chunk counts when units are cut in chunks.  A tile has >= 1 pair: at most
+      // min(max_tiles, P) tiles.
       const int mt = (int)std::min<long long>(L.max_tiles, P);
       const int nrw = (R + 31) / 32;
       L.dy_u1 = mt * ((I + 127) / 128);
@@ -204,7 +200,8 @@ Layout make_layout(int T, int H, int E, int I, int k, unsigned flags, bool forwa
       if (DY_CH1 > 1) L.dy_part1 = take(sizeof(float) * (size_t)L.dy_u1 * DY_CH1 * R * 256);
       if (DY_CH2 > 1) L.dy_part2 = take(sizeof(float) * (size_t)L.dy_u2 * DY_CH2 * R * 256);
       L.dy_ctr = L.n_counters;
-      L.n_counters += 1 + (L.dy_u1 + L.dy_u2) * nrw;
+      // per-(unit, row warp) chunk counts only when units are cut in several chunks
+      L.n_counters += 1 + (DY_CH1 > 1 ? L.dy_u1 * nrw : 0) + (DY_CH2 > 1 ? L.dy_u2 * nrw : 0);
     }
     L.counters = take(sizeof(int32_t) * L.n_counters);
   }
@@ -328,6 +325,9 @@ DeviceState* device_state(int* dev_out) {
             cudaSuccess ||
         cudaFuncSetAttribute(expert_ffn_dynamic_kernel<64>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, dy_smem_bytes<64>()) !=
+            cudaSuccess ||
+        cudaFuncSetAttribute(expert_ffn_dynamic_kernel<128>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, dy_smem_bytes<128>()) !=
             cudaSuccess ||
         cudaFuncSetAttribute(GEMM_FFN_SMALL, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              pgemm_smem_bytes<kSmallStages, 4, true>()) != cudaSuccess ||
@@ -689,19 +689,13 @@ moe_status_t moe_forward(const void* x, const void* w_router, const float* route
     const int smem = pgemm_smem_bytes<kGemmStages, 4>();
     const PGemm g1{(I + 127) / 128, H, I, hbuf, I, partials, ctr1};
     const PGemm g2{(H + 255) / 256, I, H, obuf, H, partials2, ctr2};
-    if (!use_fused_ffn(T, k, flags)) {
-      launch(true, GEMM_GEGLU, dim3(G), dim3(pgemm_threads(true)), smem, tm_xp, tm_wg, tm_wu,
-             tm_xp, tm_wg, tl, g1, g1, h_ready);
-      if (const moe_status_t ls = launched(); ls != MOE_OK) return ls;
-      launch(true, GEMM_STORE, dim3(G), dim3(pgemm_threads(false)), smem, tm_h, tm_wd, tm_wd,
-             tm_h, tm_wd, tl, g2, g2, h_ready);
-    } else if (const int R = dy_rows(T, flags); R > 0) {
-      // at most R rows per tile, work handed out dynamically in k-chunks
+    if (const int R = dy_rows(T, flags); R > 0) {
+      // at most R rows per tile, whole units handed out from a shared counter
       CUtensorMap tm_hr;
       if (!make_map_2d(&tm_hr, hbuf, I, P, R, 64)) return cuda_failed(-1);
       int32_t* dctr = gemm_counters + L.dy_ctr;
       const int nrw = (R + 31) / 32;
-      const DyState dys{dctr, dctr + 1, dctr + 1 + L.dy_u1 * nrw,
+      const DyState dys{dctr, dctr + 1, dctr + 1 + (DY_CH1 > 1 ? L.dy_u1 * nrw : 0),
                         reinterpret_cast<float*>(ws + L.dy_part1),
                         reinterpret_cast<float*>(ws + L.dy_part2)};
       auto go = [&](auto kernel, int smem) {
@@ -711,9 +705,17 @@ moe_status_t moe_forward(const void* x, const void* w_router, const float* route
       if (R == 8) go(expert_ffn_dynamic_kernel<8>, dy_smem_bytes<8>());
       else if (R == 16) go(expert_ffn_dynamic_kernel<16>, dy_smem_bytes<16>());
       else if (R == 32) go(expert_ffn_dynamic_kernel<32>, dy_smem_bytes<32>());
-      else go(expert_ffn_dynamic_kernel<64>, dy_smem_bytes<64>());
+      else if (R == 64) go(expert_ffn_dynamic_kernel<64>, dy_smem_bytes<64>());
+      else go(expert_ffn_dynamic_kernel<128>, dy_smem_bytes<128>());
+    } else if (flags & MOE_FLAG_UNFUSED_FFN) {
+      // static stream-K schedule, GEMM-1 (+GEGLU) and GEMM-2 as two launches
+      launch(true, GEMM_GEGLU, dim3(G), dim3(pgemm_threads(true)), smem, tm_xp, tm_wg, tm_wu,
+             tm_xp, tm_wg, tl, g1, g1, h_ready);
+      if (const moe_status_t ls = launched(); ls != MOE_OK) return ls;
+      launch(true, GEMM_STORE, dim3(G), dim3(pgemm_threads(false)), smem, tm_h, tm_wd, tm_wd,
+             tm_h, tm_wd, tl, g2, g2, h_ready);
     } else if (T <= PG_SMALL_ROWS) {
-      // every tile has at most T <= 8 rows: 8-row A slots (and an 8-row box over h)
+      // static schedule in one launch; every tile has at most T <= 8 rows: 8-row A slots (and an 8-row box over h)
       CUtensorMap tm_h8;
       if (!make_map_2d(&tm_h8, hbuf, I, P, PG_SMALL_ROWS, 64)) return cuda_failed(-1);
       launch(true, GEMM_FFN_SMALL, dim3(G), dim3(pgemm_threads(true)),

@@ -72,14 +72,14 @@ enum {
    * MOE_ERR_INVALID_ARG. */
   MOE_FLAG_DECODE_TILES = 1u << 4,
   MOE_FLAG_PREFILL_TILES = 1u << 5,
-  /* Prefill tiles run GEMM-1 (+GEGLU) and GEMM-2 as one persistent launch for T*k <= 1024
-   * (a CTA moves on to GEMM-2 tiles as soon as the GEMM-1 tiles they read are stored) and
-   * as two launches above.  For T <= 8 the default single launch hands its work out
-   * dynamically (CTAs take k-chunks from a shared counter); its GEMM-1 sums are split in
-   * two chunks, so its bytes can differ from the other forms in the last bit of a few
-   * elements (it is deterministic).  MOE_FLAG_FUSED_FFN forces the single launch with a
-   * static schedule, MOE_FLAG_UNFUSED_FFN two launches; these two give the same bytes.
-   * Setting both is MOE_ERR_INVALID_ARG. */
+  /* Prefill tiles run GEMM-1 (+GEGLU) and GEMM-2 as one persistent launch that hands its
+   * work out dynamically: CTAs take whole (row tile, column block) units of GEMM-1, then of
+   * GEMM-2, from a shared counter, and a GEMM-2 unit starts as soon as the GEMM-1 tiles it
+   * reads are stored.  Every output tile is summed over its full K in one accumulator.
+   * MOE_FLAG_FUSED_FFN forces one launch with a static stream-K schedule, and
+   * MOE_FLAG_UNFUSED_FFN two launches with that schedule; these two give the same bytes, but
+   * stream-K splits the sums of some tiles across CTAs, so their bytes can differ from the
+   * default's in the last bit of a few elements.  Setting both is MOE_ERR_INVALID_ARG. */
   MOE_FLAG_UNFUSED_FFN = 1u << 6,
   MOE_FLAG_FUSED_FFN = 1u << 7
 };

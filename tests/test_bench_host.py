@@ -64,3 +64,15 @@ def test_reference_arm_json_line():
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["d2h_bytes_per_step"] == 0
     assert d["metric"] == json.load(open(os.path.join(ROOT, "BASELINE.json")))["metric"]
+
+
+def test_ffn_kernel_name_follows_the_library_rule():
+    # the default form is the dynamic FFN with an A slot of the smallest of 8..128 rows >= T
+    assert bench.ffn_kernel_name(1, "auto") == "expert_ffn_dynamic_kernel<8>"
+    assert bench.ffn_kernel_name(9, "auto") == "expert_ffn_dynamic_kernel<16>"
+    assert bench.ffn_kernel_name(64, "prefill") == "expert_ffn_dynamic_kernel<64>"
+    assert bench.ffn_kernel_name(65, "auto") == "expert_ffn_dynamic_kernel<128>"
+    assert bench.ffn_kernel_name(32768, "auto") == "expert_ffn_dynamic_kernel<128>"
+    assert "+" in bench.ffn_kernel_name(4096, "unfused")          # two launches
+    assert bench.ffn_kernel_name(8, "fused").endswith(",1>")       # 8-row A slots
+    assert bench.ffn_kernel_name(8, "decode").startswith("grouped_gemm_decode_kernel")

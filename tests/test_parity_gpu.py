@@ -217,8 +217,9 @@ def test_graph_replay_matches_direct_call(gemma_w):
     (8, "auto", 3),        # decode front end (router + dispatch), expert FFN, combine
     (8, "unfused", 4),     # ... with GEMM-1 and GEMM-2 as two launches
     (64, "auto", 5),       # fp64 router 2, single-CTA dispatch, expert FFN, combine
-    (4096, "auto", 10),    # screen router 4, dispatch 3, GEMM-1, GEMM-2, combine
-    (4096, "fused", 9),    # ... with GEMM-1 and GEMM-2 in one launch
+    (4096, "auto", 9),     # screen router 4, dispatch 3, expert FFN, combine
+    (4096, "unfused", 10), # ... with GEMM-1 and GEMM-2 as two launches
+    (4096, "fused", 9),    # ... static stream-K schedule in one launch
 ])
 def test_kernel_count_per_forward(T, tiles, expected, gemma_w):
     x, c, g = layer_inputs(wl.CONFIGS["decode"], gemma_w, T=T)
