@@ -199,7 +199,7 @@ def forward(x: torch.Tensor, w_router: torch.Tensor, w_gate: torch.Tensor, w_up:
             "perm": torch.empty(T * k, dtype=torch.int32, device=dev),
             "topk_ids": torch.empty((T, k), dtype=torch.int32, device=dev),
             "topk_weights": torch.empty((T, k), dtype=torch.float32, device=dev),
-            "router_stats": torch.zeros(4, dtype=torch.int32, device=dev),
+            "router_stats": torch.zeros(5, dtype=torch.int32, device=dev),
         }
         a = AuxOut(*(aux_d[n].data_ptr() for n, _ in AuxOut._fields_))
     nbytes = workspace_bytes(T, H, E, I, k, flags)
@@ -217,7 +217,7 @@ def router_stats(aux: dict) -> dict:
     u = [x & 0xFFFFFFFF for x in v]
     return {"candidates": u[0], "exact_recomputes": u[1],
             "max_screen_err_ratio": struct.unpack("<f", struct.pack("<I", u[2]))[0],
-            "path": "screen" if u[3] == 1 else "fp64"}
+            "path": "screen" if u[3] == 1 else "fp64", "fp64_rechecks": u[4]}
 
 
 def workspace_bytes(T: int, H: int, E: int, I: int, k: int, flags: int = 0) -> int:

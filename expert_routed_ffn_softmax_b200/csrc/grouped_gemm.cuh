@@ -134,7 +134,11 @@ __global__ void __launch_bounds__(128, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const int nk = K / GM_BK;
+  // K may be split over gridDim.y CTAs (EPI_F32 only): this CTA sums k-blocks [kb0, kb1)
+  // and stores its partial tile in slice blockIdx.y of the output
+  const int nk_all = K / GM_BK;
+  const int kb0 = (int)((long long)nk_all * blockIdx.y / gridDim.y);
+  const int nk = (int)((long long)nk_all * (blockIdx.y + 1) / gridDim.y) - kb0;
 
   if (warp == 0 && lane == 0) {
     // ---------------------------------------------------------------- TMA producer
@@ -149,18 +153,19 @@ __global__ void __launch_bounds__(128, 1)
       const uint32_t sA = base + s * STAGE_BYTES;
       const uint32_t sB = sA + GM_A_BYTES;
       mbar_arrive_expect_tx(full_bar(s), STAGE_BYTES);
-      tma_load_2d(sA, &tmA, full_bar(s), kc * GM_BK, row0);
+      const int kx = (kb0 + kc) * GM_BK;
+      tma_load_2d(sA, &tmA, full_bar(s), kx, row0);
       if (MODE == EPI_GEGLU) {
 #pragma unroll
         for (int j = 0; j < NSLAB / 2; ++j) {
-          tma_load_3d(sB + j * GM_SLAB_BYTES, &tmB0, full_bar(s), n0 + 64 * j, kc * GM_BK, e);
+          tma_load_3d(sB + j * GM_SLAB_BYTES, &tmB0, full_bar(s), n0 + 64 * j, kx, e);
           tma_load_3d(sB + (NSLAB / 2 + j) * GM_SLAB_BYTES, &tmB1, full_bar(s), n0 + 64 * j,
-                      kc * GM_BK, e);
+                      kx, e);
         }
       } else {
 #pragma unroll
         for (int j = 0; j < NSLAB; ++j)
-          tma_load_3d(sB + j * GM_SLAB_BYTES, &tmB0, full_bar(s), n0 + 64 * j, kc * GM_BK, e);
+          tma_load_3d(sB + j * GM_SLAB_BYTES, &tmB0, full_bar(s), n0 + 64 * j, kx, e);
       }
       *n_issued = kc + 1;
     }
@@ -239,7 +244,8 @@ __global__ void __launch_bounds__(128, 1)
       }
     }
   } else {
-    float* orow = static_cast<float*>(out_ptr) + (size_t)(row0 + r) * ldo;
+    float* orow = static_cast<float*>(out_ptr) +
+                  ((size_t)blockIdx.y * tiles.uniform_rows + row0 + r) * ldo;
 #pragma unroll 1
     for (int c = 0; c < BN; c += 32) {
       uint32_t v[32];

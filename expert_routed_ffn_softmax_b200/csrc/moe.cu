@@ -32,6 +32,7 @@ constexpr int kStreamKCounters = 4 * 2 * kMaxGemmCtas;   // per GEMM: 4 per spli
 constexpr int kFrontSmemMax = 200 * 1024;        // decode front kernel's dynamic smem cap
 
 constexpr double kScreenC = 1.0 / 1024.0;        // screen error bound / (|x| |w|)
+constexpr int kRouterStats = 5;                  // words of moe_aux_t::router_stats
 constexpr unsigned kKnownFlags = MOE_FLAG_NO_RENORM | MOE_FLAG_ROUTER_FP64 |
                                  MOE_FLAG_ROUTER_SCREEN | MOE_FLAG_PROFILE_STAGES |
                                  MOE_FLAG_DECODE_TILES | MOE_FLAG_PREFILL_TILES |
@@ -97,6 +98,13 @@ bool use_decode_front(int T, int H, int E, unsigned flags) {
 
 size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 
+// K split of the screen GEMM: enough (row tile, K slice) CTAs to cover the SMs of a B200
+// (148), at most 8 slices and at least one 64-wide k-block per slice.
+int screen_ksplit(int T, int H) {
+  const int mt = (T + 127) / 128;
+  return std::max(1, std::min({8, 148 / std::max(1, mt), H / 64}));
+}
+
 bool shape_supported(int T, int H, int E, int I, int k, bool need_I) {
   if (T < 1 || T > 1048576) return false;
   if (H < 64 || H > 16384 || H % 64) return false;
@@ -127,7 +135,8 @@ struct Layout {
   bool screen = false;
   int ks = 0, hs = 0, nchunks = 0, max_tiles = 0, bm = 0;
   size_t part_logit = 0, part_xn2 = 0, part_wn2 = 0, stats = 0, ids = 0, wts = 0;
-  size_t scr = 0, wrT = 0, wn2 = 0;
+  size_t scr = 0, wrT = 0, wn = 0;
+  int screen_ks = 1;   // K split of the screen GEMM (partial-sum slices in scr)
   size_t chunk_counts = 0, chunk_base = 0, counts = 0, offsets = 0, perm = 0, inv = 0;
   size_t tile_num = 0, tile_expert = 0, tile_row0 = 0, tile_rows = 0;
   size_t xp = 0, hbuf = 0, obuf = 0;
@@ -147,11 +156,12 @@ Layout make_layout(int T, int H, int E, int I, int k, unsigned flags, bool forwa
   };
   const size_t P = (size_t)T * k;
   L.screen = router_uses_screen(T, E, flags);
-  L.stats = take(8 * sizeof(unsigned));   // router statistics [4], front-end counter [1]
+  L.stats = take(8 * sizeof(unsigned));   // router statistics [5]; [7] front-end counter
   if (L.screen) {
-    L.scr = take(sizeof(float) * (size_t)T * E);
+    L.screen_ks = screen_ksplit(T, H);
+    L.scr = take(sizeof(float) * (size_t)L.screen_ks * T * E);
     L.wrT = take(2 * (size_t)E * H);
-    L.wn2 = take(sizeof(double) * E);
+    L.wn = take(sizeof(double) * E);
   } else {
     L.ks = router_ksplit(T, H);
     L.hs = H / L.ks;
@@ -420,7 +430,7 @@ moe_status_t launch_router(const __nv_bfloat16* x, const __nv_bfloat16* wr, cons
                            int T, int H, int E, int k, unsigned flags, int32_t* ids, float* wts,
                            unsigned* stats, uint8_t* ws, const Layout& L, const DeviceState& d,
                            cudaStream_t st, bool pdl) {
-  MOE_TRY_CUDA(cudaMemsetAsync(stats, 0, 4 * sizeof(unsigned), st));
+  MOE_TRY_CUDA(cudaMemsetAsync(stats, 0, kRouterStats * sizeof(unsigned), st));
   const Launch launch{st, pdl};
   const double u = std::ldexp(1.0, -53);
   const double n = (double)H + 8.0;
@@ -431,26 +441,27 @@ moe_status_t launch_router(const __nv_bfloat16* x, const __nv_bfloat16* wr, cons
   if (L.screen) {
     float* scr = reinterpret_cast<float*>(ws + L.scr);
     __nv_bfloat16* wrT = reinterpret_cast<__nv_bfloat16*>(ws + L.wrT);
-    double* wn2 = reinterpret_cast<double*>(ws + L.wn2);
+    double* wn = reinterpret_cast<double*>(ws + L.wn);
     launch(false, router_transpose_kernel, dim3((H + 31) / 32, (E + 31) / 32), dim3(32, 8), 0, wr,
            H, E, wrT);
-    launch(true, router_wnorm_kernel, dim3((E + 7) / 8), dim3(256), 0, wrT, H, E, wn2);
+    launch(true, router_wnorm_kernel, dim3(E), dim3(256), 0, wrT, H, E, wn);
     CUtensorMap tm_x, tm_wr;
     if (!make_map_2d(&tm_x, x, H, T, GM_BM) || !make_map_3d(&tm_wr, wr, E, H, 1))
       return cuda_failed(-1);   // a tensor map could not be encoded
     const TileList tl{nullptr, nullptr, nullptr, nullptr, T};
     const int nb = (E + 127) / 128;
     const int mt = (T + GM_BM - 1) / GM_BM;
-    launch(true, GEMM_SCREEN, dim3(nb * mt), dim3(128), gemm_smem_bytes<kGemmStages, 2>(), tm_x,
-           tm_wr, tm_wr, tl, nb, H, E, (void*)scr, E);
+    launch(true, GEMM_SCREEN, dim3(nb * mt, L.screen_ks), dim3(128),
+           gemm_smem_bytes<kGemmStages, 2>(), tm_x, tm_wr, tm_wr, tl, nb, H, E, (void*)scr, E);
+    const long long kstride = (long long)T * E;
     if (E <= 128)
       launch(true, router_screen_select_kernel<4>, dim3(warps_blocks), dim3(32 * kScreenWarps), 0,
-             (const float*)scr, x, (const __nv_bfloat16*)wrT, (const double*)wn2, bias, T, H, E, k,
-             kScreenC, beta_scale, ids, wts, stats);
+             (const float*)scr, L.screen_ks, kstride, x, (const __nv_bfloat16*)wrT,
+             (const double*)wn, bias, T, H, E, k, kScreenC, beta_scale, ids, wts, stats);
     else
       launch(true, router_screen_select_kernel<8>, dim3(warps_blocks), dim3(32 * kScreenWarps), 0,
-             (const float*)scr, x, (const __nv_bfloat16*)wrT, (const double*)wn2, bias, T, H, E, k,
-             kScreenC, beta_scale, ids, wts, stats);
+             (const float*)scr, L.screen_ks, kstride, x, (const __nv_bfloat16*)wrT,
+             (const double*)wn, bias, T, H, E, k, kScreenC, beta_scale, ids, wts, stats);
     return launched();
   }
   double* part_logit = reinterpret_cast<double*>(ws + L.part_logit);
@@ -620,9 +631,16 @@ moe_status_t moe_forward(const void* x, const void* w_router, const float* route
   // Dependent launches, except while stage events sit between the kernels.
   const Launch launch{st, !prof.on};
   if (use_decode_front(T, H, E, flags)) {
-    // 1+2. router and dispatch in one launch: one 8-CTA cluster per token.  stats[4] is the
-    // front end's token counter (zero at launch, left zero).
-    MOE_TRY_CUDA(cudaMemsetAsync(stats, 0, 8 * sizeof(unsigned), st));
+    // 1+2. router and dispatch in one launch: one 8-CTA cluster per token.  Word 7 of the
+    // workspace statistics is the front end's token counter (zero at launch, left zero).
+    unsigned* ws_stats = reinterpret_cast<unsigned*>(ws + L.stats);
+    unsigned* front_done = ws_stats + 7;
+    if (stats == ws_stats) {
+      MOE_TRY_CUDA(cudaMemsetAsync(ws_stats, 0, 8 * sizeof(unsigned), st));
+    } else {
+      MOE_TRY_CUDA(cudaMemsetAsync(stats, 0, kRouterStats * sizeof(unsigned), st));
+      MOE_TRY_CUDA(cudaMemsetAsync(front_done, 0, sizeof(unsigned), st));
+    }
     const double u = std::ldexp(1.0, -53), n = (double)H + 8.0;
     const double beta_scale = 2.0 * (n * u / (1.0 - n * u)) * 1.01;
     launch(false, decode_front_kernel<4>, dim3(kFrontRanks * T), dim3(32 * kFrontWarps),
@@ -630,7 +648,7 @@ moe_status_t moe_forward(const void* x, const void* w_router, const float* route
            static_cast<const __nv_bfloat16*>(w_router), router_bias, T, H, E, k,
            (flags & MOE_FLAG_NO_RENORM) ? 0 : 1, beta_scale, ids, wts, stats, counts, offsets, perm,
            inv, tile_num, tile_expert, tile_row0, tile_rows, gemm_counters, L.n_counters, L.bm,
-           stats + 4);
+           front_done);
     if (dec)   // decode tiles read a gathered copy of the routed rows
       launch(true, gather_rows_kernel, dim3(std::min((P + 7) / 8, gsm)), dim3(256), 0,
              static_cast<const uint4*>(x), (const int32_t*)perm, P, k, H / 8,

@@ -479,211 +479,475 @@ __global__ void __launch_bounds__(256) router_transpose_kernel(const __nv_bfloat
   }
 }
 
-// wn2[e] = sum_h Wr[h][e]^2 in fp64 (one warp per expert, over the transposed rows).
+// wn[e] >= |W[:, e]|_2: sum_h Wr[h][e]^2 in fp64 (every square exact), one 256-thread block
+// per expert over its transposed row, lanes then warps added in a fixed order; then the
+// square root, raised by 1e-6 relative to cover its rounding and the sum's.
 __global__ void __launch_bounds__(256) router_wnorm_kernel(const __nv_bfloat16* __restrict__ wrT,
-                                                           int H, int E, double* __restrict__ wn2) {
+                                                           int H, int E, double* __restrict__ wn) {
   pdl_trigger();
   pdl_wait();
-  const int lane = threadIdx.x & 31;
-  const int e = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-  if (e >= E) return;
+  __shared__ double s_part[8];
+  const int e = blockIdx.x, lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const uint32_t* row = reinterpret_cast<const uint32_t*>(wrT + (size_t)e * H);
   double s = 0.0;
-  for (int h = lane; h < H; h += 32) {
-    const double v = (double)__bfloat162float(wrT[(size_t)e * H + h]);
-    s = fma(v, v, s);
+  for (int p = threadIdx.x; 2 * p < H; p += 256) {
+    const uint32_t w2 = __ldg(row + p);
+    const double a = (double)__uint_as_float(w2 << 16), b = (double)__uint_as_float(w2 & 0xffff0000u);
+    s = fma(b, b, fma(a, a, s));
   }
 #pragma unroll
   for (int off = 16; off; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
-  if (lane == 0) wn2[e] = s;
+  if (lane == 0) s_part[warp] = s;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    double t = 0.0;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) t += s_part[w];
+    wn[e] = sqrt(t) * (1.0 + 1e-6);
+  }
 }
 
 constexpr int kScreenWarps = 8;
 
+// Weight accuracy of the pair-sum recheck: its values are kept only when the renormalised
+// weights they give are provably within this of the weights of the fp64 logits.  With every
+// logit off by at most b, each weight w_r moves by at most w_r (e^{2b} - 1), so
+// 2 b max_r w_r bounds the difference to first order (b <= 1e-4 here, the second order is
+// below 1e-4 of it); the fp32 store adds at most 2^-24 w_r.
+constexpr double kPairWeightErr = 8e-6;
+
+// Order-preserving maps onto unsigned integers (a larger value gets a larger key).
+__device__ __forceinline__ uint32_t ord_f32(float f) {
+  const uint32_t b = __float_as_uint(f);
+  return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+__device__ __forceinline__ float unord_f32(uint32_t k) {
+  return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
+}
+// Doubles: -0 is taken as +0 and NaN maps to 1, below every number (0 marks an empty slot).
+__device__ __forceinline__ uint64_t ord_f64(double d) {
+  if (isnan(d)) return 1ull;
+  const uint64_t b = (uint64_t)__double_as_longlong(d == 0.0 ? 0.0 : d);
+  return (b >> 63) ? ~b : (b | 0x8000000000000000ull);
+}
+__device__ __forceinline__ double unord_f64(uint64_t k) {
+  return __longlong_as_double((long long)((k >> 63) ? (k & 0x7fffffffffffffffull) : ~k));
+}
+
+// x_lo w_lo + x_hi w_hi for two packed bf16 pairs with ONE fp32 rounding: bf16 x bf16 is
+// exact in fp32 (8-bit significands), so the first fused multiply-add (onto +0) is exact
+// and the second rounds once.  Error <= 2^-24 |sum| (or <= 2^-150 in the subnormal range).
+__device__ __forceinline__ float bf16_pair_dot(uint32_t xw, uint32_t ww) {
+  float d;
+  asm("{.reg .b16 xl, xh, wl, wh;\n\t.reg .f32 p;\n\t"
+      "mov.b32 {xl, xh}, %1;\n\tmov.b32 {wl, wh}, %2;\n\t"
+      "fma.rn.f32.bf16 p, xl, wl, 0f00000000;\n\t"
+      "fma.rn.f32.bf16 %0, xh, wh, p;\n\t}"
+      : "=f"(d)
+      : "r"(xw), "r"(ww));
+  return d;
+}
+
+// Dot products of one token row x with G candidate rows of W^T (wrow[u]), split over the
+// warp: lane l owns h = 256 j + 8 l + i (i < 8), read as 16-byte vectors; a fixed xor tree
+// adds the lanes in fp64.  Two precisions:
+//   PAIRS: each pair (h, h+1) summed with one fp32 rounding (bf16_pair_dot), the pair sums
+//     accumulated in fp64.  |result - sum_h x_h w_h| <= 2^-24 sum_h |x_h w_h| + H 2^-150
+//     + the fp64 accumulation's error (well inside the fp64 bound beta).
+//   !PAIRS: every value converted to fp64, fp64 fused multiply-adds (error inside beta).
+template <bool PAIRS, int G>
+__device__ __forceinline__ void screen_dot(const __nv_bfloat16* __restrict__ xr,
+                                           const uint4* (&wrow)[G], int H, double (&acc)[G]) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int u = 0; u < G; ++u) acc[u] = 0.0;
+  const uint4* xv4 = reinterpret_cast<const uint4*>(xr);
+#pragma unroll 4
+  for (int v = lane; 8 * v < H; v += 32) {   // 16-byte vector index within the row
+    const uint4 xq = __ldg(xv4 + v);
+    uint4 wq[G];
+#pragma unroll
+    for (int u = 0; u < G; ++u) wq[u] = __ldg(wrow[u] + v);
+    const uint32_t* xw = reinterpret_cast<const uint32_t*>(&xq);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+#pragma unroll
+      for (int u = 0; u < G; ++u) {
+        const uint32_t ww = reinterpret_cast<const uint32_t*>(&wq[u])[i];
+        if constexpr (PAIRS) {
+          acc[u] += (double)bf16_pair_dot(xw[i], ww);
+        } else {
+          acc[u] = fma((double)__uint_as_float(xw[i] << 16), (double)__uint_as_float(ww << 16),
+                       acc[u]);
+          acc[u] = fma((double)__uint_as_float(xw[i] & 0xffff0000u),
+                       (double)__uint_as_float(ww & 0xffff0000u), acc[u]);
+        }
+      }
+    }
+  }
+#pragma unroll
+  for (int u = 0; u < G; ++u) {
+#pragma unroll
+    for (int off = 16; off; off >>= 1) acc[u] += __shfl_xor_sync(0xffffffffu, acc[u], off);
+  }
+}
+
+// Recompute the nc candidates of this warp's token (ids in cand[]) into val[] (+ bias),
+// four rows at a time and two for a tail of at most two.
+template <bool PAIRS>
+__device__ __forceinline__ void screen_recheck(const __nv_bfloat16* __restrict__ xr,
+                                               const __nv_bfloat16* __restrict__ wrT,
+                                               const float* __restrict__ bias, int H,
+                                               const int* cand, int nc, double* val) {
+  const int lane = threadIdx.x & 31;
+  __syncwarp();   // every lane is done reading val
+  for (int c0 = 0; c0 < nc;) {
+    if (nc - c0 > 2) {
+      const uint4* wrow[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        wrow[u] = reinterpret_cast<const uint4*>(wrT + (size_t)cand[min(c0 + u, nc - 1)] * H);
+      double acc[4];
+      screen_dot<PAIRS, 4>(xr, wrow, H, acc);
+      double v = acc[0];
+#pragma unroll
+      for (int u = 1; u < 4; ++u)
+        if (lane == u) v = acc[u];
+      if (lane < 4 && c0 + lane < nc) {
+        const int e = cand[c0 + lane];
+        val[c0 + lane] = bias ? v + (double)bias[e] : v;
+      }
+      c0 += 4;
+    } else {
+      const uint4* wrow[2];
+#pragma unroll
+      for (int u = 0; u < 2; ++u)
+        wrow[u] = reinterpret_cast<const uint4*>(wrT + (size_t)cand[min(c0 + u, nc - 1)] * H);
+      double acc[2];
+      screen_dot<PAIRS, 2>(xr, wrow, H, acc);
+      const double v = lane == 1 ? acc[1] : acc[0];
+      if (lane < 2 && c0 + lane < nc) {
+        const int e = cand[c0 + lane];
+        val[c0 + lane] = bias ? v + (double)bias[e] : v;
+      }
+      c0 += 2;
+    }
+  }
+  __syncwarp();
+}
+
+// k rounds of a warp-wide argmax by (value desc, id asc) over the slots (id INT_MAX = empty;
+// at least k slots are filled).  Each round takes every lane's best free slot and reduces
+// the 64-bit value keys and then the ids with redux.sync.  On return every lane holds the
+// selected ids, values and bounds in rank order; `taken` marks the lane's selected slots.
+template <int EPL>
+__device__ __forceinline__ void warp_rank_select(const double (&V)[EPL], const double (&B)[EPL],
+                                                 const int (&id)[EPL], int k,
+                                                 bool (&taken)[EPL], int (&sel_e)[8],
+                                                 double (&sel_v)[8], double (&sel_b)[8]) {
+  uint64_t key[EPL];
+#pragma unroll
+  for (int i = 0; i < EPL; ++i) {
+    taken[i] = false;
+    key[i] = id[i] != INT_MAX ? ord_f64(V[i]) : 0ull;
+  }
+#pragma unroll
+  for (int r = 0; r < 8; ++r) {
+    sel_e[r] = INT_MAX;
+    sel_v[r] = 0.0;
+    sel_b[r] = 0.0;
+    if (r < k) {
+      uint64_t bk = 0;
+      int bid = INT_MAX;
+      double bb = 0.0;
+#pragma unroll
+      for (int i = 0; i < EPL; ++i)
+        if (!taken[i] && key[i] != 0 && (key[i] > bk || (key[i] == bk && id[i] < bid))) {
+          bk = key[i];
+          bid = id[i];
+          bb = B[i];
+        }
+      const uint32_t hi = (uint32_t)(bk >> 32), lo = (uint32_t)bk;
+      const uint32_t mhi = __reduce_max_sync(0xffffffffu, hi);
+      const uint32_t mlo = __reduce_max_sync(0xffffffffu, hi == mhi ? lo : 0u);
+      const bool top = bk != 0 && hi == mhi && lo == mlo;
+      const int wid = __reduce_min_sync(0xffffffffu, top ? bid : INT_MAX);
+      const unsigned wl = __ballot_sync(0xffffffffu, top && bid == wid);
+      sel_e[r] = wid;
+      sel_v[r] = unord_f64(((uint64_t)mhi << 32) | mlo);
+      sel_b[r] = __shfl_sync(0xffffffffu, bb, __ffs(wl) - 1);
+#pragma unroll
+      for (int i = 0; i < EPL; ++i)
+        if (id[i] == wid) taken[i] = true;
+    }
+  }
+}
+
+// Rank the candidates (slot c = lane + 32 i) by their recomputed values and check every
+// decision against B_e = beta_e + c_extra |x| |w_e| + abs_extra.  Returns true when all of
+// them hold; V, cid, taken, sel_* describe the ranking either way, b_max = max selected B.
+template <int EPL>
+__device__ __forceinline__ bool screen_rank_verify(const int* cand, const double* val, int nc,
+                                                   const double* __restrict__ wn,
+                                                   const float* __restrict__ bias, double xn,
+                                                   double beta_scale, double c_extra,
+                                                   double abs_extra, int k, double (&V)[EPL],
+                                                   int (&cid)[EPL], bool (&taken)[EPL],
+                                                   int (&sel_e)[8], double (&sel_v)[8],
+                                                   double& b_max) {
+  const int lane = threadIdx.x & 31;
+  bool ok = true;
+  double B[EPL];
+#pragma unroll
+  for (int i = 0; i < EPL; ++i) {
+    const int c = lane + 32 * i;
+    cid[i] = INT_MAX;
+    V[i] = -DBL_MAX;
+    B[i] = 0.0;
+    if (c < nc) {
+      const int e = cand[c];
+      cid[i] = e;
+      V[i] = val[c];
+      ok = ok && isfinite(V[i]);
+      const double xw = xn * wn[e];
+      B[i] = beta_scale * (xw + (bias ? fabs((double)bias[e]) : 0.0)) + c_extra * xw + abs_extra;
+    }
+  }
+  double sel_b[8];
+  warp_rank_select<EPL>(V, B, cid, k, taken, sel_e, sel_v, sel_b);
+  b_max = 0.0;
+#pragma unroll
+  for (int r = 0; r < 8; ++r)
+    if (r < k) b_max = fmax(b_max, sel_b[r]);
+  ok = ok && isfinite(b_max);
+#pragma unroll
+  for (int r = 0; r + 1 < 8; ++r)
+    if (r + 1 < k) ok = ok && (sel_v[r] - sel_v[r + 1] > sel_b[r] + sel_b[r + 1]);
+  double v_last = sel_v[0], b_last = sel_b[0];
+#pragma unroll
+  for (int r = 1; r < 8; ++r)
+    if (r == k - 1) {
+      v_last = sel_v[r];
+      b_last = sel_b[r];
+    }
+#pragma unroll
+  for (int i = 0; i < EPL; ++i)
+    if (cid[i] != INT_MAX && !taken[i]) ok = ok && (v_last - V[i] > b_last + B[i]);
+  return __all_sync(0xffffffffu, ok);
+}
+
+// Screen path, one warp per token.  screen: ks fp32 partial-sum slices of kstride floats
+// each ([T][E] per slice, added here in fp64 in slice order).
 // stats[0] += candidates, stats[1] += exact recomputations,
 // stats[2] = max over candidates of |screen - L| / (|x| |w|) (float bits, atomicMax),
-// stats[3] = 1 (the screen path).
+// stats[3] = 1 (the screen path), stats[4] += tokens recomputed in fp64 (second tier).
 template <int EPL>
-__global__ void __launch_bounds__(256, 3) router_screen_select_kernel(
-    const float* __restrict__ screen, const __nv_bfloat16* __restrict__ x,
-    const __nv_bfloat16* __restrict__ wrT, const double* __restrict__ wn2,
-    const float* __restrict__ bias, int T, int H, int E, int k, double screen_c,
-    double beta_scale, int32_t* __restrict__ ids, float* __restrict__ wts,
+__global__ void __launch_bounds__(256, 2) router_screen_select_kernel(
+    const float* __restrict__ screen, int ks, long long kstride,
+    const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __restrict__ wrT,
+    const double* __restrict__ wn, const float* __restrict__ bias, int T, int H, int E, int k,
+    double screen_c, double beta_scale, int32_t* __restrict__ ids, float* __restrict__ wts,
     unsigned* __restrict__ stats) {
   pdl_trigger();
   pdl_wait();
-  if (blockIdx.x == 0 && threadIdx.x == 0) stats[3] = 1;   // path: screen + fp64 recheck
+  if (blockIdx.x == 0 && threadIdx.x == 0) stats[3] = 1;   // path: screen + recheck
   __shared__ int s_cand[kScreenWarps][32 * EPL];
   __shared__ double s_val[kScreenWarps][32 * EPL];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const unsigned lt = (1u << lane) - 1u;
+  // bound of the pair sums: 2^-24 sum |x_h w_h| <= 2^-24 |x| |w| (+ 1%), underflow H 2^-150
+  const double pair_c = 1.01 * 0x1p-24, pair_abs = (double)H * 0x1p-149;
   // statistics are gathered per warp and published once, not per token
-  unsigned st_cand = 0, st_exact = 0;
+  unsigned st_cand = 0, st_exact = 0, st_fp64 = 0;
   float st_err = 0.f;
   for (int t = blockIdx.x * kScreenWarps + warp; t < T; t += gridDim.x * kScreenWarps) {
     const __nv_bfloat16* xr = x + (size_t)t * H;
-    double xn2 = 0.0;
-    for (int h = lane; h < H; h += 32) {
-      const double v = (double)__bfloat162float(xr[h]);
-      xn2 = fma(v, v, xn2);
+    // |x_t| bound: squares of bf16 values are exact in fp32; each lane sums its H/32 of them
+    // in fp32 (relative error < (H/32) 2^-24, + H/32 2^-150 for underflow), 16-byte loads
+    float q = 0.f;
+    {
+      const uint4* xv4 = reinterpret_cast<const uint4*>(xr);
+#pragma unroll 4
+      for (int v = lane; 8 * v < H; v += 32) {
+        const uint4 xq = __ldg(xv4 + v);
+        q += bf16_pair_dot(xq.x, xq.x) + bf16_pair_dot(xq.y, xq.y) +
+             bf16_pair_dot(xq.z, xq.z) + bf16_pair_dot(xq.w, xq.w);
+      }
     }
+    double xn2 = (double)q;
 #pragma unroll
     for (int off = 16; off; off >>= 1) xn2 += __shfl_xor_sync(0xffffffffu, xn2, off);
+    xn2 = xn2 * (1.0 + (double)(H / 32 + 2) * 0x1p-23) + (double)H * 0x1p-149;
+    if (!isfinite(xn2)) {   // fp32 overflow: the norm again in fp64
+      xn2 = 0.0;
+      for (int h = lane; h < H; h += 32) {
+        const double v = (double)__bfloat162float(xr[h]);
+        xn2 = fma(v, v, xn2);
+      }
+#pragma unroll
+      for (int off = 16; off; off >>= 1) xn2 += __shfl_xor_sync(0xffffffffu, xn2, off);
+    }
     const double xn = sqrt(xn2) * (1.0 + 1e-6);
 
+    // Screened logits S, their bounds D, and a threshold tau below the k-th largest lower
+    // bound S - D: tau = min of S - D over k experts of the largest S (any k experts give a
+    // valid tau; the largest S make it tight).  An expert with S + D < tau cannot reach the
+    // top-k, in exact arithmetic or in either fp64 summation order.
     double S[EPL], D[EPL];
-    int eid[EPL];
+    uint32_t skey[EPL];
     bool finite = true;
 #pragma unroll
     for (int i = 0; i < EPL; ++i) {
       const int e = lane + 32 * i;
-      eid[i] = e < E ? e : INT_MAX;
       S[i] = -DBL_MAX;
       D[i] = 0.0;
+      skey[i] = 0u;
       if (e < E) {
-        const double sv = (double)screen[(size_t)t * E + e];
-        const double wn = sqrt(wn2[e]) * (1.0 + 1e-6);
-        const double beta = beta_scale * (xn * wn + (bias ? fabs((double)bias[e]) : 0.0));
+        double sv = 0.0;
+        for (int z = 0; z < ks; ++z) sv += (double)screen[z * kstride + (size_t)t * E + e];
+        const double xw = xn * wn[e];
+        const double beta = beta_scale * (xw + (bias ? fabs((double)bias[e]) : 0.0));
         if (isfinite(sv)) {
           S[i] = bias ? sv + (double)bias[e] : sv;
-          D[i] = screen_c * xn * wn + 4.0 * beta;
+          D[i] = screen_c * xw + 4.0 * beta;
+          // 24 high bits of the value, then 255 - e: unique keys, larger S first
+          skey[i] = (ord_f32((float)S[i]) & 0xffffff00u) | (uint32_t)(255 - e);
         } else {
           finite = false;
         }
       }
     }
     finite = __all_sync(0xffffffffu, finite);
-    bool taken[EPL];
-    int sel_e[8];
-    double sel_v[8];
     double tau = -DBL_MAX;
     if (finite) {
-      warp_topk_ids<EPL>(S, eid, k, taken, sel_e, sel_v);
-      for (int r = 0; r < k; ++r)
-        tau = fmin(tau == -DBL_MAX ? DBL_MAX : tau, sel_v[r] - warp_value_of<EPL>(D, eid, sel_e[r]));
+      float lo_min = FLT_MAX;
+      bool chosen[EPL];
+#pragma unroll
+      for (int i = 0; i < EPL; ++i) chosen[i] = false;
+#pragma unroll
+      for (int r = 0; r < 8; ++r) {
+        if (r < k) {
+          uint32_t m = 0u;
+#pragma unroll
+          for (int i = 0; i < EPL; ++i)
+            if (!chosen[i]) m = max(m, skey[i]);
+          const uint32_t w = __reduce_max_sync(0xffffffffu, m);
+#pragma unroll
+          for (int i = 0; i < EPL; ++i)
+            if (w != 0u && skey[i] == w) chosen[i] = true;
+        }
+      }
+#pragma unroll
+      for (int i = 0; i < EPL; ++i)
+        if (chosen[i]) lo_min = fminf(lo_min, __double2float_rd(S[i] - D[i]));
+      tau = (double)unord_f32(__reduce_min_sync(0xffffffffu, ord_f32(lo_min)));
     }
     // Compact the candidates in ascending expert id.
     int nc = 0;
+    int* cand = s_cand[warp];
+    double* val = s_val[warp];
 #pragma unroll
     for (int i = 0; i < EPL; ++i) {
-      const bool c = eid[i] != INT_MAX && (!finite || S[i] + D[i] >= tau);
+      const int e = lane + 32 * i;
+      const bool c = e < E && (!finite || S[i] + D[i] >= tau);
       const unsigned m = __ballot_sync(0xffffffffu, c);
-      if (c) s_cand[warp][nc + __popc(m & lt)] = eid[i];
+      if (c) cand[nc + __popc(m & lt)] = e;
       nc += __popc(m);
     }
     __syncwarp();
 
-    // fp64 recheck of the candidates, 4 at a time.  Lane l owns h = 256 j + 8 l + i
-    // (i < 8), read as 16-byte vectors of x and of the transposed W rows; it sums its h in
-    // ascending order, then a fixed xor tree adds the lanes.
-    const int nj = (H + 255) / 256;
-    for (int c0 = 0; c0 < nc; c0 += 4) {
-      const uint4* wrow[4];
-      double acc[4] = {0.0, 0.0, 0.0, 0.0};
+    // First recheck: fp32 pair sums.  Kept when every ranking decision clears the pair-sum
+    // bound and the weights they give are within kPairWeightErr of the fp64 ones.
+    screen_recheck<true>(xr, wrT, bias, H, cand, nc, val);
+    double V[EPL];
+    int cid[EPL];
+    bool taken[EPL];
+    int sel_e[8];
+    double sel_v[8];
+    double b_max;
+    bool ok = screen_rank_verify<EPL>(cand, val, nc, wn, bias, xn, beta_scale, pair_c, pair_abs,
+                                      k, V, cid, taken, sel_e, sel_v, b_max);
+    // this lane's share of the renormalised weights: lane r < k holds exp(L_r - L_0)
+    double my_v = sel_v[0];
+    int my_e = sel_e[0];
 #pragma unroll
-      for (int u = 0; u < 4; ++u)
-        wrow[u] = reinterpret_cast<const uint4*>(wrT + (size_t)s_cand[warp][min(c0 + u, nc - 1)] * H);
-      const uint4* xv4 = reinterpret_cast<const uint4*>(xr);
-#pragma unroll 4
-      for (int jj = 0; jj < nj; ++jj) {
-        const int v = jj * 32 + lane;           // 16-byte vector index within the row
-        if (v * 8 < H) {
-          const uint4 xq = __ldg(xv4 + v);
-          uint4 wq[4];
+    for (int r = 1; r < 8; ++r)
+      if (lane == r) {
+        my_v = sel_v[r];
+        my_e = sel_e[r];
+      }
+    double ev = lane < k ? exp(my_v - sel_v[0]) : 0.0;
+    double denom = ev;
 #pragma unroll
-          for (int u = 0; u < 4; ++u) wq[u] = __ldg(wrow[u] + v);
-          const __nv_bfloat162* xp2 = reinterpret_cast<const __nv_bfloat162*>(&xq);
+    for (int off = 16; off; off >>= 1) denom += __shfl_xor_sync(0xffffffffu, denom, off);
+    ok = ok && 2.0 * b_max / denom <= kPairWeightErr;   // 1 / denom: the largest weight
+    if (!ok) {
+      // Second recheck: fp64 products and sums, checked against the fp64 bound alone.
+      ++st_fp64;
+      screen_recheck<false>(xr, wrT, bias, H, cand, nc, val);
+      ok = screen_rank_verify<EPL>(cand, val, nc, wn, bias, xn, beta_scale, 0.0, 0.0, k, V, cid,
+                                   taken, sel_e, sel_v, b_max);
+      if (!ok) {
+        // Too close to call: each lane recomputes its candidates as one FMA chain in
+        // ascending h (the definition's sequence of roundings), then the warp ranks again.
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const float2 xf = __bfloat1622float2(xp2[i]);
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-              const float2 wf = __bfloat1622float2(reinterpret_cast<const __nv_bfloat162*>(&wq[u])[i]);
-              acc[u] = fma((double)xf.x, (double)wf.x, acc[u]);
-              acc[u] = fma((double)xf.y, (double)wf.y, acc[u]);
-            }
+        for (int i = 0; i < EPL; ++i) {
+          if (cid[i] != INT_MAX) {
+            const __nv_bfloat16* wrow = wrT + (size_t)cid[i] * H;
+            double a = 0.0;
+            for (int h = 0; h < H; ++h)
+              a = fma((double)__bfloat162float(xr[h]), (double)__bfloat162float(wrow[h]), a);
+            V[i] = bias ? a + (double)bias[cid[i]] : a;
           }
         }
-      }
+        double Bz[EPL], sel_bz[8];
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-#pragma unroll
-        for (int off = 16; off; off >>= 1) acc[u] += __shfl_xor_sync(0xffffffffu, acc[u], off);
+        for (int i = 0; i < EPL; ++i) Bz[i] = 0.0;
+        warp_rank_select<EPL>(V, Bz, cid, k, taken, sel_e, sel_v, sel_bz);
+        ++st_exact;
       }
-      if (lane < 4 && c0 + lane < nc) {
-        double v = acc[0];
+      my_v = sel_v[0];
+      my_e = sel_e[0];
 #pragma unroll
-        for (int u = 1; u < 4; ++u)
-          if (lane == u) v = acc[u];
-        const int e = s_cand[warp][c0 + lane];
-        s_val[warp][c0 + lane] = bias ? v + (double)bias[e] : v;
-      }
+      for (int r = 1; r < 8; ++r)
+        if (lane == r) {
+          my_v = sel_v[r];
+          my_e = sel_e[r];
+        }
+      ev = lane < k ? exp(my_v - sel_v[0]) : 0.0;
+      denom = ev;
+#pragma unroll
+      for (int off = 16; off; off >>= 1) denom += __shfl_xor_sync(0xffffffffu, denom, off);
     }
-    __syncwarp();
-
-    // Rank the candidates (slot c = lane + 32 i) and verify every decision.
-    double V[EPL], B[EPL];
-    int cid[EPL];
+    // largest |screen - L| / (|x| |w|) over the candidates, L from the last recheck
     float err = 0.f;
-#pragma unroll
-    for (int i = 0; i < EPL; ++i) {
-      const int c = lane + 32 * i;
-      cid[i] = INT_MAX;
-      V[i] = -DBL_MAX;
-      B[i] = 0.0;
-      if (c < nc) {
-        const int e = s_cand[warp][c];
-        cid[i] = e;
-        V[i] = s_val[warp][c];
-        const double wn = sqrt(wn2[e]) * (1.0 + 1e-6);
-        B[i] = beta_scale * (xn * wn + (bias ? fabs((double)bias[e]) : 0.0));
-        const double L0 = bias ? V[i] - (double)bias[e] : V[i];
-        if (finite) err = fmaxf(err, (float)(fabs((double)screen[(size_t)t * E + e] - L0) / (xn * wn)));
-      }
-    }
-    warp_topk_ids<EPL>(V, cid, k, taken, sel_e, sel_v);
-    double sel_b[8];
-    for (int r = 0; r < k; ++r) sel_b[r] = warp_value_of<EPL>(B, cid, sel_e[r]);
-    bool ok = true;
-    for (int r = 0; r + 1 < k; ++r) ok = ok && (sel_v[r] - sel_v[r + 1] > sel_b[r] + sel_b[r + 1]);
-#pragma unroll
-    for (int i = 0; i < EPL; ++i)
-      if (cid[i] != INT_MAX && !taken[i]) ok = ok && (sel_v[k - 1] - V[i] > sel_b[k - 1] + B[i]);
-    ok = __all_sync(0xffffffffu, ok);
-    if (!ok) {
-      // Too close to call: each lane recomputes its candidates as one FMA chain in
-      // ascending h (the definition's sequence of roundings), then the warp ranks again.
+    if (finite) {
 #pragma unroll
       for (int i = 0; i < EPL; ++i) {
         if (cid[i] != INT_MAX) {
-          const __nv_bfloat16* wrow = wrT + (size_t)cid[i] * H;
-          double a = 0.0;
-          for (int h = 0; h < H; ++h)
-            a = fma((double)__bfloat162float(xr[h]), (double)__bfloat162float(wrow[h]), a);
-          V[i] = bias ? a + (double)bias[cid[i]] : a;
+          const int e = cid[i];
+          double sv = 0.0;
+          for (int z = 0; z < ks; ++z) sv += (double)screen[z * kstride + (size_t)t * E + e];
+          const double L0 = bias ? V[i] - (double)bias[e] : V[i];
+          err = fmaxf(err, (float)(fabs(sv - L0) / (xn * wn[e])));
         }
       }
-      warp_topk_ids<EPL>(V, cid, k, taken, sel_e, sel_v);
     }
-#pragma unroll
-    for (int off = 16; off; off >>= 1) err = fmaxf(err, __shfl_xor_sync(0xffffffffu, err, off));
     st_cand += (unsigned)nc;
-    st_exact += ok ? 0u : 1u;
-    st_err = fmaxf(st_err, err);
+    st_err = fmaxf(st_err, err);   // lanes differ; the block-wide max is taken below
 
-    // Renormalised weights: softmax over the k selected logits.
-    const double m = sel_v[0];
-    double denom = 0.0;
-    for (int r = 0; r < k; ++r) denom += exp(sel_v[r] - m);
-    for (int r = 0; r < k; ++r)
-      if (lane == r) {
-        ids[(size_t)t * k + r] = sel_e[r];
-        wts[(size_t)t * k + r] = (float)(exp(sel_v[r] - m) / denom);
-      }
+    // Renormalised weights: softmax over the k selected logits, lane r writes slot r.
+    if (lane < k) {
+      ids[(size_t)t * k + lane] = my_e;
+      wts[(size_t)t * k + lane] = (float)(ev / denom);
+    }
     __syncwarp();
   }
+  st_err = __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(st_err)));
   if (lane == 0 && st_cand) {
     atomicAdd(&stats[0], st_cand);
     if (st_exact) atomicAdd(&stats[1], st_exact);
+    if (st_fp64) atomicAdd(&stats[4], st_fp64);
     atomicMax(&stats[2], __float_as_uint(st_err));
   }
 }

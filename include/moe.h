@@ -39,7 +39,7 @@
 extern "C" {
 #endif
 
-#define MOE_ABI_VERSION 1
+#define MOE_ABI_VERSION 2
 
 typedef enum {
   MOE_OK = 0,
@@ -91,10 +91,12 @@ typedef struct {
   int32_t *perm;           /* [T*k]  expert-sorted position -> pair index t*k+j       */
   int32_t *topk_ids;       /* [T*k]  as moe_route                                     */
   float *topk_weights;     /* [T*k]  as moe_route                                     */
-  uint32_t *router_stats;  /* [4]    {candidates recomputed in fp64, tokens that needed
-                            *         the exact sequential recomputation, largest screen
-                            *         error / (|x_t| |w_e|) seen (float bits), path:
-                            *         0 = fp64 logits, 1 = tensor-core screen}           */
+  uint32_t *router_stats;  /* [5]    {candidates recomputed, tokens that needed the exact
+                            *         sequential recomputation, largest screen error /
+                            *         (|x_t| |w_e|) seen (float bits), path: 0 = fp64
+                            *         logits, 1 = tensor-core screen, tokens whose fp32
+                            *         pair-sum recheck was too close to call and were
+                            *         recomputed in fp64 (screen path)}                 */
 } moe_aux_t;
 
 /* ABI version of the loaded library (MOE_ABI_VERSION at build time). */

@@ -165,7 +165,26 @@ def test_k_equals_E_and_exact_ties():
             ref = oracle.forward(x, w["w_router"], w["w_gate"], w["w_up"], w["w_down"], k)
             check_routing(aux, ref, cfg.E)
             check_y(y, ref["y"])
-            assert moe.router_stats(aux)["exact_recomputes"] > 0    # the ties went the exact way
+            st = moe.router_stats(aux)
+            assert st["exact_recomputes"] > 0    # the ties went the exact way
+            if router == "screen":               # ... through the fp64 recheck first
+                assert st["fp64_rechecks"] >= st["exact_recomputes"]
+
+
+def test_screen_pair_sums_settle_most_tokens(gemma_w):
+    """On the Gemma-shaped batch the fp32 pair-sum recheck decides the routing (and weights)
+    of most tokens; the ones it leaves go through fp64, and the result matches the oracle."""
+    x, c, g = layer_inputs(wl.CONFIGS["prefill"], gemma_w)
+    T = x.shape[0]
+    _, aux = gpu_forward(x, g, 8, router="screen")
+    st = moe.router_stats(aux)
+    assert st["path"] == "screen"
+    assert 8 * T <= st["candidates"] <= 32 * T, st
+    assert st["fp64_rechecks"] <= T // 4, st
+    ids, w_ref, _ = oracle.route(x, c["w_router"], 8)
+    assert np.array_equal(aux["topk_ids"].cpu().numpy(), ids)
+    w = aux["topk_weights"].cpu().numpy().astype(np.float64)
+    assert np.max(np.abs(w - w_ref)) <= W_ABS
 
 
 def test_determinism(gemma_w):
