@@ -102,7 +102,7 @@ size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 // (148), at most 8 slices and at least one 64-wide k-block per slice.
 int screen_ksplit(int T, int H) {
   const int mt = (T + 127) / 128;
-  return std::max(1, std::min({8, 148 / std::max(1, mt), H / 64}));
+  return std::max(1, std::min({kMaxScreenSplit, 148 / std::max(1, mt), H / 64}));
 }
 
 bool shape_supported(int T, int H, int E, int I, int k, bool need_I) {

@@ -592,43 +592,45 @@ __device__ __forceinline__ void screen_dot(const __nv_bfloat16* __restrict__ xr,
   }
 }
 
-// Recompute the nc candidates of this warp's token (ids in cand[]) into val[] (+ bias),
-// four rows at a time and two for a tail of at most two.
+// Recompute n candidates of this warp's token into val[] (+ bias): slot j is
+// sub ? sub[j] : j, its expert cand[slot].  Four rows at a time, two for a tail of <= 2.
 template <bool PAIRS>
 __device__ __forceinline__ void screen_recheck(const __nv_bfloat16* __restrict__ xr,
                                                const __nv_bfloat16* __restrict__ wrT,
                                                const float* __restrict__ bias, int H,
-                                               const int* cand, int nc, double* val) {
+                                               const int* cand, const int* sub, int n,
+                                               double* val) {
   const int lane = threadIdx.x & 31;
   __syncwarp();   // every lane is done reading val
-  for (int c0 = 0; c0 < nc;) {
-    if (nc - c0 > 2) {
+  auto slot = [&](int j) { return sub ? sub[j] : j; };
+  for (int c0 = 0; c0 < n;) {
+    if (n - c0 > 2) {
       const uint4* wrow[4];
 #pragma unroll
       for (int u = 0; u < 4; ++u)
-        wrow[u] = reinterpret_cast<const uint4*>(wrT + (size_t)cand[min(c0 + u, nc - 1)] * H);
+        wrow[u] = reinterpret_cast<const uint4*>(wrT + (size_t)cand[slot(min(c0 + u, n - 1))] * H);
       double acc[4];
       screen_dot<PAIRS, 4>(xr, wrow, H, acc);
       double v = acc[0];
 #pragma unroll
       for (int u = 1; u < 4; ++u)
         if (lane == u) v = acc[u];
-      if (lane < 4 && c0 + lane < nc) {
-        const int e = cand[c0 + lane];
-        val[c0 + lane] = bias ? v + (double)bias[e] : v;
+      if (lane < 4 && c0 + lane < n) {
+        const int c = slot(c0 + lane), e = cand[c];
+        val[c] = bias ? v + (double)bias[e] : v;
       }
       c0 += 4;
     } else {
       const uint4* wrow[2];
 #pragma unroll
       for (int u = 0; u < 2; ++u)
-        wrow[u] = reinterpret_cast<const uint4*>(wrT + (size_t)cand[min(c0 + u, nc - 1)] * H);
+        wrow[u] = reinterpret_cast<const uint4*>(wrT + (size_t)cand[slot(min(c0 + u, n - 1))] * H);
       double acc[2];
       screen_dot<PAIRS, 2>(xr, wrow, H, acc);
       const double v = lane == 1 ? acc[1] : acc[0];
-      if (lane < 2 && c0 + lane < nc) {
-        const int e = cand[c0 + lane];
-        val[c0 + lane] = bias ? v + (double)bias[e] : v;
+      if (lane < 2 && c0 + lane < n) {
+        const int c = slot(c0 + lane), e = cand[c];
+        val[c] = bias ? v + (double)bias[e] : v;
       }
       c0 += 2;
     }
@@ -684,19 +686,21 @@ __device__ __forceinline__ void warp_rank_select(const double (&V)[EPL], const d
 }
 
 // Rank the candidates (slot c = lane + 32 i) by their recomputed values and check every
-// decision against B_e = beta_e + c_extra |x| |w_e| + abs_extra.  Returns true when all of
-// them hold; V, cid, taken, sel_* describe the ranking either way, b_max = max selected B.
+// decision against B_e = beta_e, plus c_extra |x| |w_e| + abs_extra for a slot whose value
+// is a pair sum (prec[c] == 0 or prec == nullptr).  Returns true when all of them hold;
+// V, cid, taken, sel_* describe the ranking either way, b_max = max selected B, and need[i]
+// marks the slots of the decisions that failed (and of non-finite values).
 template <int EPL>
-__device__ __forceinline__ bool screen_rank_verify(const int* cand, const double* val, int nc,
+__device__ __forceinline__ bool screen_rank_verify(const int* cand, const double* val,
+                                                   const uint8_t* prec, int nc,
                                                    const double* __restrict__ wn,
                                                    const float* __restrict__ bias, double xn,
                                                    double beta_scale, double c_extra,
                                                    double abs_extra, int k, double (&V)[EPL],
                                                    int (&cid)[EPL], bool (&taken)[EPL],
-                                                   int (&sel_e)[8], double (&sel_v)[8],
-                                                   double& b_max) {
+                                                   bool (&need)[EPL], int (&sel_e)[8],
+                                                   double (&sel_v)[8], double& b_max) {
   const int lane = threadIdx.x & 31;
-  bool ok = true;
   double B[EPL];
 #pragma unroll
   for (int i = 0; i < EPL; ++i) {
@@ -704,13 +708,15 @@ __device__ __forceinline__ bool screen_rank_verify(const int* cand, const double
     cid[i] = INT_MAX;
     V[i] = -DBL_MAX;
     B[i] = 0.0;
+    need[i] = false;
     if (c < nc) {
       const int e = cand[c];
       cid[i] = e;
       V[i] = val[c];
-      ok = ok && isfinite(V[i]);
+      need[i] = !isfinite(V[i]);
       const double xw = xn * wn[e];
-      B[i] = beta_scale * (xw + (bias ? fabs((double)bias[e]) : 0.0)) + c_extra * xw + abs_extra;
+      B[i] = beta_scale * (xw + (bias ? fabs((double)bias[e]) : 0.0));
+      if (!(prec && prec[c])) B[i] += c_extra * xw + abs_extra;
     }
   }
   double sel_b[8];
@@ -719,28 +725,49 @@ __device__ __forceinline__ bool screen_rank_verify(const int* cand, const double
 #pragma unroll
   for (int r = 0; r < 8; ++r)
     if (r < k) b_max = fmax(b_max, sel_b[r]);
-  ok = ok && isfinite(b_max);
+  // adjacent selected pairs that are not separated (bit r: ranks r and r + 1)
+  unsigned bad = 0u;
 #pragma unroll
   for (int r = 0; r + 1 < 8; ++r)
-    if (r + 1 < k) ok = ok && (sel_v[r] - sel_v[r + 1] > sel_b[r] + sel_b[r + 1]);
+    if (r + 1 < k && !(sel_v[r] - sel_v[r + 1] > sel_b[r] + sel_b[r + 1])) bad |= 1u << r;
   double v_last = sel_v[0], b_last = sel_b[0];
+  int e_last = sel_e[0];
 #pragma unroll
   for (int r = 1; r < 8; ++r)
     if (r == k - 1) {
       v_last = sel_v[r];
       b_last = sel_b[r];
+      e_last = sel_e[r];
     }
+  // unselected candidates not separated from the k-th
+  bool bnd = false;
 #pragma unroll
   for (int i = 0; i < EPL; ++i)
-    if (cid[i] != INT_MAX && !taken[i]) ok = ok && (v_last - V[i] > b_last + B[i]);
-  return __all_sync(0xffffffffu, ok);
+    if (cid[i] != INT_MAX && !taken[i] && !(v_last - V[i] > b_last + B[i])) {
+      need[i] = true;
+      bnd = true;
+    }
+  bnd = __any_sync(0xffffffffu, bnd);
+#pragma unroll
+  for (int i = 0; i < EPL; ++i) {
+    if (cid[i] == INT_MAX) continue;
+    if (bnd && cid[i] == e_last) need[i] = true;
+#pragma unroll
+    for (int r = 0; r + 1 < 8; ++r)
+      if (((bad >> r) & 1u) && (cid[i] == sel_e[r] || cid[i] == sel_e[r + 1])) need[i] = true;
+  }
+  bool any = false;
+#pragma unroll
+  for (int i = 0; i < EPL; ++i) any = any || need[i];
+  return !__any_sync(0xffffffffu, any) && isfinite(b_max);
 }
 
-// Screen path, one warp per token.  screen: ks fp32 partial-sum slices of kstride floats
-// each ([T][E] per slice, added here in fp64 in slice order).
+// Screen path, one warp per token.  screen: ks <= kMaxScreenSplit fp32 partial-sum slices
+// of kstride floats each ([T][E] per slice, added here in fp64 in slice order).
 // stats[0] += candidates, stats[1] += exact recomputations,
 // stats[2] = max over candidates of |screen - L| / (|x| |w|) (float bits, atomicMax),
-// stats[3] = 1 (the screen path), stats[4] += tokens recomputed in fp64 (second tier).
+// stats[3] = 1 (the screen path), stats[4] += tokens with a candidate recomputed in fp64.
+constexpr int kMaxScreenSplit = 8;
 template <int EPL>
 __global__ void __launch_bounds__(256, 2) router_screen_select_kernel(
     const float* __restrict__ screen, int ks, long long kstride,
@@ -752,16 +779,41 @@ __global__ void __launch_bounds__(256, 2) router_screen_select_kernel(
   pdl_wait();
   if (blockIdx.x == 0 && threadIdx.x == 0) stats[3] = 1;   // path: screen + recheck
   __shared__ int s_cand[kScreenWarps][32 * EPL];
+  __shared__ int s_sub[kScreenWarps][32 * EPL];
   __shared__ double s_val[kScreenWarps][32 * EPL];
+  __shared__ float s_scr[kScreenWarps][32 * EPL];   // screen sums by expert (statistic)
+  __shared__ uint8_t s_prec[kScreenWarps][32 * EPL];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const unsigned lt = (1u << lane) - 1u;
   // bound of the pair sums: 2^-24 sum |x_h w_h| <= 2^-24 |x| |w| (+ 1%), underflow H 2^-150
   const double pair_c = 1.01 * 0x1p-24, pair_abs = (double)H * 0x1p-149;
+  int* cand = s_cand[warp];
+  int* sub = s_sub[warp];
+  double* val = s_val[warp];
+  uint8_t* prec = s_prec[warp];
   // statistics are gathered per warp and published once, not per token
   unsigned st_cand = 0, st_exact = 0, st_fp64 = 0;
   float st_err = 0.f;
   for (int t = blockIdx.x * kScreenWarps + warp; t < T; t += gridDim.x * kScreenWarps) {
     const __nv_bfloat16* xr = x + (size_t)t * H;
+    // Screen sums first: every partial of every slot in flight at once.
+    double sv[EPL];
+    {
+      float part[kMaxScreenSplit][EPL];
+#pragma unroll
+      for (int z = 0; z < kMaxScreenSplit; ++z)
+#pragma unroll
+        for (int i = 0; i < EPL; ++i)
+          part[z][i] = (z < ks && lane + 32 * i < E)
+                           ? __ldg(screen + z * kstride + (size_t)t * E + lane + 32 * i)
+                           : 0.f;
+#pragma unroll
+      for (int i = 0; i < EPL; ++i) {
+        sv[i] = 0.0;
+#pragma unroll
+        for (int z = 0; z < kMaxScreenSplit; ++z) sv[i] += (double)part[z][i];
+      }
+    }
     // |x_t| bound: squares of bf16 values are exact in fp32; each lane sums its H/32 of them
     // in fp32 (relative error < (H/32) 2^-24, + H/32 2^-150 for underflow), 16-byte loads
     float q = 0.f;
@@ -803,12 +855,11 @@ __global__ void __launch_bounds__(256, 2) router_screen_select_kernel(
       D[i] = 0.0;
       skey[i] = 0u;
       if (e < E) {
-        double sv = 0.0;
-        for (int z = 0; z < ks; ++z) sv += (double)screen[z * kstride + (size_t)t * E + e];
+        s_scr[warp][e] = (float)sv[i];
         const double xw = xn * wn[e];
         const double beta = beta_scale * (xw + (bias ? fabs((double)bias[e]) : 0.0));
-        if (isfinite(sv)) {
-          S[i] = bias ? sv + (double)bias[e] : sv;
+        if (isfinite(sv[i])) {
+          S[i] = bias ? sv[i] + (double)bias[e] : sv[i];
           D[i] = screen_c * xw + 4.0 * beta;
           // 24 high bits of the value, then 255 - e: unique keys, larger S first
           skey[i] = (ord_f32((float)S[i]) & 0xffffff00u) | (uint32_t)(255 - e);
@@ -844,49 +895,79 @@ __global__ void __launch_bounds__(256, 2) router_screen_select_kernel(
     }
     // Compact the candidates in ascending expert id.
     int nc = 0;
-    int* cand = s_cand[warp];
-    double* val = s_val[warp];
 #pragma unroll
     for (int i = 0; i < EPL; ++i) {
       const int e = lane + 32 * i;
       const bool c = e < E && (!finite || S[i] + D[i] >= tau);
       const unsigned m = __ballot_sync(0xffffffffu, c);
-      if (c) cand[nc + __popc(m & lt)] = e;
+      if (c) {
+        cand[nc + __popc(m & lt)] = e;
+        prec[nc + __popc(m & lt)] = 0;
+      }
       nc += __popc(m);
     }
     __syncwarp();
 
     // First recheck: fp32 pair sums.  Kept when every ranking decision clears the pair-sum
     // bound and the weights they give are within kPairWeightErr of the fp64 ones.
-    screen_recheck<true>(xr, wrT, bias, H, cand, nc, val);
+    screen_recheck<true>(xr, wrT, bias, H, cand, nullptr, nc, val);
     double V[EPL];
     int cid[EPL];
-    bool taken[EPL];
+    bool taken[EPL], need[EPL];
     int sel_e[8];
     double sel_v[8];
     double b_max;
-    bool ok = screen_rank_verify<EPL>(cand, val, nc, wn, bias, xn, beta_scale, pair_c, pair_abs,
-                                      k, V, cid, taken, sel_e, sel_v, b_max);
+    bool ok = screen_rank_verify<EPL>(cand, val, prec, nc, wn, bias, xn, beta_scale, pair_c,
+                                      pair_abs, k, V, cid, taken, need, sel_e, sel_v, b_max);
     // this lane's share of the renormalised weights: lane r < k holds exp(L_r - L_0)
-    double my_v = sel_v[0];
-    int my_e = sel_e[0];
+    auto lane_weight = [&](double& ev, double& denom, int& my_e) {
+      double my_v = sel_v[0];
+      my_e = sel_e[0];
 #pragma unroll
-    for (int r = 1; r < 8; ++r)
-      if (lane == r) {
-        my_v = sel_v[r];
-        my_e = sel_e[r];
-      }
-    double ev = lane < k ? exp(my_v - sel_v[0]) : 0.0;
-    double denom = ev;
+      for (int r = 1; r < 8; ++r)
+        if (lane == r) {
+          my_v = sel_v[r];
+          my_e = sel_e[r];
+        }
+      ev = lane < k ? exp(my_v - sel_v[0]) : 0.0;
+      denom = ev;
 #pragma unroll
-    for (int off = 16; off; off >>= 1) denom += __shfl_xor_sync(0xffffffffu, denom, off);
-    ok = ok && 2.0 * b_max / denom <= kPairWeightErr;   // 1 / denom: the largest weight
-    if (!ok) {
-      // Second recheck: fp64 products and sums, checked against the fp64 bound alone.
+      for (int off = 16; off; off >>= 1) denom += __shfl_xor_sync(0xffffffffu, denom, off);
+    };
+    double ev, denom;
+    int my_e;
+    lane_weight(ev, denom, my_e);
+    const bool weights_ok = 2.0 * b_max / denom <= kPairWeightErr;   // 1 / denom: max weight
+    if (!ok || !weights_ok) {
       ++st_fp64;
-      screen_recheck<false>(xr, wrT, bias, H, cand, nc, val);
-      ok = screen_rank_verify<EPL>(cand, val, nc, wn, bias, xn, beta_scale, 0.0, 0.0, k, V, cid,
-                                   taken, sel_e, sel_v, b_max);
+      // Second recheck in fp64: only the slots of the failed decisions when the weights were
+      // fine, every candidate otherwise; each recomputed slot then carries the fp64 bound.
+      int ns = 0;
+      if (weights_ok) {
+#pragma unroll
+        for (int i = 0; i < EPL; ++i) {
+          const unsigned m = __ballot_sync(0xffffffffu, need[i]);
+          if (need[i]) sub[ns + __popc(m & lt)] = lane + 32 * i;
+          ns += __popc(m);
+        }
+        __syncwarp();
+      }
+      if (ns > 0 && ns < nc) {
+        screen_recheck<false>(xr, wrT, bias, H, cand, sub, ns, val);
+        for (int j = lane; j < ns; j += 32) prec[sub[j]] = 1;
+        __syncwarp();
+        ok = screen_rank_verify<EPL>(cand, val, prec, nc, wn, bias, xn, beta_scale, pair_c,
+                                     pair_abs, k, V, cid, taken, need, sel_e, sel_v, b_max);
+        lane_weight(ev, denom, my_e);
+        ok = ok && 2.0 * b_max / denom <= kPairWeightErr;
+      } else {
+        ok = false;
+      }
+      if (!ok) {
+        screen_recheck<false>(xr, wrT, bias, H, cand, nullptr, nc, val);
+        ok = screen_rank_verify<EPL>(cand, val, nullptr, nc, wn, bias, xn, beta_scale, 0.0, 0.0,
+                                     k, V, cid, taken, need, sel_e, sel_v, b_max);
+      }
       if (!ok) {
         // Too close to call: each lane recomputes its candidates as one FMA chain in
         // ascending h (the definition's sequence of roundings), then the warp ranks again.
@@ -906,18 +987,7 @@ __global__ void __launch_bounds__(256, 2) router_screen_select_kernel(
         warp_rank_select<EPL>(V, Bz, cid, k, taken, sel_e, sel_v, sel_bz);
         ++st_exact;
       }
-      my_v = sel_v[0];
-      my_e = sel_e[0];
-#pragma unroll
-      for (int r = 1; r < 8; ++r)
-        if (lane == r) {
-          my_v = sel_v[r];
-          my_e = sel_e[r];
-        }
-      ev = lane < k ? exp(my_v - sel_v[0]) : 0.0;
-      denom = ev;
-#pragma unroll
-      for (int off = 16; off; off >>= 1) denom += __shfl_xor_sync(0xffffffffu, denom, off);
+      lane_weight(ev, denom, my_e);
     }
     // largest |screen - L| / (|x| |w|) over the candidates, L from the last recheck
     float err = 0.f;
@@ -926,15 +996,13 @@ __global__ void __launch_bounds__(256, 2) router_screen_select_kernel(
       for (int i = 0; i < EPL; ++i) {
         if (cid[i] != INT_MAX) {
           const int e = cid[i];
-          double sv = 0.0;
-          for (int z = 0; z < ks; ++z) sv += (double)screen[z * kstride + (size_t)t * E + e];
           const double L0 = bias ? V[i] - (double)bias[e] : V[i];
-          err = fmaxf(err, (float)(fabs(sv - L0) / (xn * wn[e])));
+          err = fmaxf(err, (float)(fabs((double)s_scr[warp][e] - L0) / (xn * wn[e])));
         }
       }
     }
     st_cand += (unsigned)nc;
-    st_err = fmaxf(st_err, err);   // lanes differ; the block-wide max is taken below
+    st_err = fmaxf(st_err, err);   // lanes differ; the warp-wide max is taken below
 
     // Renormalised weights: softmax over the k selected logits, lane r writes slot r.
     if (lane < k) {
