@@ -41,15 +41,12 @@ __global__ void __launch_bounds__(256) dispatch_count_kernel(const int32_t* __re
 // (expert, first sorted row, rows in tile), in expert order.  Also zeroes the split-unit
 // counters the grouped GEMMs use.  Thread e walks its column of chunk counts with 8 loads
 // in flight; warp 0 scans the experts (8 per lane) with shuffles.
-__global__ void __launch_bounds__(256) dispatch_scan_kernel(
+__device__ __forceinline__ void dispatch_scan_block(
     const int32_t* __restrict__ chunk_counts, int nchunks, int E, int P, int BM,
     int32_t* __restrict__ counts, int32_t* __restrict__ offsets, int32_t* __restrict__ chunk_base,
     int32_t* __restrict__ tile_num, int32_t* __restrict__ tile_expert,
     int32_t* __restrict__ tile_row0, int32_t* __restrict__ tile_rows,
-    int32_t* __restrict__ gemm_counters, int n_counters) {
-  pdl_trigger();
-  pdl_wait();
-  __shared__ int s_cnt[256], s_off[256], s_tstart[256];
+    int32_t* __restrict__ gemm_counters, int n_counters, int* s_cnt, int* s_off, int* s_tstart) {
   for (int i = threadIdx.x; i < n_counters; i += blockDim.x) gemm_counters[i] = 0;
   const int e = threadIdx.x, lane = threadIdx.x & 31;
   int run = 0;
@@ -121,44 +118,56 @@ __global__ void __launch_bounds__(256) dispatch_scan_kernel(
   }
 }
 
+__global__ void __launch_bounds__(256) dispatch_scan_kernel(
+    const int32_t* __restrict__ chunk_counts, int nchunks, int E, int P, int BM,
+    int32_t* __restrict__ counts, int32_t* __restrict__ offsets, int32_t* __restrict__ chunk_base,
+    int32_t* __restrict__ tile_num, int32_t* __restrict__ tile_expert,
+    int32_t* __restrict__ tile_row0, int32_t* __restrict__ tile_rows,
+    int32_t* __restrict__ gemm_counters, int n_counters) {
+  pdl_trigger();
+  pdl_wait();
+  __shared__ int s_cnt[256], s_off[256], s_tstart[256];
+  dispatch_scan_block(chunk_counts, nchunks, E, P, BM, counts, offsets, chunk_base, tile_num,
+                      tile_expert, tile_row0, tile_rows, gemm_counters, n_counters, s_cnt, s_off,
+                      s_tstart);
+}
+
 // One CTA of 8 warps per chunk: warp w takes pairs [256 w, 256 w + 256) of the chunk
 // (8 per lane, loaded up front), counts them per expert, the warps' counts are scanned in
 // warp order per expert, and each warp ranks its pairs in order with __match_any_sync:
 // pos = chunk_base[c][e] + pairs of e in earlier warps + rank within the warp's earlier
 // pairs.  perm[pos] = q, inv[q] = pos.  Dynamic shared memory: 9 * E ints.
 constexpr int kRankWarps = 8;
-__global__ void __launch_bounds__(32 * kRankWarps) dispatch_rank_kernel(
-    const int32_t* __restrict__ ids, int P, int E, const int32_t* __restrict__ chunk_base,
-    int32_t* __restrict__ perm, int32_t* __restrict__ inv) {
-  pdl_trigger();
-  pdl_wait();
-  extern __shared__ int rank_sm[];
-  int* wcnt = rank_sm;                   // [kRankWarps][E] pairs of e in warp w
-  int* base = rank_sm + kRankWarps * E;  // [E] chunk base
+constexpr int kRankSub = kDispatchChunk / kRankWarps;   // 256 pairs per warp
+
+// This warp's pairs of chunk c (expert ids; -1 past P, -2 for an id out of range) and its
+// per-expert counts in wcnt[warp][e] (zeroed by the caller).
+__device__ __forceinline__ void rank_load_count(const int32_t* __restrict__ ids, int P, int E,
+                                                int c, int* wcnt, int (&ev)[kRankSub / 32]) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  constexpr int kSub = kDispatchChunk / kRankWarps;   // 256 pairs per warp
-  const int q0 = blockIdx.x * kDispatchChunk + warp * kSub;
-  for (int i = threadIdx.x; i < kRankWarps * E; i += blockDim.x) wcnt[i] = 0;
-  for (int i = threadIdx.x; i < E; i += blockDim.x) base[i] = chunk_base[(size_t)blockIdx.x * E + i];
-  int ev[kSub / 32];
+  const int q0 = c * kDispatchChunk + warp * kRankSub;
 #pragma unroll
-  for (int it = 0; it < kSub / 32; ++it) {
+  for (int it = 0; it < kRankSub / 32; ++it) {
     const int q = q0 + 32 * it + lane;
     int e = q < P ? __ldcg(ids + q) : -1;
     if (q < P && (unsigned)e >= (unsigned)E) e = -2;   // counted as an error already
     ev[it] = e;
   }
-  __syncthreads();
-  const unsigned lt = (1u << lane) - 1u;
-  // per-warp counts
 #pragma unroll
-  for (int it = 0; it < kSub / 32; ++it) {
+  for (int it = 0; it < kRankSub / 32; ++it) {
     const int e = ev[it];
     const unsigned grp = __match_any_sync(0xffffffffu, e);
     if (e >= 0 && lane == 31 - __clz(grp)) wcnt[warp * E + e] += __popc(grp);
     __syncwarp();
   }
-  __syncthreads();
+}
+
+// After the warps' counts and base[e] = chunk_base[c][e] are in shared memory (and a block
+// barrier): scan the counts over the warps, then place every pair.
+__device__ __forceinline__ void rank_place(int E, int c, int* wcnt, const int* base,
+                                           const int (&ev)[kRankSub / 32],
+                                           int32_t* __restrict__ perm, int32_t* __restrict__ inv) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   // exclusive scan over the warps, per expert (in place): wcnt[w][e] = pairs of e in warps < w
   for (int e = threadIdx.x; e < E; e += blockDim.x) {
     int run = base[e];
@@ -171,8 +180,10 @@ __global__ void __launch_bounds__(32 * kRankWarps) dispatch_rank_kernel(
   }
   __syncthreads();
   int* wb = wcnt + warp * E;   // this warp's running base per expert
+  const unsigned lt = (1u << lane) - 1u;
+  const int q0 = c * kDispatchChunk + warp * kRankSub;
 #pragma unroll
-  for (int it = 0; it < kSub / 32; ++it) {
+  for (int it = 0; it < kRankSub / 32; ++it) {
     const int q = q0 + 32 * it + lane;
     const int e = ev[it];
     const unsigned grp = __match_any_sync(0xffffffffu, e);
@@ -186,6 +197,76 @@ __global__ void __launch_bounds__(32 * kRankWarps) dispatch_rank_kernel(
       inv[q] = pos;
     }
   }
+}
+
+__global__ void __launch_bounds__(32 * kRankWarps) dispatch_rank_kernel(
+    const int32_t* __restrict__ ids, int P, int E, const int32_t* __restrict__ chunk_base,
+    int32_t* __restrict__ perm, int32_t* __restrict__ inv) {
+  pdl_trigger();
+  pdl_wait();
+  extern __shared__ int rank_sm[];
+  int* wcnt = rank_sm;                   // [kRankWarps][E] pairs of e in warp w
+  int* base = rank_sm + kRankWarps * E;  // [E] chunk base
+  const int c = blockIdx.x;
+  for (int i = threadIdx.x; i < kRankWarps * E; i += blockDim.x) wcnt[i] = 0;
+  for (int i = threadIdx.x; i < E; i += blockDim.x) base[i] = chunk_base[(size_t)c * E + i];
+  __syncthreads();
+  int ev[kRankSub / 32];
+  rank_load_count(ids, P, E, c, wcnt, ev);
+  __syncthreads();
+  rank_place(E, c, wcnt, base, ev, perm, inv);
+}
+
+// The three kernels above in one launch, for few chunks (every CTA must be resident at
+// once, so at most the SM count): CTA c counts chunk c and publishes its counts; the CTA that arrives last (a counter)
+// runs the scan and raises a flag; every CTA waits (bounded) for the flag, reads its chunk's
+// bases and ranks its pairs.  sync[0] (arrivals) and sync[1] (flag) are zero at launch.
+// Dynamic shared memory: (kRankWarps + 1) * E ints.
+__global__ void __launch_bounds__(32 * kRankWarps) dispatch_fused_kernel(
+    const int32_t* __restrict__ ids, int P, int E, int BM, int nchunks,
+    int32_t* __restrict__ chunk_counts, int32_t* __restrict__ chunk_base,
+    int32_t* __restrict__ counts, int32_t* __restrict__ offsets, int32_t* __restrict__ perm,
+    int32_t* __restrict__ inv, int32_t* __restrict__ tile_num, int32_t* __restrict__ tile_expert,
+    int32_t* __restrict__ tile_row0, int32_t* __restrict__ tile_rows,
+    int32_t* __restrict__ gemm_counters, int n_counters, int* __restrict__ sync) {
+  pdl_trigger();
+  pdl_wait();
+  extern __shared__ int rank_sm[];
+  int* wcnt = rank_sm;
+  int* base = rank_sm + kRankWarps * E;
+  __shared__ int s_cnt[256], s_off[256], s_tstart[256];
+  __shared__ int s_last, s_ok;
+  const int c = blockIdx.x;
+  for (int i = threadIdx.x; i < kRankWarps * E; i += blockDim.x) wcnt[i] = 0;
+  __syncthreads();
+  int ev[kRankSub / 32];
+  rank_load_count(ids, P, E, c, wcnt, ev);
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    int n = 0;
+#pragma unroll
+    for (int w = 0; w < kRankWarps; ++w) n += wcnt[w * E + e];
+    chunk_counts[(size_t)c * E + e] = n;
+  }
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) s_last = atomicAdd(&sync[0], 1) == nchunks - 1;
+  __syncthreads();
+  if (s_last) {
+    __threadfence();   // every chunk's counts before reading them
+    dispatch_scan_block(chunk_counts, nchunks, E, P, BM, counts, offsets, chunk_base, tile_num,
+                        tile_expert, tile_row0, tile_rows, gemm_counters, n_counters, s_cnt,
+                        s_off, s_tstart);
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) red_release_add_gpu(&sync[1], 1);
+  }
+  if (threadIdx.x == 0) s_ok = wait_counter_geq(&sync[1], 1);
+  __syncthreads();
+  if (!s_ok) return;   // timed out: the error word is set
+  for (int i = threadIdx.x; i < E; i += blockDim.x) base[i] = __ldcg(chunk_base + (size_t)c * E + i);
+  __syncthreads();
+  rank_place(E, c, wcnt, base, ev, perm, inv);
 }
 
 // Whole dispatch for a batch of at most one chunk (P <= kDispatchChunk) by one CTA (any

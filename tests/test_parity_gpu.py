@@ -232,13 +232,29 @@ def test_graph_replay_matches_direct_call(gemma_w):
     assert torch.equal(y2, moe.forward(x2, g["w_router"], g["w_gate"], g["w_up"], g["w_down"], 8))
 
 
+def test_dispatch_three_launches_for_many_chunks(gemma_w):
+    """Past 32 chunks of 2048 pairs the dispatch runs as three launches (count, scan, rank)
+    instead of one; its counts, offsets and permutation must still be the oracle's for the
+    ids the router chose."""
+    T = 2048 * 160 // 8   # 160 chunks of 2048 pairs at k = 8
+    x, c, g = layer_inputs(wl.CONFIGS["prefill"], gemma_w, T=T)
+    y, aux = gpu_forward(x, g, 8)
+    assert moe.last_kernel_count() == 4 + 3 + 1 + 1
+    ids = aux["topk_ids"].cpu().numpy()
+    counts, offsets, perm, _ = oracle.dispatch(ids, 128)
+    assert np.array_equal(aux["expert_counts"].cpu().numpy(), counts)
+    assert np.array_equal(aux["expert_offsets"].cpu().numpy(), offsets)
+    assert np.array_equal(aux["perm"].cpu().numpy(), perm)
+    assert torch.isfinite(y.float()).all()
+
+
 @pytest.mark.parametrize("T,tiles,expected", [
     (8, "auto", 3),        # decode front end (router + dispatch), expert FFN, combine
     (8, "unfused", 4),     # ... with GEMM-1 and GEMM-2 as two launches
     (64, "auto", 5),       # fp64 router 2, single-CTA dispatch, expert FFN, combine
-    (4096, "auto", 9),     # screen router 4, dispatch 3, expert FFN, combine
-    (4096, "unfused", 10), # ... with GEMM-1 and GEMM-2 as two launches
-    (4096, "fused", 9),    # ... static stream-K schedule in one launch
+    (4096, "auto", 7),     # screen router 4, one-launch dispatch, expert FFN, combine
+    (4096, "unfused", 8),  # ... with GEMM-1 and GEMM-2 as two launches
+    (4096, "fused", 7),    # ... static stream-K schedule in one launch
 ])
 def test_kernel_count_per_forward(T, tiles, expected, gemma_w):
     x, c, g = layer_inputs(wl.CONFIGS["decode"], gemma_w, T=T)
