@@ -3,8 +3,10 @@
     python bench.py [--gpus N] [--steps K] [--warmup W] [--config decode] [--impl reference]
 
 A step is one moe_forward over one batch (router, dispatch, GEMM-1 + GEGLU, GEMM-2,
-combine) with inputs resident in HBM.  L2 is flushed (256 MB write, untimed) before
-every step; each step is timed with CUDA events on the launching stream.  Rank 0 prints
+combine) with inputs resident in HBM.  L2 is flushed before every step, untimed: a 256 MB
+write, then a 256 MB read, so that the dirty lines the write leaves are written back before
+the step rather than during it; each step is timed with CUDA events on the launching
+stream.  Rank 0 prints
 one JSON line.  With N > 1 (torchrun) every rank runs its own batch on its own GPU (weak
 scaling, no collective on the data path) and the reported time is the max over ranks.
 
@@ -264,7 +266,13 @@ def run_native(args, cfg) -> None:
     g = {k: (v.to(dev) if v is not None else None) for k, v in d.items()}
     x = x_cpu.to(dev)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    flush_rd = torch.zeros(L2_FLUSH_BYTES // 8, dtype=torch.int64, device=dev)
     stream = torch.cuda.current_stream()
+
+    def flush_l2():
+        # write more than L2 holds, then read more than it holds: L2 ends cold and clean
+        flush.zero_()
+        flush_rd.max()
 
     y0, aux = moe.forward(x, g["w_router"], g["w_gate"], g["w_up"], g["w_down"], cfg.k,
                           bias=g["bias"], aux=True, tiles=args.tiles)
@@ -278,7 +286,7 @@ def run_native(args, cfg) -> None:
     graph = moe.ForwardGraph(x, g["w_router"], g["w_gate"], g["w_up"], g["w_down"], cfg.k,
                              bias=g["bias"], tiles=args.tiles)
     for _ in range(args.warmup):
-        flush.zero_()
+        flush_l2()
         graph.replay()
     torch.cuda.synchronize()
     if not torch.equal(graph.y, y0):
@@ -293,7 +301,7 @@ def run_native(args, cfg) -> None:
         dist.barrier()
     torch.cuda.synchronize()
     for i in range(args.steps):
-        flush.zero_()
+        flush_l2()
         ev[i][0].record(stream)
         graph.replay()
         ev[i][1].record(stream)
@@ -312,7 +320,7 @@ def run_native(args, cfg) -> None:
     stage_acc: dict[str, list[float]] = {}
     try:
         for _ in range(max(3, min(args.steps, 20))):
-            flush.zero_()
+            flush_l2()
             pgraph.replay()
             for k, v in moe.last_stage_times().items():
                 stage_acc.setdefault(k, []).append(v)
@@ -327,7 +335,7 @@ def run_native(args, cfg) -> None:
     e2e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
               for _ in range(args.steps)]
     for i in range(args.warmup + args.steps):
-        flush.zero_()
+        flush_l2()
         if i >= args.warmup:
             e2e_ev[i - args.warmup][0].record(stream)
         graph.x.copy_(x_host, non_blocking=True)
@@ -379,7 +387,7 @@ def run_native(args, cfg) -> None:
                                    f"I={cfg.I} (routed MoE FFN layer, Gemma-4-26B-A4B shape)",
                        "global_batch": world * cfg.T, "tokens_per_gpu": cfg.T,
                        "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
-                       "l2": "flushed before every step (256 MB write, untimed)"},
+                       "l2": "flushed before every step (256 MB write then 256 MB read, untimed)"},
             "roofline": roof,
             "step_roofline": {
                 "hbm_frac": acc["step_bytes"] / step_s / (pk["hbm_gbs"] * 1e9),
