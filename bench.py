@@ -411,6 +411,115 @@ def run_native(args, cfg) -> None:
         dist.destroy_process_group()
 
 
+def run_dense(args, cfg) -> None:
+    """--dense: the dense GEGLU MLP beside the MoE (intermediate workloads.DENSE_I) on the
+    config's x, one GPU; same timing rules as the layer (clean L2 before every step)."""
+    import expert_routed_ffn_softmax_b200 as moe
+    if int(os.environ.get("WORLD_SIZE", "1")) != 1 or args.gpus != 1:
+        raise SystemExit("--dense runs on one GPU")
+    dev = torch.device("cuda", 0)
+    I = wl.DENSE_I if cfg.H == 2816 else 2 * cfg.I
+    w = wl.make_dense_weights(cfg.H, I)
+    g = {k: v.to(dev) for k, v in w.items()}
+    x_cpu = wl.make_x(cfg)
+    x = x_cpu.to(dev)
+    y = torch.empty((cfg.T, cfg.H), dtype=torch.bfloat16, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    flush_rd = torch.zeros(L2_FLUSH_BYTES // 8, dtype=torch.int64, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def flush_l2():
+        flush.zero_()
+        flush_rd.max()
+
+    def step():
+        moe.dense_ffn(x, g["w_gate"], g["w_up"], g["w_down"], out=y)
+
+    for _ in range(args.warmup):
+        flush_l2()
+        step()
+    torch.cuda.synchronize()
+    if moe.sync_status() != 0:
+        raise SystemExit("device status not OK after the warm-up")
+    launches = moe.last_kernel_count()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    clocks = ClockSampler(dev)
+    clocks.start()
+    torch.cuda.synchronize()
+    for i in range(args.steps):
+        flush_l2()
+        ev[i][0].record(stream)
+        step()
+        ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    ms = sum(a.elapsed_time(b) for a, b in ev) / args.steps
+    # end to end: pinned x in, y out, every step
+    x_host = x_cpu.pin_memory()
+    y_host = torch.empty((cfg.T, cfg.H), dtype=torch.bfloat16).pin_memory()
+    e2e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(args.steps)]
+    for i in range(args.warmup + args.steps):
+        flush_l2()
+        if i >= args.warmup:
+            e2e_ev[i - args.warmup][0].record(stream)
+        x.copy_(x_host, non_blocking=True)
+        step()
+        y_host.copy_(y, non_blocking=True)
+        if i >= args.warmup:
+            e2e_ev[i - args.warmup][1].record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = sum(a.elapsed_time(b) for a, b in e2e_ev) / args.steps
+    pk = peaks()
+    wbytes = 3 * cfg.H * I * 2
+    kb = wbytes + 2 * cfg.T * cfg.H * 2
+    kf = cfg.T * (2 * cfg.H * 2 * I + 2 * I * cfg.H)
+    ridge = pk["bf16_tflops"] * 1e12 / (pk["hbm_gbs"] * 1e9)
+    rname = next(r for r in (8, 16, 32, 64, 128) if cfg.T <= r or r == 128)
+    if kf / kb < ridge:
+        a = kb / (ms * 1e-3) / 1e9
+        roof = {"bound": "hbm", "achieved": a, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                "frac": a / pk["hbm_gbs"], "traffic": None,
+                "kernel": f"expert_ffn_dynamic_kernel<{rname}> (one expert, all rows)",
+                "peak_source": pk["source"] + " hbm_gbs"}
+    else:
+        a = kf / (ms * 1e-3) / 1e12
+        roof = {"bound": "tensor", "achieved": a, "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
+                "frac": a / pk["bf16_tflops"], "traffic": None,
+                "kernel": f"expert_ffn_dynamic_kernel<{rname}> (one expert, all rows)",
+                "peak_source": pk["source"] + " bf16_tflops (burst)",
+                "frac_of_sustained": a / pk["bf16_tflops_sustained"]}
+    line = {
+        "metric": "dense GEGLU MLP tokens/s (the MLP beside the MoE)", "value": cfg.T / (ms * 1e-3),
+        "unit": UNIT, "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": f"dense MLP: T={cfg.T} H={cfg.H} I={I} (x of the {cfg.name} config)",
+                   "global_batch": cfg.T, "parallelism": "single GPU",
+                   "l2": "flushed before every step (256 MB write then 256 MB read, untimed)"},
+        "roofline": roof, "gpu_launches": launches * args.steps, "clocks": clk,
+        "e2e": {"value": cfg.T / (e2e_ms * 1e-3), "unit": UNIT,
+                "h2d_bytes_per_step": cfg.T * cfg.H * 2, "d2h_bytes_per_step": cfg.T * cfg.H * 2},
+    }
+    if not args.no_cpu_baseline:
+        import oracle
+        cores = len(os.sched_getaffinity(0))
+        oracle.set_threads(cores)
+        rows = list(range(min(cfg.T, 8)))
+        n, t_total = 0, 0.0
+        while t_total < args.cpu_seconds or n == 0:
+            t0 = time.perf_counter()
+            oracle.dense_ffn(x_cpu, w["w_gate"], w["w_up"], w["w_down"], rows=rows)
+            t_total += time.perf_counter() - t0
+            n += 1
+        line["cpu_baseline"] = {"value": n * len(rows) / t_total, "unit": UNIT,
+                                "cores": oracle.get_threads(), "kind": "oracle",
+                                "sample": f"{n} x the dense MLP of the first {len(rows)} tokens "
+                                          f"({t_total:.1f} s of fp64 CPU work)"}
+    print(json.dumps(line), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -423,10 +532,14 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--tiles", default="auto", choices=["auto", "decode", "prefill", "fused", "unfused"],
                     help="expert-GEMM tile family (default: the library's choice)")
+    ap.add_argument("--dense", action="store_true",
+                    help="time the dense GEGLU MLP beside the MoE instead of the MoE layer")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)     # at least 3 untimed warm-up steps
     cfg = wl.CONFIGS[args.config]
-    if args.impl == "reference":
+    if args.dense:
+        run_dense(args, cfg)
+    elif args.impl == "reference":
         run_reference(args, cfg)
     else:
         run_native(args, cfg)

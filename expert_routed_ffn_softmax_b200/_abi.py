@@ -33,8 +33,8 @@ MOE_FLAG_UNFUSED_FFN = 1 << 6
 MOE_FLAG_FUSED_FFN = 1 << 7
 
 _ROUTER_FLAGS = {"auto": 0, "fp64": MOE_FLAG_ROUTER_FP64, "screen": MOE_FLAG_ROUTER_SCREEN}
-# Prefill tiles run GEMM-1 and GEMM-2 as one persistent launch ("fused") or two
-# ("unfused"); "prefill" leaves that choice to the library (fused for T*k <= 1024).
+# "auto"/"prefill": the dynamically scheduled expert FFN (one launch); "fused" / "unfused":
+# the statically scheduled forms in one or two launches; "decode": the swap-AB decode tiles.
 _TILE_FLAGS = {"auto": 0, "decode": MOE_FLAG_DECODE_TILES, "prefill": MOE_FLAG_PREFILL_TILES,
                "fused": MOE_FLAG_PREFILL_TILES | MOE_FLAG_FUSED_FFN,
                "unfused": MOE_FLAG_PREFILL_TILES | MOE_FLAG_UNFUSED_FFN}
@@ -49,6 +49,8 @@ SIGNATURES = {
     "moe_route": (_I, [_P, _P, _P, _I, _I, _I, _I, _U, _P, _P, _P, _SZ, _P]),
     "moe_route_static": (_I, [_P, _P, _P, _I, _I, _I, _I, _U, _P, _P, _P]),
     "moe_forward": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _U, _P, _P, _P, _SZ, _P]),
+    "moe_dense_workspace_size": (_SZ, [_I, _I, _I]),
+    "moe_dense_ffn": (_I, [_P, _P, _P, _P, _I, _I, _I, _P, _P, _SZ, _P]),
     "moe_sync_status": (_I, [_P]),
     "moe_last_stage_times": (_I, [ctypes.POINTER(ctypes.c_float), _I]),
     "moe_stage_name": (ctypes.c_char_p, [_I]),
@@ -208,6 +210,32 @@ def forward(x: torch.Tensor, w_router: torch.Tensor, w_gate: torch.Tensor, w_up:
                          None if a is None else ctypes.byref(a), ws.data_ptr(), ws.numel(),
                          _stream_ptr(stream)), "moe_forward")
     return (y, aux_d) if aux else y
+
+
+def dense_ffn(x: torch.Tensor, w_gate: torch.Tensor, w_up: torch.Tensor, w_down: torch.Tensor,
+              out: torch.Tensor | None = None, stream=None,
+              workspace_buf: torch.Tensor | None = None) -> torch.Tensor:
+    """The dense GEGLU MLP beside the MoE -> y bf16 [T,H]:
+    y = (gelu_tanh(x W_gate) * (x W_up)) W_down, W_gate/W_up [H,I], W_down [I,H]."""
+    L = load()
+    T, H = x.shape
+    I = w_gate.shape[1]
+    dev = x.device
+    px = _dev(x, "x", torch.bfloat16, (T, H))
+    pg = _dev(w_gate, "w_gate", torch.bfloat16, (H, I))
+    pu = _dev(w_up, "w_up", torch.bfloat16, (H, I))
+    pd = _dev(w_down, "w_down", torch.bfloat16, (I, H))
+    y = torch.empty((T, H), dtype=torch.bfloat16, device=dev) if out is None else out
+    py = _dev(y, "out", torch.bfloat16, (T, H))
+    if T == 0:
+        return y
+    nbytes = L.moe_dense_workspace_size(T, H, I)
+    if nbytes == 0:
+        raise MoEError(MOE_ERR_UNSUPPORTED, "moe_dense_workspace_size")
+    ws = workspace(nbytes, dev) if workspace_buf is None else workspace_buf
+    _check(L.moe_dense_ffn(px, pg, pu, pd, T, H, I, py, ws.data_ptr(), ws.numel(),
+                           _stream_ptr(stream)), "moe_dense_ffn")
+    return y
 
 
 def router_stats(aux: dict) -> dict:

@@ -153,7 +153,7 @@ __global__ void __launch_bounds__(PG_MAX_THREADS, 1)
   pdl_wait();   // the tile list, counters and x come from the previous kernels
   int n_tiles = 0;
   if (!(*reinterpret_cast<volatile unsigned*>(&g_error_word) & MOE_DEVERR_TIMEOUT))
-    n_tiles = *tiles.num;
+    n_tiles = tiles.uniform_rows > 0 ? (tiles.uniform_rows + GM_BM - 1) / GM_BM : *tiles.num;
   const int U1 = n_tiles * g1.n_blocks, U2 = n_tiles * g2.n_blocks;
   const int nk1 = g1.K / GM_BK, nk2 = g2.K / GM_BK;
   const int ch1 = min(DY_CH1, nk1), ch2 = min(DY_CH2, nk2);
@@ -466,7 +466,8 @@ __global__ void __launch_bounds__(PG_MAX_THREADS, 1)
         const int r = gw * (R / 2) + 4 * u + sub;
         src[u] = nullptr;
         if (r < rows) {
-          const int t = __ldg(tiles.perm + row0 + r) / tiles.k;
+          // the routed pair's token, or (no permutation: one dense layer) the row itself
+          const int t = tiles.perm ? __ldg(tiles.perm + row0 + r) / tiles.k : row0 + r;
           if (t >= 0 && t < tiles.src_rows)
             src[u] = tiles.src + (size_t)t * tiles.ld + 8 * ch;
           else

@@ -771,6 +771,87 @@ moe_status_t moe_forward(const void* x, const void* w_router, const float* route
   return MOE_OK;
 }
 
+// ----------------------------------------------------------------------------- dense MLP
+// The dense GEGLU MLP beside the MoE: the expert FFN kernel with every row in one "expert"
+// (uniform tiles of 128 rows, no permutation), GEMM-2 writing y in token order.
+// Workspace: h [T][I] bf16, then the unit counter and the h-ready counters (one per row
+// tile, plus their total).
+struct DenseLayout {
+  size_t hbuf = 0, counters = 0, total = 0;
+  int n_tiles = 0, n_counters = 0;
+};
+
+DenseLayout dense_layout(int T, int I) {
+  DenseLayout L;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off = align256(off + bytes);
+    return o;
+  };
+  L.n_tiles = (T + GM_BM - 1) / GM_BM;
+  L.hbuf = take(2 * (size_t)T * I);
+  L.n_counters = 1 + L.n_tiles + 1;
+  L.counters = take(sizeof(int32_t) * L.n_counters);
+  L.total = off;
+  return L;
+}
+
+size_t moe_dense_workspace_size(int T, int H, int I) {
+  if (T < 1 || T > 1048576 || H < 64 || H > 16384 || H % 64 || I < 64 || I > 8192 || I % 64)
+    return 0;
+  return dense_layout(T, I).total;
+}
+
+moe_status_t moe_dense_ffn(const void* x, const void* w_gate, const void* w_up,
+                           const void* w_down, int T, int H, int I, void* y, void* workspace,
+                           size_t workspace_bytes, void* stream) {
+  if (T < 0 || H <= 0 || I <= 0) return MOE_ERR_INVALID_ARG;
+  if (T == 0) return MOE_OK;
+  if (!x || !w_gate || !w_up || !w_down || !y || !workspace) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(w_gate) || !aligned16(w_up) || !aligned16(w_down) ||
+      !aligned16(y) || !aligned16(workspace))
+    return MOE_ERR_INVALID_ARG;
+  if (x == y) return MOE_ERR_INVALID_ARG;
+  if (moe_dense_workspace_size(T, H, I) == 0) return MOE_ERR_UNSUPPORTED;
+  const DenseLayout L = dense_layout(T, I);
+  if (workspace_bytes < L.total) return MOE_ERR_NO_WORKSPACE;
+  int dev = 0;
+  DeviceState* d = device_state(&dev);
+  if (!d) return MOE_ERR_CUDA;
+  t_kernels = 0;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  __nv_bfloat16* hbuf = reinterpret_cast<__nv_bfloat16*>(ws + L.hbuf);
+  int32_t* ctr = reinterpret_cast<int32_t*>(ws + L.counters);
+  MOE_TRY_CUDA(cudaMemsetAsync(ctr, 0, sizeof(int32_t) * L.n_counters, st));
+
+  const int R = dy_rows(T, 0);
+  CUtensorMap tm_wg, tm_wu, tm_wd, tm_hr;
+  if (!make_map_slabs(&tm_wg, w_gate, I, H, 1, 64, 2) ||
+      !make_map_slabs(&tm_wu, w_up, I, H, 1, 64, 2) ||
+      !make_map_slabs(&tm_wd, w_down, H, I, 1, 64, 4) || !make_map_2d(&tm_hr, hbuf, I, T, R, 64))
+    return cuda_failed(-1);   // a tensor map could not be encoded
+  const TileList tl{nullptr, nullptr, nullptr, nullptr, T,
+                    nullptr, 1,       static_cast<const __nv_bfloat16*>(x), H, T};
+  const PGemm g1{(I + 127) / 128, H, I, hbuf, I, nullptr, nullptr};
+  const PGemm g2{(H + 255) / 256, I, H, y, H, nullptr, nullptr};
+  int32_t* h_ready = ctr + 1;
+  const DyState dys{ctr, ctr + 1, ctr + 1, nullptr, nullptr};
+  const int G = std::min(std::max(1, d->num_sms), kMaxGemmCtas);
+  const Launch launch{st, false};
+  auto go = [&](auto kernel, int smem) {
+    launch(false, kernel, dim3(G), dim3(pgemm_threads(true)), smem, tm_wg, tm_wu, tm_hr, tm_wd,
+           tl, g1, g2, h_ready, dys);
+  };
+  if (R == 8) go(expert_ffn_dynamic_kernel<8>, dy_smem_bytes<8>());
+  else if (R == 16) go(expert_ffn_dynamic_kernel<16>, dy_smem_bytes<16>());
+  else if (R == 32) go(expert_ffn_dynamic_kernel<32>, dy_smem_bytes<32>());
+  else if (R == 64) go(expert_ffn_dynamic_kernel<64>, dy_smem_bytes<64>());
+  else go(expert_ffn_dynamic_kernel<128>, dy_smem_bytes<128>());
+  return launched();
+}
+
 moe_status_t moe_route_static(const void* x, const void* w_router, const float* router_bias,
                               int T, int H, int E, int k, unsigned flags, int32_t* topk_ids,
                               float* topk_weights, void* stream) {

@@ -100,6 +100,26 @@ def make_weights(cfg: MoEConfig, seed: int = 0) -> dict:
     }
 
 
+DENSE_I = 2112   # intermediate of the dense MLP that runs beside the MoE in every layer
+
+
+def make_dense_weights(H: int, I: int, seed: int = 0) -> dict:
+    """Weights of the dense GEGLU MLP beside the MoE: w_gate, w_up [H,I], w_down [I,H], bf16,
+    N(0, 0.02^2) from their own stream (seed + 1000), so the MoE weights do not change."""
+    rng = np.random.default_rng(seed + 1000)
+    std = np.float32(WEIGHT_STD)
+
+    def draw(shape):
+        a = rng.standard_normal(size=shape, dtype=np.float32)
+        a *= std
+        return bf16_from_f32(a)
+
+    w_gate = draw((H, I))
+    w_up = draw((H, I))
+    w_down = draw((I, H))
+    return {"w_gate": w_gate, "w_up": w_up, "w_down": w_down}
+
+
 def make_x(cfg: MoEConfig, seed: int = 0, T: int | None = None) -> torch.Tensor:
     """Token activations x [T,H] bf16 on the CPU."""
     T = cfg.T if T is None else T

@@ -163,6 +163,28 @@ moe_status_t moe_forward(const void *x, const void *w_router, const float *route
                          void *workspace, size_t workspace_bytes, void *stream);
 
 /*
+ * moe_dense_ffn -- the dense MLP that runs beside the MoE in every layer ("每层同时有 Dense
+ * MLP 和 MoE", gate/up/down, intermediate 2112, GELU: cann-recipes-infer "Gemma-4-26B-A4B
+ * 模型优化报告", §1 模型概况), in the experts' GEGLU form:
+ *
+ *   y = (gelu_tanh(x W_gate) * (x W_up)) W_down
+ *   Precision: bf16 operands, fp32 accumulation; h and y are rounded to bf16.
+ *
+ *   x       (device) bf16 [T, H]
+ *   w_gate, w_up  (device) bf16 [H, I]  (I contiguous)
+ *   w_down  (device) bf16 [I, H]  (H contiguous)
+ *   y       (device) bf16 [T, H]  output (may not alias x)
+ *   workspace (device) >= moe_dense_workspace_size(T, H, I) bytes, else MOE_ERR_NO_WORKSPACE
+ *   Shapes as moe_forward (H, I multiples of 64); T == 0 launches nothing.  One kernel
+ *   launch (the expert FFN kernel with every row in one "expert"); y rows are written in
+ *   token order, so no combine is needed.
+ */
+size_t moe_dense_workspace_size(int T, int H, int I);
+moe_status_t moe_dense_ffn(const void *x, const void *w_gate, const void *w_up,
+                           const void *w_down, int T, int H, int I, void *y, void *workspace,
+                           size_t workspace_bytes, void *stream);
+
+/*
  * moe_route_static -- moe_route for callers that cannot allocate device memory.
  *
  * The pages have no counterpart of this call; it exists for the library's users.  Some

@@ -142,6 +142,18 @@ def expert_ffn(x_row, w_gate, w_up, w_down, e: int) -> np.ndarray:
     return out
 
 
+def dense_ffn(x, w_gate, w_up, w_down, rows=None) -> np.ndarray:
+    """The dense MLP beside the MoE (cann-recipes-infer "Gemma-4-26B-A4B 模型优化报告",
+    §1 模型概况: every layer has a dense gate/up/down MLP, intermediate 2112, GELU), read in
+    the experts' GEGLU form: y[t] = (gelu_tanh(x[t] W_gate) * (x[t] W_up)) W_down, in fp64
+    with no intermediate rounding -- the expert FFN with one expert.
+    w_gate, w_up [H,I]; w_down [I,H] -> y [len(rows) or T, H] float64."""
+    T = x.shape[0]
+    rows = range(T) if rows is None else rows
+    wg, wu, wd = w_gate[None], w_up[None], w_down[None]
+    return np.stack([expert_ffn(x[t], wg, wu, wd, 0) for t in rows])
+
+
 def forward(x, w_router, w_gate, w_up, w_down, k: int, bias=None, renorm: bool = True,
             tokens=None):
     """Whole layer in fp64.  Routes every token; computes y only for `tokens` (all if None).

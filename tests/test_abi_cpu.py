@@ -105,3 +105,18 @@ def test_host_argument_checks(lib):
     assert r(FAKE, FAKE, None, 8, 2816, 128, 8, 0, FAKE, FAKE, FAKE, 16, None) == \
         _abi.MOE_ERR_NO_WORKSPACE
     assert r(FAKE, None, None, 8, 2816, 128, 8, 0, FAKE, FAKE, FAKE, 1 << 30, None) == 1
+
+
+def test_dense_ffn_host_checks(lib):
+    f = lib.moe_dense_ffn
+    # h [T, I] bf16 plus the counters: at least 2 * T * I bytes
+    assert lib.moe_dense_workspace_size(2048, 2816, 2112) >= 2 * 2048 * 2112
+    assert lib.moe_dense_workspace_size(8, 2816, 2100) == 0      # I % 64 != 0
+    assert lib.moe_dense_workspace_size(0, 2816, 2112) == 0
+    w = (FAKE, FAKE, FAKE, FAKE)
+    assert f(*w, 0, 2816, 2112, FAKE + 4096, FAKE, 1 << 30, None) == 0           # T == 0
+    assert f(None, FAKE, FAKE, FAKE, 8, 2816, 2112, FAKE + 4096, FAKE, 1 << 30, None) == 1
+    assert f(*w, 8, 2816, 2112, FAKE, FAKE, 1 << 30, None) == 1                   # y == x
+    assert f(FAKE + 2, FAKE, FAKE, FAKE, 8, 2816, 2112, FAKE + 4096, FAKE, 1 << 30, None) == 1
+    assert f(*w, 8, 2816, 2100, FAKE + 4096, FAKE, 1 << 30, None) == _abi.MOE_ERR_UNSUPPORTED
+    assert f(*w, 8, 2816, 2112, FAKE + 4096, FAKE, 1024, None) == _abi.MOE_ERR_NO_WORKSPACE

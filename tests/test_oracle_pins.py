@@ -232,6 +232,22 @@ def test_single_expert_equals_dense_geglu_ffn():
     assert np.max(np.abs(out["y"] - swapped)) > 1e-3
 
 
+def test_dense_mlp_oracle_is_the_library_formula():
+    """The dense MLP beside the MoE: the oracle's one-expert FFN against the plain formula
+    (torch fp64), on every row and on a subset of rows; gate/up swapped must differ."""
+    rng = np.random.default_rng(12)
+    T, H, I = 5, 128, 192
+    x = rand_bf16(rng, (T, H))
+    wg, wu = rand_bf16(rng, (H, I), 0.02), rand_bf16(rng, (H, I), 0.02)
+    wd = rand_bf16(rng, (I, H), 0.02)
+    ref = dense_ffn_torch(x, wg, wu, wd).numpy()
+    np.testing.assert_allclose(oracle.dense_ffn(x, wg, wu, wd), ref, rtol=1e-12, atol=1e-14)
+    np.testing.assert_allclose(oracle.dense_ffn(x, wg, wu, wd, rows=[3, 0]), ref[[3, 0]],
+                               rtol=1e-12, atol=1e-14)
+    swapped = dense_ffn_torch(x, wu, wg, wd).numpy()
+    assert np.max(np.abs(oracle.dense_ffn(x, wg, wu, wd) - swapped)) > 1e-3
+
+
 def _tiny_layer(seed=10, T=16, H=256, E=8, k=2, I=128):
     rng = np.random.default_rng(seed)
     return dict(x=rand_bf16(rng, (T, H)), w_router=rand_bf16(rng, (H, E), 0.02),
