@@ -1,30 +1,29 @@
-// ffn_dynamic.cuh -- the expert FFN (GEMM-1 + GEGLU, then GEMM-2) of a batch of at most 8
-// tokens in one persistent launch whose CTAs take their work from a shared counter.
+// ffn_dynamic.cuh -- the expert FFN (GEMM-1 + GEGLU, then GEMM-2) of a batch in one
+// persistent launch whose CTAs take their work from a shared counter.
 //
-// A decode step streams the weights of every chosen expert once; the layer's time is that
-// stream.  With a fixed split of the work each CTA streams the same bytes, but SMs do not
-// stream at the same rate, so the slowest CTA sets the end, and GEMM-2 can only start a tile
-// once GEMM-1 has stored it.  Here the work is cut into chunks of a few 64-deep k-steps
-// (CH1 chunks per GEMM-1 unit = (tile, 128 features), CH2 per GEMM-2 unit = (tile, 256
-// columns)), handed out in order from one global counter: every GEMM-1 chunk before any
-// GEMM-2 chunk, so a CTA never waits for work that is handed out after its own.  A chunk's
-// fp32 partial (at most R rows x 256 columns) goes to global memory; the CTA that completes
-// a unit's last chunk adds the unit's partials in chunk order (deterministic whatever the
-// timing), applies GEGLU (GEMM-1) or rounds (GEMM-2) and stores the rows.  GEMM-1 units
-// publish h_ready[tile]; a GEMM-2 chunk's TMA load of h waits for it.
+// The work is cut into units -- (row tile, 128 GEMM-1 features) and (row tile, 256 GEMM-2
+// columns) -- handed out in order from one global counter: every GEMM-1 unit before any
+// GEMM-2 unit, so a CTA never waits for work that is handed out after its own, and SMs that
+// stream faster simply take more units (with a fixed split the slowest SM sets the end).
+// Each unit is summed over its whole K in one TMEM accumulator (two alternate, so one
+// unit's epilogue overlaps the next unit's mainloop) and its epilogue works straight from
+// TMEM: GEGLU and a bf16 store of h (GEMM-1), a bf16 store of the expert output (GEMM-2).
+// A GEMM-1 unit then publishes h_ready[tile]; a GEMM-2 unit issues its W_down loads for
+// the first stages, waits for h_ready, then loads its h rows.
 //
 // Roles as in gemm_persistent.cuh (TMA thread, MMA thread, 4 epilogue warps, 2 gather
-// warps), with A slots of R <= 64 rows (batches of T <= R tokens).  The TMA thread takes chunk ids and
-// passes them to the other roles through a ring of descriptors in shared memory (full /
-// empty mbarriers).  Every wait is bounded.
+// warps), with A slots of R = 8 ... 128 rows (every tile has at most R rows).  The TMA
+// thread takes unit ids and passes them to the other roles through a ring of descriptors
+// in shared memory (full / empty mbarriers).  A tile list from the dispatch describes the
+// routed rows (expert, first sorted row, rows; the A rows gathered from x through perm);
+// without a list (TileList::uniform_rows) the rows of x form one "expert" in 128-row
+// tiles, which is how the dense MLP beside the MoE runs.  Every wait is bounded.
 #pragma once
 #include "gemm_persistent.cuh"
 
 namespace moe {
 
-constexpr int DY_RING = 8;                           // chunk descriptors in flight per CTA
-constexpr int DY_CH1 = 1;                            // chunks per GEMM-1 unit
-constexpr int DY_CH2 = 1;                            // chunks per GEMM-2 unit
+constexpr int DY_RING = 8;                           // unit descriptors in flight per CTA
 
 // R = rows of a tile's A slot: 8, 16, 32 or 64 for batches of T <= R tokens (at most T
 // rows per tile), 128 for any batch (tiles are at most 128 rows).  The MMA reads 128 rows
@@ -37,16 +36,11 @@ struct DyShape {
   static constexpr int STAGE_BYTES = A_BYTES + 4 * GM_SLAB_BYTES;
   static constexpr int STAGES = R <= 32 ? 6 : R == 64 ? 5 : 4;
   static constexpr int ROW_WARPS = (R + 31) / 32;    // epilogue warps holding rows
-  static constexpr int PART_FLOATS = R * 256;        // one chunk's partial tile
   static constexpr int SMEM = 1024 + STAGES * STAGE_BYTES + 2048;
 };
 
 struct DyState {
-  int* next;       // [1] next chunk id; zero at launch
-  int* done1;      // [U1][ROW_WARPS] finished chunks per GEMM-1 unit; zero at launch
-  int* done2;      // [U2][ROW_WARPS] finished chunks per GEMM-2 unit; zero at launch
-  float* part1;    // [U1 * CH1][R][256] (unused when CH1 == 1)
-  float* part2;    // [U2 * CH2][R][256] (unused when CH2 == 1)
+  int* next;       // [1] next unit id; zero at launch
 };
 
 template <int R>
@@ -54,29 +48,16 @@ __host__ __device__ inline int dy_smem_bytes() {
   return DyShape<R>::SMEM;
 }
 
-// A chunk: phase 0 = GEMM-1, 1 = GEMM-2; unit; chunk index j within the unit; k-steps
-// [kb, ke).  A unit of nk k-steps has ch = min(CH, nk) chunks, none empty.
+// A unit: phase 0 = GEMM-1, 1 = GEMM-2; unit index within its GEMM; k-steps [kb, ke).
 struct DyChunk {
-  int phase, unit, j, kb, ke;
+  int phase, unit, kb, ke;
 };
-__device__ __forceinline__ DyChunk dy_decode(int c, int U1, int nk1, int nk2, int ch1,
-                                             int ch2) {
+__device__ __forceinline__ DyChunk dy_decode(int c, int U1, int nk1, int nk2) {
   DyChunk d;
-  const int total1 = U1 * ch1;
-  if (c < total1) {
-    d.phase = 0;
-    d.unit = c / ch1;
-    d.j = c - d.unit * ch1;
-    d.kb = d.j * nk1 / ch1;
-    d.ke = (d.j + 1) * nk1 / ch1;
-  } else {
-    d.phase = 1;
-    const int c2 = c - total1;
-    d.unit = c2 / ch2;
-    d.j = c2 - d.unit * ch2;
-    d.kb = d.j * nk2 / ch2;
-    d.ke = (d.j + 1) * nk2 / ch2;
-  }
+  d.phase = c < U1 ? 0 : 1;
+  d.unit = c < U1 ? c : c - U1;
+  d.kb = 0;
+  d.ke = c < U1 ? nk1 : nk2;
   return d;
 }
 
@@ -94,9 +75,7 @@ __global__ void __launch_bounds__(PG_MAX_THREADS, 1)
   constexpr int STAGE_BYTES = SH::STAGE_BYTES;
   constexpr int DY_STAGES = SH::STAGES;
   constexpr int NRW = SH::ROW_WARPS;
-  constexpr int PARTF = SH::PART_FLOATS;
   constexpr uint32_t TMEM_COLS = 2 * BN;
-  static_assert(DY_CH1 >= 1 && DY_CH2 >= 1, "chunks");
 
   pdl_trigger();
   extern __shared__ uint8_t dsm_raw[];
@@ -115,7 +94,7 @@ __global__ void __launch_bounds__(PG_MAX_THREADS, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 4);
   volatile int* n_issued = reinterpret_cast<volatile int*>(misc + 8);
   volatile int* n_consumed = reinterpret_cast<volatile int*>(misc + 12);
-  volatile int* ring = reinterpret_cast<volatile int*>(misc + 16);   // [DY_RING] chunk ids
+  volatile int* ring = reinterpret_cast<volatile int*>(misc + 16);   // [DY_RING] unit ids
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   // arrivals that release a descriptor: MMA thread, 4 epilogue warps, 2 gather warps
@@ -156,8 +135,7 @@ __global__ void __launch_bounds__(PG_MAX_THREADS, 1)
     n_tiles = tiles.uniform_rows > 0 ? (tiles.uniform_rows + GM_BM - 1) / GM_BM : *tiles.num;
   const int U1 = n_tiles * g1.n_blocks, U2 = n_tiles * g2.n_blocks;
   const int nk1 = g1.K / GM_BK, nk2 = g2.K / GM_BK;
-  const int ch1 = min(DY_CH1, nk1), ch2 = min(DY_CH2, nk2);
-  const int total = U1 * ch1 + U2 * ch2;
+  const int total = U1 + U2;
   const int h_target = NRW * g1.n_blocks;   // one release per (GEMM-1 unit, row warp)
 
   // Read descriptor i (bounded wait); every reader then releases it.  -1 = no more work,
@@ -184,14 +162,14 @@ __global__ void __launch_bounds__(PG_MAX_THREADS, 1)
         ring[r] = stop ? -1 : c;
         mbar_arrive(dfull_bar(r));
         if (stop) break;
-        const int cnext = atomicAdd(dy.next, 1);   // claimed one chunk ahead
-        const DyChunk d = dy_decode(c, U1, nk1, nk2, ch1, ch2);
+        const int cnext = atomicAdd(dy.next, 1);   // claimed one unit ahead
+        const DyChunk d = dy_decode(c, U1, nk1, nk2);
         int e, row0, rows, n0;
         if (d.phase == 0)
           pg_tile_info<EPI_GEGLU, NSLAB>(tiles, g1.n_blocks, d.unit, e, row0, rows, n0);
         else
           pg_tile_info<EPI_STORE, NSLAB>(tiles, g2.n_blocks, d.unit, e, row0, rows, n0);
-        // Issue stage `kc` of the chunk: wait for the slot; B (and, unless deferred, A).
+        // Issue stage `kc` of the unit: wait for the slot; B (and, unless deferred, A).
         auto stage_in = [&](int kc, int qq, bool with_a) -> bool {
           const int s = qq % DY_STAGES;
           if (*abort_flag ||
@@ -256,7 +234,7 @@ __global__ void __launch_bounds__(PG_MAX_THREADS, 1)
           if (c == -2) *abort_flag = 1;
           break;
         }
-        const DyChunk d = dy_decode(c, U1, nk1, nk2, ch1, ch2);
+        const DyChunk d = dy_decode(c, U1, nk1, nk2);
         const int b = i & 1, use = i >> 1;
         if (use >= 1 && !mbar_wait(tempty_bar(b), (use - 1) & 1)) {
           *abort_flag = 1;
@@ -307,7 +285,7 @@ __global__ void __launch_bounds__(PG_MAX_THREADS, 1)
         if (c == -2) *abort_flag = 1;
         break;
       }
-      const DyChunk d = dy_decode(c, U1, nk1, nk2, ch1, ch2);
+      const DyChunk d = dy_decode(c, U1, nk1, nk2);
       const int b = i & 1, use = i >> 1;
       bool got = mbar_wait(tfull_bar(b), use & 1);
       tc_fence_after();
@@ -322,102 +300,32 @@ __global__ void __launch_bounds__(PG_MAX_THREADS, 1)
         pg_tile_info<EPI_GEGLU, NSLAB>(tiles, g.n_blocks, d.unit, e, row0, rows, n0);
       else
         pg_tile_info<EPI_STORE, NSLAB>(tiles, g.n_blocks, d.unit, e, row0, rows, n0);
-      const int nch = d.phase == 0 ? ch1 : ch2;
       const int r_local = quad * 32 + lane;
       const bool row_ok = rows_warp && r_local < rows && r_local < R;
       const uint32_t trow = tmem + b * BN + (static_cast<uint32_t>(quad * 32) << 16);
-      if (nch == 1) {
-        // the whole unit in one chunk: epilogue straight from TMEM
-        if (rows_warp) {
-          const int NC = d.phase == 0 ? BN / 2 : BN;
+      // epilogue straight from TMEM
+      if (rows_warp) {
+        const int NC = d.phase == 0 ? BN / 2 : BN;
 #pragma unroll 1
-          for (int cc = 0; cc < NC; cc += 32) {
-            uint32_t gv[32], uv[32];
-            tmem_ld_32x32b_x32(trow + cc, gv);
-            if (d.phase == 0) tmem_ld_32x32b_x32(trow + BN / 2 + cc, uv);
-            tmem_ld_wait();
-            if (row_ok) {
-              if (d.phase == 0)
-                pg_store32<EPI_GEGLU, NSLAB>(g.out, g.ldo, row0 + r_local, n0, cc, g.N_total,
-                                             reinterpret_cast<const float*>(gv),
-                                             reinterpret_cast<const float*>(uv));
-              else
-                pg_store32<EPI_STORE, NSLAB>(g.out, g.ldo, row0 + r_local, n0, cc, g.N_total,
-                                             reinterpret_cast<const float*>(gv),
-                                             reinterpret_cast<const float*>(uv));
-            }
-          }
-        }
-        tc_fence_before();
-        mbar_arrive(tempty_bar(b));
-      } else {
-        float* part = (d.phase == 0 ? dy.part1 + (size_t)d.unit * DY_CH1 * PARTF
-                                    : dy.part2 + (size_t)d.unit * DY_CH2 * PARTF);
-        if (rows_warp) {
-          // this chunk's partial rows -> global
-          float* prow = part + (size_t)d.j * PARTF + (size_t)r_local * 256;
-#pragma unroll 1
-          for (int cc = 0; cc < BN; cc += 32) {
-            uint32_t v[32];
-            tmem_ld_32x32b_x32(trow + cc, v);
-            tmem_ld_wait();
-            if (row_ok) {
-#pragma unroll
-              for (int k4 = 0; k4 < 8; ++k4)
-                reinterpret_cast<uint4*>(prow + cc)[k4] =
-                    make_uint4(v[4 * k4], v[4 * k4 + 1], v[4 * k4 + 2], v[4 * k4 + 3]);
-            }
-          }
-        }
-        tc_fence_before();
-        mbar_arrive(tempty_bar(b));
-        if (!rows_warp) continue;
-        __threadfence();
-        __syncwarp();
-        int last = 0;
-        if (lane == 0) {
-          int* ctr = (d.phase == 0 ? dy.done1 : dy.done2) + d.unit * NRW + quad;
-          last = atomicAdd(ctr, 1) == nch - 1;
-        }
-        last = __shfl_sync(0xffffffffu, last, 0);
-        if (!last) continue;
-        // the unit's last chunk: add the partials in chunk order and finish the rows
-        __threadfence();
-        if (row_ok) {
-          constexpr int NC1 = BN / 2;
-          const int NC = d.phase == 0 ? NC1 : BN;
-#pragma unroll 1
-          for (int cc = 0; cc < NC; cc += 32) {
-            float gsum[32], usum[32];
-#pragma unroll
-            for (int k2 = 0; k2 < 32; ++k2) gsum[k2] = usum[k2] = 0.f;
-            for (int jj = 0; jj < nch; ++jj) {
-              const float* src = part + (size_t)jj * PARTF + (size_t)r_local * 256;
-#pragma unroll
-              for (int k4 = 0; k4 < 8; ++k4) {
-                const float4 a4 = __ldcg(reinterpret_cast<const float4*>(src + cc) + k4);
-                gsum[4 * k4] += a4.x;
-                gsum[4 * k4 + 1] += a4.y;
-                gsum[4 * k4 + 2] += a4.z;
-                gsum[4 * k4 + 3] += a4.w;
-                if (d.phase == 0) {
-                  const float4 bq = __ldcg(reinterpret_cast<const float4*>(src + NC1 + cc) + k4);
-                  usum[4 * k4] += bq.x;
-                  usum[4 * k4 + 1] += bq.y;
-                  usum[4 * k4 + 2] += bq.z;
-                  usum[4 * k4 + 3] += bq.w;
-                }
-              }
-            }
+        for (int cc = 0; cc < NC; cc += 32) {
+          uint32_t gv[32], uv[32];
+          tmem_ld_32x32b_x32(trow + cc, gv);
+          if (d.phase == 0) tmem_ld_32x32b_x32(trow + BN / 2 + cc, uv);
+          tmem_ld_wait();
+          if (row_ok) {
             if (d.phase == 0)
-              pg_store32<EPI_GEGLU, NSLAB>(g.out, g.ldo, row0 + r_local, n0, cc, g.N_total, gsum,
-                                           usum);
+              pg_store32<EPI_GEGLU, NSLAB>(g.out, g.ldo, row0 + r_local, n0, cc, g.N_total,
+                                           reinterpret_cast<const float*>(gv),
+                                           reinterpret_cast<const float*>(uv));
             else
-              pg_store32<EPI_STORE, NSLAB>(g.out, g.ldo, row0 + r_local, n0, cc, g.N_total, gsum,
-                                           usum);
+              pg_store32<EPI_STORE, NSLAB>(g.out, g.ldo, row0 + r_local, n0, cc, g.N_total,
+                                           reinterpret_cast<const float*>(gv),
+                                           reinterpret_cast<const float*>(uv));
           }
         }
       }
+      tc_fence_before();
+      mbar_arrive(tempty_bar(b));
       if (d.phase == 0 && rows_warp) {
         // publish this warp's h rows of the unit to the GEMM-2 TMA loads
         fence_proxy_async_global();
@@ -431,8 +339,8 @@ __global__ void __launch_bounds__(PG_MAX_THREADS, 1)
     }
   } else {
     // -------------------------------------------------------------- A-row gather (warps 6-7)
-    // GEMM-1 chunks: the <= R rows of the tile, 16-byte cp.async into the 128-byte-swizzled
-    // slot (chunk c of row r at byte 128 r + 16 (c ^ r)).  GEMM-2 chunks: nothing (the TMA
+    // GEMM-1 units: the <= R rows of the tile, 16-byte cp.async into the 128-byte-swizzled
+    // slot (chunk c of row r at byte 128 r + 16 (c ^ r)).  GEMM-2 units: nothing (the TMA
     // thread arrives in their place), but the stage count must follow.
     const int gw = warp - 6, sub = lane >> 3, ch = lane & 7;
     int q = 0;
@@ -446,7 +354,7 @@ __global__ void __launch_bounds__(PG_MAX_THREADS, 1)
         if (c == -2) *abort_flag = 1;
         break;
       }
-      const DyChunk d = dy_decode(c, U1, nk1, nk2, ch1, ch2);
+      const DyChunk d = dy_decode(c, U1, nk1, nk2);
       if (d.phase == 1) {
         q += d.ke - d.kb;
         continue;

@@ -142,8 +142,8 @@ struct Layout {
   size_t dsync = 0;   // one-launch dispatch: arrivals, flag
   size_t tile_num = 0, tile_expert = 0, tile_row0 = 0, tile_rows = 0;
   size_t xp = 0, hbuf = 0, obuf = 0;
-  size_t partials = 0, partials2 = 0, counters = 0, dy_part1 = 0, dy_part2 = 0;
-  int dy_u1 = 0, dy_u2 = 0, dy_ctr = 0;   // dynamic small-batch FFN: units, counter offset
+  size_t partials = 0, partials2 = 0, counters = 0;
+  int dy_ctr = 0;   // dynamic FFN: offset of its unit counter among the counters
   int n_counters = 0;
   size_t total = 0;
 };
@@ -203,18 +203,9 @@ Layout make_layout(int T, int H, int E, int I, int k, unsigned flags, bool forwa
     }
     L.n_counters = 2 * kStreamKCounters + L.max_tiles + 1;
     if (R > 0) {
-      // dynamic FFN: the unit counter, and per-chunk partial tiles and per-(unit, row warp)
-      // chunk counts when units are cut in chunks.  A tile has >= 1 pair: at most
-      // min(max_tiles, P) tiles.
-      const int mt = (int)std::min<long long>(L.max_tiles, P);
-      const int nrw = (R + 31) / 32;
-      L.dy_u1 = mt * ((I + 127) / 128);
-      L.dy_u2 = mt * ((H + 255) / 256);
-      if (DY_CH1 > 1) L.dy_part1 = take(sizeof(float) * (size_t)L.dy_u1 * DY_CH1 * R * 256);
-      if (DY_CH2 > 1) L.dy_part2 = take(sizeof(float) * (size_t)L.dy_u2 * DY_CH2 * R * 256);
+      // dynamic FFN: its unit counter
       L.dy_ctr = L.n_counters;
-      // per-(unit, row warp) chunk counts only when units are cut in several chunks
-      L.n_counters += 1 + (DY_CH1 > 1 ? L.dy_u1 * nrw : 0) + (DY_CH2 > 1 ? L.dy_u2 * nrw : 0);
+      L.n_counters += 1;
     }
     L.counters = take(sizeof(int32_t) * L.n_counters);
   }
@@ -726,10 +717,7 @@ moe_status_t moe_forward(const void* x, const void* w_router, const float* route
       CUtensorMap tm_hr;
       if (!make_map_2d(&tm_hr, hbuf, I, P, R, 64)) return cuda_failed(-1);
       int32_t* dctr = gemm_counters + L.dy_ctr;
-      const int nrw = (R + 31) / 32;
-      const DyState dys{dctr, dctr + 1, dctr + 1 + (DY_CH1 > 1 ? L.dy_u1 * nrw : 0),
-                        reinterpret_cast<float*>(ws + L.dy_part1),
-                        reinterpret_cast<float*>(ws + L.dy_part2)};
+      const DyState dys{dctr};
       auto go = [&](auto kernel, int smem) {
         launch(true, kernel, dim3(G), dim3(pgemm_threads(true)), smem, tm_wg, tm_wu, tm_hr, tm_wd,
                tl, g1, g2, h_ready, dys);
@@ -837,7 +825,7 @@ moe_status_t moe_dense_ffn(const void* x, const void* w_gate, const void* w_up,
   const PGemm g1{(I + 127) / 128, H, I, hbuf, I, nullptr, nullptr};
   const PGemm g2{(H + 255) / 256, I, H, y, H, nullptr, nullptr};
   int32_t* h_ready = ctr + 1;
-  const DyState dys{ctr, ctr + 1, ctr + 1, nullptr, nullptr};
+  const DyState dys{ctr};
   const int G = std::min(std::max(1, d->num_sms), kMaxGemmCtas);
   const Launch launch{st, false};
   auto go = [&](auto kernel, int smem) {
