@@ -12,6 +12,9 @@
 // Eight warps put two on each SM sub-partition, whose 16K registers then allow up to 255
 // per thread (ten warps would put three on one and cap every thread at 168).
 //
+// The warp roles, operand layouts and epilogue helpers here are shared with the default,
+// dynamically scheduled expert FFN (ffn_dynamic.cuh).  This file's kernel is the statically
+// scheduled form, run when a flag asks for it (one launch for both GEMMs, or two):
 // Schedule over U = tiles x column blocks units of nk k-steps each, G CTAs:
 //   * whole units, round robin (unit g + i*G), for all but the last one-to-two waves;
 //   * the remaining R units (G <= R < 2G, or all of them when U < 2G) are cut into G equal
