@@ -15,6 +15,11 @@
 //      When a decision is closer than that (a near-tie or an exact tie), the warp
 //      recomputes every logit of that token sequentially in ascending h -- the same
 //      sequence of roundings as the ascending-order definition -- and ranks those.
+// Large batches take the screen path at the end of this file instead: a tensor-core screen
+// picks each token's candidates, whose logits are recomputed first as fp32 pair sums of
+// the exact products (bounded error, one fp32 -> fp64 conversion per pair), then -- only
+// for the candidates of decisions those cannot settle -- in fp64, then, if still too close,
+// by the same sequential ascending-h chains.
 #pragma once
 #include <cfloat>
 #include <climits>
