@@ -52,13 +52,13 @@ def peaks() -> dict:
 
 # ----------------------------------------------------------------------------- clocks
 class ClockSampler:
-    """SM clock and clock-event reasons sampled through NVML every few ms while the timed
-    region runs (reads only; nothing is set)."""
+    """SM clock and clock-event reasons sampled through NVML every millisecond while the
+    timed region runs (reads only; nothing is set)."""
 
     REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
                0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown"}
 
-    def __init__(self, device: torch.device, period_s: float = 0.005):
+    def __init__(self, device: torch.device, period_s: float = 0.001):
         self.period = period_s
         self.samples: list[tuple[float, int, int]] = []
         self.h = None
@@ -187,6 +187,132 @@ def job_throughput(world: int, tokens_per_rank: int, max_ms: float) -> float:
     return world * tokens_per_rank / (max_ms * 1e-3)
 
 
+TENSOR_BOUND_CONFIGS = ("skewed", "sweep_T32768")
+
+
+def time_layer(moe, cfg, args, g, x_cpu, dev, stream, flush_l2, dist, e2e: bool) -> dict:
+    """Time args.steps graph replays of one moe_forward over cfg's batch (L2 flushed, untimed,
+    before every step); per-stage device times from a second graph with the library's stage
+    events; optionally the end-to-end time with pinned host buffers.  Device times are the
+    max over ranks."""
+    x = x_cpu.to(dev)
+    y0, aux = moe.forward(x, g["w_router"], g["w_gate"], g["w_up"], g["w_down"], cfg.k,
+                          bias=g["bias"], aux=True, tiles=args.tiles)
+    if moe.sync_status() != 0:
+        raise SystemExit(f"device status not OK after the first forward ({cfg.name})")
+    counts = aux["expert_counts"].cpu().numpy()
+    acc = algorithmic(cfg, counts, g["bias"] is not None)
+    rstats = moe.router_stats(aux)
+    del aux
+
+    # The step as a serving loop runs it: one captured moe_forward per batch (graph replay).
+    graph = moe.ForwardGraph(x, g["w_router"], g["w_gate"], g["w_up"], g["w_down"], cfg.k,
+                             bias=g["bias"], tiles=args.tiles)
+    for _ in range(args.warmup):
+        flush_l2()
+        graph.replay()
+    torch.cuda.synchronize()
+    if not torch.equal(graph.y, y0):
+        raise SystemExit(f"graph replay differs from the direct call ({cfg.name})")
+    del y0
+
+    # ---- timed region: K steps, L2 flushed (untimed) before each
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    clocks = ClockSampler(dev)
+    clocks.start()
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    for i in range(args.steps):
+        flush_l2()
+        ev[i][0].record(stream)
+        graph.replay()
+        ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    clk = clocks.stop()
+    step_ms = [a.elapsed_time(b) for a, b in ev]
+    ms = sum(step_ms) / len(step_ms)
+    if moe.sync_status() != 0:
+        raise SystemExit(f"device status not OK after the timed steps ({cfg.name})")
+
+    # ---- per-stage device times: a graph of the same call with the library's stage events
+    pgraph = moe.ForwardGraph(x, g["w_router"], g["w_gate"], g["w_up"], g["w_down"], cfg.k,
+                              bias=g["bias"], profile=True, tiles=args.tiles)
+    stage_acc: dict[str, list[float]] = {}
+    try:
+        for _ in range(max(3, min(args.steps, 20))):
+            flush_l2()
+            pgraph.replay()
+            for k, v in moe.last_stage_times().items():
+                stage_acc.setdefault(k, []).append(v)
+    except RuntimeError as exc:
+        print(f"stage timing unavailable: {exc}", file=sys.stderr)
+    stages = {k: sum(v) / len(v) for k, v in stage_acc.items()}
+    del pgraph
+
+    e2e_ms = None
+    if e2e:
+        # ---- end to end through the public API with host buffers (pinned), L2 flushed
+        x_host = x_cpu.pin_memory()
+        y_host = torch.empty((cfg.T, cfg.H), dtype=torch.bfloat16).pin_memory()
+        e2e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                  for _ in range(args.steps)]
+        for i in range(args.warmup + args.steps):
+            flush_l2()
+            if i >= args.warmup:
+                e2e_ev[i - args.warmup][0].record(stream)
+            graph.x.copy_(x_host, non_blocking=True)
+            graph.replay()
+            y_host.copy_(graph.y, non_blocking=True)
+            if i >= args.warmup:
+                e2e_ev[i - args.warmup][1].record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = sum(a.elapsed_time(b) for a, b in e2e_ev) / args.steps
+    kernels = graph.kernels_per_replay
+    del graph
+    vals = [ms, stages.get("expert_ffn", 0.0)] + ([e2e_ms] if e2e else [])
+    vals = max_over_ranks(vals, dist, dev)
+    ms, ffn_ms = vals[0], vals[1]
+    if e2e:
+        e2e_ms = vals[2]
+    if "expert_ffn" in stages:
+        stages["expert_ffn"] = ffn_ms
+    return {"ms": ms, "e2e_ms": e2e_ms, "acc": acc, "rstats": rstats, "stages": stages,
+            "clocks": clk, "kernels": kernels, "step_ms": step_ms}
+
+
+def tensor_bound_entry(cfg, m: dict, world: int, pk: dict) -> dict:
+    """Summary of one large-batch config: tokens/s, the expert FFN's tensor throughput
+    against the measured burst and sustained bf16 peaks, and the whole step's."""
+    acc = m["acc"]
+    kf = acc["gemm1_flops"] + acc["gemm2_flops"]
+    ffn_ms = m["stages"].get("expert_ffn", 0.0)
+    ffn_tf = kf / (ffn_ms * 1e-3) / 1e12 if ffn_ms > 0 else None
+    step_tf = acc["step_flops"] / (m["ms"] * 1e-3) / 1e12
+    return {
+        "workload": f"{cfg.name}: T={cfg.T} H={cfg.H} E={cfg.E} k={cfg.k} I={cfg.I}"
+                    + (" (router bias b_e = 2 ln(1/(e+1)))" if cfg.skew_bias else ""),
+        "value": job_throughput(world, cfg.T, m["ms"]), "unit": UNIT,
+        "ms_per_step": m["ms"],
+        "expert_ffn": {"kernel": ffn_kernel_name(cfg.T, "auto"), "ms": ffn_ms,
+                       "achieved_tflops": ffn_tf,
+                       "frac_of_burst": None if ffn_tf is None else ffn_tf / pk["bf16_tflops"],
+                       "frac_of_sustained": None if ffn_tf is None
+                       else ffn_tf / pk["bf16_tflops_sustained"],
+                       "algorithmic_flops": kf},
+        "step_tensor_frac": step_tf * 1e12 / (pk["bf16_tflops"] * 1e12),
+        "active_experts": acc["active_experts"],
+        "stages_ms": m["stages"],
+        "router_stats": m["rstats"],
+        "clocks": m["clocks"],
+        "gpu_launches": m["kernels"] * m["_steps"],
+    }
+
+
+
 # ----------------------------------------------------------------------------- arms
 def run_reference(args, cfg) -> None:
     import oracle
@@ -264,7 +390,6 @@ def run_native(args, cfg) -> None:
     d = wl.make_weights(cfg)
     x_cpu = wl.make_x(cfg, seed=rank)
     g = {k: (v.to(dev) if v is not None else None) for k, v in d.items()}
-    x = x_cpu.to(dev)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     flush_rd = torch.zeros(L2_FLUSH_BYTES // 8, dtype=torch.int64, device=dev)
     stream = torch.cuda.current_stream()
@@ -274,80 +399,19 @@ def run_native(args, cfg) -> None:
         flush.zero_()
         flush_rd.max()
 
-    y0, aux = moe.forward(x, g["w_router"], g["w_gate"], g["w_up"], g["w_down"], cfg.k,
-                          bias=g["bias"], aux=True, tiles=args.tiles)
-    if moe.sync_status() != 0:
-        raise SystemExit("device status not OK after the first forward")
-    counts = aux["expert_counts"].cpu().numpy()
-    acc = algorithmic(cfg, counts, d["bias"] is not None)
-    rstats = moe.router_stats(aux)
-
-    # The step as a serving loop runs it: one captured moe_forward per batch (graph replay).
-    graph = moe.ForwardGraph(x, g["w_router"], g["w_gate"], g["w_up"], g["w_down"], cfg.k,
-                             bias=g["bias"], tiles=args.tiles)
-    for _ in range(args.warmup):
-        flush_l2()
-        graph.replay()
-    torch.cuda.synchronize()
-    if not torch.equal(graph.y, y0):
-        raise SystemExit("graph replay differs from the direct call")
-
-    # ---- timed region: K steps, L2 flushed (untimed) before each
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-          for _ in range(args.steps)]
-    clocks = ClockSampler(dev)
-    clocks.start()
-    if dist:
-        dist.barrier()
-    torch.cuda.synchronize()
-    for i in range(args.steps):
-        flush_l2()
-        ev[i][0].record(stream)
-        graph.replay()
-        ev[i][1].record(stream)
-    torch.cuda.synchronize()
-    if dist:
-        dist.barrier()
-    clk = clocks.stop()
-    step_ms = [a.elapsed_time(b) for a, b in ev]
-    ms = sum(step_ms) / len(step_ms)
-    if moe.sync_status() != 0:
-        raise SystemExit("device status not OK after the timed steps")
-
-    # ---- per-stage device times: a graph of the same call with the library's stage events
-    pgraph = moe.ForwardGraph(x, g["w_router"], g["w_gate"], g["w_up"], g["w_down"], cfg.k,
-                              bias=g["bias"], profile=True, tiles=args.tiles)
-    stage_acc: dict[str, list[float]] = {}
-    try:
-        for _ in range(max(3, min(args.steps, 20))):
-            flush_l2()
-            pgraph.replay()
-            for k, v in moe.last_stage_times().items():
-                stage_acc.setdefault(k, []).append(v)
-    except RuntimeError as exc:
-        print(f"stage timing unavailable: {exc}", file=sys.stderr)
-    stages = {k: sum(v) / len(v) for k, v in stage_acc.items()}
-    del pgraph
-
-    # ---- end to end through the public API with host buffers (pinned), L2 flushed
-    x_host = x_cpu.pin_memory()
-    y_host = torch.empty((cfg.T, cfg.H), dtype=torch.bfloat16).pin_memory()
-    e2e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-              for _ in range(args.steps)]
-    for i in range(args.warmup + args.steps):
-        flush_l2()
-        if i >= args.warmup:
-            e2e_ev[i - args.warmup][0].record(stream)
-        graph.x.copy_(x_host, non_blocking=True)
-        graph.replay()
-        y_host.copy_(graph.y, non_blocking=True)
-        if i >= args.warmup:
-            e2e_ev[i - args.warmup][1].record(stream)
-    torch.cuda.synchronize()
-    e2e_ms = sum(a.elapsed_time(b) for a, b in e2e_ev) / args.steps
-
-    ms, e2e_ms = max_over_ranks([ms, e2e_ms], dist, dev)
-
+    m = time_layer(moe, cfg, args, g, x_cpu, dev, stream, flush_l2, dist, e2e=True)
+    ms, e2e_ms = m["ms"], m["e2e_ms"]
+    acc, rstats, stages, clk, graph_kernels, step_ms = (m["acc"], m["rstats"], m["stages"],
+                                                       m["clocks"], m["kernels"], m["step_ms"])
+    # the tensor-bound configs (large batches), same timing rules, reported beside the line
+    tensor_bound = []
+    if not args.no_tensor_bound:
+        for name in TENSOR_BOUND_CONFIGS:
+            c2 = wl.CONFIGS[name]
+            g2 = dict(g, bias=(wl.skew_bias(c2.E).to(dev) if c2.skew_bias else None))
+            m2 = time_layer(moe, c2, args, g2, wl.make_x(c2, seed=rank), dev, stream, flush_l2,
+                            dist, e2e=False)
+            tensor_bound.append((c2, m2))
     if rank == 0:
         pk = peaks()
         # the dominant kernel: the expert FFN (GEMM-1 + GEGLU and GEMM-2; one launch unless
@@ -399,10 +463,15 @@ def run_native(args, cfg) -> None:
             "e2e": {"value": job_throughput(world, cfg.T, e2e_ms), "unit": UNIT,
                     "h2d_bytes_per_step": cfg.T * cfg.H * 2,
                     "d2h_bytes_per_step": cfg.T * cfg.H * 2},
-            "gpu_launches": graph.kernels_per_replay * args.steps,
+            "gpu_launches": graph_kernels * args.steps,
             "clocks": clk,
             "step_ms_p10_p50_p90": [float(np.percentile(step_ms, q)) for q in (10, 50, 90)],
         }
+        if tensor_bound:
+            line["tensor_bound"] = []
+            for c2, m2 in tensor_bound:
+                m2["_steps"] = args.steps
+                line["tensor_bound"].append(tensor_bound_entry(c2, m2, world, pk))
         if not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline(cfg, d, x_cpu, args.cpu_seconds)
         print(json.dumps(line), flush=True)
@@ -532,6 +601,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--tiles", default="auto", choices=["auto", "decode", "prefill", "fused", "unfused"],
                     help="expert-GEMM tile family (default: the library's choice)")
+    ap.add_argument("--no-tensor-bound", action="store_true",
+                    help="skip the large-batch (tensor-bound) configs reported beside the line")
     ap.add_argument("--dense", action="store_true",
                     help="time the dense GEGLU MLP beside the MoE instead of the MoE layer")
     args = ap.parse_args()

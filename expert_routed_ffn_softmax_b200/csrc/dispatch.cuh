@@ -385,23 +385,33 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const uint4* __restric
                                                           int k, int nvec, uint4* __restrict__ xp) {
   pdl_trigger();
   pdl_wait();
+  // After a timeout upstream perm may be stale: skip the work (the error word says why).
+  if (*reinterpret_cast<volatile unsigned*>(&g_error_word) & MOE_DEVERR_TIMEOUT) return;
   const long long total = (long long)P * nvec;
   const long long nthr = (long long)gridDim.x * blockDim.x;
   for (long long b0 = (long long)blockIdx.x * blockDim.x + threadIdx.x; b0 < total;
        b0 += 8 * nthr) {
     uint4 r[8];
+    bool ok[8];
 #pragma unroll
     for (int u = 0; u < 8; ++u) {
       const long long idx = b0 + u * nthr;
+      ok[u] = false;
       if (idx < total) {
         const int pos = (int)(idx / nvec), v = (int)(idx - (long long)pos * nvec);
-        r[u] = x[(size_t)(perm[pos] / k) * nvec + v];
+        const int q = perm[pos];
+        if ((unsigned)q < (unsigned)P) {   // the source row t = q / k is then < T
+          r[u] = x[(size_t)(q / k) * nvec + v];
+          ok[u] = true;
+        } else {
+          raise_error(MOE_DEVERR_BAD_INDEX);
+        }
       }
     }
 #pragma unroll
     for (int u = 0; u < 8; ++u) {
       const long long idx = b0 + u * nthr;
-      if (idx < total) xp[idx] = r[u];
+      if (ok[u]) xp[idx] = r[u];
     }
   }
 }
@@ -417,7 +427,10 @@ __global__ void __launch_bounds__(256) combine_kernel(const uint4* __restrict__ 
                                                       int nvec, uint4* __restrict__ y) {
   pdl_trigger();
   pdl_wait();
+  // After a timeout upstream inv may be stale: skip the work (the error word says why).
+  if (*reinterpret_cast<volatile unsigned*>(&g_error_word) & MOE_DEVERR_TIMEOUT) return;
   const int lane = threadIdx.x & 31;
+  const int P = T * k;
   const int nch = (nvec + kCombineChunkVec - 1) / kCombineChunkVec;
   const long long items = (long long)T * nch;
   const long long nwarps = (long long)gridDim.x * (blockDim.x >> 5);
@@ -429,6 +442,11 @@ __global__ void __launch_bounds__(256) combine_kernel(const uint4* __restrict__ 
     if (lane < k) {
       myp = __ldg(inv + (size_t)t * k + lane);
       myw = __ldg(w + (size_t)t * k + lane);
+      if ((unsigned)myp >= (unsigned)P) {   // never written so: read nothing for this slot
+        raise_error(MOE_DEVERR_BAD_INDEX);
+        myp = 0;
+        myw = 0.f;
+      }
     }
     int pos[8];
     float wj[8];

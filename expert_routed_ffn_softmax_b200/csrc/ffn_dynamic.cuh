@@ -61,11 +61,22 @@ __device__ __forceinline__ DyChunk dy_decode(int c, int U1, int nk1, int nk2) {
   return d;
 }
 
-// tmH: h rows, box R rows x 64 columns.
+// A GEMM-1 column block covers 128 features: 128 gate and 128 up columns in one N = 256
+// MMA.  When I % 128 == 64 the last block has 64 features; it runs an N = 128 MMA (gate in
+// slab 0, up in slab 1, loaded with the one-slab maps tmWg1 / tmWu1) instead of computing
+// 128 zero-filled columns.
+__device__ __forceinline__ bool dy_narrow_block(const DyChunk& d, const PGemm& g1) {
+  return d.phase == 0 && (g1.N_total & 127) != 0 && d.unit % g1.n_blocks == g1.n_blocks - 1;
+}
+
+// tmH: h rows, box R rows x 64 columns.  tmWg / tmWu: two-slab boxes; tmWg1 / tmWu1: one-slab
+// boxes (the narrow last GEMM-1 block).
 template <int R>
 __global__ void __launch_bounds__(PG_MAX_THREADS, 1)
     expert_ffn_dynamic_kernel(const __grid_constant__ CUtensorMap tmWg,
                               const __grid_constant__ CUtensorMap tmWu,
+                              const __grid_constant__ CUtensorMap tmWg1,
+                              const __grid_constant__ CUtensorMap tmWu1,
                               const __grid_constant__ CUtensorMap tmH,
                               const __grid_constant__ CUtensorMap tmWd, TileList tiles,
                               PGemm g1, PGemm g2, int* __restrict__ h_ready, DyState dy) {
@@ -118,6 +129,10 @@ __global__ void __launch_bounds__(PG_MAX_THREADS, 1)
     fence_barrier_init();
     tma_prefetch_desc(&tmWg);
     tma_prefetch_desc(&tmWu);
+    if (g1.N_total & 127) {
+      tma_prefetch_desc(&tmWg1);
+      tma_prefetch_desc(&tmWu1);
+    }
     tma_prefetch_desc(&tmH);
     tma_prefetch_desc(&tmWd);
   }
@@ -169,6 +184,7 @@ __global__ void __launch_bounds__(PG_MAX_THREADS, 1)
           pg_tile_info<EPI_GEGLU, NSLAB>(tiles, g1.n_blocks, d.unit, e, row0, rows, n0);
         else
           pg_tile_info<EPI_STORE, NSLAB>(tiles, g2.n_blocks, d.unit, e, row0, rows, n0);
+        const bool narrow = dy_narrow_block(d, g1);
         // Issue stage `kc` of the unit: wait for the slot; B (and, unless deferred, A).
         auto stage_in = [&](int kc, int qq, bool with_a) -> bool {
           const int s = qq % DY_STAGES;
@@ -179,7 +195,11 @@ __global__ void __launch_bounds__(PG_MAX_THREADS, 1)
           }
           const uint32_t sA = base + s * STAGE_BYTES;
           const uint32_t sB = sA + A_BYTES;
-          if (d.phase == 0) {
+          if (narrow) {
+            mbar_arrive_expect_tx(full_bar(s), 2 * GM_SLAB_BYTES);
+            tma_load_4d(sB, &tmWg1, full_bar(s), 0, kc * GM_BK, n0 / 64, e);
+            tma_load_4d(sB + GM_SLAB_BYTES, &tmWu1, full_bar(s), 0, kc * GM_BK, n0 / 64, e);
+          } else if (d.phase == 0) {
             mbar_arrive_expect_tx(full_bar(s), NSLAB * GM_SLAB_BYTES);
             tma_load_4d(sB, &tmWg, full_bar(s), 0, kc * GM_BK, n0 / 64, e);
             tma_load_4d(sB + (NSLAB / 2) * GM_SLAB_BYTES, &tmWu, full_bar(s), 0, kc * GM_BK,
@@ -225,7 +245,8 @@ __global__ void __launch_bounds__(PG_MAX_THREADS, 1)
   } else if (warp == 1) {
     if (lane == 0) {
       // ------------------------------------------------------------ MMA issuer
-      constexpr uint32_t idesc = idesc_bf16_f32(GM_BM, BN, false, true);
+      constexpr uint32_t idesc_full = idesc_bf16_f32(GM_BM, BN, false, true);
+      constexpr uint32_t idesc_narrow = idesc_bf16_f32(GM_BM, BN / 2, false, true);
       int q = 0;
       for (int i = 0;; ++i) {
         const int c = read_desc(i);
@@ -235,6 +256,7 @@ __global__ void __launch_bounds__(PG_MAX_THREADS, 1)
           break;
         }
         const DyChunk d = dy_decode(c, U1, nk1, nk2);
+        const uint32_t idesc = dy_narrow_block(d, g1) ? idesc_narrow : idesc_full;
         const int b = i & 1, use = i >> 1;
         if (use >= 1 && !mbar_wait(tempty_bar(b), (use - 1) & 1)) {
           *abort_flag = 1;
@@ -305,12 +327,14 @@ __global__ void __launch_bounds__(PG_MAX_THREADS, 1)
       const uint32_t trow = tmem + b * BN + (static_cast<uint32_t>(quad * 32) << 16);
       // epilogue straight from TMEM
       if (rows_warp) {
-        const int NC = d.phase == 0 ? BN / 2 : BN;
+        // GEMM-1: gate columns [0, NC), up columns [NC, 2 NC) of the accumulator
+        const bool narrow = dy_narrow_block(d, g1);
+        const int NC = d.phase == 0 ? (narrow ? BN / 4 : BN / 2) : BN;
 #pragma unroll 1
         for (int cc = 0; cc < NC; cc += 32) {
           uint32_t gv[32], uv[32];
           tmem_ld_32x32b_x32(trow + cc, gv);
-          if (d.phase == 0) tmem_ld_32x32b_x32(trow + BN / 2 + cc, uv);
+          if (d.phase == 0) tmem_ld_32x32b_x32(trow + NC + cc, uv);
           tmem_ld_wait();
           if (row_ok) {
             if (d.phase == 0)

@@ -713,14 +713,18 @@ moe_status_t moe_forward(const void* x, const void* w_router, const float* route
     const PGemm g1{(I + 127) / 128, H, I, hbuf, I, partials, ctr1};
     const PGemm g2{(H + 255) / 256, I, H, obuf, H, partials2, ctr2};
     if (const int R = dy_rows(T, flags); R > 0) {
-      // at most R rows per tile, whole units handed out from a shared counter
-      CUtensorMap tm_hr;
-      if (!make_map_2d(&tm_hr, hbuf, I, P, R, 64)) return cuda_failed(-1);
+      // at most R rows per tile, whole units handed out from a shared counter; one-slab
+      // weight maps for a narrow last GEMM-1 block (I % 128 == 64)
+      CUtensorMap tm_hr, tm_wg1, tm_wu1;
+      if (!make_map_2d(&tm_hr, hbuf, I, P, R, 64) ||
+          !make_map_slabs(&tm_wg1, w_gate, I, H, E, 64, 1) ||
+          !make_map_slabs(&tm_wu1, w_up, I, H, E, 64, 1))
+        return cuda_failed(-1);
       int32_t* dctr = gemm_counters + L.dy_ctr;
       const DyState dys{dctr};
       auto go = [&](auto kernel, int smem) {
-        launch(true, kernel, dim3(G), dim3(pgemm_threads(true)), smem, tm_wg, tm_wu, tm_hr, tm_wd,
-               tl, g1, g2, h_ready, dys);
+        launch(true, kernel, dim3(G), dim3(pgemm_threads(true)), smem, tm_wg, tm_wu, tm_wg1,
+               tm_wu1, tm_hr, tm_wd, tl, g1, g2, h_ready, dys);
       };
       if (R == 8) go(expert_ffn_dynamic_kernel<8>, dy_smem_bytes<8>());
       else if (R == 16) go(expert_ffn_dynamic_kernel<16>, dy_smem_bytes<16>());
@@ -815,9 +819,11 @@ moe_status_t moe_dense_ffn(const void* x, const void* w_gate, const void* w_up,
   MOE_TRY_CUDA(cudaMemsetAsync(ctr, 0, sizeof(int32_t) * L.n_counters, st));
 
   const int R = dy_rows(T, 0);
-  CUtensorMap tm_wg, tm_wu, tm_wd, tm_hr;
+  CUtensorMap tm_wg, tm_wu, tm_wg1, tm_wu1, tm_wd, tm_hr;
   if (!make_map_slabs(&tm_wg, w_gate, I, H, 1, 64, 2) ||
       !make_map_slabs(&tm_wu, w_up, I, H, 1, 64, 2) ||
+      !make_map_slabs(&tm_wg1, w_gate, I, H, 1, 64, 1) ||
+      !make_map_slabs(&tm_wu1, w_up, I, H, 1, 64, 1) ||
       !make_map_slabs(&tm_wd, w_down, H, I, 1, 64, 4) || !make_map_2d(&tm_hr, hbuf, I, T, R, 64))
     return cuda_failed(-1);   // a tensor map could not be encoded
   const TileList tl{nullptr, nullptr, nullptr, nullptr, T,
@@ -829,8 +835,8 @@ moe_status_t moe_dense_ffn(const void* x, const void* w_gate, const void* w_up,
   const int G = std::min(std::max(1, d->num_sms), kMaxGemmCtas);
   const Launch launch{st, false};
   auto go = [&](auto kernel, int smem) {
-    launch(false, kernel, dim3(G), dim3(pgemm_threads(true)), smem, tm_wg, tm_wu, tm_hr, tm_wd,
-           tl, g1, g2, h_ready, dys);
+    launch(false, kernel, dim3(G), dim3(pgemm_threads(true)), smem, tm_wg, tm_wu, tm_wg1, tm_wu1,
+           tm_hr, tm_wd, tl, g1, g2, h_ready, dys);
   };
   if (R == 8) go(expert_ffn_dynamic_kernel<8>, dy_smem_bytes<8>());
   else if (R == 16) go(expert_ffn_dynamic_kernel<16>, dy_smem_bytes<16>());

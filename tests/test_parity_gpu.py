@@ -217,19 +217,65 @@ def test_bounded_wait_reports_timeout_and_context_survives(gemma_w):
     run_case(wl.CONFIGS["decode"], gemma_w, 10**9)                 # context still usable
 
 
-def test_graph_replay_matches_direct_call(gemma_w):
-    x, c, g = layer_inputs(wl.CONFIGS["decode"], gemma_w)
-    x = x.cuda()
+def test_graph_replay_matches_oracle_and_direct_call(gemma_w):
+    """A captured moe_forward replays to the oracle's y (within the layer tolerance) and to
+    the direct call's bytes, and picks up new activations copied into its input buffer."""
+    x_cpu, c, g = layer_inputs(wl.CONFIGS["decode"], gemma_w)
+    x = x_cpu.cuda()
     y_direct = moe.forward(x, g["w_router"], g["w_gate"], g["w_up"], g["w_down"], 8)
     fg = moe.ForwardGraph(x, g["w_router"], g["w_gate"], g["w_up"], g["w_down"], 8)
+    ref = oracle.forward(x_cpu, c["w_router"], c["w_gate"], c["w_up"], c["w_down"], 8)
     for _ in range(3):
-        assert torch.equal(fg.replay(), y_direct)
+        y = fg.replay()
+        assert moe.sync_status() == 0
+        check_y(y, ref["y"])
+        assert torch.equal(y, y_direct)
     # new activations copied into the captured input buffer are picked up by the replay
-    x2 = wl.make_x(wl.CONFIGS["decode"], seed=7).cuda()
-    fg.x.copy_(x2)
+    x2_cpu = wl.make_x(wl.CONFIGS["decode"], seed=7)
+    fg.x.copy_(x2_cpu.cuda())
     y2 = fg.replay()
     assert moe.sync_status() == 0
-    assert torch.equal(y2, moe.forward(x2, g["w_router"], g["w_gate"], g["w_up"], g["w_down"], 8))
+    ref2 = oracle.forward(x2_cpu, c["w_router"], c["w_gate"], c["w_up"], c["w_down"], 8)
+    check_y(y2, ref2["y"])
+    assert torch.equal(y2, moe.forward(x2_cpu.cuda(), g["w_router"], g["w_gate"], g["w_up"],
+                                       g["w_down"], 8))
+
+
+def test_forward_and_dense_mlp_on_two_streams(gemma_w):
+    """The MoE layer and the dense MLP beside it, issued on two streams so that their
+    kernels overlap (each persistent expert-FFN grid then finds part of the GPU taken),
+    each with its own workspace: both outputs match the oracle, three times over, and the
+    device status stays OK (a bounded wait that ran out would read MOE_ERR_TIMEOUT)."""
+    cfg = wl.CONFIGS["prefill"]
+    x_cpu, c, g = layer_inputs(cfg, gemma_w)
+    wd_cpu = wl.make_dense_weights(cfg.H, wl.DENSE_I)
+    gd = {k: v.cuda() for k, v in wd_cpu.items()}
+    x = x_cpu.cuda()
+    lib = moe.load()
+    ws1 = torch.empty(moe._abi.workspace_bytes(cfg.T, cfg.H, cfg.E, cfg.I, cfg.k), dtype=torch.uint8,
+                      device="cuda")
+    ws2 = torch.empty(lib.moe_dense_workspace_size(cfg.T, cfg.H, wl.DENSE_I), dtype=torch.uint8,
+                      device="cuda")
+    s1, s2 = torch.cuda.Stream(), torch.cuda.Stream()
+    rows = sample_tokens(cfg.T, 48, seed=11)
+    ref = oracle.forward(x_cpu, c["w_router"], c["w_gate"], c["w_up"], c["w_down"], cfg.k,
+                         tokens=rows)
+    ref_d = oracle.dense_ffn(x_cpu, wd_cpu["w_gate"], wd_cpu["w_up"], wd_cpu["w_down"],
+                             rows=rows.tolist())
+    torch.cuda.synchronize()
+    for _ in range(3):
+        with torch.cuda.stream(s1):
+            y, aux = moe.forward(x, g["w_router"], g["w_gate"], g["w_up"], g["w_down"], cfg.k,
+                                 aux=True, workspace_buf=ws1, stream=s1)
+        with torch.cuda.stream(s2):
+            yd = moe.dense_ffn(x, gd["w_gate"], gd["w_up"], gd["w_down"], workspace_buf=ws2,
+                               stream=s2)
+        torch.cuda.synchronize()
+        assert moe.sync_status() == 0
+        idx = torch.from_numpy(rows).cuda()
+        check_routing(aux, ref, cfg.E)
+        check_y(y[idx], ref["y"])
+        check_y(yd[idx], ref_d)
 
 
 def test_dispatch_three_launches_for_many_chunks(gemma_w):
