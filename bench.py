@@ -136,21 +136,14 @@ def algorithmic(cfg: wl.MoEConfig, counts: np.ndarray, has_bias: bool) -> dict:
 
 def ffn_kernel_name(T: int, tiles: str) -> str:
     """The expert-FFN kernel(s) the library launches for T tokens and a tile family."""
-    if tiles == "decode":
-        return "grouped_gemm_decode_kernel<EPI_GEGLU>+<EPI_STORE>"
-    if tiles == "unfused":
-        return "grouped_gemm_persistent_kernel<4,EPI_GEGLU,4,1,0>+<4,EPI_STORE,4,0,0>"
-    if tiles == "fused":
-        return ("grouped_gemm_persistent_kernel<6,EPI_GEGLU,4,1,1,1>" if T <= 8
-                else "grouped_gemm_persistent_kernel<4,EPI_GEGLU,4,1,1>")
-    rows = next(r for r in (8, 16, 32, 64, 128) if T <= r or r == 128)
-    return f"expert_ffn_dynamic_kernel<{rows}>"
+    from expert_routed_ffn_softmax_b200 import _abi
+    return _abi.ffn_kernel_name(T, tiles)
 
 
 def kernel_source_sha() -> str:
     h = hashlib.sha256()
-    for f in ("grouped_gemm.cuh", "gemm_persistent.cuh", "ffn_dynamic.cuh", "gemm_decode.cuh",
-              "ptx.cuh"):
+    for f in ("grouped_gemm.cuh", "gemm_persistent.cuh", "ffn_dynamic.cuh", "ffn_pair.cuh",
+              "gemm_decode.cuh", "ptx.cuh"):
         h.update(open(os.path.join(ROOT, "expert_routed_ffn_softmax_b200", "csrc", f), "rb").read())
     return h.hexdigest()[:16]
 
@@ -297,7 +290,7 @@ def tensor_bound_entry(cfg, m: dict, world: int, pk: dict) -> dict:
                     + (" (router bias b_e = 2 ln(1/(e+1)))" if cfg.skew_bias else ""),
         "value": job_throughput(world, cfg.T, m["ms"]), "unit": UNIT,
         "ms_per_step": m["ms"],
-        "expert_ffn": {"kernel": ffn_kernel_name(cfg.T, "auto"), "ms": ffn_ms,
+        "expert_ffn": {"kernel": ffn_kernel_name(cfg.T, m["_tiles"]), "ms": ffn_ms,
                        "achieved_tflops": ffn_tf,
                        "frac_of_burst": None if ffn_tf is None else ffn_tf / pk["bf16_tflops"],
                        "frac_of_sustained": None if ffn_tf is None
@@ -471,6 +464,7 @@ def run_native(args, cfg) -> None:
             line["tensor_bound"] = []
             for c2, m2 in tensor_bound:
                 m2["_steps"] = args.steps
+                m2["_tiles"] = args.tiles
                 line["tensor_bound"].append(tensor_bound_entry(c2, m2, world, pk))
         if not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline(cfg, d, x_cpu, args.cpu_seconds)
@@ -599,7 +593,8 @@ def main():
     ap.add_argument("--ref-tokens", type=int, default=8)
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--tiles", default="auto", choices=["auto", "decode", "prefill", "fused", "unfused"],
+    ap.add_argument("--tiles", default="auto",
+                    choices=["auto", "decode", "prefill", "pairs", "single", "fused", "unfused"],
                     help="expert-GEMM tile family (default: the library's choice)")
     ap.add_argument("--no-tensor-bound", action="store_true",
                     help="skip the large-batch (tensor-bound) configs reported beside the line")

@@ -11,8 +11,10 @@ x, weights and outputs are CUDA tensors (bf16 operands, int32 ids, fp32 routing 
 all arithmetic runs in libmoe_b200.so.  ``workloads`` (seeded synthetic inputs) can be
 imported without a GPU.
 """
-from ._abi import (ForwardGraph, MoEError, dense_ffn, forward, last_kernel_count,  # noqa: F401
-                   last_stage_times, load, route, router_stats, status_string, sync_status)
+from ._abi import (ForwardGraph, MoEError, dense_ffn, ffn_kernel_name, forward,  # noqa: F401
+                   last_kernel_count, last_stage_times, load, route, router_stats, status_string,
+                   sync_status)
 
 __all__ = ["route", "forward", "dense_ffn", "ForwardGraph", "sync_status", "last_stage_times",
-           "load", "router_stats", "status_string", "MoEError", "last_kernel_count"]
+           "load", "router_stats", "status_string", "MoEError", "last_kernel_count",
+           "ffn_kernel_name"]

@@ -31,11 +31,16 @@ MOE_FLAG_DECODE_TILES = 1 << 4
 MOE_FLAG_PREFILL_TILES = 1 << 5
 MOE_FLAG_UNFUSED_FFN = 1 << 6
 MOE_FLAG_FUSED_FFN = 1 << 7
+MOE_FLAG_FFN_PAIRS = 1 << 8
+MOE_FLAG_FFN_SINGLE = 1 << 9
 
 _ROUTER_FLAGS = {"auto": 0, "fp64": MOE_FLAG_ROUTER_FP64, "screen": MOE_FLAG_ROUTER_SCREEN}
-# "auto"/"prefill": the dynamically scheduled expert FFN (one launch); "fused" / "unfused":
-# the statically scheduled forms in one or two launches; "decode": the swap-AB decode tiles.
+# "auto"/"prefill": the dynamically scheduled expert FFN (one launch; CTA pairs for large
+# batches); "pairs" / "single": that kernel on CTA pairs (256-row tiles) or single CTAs
+# (128-row tiles) for batches of more than 64 tokens; "fused" / "unfused": the statically
+# scheduled forms in one or two launches; "decode": the swap-AB decode tiles.
 _TILE_FLAGS = {"auto": 0, "decode": MOE_FLAG_DECODE_TILES, "prefill": MOE_FLAG_PREFILL_TILES,
+               "pairs": MOE_FLAG_FFN_PAIRS, "single": MOE_FLAG_FFN_SINGLE,
                "fused": MOE_FLAG_PREFILL_TILES | MOE_FLAG_FUSED_FFN,
                "unfused": MOE_FLAG_PREFILL_TILES | MOE_FLAG_UNFUSED_FFN}
 
@@ -52,6 +57,8 @@ SIGNATURES = {
     "moe_dense_workspace_size": (_SZ, [_I, _I, _I]),
     "moe_dense_ffn": (_I, [_P, _P, _P, _P, _I, _I, _I, _P, _P, _SZ, _P]),
     "moe_sync_status": (_I, [_P]),
+    "moe_pair_min_tokens": (_I, []),
+    "moe_ffn_kernel_name": (ctypes.c_char_p, [_I, _U]),
     "moe_last_stage_times": (_I, [ctypes.POINTER(ctypes.c_float), _I]),
     "moe_stage_name": (ctypes.c_char_p, [_I]),
     "moe_last_cuda_error": (_I, []),
@@ -269,6 +276,13 @@ def last_stage_times() -> dict[str, float]:
     if n < 0:
         raise RuntimeError("no profiled moe_forward call yet")
     return {L.moe_stage_name(i).decode(): float(buf[i]) for i in range(n)}
+
+
+def ffn_kernel_name(T: int, tiles: str = "auto") -> str:
+    """The expert-FFN kernel moe_forward launches for T tokens with this tile choice."""
+    if tiles not in _TILE_FLAGS:
+        raise ValueError(f"tiles must be one of {sorted(_TILE_FLAGS)}")
+    return load().moe_ffn_kernel_name(int(T), _TILE_FLAGS[tiles]).decode()
 
 
 def last_kernel_count() -> int:

@@ -38,10 +38,6 @@ __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_
       : "memory");
 }
 
-__device__ __forceinline__ void st_cluster_u32(uint32_t addr, uint32_t v) {
-  asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
-}
-
 // Dynamic shared memory layout (bytes from a 16-byte aligned base):
 //   W   max(hs*E*2, 2*NW*E*8)    W_router slice (bf16), later the cross-warp reduction
 //   XS  hs*8                     the token's x slice as doubles

@@ -18,6 +18,7 @@
 #include "grouped_gemm.cuh"
 #include "gemm_persistent.cuh"
 #include "ffn_dynamic.cuh"
+#include "ffn_pair.cuh"
 #include "decode_front.cuh"
 #include "gemm_decode.cuh"
 
@@ -37,7 +38,10 @@ constexpr int kFusedDispatchMaxChunks = 32;      // one-launch dispatch up to th
 constexpr unsigned kKnownFlags = MOE_FLAG_NO_RENORM | MOE_FLAG_ROUTER_FP64 |
                                  MOE_FLAG_ROUTER_SCREEN | MOE_FLAG_PROFILE_STAGES |
                                  MOE_FLAG_DECODE_TILES | MOE_FLAG_PREFILL_TILES |
-                                 MOE_FLAG_UNFUSED_FFN | MOE_FLAG_FUSED_FFN;
+                                 MOE_FLAG_UNFUSED_FFN | MOE_FLAG_FUSED_FFN |
+                                 MOE_FLAG_FFN_PAIRS | MOE_FLAG_FFN_SINGLE;
+// Batches of at least this many tokens run the expert FFN on CTA pairs by default.
+constexpr int kPairMinTokens = 2048;
 
 #define GEMM_GEGLU grouped_gemm_persistent_kernel<kGemmStages, EPI_GEGLU, 4, true>
 #define GEMM_FFN grouped_gemm_persistent_kernel<kGemmStages, EPI_GEGLU, 4, true, true>
@@ -52,6 +56,11 @@ bool flags_ok(unsigned flags) {
   if ((flags & MOE_FLAG_ROUTER_FP64) && (flags & MOE_FLAG_ROUTER_SCREEN)) return false;
   if ((flags & MOE_FLAG_DECODE_TILES) && (flags & MOE_FLAG_PREFILL_TILES)) return false;
   if ((flags & MOE_FLAG_UNFUSED_FFN) && (flags & MOE_FLAG_FUSED_FFN)) return false;
+  const unsigned tiles = MOE_FLAG_FFN_PAIRS | MOE_FLAG_FFN_SINGLE;
+  if ((flags & tiles) == tiles) return false;
+  if ((flags & tiles) &&
+      (flags & (MOE_FLAG_FUSED_FFN | MOE_FLAG_UNFUSED_FFN | MOE_FLAG_DECODE_TILES)))
+    return false;
   return true;
 }
 
@@ -77,6 +86,13 @@ bool router_uses_screen(int T, int E, unsigned flags) {
 int dy_rows(int T, unsigned flags) {
   if (flags & (MOE_FLAG_FUSED_FFN | MOE_FLAG_UNFUSED_FFN | MOE_FLAG_DECODE_TILES)) return 0;
   return T <= 8 ? 8 : T <= 16 ? 16 : T <= 32 ? 32 : T <= 64 ? 64 : 128;
+}
+
+// The dynamic FFN on CTA pairs (256-row tiles, tcgen05 cta_group::2): batches of more than
+// 64 tokens, from kPairMinTokens tokens by default.
+bool use_pair_ffn(int T, unsigned flags) {
+  if (dy_rows(T, flags) != 128 || (flags & MOE_FLAG_FFN_SINGLE)) return false;
+  return (flags & MOE_FLAG_FFN_PAIRS) || T >= kPairMinTokens;
 }
 
 // Batches of at most 16 tokens (so at most 16 rows per expert) use the decode GEMMs.
@@ -173,7 +189,7 @@ Layout make_layout(int T, int H, int E, int I, int k, unsigned flags, bool forwa
   }
   if (forward) {
     L.nchunks = (int)((P + kDispatchChunk - 1) / kDispatchChunk);
-    L.bm = use_decode_gemm(T, H, I, flags) ? DG_BN : GM_BM;
+    L.bm = use_decode_gemm(T, H, I, flags) ? DG_BN : use_pair_ffn(T, flags) ? PR_ROWS : GM_BM;
     L.max_tiles = (int)(P / L.bm) + E;
     L.ids = take(sizeof(int32_t) * P);
     L.wts = take(sizeof(float) * P);
@@ -333,6 +349,8 @@ DeviceState* device_state(int* dev_out) {
         cudaFuncSetAttribute(expert_ffn_dynamic_kernel<128>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, dy_smem_bytes<128>()) !=
             cudaSuccess ||
+        cudaFuncSetAttribute(expert_ffn_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             PR_SMEM) != cudaSuccess ||
         cudaFuncSetAttribute(GEMM_FFN_SMALL, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              pgemm_smem_bytes<kSmallStages, 4, true>()) != cudaSuccess ||
         cudaFuncSetAttribute(GEMM_STORE, cudaFuncAttributeMaxDynamicSharedMemorySize, gs) !=
@@ -726,7 +744,14 @@ moe_status_t moe_forward(const void* x, const void* w_router, const float* route
         launch(true, kernel, dim3(G), dim3(pgemm_threads(true)), smem, tm_wg, tm_wu, tm_wg1,
                tm_wu1, tm_hr, tm_wd, tl, g1, g2, h_ready, dys);
       };
-      if (R == 8) go(expert_ffn_dynamic_kernel<8>, dy_smem_bytes<8>());
+      if (L.bm == PR_ROWS) {
+        // CTA pairs (2-CTA clusters, an even grid): 2-slab W_down boxes, each CTA loading
+        // 128 of a block's 256 columns
+        CUtensorMap tm_wd2;
+        if (!make_map_slabs(&tm_wd2, w_down, H, I, E, 64, 2)) return cuda_failed(-1);
+        launch(true, expert_ffn_pair_kernel, dim3(std::max(2, G & ~1)), dim3(pgemm_threads(true)), PR_SMEM,
+               tm_wg, tm_wu, tm_wg1, tm_wu1, tm_hr, tm_wd2, tl, g1, g2, h_ready, dys);
+      } else if (R == 8) go(expert_ffn_dynamic_kernel<8>, dy_smem_bytes<8>());
       else if (R == 16) go(expert_ffn_dynamic_kernel<16>, dy_smem_bytes<16>());
       else if (R == 32) go(expert_ffn_dynamic_kernel<32>, dy_smem_bytes<32>());
       else if (R == 64) go(expert_ffn_dynamic_kernel<64>, dy_smem_bytes<64>());
@@ -838,7 +863,13 @@ moe_status_t moe_dense_ffn(const void* x, const void* w_gate, const void* w_up,
     launch(false, kernel, dim3(G), dim3(pgemm_threads(true)), smem, tm_wg, tm_wu, tm_wg1, tm_wu1,
            tm_hr, tm_wd, tl, g1, g2, h_ready, dys);
   };
-  if (R == 8) go(expert_ffn_dynamic_kernel<8>, dy_smem_bytes<8>());
+  if (use_pair_ffn(T, 0)) {
+    // CTA pairs over 256-row tiles of x (the counters above cover ceil(T / 128) tiles)
+    CUtensorMap tm_wd2;
+    if (!make_map_slabs(&tm_wd2, w_down, H, I, 1, 64, 2)) return cuda_failed(-1);
+    launch(false, expert_ffn_pair_kernel, dim3(std::max(2, G & ~1)), dim3(pgemm_threads(true)),
+           PR_SMEM, tm_wg, tm_wu, tm_wg1, tm_wu1, tm_hr, tm_wd2, tl, g1, g2, h_ready, dys);
+  } else if (R == 8) go(expert_ffn_dynamic_kernel<8>, dy_smem_bytes<8>());
   else if (R == 16) go(expert_ffn_dynamic_kernel<16>, dy_smem_bytes<16>());
   else if (R == 32) go(expert_ffn_dynamic_kernel<32>, dy_smem_bytes<32>());
   else if (R == 64) go(expert_ffn_dynamic_kernel<64>, dy_smem_bytes<64>());
@@ -893,6 +924,27 @@ moe_status_t moe_sync_status(void* stream) {
   if (w & MOE_DEVERR_TIMEOUT) return MOE_ERR_TIMEOUT;
   if (w) return MOE_ERR_CUDA;
   return MOE_OK;
+}
+
+int moe_pair_min_tokens(void) { return kPairMinTokens; }
+
+const char* moe_ffn_kernel_name(int T, unsigned flags) {
+  if (T < 1 || !flags_ok(flags)) return "";
+  if (flags & MOE_FLAG_DECODE_TILES)
+    return T <= kDecodeMaxTokens ? "grouped_gemm_decode_kernel<EPI_GEGLU>+<EPI_STORE>" : "";
+  if (flags & MOE_FLAG_UNFUSED_FFN)
+    return "grouped_gemm_persistent_kernel<4,EPI_GEGLU,4,1,0>+<4,EPI_STORE,4,0,0>";
+  if (flags & MOE_FLAG_FUSED_FFN)
+    return T <= PG_SMALL_ROWS ? "grouped_gemm_persistent_kernel<6,EPI_GEGLU,4,1,1,1>"
+                              : "grouped_gemm_persistent_kernel<4,EPI_GEGLU,4,1,1>";
+  if (use_pair_ffn(T, flags)) return "expert_ffn_pair_kernel";
+  switch (dy_rows(T, flags)) {
+    case 8: return "expert_ffn_dynamic_kernel<8>";
+    case 16: return "expert_ffn_dynamic_kernel<16>";
+    case 32: return "expert_ffn_dynamic_kernel<32>";
+    case 64: return "expert_ffn_dynamic_kernel<64>";
+    default: return "expert_ffn_dynamic_kernel<128>";
+  }
 }
 
 int moe_last_cuda_error(void) { return t_last_cuda_error; }

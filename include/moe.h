@@ -39,7 +39,7 @@
 extern "C" {
 #endif
 
-#define MOE_ABI_VERSION 2
+#define MOE_ABI_VERSION 3
 
 typedef enum {
   MOE_OK = 0,
@@ -81,7 +81,17 @@ enum {
    * stream-K splits the sums of some tiles across CTAs, so their bytes can differ from the
    * default's in the last bit of a few elements.  Setting both is MOE_ERR_INVALID_ARG. */
   MOE_FLAG_UNFUSED_FFN = 1u << 6,
-  MOE_FLAG_FUSED_FFN = 1u << 7
+  MOE_FLAG_FUSED_FFN = 1u << 7,
+  /* Tiles of the default (dynamically scheduled) expert FFN for batches of more than 64
+   * tokens: CTA pairs -- a 2-CTA cluster computes 256 sorted rows x 256 columns with one
+   * tcgen05.mma.cta_group::2, each CTA loading its own 128 rows and half of the weight
+   * columns -- or single CTAs with 128-row tiles.  By default batches of at least
+   * moe_pair_min_tokens() tokens use pairs.  Both give the same bytes (every output element
+   * is the same fp32 sum over K in the same order).  Setting both, or either with
+   * MOE_FLAG_FUSED_FFN / MOE_FLAG_UNFUSED_FFN / MOE_FLAG_DECODE_TILES, is MOE_ERR_INVALID_ARG;
+   * at 64 tokens or fewer both are ignored (the A tiles then hold at most 64 rows). */
+  MOE_FLAG_FFN_PAIRS = 1u << 8,
+  MOE_FLAG_FFN_SINGLE = 1u << 9
 };
 
 /* Optional caller-owned device outputs of moe_forward (any member may be NULL). */
@@ -211,6 +221,14 @@ moe_status_t moe_dense_ffn(const void *x, const void *w_gate, const void *w_up,
 moe_status_t moe_route_static(const void *x, const void *w_router, const float *router_bias,
                               int T, int H, int E, int k, unsigned flags, int32_t *topk_ids,
                               float *topk_weights, void *stream);
+
+/* Smallest batch (tokens) for which moe_forward and moe_dense_ffn run the expert FFN on
+ * CTA pairs by default (see MOE_FLAG_FFN_PAIRS). */
+int moe_pair_min_tokens(void);
+
+/* Name of the expert-FFN kernel moe_forward launches for a batch of T tokens with these
+ * flags (static storage; "" for an invalid combination). */
+const char *moe_ffn_kernel_name(int T, unsigned flags);
 
 /* Synchronise `stream`, then read and clear this device's error word.
  * MOE_OK, MOE_ERR_TIMEOUT (a bounded device wait ran out), or MOE_ERR_CUDA (a CUDA error,

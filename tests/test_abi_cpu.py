@@ -39,7 +39,7 @@ def test_library_exports_every_declared_symbol(lib):
 
 
 def test_abi_version_and_status_strings(lib):
-    assert lib.moe_abi_version() == 2
+    assert lib.moe_abi_version() == 3
     assert _abi.status_string(0) == "MOE_OK"
     assert _abi.status_string(5) == "MOE_ERR_TIMEOUT"
     assert _abi.status_string(99) == "MOE_ERR_UNKNOWN"
@@ -87,7 +87,10 @@ def test_host_argument_checks(lib):
     assert f(*ok, 8, 2816, 128, 704, 8, 1 << 12, FAKE + 4096, None, FAKE, 1 << 30, None) == 1
     for both in (_abi.MOE_FLAG_ROUTER_FP64 | _abi.MOE_FLAG_ROUTER_SCREEN,   # contradictory
                  _abi.MOE_FLAG_FUSED_FFN | _abi.MOE_FLAG_UNFUSED_FFN,
-                 _abi.MOE_FLAG_DECODE_TILES | _abi.MOE_FLAG_PREFILL_TILES):
+                 _abi.MOE_FLAG_DECODE_TILES | _abi.MOE_FLAG_PREFILL_TILES,
+                 _abi.MOE_FLAG_FFN_PAIRS | _abi.MOE_FLAG_FFN_SINGLE,
+                 _abi.MOE_FLAG_FFN_PAIRS | _abi.MOE_FLAG_FUSED_FFN,
+                 _abi.MOE_FLAG_FFN_SINGLE | _abi.MOE_FLAG_DECODE_TILES):
         assert f(*ok, 8, 2816, 128, 704, 8, both, FAKE + 4096, None, FAKE, 1 << 30, None) == 1
         assert lib.moe_workspace_size(8, 2816, 128, 704, 8, both) == 0
     # misaligned pointer
@@ -120,3 +123,24 @@ def test_dense_ffn_host_checks(lib):
     assert f(FAKE + 2, FAKE, FAKE, FAKE, 8, 2816, 2112, FAKE + 4096, FAKE, 1 << 30, None) == 1
     assert f(*w, 8, 2816, 2100, FAKE + 4096, FAKE, 1 << 30, None) == _abi.MOE_ERR_UNSUPPORTED
     assert f(*w, 8, 2816, 2112, FAKE + 4096, FAKE, 1024, None) == _abi.MOE_ERR_NO_WORKSPACE
+
+
+def test_ffn_kernel_choice(lib):
+    """Which expert-FFN kernel a batch gets: the dynamic kernel with A slots of 8..128 rows,
+    CTA pairs from moe_pair_min_tokens() tokens (or when forced above 64 tokens)."""
+    pmin = lib.moe_pair_min_tokens()
+    assert 64 < pmin <= 1 << 20
+    assert _abi.ffn_kernel_name(1) == "expert_ffn_dynamic_kernel<8>"
+    assert _abi.ffn_kernel_name(8) == "expert_ffn_dynamic_kernel<8>"
+    assert _abi.ffn_kernel_name(64) == "expert_ffn_dynamic_kernel<64>"
+    assert _abi.ffn_kernel_name(pmin - 1) == "expert_ffn_dynamic_kernel<128>"
+    assert _abi.ffn_kernel_name(pmin) == "expert_ffn_pair_kernel"
+    assert _abi.ffn_kernel_name(pmin, "single") == "expert_ffn_dynamic_kernel<128>"
+    assert _abi.ffn_kernel_name(65, "pairs") == "expert_ffn_pair_kernel"
+    assert _abi.ffn_kernel_name(64, "pairs") == "expert_ffn_dynamic_kernel<64>"
+    assert _abi.ffn_kernel_name(8, "decode").startswith("grouped_gemm_decode_kernel")
+    assert lib.moe_ffn_kernel_name(8, _abi.MOE_FLAG_FFN_PAIRS | _abi.MOE_FLAG_FFN_SINGLE) == b""
+    # pair tiles of 256 rows need fewer tile-list entries, not more workspace
+    single = lib.moe_workspace_size(4096, 2816, 128, 704, 8, _abi.MOE_FLAG_FFN_SINGLE)
+    pairs = lib.moe_workspace_size(4096, 2816, 128, 704, 8, _abi.MOE_FLAG_FFN_PAIRS)
+    assert 0 < pairs <= single

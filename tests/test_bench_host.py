@@ -67,12 +67,15 @@ def test_reference_arm_json_line():
 
 
 def test_ffn_kernel_name_follows_the_library_rule():
+    from expert_routed_ffn_softmax_b200 import build
+    build.build()
     # the default form is the dynamic FFN with an A slot of the smallest of 8..128 rows >= T
     assert bench.ffn_kernel_name(1, "auto") == "expert_ffn_dynamic_kernel<8>"
     assert bench.ffn_kernel_name(9, "auto") == "expert_ffn_dynamic_kernel<16>"
     assert bench.ffn_kernel_name(64, "prefill") == "expert_ffn_dynamic_kernel<64>"
     assert bench.ffn_kernel_name(65, "auto") == "expert_ffn_dynamic_kernel<128>"
-    assert bench.ffn_kernel_name(32768, "auto") == "expert_ffn_dynamic_kernel<128>"
+    assert bench.ffn_kernel_name(32768, "auto") == "expert_ffn_pair_kernel"      # CTA pairs
+    assert bench.ffn_kernel_name(32768, "single") == "expert_ffn_dynamic_kernel<128>"
     assert "+" in bench.ffn_kernel_name(4096, "unfused")          # two launches
     assert bench.ffn_kernel_name(8, "fused").endswith(",1>")       # 8-row A slots
     assert bench.ffn_kernel_name(8, "decode").startswith("grouped_gemm_decode_kernel")

@@ -129,6 +129,41 @@ def test_forward_tile_families(name, T, tiles, gemma_w):
     run_case(wl.CONFIGS[name], gemma_w, 64, T=T, tiles=tiles)
 
 
+# CTA-pair tiles (256 rows per pair, tcgen05 cta_group::2) and single-CTA tiles (128 rows) of
+# the dynamic expert FFN, each forced at batch sizes where the other is the default.  At
+# T = 65 and 300 every expert has fewer than 128 rows (the second CTA of every pair has no
+# rows); at T = 2048 and 4096 experts have around 128 and 256 rows (pair tiles whose second
+# half is empty, partly filled or full, and experts with an odd number of 128-row tiles);
+# tiny T = 1000 has 250 rows per expert and H = 256 (one GEMM-2 block).
+PAIR_CASES = [("tiny", 1000), ("decode", 65), ("decode", 300), ("prefill", 2048),
+              ("sweep_T4096", 4096)]
+
+
+@pytest.mark.parametrize("tiles", ["pairs", "single"])
+@pytest.mark.parametrize("name,T", PAIR_CASES, ids=[f"{n}_T{t}" for n, t in PAIR_CASES])
+def test_forward_pair_and_single_cta_tiles(name, T, tiles, gemma_w):
+    run_case(wl.CONFIGS[name], gemma_w, 256, T=T, tiles=tiles)
+
+
+def test_skewed_on_single_cta_tiles(gemma_w):
+    """The skewed batch (experts from empty to 16k rows) on 128-row single-CTA tiles (its
+    default is CTA pairs, covered by test_forward_parity)."""
+    assert moe.ffn_kernel_name(16384) == "expert_ffn_pair_kernel"
+    run_case(wl.CONFIGS["skewed"], gemma_w, 128, tiles="single")
+
+
+@pytest.mark.parametrize("T", [65, 300, 2048, 4096])
+def test_pair_tiles_match_single_cta_tiles_bitwise(T, gemma_w):
+    """Every output element is the same fp32 sum over K in the same k-step order whether its
+    row sits in a 128-row single-CTA tile or in a 256-row CTA pair, so the bytes agree."""
+    x, c, g = layer_inputs(wl.CONFIGS["decode"], gemma_w, T=T)
+    x = x.cuda()
+    y1 = moe.forward(x, g["w_router"], g["w_gate"], g["w_up"], g["w_down"], 8, tiles="pairs")
+    y2 = moe.forward(x, g["w_router"], g["w_gate"], g["w_up"], g["w_down"], 8, tiles="single")
+    assert moe.sync_status() == 0
+    assert torch.equal(y1, y2)
+
+
 def test_forward_no_renorm(gemma_w):
     run_case(wl.CONFIGS["tiny"], gemma_w, 10**9, renorm=False)
     run_case(wl.CONFIGS["decode"], gemma_w, 10**9, renorm=False)
@@ -299,7 +334,8 @@ def test_dispatch_three_launches_for_many_chunks(gemma_w):
     (8, 2816, 2112, None),         # Gemma dense MLP at decode, every row
     (1, 2816, 2112, None),
     (200, 2816, 2112, "sample"),   # two row tiles, the second ragged (72 rows)
-    (2048, 2816, 2112, "sample"),
+    (2048, 2816, 2112, "sample"),  # CTA pairs: 8 tiles of 256 rows
+    (2500, 2816, 2112, "sample"),  # CTA pairs, the last tile 196 rows (128 + 68)
 ])
 def test_dense_ffn_parity(T, H, I, rows):
     """The dense GEGLU MLP beside the MoE against the fp64 oracle (same bf16 inputs):
@@ -373,5 +409,7 @@ def test_other_shapes(cfg, router, gemma_w):
         return
     run_case(cfg, gemma_w, 10**9, router=router)
     run_case(cfg, gemma_w, 10**9, router=router, tiles="unfused")
+    if cfg.T > 64:
+        run_case(cfg, gemma_w, 10**9, router=router, tiles="pairs")
     if router != "screen":   # the screen path renormalises only
         run_case(cfg, gemma_w, 10**9, router=router, renorm=False)
