@@ -583,6 +583,87 @@ def run_dense(args, cfg) -> None:
     print(json.dumps(line), flush=True)
 
 
+def run_ep(args, cfg) -> None:
+    """--ep: the expert-parallel layer (expert_routed_ffn_softmax_b200.ep) with E / N experts on
+    each of N ranks (NCCL), every rank bringing its own batch of cfg's shape; the AllToAll
+    form above 64 tokens per rank, the AllGather (decode) form at or below.  Same timing
+    rules as the default run (untimed L2 flush before every step, CUDA events on the launching
+    stream, max over ranks)."""
+    import datetime
+    import torch.distributed as dist
+    from expert_routed_ffn_softmax_b200 import ep
+    import expert_routed_ffn_softmax_b200 as moe
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+    os.environ.setdefault("MASTER_PORT", "29731")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist.init_process_group("nccl", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=120), device_id=dev)
+    try:
+        w = wl.make_weights(cfg)
+        lo, hi = ep.expert_range(cfg.E, world, rank)
+        g = {"w_router": w["w_router"].to(dev),
+             "w_gate": w["w_gate"][lo:hi].contiguous().to(dev),
+             "w_up": w["w_up"][lo:hi].contiguous().to(dev),
+             "w_down": w["w_down"][lo:hi].contiguous().to(dev)}
+        bias = w["bias"].to(dev) if w["bias"] is not None else None
+        layer = ep.ExpertParallelMoE(g["w_router"], g["w_gate"], g["w_up"], g["w_down"], cfg.E,
+                                     cfg.k, ep.TorchComm(), bias=bias)
+        mode = "allgather" if cfg.T <= 64 else "alltoall"
+        x = wl.make_x(cfg, seed=rank).to(dev)
+        flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+        flush_rd = torch.zeros(L2_FLUSH_BYTES // 8, dtype=torch.int64, device=dev)
+        stream = torch.cuda.current_stream()
+        for _ in range(args.warmup):
+            flush.zero_()
+            flush_rd.max()
+            layer.forward(x, mode)
+        torch.cuda.synchronize()
+        if moe.sync_status() != 0:
+            raise SystemExit("device status not OK after the warm-up")
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(args.steps)]
+        clocks = ClockSampler(dev)
+        clocks.start()
+        dist.barrier()
+        torch.cuda.synchronize()
+        for i in range(args.steps):
+            flush.zero_()
+            flush_rd.max()
+            ev[i][0].record(stream)
+            layer.forward(x, mode)
+            ev[i][1].record(stream)
+        torch.cuda.synchronize()
+        dist.barrier()
+        clk = clocks.stop()
+        ms = sum(a.elapsed_time(b) for a, b in ev) / args.steps
+        ms = max_over_ranks([ms], dist, dev)[0]
+        if rank == 0:
+            line = {
+                "metric": METRIC, "value": job_throughput(world, cfg.T, ms), "unit": UNIT,
+                "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+                "data": "synthetic",
+                "config": {"workload": f"{cfg.name}: T={cfg.T} per rank, H={cfg.H} E={cfg.E} "
+                                       f"k={cfg.k} I={cfg.I}, experts split over the ranks",
+                           "global_batch": world * cfg.T, "tokens_per_gpu": cfg.T,
+                           "parallelism": f"ep{world} ({mode})",
+                           "l2": "flushed before every step (256 MB write then 256 MB read, untimed)"},
+                "clocks": clk,
+                "note": "host-synchronising split-size exchange per step (counts to the host)",
+            }
+            print(json.dumps(line), flush=True)
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -598,6 +679,8 @@ def main():
                     help="expert-GEMM tile family (default: the library's choice)")
     ap.add_argument("--no-tensor-bound", action="store_true",
                     help="skip the large-batch (tensor-bound) configs reported beside the line")
+    ap.add_argument("--ep", action="store_true",
+                    help="time the expert-parallel layer (experts split over the ranks, NCCL)")
     ap.add_argument("--dense", action="store_true",
                     help="time the dense GEGLU MLP beside the MoE instead of the MoE layer")
     args = ap.parse_args()
@@ -605,6 +688,8 @@ def main():
     cfg = wl.CONFIGS[args.config]
     if args.dense:
         run_dense(args, cfg)
+    elif args.ep and args.impl != "reference":
+        run_ep(args, cfg)
     elif args.impl == "reference":
         run_reference(args, cfg)
     else:

@@ -33,8 +33,14 @@ MOE_FLAG_UNFUSED_FFN = 1 << 6
 MOE_FLAG_FUSED_FFN = 1 << 7
 MOE_FLAG_FFN_PAIRS = 1 << 8
 MOE_FLAG_FFN_SINGLE = 1 << 9
+MOE_FLAG_FFN_ROWS_COPY = 1 << 10
+MOE_FLAG_FFN_ROWS_GATHER = 1 << 11
+MOE_COMBINE_F32 = 1 << 0
 
 _ROUTER_FLAGS = {"auto": 0, "fp64": MOE_FLAG_ROUTER_FP64, "screen": MOE_FLAG_ROUTER_SCREEN}
+# How GEMM-1 of the dynamic FFN gets its A rows above 64 tokens: copied into an expert-sorted
+# buffer first and loaded by TMA, or gathered from x inside the FFN kernel.
+_ROWS_FLAGS = {"auto": 0, "copy": MOE_FLAG_FFN_ROWS_COPY, "gather": MOE_FLAG_FFN_ROWS_GATHER}
 # "auto"/"prefill": the dynamically scheduled expert FFN (one launch; CTA pairs for large
 # batches); "pairs" / "single": that kernel on CTA pairs (256-row tiles) or single CTAs
 # (128-row tiles) for batches of more than 64 tokens; "fused" / "unfused": the statically
@@ -56,8 +62,13 @@ SIGNATURES = {
     "moe_forward": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _U, _P, _P, _P, _SZ, _P]),
     "moe_dense_workspace_size": (_SZ, [_I, _I, _I]),
     "moe_dense_ffn": (_I, [_P, _P, _P, _P, _I, _I, _I, _P, _P, _SZ, _P]),
+    "moe_dispatch_workspace_size": (_SZ, [_I, _I, _I]),
+    "moe_dispatch": (_I, [_P, _I, _I, _I, _P, _P, _P, _P, _P, _SZ, _P]),
+    "moe_gather_rows": (_I, [_P, _P, _I, _I, _I, _I, _P, _P]),
+    "moe_expert_ffn_workspace_size": (_SZ, [_I, _I, _I, _I, _I]),
+    "moe_expert_ffn": (_I, [_P, _I, _P, _P, _I, _P, _P, _P, _I, _I, _I, _P, _P, _SZ, _P]),
+    "moe_combine": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _U, _P, _P]),
     "moe_sync_status": (_I, [_P]),
-    "moe_pair_min_tokens": (_I, []),
     "moe_ffn_kernel_name": (ctypes.c_char_p, [_I, _U]),
     "moe_last_stage_times": (_I, [ctypes.POINTER(ctypes.c_float), _I]),
     "moe_stage_name": (ctypes.c_char_p, [_I]),
@@ -143,17 +154,20 @@ def _dev(t: torch.Tensor, name: str, dtype: torch.dtype, shape: tuple) -> int:
     return t.data_ptr()
 
 
-def _flags(renorm: bool, router: str, profile: bool = False, tiles: str = "auto") -> int:
+def _flags(renorm: bool, router: str, profile: bool = False, tiles: str = "auto",
+           rows: str = "auto") -> int:
     if router not in _ROUTER_FLAGS:
         raise ValueError(f"router must be one of {sorted(_ROUTER_FLAGS)}")
     if tiles not in _TILE_FLAGS:
         raise ValueError(f"tiles must be one of {sorted(_TILE_FLAGS)}")
+    if rows not in _ROWS_FLAGS:
+        raise ValueError(f"rows must be one of {sorted(_ROWS_FLAGS)}")
     return ((0 if renorm else MOE_FLAG_NO_RENORM) | _ROUTER_FLAGS[router] | _TILE_FLAGS[tiles]
-            | (MOE_FLAG_PROFILE_STAGES if profile else 0))
+            | _ROWS_FLAGS[rows] | (MOE_FLAG_PROFILE_STAGES if profile else 0))
 
 
 def route(x: torch.Tensor, w_router: torch.Tensor, k: int, bias: torch.Tensor | None = None,
-          renorm: bool = True, router: str = "auto", stream=None):
+          renorm: bool = True, router: str = "auto", stream=None, workspace_buf=None):
     """Router of the MoE layer -> (topk_ids int32 [T,k], topk_weights float32 [T,k]).
 
     router: "auto" (tensor-core screen + fp64 recheck for T >= 256, fp64 logits below),
@@ -171,7 +185,7 @@ def route(x: torch.Tensor, w_router: torch.Tensor, k: int, bias: torch.Tensor | 
     nbytes = L.moe_route_workspace_size(T, H, E, k, flags) if T > 0 else 0
     if T > 0 and nbytes == 0:
         raise MoEError(MOE_ERR_UNSUPPORTED, "moe_route_workspace_size")
-    ws = workspace(nbytes, dev)
+    ws = workspace(nbytes, dev) if workspace_buf is None else workspace_buf
     _check(L.moe_route(px, pw, pb, T, H, E, k, flags, ids.data_ptr(), wts.data_ptr(),
                        ws.data_ptr(), ws.numel(), _stream_ptr(stream)), "moe_route")
     return ids, wts
@@ -181,7 +195,7 @@ def forward(x: torch.Tensor, w_router: torch.Tensor, w_gate: torch.Tensor, w_up:
             w_down: torch.Tensor, k: int, bias: torch.Tensor | None = None, renorm: bool = True,
             aux: bool = False, out: torch.Tensor | None = None, profile: bool = False,
             stream=None, workspace_buf: torch.Tensor | None = None, router: str = "auto",
-            tiles: str = "auto"):
+            tiles: str = "auto", rows: str = "auto"):
     """The routed MoE FFN layer -> y bf16 [T,H] (and a dict of routing outputs if aux).
 
     workspace_buf: optional caller-owned uint8 CUDA tensor used as the workspace (else a
@@ -198,7 +212,7 @@ def forward(x: torch.Tensor, w_router: torch.Tensor, w_gate: torch.Tensor, w_up:
     pb = None if bias is None else _dev(bias, "bias", torch.float32, (E,))
     y = torch.empty((T, H), dtype=torch.bfloat16, device=dev) if out is None else out
     py = _dev(y, "out", torch.bfloat16, (T, H))
-    flags = _flags(renorm, router, profile, tiles)
+    flags = _flags(renorm, router, profile, tiles, rows)
     a = None
     aux_d = None
     if aux:
@@ -245,6 +259,97 @@ def dense_ffn(x: torch.Tensor, w_gate: torch.Tensor, w_up: torch.Tensor, w_down:
     return y
 
 
+# ----------------------------------------------------------------------------- steps alone
+def dispatch(topk_ids: torch.Tensor, E: int, stream=None, workspace_buf=None):
+    """moe_dispatch: topk_ids int32 [T,k] -> (counts [E], offsets [E+1], perm [T*k],
+    inv [T*k]), int32 CUDA tensors."""
+    L = load()
+    T, k = topk_ids.shape
+    dev = topk_ids.device
+    pids = _dev(topk_ids, "topk_ids", torch.int32, (T, k))
+    counts = torch.empty(E, dtype=torch.int32, device=dev)
+    offsets = torch.empty(E + 1, dtype=torch.int32, device=dev)
+    perm = torch.empty(T * k, dtype=torch.int32, device=dev)
+    inv = torch.empty(T * k, dtype=torch.int32, device=dev)
+    if T == 0:
+        return counts.zero_(), offsets.zero_(), perm, inv
+    nbytes = L.moe_dispatch_workspace_size(T, E, k)
+    if nbytes == 0:
+        raise MoEError(MOE_ERR_UNSUPPORTED, "moe_dispatch_workspace_size")
+    ws = workspace(nbytes, dev) if workspace_buf is None else workspace_buf
+    _check(L.moe_dispatch(pids, T, E, k, counts.data_ptr(), offsets.data_ptr(), perm.data_ptr(),
+                          inv.data_ptr(), ws.data_ptr(), ws.numel(), _stream_ptr(stream)),
+           "moe_dispatch")
+    return counts, offsets, perm, inv
+
+
+def gather_rows(x: torch.Tensor, perm: torch.Tensor, k: int, out: torch.Tensor | None = None,
+                stream=None) -> torch.Tensor:
+    """moe_gather_rows: out[r] = x[perm[r] // k] for every entry of perm (a 1-D int32 CUDA
+    tensor of pair indices, possibly a slice of dispatch()'s perm)."""
+    L = load()
+    T, H = x.shape
+    n = perm.numel()
+    px = _dev(x, "x", torch.bfloat16, (T, H))
+    pp = _dev(perm, "perm", torch.int32, (n,))
+    xp = torch.empty((n, H), dtype=torch.bfloat16, device=x.device) if out is None else out
+    po = _dev(xp, "out", torch.bfloat16, (n, H))
+    if n:
+        _check(L.moe_gather_rows(px, pp, n, T, H, k, po, _stream_ptr(stream)), "moe_gather_rows")
+    return xp
+
+
+def expert_ffn(xs: torch.Tensor, seg_rows: torch.Tensor, seg_expert: torch.Tensor,
+               w_gate: torch.Tensor, w_up: torch.Tensor, w_down: torch.Tensor,
+               out: torch.Tensor | None = None, stream=None, workspace_buf=None) -> torch.Tensor:
+    """moe_expert_ffn: the GEGLU expert FFN of every row of xs [N,H] (bf16), whose rows form
+    consecutive segments: seg_rows[i] rows of expert seg_expert[i] (int32 CUDA tensors)."""
+    L = load()
+    N, H = xs.shape
+    E, _, I = w_gate.shape
+    n_seg = seg_rows.numel()
+    dev = xs.device
+    px = _dev(xs, "xs", torch.bfloat16, (N, H))
+    pr = _dev(seg_rows, "seg_rows", torch.int32, (n_seg,))
+    pe = _dev(seg_expert, "seg_expert", torch.int32, (n_seg,))
+    pg = _dev(w_gate, "w_gate", torch.bfloat16, (E, H, I))
+    pu = _dev(w_up, "w_up", torch.bfloat16, (E, H, I))
+    pd = _dev(w_down, "w_down", torch.bfloat16, (E, I, H))
+    o = torch.empty((N, H), dtype=torch.bfloat16, device=dev) if out is None else out
+    po = _dev(o, "out", torch.bfloat16, (N, H))
+    if N == 0 or n_seg == 0:
+        return o
+    nbytes = L.moe_expert_ffn_workspace_size(N, H, E, I, n_seg)
+    if nbytes == 0:
+        raise MoEError(MOE_ERR_UNSUPPORTED, "moe_expert_ffn_workspace_size")
+    ws = workspace(nbytes, dev) if workspace_buf is None else workspace_buf
+    _check(L.moe_expert_ffn(px, N, pr, pe, n_seg, pg, pu, pd, H, E, I, po, ws.data_ptr(),
+                            ws.numel(), _stream_ptr(stream)), "moe_expert_ffn")
+    return o
+
+
+def combine(o: torch.Tensor, inv: torch.Tensor, topk_weights: torch.Tensor, row_lo: int = 0,
+            row_hi: int | None = None, fp32: bool = False, out: torch.Tensor | None = None,
+            stream=None) -> torch.Tensor:
+    """moe_combine: y[t] = sum_j w[t,j] o[inv[t,j]] over the slots whose sorted row lies in
+    [row_lo, row_hi) -> y [T,H], bf16 (or fp32 with fp32=True)."""
+    L = load()
+    T, k = topk_weights.shape
+    P, H = o.shape
+    row_hi = T * k if row_hi is None else row_hi
+    po = _dev(o, "o", torch.bfloat16, (P, H))
+    pi = _dev(inv, "inv", torch.int32, (T * k,))
+    pw = _dev(topk_weights, "topk_weights", torch.float32, (T, k))
+    dt = torch.float32 if fp32 else torch.bfloat16
+    y = torch.empty((T, H), dtype=dt, device=o.device) if out is None else out
+    py = _dev(y, "out", dt, (T, H))
+    if T:
+        _check(L.moe_combine(po, pi, pw, T, k, H, row_lo, row_hi,
+                             MOE_COMBINE_F32 if fp32 else 0, py, _stream_ptr(stream)),
+               "moe_combine")
+    return y
+
+
 def router_stats(aux: dict) -> dict:
     """Decode aux["router_stats"] of a forward(..., aux=True) call."""
     import struct
@@ -278,11 +383,9 @@ def last_stage_times() -> dict[str, float]:
     return {L.moe_stage_name(i).decode(): float(buf[i]) for i in range(n)}
 
 
-def ffn_kernel_name(T: int, tiles: str = "auto") -> str:
+def ffn_kernel_name(T: int, tiles: str = "auto", rows: str = "auto") -> str:
     """The expert-FFN kernel moe_forward launches for T tokens with this tile choice."""
-    if tiles not in _TILE_FLAGS:
-        raise ValueError(f"tiles must be one of {sorted(_TILE_FLAGS)}")
-    return load().moe_ffn_kernel_name(int(T), _TILE_FLAGS[tiles]).decode()
+    return load().moe_ffn_kernel_name(int(T), _flags(True, "auto", False, tiles, rows)).decode()
 
 
 def last_kernel_count() -> int:
@@ -302,17 +405,17 @@ class ForwardGraph:
     """
 
     def __init__(self, x, w_router, w_gate, w_up, w_down, k, bias=None, renorm=True,
-                 profile=False, router="auto", tiles="auto"):
+                 profile=False, router="auto", tiles="auto", rows="auto"):
         self.x = x
         T, H = x.shape
         E, _, I = w_gate.shape
         self.y = torch.empty((T, H), dtype=torch.bfloat16, device=x.device)
-        flags = _flags(renorm, router, profile, tiles)
+        flags = _flags(renorm, router, profile, tiles, rows)
         self.workspace = torch.empty(max(1, workspace_bytes(T, H, E, I, k, flags)),
                                      dtype=torch.uint8, device=x.device)
         self._args = (w_router, w_gate, w_up, w_down, k)
         self._kw = dict(bias=bias, renorm=renorm, profile=profile, workspace_buf=self.workspace,
-                        router=router, tiles=tiles)
+                        router=router, tiles=tiles, rows=rows)
         forward(self.x, *self._args, out=self.y, **self._kw)    # set-up + workspace, uncaptured
         torch.cuda.synchronize(x.device)
         self.graph = torch.cuda.CUDAGraph()

@@ -378,11 +378,13 @@ __global__ void __launch_bounds__(256) dispatch_small_kernel(
                        s_tstart);
 }
 
-// Xp[pos, :] = x[perm[pos] / k, :]   (16-byte vectors over all (row, vector) pairs,
-// 8 loads per thread issued before the stores)
+// Xp[pos, :] = x[perm[pos] / k, :] for pos < P   (16-byte vectors over all (row, vector)
+// pairs, 8 loads per thread issued before the stores).  perm holds pair indices t*k + j below
+// n_pairs (it may be a slice of a longer permutation).
 __global__ void __launch_bounds__(256) gather_rows_kernel(const uint4* __restrict__ x,
                                                           const int32_t* __restrict__ perm, int P,
-                                                          int k, int nvec, uint4* __restrict__ xp) {
+                                                          int k, int n_pairs, int nvec,
+                                                          uint4* __restrict__ xp) {
   pdl_trigger();
   pdl_wait();
   // After a timeout upstream perm may be stale: skip the work (the error word says why).
@@ -400,7 +402,7 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const uint4* __restric
       if (idx < total) {
         const int pos = (int)(idx / nvec), v = (int)(idx - (long long)pos * nvec);
         const int q = perm[pos];
-        if ((unsigned)q < (unsigned)P) {   // the source row t = q / k is then < T
+        if ((unsigned)q < (unsigned)n_pairs) {   // the source row t = q / k is then < T
           r[u] = x[(size_t)(q / k) * nvec + v];
           ok[u] = true;
         } else {
@@ -416,15 +418,20 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const uint4* __restric
   }
 }
 
-// y[t, :] = sum_{j ascending} w[t,j] * O[inv[t,j], :]   (fp32, one bf16 rounding)
+// y[t, :] = sum_{j ascending} w[t,j] * O[inv[t,j], :]   (fp32, one rounding to the output)
 // One warp per item (token t, chunk c of 64 16-byte vectors of the row): lanes j < k fetch
 // slot j's row and weight, which the warp shares by shuffles; then each lane loads its two
-// vectors of all k rows (16 loads in flight) and sums them in slot order.
+// vectors of all k rows (16 loads in flight) and sums them in slot order.  Only sorted rows
+// in [row_lo, row_hi) contribute (the rest count as zero): the whole layer passes [0, T*k);
+// an expert-parallel rank passes the rows of its own experts and writes an fp32 partial sum
+// (F32OUT) for the cross-rank reduction.  y holds 8 values per 16-byte vector of O.
 constexpr int kCombineChunkVec = 64;
+template <bool F32OUT>
 __global__ void __launch_bounds__(256) combine_kernel(const uint4* __restrict__ O,
                                                       const int32_t* __restrict__ inv,
                                                       const float* __restrict__ w, int T, int k,
-                                                      int nvec, uint4* __restrict__ y) {
+                                                      int nvec, int row_lo, int row_hi,
+                                                      void* __restrict__ y_out) {
   pdl_trigger();
   pdl_wait();
   // After a timeout upstream inv may be stale: skip the work (the error word says why).
@@ -439,15 +446,21 @@ __global__ void __launch_bounds__(256) combine_kernel(const uint4* __restrict__ 
     const int t = (int)(it / nch), c = (int)(it - (long long)t * nch);
     int myp = 0;
     float myw = 0.f;
+    bool myon = false;
     if (lane < k) {
       myp = __ldg(inv + (size_t)t * k + lane);
       myw = __ldg(w + (size_t)t * k + lane);
       if ((unsigned)myp >= (unsigned)P) {   // never written so: read nothing for this slot
         raise_error(MOE_DEVERR_BAD_INDEX);
+      } else {
+        myon = myp >= row_lo && myp < row_hi;
+      }
+      if (!myon) {
         myp = 0;
         myw = 0.f;
       }
     }
+    const unsigned on = __ballot_sync(0xffffffffu, myon);
     int pos[8];
     float wj[8];
 #pragma unroll
@@ -460,8 +473,10 @@ __global__ void __launch_bounds__(256) combine_kernel(const uint4* __restrict__ 
     uint4 r0[8], r1[8];
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
-      if (j < k && ok0) r0[j] = __ldcs(O + (size_t)pos[j] * nvec + v0);
-      if (j < k && ok1) r1[j] = __ldcs(O + (size_t)pos[j] * nvec + v1);
+      r0[j] = r1[j] = make_uint4(0u, 0u, 0u, 0u);
+      const bool use = j < k && ((on >> j) & 1u);
+      if (use && ok0) r0[j] = __ldcs(O + (size_t)pos[j] * nvec + v0);
+      if (use && ok1) r1[j] = __ldcs(O + (size_t)pos[j] * nvec + v1);
     }
 #pragma unroll
     for (int half = 0; half < 2; ++half) {
@@ -472,7 +487,7 @@ __global__ void __launch_bounds__(256) combine_kernel(const uint4* __restrict__ 
       for (int i = 0; i < 8; ++i) acc[i] = 0.f;
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
-        if (j < k) {
+        if (j < k && ((on >> j) & 1u)) {
           const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&r[j]);
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
@@ -482,12 +497,71 @@ __global__ void __launch_bounds__(256) combine_kernel(const uint4* __restrict__ 
           }
         }
       }
-      uint4 out;
-      out.x = pack_bf16x2(acc[0], acc[1]);
-      out.y = pack_bf16x2(acc[2], acc[3]);
-      out.z = pack_bf16x2(acc[4], acc[5]);
-      out.w = pack_bf16x2(acc[6], acc[7]);
-      y[(size_t)t * nvec + (half == 0 ? v0 : v1)] = out;
+      const size_t vi = (size_t)t * nvec + (half == 0 ? v0 : v1);
+      if (F32OUT) {
+        float4* yo = static_cast<float4*>(y_out) + 2 * vi;
+        yo[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+        yo[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
+      } else {
+        uint4 out;
+        out.x = pack_bf16x2(acc[0], acc[1]);
+        out.y = pack_bf16x2(acc[2], acc[3]);
+        out.z = pack_bf16x2(acc[4], acc[5]);
+        out.w = pack_bf16x2(acc[6], acc[7]);
+        static_cast<uint4*>(y_out)[vi] = out;
+      }
+    }
+  }
+}
+
+// Tile list of a grouped FFN over caller-given row segments (one CTA): segment i holds
+// seg_rows[i] consecutive rows of local expert seg_expert[i], segments back to back from row
+// 0.  Tiles of BM rows never cross a segment.  Also zeroes the FFN's counters.  A segment
+// with an expert id outside [0, E) or a negative row count raises BAD_INDEX and gets no tiles;
+// segments that add up to more than N rows (the rows the caller's buffers hold) raise
+// BAD_INDEX and produce no tiles at all, so nothing is read or written past row N.
+constexpr int kMaxSegments = 1024;
+__global__ void __launch_bounds__(256) segment_tiles_kernel(
+    const int32_t* __restrict__ seg_rows, const int32_t* __restrict__ seg_expert, int n_seg,
+    int N, int E, int BM, int max_tiles, int32_t* __restrict__ tile_num,
+    int32_t* __restrict__ tile_expert, int32_t* __restrict__ tile_row0,
+    int32_t* __restrict__ tile_rows, int32_t* __restrict__ counters, int n_counters) {
+  pdl_trigger();
+  pdl_wait();
+  __shared__ int s_start[kMaxSegments], s_tstart[kMaxSegments];
+  for (int i = threadIdx.x; i < n_counters; i += blockDim.x) counters[i] = 0;
+  if (threadIdx.x == 0) {
+    // segments are few (ranks x local experts): a serial scan keeps the order obvious
+    int row = 0, tt = 0;
+    for (int i = 0; i < n_seg; ++i) {
+      int n = __ldg(seg_rows + i);
+      const int e = __ldg(seg_expert + i);
+      if (n < 0 || (n > 0 && (unsigned)e >= (unsigned)E)) {
+        raise_error(MOE_DEVERR_BAD_INDEX);
+        n = -1;
+      }
+      s_start[i] = row;
+      s_tstart[i] = n > 0 ? tt : -1;
+      if (n > 0) {
+        row += n;
+        tt += (n + BM - 1) / BM;
+      }
+    }
+    if (row > N || tt > max_tiles) {   // more rows than the caller's buffers hold
+      raise_error(MOE_DEVERR_BAD_INDEX);
+      tt = 0;
+    }
+    *tile_num = tt;
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < n_seg; i += blockDim.x) {
+    const int t0 = s_tstart[i];
+    if (t0 < 0 || *tile_num == 0) continue;
+    const int n = __ldg(seg_rows + i), e = __ldg(seg_expert + i);
+    for (int m = 0; m * BM < n; ++m) {
+      tile_expert[t0 + m] = e;
+      tile_row0[t0 + m] = s_start[i] + m * BM;
+      tile_rows[t0 + m] = min(BM, n - m * BM);
     }
   }
 }

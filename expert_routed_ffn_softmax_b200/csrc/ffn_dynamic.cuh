@@ -70,13 +70,15 @@ __device__ __forceinline__ bool dy_narrow_block(const DyChunk& d, const PGemm& g
 }
 
 // tmH: h rows, box R rows x 64 columns.  tmWg / tmWu: two-slab boxes; tmWg1 / tmWu1: one-slab
-// boxes (the narrow last GEMM-1 block).
+// boxes (the narrow last GEMM-1 block).  tmX: GEMM-1's A rows when tiles.a_tma (box R rows x
+// 64 columns of a contiguous row-major tensor), else unused.
 template <int R>
 __global__ void __launch_bounds__(PG_MAX_THREADS, 1)
     expert_ffn_dynamic_kernel(const __grid_constant__ CUtensorMap tmWg,
                               const __grid_constant__ CUtensorMap tmWu,
                               const __grid_constant__ CUtensorMap tmWg1,
                               const __grid_constant__ CUtensorMap tmWu1,
+                              const __grid_constant__ CUtensorMap tmX,
                               const __grid_constant__ CUtensorMap tmH,
                               const __grid_constant__ CUtensorMap tmWd, TileList tiles,
                               PGemm g1, PGemm g2, int* __restrict__ h_ready, DyState dy) {
@@ -133,6 +135,7 @@ __global__ void __launch_bounds__(PG_MAX_THREADS, 1)
       tma_prefetch_desc(&tmWg1);
       tma_prefetch_desc(&tmWu1);
     }
+    if (tiles.a_tma) tma_prefetch_desc(&tmX);
     tma_prefetch_desc(&tmH);
     tma_prefetch_desc(&tmWd);
   }
@@ -195,15 +198,23 @@ __global__ void __launch_bounds__(PG_MAX_THREADS, 1)
           }
           const uint32_t sA = base + s * STAGE_BYTES;
           const uint32_t sB = sA + A_BYTES;
-          if (narrow) {
-            mbar_arrive_expect_tx(full_bar(s), 2 * GM_SLAB_BYTES);
-            tma_load_4d(sB, &tmWg1, full_bar(s), 0, kc * GM_BK, n0 / 64, e);
-            tma_load_4d(sB + GM_SLAB_BYTES, &tmWu1, full_bar(s), 0, kc * GM_BK, n0 / 64, e);
-          } else if (d.phase == 0) {
-            mbar_arrive_expect_tx(full_bar(s), NSLAB * GM_SLAB_BYTES);
-            tma_load_4d(sB, &tmWg, full_bar(s), 0, kc * GM_BK, n0 / 64, e);
-            tma_load_4d(sB + (NSLAB / 2) * GM_SLAB_BYTES, &tmWu, full_bar(s), 0, kc * GM_BK,
-                        n0 / 64, e);
+          if (d.phase == 0) {
+            const uint32_t b_bytes = (narrow ? 2 : NSLAB) * GM_SLAB_BYTES;
+            if (tiles.a_tma) {
+              mbar_arrive_expect_tx(full_bar(s), b_bytes + A_BYTES);
+              mbar_arrive_cnt(full_bar(s), PG_GATHER_THREADS);   // in place of the gather warps
+              tma_load_2d(sA, &tmX, full_bar(s), kc * GM_BK, row0);
+            } else {
+              mbar_arrive_expect_tx(full_bar(s), b_bytes);
+            }
+            if (narrow) {
+              tma_load_4d(sB, &tmWg1, full_bar(s), 0, kc * GM_BK, n0 / 64, e);
+              tma_load_4d(sB + GM_SLAB_BYTES, &tmWu1, full_bar(s), 0, kc * GM_BK, n0 / 64, e);
+            } else {
+              tma_load_4d(sB, &tmWg, full_bar(s), 0, kc * GM_BK, n0 / 64, e);
+              tma_load_4d(sB + (NSLAB / 2) * GM_SLAB_BYTES, &tmWu, full_bar(s), 0, kc * GM_BK,
+                          n0 / 64, e);
+            }
           } else {
             mbar_arrive_expect_tx(full_bar(s), A_BYTES + NSLAB * GM_SLAB_BYTES);
             mbar_arrive_cnt(full_bar(s), PG_GATHER_THREADS);   // in place of the gather warps
@@ -272,7 +283,7 @@ __global__ void __launch_bounds__(PG_MAX_THREADS, 1)
             break;
           }
           *n_consumed = q + 1;
-          if (d.phase == 0) fence_proxy_async_smem();   // A came through the generic proxy
+          if (d.phase == 0 && !tiles.a_tma) fence_proxy_async_smem();   // A came by cp.async
           tc_fence_after();
           const uint32_t sA = base + s * STAGE_BYTES;
           const uint32_t sB = sA + A_BYTES;
@@ -364,8 +375,9 @@ __global__ void __launch_bounds__(PG_MAX_THREADS, 1)
   } else {
     // -------------------------------------------------------------- A-row gather (warps 6-7)
     // GEMM-1 units: the <= R rows of the tile, 16-byte cp.async into the 128-byte-swizzled
-    // slot (chunk c of row r at byte 128 r + 16 (c ^ r)).  GEMM-2 units: nothing (the TMA
-    // thread arrives in their place), but the stage count must follow.
+    // slot (chunk c of row r at byte 128 r + 16 (c ^ r)).  GEMM-2 units, and GEMM-1 units
+    // whose A rows come by TMA: nothing (the TMA thread arrives in their place), but the
+    // stage count must follow.
     const int gw = warp - 6, sub = lane >> 3, ch = lane & 7;
     int q = 0;
     for (int i = 0;; ++i) {
@@ -379,7 +391,7 @@ __global__ void __launch_bounds__(PG_MAX_THREADS, 1)
         break;
       }
       const DyChunk d = dy_decode(c, U1, nk1, nk2);
-      if (d.phase == 1) {
+      if (d.phase == 1 || tiles.a_tma) {
         q += d.ke - d.kb;
         continue;
       }

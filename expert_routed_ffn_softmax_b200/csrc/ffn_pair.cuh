@@ -24,9 +24,11 @@
 //                  form, whose byte count lands on rank 0's full barrier; rank 0 announces
 //                  the bytes of both.  No load uses cluster multicast.
 //   warp 1 lane 0  rank 0: MMA issuer (tcgen05.mma.cta_group::2; commits arrive on both
-//                  CTAs' barriers).  Rank 1: forwards "A rows landed" -- its gather warps
-//                  complete a local barrier, this thread then arrives on rank 0's full
-//                  barrier (cp.async cannot signal another CTA's barrier).
+//                  CTAs' barriers).  Rank 1: forwards "A rows landed" for the stages whose A
+//                  rows its gather warps copy -- they complete a local barrier, this thread
+//                  then arrives on rank 0's full barrier (cp.async cannot signal another CTA's
+//                  barrier).  Stages loaded by TMA alone need no forward: their bytes count on
+//                  rank 0's barrier and rank 0's producer arrives for rank 1.
 //   warps 2-5      epilogue from this CTA's TMEM (its 128 rows): GEGLU + bf16 h, or bf16 O;
 //                  releases the accumulator to rank 0 and publishes h_ready.
 //   warps 6-7      GEMM-1 A-row gather of this CTA's 128 rows from x through perm (cp.async
@@ -49,6 +51,7 @@ constexpr int PR_SMEM = 1024 + PR_STAGES * PR_STAGE_BYTES + 2048;
 constexpr int PR_DESC_READERS = 7 + 8;
 constexpr int PR_EPI_WARPS = 8;                        // accumulator releases per unit (both CTAs)
 
+
 // (expert, first sorted row, rows <= 256, first output column) of pair unit `unit`.
 __device__ __forceinline__ void pr_tile_info(const TileList& tiles, int n_blocks, int unit,
                                              bool geglu, int& e, int& row0, int& rows, int& n0) {
@@ -67,12 +70,14 @@ __device__ __forceinline__ void pr_tile_info(const TileList& tiles, int n_blocks
 }
 
 // tmWg / tmWu: two-slab boxes of W_gate / W_up; tmWg1 / tmWu1: one-slab boxes (narrow last
-// GEMM-1 block); tmH: 128 rows x 64 columns of h; tmWd: two-slab boxes of W_down.
+// GEMM-1 block); tmX: 128 rows x 64 columns of GEMM-1's A rows when tiles.a_tma; tmH: 128
+// rows x 64 columns of h; tmWd: two-slab boxes of W_down.
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PG_MAX_THREADS, 1)
     expert_ffn_pair_kernel(const __grid_constant__ CUtensorMap tmWg,
                            const __grid_constant__ CUtensorMap tmWu,
                            const __grid_constant__ CUtensorMap tmWg1,
                            const __grid_constant__ CUtensorMap tmWu1,
+                           const __grid_constant__ CUtensorMap tmX,
                            const __grid_constant__ CUtensorMap tmH,
                            const __grid_constant__ CUtensorMap tmWd, TileList tiles, PGemm g1,
                            PGemm g2, int* __restrict__ h_ready, DyState dy) {
@@ -114,7 +119,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PG_MAX_THREADS, 1)
       // thread for them), rank 1's forwarder
       mbar_init(full_bar(s), 1 + PG_GATHER_THREADS + 1);
       mbar_init(empty_bar(s), 1);
-      mbar_init(afull_bar(s), PG_GATHER_THREADS);   // rank 1: its gather threads
+      mbar_init(afull_bar(s), PG_GATHER_THREADS);   // rank 1: its gather threads (per
+                                                     // gathered stage, in gather order)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(tfull_bar(b), 1);
@@ -134,6 +140,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PG_MAX_THREADS, 1)
       tma_prefetch_desc(&tmWg1);
       tma_prefetch_desc(&tmWu1);
     }
+    if (tiles.a_tma) tma_prefetch_desc(&tmX);
     tma_prefetch_desc(&tmH);
     tma_prefetch_desc(&tmWd);
   }
@@ -177,7 +184,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PG_MAX_THREADS, 1)
       while (true) {
         if (leader) {
           const int r = i % DY_RING;
-          if (i >= DY_RING && !mbar_wait_cl(dempty_bar(r), ((i / DY_RING) - 1) & 1)) {
+          if (i >= DY_RING && !mbar_wait(dempty_bar(r), ((i / DY_RING) - 1) & 1)) {
             *abort_flag = 1;
             break;
           }
@@ -186,7 +193,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PG_MAX_THREADS, 1)
           ring[r] = v;
           st_cluster_u32(at_peer(ring_addr + 4u * r), static_cast<uint32_t>(v));
           mbar_arrive(dfull_bar(r));
-          mbar_arrive_remote(at_peer(dfull_bar(r)));   // release: the ring store first
+          mbar_arrive_remote_publish(at_peer(dfull_bar(r)));   // after the ring store
           if (stop) break;
         } else {
           c = read_desc(i);
@@ -206,24 +213,32 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PG_MAX_THREADS, 1)
         // deferred, its h rows); the bytes count on rank 0's full barrier.
         auto stage_in = [&](int kc, int qq, bool with_a) -> bool {
           const int s = qq % S;
-          if (*abort_flag || (qq >= S && !mbar_wait_cl(empty_bar(s), ((qq / S) - 1) & 1))) {
+          if (*abort_flag || (qq >= S && !mbar_wait(empty_bar(s), ((qq / S) - 1) & 1))) {
             *abort_flag = 1;
             return false;
           }
           const uint32_t sA = base + s * PR_STAGE_BYTES;
           const uint32_t sB = sA + PR_A_BYTES;
           const uint32_t fb = leader ? full_bar(s) : at_leader(full_bar(s));
+          // Rank 0 announces the bytes of both CTAs; on a stage without gathered rows it
+          // also arrives for both CTAs' gather warps and for rank 1's forwarder.
           if (d.phase == 0) {
-            if (leader)
-              mbar_arrive_expect_tx(fb, narrow ? 2 * GM_SLAB_BYTES : 2 * PR_B_BYTES);
+            const uint32_t b_bytes = narrow ? 2 * GM_SLAB_BYTES : 2 * PR_B_BYTES;
+            if (leader) {
+              if (tiles.a_tma) {
+                mbar_arrive_expect_tx(fb, b_bytes + 2 * PR_A_BYTES);
+                mbar_arrive_cnt(fb, PG_GATHER_THREADS + 1);
+              } else {
+                mbar_arrive_expect_tx(fb, b_bytes);
+              }
+            }
+            if (tiles.a_tma) tma_load_2d_pair(sA, &tmX, fb, kc * GM_BK, row0 + half0);
             const CUtensorMap* m = narrow ? (leader ? &tmWg1 : &tmWu1) : (leader ? &tmWg : &tmWu);
             tma_load_4d_pair(sB, m, fb, 0, kc * GM_BK, n0 / 64, e);
           } else {
             if (leader) {
               mbar_arrive_expect_tx(fb, 2 * (PR_A_BYTES + PR_B_BYTES));
-              mbar_arrive_cnt(fb, PG_GATHER_THREADS);      // in place of the gather warps
-            } else {
-              mbar_arrive_cnt(afull_bar(s), PG_GATHER_THREADS);
+              mbar_arrive_cnt(fb, PG_GATHER_THREADS + 1);
             }
             tma_load_4d_pair(sB, &tmWd, fb, 0, kc * GM_BK, n0 / 64 + (leader ? 0 : 2), e);
             if (with_a) tma_load_2d_pair(sA, &tmH, fb, kc * GM_BK, row0 + half0);
@@ -266,7 +281,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PG_MAX_THREADS, 1)
       if (!*abort_flag) {
         const int qe = *n_issued;
         for (int qq = max(0, qe - S); qq < qe; ++qq)
-          if (!mbar_wait_cl(empty_bar(qq % S), (qq / S) & 1)) {
+          if (!mbar_wait(empty_bar(qq % S), (qq / S) & 1)) {
             *abort_flag = 1;
             break;
           }
@@ -288,7 +303,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PG_MAX_THREADS, 1)
         const DyChunk d = dy_decode(c, U1, nk1, nk2);
         const uint32_t idesc = dy_narrow_block(d, g1) ? idesc_narrow : idesc_full;
         const int b = i & 1, use = i >> 1;
-        if (use >= 1 && !mbar_wait_cl(tempty_bar(b), (use - 1) & 1)) {
+        if (use >= 1 && !mbar_wait(tempty_bar(b), (use - 1) & 1)) {
           *abort_flag = 1;
           break;
         }
@@ -297,12 +312,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PG_MAX_THREADS, 1)
         bool ok = true;
         for (int kc = d.kb; kc < d.ke; ++kc, ++q) {
           const int s = q % S;
-          if (!mbar_wait_cl(full_bar(s), (q / S) & 1)) {
+          if (!mbar_wait(full_bar(s), (q / S) & 1)) {
             ok = false;
             break;
           }
           *n_consumed = q + 1;
-          if (d.phase == 0) fence_proxy_async_smem();   // A came through the generic proxy
+          if (d.phase == 0 && !tiles.a_tma) fence_proxy_async_smem();   // A came by cp.async
           tc_fence_after();
           const uint32_t sA = base + s * PR_STAGE_BYTES;
           const uint32_t sB = sA + PR_A_BYTES;
@@ -322,7 +337,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PG_MAX_THREADS, 1)
       }
     } else if (lane == 0) {
       // ------------------------------------------------ A-rows-landed forwarder (rank 1)
-      int q = 0;
+      // q: stage (shared-memory slot q % S); qa: gathered stage (A barrier qa % S)
+      int q = 0, qa = 0;
       for (int i = 0;; ++i) {
         const int c = read_desc(i);
         release_desc(i);
@@ -331,14 +347,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PG_MAX_THREADS, 1)
           break;
         }
         const DyChunk d = dy_decode(c, U1, nk1, nk2);
+        if (d.phase == 1 || tiles.a_tma) {
+          q += d.ke - d.kb;
+          continue;
+        }
         bool ok = true;
-        for (int kc = d.kb; kc < d.ke; ++kc, ++q) {
+        for (int kc = d.kb; kc < d.ke; ++kc, ++q, ++qa) {
           const int s = q % S;
-          if (!mbar_wait_cl(afull_bar(s), (q / S) & 1)) {
+          if (!mbar_wait(afull_bar(qa % S), (qa / S) & 1)) {
             ok = false;
             break;
           }
-          fence_proxy_async_cluster();   // the gathered rows, for the pair MMA's reads
+          fence_proxy_async_smem();   // the gathered rows, for the pair MMA's reads
           mbar_arrive_remote(at_leader(full_bar(s)));
         }
         if (!ok) {
@@ -363,7 +383,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PG_MAX_THREADS, 1)
       }
       const DyChunk d = dy_decode(c, U1, nk1, nk2);
       const int b = i & 1, use = i >> 1;
-      bool got = mbar_wait_cl(tfull_bar(b), use & 1);
+      bool got = mbar_wait(tfull_bar(b), use & 1);
       tc_fence_after();
       got = __all_sync(0xffffffffu, got && !*abort_flag);
       if (!got) {
@@ -421,10 +441,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PG_MAX_THREADS, 1)
     // -------------------------------------------------------------- A-row gather (warps 6-7)
     // GEMM-1 units: this CTA's <= 128 rows of the pair tile, 16-byte cp.async into the
     // 128-byte-swizzled slot (chunk c of row r at byte 128 r + 16 (c ^ r)); rank 0's complete
-    // its full barrier, rank 1's its local A barrier (forwarded by warp 1).  GEMM-2 units:
-    // nothing (the TMA thread arrives in their place), but the stage count must follow.
+    // its full barrier, rank 1's its local A barrier (forwarded by warp 1).  GEMM-2 units,
+    // and GEMM-1 units whose A rows come by TMA: nothing (rank 0's TMA thread arrives in
+    // their place), but the stage count must follow.
     const int gw = warp - 6, sub = lane >> 3, ch = lane & 7;
-    int q = 0;
+    int q = 0, qa = 0;   // stage, gathered stage (rank 1's A barrier qa % S)
     for (int i = 0;; ++i) {
       int c = 0;
       if (lane == 0) c = read_desc(i);
@@ -436,7 +457,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PG_MAX_THREADS, 1)
         break;
       }
       const DyChunk d = dy_decode(c, U1, nk1, nk2);
-      if (d.phase == 1) {
+      if (d.phase == 1 || tiles.a_tma) {
         q += d.ke - d.kb;
         continue;
       }
@@ -466,9 +487,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PG_MAX_THREADS, 1)
         doff[u] = static_cast<uint32_t>(r * 128 + ((ch ^ (r & 7)) << 4));
       }
       bool stop = false;
-      for (int kc = d.kb; kc < d.ke; ++kc, ++q) {
+      for (int kc = d.kb; kc < d.ke; ++kc, ++q, ++qa) {
         const int s = q % S;
-        bool ok = !*abort_flag && (q < S || mbar_wait_cl(empty_bar(s), ((q / S) - 1) & 1));
+        bool ok = !*abort_flag && (q < S || mbar_wait(empty_bar(s), ((q / S) - 1) & 1));
         if (!__all_sync(0xffffffffu, ok)) {
           *abort_flag = 1;
           stop = true;
@@ -478,7 +499,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PG_MAX_THREADS, 1)
 #pragma unroll
         for (int u = 0; u < NI; ++u)
           if (src[u] != nullptr) cp_async_16(sA + doff[u], src[u] + kc * GM_BK);
-        cp_async_arrive_noinc(leader ? full_bar(s) : afull_bar(s));
+        cp_async_arrive_noinc(leader ? full_bar(s) : afull_bar(qa % S));
       }
       if (stop) break;
     }

@@ -47,6 +47,9 @@ struct TileList {
   const __nv_bfloat16* src = nullptr;
   int ld = 0;         // row stride of src (elements; a multiple of 8)
   int src_rows = 0;   // rows of src
+  // 1: the A rows of GEMM-1 are rows row0.. of a contiguous row-major tensor (the tile's rows
+  // already in sorted order), loaded by TMA like GEMM-2's h rows; the gather warps idle.
+  int a_tma = 0;
 };
 
 template <int NSLAB>

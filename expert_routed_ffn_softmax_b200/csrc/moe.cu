@@ -39,9 +39,16 @@ constexpr unsigned kKnownFlags = MOE_FLAG_NO_RENORM | MOE_FLAG_ROUTER_FP64 |
                                  MOE_FLAG_ROUTER_SCREEN | MOE_FLAG_PROFILE_STAGES |
                                  MOE_FLAG_DECODE_TILES | MOE_FLAG_PREFILL_TILES |
                                  MOE_FLAG_UNFUSED_FFN | MOE_FLAG_FUSED_FFN |
-                                 MOE_FLAG_FFN_PAIRS | MOE_FLAG_FFN_SINGLE;
-// Batches of at least this many tokens run the expert FFN on CTA pairs by default.
-constexpr int kPairMinTokens = 2048;
+                                 MOE_FLAG_FFN_PAIRS | MOE_FLAG_FFN_SINGLE |
+                                 MOE_FLAG_FFN_ROWS_COPY | MOE_FLAG_FFN_ROWS_GATHER;
+// Default tile form of the routed layer's expert FFN: single CTAs at every batch size.
+// Measured on B200 (FFN stage, T = 32768): single CTAs 3.14 ms with the in-kernel row gather;
+// CTA pairs 3.78 ms with it -- the second CTA's gathered rows must be forwarded to the MMA's
+// barrier -- and 2.96 ms (single CTAs 3.01 ms) when the rows are first copied in expert order
+// and loaded by TMA, but that copy costs 0.58 ms.  The dense MLP, whose rows need no copy,
+// runs on pairs from kDensePairMinTokens tokens (T = 32768: 0.85 ms, 0.83 of the bf16 peak).
+constexpr int kPairMinTokens = 1 << 30;
+constexpr int kDensePairMinTokens = 2048;
 
 #define GEMM_GEGLU grouped_gemm_persistent_kernel<kGemmStages, EPI_GEGLU, 4, true>
 #define GEMM_FFN grouped_gemm_persistent_kernel<kGemmStages, EPI_GEGLU, 4, true, true>
@@ -57,8 +64,9 @@ bool flags_ok(unsigned flags) {
   if ((flags & MOE_FLAG_DECODE_TILES) && (flags & MOE_FLAG_PREFILL_TILES)) return false;
   if ((flags & MOE_FLAG_UNFUSED_FFN) && (flags & MOE_FLAG_FUSED_FFN)) return false;
   const unsigned tiles = MOE_FLAG_FFN_PAIRS | MOE_FLAG_FFN_SINGLE;
-  if ((flags & tiles) == tiles) return false;
-  if ((flags & tiles) &&
+  const unsigned rows = MOE_FLAG_FFN_ROWS_COPY | MOE_FLAG_FFN_ROWS_GATHER;
+  if ((flags & tiles) == tiles || (flags & rows) == rows) return false;
+  if ((flags & (tiles | rows)) &&
       (flags & (MOE_FLAG_FUSED_FFN | MOE_FLAG_UNFUSED_FFN | MOE_FLAG_DECODE_TILES)))
     return false;
   return true;
@@ -89,10 +97,18 @@ int dy_rows(int T, unsigned flags) {
 }
 
 // The dynamic FFN on CTA pairs (256-row tiles, tcgen05 cta_group::2): batches of more than
-// 64 tokens, from kPairMinTokens tokens by default.
+// 64 tokens, when asked for (kPairMinTokens sets the default).
 bool use_pair_ffn(int T, unsigned flags) {
   if (dy_rows(T, flags) != 128 || (flags & MOE_FLAG_FFN_SINGLE)) return false;
   return (flags & MOE_FLAG_FFN_PAIRS) || T >= kPairMinTokens;
+}
+
+// GEMM-1's A rows for the dynamic FFN of more than 64 tokens: copied into an expert-sorted
+// buffer and loaded by TMA, or gathered inside the kernel (the default: see kPairMinTokens).
+constexpr int kRowCopyMinTokens = 1 << 30;
+bool use_row_copy(int T, unsigned flags) {
+  if (dy_rows(T, flags) != 128 || (flags & MOE_FLAG_FFN_ROWS_GATHER)) return false;
+  return (flags & MOE_FLAG_FFN_ROWS_COPY) || T >= kRowCopyMinTokens;
 }
 
 // Batches of at most 16 tokens (so at most 16 rows per expert) use the decode GEMMs.
@@ -206,7 +222,7 @@ Layout make_layout(int T, int H, int E, int I, int k, unsigned flags, bool forwa
     L.tile_rows = take(sizeof(int32_t) * L.max_tiles);
     // Xp (expert-sorted copies of the x rows) only for the decode tiles; the prefill tiles
     // gather the rows straight from x
-    if (L.bm == DG_BN) L.xp = take(2 * P * H);
+    if (L.bm == DG_BN || use_row_copy(T, flags)) L.xp = take(2 * P * H);
     L.hbuf = take(2 * P * I);
     L.obuf = take(2 * P * H);
     // stream-K split tiles of the statically scheduled GEMMs: two fp32 tile slots per CTA
@@ -663,7 +679,7 @@ moe_status_t moe_forward(const void* x, const void* w_router, const float* route
            front_done);
     if (dec)   // decode tiles read a gathered copy of the routed rows
       launch(true, gather_rows_kernel, dim3(std::min((P + 7) / 8, gsm)), dim3(256), 0,
-             static_cast<const uint4*>(x), (const int32_t*)perm, P, k, H / 8,
+             static_cast<const uint4*>(x), (const int32_t*)perm, P, k, P, H / 8,
              reinterpret_cast<uint4*>(xp));
     if (const moe_status_t ls = launched(); ls != MOE_OK) return ls;
     prof.mark();
@@ -701,16 +717,17 @@ moe_status_t moe_forward(const void* x, const void* w_router, const float* route
              (kRankWarps + 1) * E * sizeof(int),
              (const int32_t*)ids, P, E, (const int32_t*)chunk_base, perm, inv);
     }
-    if (dec)
+    if (dec || use_row_copy(T, flags))   // the routed rows, in expert order
       launch(true, gather_rows_kernel, dim3(std::min((P + 7) / 8, gsm)), dim3(256), 0,
-             static_cast<const uint4*>(x), (const int32_t*)perm, P, k, H / 8,
+             static_cast<const uint4*>(x), (const int32_t*)perm, P, k, P, H / 8,
              reinterpret_cast<uint4*>(xp));
     if (const moe_status_t ls = launched(); ls != MOE_OK) return ls;
     prof.mark();
   }
   // 3. GEMM-1 + GEGLU, 4. GEMM-2 (down)
-  const TileList tl{tile_num, tile_expert, tile_row0, tile_rows, 0, perm, k,
-                    static_cast<const __nv_bfloat16*>(x), H, T};
+  TileList tl{tile_num, tile_expert, tile_row0, tile_rows, 0, perm, k,
+              static_cast<const __nv_bfloat16*>(x), H, T};
+  tl.a_tma = use_row_copy(T, flags) ? 1 : 0;
   float* partials = reinterpret_cast<float*>(ws + L.partials);
   float* partials2 = reinterpret_cast<float*>(ws + L.partials2);
   const int G = std::min(std::max(1, d->num_sms), kMaxGemmCtas);
@@ -733,24 +750,26 @@ moe_status_t moe_forward(const void* x, const void* w_router, const float* route
     if (const int R = dy_rows(T, flags); R > 0) {
       // at most R rows per tile, whole units handed out from a shared counter; one-slab
       // weight maps for a narrow last GEMM-1 block (I % 128 == 64)
-      CUtensorMap tm_hr, tm_wg1, tm_wu1;
+      CUtensorMap tm_hr, tm_wg1, tm_wu1, tm_xr;
       if (!make_map_2d(&tm_hr, hbuf, I, P, R, 64) ||
           !make_map_slabs(&tm_wg1, w_gate, I, H, E, 64, 1) ||
-          !make_map_slabs(&tm_wu1, w_up, I, H, E, 64, 1))
+          !make_map_slabs(&tm_wu1, w_up, I, H, E, 64, 1) ||
+          !make_map_2d(&tm_xr, tl.a_tma ? (const void*)xp : x, H, tl.a_tma ? P : T, R, 64))
         return cuda_failed(-1);
       int32_t* dctr = gemm_counters + L.dy_ctr;
       const DyState dys{dctr};
       auto go = [&](auto kernel, int smem) {
         launch(true, kernel, dim3(G), dim3(pgemm_threads(true)), smem, tm_wg, tm_wu, tm_wg1,
-               tm_wu1, tm_hr, tm_wd, tl, g1, g2, h_ready, dys);
+               tm_wu1, tm_xr, tm_hr, tm_wd, tl, g1, g2, h_ready, dys);
       };
       if (L.bm == PR_ROWS) {
         // CTA pairs (2-CTA clusters, an even grid): 2-slab W_down boxes, each CTA loading
         // 128 of a block's 256 columns
         CUtensorMap tm_wd2;
         if (!make_map_slabs(&tm_wd2, w_down, H, I, E, 64, 2)) return cuda_failed(-1);
-        launch(true, expert_ffn_pair_kernel, dim3(std::max(2, G & ~1)), dim3(pgemm_threads(true)), PR_SMEM,
-               tm_wg, tm_wu, tm_wg1, tm_wu1, tm_hr, tm_wd2, tl, g1, g2, h_ready, dys);
+        launch(true, expert_ffn_pair_kernel, dim3(std::max(2, G & ~1)), dim3(pgemm_threads(true)),
+               PR_SMEM, tm_wg, tm_wu, tm_wg1, tm_wu1, tm_xr, tm_hr, tm_wd2, tl, g1, g2, h_ready,
+               dys);
       } else if (R == 8) go(expert_ffn_dynamic_kernel<8>, dy_smem_bytes<8>());
       else if (R == 16) go(expert_ffn_dynamic_kernel<16>, dy_smem_bytes<16>());
       else if (R == 32) go(expert_ffn_dynamic_kernel<32>, dy_smem_bytes<32>());
@@ -779,9 +798,9 @@ moe_status_t moe_forward(const void* x, const void* w_router, const float* route
   prof.mark();
   // 5. combine: one warp per (token, 64-vector chunk), 8 warps per block
   const long long citems = (long long)T * ((H / 8 + kCombineChunkVec - 1) / kCombineChunkVec);
-  launch(true, combine_kernel, dim3((int)std::min<long long>((citems + 7) / 8, gsm)), dim3(256),
-         0, reinterpret_cast<const uint4*>(obuf), (const int32_t*)inv, (const float*)wts, T, k,
-         H / 8, static_cast<uint4*>(y));
+  launch(true, combine_kernel<false>, dim3((int)std::min<long long>((citems + 7) / 8, gsm)),
+         dim3(256), 0, reinterpret_cast<const uint4*>(obuf), (const int32_t*)inv,
+         (const float*)wts, T, k, H / 8, 0, P, y);
   if (const moe_status_t ls = launched(); ls != MOE_OK) return ls;
   prof.mark();
   prof.finish();
@@ -844,15 +863,18 @@ moe_status_t moe_dense_ffn(const void* x, const void* w_gate, const void* w_up,
   MOE_TRY_CUDA(cudaMemsetAsync(ctr, 0, sizeof(int32_t) * L.n_counters, st));
 
   const int R = dy_rows(T, 0);
-  CUtensorMap tm_wg, tm_wu, tm_wg1, tm_wu1, tm_wd, tm_hr;
+  CUtensorMap tm_wg, tm_wu, tm_wg1, tm_wu1, tm_wd, tm_hr, tm_xr;
   if (!make_map_slabs(&tm_wg, w_gate, I, H, 1, 64, 2) ||
       !make_map_slabs(&tm_wu, w_up, I, H, 1, 64, 2) ||
       !make_map_slabs(&tm_wg1, w_gate, I, H, 1, 64, 1) ||
       !make_map_slabs(&tm_wu1, w_up, I, H, 1, 64, 1) ||
-      !make_map_slabs(&tm_wd, w_down, H, I, 1, 64, 4) || !make_map_2d(&tm_hr, hbuf, I, T, R, 64))
+      !make_map_slabs(&tm_wd, w_down, H, I, 1, 64, 4) || !make_map_2d(&tm_hr, hbuf, I, T, R, 64) ||
+      !make_map_2d(&tm_xr, x, H, T, R, 64))
     return cuda_failed(-1);   // a tensor map could not be encoded
-  const TileList tl{nullptr, nullptr, nullptr, nullptr, T,
-                    nullptr, 1,       static_cast<const __nv_bfloat16*>(x), H, T};
+  // the rows of x are the A rows in place: TMA tiles of them
+  TileList tl{nullptr, nullptr, nullptr, nullptr, T,
+              nullptr, 1,       static_cast<const __nv_bfloat16*>(x), H, T};
+  tl.a_tma = 1;
   const PGemm g1{(I + 127) / 128, H, I, hbuf, I, nullptr, nullptr};
   const PGemm g2{(H + 255) / 256, I, H, y, H, nullptr, nullptr};
   int32_t* h_ready = ctr + 1;
@@ -861,19 +883,261 @@ moe_status_t moe_dense_ffn(const void* x, const void* w_gate, const void* w_up,
   const Launch launch{st, false};
   auto go = [&](auto kernel, int smem) {
     launch(false, kernel, dim3(G), dim3(pgemm_threads(true)), smem, tm_wg, tm_wu, tm_wg1, tm_wu1,
-           tm_hr, tm_wd, tl, g1, g2, h_ready, dys);
+           tm_xr, tm_hr, tm_wd, tl, g1, g2, h_ready, dys);
   };
-  if (use_pair_ffn(T, 0)) {
+  if (dy_rows(T, 0) == 128 && T >= kDensePairMinTokens) {
     // CTA pairs over 256-row tiles of x (the counters above cover ceil(T / 128) tiles)
     CUtensorMap tm_wd2;
     if (!make_map_slabs(&tm_wd2, w_down, H, I, 1, 64, 2)) return cuda_failed(-1);
     launch(false, expert_ffn_pair_kernel, dim3(std::max(2, G & ~1)), dim3(pgemm_threads(true)),
-           PR_SMEM, tm_wg, tm_wu, tm_wg1, tm_wu1, tm_hr, tm_wd2, tl, g1, g2, h_ready, dys);
+           PR_SMEM, tm_wg, tm_wu, tm_wg1, tm_wu1, tm_xr, tm_hr, tm_wd2, tl, g1, g2, h_ready, dys);
   } else if (R == 8) go(expert_ffn_dynamic_kernel<8>, dy_smem_bytes<8>());
   else if (R == 16) go(expert_ffn_dynamic_kernel<16>, dy_smem_bytes<16>());
   else if (R == 32) go(expert_ffn_dynamic_kernel<32>, dy_smem_bytes<32>());
   else if (R == 64) go(expert_ffn_dynamic_kernel<64>, dy_smem_bytes<64>());
   else go(expert_ffn_dynamic_kernel<128>, dy_smem_bytes<128>());
+  return launched();
+}
+
+// ----------------------------------------------------------------------------- steps alone
+// The steps of moe_forward as separate calls (dispatch, row gather, grouped expert FFN over
+// row segments, combine), which an expert-parallel layer strings together around its
+// exchanges.
+}  // extern "C"
+
+namespace moe {
+namespace {
+struct DispatchLayout {
+  size_t chunk_counts = 0, chunk_base = 0, dsync = 0, tile_num = 0, tile_expert = 0;
+  size_t tile_row0 = 0, tile_rows = 0, total = 0;
+  int nchunks = 0, max_tiles = 0;
+};
+DispatchLayout dispatch_layout(int T, int E, int k) {
+  DispatchLayout L;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off = align256(off + bytes);
+    return o;
+  };
+  const size_t P = (size_t)T * k;
+  L.nchunks = (int)((P + kDispatchChunk - 1) / kDispatchChunk);
+  L.max_tiles = (int)(P / GM_BM) + E;
+  L.chunk_counts = take(sizeof(int32_t) * (size_t)L.nchunks * E);
+  L.chunk_base = take(sizeof(int32_t) * (size_t)L.nchunks * E);
+  L.dsync = take(2 * sizeof(int32_t));
+  L.tile_num = take(sizeof(int32_t));
+  L.tile_expert = take(sizeof(int32_t) * L.max_tiles);
+  L.tile_row0 = take(sizeof(int32_t) * L.max_tiles);
+  L.tile_rows = take(sizeof(int32_t) * L.max_tiles);
+  L.total = off;
+  return L;
+}
+bool dispatch_shape_ok(int T, int E, int k) {
+  return T >= 1 && T <= 1048576 && E >= 1 && E <= 256 && k >= 1 && k <= 8 && k <= E;
+}
+
+// Rows of a grouped FFN over contiguous row segments at which CTA pairs take over (its rows
+// are loaded by TMA in place, as the dense MLP's are).
+constexpr int kPairMinRows = 8 * kDensePairMinTokens;
+
+struct FfnLayout {
+  size_t tile_num = 0, tile_expert = 0, tile_row0 = 0, tile_rows = 0, hbuf = 0, counters = 0;
+  size_t total = 0;
+  int max_tiles = 0, n_counters = 0, bm = 0;
+};
+FfnLayout ffn_layout(int N, int I, int n_seg) {
+  FfnLayout L;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off = align256(off + bytes);
+    return o;
+  };
+  L.bm = N >= kPairMinRows ? PR_ROWS : GM_BM;
+  L.max_tiles = N / L.bm + n_seg;
+  L.tile_num = take(sizeof(int32_t));
+  L.tile_expert = take(sizeof(int32_t) * L.max_tiles);
+  L.tile_row0 = take(sizeof(int32_t) * L.max_tiles);
+  L.tile_rows = take(sizeof(int32_t) * L.max_tiles);
+  L.hbuf = take(2 * (size_t)N * I);
+  L.n_counters = 1 + L.max_tiles + 1;   // unit counter, h-ready per tile, their total
+  L.counters = take(sizeof(int32_t) * L.n_counters);
+  L.total = off;
+  return L;
+}
+bool ffn_shape_ok(int N, int H, int E, int I, int n_seg) {
+  return N >= 1 && N <= 8 * 1048576 && H >= 64 && H <= 16384 && H % 64 == 0 && I >= 64 &&
+         I <= 8192 && I % 64 == 0 && E >= 1 && E <= 256 && n_seg >= 1 && n_seg <= kMaxSegments;
+}
+}  // namespace
+}  // namespace moe
+
+extern "C" {
+
+size_t moe_dispatch_workspace_size(int T, int E, int k) {
+  if (!dispatch_shape_ok(T, E, k)) return 0;
+  return dispatch_layout(T, E, k).total;
+}
+
+moe_status_t moe_dispatch(const int32_t* topk_ids, int T, int E, int k, int32_t* counts,
+                          int32_t* offsets, int32_t* perm, int32_t* inv, void* workspace,
+                          size_t workspace_bytes, void* stream) {
+  if (T < 0 || E <= 0 || k < 1 || k > E) return MOE_ERR_INVALID_ARG;
+  if (T == 0) return MOE_OK;
+  if (!topk_ids || !counts || !offsets || !perm || !inv || !workspace) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(workspace)) return MOE_ERR_INVALID_ARG;
+  if (!dispatch_shape_ok(T, E, k)) return MOE_ERR_UNSUPPORTED;
+  const DispatchLayout L = dispatch_layout(T, E, k);
+  if (workspace_bytes < L.total) return MOE_ERR_NO_WORKSPACE;
+  int dev = 0;
+  DeviceState* d = device_state(&dev);
+  if (!d) return MOE_ERR_CUDA;
+  t_kernels = 0;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  const int P = T * k;
+  int32_t* chunk_counts = reinterpret_cast<int32_t*>(ws + L.chunk_counts);
+  int32_t* chunk_base = reinterpret_cast<int32_t*>(ws + L.chunk_base);
+  int32_t* dsync = reinterpret_cast<int32_t*>(ws + L.dsync);
+  int32_t* tile_num = reinterpret_cast<int32_t*>(ws + L.tile_num);
+  int32_t* tile_expert = reinterpret_cast<int32_t*>(ws + L.tile_expert);
+  int32_t* tile_row0 = reinterpret_cast<int32_t*>(ws + L.tile_row0);
+  int32_t* tile_rows = reinterpret_cast<int32_t*>(ws + L.tile_rows);
+  const Launch launch{st, true};
+  const bool fused = L.nchunks > 1 && L.nchunks <= std::min(kFusedDispatchMaxChunks, d->num_sms);
+  if (L.nchunks == 1) {
+    launch(false, dispatch_small_kernel, dim3(1), dim3(256), 0, topk_ids, P, E, GM_BM, counts,
+           offsets, perm, inv, tile_num, tile_expert, tile_row0, tile_rows, (int32_t*)nullptr, 0);
+  } else if (fused) {
+    MOE_TRY_CUDA(cudaMemsetAsync(dsync, 0, 2 * sizeof(int32_t), st));
+    launch(false, dispatch_fused_kernel, dim3(L.nchunks), dim3(32 * kRankWarps),
+           (kRankWarps + 1) * E * sizeof(int), topk_ids, P, E, GM_BM, L.nchunks, chunk_counts,
+           chunk_base, counts, offsets, perm, inv, tile_num, tile_expert, tile_row0, tile_rows,
+           (int32_t*)nullptr, 0, dsync);
+  } else {
+    launch(false, dispatch_count_kernel, dim3(L.nchunks), dim3(256), E * sizeof(int), topk_ids,
+           P, E, chunk_counts);
+    launch(true, dispatch_scan_kernel, dim3(1), dim3(256), 0, (const int32_t*)chunk_counts,
+           L.nchunks, E, P, GM_BM, counts, offsets, chunk_base, tile_num, tile_expert, tile_row0,
+           tile_rows, (int32_t*)nullptr, 0);
+    launch(true, dispatch_rank_kernel, dim3(L.nchunks), dim3(32 * kRankWarps),
+           (kRankWarps + 1) * E * sizeof(int), topk_ids, P, E, (const int32_t*)chunk_base, perm,
+           inv);
+  }
+  return launched();
+}
+
+moe_status_t moe_gather_rows(const void* x, const int32_t* perm, int n_rows, int T, int H,
+                             int k, void* xp, void* stream) {
+  if (n_rows < 0 || T < 0 || H <= 0 || k < 1) return MOE_ERR_INVALID_ARG;
+  if (n_rows == 0) return MOE_OK;
+  if (!x || !perm || !xp || !aligned16(x) || !aligned16(xp)) return MOE_ERR_INVALID_ARG;
+  if (H % 8 || (long long)T * k > 8ll * 1048576) return MOE_ERR_UNSUPPORTED;
+  int dev = 0;
+  DeviceState* d = device_state(&dev);
+  if (!d) return MOE_ERR_CUDA;
+  t_kernels = 0;
+  const Launch launch{static_cast<cudaStream_t>(stream), true};
+  const int gsm = std::max(1, d->num_sms) * 8;
+  launch(false, gather_rows_kernel, dim3(std::min((n_rows + 7) / 8, gsm)), dim3(256), 0,
+         static_cast<const uint4*>(x), perm, n_rows, k, T * k, H / 8, static_cast<uint4*>(xp));
+  return launched();
+}
+
+size_t moe_expert_ffn_workspace_size(int N, int H, int E, int I, int n_seg) {
+  if (!ffn_shape_ok(N, H, E, I, n_seg)) return 0;
+  return ffn_layout(N, I, n_seg).total;
+}
+
+moe_status_t moe_expert_ffn(const void* xs, int N, const int32_t* seg_rows,
+                            const int32_t* seg_expert, int n_seg, const void* w_gate,
+                            const void* w_up, const void* w_down, int H, int E, int I, void* out,
+                            void* workspace, size_t workspace_bytes, void* stream) {
+  if (N < 0 || n_seg < 0 || H <= 0 || E <= 0 || I <= 0) return MOE_ERR_INVALID_ARG;
+  if (N == 0 || n_seg == 0) return MOE_OK;
+  if (!xs || !seg_rows || !seg_expert || !w_gate || !w_up || !w_down || !out || !workspace)
+    return MOE_ERR_INVALID_ARG;
+  if (!aligned16(xs) || !aligned16(w_gate) || !aligned16(w_up) || !aligned16(w_down) ||
+      !aligned16(out) || !aligned16(workspace))
+    return MOE_ERR_INVALID_ARG;
+  if (xs == out) return MOE_ERR_INVALID_ARG;
+  if (!ffn_shape_ok(N, H, E, I, n_seg)) return MOE_ERR_UNSUPPORTED;
+  const FfnLayout L = ffn_layout(N, I, n_seg);
+  if (workspace_bytes < L.total) return MOE_ERR_NO_WORKSPACE;
+  int dev = 0;
+  DeviceState* d = device_state(&dev);
+  if (!d) return MOE_ERR_CUDA;
+  t_kernels = 0;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  int32_t* tile_num = reinterpret_cast<int32_t*>(ws + L.tile_num);
+  int32_t* tile_expert = reinterpret_cast<int32_t*>(ws + L.tile_expert);
+  int32_t* tile_row0 = reinterpret_cast<int32_t*>(ws + L.tile_row0);
+  int32_t* tile_rows = reinterpret_cast<int32_t*>(ws + L.tile_rows);
+  __nv_bfloat16* hbuf = reinterpret_cast<__nv_bfloat16*>(ws + L.hbuf);
+  int32_t* ctr = reinterpret_cast<int32_t*>(ws + L.counters);
+  const int R = dy_rows(N, 0);
+  CUtensorMap tm_wg, tm_wu, tm_wg1, tm_wu1, tm_wd, tm_hr, tm_xr;
+  if (!make_map_slabs(&tm_wg, w_gate, I, H, E, 64, 2) ||
+      !make_map_slabs(&tm_wu, w_up, I, H, E, 64, 2) ||
+      !make_map_slabs(&tm_wg1, w_gate, I, H, E, 64, 1) ||
+      !make_map_slabs(&tm_wu1, w_up, I, H, E, 64, 1) ||
+      !make_map_slabs(&tm_wd, w_down, H, I, E, 64, L.bm == PR_ROWS ? 2 : 4) ||
+      !make_map_2d(&tm_hr, hbuf, I, N, R, 64) || !make_map_2d(&tm_xr, xs, H, N, R, 64))
+    return cuda_failed(-1);   // a tensor map could not be encoded
+  const Launch launch{st, true};
+  launch(false, segment_tiles_kernel, dim3(1), dim3(256), 0, seg_rows, seg_expert, n_seg, N, E,
+         L.bm, L.max_tiles, tile_num, tile_expert, tile_row0, tile_rows, ctr, L.n_counters);
+  // the rows are read in place (no permutation) by TMA: sorted row r of the A operand is xs[r]
+  TileList tl{tile_num, tile_expert, tile_row0, tile_rows, 0,
+              nullptr,  1,           static_cast<const __nv_bfloat16*>(xs), H, N};
+  tl.a_tma = 1;
+  const PGemm g1{(I + 127) / 128, H, I, hbuf, I, nullptr, nullptr};
+  const PGemm g2{(H + 255) / 256, I, H, out, H, nullptr, nullptr};
+  int32_t* h_ready = ctr + 1;
+  const DyState dys{ctr};
+  const int G = std::min(std::max(1, d->num_sms), kMaxGemmCtas);
+  auto go = [&](auto kernel, int smem) {
+    launch(true, kernel, dim3(G), dim3(pgemm_threads(true)), smem, tm_wg, tm_wu, tm_wg1, tm_wu1,
+           tm_xr, tm_hr, tm_wd, tl, g1, g2, h_ready, dys);
+  };
+  if (L.bm == PR_ROWS)
+    launch(true, expert_ffn_pair_kernel, dim3(std::max(2, G & ~1)), dim3(pgemm_threads(true)),
+           PR_SMEM, tm_wg, tm_wu, tm_wg1, tm_wu1, tm_xr, tm_hr, tm_wd, tl, g1, g2, h_ready, dys);
+  else if (R == 8) go(expert_ffn_dynamic_kernel<8>, dy_smem_bytes<8>());
+  else if (R == 16) go(expert_ffn_dynamic_kernel<16>, dy_smem_bytes<16>());
+  else if (R == 32) go(expert_ffn_dynamic_kernel<32>, dy_smem_bytes<32>());
+  else if (R == 64) go(expert_ffn_dynamic_kernel<64>, dy_smem_bytes<64>());
+  else go(expert_ffn_dynamic_kernel<128>, dy_smem_bytes<128>());
+  return launched();
+}
+
+moe_status_t moe_combine(const void* o, const int32_t* inv, const float* topk_weights, int T,
+                         int k, int H, int row_lo, int row_hi, unsigned flags, void* y,
+                         void* stream) {
+  if (T < 0 || k < 1 || k > 8 || H <= 0) return MOE_ERR_INVALID_ARG;
+  if (flags & ~(unsigned)MOE_COMBINE_F32) return MOE_ERR_INVALID_ARG;
+  if (T == 0) return MOE_OK;
+  if (!o || !inv || !topk_weights || !y || !aligned16(o) || !aligned16(y))
+    return MOE_ERR_INVALID_ARG;
+  if (row_lo < 0 || row_hi < row_lo || (long long)row_hi > (long long)T * k)
+    return MOE_ERR_INVALID_ARG;
+  if (H % 8 || (long long)T * k > 8ll * 1048576) return MOE_ERR_UNSUPPORTED;
+  int dev = 0;
+  DeviceState* d = device_state(&dev);
+  if (!d) return MOE_ERR_CUDA;
+  t_kernels = 0;
+  const Launch launch{static_cast<cudaStream_t>(stream), true};
+  const int gsm = std::max(1, d->num_sms) * 8;
+  const long long citems = (long long)T * ((H / 8 + kCombineChunkVec - 1) / kCombineChunkVec);
+  const dim3 grid((int)std::min<long long>((citems + 7) / 8, gsm));
+  if (flags & MOE_COMBINE_F32)
+    launch(false, combine_kernel<true>, grid, dim3(256), 0, static_cast<const uint4*>(o), inv,
+           topk_weights, T, k, H / 8, row_lo, row_hi, y);
+  else
+    launch(false, combine_kernel<false>, grid, dim3(256), 0, static_cast<const uint4*>(o), inv,
+           topk_weights, T, k, H / 8, row_lo, row_hi, y);
   return launched();
 }
 
@@ -926,8 +1190,6 @@ moe_status_t moe_sync_status(void* stream) {
   return MOE_OK;
 }
 
-int moe_pair_min_tokens(void) { return kPairMinTokens; }
-
 const char* moe_ffn_kernel_name(int T, unsigned flags) {
   if (T < 1 || !flags_ok(flags)) return "";
   if (flags & MOE_FLAG_DECODE_TILES)
@@ -937,7 +1199,9 @@ const char* moe_ffn_kernel_name(int T, unsigned flags) {
   if (flags & MOE_FLAG_FUSED_FFN)
     return T <= PG_SMALL_ROWS ? "grouped_gemm_persistent_kernel<6,EPI_GEGLU,4,1,1,1>"
                               : "grouped_gemm_persistent_kernel<4,EPI_GEGLU,4,1,1>";
-  if (use_pair_ffn(T, flags)) return "expert_ffn_pair_kernel";
+  if (use_pair_ffn(T, flags))
+    return use_row_copy(T, flags) ? "expert_ffn_pair_kernel (rows copied)" : "expert_ffn_pair_kernel";
+  if (use_row_copy(T, flags)) return "expert_ffn_dynamic_kernel<128> (rows copied)";
   switch (dy_rows(T, flags)) {
     case 8: return "expert_ffn_dynamic_kernel<8>";
     case 16: return "expert_ffn_dynamic_kernel<16>";

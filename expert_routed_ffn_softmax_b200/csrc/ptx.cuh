@@ -147,6 +147,24 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const void* desc, uint
       : "memory");
 }
 
+// L2 prefetches: a line of global memory, or a tensor tile (no shared memory written, no
+// barrier).  Used a few stages ahead of the shared-memory pipeline so that its loads hit L2.
+__device__ __forceinline__ void prefetch_l2(const void* p) {
+  asm volatile("prefetch.global.L2 [%0];" ::"l"(reinterpret_cast<uint64_t>(p)));
+}
+__device__ __forceinline__ void tma_prefetch_2d(const void* desc, int c0, int c1) {
+  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(
+                   reinterpret_cast<uint64_t>(desc)),
+               "r"(c0), "r"(c1)
+               : "memory");
+}
+__device__ __forceinline__ void tma_prefetch_4d(const void* desc, int c0, int c1, int c2, int c3) {
+  asm volatile("cp.async.bulk.prefetch.tensor.4d.L2.global.tile [%0, {%1, %2, %3, %4}];" ::"l"(
+                   reinterpret_cast<uint64_t>(desc)),
+               "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+               : "memory");
+}
+
 // 16-byte copy global -> shared that bypasses L1 (cp.async, generic proxy).
 __device__ __forceinline__ void cp_async_16(uint32_t dst, const void* src) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
@@ -288,9 +306,18 @@ __device__ __forceinline__ void st_cluster_u32(uint32_t addr, uint32_t v) {
 // issues it; each CTA holds half of A (128 rows), half of B (N/2 columns) and, in its own
 // TMEM, its 128 rows of D.  Every tcgen05 instruction of such a kernel names cta_group::2.
 
-// Arrive (release at cluster scope) on an mbarrier of another CTA of the cluster
-// (`addr` from mapa_shared).
+// Arrive on an mbarrier of another CTA of the cluster (`addr` from mapa_shared), with the
+// default semantics (release at CTA scope): what the arrival announces is this CTA's own
+// shared memory (landed copies, a freed accumulator), which the peer reads through the
+// barrier, not through the memory hierarchy.  A cluster-scope release costs a memory fence
+// per arrival (about a microsecond, measured), so it is kept for the one place that hands
+// data to the peer: mbar_arrive_remote_publish.
 __device__ __forceinline__ void mbar_arrive_remote(uint32_t addr) {
+  asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(addr) : "memory");
+}
+// Arrive on a peer's mbarrier after storing into the peer's shared memory (st.shared::cluster):
+// release at cluster scope, so the peer, acquiring at cluster scope, sees the stores.
+__device__ __forceinline__ void mbar_arrive_remote_publish(uint32_t addr) {
   asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(addr)
                : "memory");
 }
@@ -320,12 +347,6 @@ __device__ __forceinline__ bool mbar_wait_cl(uint32_t bar, uint32_t parity) {
       return false;
     }
   }
-}
-
-// Orders the generic-proxy shared-memory writes this thread has seen (cp.async rows) with
-// later async-proxy reads of them by the pair's MMA.
-__device__ __forceinline__ void fence_proxy_async_cluster() {
-  asm volatile("fence.proxy.async.shared::cluster;" ::: "memory");
 }
 
 // TMA tile loads into this CTA's shared memory whose completion is counted on the mbarrier at

@@ -39,7 +39,7 @@
 extern "C" {
 #endif
 
-#define MOE_ABI_VERSION 3
+#define MOE_ABI_VERSION 4
 
 typedef enum {
   MOE_OK = 0,
@@ -85,13 +85,21 @@ enum {
   /* Tiles of the default (dynamically scheduled) expert FFN for batches of more than 64
    * tokens: CTA pairs -- a 2-CTA cluster computes 256 sorted rows x 256 columns with one
    * tcgen05.mma.cta_group::2, each CTA loading its own 128 rows and half of the weight
-   * columns -- or single CTAs with 128-row tiles.  By default batches of at least
-   * moe_pair_min_tokens() tokens use pairs.  Both give the same bytes (every output element
-   * is the same fp32 sum over K in the same order).  Setting both, or either with
+   * columns -- or single CTAs with 128-row tiles.  moe_ffn_kernel_name() tells which one a
+   * batch gets by default.  Both give the same bytes (every output element is the same fp32
+   * sum over K in the same order).  Setting both, or either with
    * MOE_FLAG_FUSED_FFN / MOE_FLAG_UNFUSED_FFN / MOE_FLAG_DECODE_TILES, is MOE_ERR_INVALID_ARG;
    * at 64 tokens or fewer both are ignored (the A tiles then hold at most 64 rows). */
   MOE_FLAG_FFN_PAIRS = 1u << 8,
-  MOE_FLAG_FFN_SINGLE = 1u << 9
+  MOE_FLAG_FFN_SINGLE = 1u << 9,
+  /* How the default expert FFN gets GEMM-1's A rows (the routed tokens' x rows, in expert
+   * order) for batches of more than 64 tokens: copied first into an expert-sorted buffer by
+   * one more kernel and then loaded by TMA tiles (ROWS_COPY), or gathered from x inside the
+   * FFN kernel through the permutation (ROWS_GATHER).  Both give the same bytes.  The default
+   * is moe_ffn_kernel_name()'s choice; setting both, or either with a static or decode tile
+   * family, is MOE_ERR_INVALID_ARG; at 64 tokens or fewer both are ignored. */
+  MOE_FLAG_FFN_ROWS_COPY = 1u << 10,
+  MOE_FLAG_FFN_ROWS_GATHER = 1u << 11
 };
 
 /* Optional caller-owned device outputs of moe_forward (any member may be NULL). */
@@ -195,6 +203,64 @@ moe_status_t moe_dense_ffn(const void *x, const void *w_gate, const void *w_up,
                            size_t workspace_bytes, void *stream);
 
 /*
+ * The steps of moe_forward as separate calls.  An expert-parallel layer (experts split over
+ * ranks, cann-recipes-infer "Gemma-4-26B-A4B 模型优化报告" §3 部署 EP8 with 16 experts per
+ * rank, and §6.1 方案: the double_routing AllToAll that sends each rank the rows of its
+ * experts by the per-expert "split sizes", and the local-expert AllReduce of decode) strings
+ * them together around its exchanges; moe_forward runs the same kernels in one call.
+ * Arguments are (device) caller-owned memory as above; T == 0 (or no rows) launches nothing.
+ */
+
+/* Dispatch (step a3 alone): from topk_ids [T, k] (int32, ids in [0, E)) write
+ *   counts [E]    pairs routed to each expert ("split sizes"),
+ *   offsets [E+1] their exclusive scan,
+ *   perm [T*k]    expert-sorted position -> pair index t*k + j (stable: expert by expert,
+ *                 ascending pair index within an expert),
+ *   inv [T*k]     pair index -> expert-sorted position.
+ * Limits: 1 <= E <= 256, 1 <= k <= min(8, E), T <= 1048576.  An id outside [0, E) is skipped
+ * and reported by moe_sync_status() as MOE_ERR_CUDA.  Workspace: moe_dispatch_workspace_size
+ * bytes (0 = unsupported shape). */
+size_t moe_dispatch_workspace_size(int T, int E, int k);
+moe_status_t moe_dispatch(const int32_t *topk_ids, int T, int E, int k, int32_t *counts,
+                          int32_t *offsets, int32_t *perm, int32_t *inv, void *workspace,
+                          size_t workspace_bytes, void *stream);
+
+/* Row gather: xp[r, :] = x[perm[r] / k, :] for r < n_rows.  x bf16 [T, H], xp bf16
+ * [n_rows, H], perm int32 [n_rows] of pair indices below T*k (a slice of moe_dispatch's perm
+ * selects the rows of a range of experts).  H % 8 == 0.  A pair index out of range leaves
+ * its row unwritten and is reported by moe_sync_status() as MOE_ERR_CUDA. */
+moe_status_t moe_gather_rows(const void *x, const int32_t *perm, int n_rows, int T, int H, int k,
+                             void *xp, void *stream);
+
+/* Grouped expert FFN over row segments (steps a4 + a5 alone): rows are N consecutive bf16
+ * rows xs [N, H] cut into n_seg segments, segment i holding seg_rows[i] rows of expert
+ * seg_expert[i] (both int32 [n_seg], device), back to back from row 0; for every row r of
+ * a segment of expert e
+ *     out[r, :] = (gelu_tanh(xs[r] W_gate[e]) * (xs[r] W_up[e])) W_down[e]
+ * with W_gate, W_up bf16 [E, H, I] and W_down bf16 [E, I, H] (the E experts this caller
+ * holds), out bf16 [N, H] (may not alias xs).  Precision as moe_forward.  Segments may be
+ * empty; an expert id outside [0, E), a negative count, or counts adding up to more than N
+ * are reported by moe_sync_status() as MOE_ERR_CUDA and nothing is computed.
+ * Limits: N <= 8388608, 1 <= n_seg <= 1024, shapes as moe_forward.  Workspace:
+ * moe_expert_ffn_workspace_size bytes (0 = unsupported shape). */
+size_t moe_expert_ffn_workspace_size(int N, int H, int E, int I, int n_seg);
+moe_status_t moe_expert_ffn(const void *xs, int N, const int32_t *seg_rows,
+                            const int32_t *seg_expert, int n_seg, const void *w_gate,
+                            const void *w_up, const void *w_down, int H, int E, int I, void *out,
+                            void *workspace, size_t workspace_bytes, void *stream);
+
+/* Combine (step a6 alone): y[t, :] = sum_{j ascending} topk_weights[t, j] * o[inv[t, j], :]
+ * over the slots whose expert-sorted row inv[t, j] lies in [row_lo, row_hi) (the others add
+ * nothing), summed in fp32 and rounded once to bf16 -- or, with MOE_COMBINE_F32, written as
+ * fp32 (a partial sum for a cross-rank reduction).  o bf16 [T*k, H] in expert-sorted row
+ * order (only rows in the range are read), inv int32 [T*k], topk_weights fp32 [T*k],
+ * y [T, H].  0 <= row_lo <= row_hi <= T*k; H % 8 == 0; k <= 8. */
+enum { MOE_COMBINE_F32 = 1u << 0 };
+moe_status_t moe_combine(const void *o, const int32_t *inv, const float *topk_weights, int T,
+                         int k, int H, int row_lo, int row_hi, unsigned flags, void *y,
+                         void *stream);
+
+/*
  * moe_route_static -- moe_route for callers that cannot allocate device memory.
  *
  * The pages have no counterpart of this call; it exists for the library's users.  Some
@@ -221,10 +287,6 @@ moe_status_t moe_dense_ffn(const void *x, const void *w_gate, const void *w_up,
 moe_status_t moe_route_static(const void *x, const void *w_router, const float *router_bias,
                               int T, int H, int E, int k, unsigned flags, int32_t *topk_ids,
                               float *topk_weights, void *stream);
-
-/* Smallest batch (tokens) for which moe_forward and moe_dense_ffn run the expert FFN on
- * CTA pairs by default (see MOE_FLAG_FFN_PAIRS). */
-int moe_pair_min_tokens(void);
 
 /* Name of the expert-FFN kernel moe_forward launches for a batch of T tokens with these
  * flags (static storage; "" for an invalid combination). */

@@ -6,8 +6,9 @@ path, and neither side imports the other.  The arithmetic lives in ``moe_oracle.
 (plain C, double precision, ascending-index sums); this module only builds it and
 marshals numpy arrays into it.
 
-Pinned by ``tests/test_oracle_pins.py`` against closed forms, brute force on tiny
-inputs, exact rational arithmetic and library routines.  Parity status of every
+Pinned by ``tests/test_oracle_pins.py`` and ``tests/test_nvfp4_pins.py`` against closed
+forms, brute force on tiny inputs, exact rational arithmetic, library routines and a
+hand-worked NVFP4 group (``tests/golden/nvfp4_group_example.json``).  Parity status of every
 function: pinned (see the tests), except the Gemma-faithfulness of routing details
 (no router normalisation or scaling is modelled; the pages do not describe one).
 """
@@ -21,6 +22,7 @@ import numpy as np
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "moe_oracle.c")
+_SRC_FP4 = os.path.join(_HERE, "nvfp4_oracle.c")
 _LIB = os.path.join(_HERE, "libmoe_oracle.so")
 
 # No -ffast-math: the oracle relies on IEEE double arithmetic in source order.
@@ -30,9 +32,11 @@ CFLAGS = ["-O2", "-std=gnu11", "-fopenmp", "-fPIC", "-shared", "-fno-fast-math",
 
 def build(force: bool = False) -> str:
     """Compile moe_oracle.c into libmoe_oracle.so next to it (gcc)."""
-    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+    srcs = [_SRC, _SRC_FP4]
+    if force or not os.path.exists(_LIB) or any(os.path.getmtime(_LIB) < os.path.getmtime(f)
+                                                for f in srcs):
         tmp = _LIB + f".tmp{os.getpid()}"
-        subprocess.check_call(["gcc", *CFLAGS, "-o", tmp, _SRC, "-lm"])
+        subprocess.check_call(["gcc", *CFLAGS, "-o", tmp, *srcs, "-lm"])
         os.replace(tmp, _LIB)
     return _LIB
 
@@ -59,6 +63,20 @@ def lib():
         L.oracle_expert_ffn.argtypes = [_P, _P, _P, _P, _I, _I, _I, _P]
         L.oracle_forward.argtypes = [_P, _P, _P, _P, _P, _P, _I64, _I, _I, _I, _I, _I,
                                      _P, _I64, _P, _P, _P, _P]
+        _F = ctypes.c_float
+        L.oracle_e2m1_value.restype = ctypes.c_double
+        L.oracle_e2m1_value.argtypes = [_I]
+        L.oracle_e4m3_value.restype = ctypes.c_double
+        L.oracle_e4m3_value.argtypes = [_I]
+        L.oracle_e2m1_round.argtypes = [_F]
+        L.oracle_e4m3_round.argtypes = [_F]
+        L.oracle_nvfp4_weight_scale.restype = _F
+        L.oracle_nvfp4_weight_scale.argtypes = [_P, _I64]
+        L.oracle_nvfp4_quantize.argtypes = [_P, _I64, _I, _F, _P, _P]
+        L.oracle_nvfp4_dequantize.argtypes = [_P, _P, _I64, _I, _F, _P]
+        L.oracle_expert_ffn_nvfp4.argtypes = [_P, _P, _P, _P, _I, _I, _F, _F, _P]
+        L.oracle_forward_nvfp4.argtypes = [_P, _P, _P, _P, _P, _P, _I64, _I, _I, _I, _I, _I, _F,
+                                           _F, _P, _I64, _P, _P, _P, _P]
         _lib = L
     return _lib
 
@@ -173,4 +191,104 @@ def forward(x, w_router, w_gate, w_up, w_down, k: int, bias=None, renorm: bool =
     lib().oracle_forward(_ptr(x), _ptr(wr), _ptr(b), _ptr(wg), _ptr(wu), _ptr(wd), T, H, E, I,
                          k, int(bool(renorm)), _ptr(tok), n_tok, _ptr(ids), _ptr(w), _ptr(L),
                          _ptr(y))
+    return {"ids": ids, "weights": w, "logits": L, "y": y}
+
+
+# ----------------------------------------------------------------------------- NVFP4
+# NVFP4 quantisation and the layer with NVFP4 experts (nvfp4_oracle.c; Gemma-4-26B-A4B-NVFP4
+# Ascend verification report, §2.3 量化配置 (NVFP4): weights and activations in 4-bit float,
+# group size 16).  Codes are returned one per byte (bit 3 = sign), scales as E4M3 bytes.
+
+def e2m1_value(code: int) -> float:
+    return float(lib().oracle_e2m1_value(int(code)))
+
+
+def e4m3_value(code: int) -> float:
+    return float(lib().oracle_e4m3_value(int(code)))
+
+
+def e2m1_round(v: float) -> int:
+    return int(lib().oracle_e2m1_round(float(v)))
+
+
+def e4m3_round(v: float) -> int:
+    return int(lib().oracle_e4m3_round(float(v)))
+
+
+def nvfp4_weight_scale(v) -> float:
+    """Per-tensor scale of a weight tensor: amax / (6 * 448), in fp32."""
+    a = np.ascontiguousarray(v, dtype=np.float32)
+    return float(lib().oracle_nvfp4_weight_scale(_ptr(a), a.size))
+
+
+def nvfp4_quantize(v, tensor_scale: float):
+    """v [rows, K] (fp32; K % 16 == 0) -> (codes [rows, K] uint8, scales [rows, K/16] uint8)."""
+    a = np.ascontiguousarray(v, dtype=np.float32)
+    rows, K = a.shape
+    codes = np.empty((rows, K), np.uint8)
+    scales = np.empty((rows, K // 16), np.uint8)
+    lib().oracle_nvfp4_quantize(_ptr(a), rows, K, float(tensor_scale), _ptr(codes), _ptr(scales))
+    return codes, scales
+
+
+def nvfp4_dequantize(codes, scales, tensor_scale: float) -> np.ndarray:
+    c = np.ascontiguousarray(codes, dtype=np.uint8)
+    s = np.ascontiguousarray(scales, dtype=np.uint8)
+    rows, K = c.shape
+    out = np.empty((rows, K), np.float64)
+    lib().oracle_nvfp4_dequantize(_ptr(c), _ptr(s), rows, K, float(tensor_scale), _ptr(out))
+    return out
+
+
+def quantize_expert_weights(w_gate, w_up, w_down):
+    """Quantise one layer's expert weights (bf16 [E,H,I], [E,H,I], [E,I,H]) the NVFP4 way,
+    groups of 16 along each projection's reduction axis (H for gate/up, I for down), one
+    tensor scale per expert and projection.  Returns a dict of numpy arrays:
+      {gate,up}_codes [E,I,H], {gate,up}_scales [E,I,H/16], down_codes [E,H,I],
+      down_scales [E,H,I/16] (uint8), {gate,up,down}_ts [E] (fp32)."""
+    import torch  # local: only to read the bf16 tensors
+    out = {}
+    for name, w in (("gate", w_gate), ("up", w_up), ("down", w_down)):
+        wt = w.float().transpose(1, 2).contiguous().numpy()    # [E, out, K]
+        E, N, K = wt.shape
+        codes = np.empty((E, N, K), np.uint8)
+        scales = np.empty((E, N, K // 16), np.uint8)
+        ts = np.empty(E, np.float32)
+        for e in range(E):
+            ts[e] = nvfp4_weight_scale(wt[e])
+            codes[e], scales[e] = nvfp4_quantize(wt[e], ts[e])
+        out[f"{name}_codes"], out[f"{name}_scales"], out[f"{name}_ts"] = codes, scales, ts
+    del torch
+    return out
+
+
+def dequantize_expert_weights(q: dict) -> dict:
+    """-> {gate, up}: [E, I, H], down: [E, H, I] float64 (exact dequantised values)."""
+    out = {}
+    for name in ("gate", "up", "down"):
+        c, s, ts = q[f"{name}_codes"], q[f"{name}_scales"], q[f"{name}_ts"]
+        out[name] = np.stack([nvfp4_dequantize(c[e], s[e], ts[e]) for e in range(c.shape[0])])
+    return out
+
+
+def forward_nvfp4(x, w_router, wq: dict, k: int, bias=None, renorm: bool = True,
+                  act_scale_x: float = 1.0, act_scale_h: float = 1.0, tokens=None):
+    """The layer with NVFP4 expert weights (given quantised, see quantize_expert_weights) and
+    NVFP4 activations (x before GEMM-1, h before GEMM-2, with fixed tensor scales).  Routing
+    as forward().  -> dict(ids, weights, logits, y)."""
+    xb, wr, b = _u16(x), _u16(w_router), _f32(bias)
+    T, H = xb.shape
+    E = wr.shape[1]
+    dq = dequantize_expert_weights(wq)
+    I = dq["gate"].shape[1]
+    tok = None if tokens is None else np.ascontiguousarray(tokens, dtype=np.int64)
+    n_tok = T if tok is None else len(tok)
+    ids = np.empty((T, k), np.int32)
+    w = np.empty((T, k), np.float64)
+    L = np.empty((T, E), np.float64)
+    y = np.empty((n_tok, H), np.float64)
+    g, u, d = (np.ascontiguousarray(dq[n]) for n in ("gate", "up", "down"))
+    lib().oracle_forward_nvfp4(_ptr(xb), _ptr(wr), _ptr(b), _ptr(g), _ptr(u), _ptr(d), T, H, E,
+                               I, k, int(bool(renorm)), float(act_scale_x), float(act_scale_h),
+                               _ptr(tok), n_tok, _ptr(ids), _ptr(w), _ptr(L), _ptr(y))
     return {"ids": ids, "weights": w, "logits": L, "y": y}

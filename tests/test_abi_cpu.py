@@ -39,7 +39,7 @@ def test_library_exports_every_declared_symbol(lib):
 
 
 def test_abi_version_and_status_strings(lib):
-    assert lib.moe_abi_version() == 3
+    assert lib.moe_abi_version() == 4
     assert _abi.status_string(0) == "MOE_OK"
     assert _abi.status_string(5) == "MOE_ERR_TIMEOUT"
     assert _abi.status_string(99) == "MOE_ERR_UNKNOWN"
@@ -127,20 +127,24 @@ def test_dense_ffn_host_checks(lib):
 
 def test_ffn_kernel_choice(lib):
     """Which expert-FFN kernel a batch gets: the dynamic kernel with A slots of 8..128 rows,
-    CTA pairs from moe_pair_min_tokens() tokens (or when forced above 64 tokens)."""
-    pmin = lib.moe_pair_min_tokens()
-    assert 64 < pmin <= 1 << 20
+    single CTAs gathering their rows by default; CTA pairs and copied rows when forced above
+    64 tokens."""
     assert _abi.ffn_kernel_name(1) == "expert_ffn_dynamic_kernel<8>"
     assert _abi.ffn_kernel_name(8) == "expert_ffn_dynamic_kernel<8>"
     assert _abi.ffn_kernel_name(64) == "expert_ffn_dynamic_kernel<64>"
-    assert _abi.ffn_kernel_name(pmin - 1) == "expert_ffn_dynamic_kernel<128>"
-    assert _abi.ffn_kernel_name(pmin) == "expert_ffn_pair_kernel"
-    assert _abi.ffn_kernel_name(pmin, "single") == "expert_ffn_dynamic_kernel<128>"
+    assert _abi.ffn_kernel_name(32768) == "expert_ffn_dynamic_kernel<128>"
+    assert _abi.ffn_kernel_name(32768, "pairs") == "expert_ffn_pair_kernel"
+    assert _abi.ffn_kernel_name(32768, "pairs", "copy") == "expert_ffn_pair_kernel (rows copied)"
+    assert _abi.ffn_kernel_name(4096, "single", "copy") == "expert_ffn_dynamic_kernel<128> (rows copied)"
     assert _abi.ffn_kernel_name(65, "pairs") == "expert_ffn_pair_kernel"
     assert _abi.ffn_kernel_name(64, "pairs") == "expert_ffn_dynamic_kernel<64>"
     assert _abi.ffn_kernel_name(8, "decode").startswith("grouped_gemm_decode_kernel")
     assert lib.moe_ffn_kernel_name(8, _abi.MOE_FLAG_FFN_PAIRS | _abi.MOE_FLAG_FFN_SINGLE) == b""
-    # pair tiles of 256 rows need fewer tile-list entries, not more workspace
+    both_rows = _abi.MOE_FLAG_FFN_ROWS_COPY | _abi.MOE_FLAG_FFN_ROWS_GATHER
+    assert lib.moe_workspace_size(4096, 2816, 128, 704, 8, both_rows) == 0
+    # pair tiles of 256 rows need fewer tile-list entries; copied rows need the Xp buffer
     single = lib.moe_workspace_size(4096, 2816, 128, 704, 8, _abi.MOE_FLAG_FFN_SINGLE)
     pairs = lib.moe_workspace_size(4096, 2816, 128, 704, 8, _abi.MOE_FLAG_FFN_PAIRS)
+    copy = lib.moe_workspace_size(4096, 2816, 128, 704, 8, _abi.MOE_FLAG_FFN_ROWS_COPY)
     assert 0 < pairs <= single
+    assert copy >= single + 2 * 4096 * 8 * 2816

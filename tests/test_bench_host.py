@@ -74,8 +74,8 @@ def test_ffn_kernel_name_follows_the_library_rule():
     assert bench.ffn_kernel_name(9, "auto") == "expert_ffn_dynamic_kernel<16>"
     assert bench.ffn_kernel_name(64, "prefill") == "expert_ffn_dynamic_kernel<64>"
     assert bench.ffn_kernel_name(65, "auto") == "expert_ffn_dynamic_kernel<128>"
-    assert bench.ffn_kernel_name(32768, "auto") == "expert_ffn_pair_kernel"      # CTA pairs
-    assert bench.ffn_kernel_name(32768, "single") == "expert_ffn_dynamic_kernel<128>"
+    assert bench.ffn_kernel_name(32768, "auto") == "expert_ffn_dynamic_kernel<128>"
+    assert bench.ffn_kernel_name(32768, "pairs") == "expert_ffn_pair_kernel"      # CTA pairs
     assert "+" in bench.ffn_kernel_name(4096, "unfused")          # two launches
     assert bench.ffn_kernel_name(8, "fused").endswith(",1>")       # 8-row A slots
     assert bench.ffn_kernel_name(8, "decode").startswith("grouped_gemm_decode_kernel")

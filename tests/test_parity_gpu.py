@@ -45,9 +45,10 @@ def layer_inputs(cfg, gemma_w, seed=0, T=None):
 SCREEN_C = 2.0 ** -10     # the kernel's screen error bound, in units of |x_t| |w_e|
 
 
-def gpu_forward(x, g, k, renorm=True, router="auto", tiles="auto"):
+def gpu_forward(x, g, k, renorm=True, router="auto", tiles="auto", rows="auto"):
     y, aux = moe.forward(x.cuda(), g["w_router"], g["w_gate"], g["w_up"], g["w_down"], k,
-                         bias=g["bias"], renorm=renorm, aux=True, router=router, tiles=tiles)
+                         bias=g["bias"], renorm=renorm, aux=True, router=router, tiles=tiles,
+                         rows=rows)
     assert moe.sync_status() == 0
     st = moe.router_stats(aux)
     if st["path"] == "screen":
@@ -85,10 +86,11 @@ def sample_tokens(T, n, seed=0):
     return np.unique(np.concatenate([[0, T - 1], s]))
 
 
-def run_case(cfg, gemma_w, n_sample, T=None, renorm=True, router="auto", tiles="auto"):
+def run_case(cfg, gemma_w, n_sample, T=None, renorm=True, router="auto", tiles="auto",
+             rows="auto"):
     x, c, g = layer_inputs(cfg, gemma_w, T=T)
     T = x.shape[0]
-    y, aux = gpu_forward(x, g, cfg.k, renorm, router, tiles)
+    y, aux = gpu_forward(x, g, cfg.k, renorm, router, tiles, rows)
     rows = sample_tokens(T, n_sample)
     ref = oracle.forward(x, c["w_router"], c["w_gate"], c["w_up"], c["w_down"], cfg.k,
                          bias=c["bias"], renorm=renorm, tokens=rows)
@@ -139,29 +141,35 @@ PAIR_CASES = [("tiny", 1000), ("decode", 65), ("decode", 300), ("prefill", 2048)
               ("sweep_T4096", 4096)]
 
 
+@pytest.mark.parametrize("rows", ["gather", "copy"])
 @pytest.mark.parametrize("tiles", ["pairs", "single"])
 @pytest.mark.parametrize("name,T", PAIR_CASES, ids=[f"{n}_T{t}" for n, t in PAIR_CASES])
-def test_forward_pair_and_single_cta_tiles(name, T, tiles, gemma_w):
-    run_case(wl.CONFIGS[name], gemma_w, 256, T=T, tiles=tiles)
+def test_forward_pair_and_single_cta_tiles(name, T, tiles, rows, gemma_w):
+    """Each tile form with GEMM-1's A rows gathered inside the kernel or copied to an
+    expert-sorted buffer first and loaded by TMA."""
+    run_case(wl.CONFIGS[name], gemma_w, 256, T=T, tiles=tiles, rows=rows)
 
 
-def test_skewed_on_single_cta_tiles(gemma_w):
-    """The skewed batch (experts from empty to 16k rows) on 128-row single-CTA tiles (its
-    default is CTA pairs, covered by test_forward_parity)."""
-    assert moe.ffn_kernel_name(16384) == "expert_ffn_pair_kernel"
-    run_case(wl.CONFIGS["skewed"], gemma_w, 128, tiles="single")
+def test_skewed_on_cta_pairs(gemma_w):
+    """The skewed batch (experts from empty to 16k rows) on 256-row CTA pairs, with rows
+    gathered and with rows copied (its default, single CTAs, is in test_forward_parity)."""
+    assert moe.ffn_kernel_name(16384) == "expert_ffn_dynamic_kernel<128>"
+    run_case(wl.CONFIGS["skewed"], gemma_w, 128, tiles="pairs", rows="gather")
+    run_case(wl.CONFIGS["skewed"], gemma_w, 128, tiles="pairs", rows="copy")
 
 
 @pytest.mark.parametrize("T", [65, 300, 2048, 4096])
 def test_pair_tiles_match_single_cta_tiles_bitwise(T, gemma_w):
     """Every output element is the same fp32 sum over K in the same k-step order whether its
-    row sits in a 128-row single-CTA tile or in a 256-row CTA pair, so the bytes agree."""
+    row sits in a 128-row single-CTA tile or in a 256-row CTA pair, and whether its A row was
+    gathered in the kernel or copied first, so the bytes agree."""
     x, c, g = layer_inputs(wl.CONFIGS["decode"], gemma_w, T=T)
     x = x.cuda()
-    y1 = moe.forward(x, g["w_router"], g["w_gate"], g["w_up"], g["w_down"], 8, tiles="pairs")
-    y2 = moe.forward(x, g["w_router"], g["w_gate"], g["w_up"], g["w_down"], 8, tiles="single")
+    ys = [moe.forward(x, g["w_router"], g["w_gate"], g["w_up"], g["w_down"], 8, tiles=t, rows=r)
+          for t in ("pairs", "single") for r in ("gather", "copy")]
     assert moe.sync_status() == 0
-    assert torch.equal(y1, y2)
+    for y in ys[1:]:
+        assert torch.equal(ys[0], y)
 
 
 def test_forward_no_renorm(gemma_w):
