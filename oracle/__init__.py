@@ -292,3 +292,18 @@ def forward_nvfp4(x, w_router, wq: dict, k: int, bias=None, renorm: bool = True,
                                I, k, int(bool(renorm)), float(act_scale_x), float(act_scale_h),
                                _ptr(tok), n_tok, _ptr(ids), _ptr(w), _ptr(L), _ptr(y))
     return {"ids": ids, "weights": w, "logits": L, "y": y}
+
+
+def expert_ffn_nvfp4(x_row, wg_dq, wu_dq, wd_dq, act_scale_x: float = 1.0,
+                     act_scale_h: float = 1.0) -> np.ndarray:
+    """One expert on one token row with NVFP4 activations: weights given dequantised,
+    wg_dq / wu_dq [I, H] and wd_dq [H, I] (float64).  -> o [H] float64."""
+    xr = _u16(x_row)
+    g = np.ascontiguousarray(wg_dq, dtype=np.float64)
+    u = np.ascontiguousarray(wu_dq, dtype=np.float64)
+    d = np.ascontiguousarray(wd_dq, dtype=np.float64)
+    I, H = g.shape
+    out = np.empty(H, np.float64)
+    lib().oracle_expert_ffn_nvfp4(_ptr(xr), _ptr(g), _ptr(u), _ptr(d), H, I, float(act_scale_x),
+                                  float(act_scale_h), _ptr(out))
+    return out
