@@ -80,19 +80,23 @@ class ClockSampler:
         return int(fn(self.h))
 
     def _run(self):
-        nv = self.nv
         while not self._stop.is_set():
-            try:
-                self.samples.append((time.perf_counter(),
-                                     nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM),
-                                     self._reasons()))
-            except Exception:
-                pass
+            self._sample()
             time.sleep(self.period)
+
+    def _sample(self):
+        nv = self.nv
+        try:
+            self.samples.append((time.perf_counter(),
+                                 nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM),
+                                 self._reasons()))
+        except Exception:
+            pass
 
     def start(self):
         if self.h is None:
             return
+        self._sample()          # one sample as the timed region starts, whatever its length
         self._stop = threading.Event()
         self.t = threading.Thread(target=self._run, daemon=True)
         self.t.start()
@@ -102,6 +106,7 @@ class ClockSampler:
             return None
         self._stop.set()
         self.t.join()
+        self._sample()          # and one as it ends (the GPU has just finished its last step)
         if not self.samples:
             return None
         sm = [s[1] for s in self.samples]
@@ -277,6 +282,94 @@ def time_layer(moe, cfg, args, g, x_cpu, dev, stream, flush_l2, dist, e2e: bool)
             "clocks": clk, "kernels": kernels, "step_ms": step_ms}
 
 
+FP4_EXPERT_BYTES = 3 * 2816 * 704 // 2 + 3 * 2816 * 704 // 16 + 3 * 4   # codes, scales, ts
+
+
+def time_nvfp4(moe, cfg, args, g, x_cpu, dev, stream, flush_l2, dist) -> dict:
+    """The layer with NVFP4 experts (weights quantised by the library from the bf16 set) on
+    cfg's batch: graph replays of moe_forward_nvfp4, L2 flushed before every step, stage
+    events from a second graph; device times are the max over ranks."""
+    from expert_routed_ffn_softmax_b200 import _abi
+    wq = _abi.nvfp4_quantize_layer(g["w_gate"], g["w_up"], g["w_down"])
+    x = x_cpu.to(dev)
+    y0, aux = _abi.forward_nvfp4(x, g["w_router"], wq, cfg.k, bias=g["bias"], aux=True)
+    if moe.sync_status() != 0:
+        raise SystemExit("device status not OK after the first NVFP4 forward")
+    counts = aux["expert_counts"].cpu().numpy()
+    active = int((counts > 0).sum())
+    E, I, H = cfg.E, cfg.I, cfg.H
+    flags = 0
+    nbytes = _abi.load().moe_nvfp4_workspace_size(cfg.T, H, E, I, cfg.k, flags)
+    ws = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+    ws_p = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+    y = torch.empty_like(y0)
+
+    def capture(profile, buf):
+        _abi.forward_nvfp4(x, g["w_router"], wq, cfg.k, bias=g["bias"], out=y, profile=profile,
+                           workspace_buf=buf)
+        torch.cuda.synchronize()
+        gr = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gr):
+            _abi.forward_nvfp4(x, g["w_router"], wq, cfg.k, bias=g["bias"], out=y,
+                               profile=profile, workspace_buf=buf)
+        return gr, _abi.last_kernel_count()
+
+    graph, kernels = capture(False, ws)
+    for _ in range(args.warmup):
+        flush_l2()
+        graph.replay()
+    torch.cuda.synchronize()
+    if not torch.equal(y, y0):
+        raise SystemExit("NVFP4 graph replay differs from the direct call")
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    clocks = ClockSampler(dev)
+    clocks.start()
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    for i in range(args.steps):
+        flush_l2()
+        ev[i][0].record(stream)
+        graph.replay()
+        ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    ms = sum(a.elapsed_time(b) for a, b in ev) / args.steps
+    pgraph, _ = capture(True, ws_p)
+    acc: dict[str, list[float]] = {}
+    for _ in range(max(3, min(args.steps, 20))):
+        flush_l2()
+        pgraph.replay()
+        for k2, v in _abi.last_stage_times().items():
+            acc.setdefault(k2, []).append(v)
+    stages = {k2: sum(v) / len(v) for k2, v in acc.items()}
+    del pgraph, graph
+    ms, ffn_ms = max_over_ranks([ms, stages.get("expert_ffn", 0.0)], dist, dev)
+    return {"ms": ms, "ffn_ms": ffn_ms, "stages": stages, "active": active, "clocks": clk,
+            "kernels": kernels}
+
+
+def nvfp4_entry(cfg, m: dict, world: int, pk: dict) -> dict:
+    ffn_bytes = m["active"] * FP4_EXPERT_BYTES
+    step_bytes = ffn_bytes + cfg.H * cfg.E * 2 + 2 * cfg.T * cfg.H * 2
+    ach = ffn_bytes / (m["ffn_ms"] * 1e-3) / 1e9 if m["ffn_ms"] > 0 else None
+    return {
+        "workload": f"{cfg.name}: T={cfg.T} H={cfg.H} E={cfg.E} k={cfg.k} I={cfg.I}, expert "
+                    "weights and activations NVFP4 (E2M1, E4M3 scale per 16, fp32 per tensor), "
+                    "weights quantised from the bf16 set",
+        "value": job_throughput(world, cfg.T, m["ms"]), "unit": UNIT, "ms_per_step": m["ms"],
+        "expert_ffn": {"kernels": "nvfp4_gemm1_kernel + nvfp4_gemm2_kernel", "ms": m["ffn_ms"],
+                       "algorithmic_bytes": ffn_bytes, "achieved_gbs": ach,
+                       "frac_of_hbm": None if ach is None else ach / pk["hbm_gbs"]},
+        "step_hbm_frac": step_bytes / (m["ms"] * 1e-3) / (pk["hbm_gbs"] * 1e9),
+        "active_experts": m["active"], "stages_ms": m["stages"], "clocks": m["clocks"],
+        "gpu_launches": m["kernels"] * m["_steps"],
+        "note": "reduced-precision variant of the layer (the checkpoint's format), reported "
+                "beside the bf16 line, not in place of it",
+    }
+
+
 def tensor_bound_entry(cfg, m: dict, world: int, pk: dict) -> dict:
     """Summary of one large-batch config: tokens/s, the expert FFN's tensor throughput
     against the measured burst and sustained bf16 peaks, and the whole step's."""
@@ -396,6 +489,10 @@ def run_native(args, cfg) -> None:
     ms, e2e_ms = m["ms"], m["e2e_ms"]
     acc, rstats, stages, clk, graph_kernels, step_ms = (m["acc"], m["rstats"], m["stages"],
                                                        m["clocks"], m["kernels"], m["step_ms"])
+    # the layer with NVFP4 experts at decode, same timing rules, reported beside the line
+    fp4 = None
+    if not args.no_nvfp4 and cfg.T <= 16 and (cfg.H, cfg.E, cfg.I) == (2816, 128, 704):
+        fp4 = time_nvfp4(moe, cfg, args, g, x_cpu, dev, stream, flush_l2, dist)
     # the tensor-bound configs (large batches), same timing rules, reported beside the line
     tensor_bound = []
     if not args.no_tensor_bound:
@@ -460,6 +557,9 @@ def run_native(args, cfg) -> None:
             "clocks": clk,
             "step_ms_p10_p50_p90": [float(np.percentile(step_ms, q)) for q in (10, 50, 90)],
         }
+        if fp4 is not None:
+            fp4["_steps"] = args.steps
+            line["nvfp4_decode"] = nvfp4_entry(cfg, fp4, world, pk)
         if tensor_bound:
             line["tensor_bound"] = []
             for c2, m2 in tensor_bound:
@@ -677,6 +777,8 @@ def main():
     ap.add_argument("--tiles", default="auto",
                     choices=["auto", "decode", "prefill", "pairs", "single", "fused", "unfused"],
                     help="expert-GEMM tile family (default: the library's choice)")
+    ap.add_argument("--no-nvfp4", action="store_true",
+                    help="skip the NVFP4-expert variant reported beside the decode line")
     ap.add_argument("--no-tensor-bound", action="store_true",
                     help="skip the large-batch (tensor-bound) configs reported beside the line")
     ap.add_argument("--ep", action="store_true",

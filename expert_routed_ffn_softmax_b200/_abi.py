@@ -68,6 +68,12 @@ SIGNATURES = {
     "moe_expert_ffn_workspace_size": (_SZ, [_I, _I, _I, _I, _I]),
     "moe_expert_ffn": (_I, [_P, _I, _P, _P, _I, _P, _P, _P, _I, _I, _I, _P, _P, _SZ, _P]),
     "moe_combine": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _U, _P, _P]),
+    "moe_nvfp4_quantize_workspace_size": (_SZ, [_I]),
+    "moe_nvfp4_quantize_weights": (_I, [_P, _I, _I, _I, _P, _P, _P, _P, _SZ, _P]),
+    "moe_nvfp4_quantize_rows": (_I, [_P, _I, _I, ctypes.c_float, _P, _P, _P]),
+    "moe_nvfp4_workspace_size": (_SZ, [_I, _I, _I, _I, _I, _U]),
+    "moe_forward_nvfp4": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _U, ctypes.c_float,
+                               ctypes.c_float, _P, _P, _P, _SZ, _P]),
     "moe_sync_status": (_I, [_P]),
     "moe_ffn_kernel_name": (ctypes.c_char_p, [_I, _U]),
     "moe_last_stage_times": (_I, [ctypes.POINTER(ctypes.c_float), _I]),
@@ -88,6 +94,12 @@ class MoEError(RuntimeError):
         if cuda_error:
             msg += f" [{load().moe_cuda_error_name(cuda_error).decode()}]"
         super().__init__(msg)
+
+
+class NVFP4Weights(ctypes.Structure):
+    _fields_ = [("gate_codes", _P), ("gate_scales", _P), ("gate_ts", _P),
+                ("up_codes", _P), ("up_scales", _P), ("up_ts", _P),
+                ("down_codes", _P), ("down_scales", _P), ("down_ts", _P)]
 
 
 class AuxOut(ctypes.Structure):
@@ -348,6 +360,98 @@ def combine(o: torch.Tensor, inv: torch.Tensor, topk_weights: torch.Tensor, row_
                              MOE_COMBINE_F32 if fp32 else 0, py, _stream_ptr(stream)),
                "moe_combine")
     return y
+
+
+# ----------------------------------------------------------------------------- NVFP4
+def nvfp4_quantize_weights(w: torch.Tensor, stream=None) -> dict:
+    """moe_nvfp4_quantize_weights: bf16 w [E, K, N] (N contiguous) -> {codes uint8 [E, N, K/2],
+    scales uint8 [E, N, K/16], ts float32 [E]} on w's device."""
+    L = load()
+    E, K, N = w.shape
+    dev = w.device
+    pw = _dev(w, "w", torch.bfloat16, (E, K, N))
+    codes = torch.empty((E, N, K // 2), dtype=torch.uint8, device=dev)
+    scales = torch.empty((E, N, K // 16), dtype=torch.uint8, device=dev)
+    ts = torch.empty(E, dtype=torch.float32, device=dev)
+    ws = torch.empty(max(256, L.moe_nvfp4_quantize_workspace_size(E)), dtype=torch.uint8, device=dev)
+    _check(L.moe_nvfp4_quantize_weights(pw, E, K, N, codes.data_ptr(), scales.data_ptr(),
+                                        ts.data_ptr(), ws.data_ptr(), ws.numel(),
+                                        _stream_ptr(stream)), "moe_nvfp4_quantize_weights")
+    return {"codes": codes, "scales": scales, "ts": ts}
+
+
+def nvfp4_quantize_layer(w_gate: torch.Tensor, w_up: torch.Tensor, w_down: torch.Tensor,
+                         stream=None) -> dict:
+    """The layer's expert weights (bf16, moe_forward's layout) as NVFP4: a dict of the nine
+    tensors of moe_nvfp4_weights_t (gate_codes, gate_scales, gate_ts, up_..., down_...)."""
+    out = {}
+    for name, w in (("gate", w_gate), ("up", w_up), ("down", w_down)):
+        q = nvfp4_quantize_weights(w, stream)
+        out.update({f"{name}_{k}": v for k, v in q.items()})
+    return out
+
+
+def nvfp4_quantize_rows(x: torch.Tensor, ts: float, stream=None):
+    """moe_nvfp4_quantize_rows: bf16 x [rows, K] -> (codes uint8 [rows, K/2], scales uint8
+    [rows, K/16]) with tensor scale ts."""
+    L = load()
+    rows, K = x.shape
+    px = _dev(x, "x", torch.bfloat16, (rows, K))
+    codes = torch.empty((rows, K // 2), dtype=torch.uint8, device=x.device)
+    scales = torch.empty((rows, K // 16), dtype=torch.uint8, device=x.device)
+    _check(L.moe_nvfp4_quantize_rows(px, rows, K, float(ts), codes.data_ptr(), scales.data_ptr(),
+                                     _stream_ptr(stream)), "moe_nvfp4_quantize_rows")
+    return codes, scales
+
+
+def forward_nvfp4(x: torch.Tensor, w_router: torch.Tensor, wq: dict, k: int,
+                  bias: torch.Tensor | None = None, renorm: bool = True,
+                  act_scale_x: float = 1.0, act_scale_h: float = 1.0, aux: bool = False,
+                  out: torch.Tensor | None = None, profile: bool = False, stream=None,
+                  workspace_buf: torch.Tensor | None = None, router: str = "auto"):
+    """The routed layer with NVFP4 expert weights (wq from nvfp4_quantize_layer) and NVFP4
+    activations, for T <= 16 tokens -> y bf16 [T, H] (and the routing dict if aux)."""
+    L = load()
+    T, H = x.shape
+    E = w_router.shape[1]
+    I = wq["gate_codes"].shape[1]
+    dev = x.device
+    px = _dev(x, "x", torch.bfloat16, (T, H))
+    pr = _dev(w_router, "w_router", torch.bfloat16, (H, E))
+    pb = None if bias is None else _dev(bias, "bias", torch.float32, (E,))
+    shapes = {"gate_codes": ((E, I, H // 2), torch.uint8), "gate_scales": ((E, I, H // 16), torch.uint8),
+              "up_codes": ((E, I, H // 2), torch.uint8), "up_scales": ((E, I, H // 16), torch.uint8),
+              "down_codes": ((E, H, I // 2), torch.uint8), "down_scales": ((E, H, I // 16), torch.uint8),
+              "gate_ts": ((E,), torch.float32), "up_ts": ((E,), torch.float32),
+              "down_ts": ((E,), torch.float32)}
+    wstruct = NVFP4Weights(*(_dev(wq[n], n, shapes[n][1], shapes[n][0])
+                             for n, _ in NVFP4Weights._fields_))
+    y = torch.empty((T, H), dtype=torch.bfloat16, device=dev) if out is None else out
+    py = _dev(y, "out", torch.bfloat16, (T, H))
+    flags = _flags(renorm, router, profile)
+    a = None
+    aux_d = None
+    if aux:
+        aux_d = {
+            "expert_counts": torch.empty(E, dtype=torch.int32, device=dev),
+            "expert_offsets": torch.empty(E + 1, dtype=torch.int32, device=dev),
+            "perm": torch.empty(T * k, dtype=torch.int32, device=dev),
+            "topk_ids": torch.empty((T, k), dtype=torch.int32, device=dev),
+            "topk_weights": torch.empty((T, k), dtype=torch.float32, device=dev),
+            "router_stats": torch.zeros(5, dtype=torch.int32, device=dev),
+        }
+        a = AuxOut(*(aux_d[n].data_ptr() for n, _ in AuxOut._fields_))
+    if T == 0:
+        return (y, aux_d) if aux else y
+    nbytes = L.moe_nvfp4_workspace_size(T, H, E, I, k, flags)
+    if nbytes == 0:
+        raise MoEError(MOE_ERR_UNSUPPORTED, "moe_nvfp4_workspace_size")
+    ws = workspace(nbytes, dev) if workspace_buf is None else workspace_buf
+    _check(L.moe_forward_nvfp4(px, pr, pb, ctypes.byref(wstruct), T, H, E, I, k, flags,
+                               float(act_scale_x), float(act_scale_h), py,
+                               None if a is None else ctypes.byref(a), ws.data_ptr(), ws.numel(),
+                               _stream_ptr(stream)), "moe_forward_nvfp4")
+    return (y, aux_d) if aux else y
 
 
 def router_stats(aux: dict) -> dict:

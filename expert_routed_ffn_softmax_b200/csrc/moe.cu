@@ -21,6 +21,7 @@
 #include "ffn_pair.cuh"
 #include "decode_front.cuh"
 #include "gemm_decode.cuh"
+#include "nvfp4.cuh"
 
 namespace moe {
 namespace {
@@ -31,6 +32,7 @@ constexpr int kScreenMinTokens = 256;            // default router path switch
 constexpr int kMaxGemmCtas = 256;                // >= SMs per GPU (148 on B200)
 constexpr int kStreamKCounters = 4 * 2 * kMaxGemmCtas;   // per GEMM: 4 per split unit
 constexpr int kFrontSmemMax = 200 * 1024;        // decode front kernel's dynamic smem cap
+constexpr int kFp4SmemMax = 227 * 1024;          // NVFP4 FFN kernels' dynamic smem cap
 
 constexpr double kScreenC = 1.0 / 1024.0;        // screen error bound / (|x| |w|)
 constexpr int kRouterStats = 5;                  // words of moe_aux_t::router_stats
@@ -367,6 +369,14 @@ DeviceState* device_state(int* dev_out) {
             cudaSuccess ||
         cudaFuncSetAttribute(expert_ffn_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              PR_SMEM) != cudaSuccess ||
+        cudaFuncSetAttribute(nvfp4_gemm1_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             kFp4SmemMax) != cudaSuccess ||
+        cudaFuncSetAttribute(nvfp4_gemm1_kernel<FP4_MAX_ROWS>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, kFp4SmemMax) != cudaSuccess ||
+        cudaFuncSetAttribute(nvfp4_gemm2_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             kFp4SmemMax) != cudaSuccess ||
+        cudaFuncSetAttribute(nvfp4_gemm2_kernel<FP4_MAX_ROWS>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, kFp4SmemMax) != cudaSuccess ||
         cudaFuncSetAttribute(GEMM_FFN_SMALL, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              pgemm_smem_bytes<kSmallStages, 4, true>()) != cudaSuccess ||
         cudaFuncSetAttribute(GEMM_STORE, cudaFuncAttributeMaxDynamicSharedMemorySize, gs) !=
@@ -516,6 +526,103 @@ moe_status_t launch_router(const __nv_bfloat16* x, const __nv_bfloat16* wr, cons
   return launched();
 }
 
+// Steps 1 and 2 of the layer (router, dispatch) into the buffers of `b` and the workspace's
+// tile list; with copy_rows also the copy of the routed rows into Xp in expert order.
+struct RouteBufs {
+  int32_t* ids;
+  float* wts;
+  unsigned* stats;
+  int32_t *counts, *offsets, *perm, *inv;
+};
+moe_status_t route_and_dispatch(const void* x, const void* w_router, const float* router_bias,
+                                int T, int H, int E, int k, unsigned flags, const RouteBufs& b,
+                                uint8_t* ws, const Layout& L, const DeviceState& dv,
+                                cudaStream_t st, Profiler& prof, bool copy_rows) {
+  const DeviceState* d = &dv;
+  int32_t *ids = b.ids, *counts = b.counts, *offsets = b.offsets, *perm = b.perm, *inv = b.inv;
+  float* wts = b.wts;
+  unsigned* stats = b.stats;
+  const int P = T * k;
+  int32_t* chunk_counts = reinterpret_cast<int32_t*>(ws + L.chunk_counts);
+  int32_t* chunk_base = reinterpret_cast<int32_t*>(ws + L.chunk_base);
+  int32_t* tile_num = reinterpret_cast<int32_t*>(ws + L.tile_num);
+  int32_t* tile_expert = reinterpret_cast<int32_t*>(ws + L.tile_expert);
+  int32_t* tile_row0 = reinterpret_cast<int32_t*>(ws + L.tile_row0);
+  int32_t* tile_rows = reinterpret_cast<int32_t*>(ws + L.tile_rows);
+  __nv_bfloat16* xp = reinterpret_cast<__nv_bfloat16*>(ws + L.xp);
+  int32_t* gemm_counters = reinterpret_cast<int32_t*>(ws + L.counters);
+  const int gsm = std::max(1, d->num_sms) * 8;
+  // Dependent launches, except while stage events sit between the kernels.
+  const Launch launch{st, !prof.on};
+  if (use_decode_front(T, H, E, flags)) {
+    // 1+2. router and dispatch in one launch: one 8-CTA cluster per token.  Word 7 of the
+    // workspace statistics is the front end's token counter (zero at launch, left zero).
+    unsigned* ws_stats = reinterpret_cast<unsigned*>(ws + L.stats);
+    unsigned* front_done = ws_stats + 7;
+    if (stats == ws_stats) {
+      MOE_TRY_CUDA(cudaMemsetAsync(ws_stats, 0, 8 * sizeof(unsigned), st));
+    } else {
+      MOE_TRY_CUDA(cudaMemsetAsync(stats, 0, kRouterStats * sizeof(unsigned), st));
+      MOE_TRY_CUDA(cudaMemsetAsync(front_done, 0, sizeof(unsigned), st));
+    }
+    const double u = std::ldexp(1.0, -53), n = (double)H + 8.0;
+    const double beta_scale = 2.0 * (n * u / (1.0 - n * u)) * 1.01;
+    launch(false, decode_front_kernel<4>, dim3(kFrontRanks * T), dim3(32 * kFrontWarps),
+           decode_front_smem_bytes(H, E), static_cast<const __nv_bfloat16*>(x),
+           static_cast<const __nv_bfloat16*>(w_router), router_bias, T, H, E, k,
+           (flags & MOE_FLAG_NO_RENORM) ? 0 : 1, beta_scale, ids, wts, stats, counts, offsets, perm,
+           inv, tile_num, tile_expert, tile_row0, tile_rows, gemm_counters, L.n_counters, L.bm,
+           front_done);
+    if (copy_rows)   // decode tiles read a gathered copy of the routed rows
+      launch(true, gather_rows_kernel, dim3(std::min((P + 7) / 8, gsm)), dim3(256), 0,
+             static_cast<const uint4*>(x), (const int32_t*)perm, P, k, P, H / 8,
+             reinterpret_cast<uint4*>(xp));
+    if (const moe_status_t ls = launched(); ls != MOE_OK) return ls;
+    prof.mark();
+    prof.mark();
+  } else {
+    // one-launch dispatch for 2..32 chunks (every chunk's CTA must be resident at once;
+    // measured on B200: 2 us faster at 8 and 16 chunks, 5-12 us slower at 64 and 128)
+    const bool fused_dispatch =
+        L.nchunks > 1 && L.nchunks <= std::min(kFusedDispatchMaxChunks, d->num_sms);
+    int32_t* dsync = reinterpret_cast<int32_t*>(ws + L.dsync);
+    if (fused_dispatch) MOE_TRY_CUDA(cudaMemsetAsync(dsync, 0, 2 * sizeof(int32_t), st));
+    // 1. router
+    moe_status_t s = launch_router(static_cast<const __nv_bfloat16*>(x),
+                                   static_cast<const __nv_bfloat16*>(w_router), router_bias, T, H,
+                                   E, k, flags, ids, wts, stats, ws, L, *d, st, !prof.on);
+    if (s != MOE_OK) return s;
+    prof.mark();
+    // 2. dispatch
+    if (L.nchunks == 1) {
+      launch(true, dispatch_small_kernel, dim3(1), dim3(256), 0, (const int32_t*)ids, P, E, L.bm,
+             counts, offsets, perm, inv, tile_num, tile_expert, tile_row0, tile_rows,
+             gemm_counters, L.n_counters);
+    } else if (fused_dispatch) {
+      launch(true, dispatch_fused_kernel, dim3(L.nchunks), dim3(32 * kRankWarps),
+             (kRankWarps + 1) * E * sizeof(int), (const int32_t*)ids, P, E, L.bm, L.nchunks,
+             chunk_counts, chunk_base, counts, offsets, perm, inv, tile_num, tile_expert,
+             tile_row0, tile_rows, gemm_counters, L.n_counters, dsync);
+    } else {
+      launch(true, dispatch_count_kernel, dim3(L.nchunks), dim3(256), E * sizeof(int),
+             (const int32_t*)ids, P, E, chunk_counts);
+      launch(true, dispatch_scan_kernel, dim3(1), dim3(256), 0, (const int32_t*)chunk_counts,
+             L.nchunks, E, P, L.bm, counts, offsets, chunk_base, tile_num, tile_expert, tile_row0,
+             tile_rows, gemm_counters, L.n_counters);
+      launch(true, dispatch_rank_kernel, dim3(L.nchunks), dim3(32 * kRankWarps),
+             (kRankWarps + 1) * E * sizeof(int),
+             (const int32_t*)ids, P, E, (const int32_t*)chunk_base, perm, inv);
+    }
+    if (copy_rows)   // the routed rows, in expert order
+      launch(true, gather_rows_kernel, dim3(std::min((P + 7) / 8, gsm)), dim3(256), 0,
+             static_cast<const uint4*>(x), (const int32_t*)perm, P, k, P, H / 8,
+             reinterpret_cast<uint4*>(xp));
+    if (const moe_status_t ls = launched(); ls != MOE_OK) return ls;
+    prof.mark();
+  }
+  return MOE_OK;
+}
+
 // Scratch of moe_route_static: a file-scope device array (every GPU that loads this
 // library holds it until the process exits).  Host code must not use the symbol itself as a
 // device address; moe_route_static looks its address up once per device.
@@ -625,8 +732,6 @@ moe_status_t moe_forward(const void* x, const void* w_router, const float* route
   unsigned* stats = (aux && aux->router_stats) ? aux->router_stats
                                                : reinterpret_cast<unsigned*>(ws + L.stats);
   int32_t* inv = reinterpret_cast<int32_t*>(ws + L.inv);
-  int32_t* chunk_counts = reinterpret_cast<int32_t*>(ws + L.chunk_counts);
-  int32_t* chunk_base = reinterpret_cast<int32_t*>(ws + L.chunk_base);
   int32_t* tile_num = reinterpret_cast<int32_t*>(ws + L.tile_num);
   int32_t* tile_expert = reinterpret_cast<int32_t*>(ws + L.tile_expert);
   int32_t* tile_row0 = reinterpret_cast<int32_t*>(ws + L.tile_row0);
@@ -658,71 +763,12 @@ moe_status_t moe_forward(const void* x, const void* w_router, const float* route
   const int gsm = std::max(1, d->num_sms) * 8;
   // Dependent launches, except while stage events sit between the kernels.
   const Launch launch{st, !prof.on};
-  if (use_decode_front(T, H, E, flags)) {
-    // 1+2. router and dispatch in one launch: one 8-CTA cluster per token.  Word 7 of the
-    // workspace statistics is the front end's token counter (zero at launch, left zero).
-    unsigned* ws_stats = reinterpret_cast<unsigned*>(ws + L.stats);
-    unsigned* front_done = ws_stats + 7;
-    if (stats == ws_stats) {
-      MOE_TRY_CUDA(cudaMemsetAsync(ws_stats, 0, 8 * sizeof(unsigned), st));
-    } else {
-      MOE_TRY_CUDA(cudaMemsetAsync(stats, 0, kRouterStats * sizeof(unsigned), st));
-      MOE_TRY_CUDA(cudaMemsetAsync(front_done, 0, sizeof(unsigned), st));
-    }
-    const double u = std::ldexp(1.0, -53), n = (double)H + 8.0;
-    const double beta_scale = 2.0 * (n * u / (1.0 - n * u)) * 1.01;
-    launch(false, decode_front_kernel<4>, dim3(kFrontRanks * T), dim3(32 * kFrontWarps),
-           decode_front_smem_bytes(H, E), static_cast<const __nv_bfloat16*>(x),
-           static_cast<const __nv_bfloat16*>(w_router), router_bias, T, H, E, k,
-           (flags & MOE_FLAG_NO_RENORM) ? 0 : 1, beta_scale, ids, wts, stats, counts, offsets, perm,
-           inv, tile_num, tile_expert, tile_row0, tile_rows, gemm_counters, L.n_counters, L.bm,
-           front_done);
-    if (dec)   // decode tiles read a gathered copy of the routed rows
-      launch(true, gather_rows_kernel, dim3(std::min((P + 7) / 8, gsm)), dim3(256), 0,
-             static_cast<const uint4*>(x), (const int32_t*)perm, P, k, P, H / 8,
-             reinterpret_cast<uint4*>(xp));
-    if (const moe_status_t ls = launched(); ls != MOE_OK) return ls;
-    prof.mark();
-    prof.mark();
-  } else {
-    // one-launch dispatch for 2..32 chunks (every chunk's CTA must be resident at once;
-    // measured on B200: 2 us faster at 8 and 16 chunks, 5-12 us slower at 64 and 128)
-    const bool fused_dispatch =
-        L.nchunks > 1 && L.nchunks <= std::min(kFusedDispatchMaxChunks, d->num_sms);
-    int32_t* dsync = reinterpret_cast<int32_t*>(ws + L.dsync);
-    if (fused_dispatch) MOE_TRY_CUDA(cudaMemsetAsync(dsync, 0, 2 * sizeof(int32_t), st));
-    // 1. router
-    moe_status_t s = launch_router(static_cast<const __nv_bfloat16*>(x),
-                                   static_cast<const __nv_bfloat16*>(w_router), router_bias, T, H,
-                                   E, k, flags, ids, wts, stats, ws, L, *d, st, !prof.on);
-    if (s != MOE_OK) return s;
-    prof.mark();
-    // 2. dispatch
-    if (L.nchunks == 1) {
-      launch(true, dispatch_small_kernel, dim3(1), dim3(256), 0, (const int32_t*)ids, P, E, L.bm,
-             counts, offsets, perm, inv, tile_num, tile_expert, tile_row0, tile_rows,
-             gemm_counters, L.n_counters);
-    } else if (fused_dispatch) {
-      launch(true, dispatch_fused_kernel, dim3(L.nchunks), dim3(32 * kRankWarps),
-             (kRankWarps + 1) * E * sizeof(int), (const int32_t*)ids, P, E, L.bm, L.nchunks,
-             chunk_counts, chunk_base, counts, offsets, perm, inv, tile_num, tile_expert,
-             tile_row0, tile_rows, gemm_counters, L.n_counters, dsync);
-    } else {
-      launch(true, dispatch_count_kernel, dim3(L.nchunks), dim3(256), E * sizeof(int),
-             (const int32_t*)ids, P, E, chunk_counts);
-      launch(true, dispatch_scan_kernel, dim3(1), dim3(256), 0, (const int32_t*)chunk_counts,
-             L.nchunks, E, P, L.bm, counts, offsets, chunk_base, tile_num, tile_expert, tile_row0,
-             tile_rows, gemm_counters, L.n_counters);
-      launch(true, dispatch_rank_kernel, dim3(L.nchunks), dim3(32 * kRankWarps),
-             (kRankWarps + 1) * E * sizeof(int),
-             (const int32_t*)ids, P, E, (const int32_t*)chunk_base, perm, inv);
-    }
-    if (dec || use_row_copy(T, flags))   // the routed rows, in expert order
-      launch(true, gather_rows_kernel, dim3(std::min((P + 7) / 8, gsm)), dim3(256), 0,
-             static_cast<const uint4*>(x), (const int32_t*)perm, P, k, P, H / 8,
-             reinterpret_cast<uint4*>(xp));
-    if (const moe_status_t ls = launched(); ls != MOE_OK) return ls;
-    prof.mark();
+  {
+    const RouteBufs rb{ids, wts, stats, counts, offsets, perm, inv};
+    if (const moe_status_t rs = route_and_dispatch(x, w_router, router_bias, T, H, E, k, flags, rb,
+                                                   ws, L, *d, st, prof, dec || use_row_copy(T, flags));
+        rs != MOE_OK)
+      return rs;
   }
   // 3. GEMM-1 + GEGLU, 4. GEMM-2 (down)
   TileList tl{tile_num, tile_expert, tile_row0, tile_rows, 0, perm, k,
@@ -1139,6 +1185,161 @@ moe_status_t moe_combine(const void* o, const int32_t* inv, const float* topk_we
     launch(false, combine_kernel<false>, grid, dim3(256), 0, static_cast<const uint4*>(o), inv,
            topk_weights, T, k, H / 8, row_lo, row_hi, y);
   return launched();
+}
+
+// ----------------------------------------------------------------------------- NVFP4
+size_t moe_nvfp4_quantize_workspace_size(int E) {
+  return E >= 1 ? align256(sizeof(unsigned) * (size_t)E) : 0;
+}
+
+moe_status_t moe_nvfp4_quantize_weights(const void* w, int E, int K, int N, uint8_t* codes,
+                                        uint8_t* scales, float* ts, void* workspace,
+                                        size_t workspace_bytes, void* stream) {
+  if (E <= 0 || K <= 0 || N <= 0) return MOE_ERR_INVALID_ARG;
+  if (!w || !codes || !scales || !ts || !workspace) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(w) || !aligned16(codes) || !aligned16(workspace)) return MOE_ERR_INVALID_ARG;
+  if (K % 32 || K > 16384 || N > (1 << 20) || E > 65535) return MOE_ERR_UNSUPPORTED;
+  if (workspace_bytes < moe_nvfp4_quantize_workspace_size(E)) return MOE_ERR_NO_WORKSPACE;
+  int dev = 0;
+  DeviceState* d = device_state(&dev);
+  if (!d) return MOE_ERR_CUDA;
+  t_kernels = 0;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  unsigned* amax = static_cast<unsigned*>(workspace);
+  MOE_TRY_CUDA(cudaMemsetAsync(amax, 0, sizeof(unsigned) * E, st));
+  const long long per = (long long)K * N;
+  const Launch launch{st, false};
+  launch(false, nvfp4_amax_kernel, dim3((unsigned)std::min<long long>((per + 2047) / 2048, 1024), E),
+         dim3(256), 0, static_cast<const __nv_bfloat16*>(w), per, amax);
+  launch(false, nvfp4_weight_quant_kernel, dim3((N + 255) / 256, K / 16, E), dim3(256), 0,
+         static_cast<const __nv_bfloat16*>(w), K, N, (const unsigned*)amax, codes, scales, ts);
+  return launched();
+}
+
+moe_status_t moe_nvfp4_quantize_rows(const void* x, int rows, int K, float ts, uint8_t* codes,
+                                     uint8_t* scales, void* stream) {
+  if (rows < 0 || K <= 0 || !(ts > 0.f)) return MOE_ERR_INVALID_ARG;
+  if (rows == 0) return MOE_OK;
+  if (!x || !codes || !scales || !aligned16(x) || !aligned16(codes)) return MOE_ERR_INVALID_ARG;
+  if (K % 16 || (long long)rows * K > (1ll << 34)) return MOE_ERR_UNSUPPORTED;
+  int dev = 0;
+  DeviceState* d = device_state(&dev);
+  if (!d) return MOE_ERR_CUDA;
+  t_kernels = 0;
+  const Launch launch{static_cast<cudaStream_t>(stream), false};
+  const long long groups = (long long)rows * (K / 16);
+  launch(false, nvfp4_rows_quant_kernel,
+         dim3((unsigned)std::min<long long>((groups + 255) / 256, (long long)d->num_sms * 16)),
+         dim3(256), 0, static_cast<const __nv_bfloat16*>(x), (long long)rows, K, ts, codes, scales);
+  return launched();
+}
+
+namespace {
+constexpr unsigned kFp4Flags = MOE_FLAG_NO_RENORM | MOE_FLAG_ROUTER_FP64 | MOE_FLAG_ROUTER_SCREEN |
+                               MOE_FLAG_PROFILE_STAGES;
+int fp4_max_rows(int T) { return T <= 8 ? 8 : FP4_MAX_ROWS; }
+size_t fp4_smem1(int T, int H) { return (size_t)std::min(T, FP4_MAX_ROWS) * H * 2; }
+size_t fp4_smem2(int T, int I) {
+  return (size_t)std::min(T, FP4_MAX_ROWS) * I * 2 + (size_t)fp4_max_rows(T) * 64 * (2 + 4);
+}
+// h between the two GEMMs, fp32 [T k][I], after the forward's own layout
+size_t fp4_h32_bytes(int T, int I, int k) { return ((size_t)T * k * I * 4 + 255) / 256 * 256; }
+bool fp4_shape_ok(int T, int H, int E, int I, int k) {
+  return shape_supported(T, H, E, I, k, true) && T <= FP4_MAX_ROWS &&
+         fp4_smem1(T, H) <= (size_t)kFp4SmemMax && fp4_smem2(T, I) <= (size_t)kFp4SmemMax;
+}
+}  // namespace
+
+size_t moe_nvfp4_workspace_size(int T, int H, int E, int I, int k, unsigned flags) {
+  if ((flags & ~kFp4Flags) || !flags_ok(flags) || !fp4_shape_ok(T, H, E, I, k) ||
+      !forced_path_ok(E, flags))
+    return 0;
+  return make_layout(T, H, E, I, k, flags, true).total + fp4_h32_bytes(T, I, k);
+}
+
+moe_status_t moe_forward_nvfp4(const void* x, const void* w_router, const float* router_bias,
+                               const moe_nvfp4_weights_t* w, int T, int H, int E, int I, int k,
+                               unsigned flags, float act_scale_x, float act_scale_h, void* y,
+                               const moe_aux_t* aux, void* workspace, size_t workspace_bytes,
+                               void* stream) {
+  if (T < 0 || H <= 0 || E <= 0 || I <= 0 || k < 1 || k > E) return MOE_ERR_INVALID_ARG;
+  if ((flags & ~kFp4Flags) || !flags_ok(flags)) return MOE_ERR_INVALID_ARG;
+  if (!(act_scale_x > 0.f) || !(act_scale_h > 0.f)) return MOE_ERR_INVALID_ARG;
+  if (T == 0) return MOE_OK;
+  if (!x || !w_router || !w || !y || !workspace || !w->gate_codes || !w->gate_scales ||
+      !w->gate_ts || !w->up_codes || !w->up_scales || !w->up_ts || !w->down_codes ||
+      !w->down_scales || !w->down_ts)
+    return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(w_router) || !aligned16(y) || !aligned16(workspace) ||
+      !aligned16(w->gate_codes) || !aligned16(w->up_codes) || !aligned16(w->down_codes) ||
+      (reinterpret_cast<uintptr_t>(w->gate_scales) & 1) ||
+      (reinterpret_cast<uintptr_t>(w->up_scales) & 1) ||
+      (reinterpret_cast<uintptr_t>(w->down_scales) & 1))
+    return MOE_ERR_INVALID_ARG;
+  if (x == y) return MOE_ERR_INVALID_ARG;
+  if (!fp4_shape_ok(T, H, E, I, k) || !forced_path_ok(E, flags)) return MOE_ERR_UNSUPPORTED;
+  const Layout L = make_layout(T, H, E, I, k, flags, true);
+  if (workspace_bytes < L.total + fp4_h32_bytes(T, I, k)) return MOE_ERR_NO_WORKSPACE;
+  int dev = 0;
+  DeviceState* d = device_state(&dev);
+  if (!d) return MOE_ERR_CUDA;
+  t_kernels = 0;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  const int P = T * k;
+  int32_t* ids = (aux && aux->topk_ids) ? aux->topk_ids : reinterpret_cast<int32_t*>(ws + L.ids);
+  float* wts = (aux && aux->topk_weights) ? aux->topk_weights : reinterpret_cast<float*>(ws + L.wts);
+  int32_t* counts =
+      (aux && aux->expert_counts) ? aux->expert_counts : reinterpret_cast<int32_t*>(ws + L.counts);
+  int32_t* offsets = (aux && aux->expert_offsets) ? aux->expert_offsets
+                                                  : reinterpret_cast<int32_t*>(ws + L.offsets);
+  int32_t* perm = (aux && aux->perm) ? aux->perm : reinterpret_cast<int32_t*>(ws + L.perm);
+  unsigned* stats = (aux && aux->router_stats) ? aux->router_stats
+                                               : reinterpret_cast<unsigned*>(ws + L.stats);
+  int32_t* inv = reinterpret_cast<int32_t*>(ws + L.inv);
+  int32_t* tile_num = reinterpret_cast<int32_t*>(ws + L.tile_num);
+  int32_t* tile_expert = reinterpret_cast<int32_t*>(ws + L.tile_expert);
+  int32_t* tile_row0 = reinterpret_cast<int32_t*>(ws + L.tile_row0);
+  int32_t* tile_rows = reinterpret_cast<int32_t*>(ws + L.tile_rows);
+  float* h32 = reinterpret_cast<float*>(ws + L.total);   // [P][I]
+  __nv_bfloat16* obuf = reinterpret_cast<__nv_bfloat16*>(ws + L.obuf);
+
+  Profiler prof{d, st, (flags & MOE_FLAG_PROFILE_STAGES) != 0};
+  prof.mark();
+  const RouteBufs rb{ids, wts, stats, counts, offsets, perm, inv};
+  if (const moe_status_t rs = route_and_dispatch(x, w_router, router_bias, T, H, E, k, flags, rb,
+                                                 ws, L, *d, st, prof, false);
+      rs != MOE_OK)
+    return rs;
+  // 3. GEMM-1 + GEGLU, 4. GEMM-2 (h quantised as it is staged): one CTA per (tile, group of
+  // 8 features or 64 output columns); a tile is one expert's rows (at most T <= 16), so there
+  // are at most min(E, T k) tiles
+  const Launch launch{st, !prof.on};
+  const int max_tiles = std::min(E, P);
+  const bool r8 = fp4_max_rows(T) == 8;
+  launch(true, r8 ? nvfp4_gemm1_kernel<8> : nvfp4_gemm1_kernel<FP4_MAX_ROWS>,
+         dim3(max_tiles, (I + FP4_G1_FEATS - 1) / FP4_G1_FEATS), dim3(32 * FP4_G1_FEATS),
+         fp4_smem1(T, H), static_cast<const __nv_bfloat16*>(x), (const int32_t*)perm, k, T,
+         (const int32_t*)tile_num, (const int32_t*)tile_expert, (const int32_t*)tile_row0,
+         (const int32_t*)tile_rows, w->gate_codes, w->gate_scales, w->gate_ts, w->up_codes,
+         w->up_scales, w->up_ts, H, I, act_scale_x, h32);
+  launch(true, r8 ? nvfp4_gemm2_kernel<8> : nvfp4_gemm2_kernel<FP4_MAX_ROWS>,
+         dim3(max_tiles, (H + 63) / 64), dim3(256), fp4_smem2(T, I), (const float*)h32,
+         (const int32_t*)tile_num, (const int32_t*)tile_expert, (const int32_t*)tile_row0,
+         (const int32_t*)tile_rows, w->down_codes, w->down_scales, w->down_ts, H, I, act_scale_h,
+         obuf);
+  if (const moe_status_t ls = launched(); ls != MOE_OK) return ls;
+  prof.mark();
+  // 5. combine
+  const int gsm = std::max(1, d->num_sms) * 8;
+  const long long citems = (long long)T * ((H / 8 + kCombineChunkVec - 1) / kCombineChunkVec);
+  launch(true, combine_kernel<false>, dim3((int)std::min<long long>((citems + 7) / 8, gsm)),
+         dim3(256), 0, reinterpret_cast<const uint4*>(obuf), (const int32_t*)inv,
+         (const float*)wts, T, k, H / 8, 0, P, y);
+  if (const moe_status_t ls = launched(); ls != MOE_OK) return ls;
+  prof.mark();
+  prof.finish();
+  return MOE_OK;
 }
 
 moe_status_t moe_route_static(const void* x, const void* w_router, const float* router_bias,

@@ -39,7 +39,7 @@
 extern "C" {
 #endif
 
-#define MOE_ABI_VERSION 4
+#define MOE_ABI_VERSION 5
 
 typedef enum {
   MOE_OK = 0,
@@ -259,6 +259,62 @@ enum { MOE_COMBINE_F32 = 1u << 0 };
 moe_status_t moe_combine(const void *o, const int32_t *inv, const float *topk_weights, int T,
                          int k, int H, int row_lo, int row_hi, unsigned flags, void *y,
                          void *stream);
+
+/*
+ * NVFP4 experts.  The Gemma-4-26B-A4B-NVFP4 checkpoint keeps weights AND activations in
+ * "4-bit float, group_size=16" (Gemma-4-26B-A4B-NVFP4 Ascend verification report, §2.3 量化配置
+ * (NVFP4)).  The format (its published definition): E2M1 elements (magnitudes 0, 0.5, 1, 1.5,
+ * 2, 3, 4, 6), one E4M3 scale per 16 consecutive elements along the reduction axis K, one fp32
+ * scale per tensor; value = e2m1 * e4m3 * tensor_scale.  Quantisation of a group v[16], each
+ * step one IEEE fp32 operation rounding to nearest even: amax = max |v|; s = (amax / 6) / ts;
+ * s8 = E4M3(s) (saturating at 448); S = e4m3(s8) * ts; code_i = E2M1(v_i / S) (saturating
+ * at 6, sign kept), or 0 when S == 0.  A weight tensor's ts = amax / (6 * 448).
+ *
+ * Layout of one projection with reduction depth K and N outputs (a Linear layer's weight,
+ * K contiguous): codes uint8 [E][N][K/2] (byte b of a row holds element 2b in its low nibble,
+ * 2b+1 in its high nibble), scales uint8 [E][N][K/16] (E4M3 bytes), ts fp32 [E].  The layer's
+ * projections: gate and up with K = H, N = I; down with K = I, N = H.
+ */
+typedef struct {
+  const uint8_t *gate_codes, *gate_scales; /* [E][I][H/2], [E][I][H/16] */
+  const float *gate_ts;                    /* [E]                       */
+  const uint8_t *up_codes, *up_scales;     /* [E][I][H/2], [E][I][H/16] */
+  const float *up_ts;                      /* [E]                       */
+  const uint8_t *down_codes, *down_scales; /* [E][H][I/2], [E][H][I/16] */
+  const float *down_ts;                    /* [E]                       */
+} moe_nvfp4_weights_t;
+
+/* Quantise bf16 weights w [E][K][N] (N contiguous: the layout moe_forward takes, e.g. W_gate
+ * with K = H, N = I) into the layout above: codes [E][N][K/2], scales [E][N][K/16], ts [E].
+ * K % 32 == 0, K <= 16384.  Workspace: moe_nvfp4_quantize_workspace_size(E) bytes. */
+size_t moe_nvfp4_quantize_workspace_size(int E);
+moe_status_t moe_nvfp4_quantize_weights(const void *w, int E, int K, int N, uint8_t *codes,
+                                        uint8_t *scales, float *ts, void *workspace,
+                                        size_t workspace_bytes, void *stream);
+
+/* The activation quantiser as a call of its own: x bf16 [rows][K] with tensor scale ts ->
+ * codes [rows][K/2], scales [rows][K/16] (the decisions moe_forward_nvfp4 takes on x). */
+moe_status_t moe_nvfp4_quantize_rows(const void *x, int rows, int K, float ts, uint8_t *codes,
+                                     uint8_t *scales, void *stream);
+
+/*
+ * moe_forward_nvfp4 -- the routed layer with NVFP4 expert weights and activations, for
+ * batches of 1 <= T <= 16 tokens (decode).  Router, dispatch and combine as moe_forward
+ * (bf16 router, same ids and weights); expert e on a routed row:
+ *     xq = NVFP4(x row, act_scale_x);  g = xq Wg[e];  u = xq Wu[e];  h = gelu_tanh(g) * u;
+ *     hq = NVFP4(h, act_scale_h) (groups of 16 consecutive features);  o = hq Wd[e]
+ * with the dequantised weights; products exact, sums in fp32, h quantised from fp32, o and y
+ * rounded to bf16.  act_scale_x / act_scale_h: the fixed activation tensor scales (> 0).
+ * flags: MOE_FLAG_NO_RENORM, MOE_FLAG_ROUTER_FP64 / _SCREEN, MOE_FLAG_PROFILE_STAGES only.
+ * Limits: shapes as moe_forward, T <= 16, min(T,16) * H * 2 + 2048 and min(T,16) * I * 2 + 2048
+ * bytes at most 227 KB.  Workspace: moe_nvfp4_workspace_size bytes.
+ */
+size_t moe_nvfp4_workspace_size(int T, int H, int E, int I, int k, unsigned flags);
+moe_status_t moe_forward_nvfp4(const void *x, const void *w_router, const float *router_bias,
+                               const moe_nvfp4_weights_t *w, int T, int H, int E, int I, int k,
+                               unsigned flags, float act_scale_x, float act_scale_h, void *y,
+                               const moe_aux_t *aux, void *workspace, size_t workspace_bytes,
+                               void *stream);
 
 /*
  * moe_route_static -- moe_route for callers that cannot allocate device memory.

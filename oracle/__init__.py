@@ -75,8 +75,6 @@ def lib():
         L.oracle_nvfp4_quantize.argtypes = [_P, _I64, _I, _F, _P, _P]
         L.oracle_nvfp4_dequantize.argtypes = [_P, _P, _I64, _I, _F, _P]
         L.oracle_expert_ffn_nvfp4.argtypes = [_P, _P, _P, _P, _I, _I, _F, _F, _P]
-        L.oracle_forward_nvfp4.argtypes = [_P, _P, _P, _P, _P, _P, _I64, _I, _I, _I, _I, _I, _F,
-                                           _F, _P, _I64, _P, _P, _P, _P]
         _lib = L
     return _lib
 
@@ -275,22 +273,25 @@ def forward_nvfp4(x, w_router, wq: dict, k: int, bias=None, renorm: bool = True,
                   act_scale_x: float = 1.0, act_scale_h: float = 1.0, tokens=None):
     """The layer with NVFP4 expert weights (given quantised, see quantize_expert_weights) and
     NVFP4 activations (x before GEMM-1, h before GEMM-2, with fixed tensor scales).  Routing
-    as forward().  -> dict(ids, weights, logits, y)."""
-    xb, wr, b = _u16(x), _u16(w_router), _f32(bias)
+    as forward(); y[t] = sum_j w[t,j] o_{t,j} in slot order, each o from expert_ffn_nvfp4
+    (the experts are dequantised one at a time).  -> dict(ids, weights, logits, y)."""
+    xb = _u16(x)
     T, H = xb.shape
-    E = wr.shape[1]
-    dq = dequantize_expert_weights(wq)
-    I = dq["gate"].shape[1]
-    tok = None if tokens is None else np.ascontiguousarray(tokens, dtype=np.int64)
-    n_tok = T if tok is None else len(tok)
-    ids = np.empty((T, k), np.int32)
-    w = np.empty((T, k), np.float64)
-    L = np.empty((T, E), np.float64)
-    y = np.empty((n_tok, H), np.float64)
-    g, u, d = (np.ascontiguousarray(dq[n]) for n in ("gate", "up", "down"))
-    lib().oracle_forward_nvfp4(_ptr(xb), _ptr(wr), _ptr(b), _ptr(g), _ptr(u), _ptr(d), T, H, E,
-                               I, k, int(bool(renorm)), float(act_scale_x), float(act_scale_h),
-                               _ptr(tok), n_tok, _ptr(ids), _ptr(w), _ptr(L), _ptr(y))
+    ids, w, L = route(x, w_router, k, bias=bias, renorm=renorm)
+    tok = np.arange(T) if tokens is None else np.asarray(tokens, dtype=np.int64)
+    o = {}                                   # (row, slot) -> expert output
+    for e in np.unique(ids[tok]):
+        dq = [nvfp4_dequantize(wq[f"{n}_codes"][e], wq[f"{n}_scales"][e], wq[f"{n}_ts"][e])
+              for n in ("gate", "up", "down")]
+        for r, t in enumerate(tok):
+            for j in range(k):
+                if ids[t, j] == e:
+                    o[(r, j)] = expert_ffn_nvfp4(xb[t], dq[0], dq[1], dq[2], act_scale_x,
+                                                 act_scale_h)
+    y = np.zeros((len(tok), H), np.float64)
+    for r in range(len(tok)):
+        for j in range(k):
+            y[r] += w[tok[r], j] * o[(r, j)]
     return {"ids": ids, "weights": w, "logits": L, "y": y}
 
 

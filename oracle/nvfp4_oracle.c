@@ -27,9 +27,11 @@
  *   the sign bit is the input's, also when the magnitude rounds to zero).
  * Weight tensor scale: ts = amax over the tensor / (6 * 448), one fp32 division.
  * Dequantised values are exact in double (each is a product of at most 2 + 4 + 24 significant
- * bits).  The layer computes in double with no rounding, except that the intermediate h of
- * each expert is quantised as an activation: h is rounded to fp32 first (the precision the
- * quantisation decisions are taken in).
+ * bits).  One expert on one row computes in double with no rounding, except that its
+ * intermediate h is quantised as an activation: h is rounded to fp32 first (the precision the
+ * quantisation decisions are taken in).  The layer (routing, the weighted sum over the k
+ * experts in slot order) is composed in oracle/__init__.py from the routing functions of
+ * moe_oracle.c and this file's expert.
  */
 #include <math.h>
 #include <stdint.h>
@@ -136,10 +138,6 @@ static double bf16_value(uint16_t b) {
 }
 
 double oracle_gelu_tanh(double a);
-void oracle_router_logits(const uint16_t *x, const uint16_t *wr, const float *bias, int64_t T,
-                          int H, int E, double *logits);
-void oracle_select(const double *logits, int64_t T, int E, int k, int renorm, int32_t *ids,
-                   double *weights);
 
 /* Activation quantisation of one row: v (fp32) [K] -> dequantised values [K]. */
 static void act_qdq(const float *v, int K, float ts, uint8_t *codes, uint8_t *sc, double *out) {
@@ -187,34 +185,4 @@ static void expert_ffn_q(const uint16_t *xrow, const double *wg, const double *w
 void oracle_expert_ffn_nvfp4(const uint16_t *xrow, const double *wg, const double *wu,
                              const double *wd, int H, int I, float sx, float sh, double *out) {
     expert_ffn_q(xrow, wg, wu, wd, H, I, sx, sh, out);
-}
-
-/* Whole layer with NVFP4 experts.  Router, selection and combine as oracle_forward; the
- * experts' weights given dequantised: wg, wu [E][I][H], wd [E][H][I] (doubles). */
-void oracle_forward_nvfp4(const uint16_t *x, const uint16_t *w_router, const float *bias,
-                          const double *wg, const double *wu, const double *wd, int64_t T,
-                          int H, int E, int I, int k, int renorm, float sx, float sh,
-                          const int64_t *tokens, int64_t n_tok, int32_t *ids, double *weights,
-                          double *logits, double *y) {
-    oracle_router_logits(x, w_router, bias, T, H, E, logits);
-    oracle_select(logits, T, E, k, renorm, ids, weights);
-    if (!tokens) n_tok = T;
-    const int64_t hi = (int64_t)H * I;
-#pragma omp parallel
-    {
-        double *o = (double *)malloc(sizeof(double) * (size_t)H);
-#pragma omp for schedule(dynamic, 1)
-        for (int64_t r = 0; r < n_tok; ++r) {
-            const int64_t t = tokens ? tokens[r] : r;
-            double *yr = y + r * H;
-            for (int n = 0; n < H; ++n) yr[n] = 0.0;
-            for (int j = 0; j < k; ++j) {
-                const int64_t e = ids[t * k + j];
-                expert_ffn_q(x + t * H, wg + e * hi, wu + e * hi, wd + e * hi, H, I, sx, sh, o);
-                const double w = weights[t * k + j];
-                for (int n = 0; n < H; ++n) yr[n] += w * o[n];
-            }
-        }
-        free(o);
-    }
 }
