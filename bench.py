@@ -359,7 +359,7 @@ def nvfp4_entry(cfg, m: dict, world: int, pk: dict) -> dict:
                     "weights and activations NVFP4 (E2M1, E4M3 scale per 16, fp32 per tensor), "
                     "weights quantised from the bf16 set",
         "value": job_throughput(world, cfg.T, m["ms"]), "unit": UNIT, "ms_per_step": m["ms"],
-        "expert_ffn": {"kernels": "nvfp4_gemm1_kernel + nvfp4_gemm2_kernel", "ms": m["ffn_ms"],
+        "expert_ffn": {"kernels": "nvfp4_rows_sorted_kernel + nvfp4_ffn_kernel (tcgen05 kind::mxf4nvf4)", "ms": m["ffn_ms"],
                        "algorithmic_bytes": ffn_bytes, "achieved_gbs": ach,
                        "frac_of_hbm": None if ach is None else ach / pk["hbm_gbs"]},
         "step_hbm_frac": step_bytes / (m["ms"] * 1e-3) / (pk["hbm_gbs"] * 1e9),

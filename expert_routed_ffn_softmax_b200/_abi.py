@@ -365,13 +365,14 @@ def combine(o: torch.Tensor, inv: torch.Tensor, topk_weights: torch.Tensor, row_
 # ----------------------------------------------------------------------------- NVFP4
 def nvfp4_quantize_weights(w: torch.Tensor, stream=None) -> dict:
     """moe_nvfp4_quantize_weights: bf16 w [E, K, N] (N contiguous) -> {codes uint8 [E, N, K/2],
-    scales uint8 [E, N, K/16], ts float32 [E]} on w's device."""
+    scales uint8 [E, ceil(N/128), K/64, 512] (the blocked scale layout of include/moe.h),
+    ts float32 [E]} on w's device."""
     L = load()
     E, K, N = w.shape
     dev = w.device
     pw = _dev(w, "w", torch.bfloat16, (E, K, N))
     codes = torch.empty((E, N, K // 2), dtype=torch.uint8, device=dev)
-    scales = torch.empty((E, N, K // 16), dtype=torch.uint8, device=dev)
+    scales = torch.empty((E, (N + 127) // 128, K // 64, 512), dtype=torch.uint8, device=dev)
     ts = torch.empty(E, dtype=torch.float32, device=dev)
     ws = torch.empty(max(256, L.moe_nvfp4_quantize_workspace_size(E)), dtype=torch.uint8, device=dev)
     _check(L.moe_nvfp4_quantize_weights(pw, E, K, N, codes.data_ptr(), scales.data_ptr(),
@@ -419,9 +420,11 @@ def forward_nvfp4(x: torch.Tensor, w_router: torch.Tensor, wq: dict, k: int,
     px = _dev(x, "x", torch.bfloat16, (T, H))
     pr = _dev(w_router, "w_router", torch.bfloat16, (H, E))
     pb = None if bias is None else _dev(bias, "bias", torch.float32, (E,))
-    shapes = {"gate_codes": ((E, I, H // 2), torch.uint8), "gate_scales": ((E, I, H // 16), torch.uint8),
-              "up_codes": ((E, I, H // 2), torch.uint8), "up_scales": ((E, I, H // 16), torch.uint8),
-              "down_codes": ((E, H, I // 2), torch.uint8), "down_scales": ((E, H, I // 16), torch.uint8),
+    sc_i = (E, (I + 127) // 128, H // 64, 512)   # blocked scales, N = I, K = H
+    sc_h = (E, (H + 127) // 128, I // 64, 512)   # N = H, K = I
+    shapes = {"gate_codes": ((E, I, H // 2), torch.uint8), "gate_scales": (sc_i, torch.uint8),
+              "up_codes": ((E, I, H // 2), torch.uint8), "up_scales": (sc_i, torch.uint8),
+              "down_codes": ((E, H, I // 2), torch.uint8), "down_scales": (sc_h, torch.uint8),
               "gate_ts": ((E,), torch.float32), "up_ts": ((E,), torch.float32),
               "down_ts": ((E,), torch.float32)}
     wstruct = NVFP4Weights(*(_dev(wq[n], n, shapes[n][1], shapes[n][0])

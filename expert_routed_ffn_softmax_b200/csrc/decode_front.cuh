@@ -30,14 +30,6 @@ constexpr int kFrontMaxTokens = 8;
 constexpr int kFrontWarps = 8;
 constexpr int kFrontChunks = 4;     // bulk copies of the W_router slice (2 warps each)
 
-__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes,
-                                          uint32_t bar) {
-  asm volatile(
-      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar)
-      : "memory");
-}
-
 // Dynamic shared memory layout (bytes from a 16-byte aligned base):
 //   W   max(hs*E*2, 2*NW*E*8)    W_router slice (bf16), later the cross-warp reduction
 //   XS  hs*8                     the token's x slice as doubles

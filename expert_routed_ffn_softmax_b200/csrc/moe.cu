@@ -22,6 +22,7 @@
 #include "decode_front.cuh"
 #include "gemm_decode.cuh"
 #include "nvfp4.cuh"
+#include "nvfp4_mma.cuh"
 
 namespace moe {
 namespace {
@@ -32,7 +33,6 @@ constexpr int kScreenMinTokens = 256;            // default router path switch
 constexpr int kMaxGemmCtas = 256;                // >= SMs per GPU (148 on B200)
 constexpr int kStreamKCounters = 4 * 2 * kMaxGemmCtas;   // per GEMM: 4 per split unit
 constexpr int kFrontSmemMax = 200 * 1024;        // decode front kernel's dynamic smem cap
-constexpr int kFp4SmemMax = 227 * 1024;          // NVFP4 FFN kernels' dynamic smem cap
 
 constexpr double kScreenC = 1.0 / 1024.0;        // screen error bound / (|x| |w|)
 constexpr int kRouterStats = 5;                  // words of moe_aux_t::router_stats
@@ -280,6 +280,33 @@ bool make_map_2d(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Bytes [rows][cols] (cols contiguous, cols % 16 == 0), box = 128 bytes x box_rows rows,
+// 128-byte swizzle: NVFP4 codes (two per byte) as a K-major MMA operand.
+bool make_map_u8_2d(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows,
+                    uint32_t box_rows) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols};
+  cuuint32_t box[2] = {128, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+// Stacked bytes [E][rows][cols], box = 128 bytes x 128 rows x 1 expert, 128-byte swizzle.
+bool make_map_u8_3d(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, uint64_t E) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {cols, rows, E};
+  cuuint64_t strides[2] = {cols, cols * rows};
+  cuuint32_t box[3] = {128, 128, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // Stacked [E][rows][cols] bf16 (cols contiguous), box = 64 columns x box_rows rows x 1 expert.
 bool make_map_3d(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, uint64_t E,
                  uint32_t box_rows = 64) {
@@ -369,14 +396,8 @@ DeviceState* device_state(int* dev_out) {
             cudaSuccess ||
         cudaFuncSetAttribute(expert_ffn_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              PR_SMEM) != cudaSuccess ||
-        cudaFuncSetAttribute(nvfp4_gemm1_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             kFp4SmemMax) != cudaSuccess ||
-        cudaFuncSetAttribute(nvfp4_gemm1_kernel<FP4_MAX_ROWS>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, kFp4SmemMax) != cudaSuccess ||
-        cudaFuncSetAttribute(nvfp4_gemm2_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             kFp4SmemMax) != cudaSuccess ||
-        cudaFuncSetAttribute(nvfp4_gemm2_kernel<FP4_MAX_ROWS>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, kFp4SmemMax) != cudaSuccess ||
+        cudaFuncSetAttribute(nvfp4_ffn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             F4_SMEM) != cudaSuccess ||
         cudaFuncSetAttribute(GEMM_FFN_SMALL, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              pgemm_smem_bytes<kSmallStages, 4, true>()) != cudaSuccess ||
         cudaFuncSetAttribute(GEMM_STORE, cudaFuncAttributeMaxDynamicSharedMemorySize, gs) !=
@@ -1198,7 +1219,7 @@ moe_status_t moe_nvfp4_quantize_weights(const void* w, int E, int K, int N, uint
   if (E <= 0 || K <= 0 || N <= 0) return MOE_ERR_INVALID_ARG;
   if (!w || !codes || !scales || !ts || !workspace) return MOE_ERR_INVALID_ARG;
   if (!aligned16(w) || !aligned16(codes) || !aligned16(workspace)) return MOE_ERR_INVALID_ARG;
-  if (K % 32 || K > 16384 || N > (1 << 20) || E > 65535) return MOE_ERR_UNSUPPORTED;
+  if (K % 64 || K > 16384 || N > (1 << 20) || E > 65535) return MOE_ERR_UNSUPPORTED;
   if (workspace_bytes < moe_nvfp4_quantize_workspace_size(E)) return MOE_ERR_NO_WORKSPACE;
   int dev = 0;
   DeviceState* d = device_state(&dev);
@@ -1211,7 +1232,8 @@ moe_status_t moe_nvfp4_quantize_weights(const void* w, int E, int K, int N, uint
   const Launch launch{st, false};
   launch(false, nvfp4_amax_kernel, dim3((unsigned)std::min<long long>((per + 2047) / 2048, 1024), E),
          dim3(256), 0, static_cast<const __nv_bfloat16*>(w), per, amax);
-  launch(false, nvfp4_weight_quant_kernel, dim3((N + 255) / 256, K / 16, E), dim3(256), 0,
+  launch(false, nvfp4_weight_quant_kernel, dim3(((N + 127) / 128 * 128 + 255) / 256, K / 16, E),
+         dim3(256), 0,
          static_cast<const __nv_bfloat16*>(w), K, N, (const unsigned*)amax, codes, scales, ts);
   return launched();
 }
@@ -1237,16 +1259,31 @@ moe_status_t moe_nvfp4_quantize_rows(const void* x, int rows, int K, float ts, u
 namespace {
 constexpr unsigned kFp4Flags = MOE_FLAG_NO_RENORM | MOE_FLAG_ROUTER_FP64 | MOE_FLAG_ROUTER_SCREEN |
                                MOE_FLAG_PROFILE_STAGES;
-int fp4_max_rows(int T) { return T <= 8 ? 8 : FP4_MAX_ROWS; }
-size_t fp4_smem1(int T, int H) { return (size_t)std::min(T, FP4_MAX_ROWS) * H * 2; }
-size_t fp4_smem2(int T, int I) {
-  return (size_t)std::min(T, FP4_MAX_ROWS) * I * 2 + (size_t)fp4_max_rows(T) * 64 * (2 + 4);
+// The forward's own layout, then (256-byte aligned): sorted x codes [P][H/2] and scales
+// [P][H/16], h codes [P][I/2] and scales [P][I/16], the FFN counters (unit counter, h_ready).
+struct Fp4Layout {
+  size_t xq, xsf, hq, hsf, ctr, total;
+  int n_ctr;
+};
+Fp4Layout fp4_layout(size_t at, int T, int H, int E, int I, int k) {
+  Fp4Layout F;
+  const size_t P = (size_t)T * k;
+  auto take = [&](size_t bytes) {
+    const size_t o = at;
+    at = align256(at + bytes);
+    return o;
+  };
+  F.xq = take(P * H / 2);
+  F.xsf = take(P * H / 16);
+  F.hq = take(P * I / 2);
+  F.hsf = take(P * I / 16);
+  F.n_ctr = 1 + std::min(E, (int)P);
+  F.ctr = take(sizeof(int) * F.n_ctr);
+  F.total = at;
+  return F;
 }
-// h between the two GEMMs, fp32 [T k][I], after the forward's own layout
-size_t fp4_h32_bytes(int T, int I, int k) { return ((size_t)T * k * I * 4 + 255) / 256 * 256; }
 bool fp4_shape_ok(int T, int H, int E, int I, int k) {
-  return shape_supported(T, H, E, I, k, true) && T <= FP4_MAX_ROWS &&
-         fp4_smem1(T, H) <= (size_t)kFp4SmemMax && fp4_smem2(T, I) <= (size_t)kFp4SmemMax;
+  return shape_supported(T, H, E, I, k, true) && T <= FP4_MAX_ROWS;
 }
 }  // namespace
 
@@ -1254,7 +1291,7 @@ size_t moe_nvfp4_workspace_size(int T, int H, int E, int I, int k, unsigned flag
   if ((flags & ~kFp4Flags) || !flags_ok(flags) || !fp4_shape_ok(T, H, E, I, k) ||
       !forced_path_ok(E, flags))
     return 0;
-  return make_layout(T, H, E, I, k, flags, true).total + fp4_h32_bytes(T, I, k);
+  return fp4_layout(make_layout(T, H, E, I, k, flags, true).total, T, H, E, I, k).total;
 }
 
 moe_status_t moe_forward_nvfp4(const void* x, const void* w_router, const float* router_bias,
@@ -1272,14 +1309,13 @@ moe_status_t moe_forward_nvfp4(const void* x, const void* w_router, const float*
     return MOE_ERR_INVALID_ARG;
   if (!aligned16(x) || !aligned16(w_router) || !aligned16(y) || !aligned16(workspace) ||
       !aligned16(w->gate_codes) || !aligned16(w->up_codes) || !aligned16(w->down_codes) ||
-      (reinterpret_cast<uintptr_t>(w->gate_scales) & 1) ||
-      (reinterpret_cast<uintptr_t>(w->up_scales) & 1) ||
-      (reinterpret_cast<uintptr_t>(w->down_scales) & 1))
+      !aligned16(w->gate_scales) || !aligned16(w->up_scales) || !aligned16(w->down_scales))
     return MOE_ERR_INVALID_ARG;
   if (x == y) return MOE_ERR_INVALID_ARG;
   if (!fp4_shape_ok(T, H, E, I, k) || !forced_path_ok(E, flags)) return MOE_ERR_UNSUPPORTED;
   const Layout L = make_layout(T, H, E, I, k, flags, true);
-  if (workspace_bytes < L.total + fp4_h32_bytes(T, I, k)) return MOE_ERR_NO_WORKSPACE;
+  const Fp4Layout F = fp4_layout(L.total, T, H, E, I, k);
+  if (workspace_bytes < F.total) return MOE_ERR_NO_WORKSPACE;
   int dev = 0;
   DeviceState* d = device_state(&dev);
   if (!d) return MOE_ERR_CUDA;
@@ -1301,7 +1337,6 @@ moe_status_t moe_forward_nvfp4(const void* x, const void* w_router, const float*
   int32_t* tile_expert = reinterpret_cast<int32_t*>(ws + L.tile_expert);
   int32_t* tile_row0 = reinterpret_cast<int32_t*>(ws + L.tile_row0);
   int32_t* tile_rows = reinterpret_cast<int32_t*>(ws + L.tile_rows);
-  float* h32 = reinterpret_cast<float*>(ws + L.total);   // [P][I]
   __nv_bfloat16* obuf = reinterpret_cast<__nv_bfloat16*>(ws + L.obuf);
 
   Profiler prof{d, st, (flags & MOE_FLAG_PROFILE_STAGES) != 0};
@@ -1311,23 +1346,44 @@ moe_status_t moe_forward_nvfp4(const void* x, const void* w_router, const float*
                                                  ws, L, *d, st, prof, false);
       rs != MOE_OK)
     return rs;
-  // 3. GEMM-1 + GEGLU, 4. GEMM-2 (h quantised as it is staged): one CTA per (tile, group of
-  // 8 features or 64 output columns); a tile is one expert's rows (at most T <= 16), so there
-  // are at most min(E, T k) tiles
+  // 3. the routed x rows in sorted order, quantised (and the FFN's counters zeroed);
+  // 4. GEMM-1 + GEGLU + h quantised, GEMM-2: one persistent tensor-core launch
   const Launch launch{st, !prof.on};
-  const int max_tiles = std::min(E, P);
-  const bool r8 = fp4_max_rows(T) == 8;
-  launch(true, r8 ? nvfp4_gemm1_kernel<8> : nvfp4_gemm1_kernel<FP4_MAX_ROWS>,
-         dim3(max_tiles, (I + FP4_G1_FEATS - 1) / FP4_G1_FEATS), dim3(32 * FP4_G1_FEATS),
-         fp4_smem1(T, H), static_cast<const __nv_bfloat16*>(x), (const int32_t*)perm, k, T,
-         (const int32_t*)tile_num, (const int32_t*)tile_expert, (const int32_t*)tile_row0,
-         (const int32_t*)tile_rows, w->gate_codes, w->gate_scales, w->gate_ts, w->up_codes,
-         w->up_scales, w->up_ts, H, I, act_scale_x, h32);
-  launch(true, r8 ? nvfp4_gemm2_kernel<8> : nvfp4_gemm2_kernel<FP4_MAX_ROWS>,
-         dim3(max_tiles, (H + 63) / 64), dim3(256), fp4_smem2(T, I), (const float*)h32,
-         (const int32_t*)tile_num, (const int32_t*)tile_expert, (const int32_t*)tile_row0,
-         (const int32_t*)tile_rows, w->down_codes, w->down_scales, w->down_ts, H, I, act_scale_h,
-         obuf);
+  CUtensorMap tm_wg, tm_wu, tm_wd, tm_xq, tm_hq;
+  if (!make_map_u8_3d(&tm_wg, w->gate_codes, H / 2, I, E) ||
+      !make_map_u8_3d(&tm_wu, w->up_codes, H / 2, I, E) ||
+      !make_map_u8_3d(&tm_wd, w->down_codes, I / 2, H, E) ||
+      !make_map_u8_2d(&tm_xq, ws + F.xq, H / 2, P, F4_BN) ||
+      !make_map_u8_2d(&tm_hq, ws + F.hq, I / 2, P, F4_BN))
+    return cuda_failed(-1);
+  int* ctr = reinterpret_cast<int*>(ws + F.ctr);
+  const int groups = P * (H / 16);
+  launch(true, nvfp4_rows_sorted_kernel, dim3(std::min((groups + 255) / 256, d->num_sms * 4)),
+         dim3(256), 0, static_cast<const __nv_bfloat16*>(x), (const int32_t*)perm, k, T, P, H,
+         act_scale_x, ws + F.xq, ws + F.xsf, ctr, F.n_ctr);
+  Fp4Ffn fa;
+  fa.sfa_g = w->gate_scales;
+  fa.sfa_u = w->up_scales;
+  fa.sfa_d = w->down_scales;
+  fa.ts_g = w->gate_ts;
+  fa.ts_u = w->up_ts;
+  fa.ts_d = w->down_ts;
+  fa.xsf = ws + F.xsf;
+  fa.hq = ws + F.hq;
+  fa.hsf = ws + F.hsf;
+  fa.O = obuf;
+  fa.tile_num = tile_num;
+  fa.tile_expert = tile_expert;
+  fa.tile_row0 = tile_row0;
+  fa.tile_rows = tile_rows;
+  fa.next = ctr;
+  fa.h_ready = ctr + 1;
+  fa.H = H;
+  fa.I = I;
+  fa.sx = act_scale_x;
+  fa.sh = act_scale_h;
+  launch(true, nvfp4_ffn_kernel, dim3(d->num_sms), dim3(F4_THREADS), F4_SMEM, tm_wg, tm_wu, tm_wd,
+         tm_xq, tm_hq, fa);
   if (const moe_status_t ls = launched(); ls != MOE_OK) return ls;
   prof.mark();
   // 5. combine

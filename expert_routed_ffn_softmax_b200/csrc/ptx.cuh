@@ -165,6 +165,17 @@ __device__ __forceinline__ void tma_prefetch_4d(const void* desc, int c0, int c1
                : "memory");
 }
 
+// Bulk copy global -> shared (no tensor map), completing `bytes` on the mbarrier; both
+// addresses 16-byte aligned, bytes % 16 == 0.
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes,
+                                          uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          dst),
+      "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar)
+      : "memory");
+}
+
 // 16-byte copy global -> shared that bypasses L1 (cp.async, generic proxy).
 __device__ __forceinline__ void cp_async_16(uint32_t dst, const void* src) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");

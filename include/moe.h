@@ -39,7 +39,7 @@
 extern "C" {
 #endif
 
-#define MOE_ABI_VERSION 5
+#define MOE_ABI_VERSION 6
 
 typedef enum {
   MOE_OK = 0,
@@ -272,21 +272,26 @@ moe_status_t moe_combine(const void *o, const int32_t *inv, const float *topk_we
  *
  * Layout of one projection with reduction depth K and N outputs (a Linear layer's weight,
  * K contiguous): codes uint8 [E][N][K/2] (byte b of a row holds element 2b in its low nibble,
- * 2b+1 in its high nibble), scales uint8 [E][N][K/16] (E4M3 bytes), ts fp32 [E].  The layer's
- * projections: gate and up with K = H, N = I; down with K = I, N = H.
+ * 2b+1 in its high nibble); ts fp32 [E]; scales (E4M3 bytes) in a BLOCKED layout, the one the
+ * tensor cores read: E * ceil(N/128) * (K/64) blocks of 512 bytes, ordered [e][n/128][g/4]
+ * for row n and group g (= k/16); inside a block the scale of (n, g) is byte
+ *     16 * (n % 32) + 4 * ((n % 128) / 32) + (g % 4),
+ * and rows N .. ceil(N/128)*128 - 1 hold scale 0.  The layer's projections: gate and up with
+ * K = H, N = I; down with K = I, N = H.
  */
 typedef struct {
-  const uint8_t *gate_codes, *gate_scales; /* [E][I][H/2], [E][I][H/16] */
-  const float *gate_ts;                    /* [E]                       */
-  const uint8_t *up_codes, *up_scales;     /* [E][I][H/2], [E][I][H/16] */
-  const float *up_ts;                      /* [E]                       */
-  const uint8_t *down_codes, *down_scales; /* [E][H][I/2], [E][H][I/16] */
-  const float *down_ts;                    /* [E]                       */
+  const uint8_t *gate_codes, *gate_scales; /* [E][I][H/2], blocked (N = I, K = H) */
+  const float *gate_ts;                    /* [E]                                 */
+  const uint8_t *up_codes, *up_scales;     /* [E][I][H/2], blocked (N = I, K = H) */
+  const float *up_ts;                      /* [E]                                 */
+  const uint8_t *down_codes, *down_scales; /* [E][H][I/2], blocked (N = H, K = I) */
+  const float *down_ts;                    /* [E]                                 */
 } moe_nvfp4_weights_t;
 
 /* Quantise bf16 weights w [E][K][N] (N contiguous: the layout moe_forward takes, e.g. W_gate
- * with K = H, N = I) into the layout above: codes [E][N][K/2], scales [E][N][K/16], ts [E].
- * K % 32 == 0, K <= 16384.  Workspace: moe_nvfp4_quantize_workspace_size(E) bytes. */
+ * with K = H, N = I) into the layout above: codes [E][N][K/2], blocked scales
+ * (E * ceil(N/128) * K/64 * 512 bytes, 16-byte aligned), ts [E].  K % 64 == 0, K <= 16384.
+ * Workspace: moe_nvfp4_quantize_workspace_size(E) bytes. */
 size_t moe_nvfp4_quantize_workspace_size(int E);
 moe_status_t moe_nvfp4_quantize_weights(const void *w, int E, int K, int N, uint8_t *codes,
                                         uint8_t *scales, float *ts, void *workspace,
@@ -306,8 +311,9 @@ moe_status_t moe_nvfp4_quantize_rows(const void *x, int rows, int K, float ts, u
  * with the dequantised weights; products exact, sums in fp32, h quantised from fp32, o and y
  * rounded to bf16.  act_scale_x / act_scale_h: the fixed activation tensor scales (> 0).
  * flags: MOE_FLAG_NO_RENORM, MOE_FLAG_ROUTER_FP64 / _SCREEN, MOE_FLAG_PROFILE_STAGES only.
- * Limits: shapes as moe_forward, T <= 16, min(T,16) * H * 2 + 2048 and min(T,16) * I * 2 + 2048
- * bytes at most 227 KB.  Workspace: moe_nvfp4_workspace_size bytes.
+ * The expert FFN runs on the tensor cores (block-scaled NVFP4 MMAs, scales from the blocked
+ * layout).  Limits: shapes as moe_forward, T <= 16.  Codes and scales 16-byte aligned.
+ * Workspace: moe_nvfp4_workspace_size bytes.
  */
 size_t moe_nvfp4_workspace_size(int T, int H, int E, int I, int k, unsigned flags);
 moe_status_t moe_forward_nvfp4(const void *x, const void *w_router, const float *router_bias,

@@ -39,7 +39,7 @@ def test_library_exports_every_declared_symbol(lib):
 
 
 def test_abi_version_and_status_strings(lib):
-    assert lib.moe_abi_version() == 5
+    assert lib.moe_abi_version() == 6
     assert _abi.status_string(0) == "MOE_OK"
     assert _abi.status_string(5) == "MOE_ERR_TIMEOUT"
     assert _abi.status_string(99) == "MOE_ERR_UNKNOWN"

@@ -20,6 +20,22 @@ from expert_routed_ffn_softmax_b200 import workloads as wl
 pytestmark = pytest.mark.gpu
 
 
+def unblock(scales: torch.Tensor, N: int, K: int) -> np.ndarray:
+    """Blocked weight scales [E, ceil(N/128), K/64, 512] (include/moe.h) -> [E, N, K/16]; the
+    padding rows N .. must hold 0."""
+    b = scales.cpu().numpy()
+    E = b.shape[0]
+    n = np.arange(N)[:, None]
+    g = np.arange(K // 16)[None, :]
+    byte = 16 * (n % 32) + 4 * ((n % 128) // 32) + (g % 4)
+    out = b[:, n // 128, g // 4, byte]
+    pad = np.arange(N, b.shape[1] * 128)
+    if pad.size:
+        pb = 16 * (pad[:, None] % 32) + 4 * ((pad[:, None] % 128) // 32) + (g % 4)
+        assert not b[:, pad[:, None] // 128, g // 4, pb].any()
+    return out
+
+
 def unpack(codes: torch.Tensor) -> np.ndarray:
     """Packed codes [..., K/2] (element 2b in the low nibble) -> one code per byte [..., K]."""
     b = codes.cpu().numpy()
@@ -39,12 +55,18 @@ def gemma_fp4():
     return w, q_gpu, q_ref
 
 
+def check_weights(q_gpu, q_ref):
+    for n in ("gate", "up", "down"):
+        codes = unpack(q_gpu[f"{n}_codes"])
+        assert np.array_equal(codes, q_ref[f"{n}_codes"]), n
+        N, K = codes.shape[1], codes.shape[2]
+        assert np.array_equal(unblock(q_gpu[f"{n}_scales"], N, K), q_ref[f"{n}_scales"]), n
+        assert np.array_equal(q_gpu[f"{n}_ts"].cpu().numpy(), q_ref[f"{n}_ts"]), n
+
+
 def test_weight_quantizer_matches_oracle(gemma_fp4):
     _, q_gpu, q_ref = gemma_fp4
-    for n in ("gate", "up", "down"):
-        assert np.array_equal(unpack(q_gpu[f"{n}_codes"]), q_ref[f"{n}_codes"]), n
-        assert np.array_equal(q_gpu[f"{n}_scales"].cpu().numpy(), q_ref[f"{n}_scales"]), n
-        assert np.array_equal(q_gpu[f"{n}_ts"].cpu().numpy(), q_ref[f"{n}_ts"]), n
+    check_weights(q_gpu, q_ref)
 
 
 def test_weight_quantizer_tiny_shape():
@@ -52,10 +74,7 @@ def test_weight_quantizer_tiny_shape():
     w = wl.make_weights(cfg, seed=2)
     q_gpu = _abi.nvfp4_quantize_layer(w["w_gate"].cuda(), w["w_up"].cuda(), w["w_down"].cuda())
     q_ref = oracle.quantize_expert_weights(w["w_gate"], w["w_up"], w["w_down"])
-    for n in ("gate", "up", "down"):
-        assert np.array_equal(unpack(q_gpu[f"{n}_codes"]), q_ref[f"{n}_codes"]), n
-        assert np.array_equal(q_gpu[f"{n}_scales"].cpu().numpy(), q_ref[f"{n}_scales"]), n
-        assert np.array_equal(q_gpu[f"{n}_ts"].cpu().numpy(), q_ref[f"{n}_ts"]), n
+    check_weights(q_gpu, q_ref)
 
 
 @pytest.mark.parametrize("ts", [1.0, 0.0078125, 0.37])
@@ -109,6 +128,23 @@ def test_forward_nvfp4_tiny_with_bias_and_no_renorm():
         assert moe.sync_status() == 0
         ref = oracle.forward_nvfp4(x, w["w_router"], q_ref, cfg.k, bias=bias, renorm=renorm)
         check(y, aux, ref, cfg.E)
+
+
+def test_forward_nvfp4_ragged_shape():
+    """Shapes whose K stages and 128-row blocks do not divide evenly: H = 320 (GEMM-1 K in a
+    full and a one-block stage, GEMM-2 columns in blocks of 128, 128, 64), I = 192 (GEMM-1
+    features in blocks of 128 and 64, GEMM-2 K in 3 blocks)."""
+    cfg = wl.MoEConfig("ragged", 5, 320, 8, 3, 192)
+    w = wl.make_weights(cfg, seed=4)
+    q_gpu = _abi.nvfp4_quantize_layer(w["w_gate"].cuda(), w["w_up"].cuda(), w["w_down"].cuda())
+    q_ref = oracle.quantize_expert_weights(w["w_gate"], w["w_up"], w["w_down"])
+    check_weights(q_gpu, q_ref)
+    x = wl.make_x(cfg, seed=4, T=cfg.T)
+    y, aux = _abi.forward_nvfp4(x.cuda(), w["w_router"].cuda(), q_gpu, cfg.k, act_scale_h=0.5,
+                                aux=True)
+    assert moe.sync_status() == 0
+    ref = oracle.forward_nvfp4(x, w["w_router"], q_ref, cfg.k, act_scale_h=0.5)
+    check(y, aux, ref, cfg.E)
 
 
 def test_forward_nvfp4_refuses_batches_above_16(gemma_fp4):
