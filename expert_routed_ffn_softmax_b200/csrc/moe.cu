@@ -294,6 +294,19 @@ bool make_map_u8_2d(CUtensorMap* m, const void* base, uint64_t cols, uint64_t ro
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
+// Scale lines [kb][rows][16 bytes] as (16, rows, kb), box 16 bytes x 32 rows x 4 kb, no
+// swizzle: one load fills four 512-byte scale blocks.
+bool make_map_lines(CUtensorMap* m, const void* base, uint64_t rows, uint64_t kb) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {16, rows, kb};
+  cuuint64_t strides[2] = {16, 16 * rows};
+  cuuint32_t box[3] = {16, 32, 4};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
 // Stacked bytes [E][rows][cols], box = 128 bytes x 128 rows x 1 expert, 128-byte swizzle.
 bool make_map_u8_3d(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, uint64_t E) {
   auto fn = encode_fn();
@@ -1259,24 +1272,25 @@ moe_status_t moe_nvfp4_quantize_rows(const void* x, int rows, int K, float ts, u
 namespace {
 constexpr unsigned kFp4Flags = MOE_FLAG_NO_RENORM | MOE_FLAG_ROUTER_FP64 | MOE_FLAG_ROUTER_SCREEN |
                                MOE_FLAG_PROFILE_STAGES;
-// The forward's own layout, then (256-byte aligned): sorted x codes [P][H/2] and scales
-// [P][H/16], h codes [P][I/2] and scales [P][I/16], the FFN counters (unit counter, h_ready).
+// The forward's own layout, then (256-byte aligned): sorted x codes [P][H/2], x scale lines
+// [H/64][P + 16][16], h codes [P][I/2], h scale lines [I/64][P + 16][16], the FFN counters
+// (unit counter, h_ready per tile).
 struct Fp4Layout {
-  size_t xq, xsf, hq, hsf, ctr, total;
+  size_t xq, xl, hq, hl, ctr, total;
   int n_ctr;
 };
 Fp4Layout fp4_layout(size_t at, int T, int H, int E, int I, int k) {
   Fp4Layout F;
-  const size_t P = (size_t)T * k;
+  const size_t P = (size_t)T * k, Pp = P + 16;
   auto take = [&](size_t bytes) {
     const size_t o = at;
     at = align256(at + bytes);
     return o;
   };
   F.xq = take(P * H / 2);
-  F.xsf = take(P * H / 16);
+  F.xl = take((size_t)(H / 64) * Pp * 16);
   F.hq = take(P * I / 2);
-  F.hsf = take(P * I / 16);
+  F.hl = take((size_t)(I / 64) * Pp * 16);
   F.n_ctr = 1 + std::min(E, (int)P);
   F.ctr = take(sizeof(int) * F.n_ctr);
   F.total = at;
@@ -1349,18 +1363,22 @@ moe_status_t moe_forward_nvfp4(const void* x, const void* w_router, const float*
   // 3. the routed x rows in sorted order, quantised (and the FFN's counters zeroed);
   // 4. GEMM-1 + GEGLU + h quantised, GEMM-2: one persistent tensor-core launch
   const Launch launch{st, !prof.on};
-  CUtensorMap tm_wg, tm_wu, tm_wd, tm_xq, tm_hq;
+  const int Pp = P + 16;
+  CUtensorMap tm_wg, tm_wu, tm_wd, tm_xq, tm_hq, tm_xl, tm_hl;
   if (!make_map_u8_3d(&tm_wg, w->gate_codes, H / 2, I, E) ||
       !make_map_u8_3d(&tm_wu, w->up_codes, H / 2, I, E) ||
       !make_map_u8_3d(&tm_wd, w->down_codes, I / 2, H, E) ||
       !make_map_u8_2d(&tm_xq, ws + F.xq, H / 2, P, F4_BN) ||
-      !make_map_u8_2d(&tm_hq, ws + F.hq, I / 2, P, F4_BN))
+      !make_map_u8_2d(&tm_hq, ws + F.hq, I / 2, P, F4_BN) ||
+      !make_map_lines(&tm_xl, ws + F.xl, Pp, H / 64) ||
+      !make_map_lines(&tm_hl, ws + F.hl, Pp, I / 64))
     return cuda_failed(-1);
   int* ctr = reinterpret_cast<int*>(ws + F.ctr);
-  const int groups = P * (H / 16);
-  launch(true, nvfp4_rows_sorted_kernel, dim3(std::min((groups + 255) / 256, d->num_sms * 4)),
-         dim3(256), 0, static_cast<const __nv_bfloat16*>(x), (const int32_t*)perm, k, T, P, H,
-         act_scale_x, ws + F.xq, ws + F.xsf, ctr, F.n_ctr);
+  const int items = Pp * (H / 64);
+  launch(true, nvfp4_rows_sorted_kernel, dim3(std::min((items + 127) / 128, d->num_sms * 4)),
+         dim3(128), 0, static_cast<const __nv_bfloat16*>(x), (const int32_t*)perm, k, T, P, H,
+         act_scale_x, ws + F.xq, reinterpret_cast<uint4*>(ws + F.xl),
+         reinterpret_cast<uint4*>(ws + F.hl), (I / 64) * Pp, ctr, F.n_ctr);
   Fp4Ffn fa;
   fa.sfa_g = w->gate_scales;
   fa.sfa_u = w->up_scales;
@@ -1368,9 +1386,10 @@ moe_status_t moe_forward_nvfp4(const void* x, const void* w_router, const float*
   fa.ts_g = w->gate_ts;
   fa.ts_u = w->up_ts;
   fa.ts_d = w->down_ts;
-  fa.xsf = ws + F.xsf;
+  fa.x_lines = ws + F.xl;
   fa.hq = ws + F.hq;
-  fa.hsf = ws + F.hsf;
+  fa.h_lines = ws + F.hl;
+  fa.Pp = Pp;
   fa.O = obuf;
   fa.tile_num = tile_num;
   fa.tile_expert = tile_expert;
@@ -1380,10 +1399,11 @@ moe_status_t moe_forward_nvfp4(const void* x, const void* w_router, const float*
   fa.h_ready = ctr + 1;
   fa.H = H;
   fa.I = I;
+  fa.E = E;
   fa.sx = act_scale_x;
   fa.sh = act_scale_h;
   launch(true, nvfp4_ffn_kernel, dim3(d->num_sms), dim3(F4_THREADS), F4_SMEM, tm_wg, tm_wu, tm_wd,
-         tm_xq, tm_hq, fa);
+         tm_xq, tm_hq, tm_xl, tm_hl, fa);
   if (const moe_status_t ls = launched(); ls != MOE_OK) return ls;
   prof.mark();
   // 5. combine

@@ -170,43 +170,53 @@ __global__ void __launch_bounds__(256) nvfp4_rows_quant_kernel(
 
 // ---------------------------------------------------------------- activations, sorted
 // The expert FFN's activation operand: the routed rows in expert-sorted order (row j holds
-// the token of pair perm[j]) quantised with tensor scale ts -> codes [P][K/2], compact scales
-// [P][K/16].  Also zeroes the FFN's counters (n_ctr ints).  One thread per group of 16.
+// the token of pair perm[j]) quantised with tensor scale ts -> codes [P][K/2] and scale LINES:
+// lines [K/64][Pp][16 bytes], line (kb, j) = the 4 scales of row j's groups 4 kb .. 4 kb + 3,
+// then 12 zero bytes (the rows 0-15 of a tensor-core scale block, so that 16 consecutive rows
+// of one K block are one 256-byte copy).  Pp = P + 16: rows P .. P + 15 are zero lines.
+// Also zeroes h_lines ([I/64][Pp][16], filled in later by the FFN's GEMM-1 epilogue) and the
+// FFN's counters.  One thread per (row, 64-element K block).
 __global__ void __launch_bounds__(256) nvfp4_rows_sorted_kernel(
     const __nv_bfloat16* __restrict__ x, const int32_t* __restrict__ perm, int k, int T, int P,
-    int K, float ts, uint8_t* __restrict__ codes, uint8_t* __restrict__ scales,
-    int* __restrict__ counters, int n_ctr) {
+    int K, float ts, uint8_t* __restrict__ codes, uint4* __restrict__ lines,
+    uint4* __restrict__ h_lines, int n_h_lines, int* __restrict__ counters, int n_ctr) {
   pdl_trigger();
   pdl_wait();
+  const int tid = blockIdx.x * blockDim.x + threadIdx.x, nth = gridDim.x * blockDim.x;
   if (blockIdx.x == 0)
     for (int i = threadIdx.x; i < n_ctr; i += blockDim.x) counters[i] = 0;
-  const int ng = K / 16;
-  for (int gi = blockIdx.x * blockDim.x + threadIdx.x; gi < P * ng; gi += gridDim.x * blockDim.x) {
-    const int j = gi / ng, g = gi - j * ng;
-    const int q = perm[j];
-    float v[16];
-    if ((unsigned)q >= (unsigned)(T * k)) {
-      raise_error(MOE_DEVERR_BAD_INDEX);
+  for (int i = tid; i < n_h_lines; i += nth) h_lines[i] = make_uint4(0, 0, 0, 0);
+  const int nkb = K / 64, Pp = P + 16;
+  for (int gi = tid; gi < Pp * nkb; gi += nth) {
+    const int j = gi / nkb, kb = gi - j * nkb;
+    uint32_t sc4 = 0;
+    if (j < P) {
+      const int q = perm[j];
+      const bool ok = (unsigned)q < (unsigned)(T * k);
+      if (!ok) raise_error(MOE_DEVERR_BAD_INDEX);
+      const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)(ok ? q / k : 0) * K + 64 * kb);
 #pragma unroll
-      for (int i = 0; i < 16; ++i) v[i] = 0.f;
-    } else {
-      const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)(q / k) * K + 16 * g);
+      for (int g = 0; g < 4; ++g) {
+        float v[16];
 #pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {
-        const uint4 r = __ldg(src + hh);
-        const __nv_bfloat162* pr = reinterpret_cast<const __nv_bfloat162*>(&r);
+        for (int hh = 0; hh < 2; ++hh) {
+          const uint4 r = ok ? __ldg(src + 2 * g + hh) : make_uint4(0, 0, 0, 0);
+          const __nv_bfloat162* pr = reinterpret_cast<const __nv_bfloat162*>(&r);
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const float2 f = __bfloat1622float2(pr[i]);
-          v[8 * hh + 2 * i] = f.x;
-          v[8 * hh + 2 * i + 1] = f.y;
+          for (int i = 0; i < 4; ++i) {
+            const float2 f = __bfloat1622float2(pr[i]);
+            v[8 * hh + 2 * i] = f.x;
+            v[8 * hh + 2 * i + 1] = f.y;
+          }
         }
+        uint32_t c[2], sc, dq[8];
+        nvfp4_quantize16(v, ts, c, sc, dq);
+        *reinterpret_cast<uint2*>(codes + (size_t)j * (K / 2) + 32 * kb + 8 * g) =
+            make_uint2(c[0], c[1]);
+        sc4 |= sc << (8 * g);
       }
     }
-    uint32_t c[2], sc, dq[8];
-    nvfp4_quantize16(v, ts, c, sc, dq);
-    *reinterpret_cast<uint2*>(codes + (size_t)j * (K / 2) + 8 * g) = make_uint2(c[0], c[1]);
-    scales[(size_t)j * ng + g] = static_cast<uint8_t>(sc);
+    lines[(size_t)kb * Pp + j] = make_uint4(sc4, 0, 0, 0);
   }
 }
 
