@@ -148,7 +148,7 @@ def ffn_kernel_name(T: int, tiles: str) -> str:
 def kernel_source_sha() -> str:
     h = hashlib.sha256()
     for f in ("grouped_gemm.cuh", "gemm_persistent.cuh", "ffn_dynamic.cuh", "ffn_pair.cuh",
-              "gemm_decode.cuh", "ptx.cuh"):
+              "gemm_decode.cuh", "ptx.cuh", "nvfp4.cuh", "nvfp4_mma.cuh"):
         h.update(open(os.path.join(ROOT, "expert_routed_ffn_softmax_b200", "csrc", f), "rb").read())
     return h.hexdigest()[:16]
 
@@ -361,7 +361,8 @@ def nvfp4_entry(cfg, m: dict, world: int, pk: dict) -> dict:
         "value": job_throughput(world, cfg.T, m["ms"]), "unit": UNIT, "ms_per_step": m["ms"],
         "expert_ffn": {"kernels": "nvfp4_rows_sorted_kernel + nvfp4_ffn_kernel (tcgen05 kind::mxf4nvf4)", "ms": m["ffn_ms"],
                        "algorithmic_bytes": ffn_bytes, "achieved_gbs": ach,
-                       "frac_of_hbm": None if ach is None else ach / pk["hbm_gbs"]},
+                       "frac_of_hbm": None if ach is None else ach / pk["hbm_gbs"],
+                       "traffic": ncu_traffic("nvfp4_ffn_kernel", f"{cfg.name}_nvfp4")},
         "step_hbm_frac": step_bytes / (m["ms"] * 1e-3) / (pk["hbm_gbs"] * 1e9),
         "active_experts": m["active"], "stages_ms": m["stages"], "clocks": m["clocks"],
         "gpu_launches": m["kernels"] * m["_steps"],
