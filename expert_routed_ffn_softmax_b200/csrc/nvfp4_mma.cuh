@@ -19,8 +19,8 @@
 // features (16 TMEM lanes) and publishes h_ready[tile]; a GEMM-2 unit waits for its tile's
 // count before it loads h.  A GEMM-2 epilogue writes the expert output rows in bf16.
 //
-// Roles: warp 0 producer (lane 0), warp 1 MMA issuer, warps 2-5 epilogue.  Every wait is
-// bounded.
+// Roles: warp 0 weight producer, warp 6 activation producer, warp 1 MMA issuer, warps 2-5
+// epilogue.  Every wait is bounded.
 #pragma once
 #include <cuda.h>
 #include "ptx.cuh"
@@ -30,7 +30,7 @@
 
 namespace moe {
 
-constexpr int F4_THREADS = 192;
+constexpr int F4_THREADS = 224;
 constexpr int F4_STAGES = 5;
 constexpr int F4_BN = 16;                        // token columns = max rows of a tile
 constexpr int F4_KS = 256;                       // K elements per stage (128 bytes per row)
@@ -236,7 +236,7 @@ __global__ void __launch_bounds__(F4_THREADS, 1)
   float4* ts_tab = reinterpret_cast<float4*>(tile_tab + F4_MAX_TILES);          // g, u, d scales
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  constexpr int kDescReaders = 1 + 4;   // MMA warp, 4 epilogue warps
+  constexpr int kDescReaders = 1 + 4 + 1;   // MMA warp, 4 epilogue warps, activation warp
   if (tid == 0) {
     for (int s = 0; s < F4_STAGES; ++s) {
       mbar_init(full_bar(s), 1);
@@ -307,10 +307,11 @@ __global__ void __launch_bounds__(F4_THREADS, 1)
     return ring[r];
   };
   if (warp == 0) {
-    // -------------------------------------------------------------- producer (warp 0)
+    // -------------------------------------------------------------- weight producer (warp 0)
     // Warp-uniform loop as in the MMA warp: lane 0 waits and claims units, the elected lane
-    // issues the copies (predicated).  The next unit is claimed when a unit starts and read when it ends,
-    // so the claim's round trip overlaps the unit's issue.
+    // issues the copies (predicated).  The next unit is claimed when a unit starts and read
+    // when it ends, so the claim's round trip overlaps the unit's issue.  The weights never
+    // wait for h: a GEMM-2 unit's W_down streams while warp 6 waits for the tile's h.
     int q = 0;
     int c = 0;
     if (lane == 0) c = atomicAdd(a.next, 1);
@@ -332,8 +333,7 @@ __global__ void __launch_bounds__(F4_THREADS, 1)
       }
       if (__shfl_sync(0xffffffffu, stop ? 1 : 0, 0)) break;
       const F4Unit u = f4_decode(c, U1, nb1, nb2);
-      const int4 tt = tile_tab[u.tile];
-      const int e = tt.x, row0 = tt.y;
+      const int e = tile_tab[u.tile].x;
       const bool g1 = u.phase == 0;
       const int kbt = g1 ? kb1 : kb2, nk = (kbt + 3) / 4;
       // the unit's two A operands: rows (row block rA of matrix 0) and (rB of matrix 1)
@@ -343,7 +343,8 @@ __global__ void __launch_bounds__(F4_THREADS, 1)
       const uint8_t* sfa1 = g1 ? a.sfa_u : a.sfa_d;
       const size_t blkA = ((size_t)e * (g1 ? nb1 : nbh) + rA) * kbt;   // first scale blocks
       const size_t blkB = ((size_t)e * (g1 ? nb1 : nbh) + rB) * kbt;
-      // Stage kc: the weights (A + scales) and/or the activations (B + scale lines).
+      // Stage kc's weights (A + scales); the stage's byte count includes the activations,
+      // which warp 6 loads into the same stage.
       auto weights_in = [&](int kc, int qq) -> bool {
         const int s = qq % F4_STAGES;
         int okw = !*abort_flag;
@@ -366,43 +367,8 @@ __global__ void __launch_bounds__(F4_THREADS, 1)
         __syncwarp();
         return true;
       };
-      auto acts_in = [&](int kc, int qq) {
-        const uint32_t sA = base + (qq % F4_STAGES) * F4_STAGE;
-        const uint32_t lead = elect_lane();
-        const uint32_t bar = full_bar(qq % F4_STAGES);
-        tma_load_2d_p(lead, sA + F4_OFF_B, g1 ? &tmXq : &tmHq, bar, kc * 128, row0);
-        tma_load_3d_p(lead, sA + F4_OFF_SFB, g1 ? &tmXl : &tmHl, bar, 0, row0, 4 * kc);
-        __syncwarp();
-      };
       bool okp = true;
-      int kc = 0;
-      if (!g1) {
-        // GEMM-2 needs this tile's h (GEMM-1 units of any CTA); its weights do not: load
-        // them for the first stages, then (h complete) load h for those stages
-        const int pre = min(nk, F4_STAGES);
-        for (int t2 = 0; t2 < pre && okp; ++t2) okp = weights_in(t2, q + t2);
-        if (okp) {
-          int okh = 1;
-          if (lane == 0) okh = wait_counter_geq(a.h_ready + u.tile, h_target);
-          // every lane (whichever issues the loads) acquires the count, then orders its
-          // async-proxy reads of h after it
-          okh = __shfl_sync(0xffffffffu, okh, 0);
-          (void)ld_acquire_gpu(a.h_ready + u.tile);
-          fence_proxy_async_global();
-          if (!okh) {
-            *abort_flag = 1;
-            okp = false;
-          } else {
-            for (int t2 = 0; t2 < pre; ++t2) acts_in(t2, q + t2);
-          }
-        }
-        kc = pre;
-        q += pre;
-      }
-      for (; okp && kc < nk; ++kc, ++q) {
-        okp = weights_in(kc, q);
-        if (okp) acts_in(kc, q);
-      }
+      for (int kc = 0; okp && kc < nk; ++kc, ++q) okp = weights_in(kc, q);
       if (!okp) break;
       c = __shfl_sync(0xffffffffu, cnext, 0);
     }
@@ -513,6 +479,62 @@ __global__ void __launch_bounds__(F4_THREADS, 1)
     umma_commit_p(elect_lane(), done_bar);
     if (lane == 0 && !mbar_wait_ns(done_bar, 0, kDrainLimitNs)) *abort_flag = 1;
     __syncwarp();
+  } else if (warp == 6) {
+    // -------------------------------------------------------------- activation producer
+    // The same units and stages as warp 0: per stage, the tile's 16 activation rows (x's
+    // codes for GEMM-1, h's for GEMM-2) and their scale lines, into the stage warp 0 filled
+    // or is filling (the stage's byte count, set by warp 0, covers both).  A GEMM-2 unit
+    // first waits until every GEMM-1 epilogue warp of its tile has published h.
+    int q = 0;
+    for (int i = 0;; ++i) {
+      int c = 0;
+      if (lane == 0) {
+        c = read_desc(i);
+        mbar_arrive(dempty_bar(i % F4_RING));
+      }
+      c = __shfl_sync(0xffffffffu, c, 0);
+      if (c < 0) {
+        if (c == -2) *abort_flag = 1;
+        break;
+      }
+      const F4Unit u = f4_decode(c, U1, nb1, nb2);
+      const int row0 = tile_tab[u.tile].y;
+      const bool g1 = u.phase == 0;
+      const int kbt = g1 ? kb1 : kb2, nk = (kbt + 3) / 4;
+      if (!g1) {
+        int okh = 1;
+        if (lane == 0) okh = wait_counter_geq(a.h_ready + u.tile, h_target);
+        // every lane (whichever issues the loads) acquires the count, then orders its
+        // async-proxy reads of h after it
+        okh = __shfl_sync(0xffffffffu, okh, 0);
+        (void)ld_acquire_gpu(a.h_ready + u.tile);
+        fence_proxy_async_global();
+        if (!okh) {
+          *abort_flag = 1;
+          break;
+        }
+      }
+      bool ok = true;
+      for (int kc = 0; kc < nk; ++kc, ++q) {
+        const int s = q % F4_STAGES;
+        int okw = !*abort_flag;
+        if (lane == 0 && okw && q >= F4_STAGES)
+          okw = mbar_wait(empty_bar(s), ((q / F4_STAGES) - 1) & 1);
+        if (!__shfl_sync(0xffffffffu, okw, 0)) {
+          ok = false;
+          break;
+        }
+        const uint32_t sA = base + s * F4_STAGE;
+        const uint32_t lead = elect_lane();
+        tma_load_2d_p(lead, sA + F4_OFF_B, g1 ? &tmXq : &tmHq, full_bar(s), kc * 128, row0);
+        tma_load_3d_p(lead, sA + F4_OFF_SFB, g1 ? &tmXl : &tmHl, full_bar(s), 0, row0, 4 * kc);
+        __syncwarp();
+      }
+      if (!ok) {
+        *abort_flag = 1;
+        break;
+      }
+    }
   } else {
     // -------------------------------------------------------------- epilogue (warps 2-5)
     const int quad = warp & 3;
