@@ -145,10 +145,18 @@ def ffn_kernel_name(T: int, tiles: str) -> str:
     return _abi.ffn_kernel_name(T, tiles)
 
 
-def kernel_source_sha() -> str:
+# The sources each expert-FFN kernel is built from (a capture stays valid while they do).
+KERNEL_SOURCES = {
+    "bf16": ("grouped_gemm.cuh", "gemm_persistent.cuh", "ffn_dynamic.cuh", "ffn_pair.cuh",
+             "gemm_decode.cuh", "ptx.cuh"),
+    "nvfp4": ("grouped_gemm.cuh", "gemm_persistent.cuh", "gemm_decode.cuh", "ptx.cuh",
+              "nvfp4.cuh", "nvfp4_mma.cuh"),
+}
+
+
+def kernel_source_sha(family: str = "bf16") -> str:
     h = hashlib.sha256()
-    for f in ("grouped_gemm.cuh", "gemm_persistent.cuh", "ffn_dynamic.cuh", "ffn_pair.cuh",
-              "gemm_decode.cuh", "ptx.cuh", "nvfp4.cuh", "nvfp4_mma.cuh"):
+    for f in KERNEL_SOURCES[family]:
         h.update(open(os.path.join(ROOT, "expert_routed_ffn_softmax_b200", "csrc", f), "rb").read())
     return h.hexdigest()[:16]
 
@@ -162,7 +170,7 @@ def ncu_traffic(kernel: str, workload: str) -> float | None:
         rows = json.load(open(p))
     except ValueError:
         return None
-    sha = kernel_source_sha()
+    sha = kernel_source_sha("nvfp4" if kernel.startswith("nvfp4") else "bf16")
     for r in rows:
         if r.get("kernel") == kernel and r.get("workload") == workload and r.get("source_sha") == sha:
             return float(r["dram_bytes_per_launch"])
