@@ -11,8 +11,8 @@
 // A GEMM-1 unit then publishes h_ready[tile]; a GEMM-2 unit issues its W_down loads for
 // the first stages, waits for h_ready, then loads its h rows.
 //
-// Roles as in gemm_persistent.cuh (TMA thread, MMA thread, 4 epilogue warps, 2 gather
-// warps), with A slots of R = 8 ... 128 rows (every tile has at most R rows).  The TMA
+// Roles as in gemm_persistent.cuh (TMA thread, MMA thread, 4 epilogue warps, gather warps:
+// 4 for 128-row slots, 2 otherwise), with A slots of R = 8 ... 128 rows (every tile has at most R rows).  The TMA
 // thread takes unit ids and passes them to the other roles through a ring of descriptors
 // in shared memory (full / empty mbarriers).  A tile list from the dispatch describes the
 // routed rows (expert, first sorted row, rows; the A rows gathered from x through perm);
@@ -48,6 +48,17 @@ __host__ __device__ inline int dy_smem_bytes() {
   return DyShape<R>::SMEM;
 }
 
+// Gather warps: four for 128-row slots (large batches, where GEMM-1 waits on its gathered
+// rows), two otherwise.  The kernel's threads: TMA, MMA, 4 epilogue warps, the gather warps.
+template <int R>
+__host__ __device__ constexpr int dy_gather_warps() {
+  return R == 128 ? 4 : 2;
+}
+template <int R>
+__host__ __device__ constexpr int dy_threads() {
+  return PG_THREADS + 32 * dy_gather_warps<R>();
+}
+
 // A unit: phase 0 = GEMM-1, 1 = GEMM-2; unit index within its GEMM; k-steps [kb, ke).
 struct DyChunk {
   int phase, unit, kb, ke;
@@ -73,7 +84,7 @@ __device__ __forceinline__ bool dy_narrow_block(const DyChunk& d, const PGemm& g
 // boxes (the narrow last GEMM-1 block).  tmX: GEMM-1's A rows when tiles.a_tma (box R rows x
 // 64 columns of a contiguous row-major tensor), else unused.
 template <int R>
-__global__ void __launch_bounds__(PG_MAX_THREADS, 1)
+__global__ void __launch_bounds__(PG_THREADS + 128, 1)
     expert_ffn_dynamic_kernel(const __grid_constant__ CUtensorMap tmWg,
                               const __grid_constant__ CUtensorMap tmWu,
                               const __grid_constant__ CUtensorMap tmWg1,
@@ -111,10 +122,11 @@ __global__ void __launch_bounds__(PG_MAX_THREADS, 1)
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   // arrivals that release a descriptor: MMA thread, 4 epilogue warps, 2 gather warps
-  constexpr int kDescReaders = 1 + 4 + PG_GATHER_THREADS / 32;
+  constexpr int NGW = dy_gather_warps<R>(), GATHER_THREADS = 32 * NGW;
+  constexpr int kDescReaders = 1 + 4 + NGW;
   if (tid == 0) {
     for (int s = 0; s < DY_STAGES; ++s) {
-      mbar_init(full_bar(s), 1 + PG_GATHER_THREADS);
+      mbar_init(full_bar(s), 1 + GATHER_THREADS);
       mbar_init(empty_bar(s), 1);
     }
     for (int b = 0; b < 2; ++b) {
@@ -202,7 +214,7 @@ __global__ void __launch_bounds__(PG_MAX_THREADS, 1)
             const uint32_t b_bytes = (narrow ? 2 : NSLAB) * GM_SLAB_BYTES;
             if (tiles.a_tma) {
               mbar_arrive_expect_tx(full_bar(s), b_bytes + A_BYTES);
-              mbar_arrive_cnt(full_bar(s), PG_GATHER_THREADS);   // in place of the gather warps
+              mbar_arrive_cnt(full_bar(s), GATHER_THREADS);   // in place of the gather warps
               tma_load_2d(sA, &tmX, full_bar(s), kc * GM_BK, row0);
             } else {
               mbar_arrive_expect_tx(full_bar(s), b_bytes);
@@ -217,7 +229,7 @@ __global__ void __launch_bounds__(PG_MAX_THREADS, 1)
             }
           } else {
             mbar_arrive_expect_tx(full_bar(s), A_BYTES + NSLAB * GM_SLAB_BYTES);
-            mbar_arrive_cnt(full_bar(s), PG_GATHER_THREADS);   // in place of the gather warps
+            mbar_arrive_cnt(full_bar(s), GATHER_THREADS);   // in place of the gather warps
             tma_load_4d(sB, &tmWd, full_bar(s), 0, kc * GM_BK, n0 / 64, e);
             if (with_a) tma_load_2d(sA, &tmH, full_bar(s), kc * GM_BK, row0);
           }
@@ -373,7 +385,7 @@ __global__ void __launch_bounds__(PG_MAX_THREADS, 1)
       }
     }
   } else {
-    // -------------------------------------------------------------- A-row gather (warps 6-7)
+    // -------------------------------------------------------------- A-row gather (warps 6..)
     // GEMM-1 units: the <= R rows of the tile, 16-byte cp.async into the 128-byte-swizzled
     // slot (chunk c of row r at byte 128 r + 16 (c ^ r)).  GEMM-2 units, and GEMM-1 units
     // whose A rows come by TMA: nothing (the TMA thread arrives in their place), but the
@@ -401,13 +413,13 @@ __global__ void __launch_bounds__(PG_MAX_THREADS, 1)
         raise_error(MOE_DEVERR_BAD_INDEX);
         rows = R;
       }
-      // warp 6 copies rows 0 .. R/2-1, warp 7 rows R/2 .. R-1, four rows per instruction
-      constexpr int NI = R / 8;
+      // gather warp gw copies rows gw R/NGW .. (gw + 1) R/NGW - 1, four rows per instruction
+      constexpr int NI = R / (4 * NGW);
       const __nv_bfloat16* src[NI];
       uint32_t doff[NI];
 #pragma unroll
       for (int u = 0; u < NI; ++u) {
-        const int r = gw * (R / 2) + 4 * u + sub;
+        const int r = gw * (R / NGW) + 4 * u + sub;
         src[u] = nullptr;
         if (r < rows) {
           // the routed pair's token, or (no permutation: one dense layer) the row itself

@@ -838,9 +838,9 @@ moe_status_t moe_forward(const void* x, const void* w_router, const float* route
         return cuda_failed(-1);
       int32_t* dctr = gemm_counters + L.dy_ctr;
       const DyState dys{dctr};
-      auto go = [&](auto kernel, int smem) {
-        launch(true, kernel, dim3(G), dim3(pgemm_threads(true)), smem, tm_wg, tm_wu, tm_wg1,
-               tm_wu1, tm_xr, tm_hr, tm_wd, tl, g1, g2, h_ready, dys);
+      auto go = [&](auto kernel, int smem, int threads) {
+        launch(true, kernel, dim3(G), dim3(threads), smem, tm_wg, tm_wu, tm_wg1, tm_wu1, tm_xr,
+               tm_hr, tm_wd, tl, g1, g2, h_ready, dys);
       };
       if (L.bm == PR_ROWS) {
         // CTA pairs (2-CTA clusters, an even grid): 2-slab W_down boxes, each CTA loading
@@ -850,11 +850,11 @@ moe_status_t moe_forward(const void* x, const void* w_router, const float* route
         launch(true, expert_ffn_pair_kernel, dim3(std::max(2, G & ~1)), dim3(pgemm_threads(true)),
                PR_SMEM, tm_wg, tm_wu, tm_wg1, tm_wu1, tm_xr, tm_hr, tm_wd2, tl, g1, g2, h_ready,
                dys);
-      } else if (R == 8) go(expert_ffn_dynamic_kernel<8>, dy_smem_bytes<8>());
-      else if (R == 16) go(expert_ffn_dynamic_kernel<16>, dy_smem_bytes<16>());
-      else if (R == 32) go(expert_ffn_dynamic_kernel<32>, dy_smem_bytes<32>());
-      else if (R == 64) go(expert_ffn_dynamic_kernel<64>, dy_smem_bytes<64>());
-      else go(expert_ffn_dynamic_kernel<128>, dy_smem_bytes<128>());
+      } else if (R == 8) go(expert_ffn_dynamic_kernel<8>, dy_smem_bytes<8>(), dy_threads<8>());
+      else if (R == 16) go(expert_ffn_dynamic_kernel<16>, dy_smem_bytes<16>(), dy_threads<16>());
+      else if (R == 32) go(expert_ffn_dynamic_kernel<32>, dy_smem_bytes<32>(), dy_threads<32>());
+      else if (R == 64) go(expert_ffn_dynamic_kernel<64>, dy_smem_bytes<64>(), dy_threads<64>());
+      else go(expert_ffn_dynamic_kernel<128>, dy_smem_bytes<128>(), dy_threads<128>());
     } else if (flags & MOE_FLAG_UNFUSED_FFN) {
       // static stream-K schedule, GEMM-1 (+GEGLU) and GEMM-2 as two launches
       launch(true, GEMM_GEGLU, dim3(G), dim3(pgemm_threads(true)), smem, tm_xp, tm_wg, tm_wu,
@@ -961,9 +961,9 @@ moe_status_t moe_dense_ffn(const void* x, const void* w_gate, const void* w_up,
   const DyState dys{ctr};
   const int G = std::min(std::max(1, d->num_sms), kMaxGemmCtas);
   const Launch launch{st, false};
-  auto go = [&](auto kernel, int smem) {
-    launch(false, kernel, dim3(G), dim3(pgemm_threads(true)), smem, tm_wg, tm_wu, tm_wg1, tm_wu1,
-           tm_xr, tm_hr, tm_wd, tl, g1, g2, h_ready, dys);
+  auto go = [&](auto kernel, int smem, int threads) {
+    launch(false, kernel, dim3(G), dim3(threads), smem, tm_wg, tm_wu, tm_wg1, tm_wu1, tm_xr,
+           tm_hr, tm_wd, tl, g1, g2, h_ready, dys);
   };
   if (dy_rows(T, 0) == 128 && T >= kDensePairMinTokens) {
     // CTA pairs over 256-row tiles of x (the counters above cover ceil(T / 128) tiles)
@@ -971,11 +971,11 @@ moe_status_t moe_dense_ffn(const void* x, const void* w_gate, const void* w_up,
     if (!make_map_slabs(&tm_wd2, w_down, H, I, 1, 64, 2)) return cuda_failed(-1);
     launch(false, expert_ffn_pair_kernel, dim3(std::max(2, G & ~1)), dim3(pgemm_threads(true)),
            PR_SMEM, tm_wg, tm_wu, tm_wg1, tm_wu1, tm_xr, tm_hr, tm_wd2, tl, g1, g2, h_ready, dys);
-  } else if (R == 8) go(expert_ffn_dynamic_kernel<8>, dy_smem_bytes<8>());
-  else if (R == 16) go(expert_ffn_dynamic_kernel<16>, dy_smem_bytes<16>());
-  else if (R == 32) go(expert_ffn_dynamic_kernel<32>, dy_smem_bytes<32>());
-  else if (R == 64) go(expert_ffn_dynamic_kernel<64>, dy_smem_bytes<64>());
-  else go(expert_ffn_dynamic_kernel<128>, dy_smem_bytes<128>());
+  } else if (R == 8) go(expert_ffn_dynamic_kernel<8>, dy_smem_bytes<8>(), dy_threads<8>());
+  else if (R == 16) go(expert_ffn_dynamic_kernel<16>, dy_smem_bytes<16>(), dy_threads<16>());
+  else if (R == 32) go(expert_ffn_dynamic_kernel<32>, dy_smem_bytes<32>(), dy_threads<32>());
+  else if (R == 64) go(expert_ffn_dynamic_kernel<64>, dy_smem_bytes<64>(), dy_threads<64>());
+  else go(expert_ffn_dynamic_kernel<128>, dy_smem_bytes<128>(), dy_threads<128>());
   return launched();
 }
 
@@ -1178,18 +1178,18 @@ moe_status_t moe_expert_ffn(const void* xs, int N, const int32_t* seg_rows,
   int32_t* h_ready = ctr + 1;
   const DyState dys{ctr};
   const int G = std::min(std::max(1, d->num_sms), kMaxGemmCtas);
-  auto go = [&](auto kernel, int smem) {
-    launch(true, kernel, dim3(G), dim3(pgemm_threads(true)), smem, tm_wg, tm_wu, tm_wg1, tm_wu1,
-           tm_xr, tm_hr, tm_wd, tl, g1, g2, h_ready, dys);
+  auto go = [&](auto kernel, int smem, int threads) {
+    launch(true, kernel, dim3(G), dim3(threads), smem, tm_wg, tm_wu, tm_wg1, tm_wu1, tm_xr, tm_hr,
+           tm_wd, tl, g1, g2, h_ready, dys);
   };
   if (L.bm == PR_ROWS)
     launch(true, expert_ffn_pair_kernel, dim3(std::max(2, G & ~1)), dim3(pgemm_threads(true)),
            PR_SMEM, tm_wg, tm_wu, tm_wg1, tm_wu1, tm_xr, tm_hr, tm_wd, tl, g1, g2, h_ready, dys);
-  else if (R == 8) go(expert_ffn_dynamic_kernel<8>, dy_smem_bytes<8>());
-  else if (R == 16) go(expert_ffn_dynamic_kernel<16>, dy_smem_bytes<16>());
-  else if (R == 32) go(expert_ffn_dynamic_kernel<32>, dy_smem_bytes<32>());
-  else if (R == 64) go(expert_ffn_dynamic_kernel<64>, dy_smem_bytes<64>());
-  else go(expert_ffn_dynamic_kernel<128>, dy_smem_bytes<128>());
+  else if (R == 8) go(expert_ffn_dynamic_kernel<8>, dy_smem_bytes<8>(), dy_threads<8>());
+  else if (R == 16) go(expert_ffn_dynamic_kernel<16>, dy_smem_bytes<16>(), dy_threads<16>());
+  else if (R == 32) go(expert_ffn_dynamic_kernel<32>, dy_smem_bytes<32>(), dy_threads<32>());
+  else if (R == 64) go(expert_ffn_dynamic_kernel<64>, dy_smem_bytes<64>(), dy_threads<64>());
+  else go(expert_ffn_dynamic_kernel<128>, dy_smem_bytes<128>(), dy_threads<128>());
   return launched();
 }
 
