@@ -1,5 +1,5 @@
-// nvfp4.cuh -- the expert FFN with NVFP4 weights and activations (4-bit E2M1 elements, one
-// E4M3 scale per 16 consecutive elements along the reduction axis, one fp32 scale per tensor):
+// nvfp4.cuh -- NVFP4 quantisation (4-bit E2M1 elements, one E4M3 scale per 16 consecutive
+// elements along the reduction axis, one fp32 scale per tensor):
 // the checkpoint format of Gemma-4-26B-A4B-NVFP4 ("4-bit float, group_size=16" for weights
 // and activations, Gemma-4-26B-A4B-NVFP4 Ascend verification report §2.3 量化配置 (NVFP4)).
 //
@@ -48,18 +48,6 @@ __device__ __forceinline__ uint32_t e2m1x2_to_f16x2(uint32_t byte) {
   asm("{.reg .b8 t;\n\tcvt.u8.u32 t, %1;\n\tcvt.rn.f16x2.e2m1x2 %0, t;\n\t}" : "=r"(d) : "r"(byte));
   return d;
 }
-// acc + a.lo * b.lo + a.hi * b.hi, each product exact, two fp32 roundings.
-__device__ __forceinline__ float fma2_f16_f32(uint32_t a, uint32_t b, float acc) {
-  float d;
-  asm("{.reg .f16 al, ah, bl, bh;\n\t"
-      "mov.b32 {al, ah}, %1;\n\tmov.b32 {bl, bh}, %2;\n\t"
-      "fma.rn.f32.f16 %0, al, bl, %3;\n\t"
-      "fma.rn.f32.f16 %0, ah, bh, %0;\n\t}"
-      : "=f"(d)
-      : "r"(a), "r"(b), "f"(acc));
-  return d;
-}
-
 // Quantise one group of 16 fp32 values: packed codes (8 bytes), the scale byte, and the
 // group's values code * e4m3(scale) as 8 f16x2 words (exact; the tensor scale left out).
 __device__ __forceinline__ void nvfp4_quantize16(const float (&v)[16], float ts, uint32_t (&codes)[2],

@@ -33,7 +33,6 @@ namespace moe {
 constexpr int F4_THREADS = 224;
 constexpr int F4_STAGES = 5;
 constexpr int F4_BN = 16;                        // token columns = max rows of a tile
-constexpr int F4_KS = 256;                       // K elements per stage (128 bytes per row)
 constexpr int F4_A_BYTES = 128 * 128;            // one projection's codes per stage
 constexpr int F4_SF_BYTES = 4 * 512;             // 4 scale blocks (4 K blocks of 64)
 constexpr int F4_B_BYTES = F4_BN * 128;          // activation codes per stage
@@ -78,19 +77,6 @@ __host__ __device__ constexpr uint32_t idesc_nvfp4(int M, int N) {
          (static_cast<uint32_t>(M >> 4) << 24);
 }
 
-// D[tmem] (+)= (A * scale A) (B * scale B)^T over 64 K elements, block scale per 16.
-__device__ __forceinline__ void umma_nvfp4(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
-                                           uint32_t idesc, uint32_t sfa_tmem, uint32_t sfb_tmem,
-                                           uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;"
-      "\n\t}" ::"r"(d_tmem),
-      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
-      : "memory");
-}
-
 // 1 in exactly one lane of the converged warp (the same lane at every call), else 0.  As a
 // predicate of a tcgen05 or TMA instruction this keeps the instruction on its fast issue
 // path; a predicate computed from the lane index does not (measured: several times slower).
@@ -100,13 +86,6 @@ __device__ __forceinline__ uint32_t elect_lane() {
       "{\n\t.reg .pred p;\n\telect.sync _|p, 0xffffffff;\n\tselp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(e));
   return e;
-}
-
-// Shared -> tensor memory: 32 rows of 16 bytes (a 512-byte scale block) into 32 lanes x 4
-// columns, repeated in each of the four 32-lane quarters.
-__device__ __forceinline__ void tmem_cp_32x128b_warpx4(uint32_t taddr, uint64_t sdesc) {
-  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc)
-               : "memory");
 }
 
 // Descriptor of a 512-byte block read as 32 rows of 16 bytes (no swizzle, K-major): core
@@ -124,6 +103,7 @@ __device__ __forceinline__ uint64_t smem_desc_sf_block(uint32_t saddr) {
 // lanes whose `p` is non-zero.  A stage's copies and MMAs are issued as one branch-free
 // sequence predicated by elect_lane(): a few tens of cycles per instruction, where a branch
 // around each instruction costs several times that (measured).
+// D[tmem] (+)= (A * scale A) (B * scale B)^T over 64 K elements, E4M3 block scale per 16.
 __device__ __forceinline__ void umma_nvfp4_p(uint32_t p, uint32_t d_tmem, uint64_t adesc,
                                              uint64_t bdesc, uint32_t idesc, uint32_t sfa_tmem,
                                              uint32_t sfb_tmem, uint32_t accumulate) {
@@ -136,6 +116,8 @@ __device__ __forceinline__ void umma_nvfp4_p(uint32_t p, uint32_t d_tmem, uint64
       "r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
       : "memory");
 }
+// Shared -> tensor memory: 32 rows of 16 bytes (a 512-byte scale block) into 32 lanes x 4
+// columns, repeated in each of the four 32-lane quarters (the layout the MMA reads scales in).
 __device__ __forceinline__ void tmem_cp_sf_p(uint32_t p, uint32_t taddr, uint64_t sdesc) {
   asm volatile(
       "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %0, 0;\n\t"
