@@ -148,3 +148,76 @@ def test_ffn_kernel_choice(lib):
     copy = lib.moe_workspace_size(4096, 2816, 128, 704, 8, _abi.MOE_FLAG_FFN_ROWS_COPY)
     assert 0 < pairs <= single
     assert copy >= single + 2 * 4096 * 8 * 2816
+
+
+def test_nvfp4_host_checks(lib):
+    """The NVFP4 calls refuse what they cannot run before touching the device."""
+    ws = lib.moe_nvfp4_workspace_size
+    base = lib.moe_workspace_size(8, 2816, 128, 704, 8, 0)
+    fp4 = ws(8, 2816, 128, 704, 8, 0)
+    # the forward's layout plus the sorted x and h codes (and their scale lines)
+    assert fp4 >= base + 64 * 2816 // 2 + 64 * 704 // 2
+    assert ws(16, 2816, 128, 704, 8, 0) > 0
+    assert ws(17, 2816, 128, 704, 8, 0) == 0                         # T > 16
+    assert ws(8, 2816, 128, 704, 8, _abi.MOE_FLAG_DECODE_TILES) == 0  # not an NVFP4 flag
+    assert ws(8, 2816, 128, 704, 8, _abi.MOE_FLAG_FFN_PAIRS) == 0
+    wq = _abi.NVFP4Weights(*([FAKE] * 9))
+    f = lib.moe_forward_nvfp4
+    args = lambda T=8, flags=0, sx=1.0, sh=1.0, x=FAKE, y=FAKE + 4096, w=ctypes.byref(wq), \
+        nbytes=1 << 30: (x, FAKE, None, w, T, 2816, 128, 704, 8, flags, sx, sh, y, None, FAKE,
+                         nbytes, None)
+    assert f(*args(T=0)) == 0
+    assert f(*args(sx=0.0)) == _abi.MOE_ERR_INVALID_ARG                 # scales must be > 0
+    assert f(*args(sh=-1.0)) == _abi.MOE_ERR_INVALID_ARG
+    assert f(*args(w=None)) == _abi.MOE_ERR_INVALID_ARG
+    assert f(*args(y=FAKE)) == _abi.MOE_ERR_INVALID_ARG                 # y aliasing x
+    assert f(*args(flags=_abi.MOE_FLAG_FUSED_FFN)) == _abi.MOE_ERR_INVALID_ARG
+    assert f(*args(T=17)) == _abi.MOE_ERR_UNSUPPORTED
+    assert f(*args(nbytes=1024)) == _abi.MOE_ERR_NO_WORKSPACE
+    bad = _abi.NVFP4Weights(*([FAKE] * 9))
+    bad.gate_scales = FAKE + 8                                          # scales 16-byte aligned
+    assert f(*args(w=ctypes.byref(bad))) == _abi.MOE_ERR_INVALID_ARG
+    nul = _abi.NVFP4Weights(*([FAKE] * 9))
+    nul.down_ts = None
+    assert f(*args(w=ctypes.byref(nul))) == _abi.MOE_ERR_INVALID_ARG
+    q = lib.moe_nvfp4_quantize_weights
+    big = 1 << 30
+    assert q(None, 128, 2816, 704, FAKE, FAKE, FAKE, FAKE, big, None) == _abi.MOE_ERR_INVALID_ARG
+    assert q(FAKE, 128, 2848, 704, FAKE, FAKE, FAKE, FAKE, big, None) == _abi.MOE_ERR_UNSUPPORTED
+    assert q(FAKE, 128, 2816, 704, FAKE, FAKE, FAKE, FAKE, 16, None) == _abi.MOE_ERR_NO_WORKSPACE
+    assert lib.moe_nvfp4_quantize_workspace_size(128) >= 128 * 4
+
+
+def test_step_calls_host_checks(lib):
+    """moe_dispatch, moe_gather_rows, moe_expert_ffn and moe_combine (the layer's steps as
+    calls) refuse bad arguments on the host."""
+    big = 1 << 30
+    d = lib.moe_dispatch
+    assert lib.moe_dispatch_workspace_size(8, 128, 8) > 0
+    assert d(FAKE, 0, 128, 8, FAKE, FAKE, FAKE, FAKE, FAKE, big, None) == 0          # T == 0
+    assert d(FAKE, 8, 4, 8, FAKE, FAKE, FAKE, FAKE, FAKE, big, None) == 1            # k > E
+    assert d(None, 8, 128, 8, FAKE, FAKE, FAKE, FAKE, FAKE, big, None) == 1
+    assert d(FAKE, 8, 128, 8, FAKE, FAKE, FAKE, FAKE, FAKE, 16, None) == _abi.MOE_ERR_NO_WORKSPACE
+    g = lib.moe_gather_rows
+    assert g(FAKE, FAKE, 0, 8, 2816, 8, FAKE, None) == 0                               # no rows
+    assert g(FAKE + 2, FAKE, 64, 8, 2816, 8, FAKE, None) == 1                          # misaligned x
+    assert g(FAKE, FAKE, 64, 8, 2812, 8, FAKE, None) == _abi.MOE_ERR_UNSUPPORTED      # H % 8
+    f = lib.moe_expert_ffn
+    assert lib.moe_expert_ffn_workspace_size(64, 2816, 16, 704, 16) > 0
+    assert lib.moe_expert_ffn_workspace_size(64, 2816, 16, 700, 16) == 0             # I % 64
+    assert lib.moe_expert_ffn_workspace_size(64, 2816, 16, 704, 2000) == 0           # segments
+    w = (FAKE, FAKE, FAKE)
+    assert f(FAKE, 0, FAKE, FAKE, 4, *w, 2816, 16, 704, FAKE + 4096, FAKE, big, None) == 0
+    assert f(FAKE, 64, None, FAKE, 4, *w, 2816, 16, 704, FAKE + 4096, FAKE, big, None) == 1
+    assert f(FAKE, 64, FAKE, FAKE, 4, *w, 2816, 16, 704, FAKE, FAKE, big, None) == 1   # out == xs
+    assert f(FAKE, 64, FAKE, FAKE, 4, *w, 2816, 16, 700, FAKE + 4096, FAKE, big, None) == \
+        _abi.MOE_ERR_UNSUPPORTED
+    assert f(FAKE, 64, FAKE, FAKE, 4, *w, 2816, 16, 704, FAKE + 4096, FAKE, 16, None) == \
+        _abi.MOE_ERR_NO_WORKSPACE
+    c = lib.moe_combine
+    assert c(FAKE, FAKE, FAKE, 0, 8, 2816, 0, 0, 0, FAKE, None) == 0                   # T == 0
+    assert c(FAKE, FAKE, FAKE, 8, 9, 2816, 0, 64, 0, FAKE, None) == 1                  # k > 8
+    assert c(FAKE, FAKE, FAKE, 8, 8, 2816, 0, 64, 4, FAKE, None) == 1                  # flag
+    assert c(FAKE, FAKE, FAKE, 8, 8, 2816, 10, 5, 0, FAKE, None) == 1                  # lo > hi
+    assert c(FAKE, FAKE, FAKE, 8, 8, 2816, 0, 65, 0, FAKE, None) == 1                  # hi > T k
+    assert c(FAKE, FAKE, FAKE, 8, 8, 2812, 0, 64, 0, FAKE, None) == _abi.MOE_ERR_UNSUPPORTED
