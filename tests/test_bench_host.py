@@ -79,3 +79,49 @@ def test_ffn_kernel_name_follows_the_library_rule():
     assert "+" in bench.ffn_kernel_name(4096, "unfused")          # two launches
     assert bench.ffn_kernel_name(8, "fused").endswith(",1>")       # 8-row A slots
     assert bench.ffn_kernel_name(8, "decode").startswith("grouped_gemm_decode_kernel")
+
+
+def test_nvfp4_expert_bytes_are_the_formats():
+    """Per expert: three projections of H x I codes at 4 bits, one E4M3 byte per 16 of them,
+    three fp32 tensor scales."""
+    H, I = 2816, 704
+    assert bench.FP4_EXPERT_BYTES == 3 * H * I // 2 + 3 * H * I // 16 + 3 * 4 == 3_345_420
+
+
+def test_nvfp4_entry_arithmetic():
+    from expert_routed_ffn_softmax_b200 import workloads as wl
+    cfg = wl.CONFIGS["decode"]
+    m = {"active": 57, "ffn_ms": 0.060, "ms": 0.087, "stages": {"expert_ffn": 0.060},
+         "clocks": {}, "kernels": 4, "_steps": 20}
+    e = bench.nvfp4_entry(cfg, m, 1, {"hbm_gbs": 6544.7})
+    gbs = 57 * 3_345_420 / 60e-6 / 1e9
+    assert e["expert_ffn"]["algorithmic_bytes"] == 57 * 3_345_420
+    assert abs(e["expert_ffn"]["achieved_gbs"] - gbs) < 1e-6 * gbs
+    assert abs(e["expert_ffn"]["frac_of_hbm"] - gbs / 6544.7) < 1e-9
+    assert abs(e["value"] - 8 / 0.087e-3) < 1e-6 * e["value"]       # tokens/s of one rank
+    assert e["gpu_launches"] == 80
+    e2 = bench.nvfp4_entry(cfg, m, 2, {"hbm_gbs": 6544.7})
+    assert abs(e2["value"] - 2 * e["value"]) < 1e-6 * e["value"]    # the whole job
+
+
+def test_tensor_bound_entry_arithmetic():
+    from expert_routed_ffn_softmax_b200 import workloads as wl
+    cfg = wl.CONFIGS["skewed"]
+    acc = {"gemm1_flops": 1.0e12, "gemm2_flops": 0.5e12, "step_flops": 1.6e12,
+           "active_experts": 63}
+    m = {"acc": acc, "stages": {"expert_ffn": 1.5}, "ms": 2.0, "rstats": {}, "clocks": {},
+         "kernels": 4, "_steps": 20, "_tiles": "auto"}
+    pk = {"bf16_tflops": 1662.1, "bf16_tflops_sustained": 1394.8}
+    e = bench.tensor_bound_entry(cfg, m, 1, pk)
+    tf = 1.5e12 / 1.5e-3 / 1e12
+    assert abs(e["expert_ffn"]["achieved_tflops"] - tf) < 1e-9 * tf
+    assert abs(e["expert_ffn"]["frac_of_burst"] - tf / 1662.1) < 1e-12
+    assert abs(e["expert_ffn"]["frac_of_sustained"] - tf / 1394.8) < 1e-12
+    assert abs(e["step_tensor_frac"] - (1.6e12 / 2.0e-3) / 1662.1e12) < 1e-12
+    assert "router bias" in e["workload"]
+
+
+def test_kernel_source_hashes_are_per_family():
+    a, b = bench.kernel_source_sha("bf16"), bench.kernel_source_sha("nvfp4")
+    assert a != b and len(a) == len(b) == 16
+    assert a == bench.kernel_source_sha("bf16")
