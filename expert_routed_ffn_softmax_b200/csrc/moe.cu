@@ -526,7 +526,14 @@ moe_status_t launch_router(const __nv_bfloat16* x, const __nv_bfloat16* wr, cons
     launch(true, GEMM_SCREEN, dim3(nb * mt, L.screen_ks), dim3(128),
            gemm_smem_bytes<kGemmStages, 2>(), tm_x, tm_wr, tm_wr, tl, nb, H, E, (void*)scr, E);
     const long long kstride = (long long)T * E;
-    if (E <= 128)
+    // at least four waves of 2-per-SM CTAs: the 4-per-SM form (same arithmetic)
+    const bool deep = (long long)T >= 8LL * std::max(1, d.num_sms) * kScreenWarps;
+    if (E <= 128 && deep)
+      launch(true, router_screen_select_kernel<4, 4>, dim3(warps_blocks),
+             dim3(32 * kScreenWarps), 0, (const float*)scr, L.screen_ks, kstride, x,
+             (const __nv_bfloat16*)wrT, (const double*)wn, bias, T, H, E, k, kScreenC,
+             beta_scale, ids, wts, stats);
+    else if (E <= 128)
       launch(true, router_screen_select_kernel<4>, dim3(warps_blocks), dim3(32 * kScreenWarps), 0,
              (const float*)scr, L.screen_ks, kstride, x, (const __nv_bfloat16*)wrT,
              (const double*)wn, bias, T, H, E, k, kScreenC, beta_scale, ids, wts, stats);

@@ -772,9 +772,11 @@ __device__ __forceinline__ bool screen_rank_verify(const int* cand, const double
 // stats[0] += candidates, stats[1] += exact recomputations,
 // stats[2] = max over candidates of |screen - L| / (|x| |w|) (float bits, atomicMax),
 // stats[3] = 1 (the screen path), stats[4] += tokens with a candidate recomputed in fp64.
+// MINB CTAs per SM: 2 (128 registers) keeps each token's chain of L2 round trips short; 4
+// (64 registers, some spills) hides more of them when the batch is many waves deep.
 constexpr int kMaxScreenSplit = 8;
-template <int EPL>
-__global__ void __launch_bounds__(256, 2) router_screen_select_kernel(
+template <int EPL, int MINB = 2>
+__global__ void __launch_bounds__(256, MINB) router_screen_select_kernel(
     const float* __restrict__ screen, int ks, long long kstride,
     const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __restrict__ wrT,
     const double* __restrict__ wn, const float* __restrict__ bias, int T, int H, int E, int k,

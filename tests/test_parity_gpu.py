@@ -192,6 +192,21 @@ def test_route_parity_all_tokens(name, router, gemma_w):
     print(f"{name}: min gap between the k-th and (k+1)-th logit = {gap:.3e}")
 
 
+def test_screen_select_forms_agree_bitwise(gemma_w):
+    """A batch many waves deep takes the 4-CTA-per-SM form of the screen select; the same
+    tokens routed in 2048-token slices take the 2-CTA form.  Routing is per token and both
+    forms do the same arithmetic, so ids and weight bits agree."""
+    cfg = wl.CONFIGS["sweep_T32768"]
+    x, c, g = layer_inputs(cfg, gemma_w)
+    xg = x.cuda()
+    ids, w = moe.route(xg, g["w_router"], cfg.k, router="screen")
+    parts = [moe.route(xg[s:s + 2048].contiguous(), g["w_router"], cfg.k, router="screen")
+             for s in range(0, cfg.T, 2048)]
+    assert moe.sync_status() == 0
+    assert torch.equal(ids, torch.cat([p[0] for p in parts]))
+    assert torch.equal(w.view(torch.int32), torch.cat([p[1] for p in parts]).view(torch.int32))
+
+
 def test_k_equals_E_and_exact_ties():
     """k = E; duplicated router columns and all-zero rows make exact ties, which the
     kernel must resolve through its exact recomputation, in id order."""
