@@ -560,14 +560,16 @@ __device__ __forceinline__ float bf16_pair_dot(uint32_t xw, uint32_t ww) {
 //     accumulated in fp64.  |result - sum_h x_h w_h| <= 2^-24 sum_h |x_h w_h| + H 2^-150
 //     + the fp64 accumulation's error (well inside the fp64 bound beta).
 //   !PAIRS: every value converted to fp64, fp64 fused multiply-adds (error inside beta).
-template <bool PAIRS, int G>
+// UNR: unroll of the vector loop (a shorter body issues from the instruction cache better
+// when many warps share an SM).
+template <bool PAIRS, int G, int UNR>
 __device__ __forceinline__ void screen_dot(const __nv_bfloat16* __restrict__ xr,
                                            const uint4* (&wrow)[G], int H, double (&acc)[G]) {
   const int lane = threadIdx.x & 31;
 #pragma unroll
   for (int u = 0; u < G; ++u) acc[u] = 0.0;
   const uint4* xv4 = reinterpret_cast<const uint4*>(xr);
-#pragma unroll 4
+#pragma unroll UNR
   for (int v = lane; 8 * v < H; v += 32) {   // 16-byte vector index within the row
     const uint4 xq = __ldg(xv4 + v);
     uint4 wq[G];
@@ -599,7 +601,7 @@ __device__ __forceinline__ void screen_dot(const __nv_bfloat16* __restrict__ xr,
 
 // Recompute n candidates of this warp's token into val[] (+ bias): slot j is
 // sub ? sub[j] : j, its expert cand[slot].  Four rows at a time, two for a tail of <= 2.
-template <bool PAIRS>
+template <bool PAIRS, int UNR>
 __device__ __forceinline__ void screen_recheck(const __nv_bfloat16* __restrict__ xr,
                                                const __nv_bfloat16* __restrict__ wrT,
                                                const float* __restrict__ bias, int H,
@@ -615,7 +617,7 @@ __device__ __forceinline__ void screen_recheck(const __nv_bfloat16* __restrict__
       for (int u = 0; u < 4; ++u)
         wrow[u] = reinterpret_cast<const uint4*>(wrT + (size_t)cand[slot(min(c0 + u, n - 1))] * H);
       double acc[4];
-      screen_dot<PAIRS, 4>(xr, wrow, H, acc);
+      screen_dot<PAIRS, 4, UNR>(xr, wrow, H, acc);
       double v = acc[0];
 #pragma unroll
       for (int u = 1; u < 4; ++u)
@@ -631,7 +633,7 @@ __device__ __forceinline__ void screen_recheck(const __nv_bfloat16* __restrict__
       for (int u = 0; u < 2; ++u)
         wrow[u] = reinterpret_cast<const uint4*>(wrT + (size_t)cand[slot(min(c0 + u, n - 1))] * H);
       double acc[2];
-      screen_dot<PAIRS, 2>(xr, wrow, H, acc);
+      screen_dot<PAIRS, 2, UNR>(xr, wrow, H, acc);
       const double v = lane == 1 ? acc[1] : acc[0];
       if (lane < 2 && c0 + lane < n) {
         const int c = slot(c0 + lane), e = cand[c];
@@ -773,7 +775,9 @@ __device__ __forceinline__ bool screen_rank_verify(const int* cand, const double
 // stats[2] = max over candidates of |screen - L| / (|x| |w|) (float bits, atomicMax),
 // stats[3] = 1 (the screen path), stats[4] += tokens with a candidate recomputed in fp64.
 // MINB CTAs per SM: 2 (128 registers) keeps each token's chain of L2 round trips short; 4
-// (64 registers, some spills) hides more of them when the batch is many waves deep.
+// (64 registers, some spills) hides more of them when the batch is many waves deep.  The
+// recheck loop is unrolled twice in the first form and not at all in the second (measured
+// fastest for each; the arithmetic and its order do not depend on it).
 constexpr int kMaxScreenSplit = 8;
 template <int EPL, int MINB = 2>
 __global__ void __launch_bounds__(256, MINB) router_screen_select_kernel(
@@ -782,6 +786,7 @@ __global__ void __launch_bounds__(256, MINB) router_screen_select_kernel(
     const double* __restrict__ wn, const float* __restrict__ bias, int T, int H, int E, int k,
     double screen_c, double beta_scale, int32_t* __restrict__ ids, float* __restrict__ wts,
     unsigned* __restrict__ stats) {
+  constexpr int kUnr = MINB >= 4 ? 1 : 2;
   pdl_trigger();
   pdl_wait();
   if (blockIdx.x == 0 && threadIdx.x == 0) stats[3] = 1;   // path: screen + recheck
@@ -917,7 +922,7 @@ __global__ void __launch_bounds__(256, MINB) router_screen_select_kernel(
 
     // First recheck: fp32 pair sums.  Kept when every ranking decision clears the pair-sum
     // bound and the weights they give are within kPairWeightErr of the fp64 ones.
-    screen_recheck<true>(xr, wrT, bias, H, cand, nullptr, nc, val);
+    screen_recheck<true, kUnr>(xr, wrT, bias, H, cand, nullptr, nc, val);
     double V[EPL];
     int cid[EPL];
     bool taken[EPL], need[EPL];
@@ -960,7 +965,7 @@ __global__ void __launch_bounds__(256, MINB) router_screen_select_kernel(
         __syncwarp();
       }
       if (ns > 0 && ns < nc) {
-        screen_recheck<false>(xr, wrT, bias, H, cand, sub, ns, val);
+        screen_recheck<false, kUnr>(xr, wrT, bias, H, cand, sub, ns, val);
         for (int j = lane; j < ns; j += 32) prec[sub[j]] = 1;
         __syncwarp();
         ok = screen_rank_verify<EPL>(cand, val, prec, nc, wn, bias, xn, beta_scale, pair_c,
@@ -971,7 +976,7 @@ __global__ void __launch_bounds__(256, MINB) router_screen_select_kernel(
         ok = false;
       }
       if (!ok) {
-        screen_recheck<false>(xr, wrT, bias, H, cand, nullptr, nc, val);
+        screen_recheck<false, kUnr>(xr, wrT, bias, H, cand, nullptr, nc, val);
         ok = screen_rank_verify<EPL>(cand, val, nullptr, nc, wn, bias, xn, beta_scale, 0.0, 0.0,
                                      k, V, cid, taken, need, sel_e, sel_v, b_max);
       }
